@@ -1,0 +1,217 @@
+"""CPU oracle for the quantized KV-cache codec and decode attention.
+
+TEST INFRASTRUCTURE ONLY: the tests, ``__graft_entry__.smoke()`` and the
+CPU-baseline leg of ``bench.py`` are the only callers.  The product package
+never imports this module, and this module never imports the product package;
+the two share no code.
+
+The arithmetic lives in ``kvq_oracle.c`` (plain C, built with gcc, no FMA
+contraction, no fast-math).  This file only marshals numpy arrays and holds the
+recent-window bookkeeping model used to check appends, which is pure list
+logic with no arithmetic of the method.
+
+Sources: "QKVShare: Quantized KV-Cache Handoff for Multi-Agent On-Device LLMs"
+(Metodologia: quantized card, dequantize-then-inject); "Agent Memory Below the
+Prompt: Persistent Q4 KV Cache ..." (Abstract: attention over several agents'
+4-bit caches); "Coordinated Mixed-Precision KV Cache Quantization ..."
+(Abstract: per-(agent, layer) widths, recent states kept native, only newly
+quantized blocks get a width).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kvq_oracle.c")
+_LIB_PATH = os.path.join(_HERE, "_build", "liboracle_kvq.so")
+GROUP = 64
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile kvq_oracle.c into oracle/_build/liboracle_kvq.so (gcc)."""
+    os.makedirs(os.path.dirname(_LIB_PATH), exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", "-O2", "-std=c11", "-ffp-contract=off", "-fno-fast-math",
+           "-shared", "-fPIC", "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    if _lib is None:
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64, f64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
+        lib.oracle_quantize_rows.argtypes = [P, i64, i32, i32, P, P]
+        lib.oracle_dequantize_rows.argtypes = [P, P, i64, i32, i32, P]
+        lib.oracle_unpack_rows.argtypes = [P, i64, i32, i32, P]
+        lib.oracle_affine_rows.argtypes = [P, P, i64, i32, i32, P]
+        lib.oracle_decode_attn.argtypes = [i32, i32, i32, i32, i64, P, P, P, P,
+                                           i64, P, P, P, f64, P, P]
+        for f in (lib.oracle_quantize_rows, lib.oracle_dequantize_rows,
+                  lib.oracle_unpack_rows, lib.oracle_affine_rows, lib.oracle_decode_attn):
+            f.restype = ctypes.c_int
+        _lib = lib
+    return _lib
+
+
+def _ptr(a: np.ndarray):
+    return a.ctypes.data_as(ctypes.c_void_p)
+
+
+def _c(a, dtype):
+    a = np.ascontiguousarray(a)
+    if a.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {a.dtype}")
+    return a
+
+
+def row_bytes(head_dim: int, bits: int) -> int:
+    return head_dim // 8 * bits
+
+
+def quantize(x_bf16_bits: np.ndarray, bits: int):
+    """x: uint16 (bf16 bit patterns) [..., head_dim].
+
+    Returns (codes uint8 [..., head_dim*bits/8], scalemin float32 [..., head_dim/64, 2]).
+    """
+    x = _c(x_bf16_bits, np.uint16)
+    D = x.shape[-1]
+    rows = int(np.prod(x.shape[:-1], dtype=np.int64))
+    codes = np.zeros(x.shape[:-1] + (row_bytes(D, bits),), np.uint8)
+    sm = np.zeros(x.shape[:-1] + (D // GROUP, 2), np.float32)
+    rc = _load().oracle_quantize_rows(_ptr(x), rows, D, bits, _ptr(codes), _ptr(sm))
+    if rc:
+        raise ValueError(f"oracle_quantize_rows rejected the arguments (status {rc})")
+    return codes, sm
+
+
+def dequantize(codes: np.ndarray, scalemin: np.ndarray, head_dim: int, bits: int) -> np.ndarray:
+    """Returns uint16 bf16 bit patterns [..., head_dim]."""
+    codes = _c(codes, np.uint8)
+    sm = _c(scalemin, np.float32)
+    rows = int(np.prod(codes.shape[:-1], dtype=np.int64))
+    y = np.zeros(codes.shape[:-1] + (head_dim,), np.uint16)
+    rc = _load().oracle_dequantize_rows(_ptr(codes), _ptr(sm), rows, head_dim, bits, _ptr(y))
+    if rc:
+        raise ValueError(f"oracle_dequantize_rows rejected the arguments (status {rc})")
+    return y
+
+
+def unpack(codes: np.ndarray, head_dim: int, bits: int) -> np.ndarray:
+    """Integer code values, uint8 [..., head_dim]."""
+    codes = _c(codes, np.uint8)
+    rows = int(np.prod(codes.shape[:-1], dtype=np.int64))
+    out = np.zeros(codes.shape[:-1] + (head_dim,), np.uint8)
+    rc = _load().oracle_unpack_rows(_ptr(codes), rows, head_dim, bits, _ptr(out))
+    if rc:
+        raise ValueError(f"oracle_unpack_rows rejected the arguments (status {rc})")
+    return out
+
+
+def affine(codes: np.ndarray, scalemin: np.ndarray, head_dim: int, bits: int) -> np.ndarray:
+    """Exact fp64 values mn + s*c, [..., head_dim]."""
+    codes = _c(codes, np.uint8)
+    sm = _c(scalemin, np.float32)
+    rows = int(np.prod(codes.shape[:-1], dtype=np.int64))
+    out = np.zeros(codes.shape[:-1] + (head_dim,), np.float64)
+    rc = _load().oracle_affine_rows(_ptr(codes), _ptr(sm), rows, head_dim, bits, _ptr(out))
+    if rc:
+        raise ValueError(f"oracle_affine_rows rejected the arguments (status {rc})")
+    return out
+
+
+def decode_attn(q: np.ndarray, bits: int,
+                k_codes: np.ndarray | None, k_sm: np.ndarray | None,
+                v_codes: np.ndarray | None, v_sm: np.ndarray | None,
+                k_win: np.ndarray | None, v_win: np.ndarray | None,
+                softmax_scale: float, want_probs: bool = False):
+    """One view's decode attention in fp64.
+
+    q: uint16 bf16 [H_q][D].  Packed: k_codes/v_codes uint8 [H_kv][n_p][rb],
+    k_sm/v_sm float32 [H_kv][n_p][D/64][2] (or None when n_p == 0).  Window:
+    k_win/v_win uint16 bf16 [H_kv][n_w][D] in logical (oldest-first) order
+    (or None when n_w == 0).  Returns out float64 [H_q][D] (and probabilities
+    [H_q][n_p + n_w] when want_probs).
+    """
+    q = _c(q, np.uint16)
+    Hq, D = q.shape
+    if k_codes is not None:
+        k_codes = _c(k_codes, np.uint8); v_codes = _c(v_codes, np.uint8)
+        k_sm = _c(k_sm, np.float32); v_sm = _c(v_sm, np.float32)
+        Hkv, n_p = k_codes.shape[:2]
+    else:
+        n_p = 0
+    if k_win is not None:
+        k_win = _c(k_win, np.uint16); v_win = _c(v_win, np.uint16)
+        Hkv, n_w = k_win.shape[:2]
+    else:
+        n_w = 0
+    if n_p == 0 and n_w == 0:
+        raise ValueError("empty view")
+    out = np.zeros((Hq, D), np.float64)
+    probs = np.zeros((Hq, n_p + n_w), np.float64) if want_probs else None
+    null = ctypes.c_void_p(0)
+    rc = _load().oracle_decode_attn(
+        Hq, Hkv, D, bits, n_p,
+        _ptr(k_codes) if n_p else null, _ptr(k_sm) if n_p else null,
+        _ptr(v_codes) if n_p else null, _ptr(v_sm) if n_p else null,
+        n_w, _ptr(k_win) if n_w else null, _ptr(v_win) if n_w else null,
+        _ptr(q), float(softmax_scale), _ptr(out), _ptr(probs) if want_probs else null)
+    if rc:
+        raise ValueError(f"oracle_decode_attn rejected the arguments (status {rc})")
+    return (out, probs) if want_probs else out
+
+
+class WindowModel:
+    """Bookkeeping model of one view's token placement under appends.
+
+    From "Coordinated Mixed-Precision KV Cache Quantization ..." (Abstract):
+    recent states keep native precision and only newly quantized blocks get a
+    width.  Reading used here: the cache of a view that has seen tokens
+    0..n-1 holds tokens [0, n - W) quantized, in order, and the last min(n, W)
+    tokens in a bf16 ring of W slots; appending a token when the ring is full
+    first quantizes the oldest ring token (at the view's width at that moment)
+    and appends it to the packed part, then stores the new token in the freed
+    slot.  With W == 0 every token is quantized on arrival.
+
+    Pure list logic: it tracks which token sits where, never a value.
+    """
+
+    def __init__(self, capacity_window: int, packed_tokens=(), window_tokens=(), head: int = 0):
+        self.W = capacity_window
+        self.packed = list(packed_tokens)      # token ids, oldest first
+        self.slots = [None] * capacity_window  # ring: slot -> token id
+        self.head = head
+        for i, tok in enumerate(window_tokens):
+            self.slots[(head + i) % capacity_window] = tok
+        self.n_window = len(window_tokens)
+
+    def append(self, tok):
+        """Returns the token id that was flushed into the packed part, or None."""
+        if self.W == 0:
+            self.packed.append(tok)
+            return tok
+        if self.n_window == self.W:
+            old = self.slots[self.head]
+            self.packed.append(old)
+            self.slots[self.head] = tok
+            self.head = (self.head + 1) % self.W
+            return old
+        self.slots[(self.head + self.n_window) % self.W] = tok
+        self.n_window += 1
+        return None
+
+    def window_logical(self):
+        return [self.slots[(self.head + i) % self.W] for i in range(self.n_window)]

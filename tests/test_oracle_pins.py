@@ -1,0 +1,423 @@
+"""Pins of the CPU oracle against facts fixed outside the oracle itself.
+
+The pages print no worked numeric example, so every pin here is a closed form,
+an invariant, a brute-force search, or a special case that reduces to a library
+routine (torch's float->bf16 rounding, numpy/scipy softmax, torch SDPA in fp64).
+Each targets a plausible mistake: wrong bit order, wrong rounding mode, 2^b in
+place of 2^b-1, a dropped min term, a wrong GQA head map, a transposed operand.
+"""
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from quantized_kv_cache_dequantize_b200 import workloads as wl
+
+BITS = (2, 3, 4, 8)
+
+
+def bf16_of(values):
+    """float values -> bf16 bit patterns (torch RNE); values must be exact in bf16."""
+    t = torch.tensor(np.asarray(values, np.float64), dtype=torch.float64).to(torch.bfloat16)
+    back = t.to(torch.float64).numpy()
+    assert np.array_equal(back, np.asarray(values, np.float64)), "value not exact in bf16"
+    return t.view(torch.int16).numpy().view(np.uint16)
+
+
+def bf16_to_f64(bits_u16):
+    return torch.from_numpy(np.ascontiguousarray(bits_u16).view(np.int16)).view(torch.bfloat16) \
+        .to(torch.float64).numpy()
+
+
+def packed_closed_form(codes, bits):
+    """Little-endian, LSB-first bit packing as one big integer per group."""
+    codes = list(int(c) for c in codes)
+    out = bytearray()
+    for g in range(len(codes) // 64):
+        val = 0
+        for j, c in enumerate(codes[64 * g: 64 * g + 64]):
+            val |= c << (j * bits)
+        out += val.to_bytes(8 * bits, "little")
+    return np.frombuffer(bytes(out), np.uint8)
+
+
+# ------------------------------------------------------------- packing ----
+
+@pytest.mark.parametrize("bits", BITS)
+def test_packing_closed_form_every_position_and_value(bits):
+    qmax = (1 << bits) - 1
+    rows = []
+    expect_codes = []
+    for j in range(64):
+        for c in range(qmax + 1):
+            codes = np.zeros(64, np.int64)
+            # endpoints fix mn = 0 and mx = qmax (s = 1) without touching slot j
+            codes[(j + 1) % 64] = 0
+            codes[(j + 2) % 64] = qmax
+            codes[j] = c
+            rows.append(codes.astype(np.float64))
+            expect_codes.append(codes)
+    x = bf16_of(np.stack(rows))
+    packed, sm = oracle.quantize(x, bits)
+    assert np.all(sm[..., 0] == 1.0) and np.all(sm[..., 1] == 0.0)
+    for r, codes in enumerate(expect_codes):
+        assert np.array_equal(packed[r], packed_closed_form(codes, bits)), (bits, r)
+    assert np.array_equal(oracle.unpack(packed, 64, bits), np.stack(expect_codes).astype(np.uint8))
+
+
+def test_packing_b4_nibbles_and_b8_identity():
+    rng = np.random.default_rng(0)
+    for bits in (4, 8):
+        qmax = (1 << bits) - 1
+        codes = rng.integers(0, qmax + 1, size=(16, 128))
+        codes[:, 0] = 0
+        codes[:, 64] = 0
+        codes[:, 1] = qmax
+        codes[:, 65] = qmax
+        packed, _ = oracle.quantize(bf16_of(codes.astype(np.float64)), bits)
+        if bits == 8:
+            assert np.array_equal(packed, codes.astype(np.uint8))
+        else:
+            lo, hi = codes[:, 0::2], codes[:, 1::2]
+            assert np.array_equal(packed, (lo | (hi << 4)).astype(np.uint8))
+
+
+# ------------------------------------------------------------ quantize ----
+
+@pytest.mark.parametrize("bits", BITS)
+@pytest.mark.parametrize("k", [0, 3, 4, 7])
+def test_on_grid_round_trip_is_exact(bits, k):
+    """x = mn + c * 2^-k with 0 and 2^b-1 present: codes, s, mn reproduced and
+    dequantize returns x bit for bit."""
+    rng = np.random.default_rng(100 * bits + k)
+    qmax = (1 << bits) - 1
+    s = 2.0 ** -k
+    rows, want = [], []
+    for mn in (0.0, -8.0, -2.0 ** -3, 1.5, -96.0):
+        for _ in range(8):
+            c = rng.integers(0, qmax + 1, size=128)
+            for g0 in (0, 64):
+                i0, i1 = rng.choice(64, size=2, replace=False)
+                c[g0 + i0] = 0
+                c[g0 + i1] = qmax
+            vals = mn + c * s
+            # keep only rows exact in bf16 (8 significant bits)
+            t = torch.tensor(vals).to(torch.bfloat16).to(torch.float64).numpy()
+            if np.array_equal(t, vals):
+                rows.append(vals)
+                want.append((c, mn))
+    assert len(rows) >= 8
+    x = bf16_of(np.stack(rows))
+    packed, sm = oracle.quantize(x, bits)
+    got = oracle.unpack(packed, 128, bits)
+    for r, (c, mn) in enumerate(want):
+        assert np.array_equal(got[r], c), (bits, k, r)
+        assert np.all(sm[r, :, 0] == np.float32(s))
+        assert np.all(sm[r, :, 1] == np.float32(mn))
+    y = oracle.dequantize(packed, sm, 128, bits)
+    assert np.array_equal(y, x)
+    assert np.array_equal(oracle.affine(packed, sm, 128, bits), np.stack(rows))
+
+
+def test_round_half_to_even():
+    # b=2: mn=0, mx=3 -> s=1; x=0.5,1.5,2.5 are exact ties -> 0, 2, 2
+    vals = np.zeros(64)
+    vals[0], vals[1] = 0.0, 3.0
+    vals[2:5] = [0.5, 1.5, 2.5]
+    packed, sm = oracle.quantize(bf16_of(vals[None]), 2)
+    c = oracle.unpack(packed, 64, 2)[0]
+    assert sm[0, 0, 0] == 1.0
+    assert list(c[2:5]) == [0, 2, 2]
+    # b=4: ties k+0.5 for k=0..14 -> even neighbour
+    vals = np.zeros(64)
+    vals[0], vals[1] = 0.0, 15.0
+    vals[2:17] = np.arange(15) + 0.5
+    packed, _ = oracle.quantize(bf16_of(vals[None]), 4)
+    c = oracle.unpack(packed, 64, 4)[0][2:17]
+    want = [k if k % 2 == 0 else k + 1 for k in range(15)]
+    assert list(c) == want
+
+
+def test_constant_groups():
+    for bits in BITS:
+        for v in (0.0, -0.0, 1.0, -3.5, 1e-30):
+            vals = np.full((1, 64), v)
+            x = torch.tensor(vals).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+            packed, sm = oracle.quantize(x, bits)
+            assert np.all(packed == 0)
+            assert sm[0, 0, 0] == 0.0
+            mn_bits = np.float32(sm[0, 0, 1]).view(np.uint32)
+            if v == 0.0:
+                assert mn_bits == 0  # -0 stored as +0
+            y = oracle.dequantize(packed, sm, 64, bits)
+            yv = bf16_to_f64(y)
+            assert np.all(yv == (0.0 if v == 0.0 else bf16_to_f64(x)[0, 0]))
+
+
+def random_groups(seed, n_rows, head_dim=128, outliers=True):
+    g = wl.generator(seed)
+    mask = wl.outlier_mask(g, n_rows, head_dim, 0.0, first4=outliers)
+    t = wl.normal_bf16(g, (n_rows, 1, head_dim), scale_mask=mask)[:, 0, :]
+    return wl.bf16_bits(t)
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_error_bound_endpoints_and_brute_force(bits):
+    qmax = (1 << bits) - 1
+    x = random_groups(7 + bits, 48)
+    packed, sm = oracle.quantize(x, bits)
+    codes = oracle.unpack(packed, 128, bits).astype(np.int64)
+    xv = bf16_to_f64(x)
+    for r in range(x.shape[0]):
+        for g in range(2):
+            seg = xv[r, 64 * g: 64 * g + 64]
+            cs = codes[r, 64 * g: 64 * g + 64]
+            s, mn = float(sm[r, g, 0]), float(sm[r, g, 1])
+            mx = seg.max()
+            assert mn == seg.min()
+            # scale: within one fp32 ulp of (mx - mn) / (2^b - 1)
+            exact_s = (mx - mn) / qmax
+            assert abs(s - exact_s) <= np.spacing(np.float32(s)) * 1.0
+            # endpoints
+            assert cs[np.argmin(seg)] == 0 and cs[np.argmax(seg)] == qmax
+            # error bound |x - (mn + s c)| <= s (1/2 + 2^(b-23))
+            err = np.abs(seg - (mn + s * cs))
+            assert np.all(err <= s * (0.5 + 2.0 ** (bits - 23)))
+            # brute force: nearest grid point over all codes, ties to even,
+            # measured in exact rational arithmetic; near-ties accept either
+            # neighbour, since the two fp32 roundings before the integer step
+            # move the quotient by up to 2^(b-23) (relative 2^-23 of <= 2^b)
+            S, MN = Fraction(s), Fraction(mn)
+            for i in range(64):
+                X = Fraction(seg[i])
+                dist = [abs(X - (MN + S * c)) for c in range(qmax + 1)]
+                best = min(dist)
+                cands = [c for c in range(qmax + 1) if dist[c] == best]
+                nearest = cands[0] if len(cands) == 1 else [c for c in cands if c % 2 == 0][0]
+                qstar = (X - MN) / S
+                frac = qstar - int(qstar)
+                if abs(frac - Fraction(1, 2)) < Fraction(1, 1 << (21 - bits)):
+                    assert cs[i] in (int(qstar), int(qstar) + 1)
+                else:
+                    assert cs[i] == nearest, (bits, r, g, i)
+
+
+# ---------------------------------------------------------- dequantize ----
+
+def bf16_nearest_exact(v: Fraction):
+    """Nearest bf16 value to an exact rational (ties to even), as float."""
+    if v == 0:
+        return 0.0
+    f = float(v)
+    lo = torch.tensor([f], dtype=torch.float64).to(torch.bfloat16)
+    cand = set()
+    base = lo.view(torch.int16).item() & 0xFFFF
+    for d in (-1, 0, 1):
+        b = (base + d) & 0xFFFF
+        val = torch.tensor([b], dtype=torch.int32).to(torch.int16).view(torch.bfloat16).to(torch.float64).item()
+        cand.add(val)
+    best = min(cand, key=lambda c: (abs(Fraction(c) - v), 0))
+    return best
+
+
+@pytest.mark.parametrize("bits", BITS)
+def test_dequantize_matches_library_rounding(bits):
+    x = random_groups(40 + bits, 24)
+    packed, sm = oracle.quantize(x, bits)
+    y = oracle.dequantize(packed, sm, 128, bits)
+    codes = oracle.unpack(packed, 128, bits).astype(np.float64)
+    s = np.repeat(sm[..., 0].astype(np.float64), 64, axis=-1)
+    mn = np.repeat(sm[..., 1].astype(np.float64), 64, axis=-1)
+    # c*s + mn is exact in fp64 here (<= 32 significant bits, small exponent
+    # spread), so rounding it to fp32 is the single rounding of fmaf
+    f32 = (codes * s + mn).astype(np.float32)
+    want = torch.from_numpy(f32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    assert np.array_equal(y, want)
+    # and the result is a nearest bf16 of the exact affine value (a near-tie
+    # may go either way through the fp32 step)
+    yv = bf16_to_f64(y)
+    exact = codes * s + mn
+    ulp = np.spacing(np.abs(yv).astype(np.float32)).astype(np.float64) * 2 ** 16
+    assert np.all(np.abs(yv - exact) <= 0.5 * ulp * (1 + 2 ** -10) + 1e-300)
+
+
+def test_bf16_rounding_ties():
+    # exact bf16 midpoints: 1 + 2^-8 (tie -> 1.0), 1 + 3*2^-8 (tie -> 1 + 2^-6)
+    codes = np.zeros((1, 8), np.uint8)  # b=8, 64 codes; only first used
+    for val, want in ((1.0 + 2 ** -8, 1.0), (1.0 + 3 * 2 ** -8, 1.0 + 2 ** -6),
+                      (-(1.0 + 2 ** -8), -1.0)):
+        codes = np.zeros((1, 64), np.uint8)
+        sm = np.array([[[0.0, val]]], np.float32)
+        y = oracle.dequantize(codes, sm, 64, 8)
+        assert bf16_to_f64(y)[0, 0] == want
+
+
+# ----------------------------------------------------------- attention ----
+
+def make_view(seed, Hq=4, Hkv=2, D=64, n_p=40, n_w=7, bits=4):
+    g = wl.generator(seed)
+    mask = wl.outlier_mask(g, Hkv, D, 0.0, first4=True)
+    k, v = wl.kv_pair(g, Hkv, n_p + n_w, D, mask)
+    q = wl.normal_bf16(g, (Hq, D))
+    kb, vb, qb = wl.bf16_bits(k), wl.bf16_bits(v), wl.bf16_bits(q)
+    kc, ks = oracle.quantize(kb[:, :n_p], bits)
+    vc, vs = oracle.quantize(vb[:, :n_p], bits)
+    return dict(q=qb, bits=bits, k_codes=kc, k_sm=ks, v_codes=vc, v_sm=vs,
+                k_win=kb[:, n_p:], v_win=vb[:, n_p:], D=D, Hq=Hq, Hkv=Hkv)
+
+
+def dense_kv(view):
+    D, bits = view["D"], view["bits"]
+    kp = oracle.affine(view["k_codes"], view["k_sm"], D, bits)
+    vp = oracle.affine(view["v_codes"], view["v_sm"], D, bits)
+    k = np.concatenate([kp, bf16_to_f64(view["k_win"])], axis=1)
+    v = np.concatenate([vp, bf16_to_f64(view["v_win"])], axis=1)
+    return k, v
+
+
+def run(view, scale, probs=False):
+    return oracle.decode_attn(view["q"], view["bits"], view["k_codes"], view["k_sm"],
+                              view["v_codes"], view["v_sm"], view["k_win"], view["v_win"],
+                              scale, want_probs=probs)
+
+
+def test_attention_matches_numpy_scipy_brute_force():
+    from scipy.special import softmax
+    view = make_view(11)
+    scale = 1 / 8
+    out = run(view, scale)
+    k, v = dense_kv(view)
+    q = bf16_to_f64(view["q"])
+    G = view["Hq"] // view["Hkv"]
+    for h in range(view["Hq"]):
+        logits = scale * (k[h // G] @ q[h])
+        p = softmax(logits)
+        np.testing.assert_allclose(out[h], p @ v[h // G], rtol=1e-12, atol=1e-12)
+
+
+def test_attention_matches_torch_sdpa_fp64():
+    import torch.nn.functional as F
+    view = make_view(12, Hq=8, Hkv=2, D=128, n_p=33, n_w=5)
+    scale = 0.3
+    out = run(view, scale)
+    k, v = dense_kv(view)
+    q = torch.from_numpy(bf16_to_f64(view["q"]))[None, :, None, :]
+    kk = torch.from_numpy(k)[None]
+    vv = torch.from_numpy(v)[None]
+    ref = F.scaled_dot_product_attention(q, kk, vv, scale=scale, enable_gqa=True)[0, :, 0, :]
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_window_only_view_is_textbook_bf16_attention():
+    import torch.nn.functional as F
+    g = wl.generator(13)
+    Hq, Hkv, D, n = 6, 3, 64, 19
+    k, v = wl.kv_pair(g, Hkv, n, D, None)
+    q = wl.normal_bf16(g, (Hq, D))
+    out = oracle.decode_attn(wl.bf16_bits(q), 4, None, None, None, None,
+                             wl.bf16_bits(k), wl.bf16_bits(v), 1 / 8)
+    ref = F.scaled_dot_product_attention(q.double()[None, :, None], k.double()[None], v.double()[None],
+                                         scale=1 / 8, enable_gqa=True)[0, :, 0]
+    np.testing.assert_allclose(out, ref.numpy(), rtol=1e-12, atol=1e-12)
+
+
+def test_softmax_rows_sum_to_one_and_match_probs():
+    view = make_view(14)
+    out, p = run(view, 1 / 8, probs=True)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=0, atol=1e-12)
+    assert np.all(p >= 0)
+    _, v = dense_kv(view)
+    G = view["Hq"] // view["Hkv"]
+    for h in range(view["Hq"]):
+        np.testing.assert_allclose(out[h], p[h] @ v[h // G], rtol=1e-12, atol=1e-12)
+
+
+def test_identical_keys_give_mean_of_values():
+    g = wl.generator(15)
+    Hq, Hkv, D, n = 4, 2, 64, 23
+    k1, v = wl.kv_pair(g, Hkv, n, D, None)
+    k = k1[:, :1, :].expand(Hkv, n, D).contiguous()
+    q = wl.normal_bf16(g, (Hq, D))
+    out = oracle.decode_attn(wl.bf16_bits(q), 4, None, None, None, None,
+                             wl.bf16_bits(k), wl.bf16_bits(v), 0.2)
+    mean = v.double().mean(dim=1).numpy()
+    for h in range(Hq):
+        np.testing.assert_allclose(out[h], mean[h // 2], rtol=1e-12, atol=1e-12)
+
+
+def test_dominant_logit_selects_its_value_row():
+    g = wl.generator(16)
+    Hq, Hkv, D, n = 2, 1, 64, 30
+    k = torch.zeros(Hkv, n, D)
+    k[0, 17, 0] = 40.0  # q = e_0 -> logit 40 for token 17, 0 elsewhere
+    q = torch.zeros(Hq, D)
+    q[:, 0] = 1.0
+    _, v = wl.kv_pair(g, Hkv, n, D, None)
+    out = oracle.decode_attn(wl.bf16_bits(q.bfloat16()), 4, None, None, None, None,
+                             wl.bf16_bits(k.bfloat16()), wl.bf16_bits(v), 1.0)
+    np.testing.assert_allclose(out[0], v[0, 17].double().numpy(), atol=1e-15 * 0 + 1e-15 + np.exp(-40) * 30 * 5)
+
+
+def test_token_permutation_invariance():
+    view = make_view(17, n_p=50, n_w=9)
+    base = run(view, 1 / 8)
+    rng = np.random.default_rng(0)
+    pp = rng.permutation(50)
+    pw = rng.permutation(9)
+    perm = dict(view)
+    for key in ("k_codes", "k_sm", "v_codes", "v_sm"):
+        perm[key] = view[key][:, pp]
+    for key in ("k_win", "v_win"):
+        perm[key] = view[key][:, pw]
+    np.testing.assert_allclose(run(perm, 1 / 8), base, rtol=1e-12, atol=1e-13)
+
+
+def test_gqa_identical_queries_in_group_give_identical_outputs():
+    view = make_view(18, Hq=8, Hkv=2)
+    q = view["q"].copy()
+    q[1:4] = q[0]
+    q[5:8] = q[4]
+    view["q"] = q
+    out = run(view, 1 / 8)
+    for h in range(1, 4):
+        assert np.array_equal(out[h], out[0])
+    for h in range(5, 8):
+        assert np.array_equal(out[h], out[4])
+    assert not np.allclose(out[0], out[4])
+
+
+def test_key_and_value_roles_are_not_swapped():
+    # keys all equal, values distinct: output is the mean of V, not of K
+    view = make_view(19)
+    view["k_codes"] = np.repeat(view["k_codes"][:, :1], 40, axis=1)
+    view["k_sm"] = np.repeat(view["k_sm"][:, :1], 40, axis=1)
+    view["k_win"] = np.repeat(view["k_win"][:, :1], 7, axis=1)
+    # make the window key identical to the packed key's exact value as well
+    kp = oracle.affine(view["k_codes"][:, :1], view["k_sm"][:, :1], 64, 4)
+    out = run(view, 1 / 8)
+    _, v = dense_kv(view)
+    k, _ = dense_kv(view)
+    q = bf16_to_f64(view["q"])
+    from scipy.special import softmax
+    for h in range(4):
+        p = softmax((1 / 8) * (k[h // 2] @ q[h]))
+        np.testing.assert_allclose(out[h], p @ v[h // 2], rtol=1e-12, atol=1e-12)
+    assert kp.shape[1] == 1
+
+
+# --------------------------------------------------------- window model ---
+
+@pytest.mark.parametrize("W", [0, 1, 4, 7])
+def test_window_model_invariant(W):
+    rng = np.random.default_rng(W)
+    m = oracle.WindowModel(W)
+    n = 0
+    for _ in range(40):
+        m.append(n)
+        n += 1
+        split = max(0, n - W)
+        assert m.packed == list(range(split))
+        assert (m.window_logical() if W else []) == list(range(split, n))
+    assert rng is not None
