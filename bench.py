@@ -1,0 +1,451 @@
+#!/usr/bin/env python
+"""Benchmark: batched multi-agent decode over packed 4-bit KV caches.
+
+Workload (one step = one decode token for every agent): 10 agents x 32 layers
+in Llama-3.1-8B shape (32 query / 8 KV heads, head_dim 128), each (agent,
+layer) view holding 4096 packed 4-bit tokens plus a full 128-token bf16 recent
+window.  Per layer the step runs kvq_append (the new token enters the window;
+the oldest window token is quantized into the packed part) and then
+kvq_decode_attn over the 10 agents' views of that layer; the 64 calls of a
+step are replayed from one CUDA graph.  The per-step working set (~1.9 GB) is
+far larger than L2, so no flush is needed between steps.
+
+Also measured in the same run: the bulk handoff codec (quantize then
+dequantize one agent's 32-layer x 8-head x 32768-token x 128 K and V cache,
+4-bit), kvq_decode_attn as one call over all 320 views, and the CPU oracle on
+a bounded sample of the same decode workload.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import csv
+import io
+import json
+import math
+import os
+import subprocess
+import sys
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "decode-attn packed-KV GB/s & tokens/s/agent, % of HBM peak; quantize GB/s"
+WORKLOAD = ("batched multi-agent decode, Llama-3.1-8B shape: 10 agents x 32 layers, 32 q / 8 kv heads, "
+            "head_dim 128, 4096 packed 4-bit group-64 tokens + 128-token bf16 window per view, "
+            "one decode token per agent per step")
+
+
+def peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+# ------------------------------------------------------------- byte counts --
+
+def attn_bytes(n_views, Hkv, Hq, D, n_p, n_w, bits):
+    """Algorithmic bytes of one kvq_decode_attn over n_views identical views:
+    packed K and V codes + their scale/min, bf16 window K and V, bf16 q, fp32 out."""
+    rb = D // 8 * bits
+    per_view = Hkv * (n_p * (2 * rb + 2 * (D // 64) * 8) + n_w * 2 * D * 2) + Hq * D * 2 + Hq * D * 4
+    return n_views * per_view
+
+
+def append_bytes(n_views, Hkv, D, bits):
+    """kvq_append with a full window: read the new K/V token and the flushed
+    window row, write the packed row (+ scale/min) and the window row."""
+    rb = D // 8 * bits
+    return n_views * 2 * Hkv * (D * 2 + D * 2 + rb + (D // 64) * 8 + D * 2)
+
+
+# ------------------------------------------------------------ clock sampler --
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except Exception:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        self.out = ""
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.out, _ = self.proc.communicate(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        if not getattr(self, "out", ""):
+            return None
+        rows = [r for r in csv.reader(io.StringIO(self.out)) if len(r) >= 9]
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = max((float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()), default=None)
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for name, val in zip(names, r[5:9]):
+                if val.strip().lower().startswith("active"):
+                    reasons.add(name)
+        return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
+                "reasons": sorted(reasons), "samples": len(rows)}
+
+
+# ------------------------------------------------------------------ helpers --
+
+def ev_pair():
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ------------------------------------------------------------ oracle timing --
+
+def oracle_sample(w, views_idx, device="cuda"):
+    """Time the fp64 CPU oracle on some views of the decode workload (inputs
+    regenerated from the seeds; quantization by the oracle itself, untimed).
+    Returns (seconds of attention, algorithmic bytes of those views)."""
+    import oracle
+    from quantized_kv_cache_dequantize_b200 import cache as kcache, workloads as wl
+    q_all = kcache.decode_queries(w, device=device)
+    secs, nbytes = 0.0, 0
+    for (a, l) in views_idx:
+        k, v, head = kcache.view_inputs(w, a, l, device=device)
+        n_p = w.view_len(a)
+        kb, vb = wl.bf16_bits(k), wl.bf16_bits(v)
+        bits = w.view_bits(a, l)
+        kc, ks = oracle.quantize(kb[:, :n_p], bits)
+        vc, vs = oracle.quantize(vb[:, :n_p], bits)
+        qv = wl.bf16_bits(q_all[l * w.n_agents + a])
+        t0 = time.perf_counter()
+        oracle.decode_attn(qv, bits, kc, ks, vc, vs, kb[:, n_p:], vb[:, n_p:], w.softmax_scale)
+        secs += time.perf_counter() - t0
+        nbytes += attn_bytes(1, w.n_kv_heads, w.n_q_heads, w.head_dim, n_p, w.window, bits)
+    return secs, nbytes
+
+
+def run_reference(args, rank, world):
+    """Reference arm: the CPU oracle, as it stands, on the host cores."""
+    if rank != 0:
+        return
+    from quantized_kv_cache_dequantize_b200 import workloads as wl
+    w = wl.decode_llama8b()
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    per_step = [(a, 0) for a in range(2)]
+    for s in range(args.warmup):
+        oracle_sample(w, per_step, dev)
+    secs, nbytes = 0.0, 0
+    for s in range(args.steps):
+        views = [((2 * s + a) % w.n_agents, (s // 5) % w.n_layers) for a in range(2)]
+        t, b = oracle_sample(w, views, dev)
+        secs += t
+        nbytes += b
+    gbs = nbytes / secs / 1e9
+    sample = f"2 (agent, layer) views per step ({w.n_kv_heads} kv heads x 4224 tokens each), fp64 oracle attention"
+    line = {"impl": "reference", "metric": METRIC, "value": gbs, "unit": "GB/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": secs / args.steps * 1e3,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": {"workload": WORKLOAD},
+            "cpu_baseline": {"value": gbs, "unit": "GB/s", "cores": 1, "kind": "oracle", "sample": sample},
+            "e2e": {"value": gbs, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- ours ---
+
+def run_ours(args, rank, world, local):
+    import quantized_kv_cache_dequantize_b200 as kvq
+    from quantized_kv_cache_dequantize_b200 import cache as kcache, workloads as wl
+    dev = torch.device("cuda", torch.cuda.current_device())
+    peak, peak_kind = peaks()
+    extra = {}
+
+    # ---------------- decode workload (each rank holds its own 10 agents)
+    w = wl.decode_llama8b(seed=3 + 1000 * rank)
+    steps_total = args.warmup + args.steps + 4
+    # layer-major view order: views of layer l are [l*A, (l+1)*A)
+    specs = []
+    for l in range(w.n_layers):
+        for a in range(w.n_agents):
+            specs.append(dict(n_kv_heads=w.n_kv_heads, head_dim=w.head_dim, bits=w.view_bits(a, l),
+                              cap_packed=w.view_len(a) + steps_total + 2, cap_window=w.window))
+    pool = kcache.ViewPool(specs, dev)
+    for l in range(w.n_layers):
+        for a in range(w.n_agents):
+            k, v, head = kcache.view_inputs(w, a, l, dev)
+            view = pool.views[l * w.n_agents + a]
+            n_p = w.view_len(a)
+            view.fill_packed(k[:, :n_p], v[:, :n_p])
+            view.fill_window(k[:, n_p:], v[:, n_p:], head=head)
+    views = pool.views
+    A, L = w.n_agents, w.n_layers
+    q = kcache.decode_queries(w, device=dev)                        # [L*A, Hq, D] layer-major
+    kn, vn = kcache.decode_new_tokens(w, device=dev)                # [L*A, Hkv, D]
+    out = torch.empty((L * A, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+    layer_views = [views[l * A:(l + 1) * A] for l in range(L)]
+    ws = [kvq.new_workspace(lv, w.n_q_heads, device=dev) for lv in layer_views]
+    torch.cuda.synchronize()
+
+    stream = torch.cuda.Stream()
+    n_launch_per_step = 2 * L
+
+    def step():
+        for l in range(L):
+            kvq.append(layer_views[l], kn[l * A:(l + 1) * A], vn[l * A:(l + 1) * A], stream=stream)
+            kvq.decode_attn(layer_views[l], q[l * A:(l + 1) * A], w.softmax_scale,
+                            out=out[l * A:(l + 1) * A], workspace=ws[l], stream=stream)
+
+    # capture one step in a graph; host view counters advance at capture, so
+    # the graph replays the same (full-window) append + attend each time
+    with torch.cuda.stream(stream):
+        step()  # eager warm-up of every code path
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        step()
+    stream.synchronize()
+
+    bytes_step = (attn_bytes(L * A, w.n_kv_heads, w.n_q_heads, w.head_dim, w.view_len(0) + 1, w.window, 4)
+                  + append_bytes(L * A, w.n_kv_heads, w.head_dim, 4))
+    for _ in range(args.warmup):
+        graph.replay()
+    stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    e0, e1 = ev_pair()
+    with ClockSampler(local) as clk:
+        with torch.cuda.stream(stream):
+            e0.record(stream)
+            for _ in range(args.steps):
+                graph.replay()
+            e1.record(stream)
+        stream.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    t_step = e0.elapsed_time(e1) / 1e3 / args.steps
+    t_step = max_over_ranks(t_step, world)
+    value = world * bytes_step / t_step / 1e9
+
+    # ---------------- dominant kernel: kvq_decode_attn per layer, timed alone
+    attn_layer_bytes = attn_bytes(A, w.n_kv_heads, w.n_q_heads, w.head_dim, w.view_len(0) + 1, w.window, 4)
+    evs = [ev_pair() for _ in range(args.steps * L)]
+    with torch.cuda.stream(stream):
+        for i in range(args.warmup * L):
+            l = i % L
+            kvq.decode_attn(layer_views[l], q[l * A:(l + 1) * A], w.softmax_scale, out=out[l * A:(l + 1) * A],
+                            workspace=ws[l], stream=stream)
+        for i, (a0, a1) in enumerate(evs):
+            l = i % L
+            a0.record(stream)
+            kvq.decode_attn(layer_views[l], q[l * A:(l + 1) * A], w.softmax_scale, out=out[l * A:(l + 1) * A],
+                            workspace=ws[l], stream=stream)
+            a1.record(stream)
+    stream.synchronize()
+    t_attn = float(np.mean([a0.elapsed_time(a1) for a0, a1 in evs])) / 1e3
+    attn_gbs = attn_layer_bytes / t_attn / 1e9
+
+    # ---------------- one call over all 320 views
+    ws_all = kvq.new_workspace(views, w.n_q_heads, device=dev)
+    with torch.cuda.stream(stream):
+        for _ in range(max(3, args.warmup)):
+            kvq.decode_attn(views, q, w.softmax_scale, out=out, workspace=ws_all, stream=stream)
+        b0, b1 = ev_pair()
+        b0.record(stream)
+        for _ in range(args.steps):
+            kvq.decode_attn(views, q, w.softmax_scale, out=out, workspace=ws_all, stream=stream)
+        b1.record(stream)
+    stream.synchronize()
+    t_all = b0.elapsed_time(b1) / 1e3 / args.steps
+    all_gbs = attn_bytes(L * A, w.n_kv_heads, w.n_q_heads, w.head_dim, w.view_len(0) + 1, w.window, 4) / t_all / 1e9
+
+    # ---------------- end to end through the public API with host buffers
+    q_h = q.cpu().pin_memory()
+    kn_h, vn_h = kn.cpu().pin_memory(), vn.cpu().pin_memory()
+    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = q_h.numel() * 2 + kn_h.numel() * 2 + vn_h.numel() * 2
+    d2h = out_h.numel() * 4
+
+    def e2e_step():
+        q.copy_(q_h, non_blocking=True)
+        kn.copy_(kn_h, non_blocking=True)
+        vn.copy_(vn_h, non_blocking=True)
+        graph.replay()
+        out_h.copy_(out, non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            e2e_step()
+        stream.synchronize()
+        c0, c1 = ev_pair()
+        c0.record(stream)
+        for _ in range(args.steps):
+            e2e_step()
+        c1.record(stream)
+    stream.synchronize()
+    t_e2e = max_over_ranks(c0.elapsed_time(c1) / 1e3 / args.steps, world)
+    e2e_gbs = world * bytes_step / t_e2e / 1e9
+
+    del pool, ws, ws_all, q, out
+    torch.cuda.empty_cache()
+
+    # ---------------- bulk handoff codec (quantize then dequantize), 4-bit
+    codec = None
+    if not args.skip_codec:
+        hw = wl.handoff_llama8b()
+        H = hw.n_layers * hw.n_kv_heads
+        gm = wl.generator(hw.seed)
+        mask = torch.stack([wl.outlier_mask(gm, hw.n_kv_heads, hw.head_dim, hw.outlier_frac)
+                            for _ in range(hw.n_layers)]).view(H, hw.head_dim)
+        g = wl.generator(hw.seed, device=dev)
+        kx, vx = wl.kv_pair(g, H, hw.n_tokens, hw.head_dim, mask, dev)
+        rb = hw.head_dim // 8 * hw.bits
+        kc = torch.empty((H, hw.n_tokens, rb), dtype=torch.uint8, device=dev)
+        vc = torch.empty_like(kc)
+        ks = torch.empty((H, hw.n_tokens, hw.head_dim // 64, 2), dtype=torch.float32, device=dev)
+        vs = torch.empty_like(ks)
+        ky, vy = torch.empty_like(kx), torch.empty_like(vx)
+        n_el = 2 * H * hw.n_tokens * hw.head_dim
+        codec_bytes = n_el * 2 + 2 * (kc.numel() + ks.numel() * 4)
+        qt, dt = [], []
+        with torch.cuda.stream(stream):
+            for it in range(args.warmup + args.steps):
+                a0, a1, a2 = torch.cuda.Event(True), torch.cuda.Event(True), torch.cuda.Event(True)
+                a0.record(stream)
+                kvq.quantize(kx, hw.bits, kc, ks, stream=stream)
+                kvq.quantize(vx, hw.bits, vc, vs, stream=stream)
+                a1.record(stream)
+                kvq.dequantize(kc, ks, hw.n_tokens, hw.head_dim, hw.bits, out=ky, stream=stream)
+                kvq.dequantize(vc, vs, hw.n_tokens, hw.head_dim, hw.bits, out=vy, stream=stream)
+                a2.record(stream)
+                if it >= args.warmup:
+                    qt.append((a0, a1))
+                    dt.append((a1, a2))
+        stream.synchronize()
+        tq = float(np.mean([x.elapsed_time(y) for x, y in qt])) / 1e3
+        td = float(np.mean([x.elapsed_time(y) for x, y in dt])) / 1e3
+        codec = {"workload": "bulk cache handoff, Llama-3.1-8B shape: 32 layers x 8 kv heads x 32768 tokens x "
+                             "128, K and V, 4-bit group-64, 1% K outlier channels x10",
+                 "bytes": codec_bytes,
+                 "quantize_gbs": codec_bytes / tq / 1e9, "quantize_ms": tq * 1e3,
+                 "quantize_frac": codec_bytes / tq / 1e9 / peak,
+                 "dequantize_gbs": codec_bytes / td / 1e9, "dequantize_ms": td * 1e3,
+                 "dequantize_frac": codec_bytes / td / 1e9 / peak}
+        del kx, vx, kc, vc, ks, vs, ky, vy
+        torch.cuda.empty_cache()
+
+    # ---------------- CPU oracle on a bounded sample (rank 0, N=1 only)
+    cpu = None
+    if rank == 0 and world == 1 and not args.skip_cpu:
+        sample_views = [(a, l) for l in range(0, 32, 8) for a in range(0, 10, 3)][:12]
+        secs, nb = oracle_sample(w, sample_views, dev)
+        cpu = {"value": nb / secs / 1e9, "unit": "GB/s", "cores": 1, "kind": "oracle",
+               "sample": f"{len(sample_views)} (agent, layer) views of the decode workload "
+                         f"(8 kv heads x 4224 tokens each), fp64 oracle attention, single thread"}
+
+    if rank == 0:
+        clocks = clk.summary()
+        line = {
+            "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": t_step * 1e3, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "agents_per_gpu": A, "layers": L, "n_q_heads": w.n_q_heads,
+                       "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "packed_tokens": w.view_len(0),
+                       "window": w.window, "bits": 4, "calls_per_step": "per layer: kvq_append + kvq_decode_attn",
+                       "cuda_graph": True, "l2": "working set per step ~1.9 GB > 126 MB L2, no flush"},
+            "tokens_per_s_per_agent": 1.0 / t_step,
+            "hbm_frac": value / world / peak,
+            "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
+                         "frac": attn_gbs / peak, "traffic": None,
+                         "kernel": "decode_attn_kernel<2> (one kvq_decode_attn per layer, 10 views)",
+                         "bytes_per_launch": attn_layer_bytes, "launch_us": t_attn * 1e6,
+                         "peak_kind": f"{peak_kind} (hbm_gbs)"},
+            "all_views_one_call": {"gbs": all_gbs, "frac": all_gbs / peak, "ms": t_all * 1e3},
+            "codec": codec,
+            "cpu_baseline": cpu,
+            "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                    "ms_per_step": t_e2e * 1e3},
+            "gpu_launches": n_launch_per_step * args.steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--skip-codec", action="store_true")
+    ap.add_argument("--skip-cpu", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    rank, world, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            run_reference(args, rank, world)
+        else:
+            run_ours(args, rank, world, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,209 @@
+/*
+ * kvq.h -- C ABI of the quantized KV-cache library for NVIDIA B200 (sm_100a).
+ *
+ * What the library computes (pages and sections):
+ *  - "QKVShare: Quantized KV-Cache Handoff for Multi-Agent On-Device LLMs",
+ *    Riepilogo Tecnico / Metodologia: an agent hands its KV cache to the next
+ *    one as quantized groups instead of making it re-prefill, and the
+ *    receiver rebuilds full-precision K/V from them before its forward pass
+ *    (kvq_quantize, kvq_dequantize).
+ *  - "Agent Memory Below the Prompt: Persistent Q4 KV Cache for Multi-Agent
+ *    LLM Inference on Edge Devices", Abstract: 4-bit caches are loaded
+ *    directly into the attention layer and several agents' quantized caches
+ *    are attended concurrently (kvq_decode_attn over an array of views).
+ *  - "Coordinated Mixed-Precision KV Cache Quantization for Efficient
+ *    LLM-based Multi-agent Systems", Abstract: each (agent, layer) has its own
+ *    width, recent states keep native precision, and only newly quantized
+ *    blocks take a width while older blocks stay as they are (kvq_view.bits,
+ *    the bf16 recent window, kvq_append).
+ *
+ * Quantization format (the pages leave it open; this is the library's
+ * definition):
+ *  - group = 64 consecutive elements along head_dim of one (head, token) row;
+ *  - mn, mx = min and max of the group in fp32 (a zero is stored as +0.0f);
+ *    s = (mx - mn) / (2^bits - 1), one fp32 round-to-nearest division, s = 0
+ *    when mx == mn;
+ *  - code = clamp(round_half_to_even((x - mn) / s), 0, 2^bits - 1) with
+ *    x - mn and the division each one fp32 round-to-nearest step; all codes
+ *    are 0 when s == 0;
+ *  - code j of a group occupies bits [j*bits, (j+1)*bits) of the group's
+ *    little-endian byte string, least significant bit first; a group is
+ *    8*bits bytes and the groups of a row follow in head_dim order, so a row
+ *    is row_bytes = head_dim*bits/8 bytes;
+ *  - per group one float pair {s, mn} ("scalemin");
+ *  - dequantized value: bf16_round_half_to_even(fmaf((float)code, s, mn));
+ *    attention attends over the affine value mn + s*code without the bf16
+ *    rounding.
+ *  Supported: bits in {2, 3, 4, 8}; head_dim a multiple of 64, at most 256.
+ *  Inputs with NaN or Inf, or whose group range mx - mn overflows fp32, are
+ *  outside the contract.
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned by the caller; views and
+ *    other structs are HOST memory.  The library allocates no device memory,
+ *    never synchronizes the host with the device, and enqueues all work on
+ *    `stream` (a cudaStream_t; NULL means the legacy default stream) in the
+ *    caller's current CUDA device context.
+ *  - Arguments are validated on the host before anything is enqueued; on any
+ *    error nothing is enqueued and outputs are untouched.
+ *  - KVQ_ERR_CUDA reports a failed launch (the CUDA error is left for the
+ *    caller to inspect with cudaGetLastError/cudaPeekAtLastError).
+ *  - Calls that share output or workspace memory and overlap on the GPU race;
+ *    order them on one stream.
+ */
+#ifndef KVQ_H_
+#define KVQ_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVQ_GROUP_SIZE 64
+#define KVQ_MAX_HEAD_DIM 256
+
+typedef enum kvq_status {
+    KVQ_OK = 0,
+    KVQ_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or stride */
+    KVQ_ERR_UNSUPPORTED = 2, /* bits not in {2,3,4,8}, head_dim not 64..256 step 64 */
+    KVQ_ERR_CAPACITY = 3,    /* an append would write past cap_packed */
+    KVQ_ERR_CUDA = 4         /* a kernel launch or device query failed */
+} kvq_status;
+
+/* Static, NUL-terminated name of a status code ("unknown status" otherwise). */
+const char *kvq_status_string(int32_t status);
+
+/* ABI version of this header (incremented on any incompatible change). */
+int32_t kvq_abi_version(void);
+
+/*
+ * kvq_quantize -- group-wise affine quantization of bf16 K or V rows
+ * (QKVShare, Metodologia: the quantized card; Agent Memory, Abstract: 4-bit
+ * format; CoMixKV, Abstract: widths per (agent, layer)).
+ *
+ *  x          bf16 input, element (h, t, d) at x[h*x_head_stride +
+ *             t*x_tok_stride + d] (strides in ELEMENTS; d contiguous).
+ *             x must be 16-byte aligned and both strides multiples of 8.
+ *  n_heads, n_tokens, head_dim, bits   sizes; n_heads*n_tokens may be 0
+ *             (nothing is enqueued).
+ *  codes      u8 output, row (h, t) at codes + (h*out_head_cap + t)*row_bytes;
+ *             16-byte aligned.
+ *  scalemin   float output, group g of row (h, t) at
+ *             scalemin + ((h*out_head_cap + t)*(head_dim/64) + g)*2, holding
+ *             {s, mn}; 8-byte aligned.
+ *  out_head_cap  rows per head in codes/scalemin, >= n_tokens.
+ * Result: codes and scalemin are bit-exact functions of x (see format).
+ */
+kvq_status kvq_quantize(const void *x, int64_t x_head_stride, int64_t x_tok_stride,
+                        int32_t n_heads, int64_t n_tokens, int32_t head_dim, int32_t bits,
+                        void *codes, float *scalemin, int64_t out_head_cap, void *stream);
+
+/*
+ * kvq_dequantize -- inverse of kvq_quantize into bf16 (QKVShare, Metodologia,
+ * "Percorso di Iniezione": full-precision past_key_values rebuilt from the
+ * quantized card before the receiver's forward pass).
+ *
+ *  codes, scalemin, in_head_cap   as written by kvq_quantize (same alignment).
+ *  y          bf16 output, element (h, t, d) at y[h*y_head_stride +
+ *             t*y_tok_stride + d]; 16-byte aligned, strides multiples of 8.
+ * Result: y = bf16_rne(fmaf(code, s, mn)), bit-exact.
+ */
+kvq_status kvq_dequantize(const void *codes, const float *scalemin, int64_t in_head_cap,
+                          int32_t n_heads, int64_t n_tokens, int32_t head_dim, int32_t bits,
+                          void *y, int64_t y_head_stride, int64_t y_tok_stride, void *stream);
+
+/*
+ * One (agent, layer) KV cache: n_packed quantized tokens followed by
+ * n_window bf16 recent-window tokens (CoMixKV, Abstract: recent states keep
+ * native precision).  All pointers are device memory owned by the caller.
+ *
+ *  bits          width of this view's packed tokens (2, 3, 4 or 8).
+ *  n_packed      packed tokens in use, 0 <= n_packed <= cap_packed.
+ *  cap_packed    packed rows per KV head; must be even.
+ *  n_window      valid window tokens, 0 <= n_window <= cap_window.
+ *  cap_window    window ring slots per KV head (W); 0 = no window.
+ *  window_head   ring slot of the oldest window token; window token i
+ *                (0 = oldest) lives in slot (window_head + i) % cap_window.
+ *  k_codes, v_codes        u8 [n_kv_heads][cap_packed][row_bytes], 16-B aligned.
+ *  k_scalemin, v_scalemin  float [n_kv_heads][cap_packed][head_dim/64][2], 16-B aligned.
+ *  k_window, v_window      bf16 [n_kv_heads][cap_window][head_dim], 16-B aligned
+ *                          (may be NULL when cap_window == 0).
+ * The sequence a query attends is packed tokens 0..n_packed-1, then window
+ * tokens oldest to newest.
+ */
+typedef struct kvq_view {
+    int32_t bits;
+    int32_t n_window;
+    int32_t cap_window;
+    int32_t window_head;
+    int64_t n_packed;
+    int64_t cap_packed;
+    void *k_codes;
+    void *v_codes;
+    float *k_scalemin;
+    float *v_scalemin;
+    void *k_window;
+    void *v_window;
+} kvq_view;
+
+/*
+ * kvq_append -- add one new token to each of n_views views (one decode step
+ * of several agents or layers in a single launch).  CoMixKV, Abstract: the
+ * new token enters in native precision; when the window is full its oldest
+ * token is quantized at the view's CURRENT bits and appended to the packed
+ * part, while earlier packed tokens are never touched.  With cap_window == 0
+ * the new token is quantized immediately.
+ *
+ *  views      HOST array, read and then updated in place (n_packed, n_window,
+ *             window_head) to describe the state after the append.  Each view
+ *             must have distinct device buffers from every other view.
+ *  k_new, v_new  bf16 [n_views][n_kv_heads][head_dim] device arrays, 16-B aligned.
+ * Errors: KVQ_ERR_CAPACITY if any view would need to flush while
+ * n_packed == cap_packed (nothing is enqueued and no view is changed).
+ */
+kvq_status kvq_append(kvq_view *views, int32_t n_views, int32_t n_kv_heads, int32_t head_dim,
+                      const void *k_new, const void *v_new, void *stream);
+
+/*
+ * Bytes of device workspace kvq_decode_attn needs for these views on the
+ * current device (0 when the arguments are invalid).  The workspace must be
+ * zero-filled once before its first use; every completed call leaves it
+ * ready for the next one.  Its first 4 bytes are a device status word: 0
+ * normally; 1 if a bounded wait for a copy into shared memory expired, in
+ * which case the outputs of that call are not valid.
+ */
+size_t kvq_decode_attn_workspace_size(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
+                                      int32_t n_kv_heads, int32_t head_dim);
+
+/*
+ * kvq_decode_attn -- batched split-K decode attention straight over several
+ * views' packed caches and bf16 windows (Agent Memory, Abstract:
+ * BatchQuantizedKVCache, caches loaded directly into attention; QKVShare,
+ * Significato: the fused quantized attention kernel the prototype deferred).
+ *
+ *  views      HOST array of n_views views (any mix of bits and lengths; each
+ *             view must have n_packed + n_window >= 1).
+ *  n_q_heads, n_kv_heads   n_q_heads % n_kv_heads == 0; query head h reads
+ *             KV head h / (n_q_heads / n_kv_heads).
+ *  q          bf16 [n_views][n_q_heads][head_dim] device array, 16-B aligned.
+ *  softmax_scale   logits are softmax_scale * (q . k), e.g. 1/sqrt(head_dim).
+ *  out        float [n_views][n_q_heads][head_dim] device array, 16-B aligned:
+ *             out = sum_t softmax_t * v_t over packed-then-window tokens.
+ *  workspace  device scratch of at least kvq_decode_attn_workspace_size(...)
+ *             bytes, 256-B aligned, zero-filled before first use.
+ * The result is deterministic: the same inputs on the same device give the
+ * same bits (no floating-point atomics; partial results merge in a fixed
+ * order).
+ */
+kvq_status kvq_decode_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
+                           int32_t n_kv_heads, int32_t head_dim, const void *q,
+                           float softmax_scale, float *out, void *workspace,
+                           size_t workspace_bytes, void *stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H_ */

@@ -1,1 +1,257 @@
-"""Quantized KV-cache handoff and decode attention for B200 (placeholder)."""
+"""Quantized KV-cache handoff and decode attention for NVIDIA B200 (sm_100a).
+
+A thin binding over the C ABI of ``libkvq.so`` (declared in ``include/kvq.h``).
+Every computation of the method runs in the library's CUDA kernels; this module
+only marshals torch tensors (device memory and the current stream) into the C
+calls.  There is no CPU fallback: if the library is missing, every entry point
+raises.
+
+Entry points (same names as the C ABI, without the ``kvq_`` prefix):
+  quantize, dequantize          -- bf16 rows <-> packed b-bit codes + {s, mn}
+  View, append                  -- one (agent, layer) cache; add a decode token
+  decode_attn, workspace_size   -- batched split-K attention over many views
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+from . import workloads  # noqa: F401  (seeded input generators)
+
+__all__ = ["quantize", "dequantize", "View", "append", "decode_attn", "workspace_size",
+           "KvqError", "lib", "row_bytes", "GROUP"]
+
+GROUP = 64
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB_PATH = os.path.join(_HERE, "libkvq.so")
+_lib = None
+
+KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_CUDA = range(5)
+
+
+class KvqError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        name = lib().kvq_status_string(status).decode()
+        super().__init__(f"{where}: {name}")
+        self.status = status
+
+
+class CView(ctypes.Structure):
+    """ctypes mirror of ``kvq_view``."""
+    _fields_ = [("bits", ctypes.c_int32), ("n_window", ctypes.c_int32),
+                ("cap_window", ctypes.c_int32), ("window_head", ctypes.c_int32),
+                ("n_packed", ctypes.c_int64), ("cap_packed", ctypes.c_int64),
+                ("k_codes", ctypes.c_void_p), ("v_codes", ctypes.c_void_p),
+                ("k_scalemin", ctypes.c_void_p), ("v_scalemin", ctypes.c_void_p),
+                ("k_window", ctypes.c_void_p), ("v_window", ctypes.c_void_p)]
+
+
+def lib():
+    """The loaded ``libkvq.so`` (raises if it has not been built)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(_LIB_PATH):
+            raise RuntimeError(f"libkvq.so not found at {_LIB_PATH}; build it with "
+                               "`python -m quantized_kv_cache_dequantize_b200.build`")
+        L = ctypes.CDLL(_LIB_PATH)
+        P, i32, i64, f32, sz = ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float, ctypes.c_size_t
+        L.kvq_status_string.argtypes = [i32]
+        L.kvq_status_string.restype = ctypes.c_char_p
+        L.kvq_abi_version.argtypes = []
+        L.kvq_abi_version.restype = i32
+        L.kvq_quantize.argtypes = [P, i64, i64, i32, i64, i32, i32, P, P, i64, P]
+        L.kvq_quantize.restype = i32
+        L.kvq_dequantize.argtypes = [P, P, i64, i32, i64, i32, i32, P, i64, i64, P]
+        L.kvq_dequantize.restype = i32
+        L.kvq_append.argtypes = [ctypes.POINTER(CView), i32, i32, i32, P, P, P]
+        L.kvq_append.restype = i32
+        L.kvq_decode_attn_workspace_size.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32]
+        L.kvq_decode_attn_workspace_size.restype = sz
+        L.kvq_decode_attn.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, f32, P, P, sz, P]
+        L.kvq_decode_attn.restype = i32
+        _lib = L
+    return _lib
+
+
+def row_bytes(head_dim: int, bits: int) -> int:
+    return head_dim // 8 * bits
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _check(status: int, where: str):
+    if status != KVQ_OK:
+        raise KvqError(status, where)
+
+
+def _ptr(t):
+    return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+# -------------------------------------------------------------- codec -----
+
+def quantize(x: torch.Tensor, bits: int, codes: torch.Tensor | None = None,
+             scalemin: torch.Tensor | None = None, head_cap: int | None = None, stream=None):
+    """x: bf16 CUDA tensor [H, T, D] (d contiguous; head/token strides free).
+
+    Returns (codes u8 [H, cap, D*bits/8], scalemin f32 [H, cap, D/64, 2]);
+    pass preallocated outputs to write in place."""
+    if x.dtype != torch.bfloat16 or x.dim() != 3 or x.stride(2) != 1:
+        raise ValueError("x must be a bf16 [H, T, D] tensor with contiguous last dim")
+    H, T, D = x.shape
+    cap = head_cap if head_cap is not None else (codes.shape[1] if codes is not None else T)
+    if codes is None:
+        codes = torch.empty((H, cap, row_bytes(D, bits)), dtype=torch.uint8, device=x.device)
+    if scalemin is None:
+        scalemin = torch.empty((H, cap, D // GROUP, 2), dtype=torch.float32, device=x.device)
+    _check(lib().kvq_quantize(_ptr(x), x.stride(0), x.stride(1), H, T, D, bits,
+                              _ptr(codes), _ptr(scalemin), cap, _stream(stream)), "kvq_quantize")
+    return codes, scalemin
+
+
+def dequantize(codes: torch.Tensor, scalemin: torch.Tensor, n_tokens: int, head_dim: int, bits: int,
+               out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """Inverse of quantize: bf16 [H, n_tokens, D] (or into ``out``)."""
+    H, cap = codes.shape[0], codes.shape[1]
+    if out is None:
+        out = torch.empty((H, n_tokens, head_dim), dtype=torch.bfloat16, device=codes.device)
+    _check(lib().kvq_dequantize(_ptr(codes), _ptr(scalemin), cap, H, n_tokens, head_dim, bits,
+                                _ptr(out), out.stride(0), out.stride(1), _stream(stream)),
+           "kvq_dequantize")
+    return out
+
+
+# -------------------------------------------------------------- views -----
+
+class View:
+    """One (agent, layer) cache: packed tokens + bf16 recent-window ring.
+
+    Owns (or borrows) the torch tensors behind a ``kvq_view``:
+      k_codes, v_codes          u8  [H_kv, cap_packed, D*bits/8]
+      k_scalemin, v_scalemin    f32 [H_kv, cap_packed, D/64, 2]
+      k_window, v_window        bf16 [H_kv, cap_window, D]
+    """
+
+    def __init__(self, n_kv_heads: int, head_dim: int, bits: int, cap_packed: int, cap_window: int,
+                 device="cuda", tensors: dict | None = None):
+        if cap_packed % 2:
+            cap_packed += 1
+        self.n_kv_heads, self.head_dim, self.bits = n_kv_heads, head_dim, bits
+        t = tensors or {}
+        rb = row_bytes(head_dim, bits)
+        ng = head_dim // GROUP
+        self.k_codes = t.get("k_codes", torch.zeros((n_kv_heads, cap_packed, rb), dtype=torch.uint8, device=device))
+        self.v_codes = t.get("v_codes", torch.zeros((n_kv_heads, cap_packed, rb), dtype=torch.uint8, device=device))
+        self.k_scalemin = t.get("k_scalemin", torch.zeros((n_kv_heads, cap_packed, ng, 2), dtype=torch.float32,
+                                                          device=device))
+        self.v_scalemin = t.get("v_scalemin", torch.zeros((n_kv_heads, cap_packed, ng, 2), dtype=torch.float32,
+                                                          device=device))
+        self.k_window = t.get("k_window", torch.zeros((n_kv_heads, cap_window, head_dim), dtype=torch.bfloat16,
+                                                      device=device))
+        self.v_window = t.get("v_window", torch.zeros((n_kv_heads, cap_window, head_dim), dtype=torch.bfloat16,
+                                                      device=device))
+        self.c = CView(bits=bits, n_window=0, cap_window=cap_window, window_head=0, n_packed=0,
+                       cap_packed=cap_packed)
+        self._sync_ptrs()
+
+    def _sync_ptrs(self):
+        c = self.c
+        c.k_codes, c.v_codes = self.k_codes.data_ptr(), self.v_codes.data_ptr()
+        c.k_scalemin, c.v_scalemin = self.k_scalemin.data_ptr(), self.v_scalemin.data_ptr()
+        c.k_window = self.k_window.data_ptr() if self.c.cap_window else None
+        c.v_window = self.v_window.data_ptr() if self.c.cap_window else None
+
+    # state accessors
+    @property
+    def n_packed(self) -> int:
+        return self.c.n_packed
+
+    @property
+    def n_window(self) -> int:
+        return self.c.n_window
+
+    @property
+    def cap_window(self) -> int:
+        return self.c.cap_window
+
+    @property
+    def window_head(self) -> int:
+        return self.c.window_head
+
+    def set_state(self, n_packed: int, n_window: int, window_head: int = 0, bits: int | None = None):
+        self.c.n_packed, self.c.n_window, self.c.window_head = n_packed, n_window, window_head
+        if bits is not None:
+            self.c.bits = self.bits = bits
+
+    def fill_packed(self, k: torch.Tensor, v: torch.Tensor, stream=None):
+        """Quantize bf16 K/V [H, T, D] into packed rows [0, T) (prefill handoff)."""
+        T = k.shape[1]
+        quantize(k, self.bits, self.k_codes, self.k_scalemin, stream=stream)
+        quantize(v, self.bits, self.v_codes, self.v_scalemin, stream=stream)
+        self.c.n_packed = T
+
+    def fill_window(self, k: torch.Tensor, v: torch.Tensor, head: int = 0):
+        """Place bf16 K/V [H, n, D] as the window, oldest first, starting at ring slot ``head``."""
+        n = k.shape[1]
+        W = self.c.cap_window
+        if n > W:
+            raise ValueError("more window tokens than ring slots")
+        idx = (torch.arange(n, device=k.device) + head) % W
+        self.k_window[:, idx] = k
+        self.v_window[:, idx] = v
+        self.c.n_window, self.c.window_head = n, head
+
+
+def _view_array(views):
+    arr = (CView * len(views))()
+    for i, v in enumerate(views):
+        arr[i] = v.c
+    return arr
+
+
+def append(views, k_new: torch.Tensor, v_new: torch.Tensor, stream=None):
+    """Append one token per view: k_new, v_new bf16 [n_views, H_kv, D]."""
+    views = list(views)
+    arr = _view_array(views)
+    H, D = views[0].n_kv_heads, views[0].head_dim
+    _check(lib().kvq_append(arr, len(views), H, D, _ptr(k_new), _ptr(v_new), _stream(stream)),
+           "kvq_append")
+    for i, v in enumerate(views):
+        v.c.n_packed, v.c.n_window, v.c.window_head = arr[i].n_packed, arr[i].n_window, arr[i].window_head
+
+
+def workspace_size(views, n_q_heads: int) -> int:
+    views = list(views)
+    arr = _view_array(views)
+    return int(lib().kvq_decode_attn_workspace_size(arr, len(views), n_q_heads, views[0].n_kv_heads,
+                                                    views[0].head_dim))
+
+
+def new_workspace(views, n_q_heads: int, device="cuda") -> torch.Tensor:
+    """Zero-filled workspace of the size kvq_decode_attn needs for these views."""
+    n = workspace_size(views, n_q_heads)
+    if n == 0:
+        raise KvqError(KVQ_ERR_INVALID_ARG, "kvq_decode_attn_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def decode_attn(views, q: torch.Tensor, softmax_scale: float, out: torch.Tensor | None = None,
+                workspace: torch.Tensor | None = None, stream=None, _arr=None) -> torch.Tensor:
+    """q: bf16 [n_views, H_q, D] -> fp32 [n_views, H_q, D]."""
+    views = list(views)
+    n, Hq, D = q.shape
+    arr = _arr if _arr is not None else _view_array(views)
+    if workspace is None:
+        workspace = new_workspace(views, Hq, device=q.device)
+    if out is None:
+        out = torch.empty((n, Hq, D), dtype=torch.float32, device=q.device)
+    _check(lib().kvq_decode_attn(arr, len(views), Hq, views[0].n_kv_heads, D, _ptr(q), float(softmax_scale),
+                                 _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
+           "kvq_decode_attn")
+    return out

@@ -1,0 +1,391 @@
+// kvq.cu -- C-ABI entry points of libkvq (declared in include/kvq.h):
+// argument validation on the host, work planning, and kernel launches for
+// sm_100a.  Nothing here allocates device memory or synchronizes.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstdint>
+#include <cstdlib>
+#include <cstring>
+#include <vector>
+
+#include "kvq.h"
+#include "kvq_attn.cuh"
+#include "kvq_codec.cuh"
+
+#define KVQ_API extern "C" __attribute__((visibility("default")))
+
+namespace {
+
+constexpr int kAbiVersion = 1;
+
+bool bits_supported(int32_t bits) { return bits == 2 || bits == 3 || bits == 4 || bits == 8; }
+bool head_dim_supported(int32_t d) { return d >= 64 && d <= KVQ_MAX_HEAD_DIM && d % 64 == 0; }
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+int64_t row_bytes(int32_t head_dim, int32_t bits) { return (int64_t)head_dim / 8 * bits; }
+
+int device_sm_count() {
+    int dev = 0, sms = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return 148;
+    }
+    if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || sms <= 0) {
+        (void)cudaGetLastError();
+        return 148;
+    }
+    return sms;
+}
+
+template <int B, int NG>
+void launch_codec(bool quant, const kvq::CodecArgs &a, cudaStream_t st) {
+    const int64_t groups = a.n_tokens * NG;
+    const int64_t warps_needed = (groups + 15) / 16;
+    const int sms = device_sm_count();
+    int64_t blocks = (warps_needed + 7) / 8;  // 8 warps per block
+    const int64_t cap = std::max<int64_t>(1, (int64_t)sms * 8 / std::max(1, a.n_heads));
+    blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, std::max<int64_t>(cap, 4)));
+    dim3 grid((unsigned)blocks, (unsigned)a.n_heads);
+    if (quant)
+        kvq::quantize_kernel<B, NG><<<grid, 256, 0, st>>>(a);
+    else
+        kvq::dequantize_kernel<B, NG><<<grid, 256, 0, st>>>(a);
+}
+
+template <int B>
+void launch_codec_ng(bool quant, int ng, const kvq::CodecArgs &a, cudaStream_t st) {
+    switch (ng) {
+        case 1: launch_codec<B, 1>(quant, a, st); break;
+        case 2: launch_codec<B, 2>(quant, a, st); break;
+        case 3: launch_codec<B, 3>(quant, a, st); break;
+        default: launch_codec<B, 4>(quant, a, st); break;
+    }
+}
+
+kvq_status codec(bool quant, const void *x, int64_t hs, int64_t ts, int32_t n_heads, int64_t n_tokens,
+                 int32_t head_dim, int32_t bits, const void *codes, const float *scalemin, int64_t cap,
+                 void *stream) {
+    if (!bits_supported(bits) || !head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
+    if (n_heads < 0 || n_tokens < 0 || cap < n_tokens || n_heads > 65535) return KVQ_ERR_INVALID_ARG;
+    if (n_heads == 0 || n_tokens == 0) return KVQ_OK;
+    if (!x || !codes || !scalemin) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(x, 16) || !aligned(codes, 16) || !aligned(scalemin, 8)) return KVQ_ERR_INVALID_ARG;
+    if (hs < 0 || ts < 0 || hs % 8 || ts % 8) return KVQ_ERR_INVALID_ARG;
+    // dequantize writes rows: consecutive tokens and heads may not share a row
+    if (!quant && ((n_tokens > 1 && ts < head_dim) || (n_heads > 1 && hs < head_dim))) return KVQ_ERR_INVALID_ARG;
+    kvq::CodecArgs a;
+    a.x = static_cast<const uint16_t *>(x);
+    a.x_head_stride = hs;
+    a.x_tok_stride = ts;
+    a.n_tokens = n_tokens;
+    a.n_heads = n_heads;
+    a.codes = static_cast<uint8_t *>(const_cast<void *>(codes));
+    a.scalemin = const_cast<float *>(scalemin);
+    a.head_cap = cap;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int ng = head_dim / 64;
+    switch (bits) {
+        case 2: launch_codec_ng<2>(quant, ng, a, st); break;
+        case 3: launch_codec_ng<3>(quant, ng, a, st); break;
+        case 4: launch_codec_ng<4>(quant, ng, a, st); break;
+        default: launch_codec_ng<8>(quant, ng, a, st); break;
+    }
+    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+// ------------------------------------------------------ decode planning ---
+
+struct AttnLaunch {
+    int v0, v1;          // views [v0, v1)
+    int total_chunks;
+};
+
+struct AttnPlan {
+    int chunk = 0;
+    int ring_bytes = 0;
+    size_t smem = 0;
+    int head_blocks = 0;
+    std::vector<AttnLaunch> launches;
+    size_t counters_off = 0, partials_off = 0, total = 0;
+};
+
+int env_int(const char *name, int dflt) {
+    const char *s = std::getenv(name);
+    if (!s || !*s) return dflt;
+    const long v = std::strtol(s, nullptr, 10);
+    return v > 0 ? (int)v : dflt;
+}
+
+kvq_status validate_views(const kvq_view *views, int32_t n_views, int32_t head_dim, bool need_nonempty) {
+    if (!views || n_views <= 0) return KVQ_ERR_INVALID_ARG;
+    for (int i = 0; i < n_views; ++i) {
+        const kvq_view &v = views[i];
+        if (v.n_packed < 0 || v.cap_packed < v.n_packed || (v.cap_packed & 1)) return KVQ_ERR_INVALID_ARG;
+        if (v.cap_packed > INT32_MAX) return KVQ_ERR_INVALID_ARG;
+        if (v.cap_window < 0 || v.n_window < 0 || v.n_window > v.cap_window) return KVQ_ERR_INVALID_ARG;
+        if (v.cap_window > 0 && (v.window_head < 0 || v.window_head >= v.cap_window)) return KVQ_ERR_INVALID_ARG;
+        if (need_nonempty && v.n_packed + v.n_window <= 0) return KVQ_ERR_INVALID_ARG;
+        if (v.cap_packed > 0 || v.n_packed > 0) {
+            if (!bits_supported(v.bits)) return KVQ_ERR_UNSUPPORTED;
+            if (!v.k_codes || !v.v_codes || !v.k_scalemin || !v.v_scalemin) return KVQ_ERR_INVALID_ARG;
+            if (!aligned(v.k_codes, 16) || !aligned(v.v_codes, 16) || !aligned(v.k_scalemin, 16) ||
+                !aligned(v.v_scalemin, 16))
+                return KVQ_ERR_INVALID_ARG;
+        }
+        if (v.cap_window > 0) {
+            if (!v.k_window || !v.v_window || !aligned(v.k_window, 16) || !aligned(v.v_window, 16))
+                return KVQ_ERR_INVALID_ARG;
+        }
+    }
+    (void)head_dim;
+    return KVQ_OK;
+}
+
+kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, int32_t n_kv_heads,
+                     int32_t head_dim, AttnPlan &plan) {
+    if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
+    if (n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads || n_kv_heads > 65535)
+        return KVQ_ERR_INVALID_ARG;
+    const kvq_status vs = validate_views(views, n_views, head_dim, true);
+    if (vs != KVQ_OK) return vs;
+    const int ng = head_dim / 64;
+    const int group = n_q_heads / n_kv_heads;
+    plan.head_blocks = (group + kvq::kHeadsPerCta - 1) / kvq::kHeadsPerCta;
+    if (plan.head_blocks > 65535) return KVQ_ERR_UNSUPPORTED;
+
+    // chunk size: aim for ~4 CTAs per SM over the whole call, in 16-token
+    // tiles, at least 256 tokens so a CTA amortises its set-up
+    int64_t total_tokens = 0;
+    uint32_t stage_max = 0;
+    for (int i = 0; i < n_views; ++i) {
+        total_tokens += views[i].n_packed + views[i].n_window;
+        if (views[i].n_packed > 0)
+            stage_max = std::max<uint32_t>(stage_max, (uint32_t)(32 * row_bytes(head_dim, views[i].bits) + 256 * ng));
+        if (views[i].n_window > 0) stage_max = std::max<uint32_t>(stage_max, (uint32_t)(32 * head_dim));
+    }
+    total_tokens *= (int64_t)n_kv_heads * plan.head_blocks;
+    const int64_t target_ctas = (int64_t)device_sm_count() * 4;
+    int64_t chunk = (total_tokens + target_ctas - 1) / target_ctas;
+    chunk = std::max<int64_t>(256, std::min<int64_t>(chunk, 8192));
+    chunk = (chunk + 63) / 64 * 64;
+    plan.chunk = env_int("KVQ_CHUNK_TOKENS", (int)chunk);
+    plan.chunk = std::max(16, plan.chunk / 16 * 16);
+
+    int ring = std::max<int>(16384, (int)(2 * stage_max));
+    ring = std::max(ring, 64 + 32 * head_dim);
+    ring = (ring + 127) / 128 * 128;
+    plan.ring_bytes = ring;
+    const size_t header = (size_t)((8 * head_dim * 2 + 8 * ng * 4 + kvq::kAttnWarps * kvq::kMaxStages * 8 + 16 + 127) & ~127);
+    plan.smem = header + (size_t)kvq::kAttnWarps * ring;
+    if (plan.smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;
+
+    int64_t max_chunks = 0;
+    int max_views = 0;
+    for (int v0 = 0; v0 < n_views; v0 += kvq::kAttnMaxViews) {
+        const int v1 = std::min<int>(n_views, v0 + kvq::kAttnMaxViews);
+        int64_t chunks = 0;
+        for (int i = v0; i < v1; ++i) {
+            chunks += (views[i].n_packed + plan.chunk - 1) / plan.chunk;
+            chunks += (views[i].n_window + plan.chunk - 1) / plan.chunk;
+        }
+        if (chunks > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
+        plan.launches.push_back({v0, v1, (int)chunks});
+        max_chunks = std::max(max_chunks, chunks);
+        max_views = std::max(max_views, v1 - v0);
+    }
+    const size_t units = (size_t)max_views * n_kv_heads * plan.head_blocks;
+    plan.counters_off = 256;
+    plan.partials_off = plan.counters_off + (units * 4 + 255) / 256 * 256;
+    const size_t part_floats = (size_t)max_chunks * n_kv_heads * plan.head_blocks * kvq::kHeadsPerCta * (head_dim + 2);
+    plan.total = plan.partials_off + part_floats * 4;
+    return KVQ_OK;
+}
+
+template <int NG>
+kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n_q_heads, int32_t n_kv_heads,
+                          const void *q, float scale, float *out, uint8_t *ws, cudaStream_t st) {
+    static int configured_smem[64] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (dev < 64 && configured_smem[dev] < (int)plan.smem) {
+        if (cudaFuncSetAttribute(kvq::decode_attn_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)plan.smem) != cudaSuccess)
+            return KVQ_ERR_CUDA;
+        configured_smem[dev] = (int)plan.smem;
+    }
+    kvq::AttnParams prm;
+    std::memset(&prm, 0, sizeof prm);
+    prm.q = static_cast<const uint16_t *>(q);
+    prm.out = out;
+    prm.status = reinterpret_cast<uint32_t *>(ws);
+    prm.counters = reinterpret_cast<uint32_t *>(ws + plan.counters_off);
+    prm.partials = reinterpret_cast<float *>(ws + plan.partials_off);
+    prm.timeout_ns = 2000000000ull;
+    prm.scale_log2 = scale * 1.4426950408889634f;
+    prm.n_q_heads = n_q_heads;
+    prm.n_kv_heads = n_kv_heads;
+    prm.group = n_q_heads / n_kv_heads;
+    prm.head_blocks = plan.head_blocks;
+    prm.chunk = plan.chunk;
+    prm.ring_bytes = plan.ring_bytes;
+    for (const AttnLaunch &L : plan.launches) {
+        prm.n_views = L.v1 - L.v0;
+        int begin = 0;
+        for (int i = L.v0; i < L.v1; ++i) {
+            const kvq_view &v = views[i];
+            kvq::AttnView &d = prm.views[i - L.v0];
+            d.codes[0] = static_cast<const uint8_t *>(v.k_codes);
+            d.codes[1] = static_cast<const uint8_t *>(v.v_codes);
+            d.scalemin[0] = v.k_scalemin;
+            d.scalemin[1] = v.v_scalemin;
+            d.window[0] = static_cast<const uint16_t *>(v.k_window);
+            d.window[1] = static_cast<const uint16_t *>(v.v_window);
+            d.cap_packed = v.cap_packed;
+            d.n_packed = (int32_t)v.n_packed;
+            d.n_window = v.n_window;
+            d.cap_window = v.cap_window;
+            d.window_head = v.window_head;
+            d.bits = v.n_packed > 0 ? v.bits : 4;
+            d.n_chunks_packed = (int32_t)((v.n_packed + plan.chunk - 1) / plan.chunk);
+            d.n_chunks = d.n_chunks_packed + (v.n_window + plan.chunk - 1) / plan.chunk;
+            d.chunk_begin = begin;
+            d.view_index = i;
+            begin += d.n_chunks;
+        }
+        dim3 grid((unsigned)L.total_chunks, (unsigned)n_kv_heads, (unsigned)plan.head_blocks);
+        kvq::decode_attn_kernel<NG><<<grid, kvq::kAttnThreads, plan.smem, st>>>(prm);
+        if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+    }
+    return KVQ_OK;
+}
+
+}  // namespace
+
+// ================================================================ C ABI ===
+
+KVQ_API const char *kvq_status_string(int32_t status) {
+    switch (status) {
+        case KVQ_OK: return "KVQ_OK";
+        case KVQ_ERR_INVALID_ARG: return "KVQ_ERR_INVALID_ARG";
+        case KVQ_ERR_UNSUPPORTED: return "KVQ_ERR_UNSUPPORTED";
+        case KVQ_ERR_CAPACITY: return "KVQ_ERR_CAPACITY";
+        case KVQ_ERR_CUDA: return "KVQ_ERR_CUDA";
+        default: return "unknown status";
+    }
+}
+
+KVQ_API int32_t kvq_abi_version(void) { return kAbiVersion; }
+
+KVQ_API kvq_status kvq_quantize(const void *x, int64_t x_head_stride, int64_t x_tok_stride, int32_t n_heads,
+                                int64_t n_tokens, int32_t head_dim, int32_t bits, void *codes, float *scalemin,
+                                int64_t out_head_cap, void *stream) {
+    return codec(true, x, x_head_stride, x_tok_stride, n_heads, n_tokens, head_dim, bits, codes, scalemin,
+                 out_head_cap, stream);
+}
+
+KVQ_API kvq_status kvq_dequantize(const void *codes, const float *scalemin, int64_t in_head_cap, int32_t n_heads,
+                                  int64_t n_tokens, int32_t head_dim, int32_t bits, void *y, int64_t y_head_stride,
+                                  int64_t y_tok_stride, void *stream) {
+    return codec(false, y, y_head_stride, y_tok_stride, n_heads, n_tokens, head_dim, bits, codes, scalemin,
+                 in_head_cap, stream);
+}
+
+KVQ_API kvq_status kvq_append(kvq_view *views, int32_t n_views, int32_t n_kv_heads, int32_t head_dim,
+                              const void *k_new, const void *v_new, void *stream) {
+    if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
+    if (n_kv_heads <= 0 || n_kv_heads > 65535) return KVQ_ERR_INVALID_ARG;
+    const kvq_status vs = validate_views(views, n_views, head_dim, false);
+    if (vs != KVQ_OK) return vs;
+    if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return KVQ_ERR_INVALID_ARG;
+    // first pass: every view must be able to take the token
+    for (int i = 0; i < n_views; ++i) {
+        const kvq_view &v = views[i];
+        const bool flush = v.cap_window == 0 || v.n_window == v.cap_window;
+        if (flush) {
+            if (!bits_supported(v.bits)) return KVQ_ERR_UNSUPPORTED;
+            if (v.n_packed >= v.cap_packed) return KVQ_ERR_CAPACITY;
+        }
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const int ng = head_dim / 64;
+    for (int v0 = 0; v0 < n_views; v0 += kvq::kAppendMaxViews) {
+        const int v1 = std::min<int>(n_views, v0 + kvq::kAppendMaxViews);
+        kvq::AppendArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.k_new = static_cast<const uint16_t *>(k_new) + (int64_t)v0 * n_kv_heads * head_dim;
+        a.v_new = static_cast<const uint16_t *>(v_new) + (int64_t)v0 * n_kv_heads * head_dim;
+        a.n_views = v1 - v0;
+        a.n_kv_heads = n_kv_heads;
+        for (int i = v0; i < v1; ++i) {
+            const kvq_view &v = views[i];
+            kvq::AppendView &d = a.views[i - v0];
+            d.codes[0] = static_cast<uint8_t *>(v.k_codes);
+            d.codes[1] = static_cast<uint8_t *>(v.v_codes);
+            d.scalemin[0] = v.k_scalemin;
+            d.scalemin[1] = v.v_scalemin;
+            d.window[0] = static_cast<uint16_t *>(v.k_window);
+            d.window[1] = static_cast<uint16_t *>(v.v_window);
+            d.cap_packed = v.cap_packed;
+            d.cap_window = v.cap_window;
+            d.bits = v.bits;
+            d.packed_row = v.n_packed;
+            if (v.cap_window == 0) {
+                d.flush = 1;
+                d.slot = -1;
+            } else if (v.n_window == v.cap_window) {
+                d.flush = 1;
+                d.slot = v.window_head;
+            } else {
+                d.flush = 0;
+                d.slot = (v.window_head + v.n_window) % v.cap_window;
+            }
+        }
+        dim3 grid((unsigned)(v1 - v0), (unsigned)n_kv_heads, 2);
+        switch (ng) {
+            case 1: kvq::append_kernel<1><<<grid, 32, 0, st>>>(a); break;
+            case 2: kvq::append_kernel<2><<<grid, 32, 0, st>>>(a); break;
+            case 3: kvq::append_kernel<3><<<grid, 32, 0, st>>>(a); break;
+            default: kvq::append_kernel<4><<<grid, 32, 0, st>>>(a); break;
+        }
+        if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+    }
+    // the launch is enqueued: advance the host-side counters
+    for (int i = 0; i < n_views; ++i) {
+        kvq_view &v = views[i];
+        if (v.cap_window == 0) {
+            v.n_packed += 1;
+        } else if (v.n_window == v.cap_window) {
+            v.n_packed += 1;
+            v.window_head = (v.window_head + 1) % v.cap_window;
+        } else {
+            v.n_window += 1;
+        }
+    }
+    return KVQ_OK;
+}
+
+KVQ_API size_t kvq_decode_attn_workspace_size(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
+                                              int32_t n_kv_heads, int32_t head_dim) {
+    AttnPlan plan;
+    if (plan_attn(views, n_views, n_q_heads, n_kv_heads, head_dim, plan) != KVQ_OK) return 0;
+    return plan.total;
+}
+
+KVQ_API kvq_status kvq_decode_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, int32_t n_kv_heads,
+                                   int32_t head_dim, const void *q, float softmax_scale, float *out, void *workspace,
+                                   size_t workspace_bytes, void *stream) {
+    AttnPlan plan;
+    const kvq_status ps = plan_attn(views, n_views, n_q_heads, n_kv_heads, head_dim, plan);
+    if (ps != KVQ_OK) return ps;
+    if (!q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
+    if (workspace_bytes < plan.total) return KVQ_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    switch (head_dim / 64) {
+        case 1: return launch_attn_ng<1>(plan, views, n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st);
+        case 2: return launch_attn_ng<2>(plan, views, n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st);
+        case 3: return launch_attn_ng<3>(plan, views, n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st);
+        default: return launch_attn_ng<4>(plan, views, n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st);
+    }
+}

@@ -1,0 +1,717 @@
+// kvq_attn.cuh -- batched split-K decode attention straight over packed b-bit
+// KV caches plus a bf16 recent window.
+//
+// "Agent Memory Below the Prompt: Persistent Q4 KV Cache for Multi-Agent LLM
+// Inference on Edge Devices", Abstract: quantized caches go directly into the
+// attention layer and several agents' caches are attended at once
+// (BatchQuantizedKVCache).  "QKVShare ...", Significato e Affermazioni: a
+// fused quantized attention kernel in place of dequantize-then-attend.
+// "Coordinated Mixed-Precision KV Cache Quantization ...", Abstract: a width
+// per (agent, layer) and recent states kept in native precision.
+//
+// Work unit: (view, KV head, block of <= 8 query heads, chunk of tokens).
+// A CTA of 4 warps owns one unit; each warp streams 16-token tiles of the
+// chunk through its own ring of shared-memory stages filled by 1-D bulk async
+// copies (one elected lane issues them; an mbarrier per stage counts the
+// bytes).  Per tile, on tensor cores (mma.m16n8k16 bf16 -> fp32):
+//   QK:  S^T[token][head] = codes[token][d] . q[d][head], one accumulator per
+//        64-element group; the affine dequantisation is folded into the
+//        epilogue:  logit = sum_g s_g * acc_g + mn_g * sum_{d in g} q_d.
+//        Codes become exact bf16 integers with a LOP3 "magic exponent"
+//        (128 + c) and one bf16x2 FMA; q is bf16 already, so every product is
+//        exact.
+//   softmax: online (running max and sum per head, base 2).
+//   PV:  O^T[d][head] += codes^T[d][token] . (p * s)[token][head] plus the
+//        min term sum_t p_t * mn_t per group; p*s is split into two bf16
+//        terms (hi + lo, relative error <= 2^-17), and the 16x8 probability
+//        tile is moved from the QK accumulator layout to the B-operand layout
+//        with movmatrix.
+// Window tiles (bf16 K/V) use the same tile loop with the values as operands.
+// Each CTA merges its warps in a fixed order; the last CTA of a unit (an
+// atomic arrival counter, never a spin) merges the chunks in chunk order, so
+// results are bitwise reproducible.
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "kvq_ptx.cuh"
+
+namespace kvq {
+
+constexpr int kAttnWarps = 4;
+constexpr int kAttnThreads = 32 * kAttnWarps;
+constexpr int kTile = 16;
+constexpr int kMaxStages = 8;
+constexpr int kHeadsPerCta = 8;
+constexpr int kAttnMaxViews = 96;
+
+struct AttnView {
+    const uint8_t *codes[2];     // K, V packed rows [H_kv][cap][RB]
+    const float *scalemin[2];    // [H_kv][cap][NG][2]
+    const uint16_t *window[2];   // bf16 [H_kv][cap_w][D]
+    int64_t cap_packed;
+    int32_t n_packed;
+    int32_t n_window;
+    int32_t cap_window;
+    int32_t window_head;
+    int32_t bits;
+    int32_t n_chunks_packed;
+    int32_t n_chunks;            // packed + window chunks
+    int32_t chunk_begin;         // first chunk index of this view in the launch
+    int32_t view_index;          // row of q / out
+    int32_t pad_;
+};
+
+struct AttnParams {
+    const uint16_t *q;           // bf16 [n_views_total][Hq][D]
+    float *out;                  // fp32 [n_views_total][Hq][D]
+    float *partials;             // workspace
+    uint32_t *counters;          // workspace
+    uint32_t *status;            // workspace word 0
+    uint64_t timeout_ns;
+    float scale_log2;            // softmax_scale * log2(e)
+    int32_t n_views;
+    int32_t n_q_heads;
+    int32_t n_kv_heads;
+    int32_t group;               // n_q_heads / n_kv_heads
+    int32_t head_blocks;         // ceil(group / 8)
+    int32_t chunk;               // tokens per chunk, multiple of 16
+    int32_t ring_bytes;          // shared-memory ring per warp
+    AttnView views[kAttnMaxViews];
+};
+
+// ------------------------------------------------------- code unpacking ---
+//
+// QK operand: lane (gid, tig) holds, for one token row and one group, the 16
+// codes [16*tig, 16*tig + 16) of the group (2*B bytes at byte 2*B*tig).  They
+// become 8 bf16x2 registers r = 0..7; register r holds codes
+// (qk_code<B>(r, 0), qk_code<B>(r, 1)) in its (low, high) halves and feeds
+// k-step r/2, half r%2 of the group's four m16n8k16 steps.  The same map
+// places q in the B operand, so the dot product sums matching elements.
+
+template <int B>
+__host__ __device__ constexpr int qk_code(int r, int e) {
+    return B == 2 ? r + 8 * e : B == 3 ? r + 8 * e : B == 4 ? ((r < 4 ? r : r + 4) + 4 * e) : 2 * r + e;
+}
+
+// (bits at offset o in each 16-bit half) -> exact bf16 integers c, 2 per word
+template <int O>
+__device__ __forceinline__ uint32_t bf16_codes(uint32_t w, uint32_t mask_at_o) {
+    // 128 + c*2^O  ->  c   (exact: (128 + c 2^O) * 2^-O - 128 * 2^-O)
+    constexpr uint32_t kMagic = 0x43004300u;  // 128.0 in both halves
+    constexpr uint32_t kScale = (O == 0) ? 0x3F803F80u : (O == 2) ? 0x3E803E80u : (O == 3) ? 0x3E003E00u : 0x3D803D80u;
+    constexpr uint32_t kBias = (O == 0) ? 0xC300C300u : (O == 2) ? 0xC200C200u : (O == 3) ? 0xC180C180u : 0xC100C100u;
+    static_assert(O == 0 || O == 2 || O == 3 || O == 4, "offset");
+    return fma_bf16x2(lop3_and_or(w, mask_at_o, kMagic), kScale, kBias);
+}
+
+template <int B>
+__device__ __forceinline__ void qk_unpack(const uint8_t *seg, uint32_t (&r)[8]);
+
+template <>
+__device__ __forceinline__ void qk_unpack<2>(const uint8_t *seg, uint32_t (&r)[8]) {
+    // 16 codes x 2 bits = one word; code j at bit 2j.  Low half: codes 0..7,
+    // high half: codes 8..15; register r = (c_r, c_{r+8}).
+    const uint32_t w = *reinterpret_cast<const uint32_t *>(seg);
+    const uint32_t w6 = w >> 6, w12 = w >> 12;
+    r[0] = bf16_codes<0>(w, 0x00030003u);
+    r[1] = bf16_codes<2>(w, 0x000C000Cu);
+    r[2] = bf16_codes<4>(w, 0x00300030u);
+    r[3] = bf16_codes<0>(w6, 0x00030003u);
+    r[4] = bf16_codes<2>(w6, 0x000C000Cu);
+    r[5] = bf16_codes<4>(w6, 0x00300030u);
+    r[6] = bf16_codes<0>(w12, 0x00030003u);
+    r[7] = bf16_codes<2>(w12, 0x000C000Cu);
+}
+
+template <>
+__device__ __forceinline__ void qk_unpack<3>(const uint8_t *seg, uint32_t (&r)[8]) {
+    // 16 codes x 3 bits = 6 bytes at a 2-byte-aligned address; code j at bit
+    // 3j.  Register 2k+e = (c_{2k+e}, c_{2k+8+e}): the 16-bit windows at bits
+    // 6k and 6k+24 are paired into one word, codes at offsets 0 and 3.
+    const uintptr_t addr = reinterpret_cast<uintptr_t>(seg);
+    const uint32_t *wp = reinterpret_cast<const uint32_t *>(addr & ~uintptr_t(3));
+    const uint32_t sh = (uint32_t)(addr & 3u) * 8u;  // 0 or 16
+    const uint32_t w0 = wp[0], w1 = wp[1];
+    const uint32_t lo = __funnelshift_r(w0, w1, sh);  // bits 0..31 of the segment
+    const uint32_t hi = w1 >> sh;                     // bits 32..47 (low 16 bits valid)
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int a = 6 * k, b = 6 * k + 24;
+        const uint32_t fa = (a == 0) ? lo : __funnelshift_r(lo, hi, a);
+        const uint32_t fb = (b < 32) ? __funnelshift_r(lo, hi, b) : (hi >> (b - 32));
+        const uint32_t pw = prmt(fa, fb, 0x5410u);
+        r[2 * k] = bf16_codes<0>(pw, 0x00070007u);
+        r[2 * k + 1] = bf16_codes<3>(pw, 0x00380038u);
+    }
+}
+
+template <>
+__device__ __forceinline__ void qk_unpack<4>(const uint8_t *seg, uint32_t (&r)[8]) {
+    // 16 codes x 4 bits = 2 words; register k = (c_k, c_{k+4}) from word 0,
+    // register 4+k = (c_{8+k}, c_{12+k}) from word 1.
+    const uint2 w = *reinterpret_cast<const uint2 *>(seg);
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        r[k] = bf16_codes<0>(w.x >> (4 * k), 0x000F000Fu);
+        r[4 + k] = bf16_codes<0>(w.y >> (4 * k), 0x000F000Fu);
+    }
+}
+
+__device__ __forceinline__ float byte_to_f32(uint32_t w, uint32_t sel) {
+    // prmt places the selected byte under exponent 2^23; subtracting 2^23
+    // leaves the byte's value exactly.
+    return __fsub_rn(__uint_as_float(prmt(w, 0x4B000000u, sel)), 8388608.0f);
+}
+
+template <>
+__device__ __forceinline__ void qk_unpack<8>(const uint8_t *seg, uint32_t (&r)[8]) {
+    // 16 bytes; register r = (c_{2r}, c_{2r+1}).
+    const uint4 w = *reinterpret_cast<const uint4 *>(seg);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        r[2 * k] = pack_bf16x2(byte_to_f32(ws[k], 0x7440u), byte_to_f32(ws[k], 0x7441u));
+        r[2 * k + 1] = pack_bf16x2(byte_to_f32(ws[k], 0x7442u), byte_to_f32(ws[k], 0x7443u));
+    }
+}
+
+// PV operand: lane (gid, tig) holds, for two tokens a and b and one group, the
+// 8 codes [8*gid, 8*gid + 8) (B bytes at byte B*gid); register u = 0..7 holds
+// (code u of token a, code u of token b).
+template <int B>
+__device__ __forceinline__ void pv_unpack(const uint8_t *sa, const uint8_t *sb, uint32_t (&r)[8]);
+
+template <>
+__device__ __forceinline__ void pv_unpack<2>(const uint8_t *sa, const uint8_t *sb, uint32_t (&r)[8]) {
+    // 2 bytes per token at a 2-byte-aligned address
+    const uintptr_t a = reinterpret_cast<uintptr_t>(sa);
+    const uint32_t wa = *reinterpret_cast<const uint32_t *>(a & ~uintptr_t(3));
+    const uint32_t wb = *reinterpret_cast<const uint32_t *>(reinterpret_cast<uintptr_t>(sb) & ~uintptr_t(3));
+    const uint32_t p = prmt(wa, wb, (a & 2u) ? 0x7632u : 0x5410u);
+    const uint32_t p6 = p >> 6, p12 = p >> 12;
+    r[0] = bf16_codes<0>(p, 0x00030003u);
+    r[1] = bf16_codes<2>(p, 0x000C000Cu);
+    r[2] = bf16_codes<4>(p, 0x00300030u);
+    r[3] = bf16_codes<0>(p6, 0x00030003u);
+    r[4] = bf16_codes<2>(p6, 0x000C000Cu);
+    r[5] = bf16_codes<4>(p6, 0x00300030u);
+    r[6] = bf16_codes<0>(p12, 0x00030003u);
+    r[7] = bf16_codes<2>(p12, 0x000C000Cu);
+}
+
+__device__ __forceinline__ uint32_t load24(const uint8_t *s) {
+    // 3 bytes at any address, as the low 24 bits of a word
+    const uintptr_t a = reinterpret_cast<uintptr_t>(s);
+    const uint32_t *wp = reinterpret_cast<const uint32_t *>(a & ~uintptr_t(3));
+    return __funnelshift_r(wp[0], wp[1], (uint32_t)(a & 3u) * 8u);
+}
+
+template <>
+__device__ __forceinline__ void pv_unpack<3>(const uint8_t *sa, const uint8_t *sb, uint32_t (&r)[8]) {
+    const uint32_t xa = load24(sa), xb = load24(sb);
+    const uint32_t p1 = prmt(xa, xb, 0x5410u);               // codes 0..4 (+bit 15) of a | of b
+    const uint32_t p2 = prmt(xa >> 15, xb >> 15, 0x5410u);   // codes 5..7
+    const uint32_t p16 = p1 >> 6, p112 = p1 >> 12, p26 = p2 >> 6;
+    r[0] = bf16_codes<0>(p1, 0x00070007u);
+    r[1] = bf16_codes<3>(p1, 0x00380038u);
+    r[2] = bf16_codes<0>(p16, 0x00070007u);
+    r[3] = bf16_codes<3>(p16, 0x00380038u);
+    r[4] = bf16_codes<0>(p112, 0x00070007u);
+    r[5] = bf16_codes<0>(p2, 0x00070007u);
+    r[6] = bf16_codes<3>(p2, 0x00380038u);
+    r[7] = bf16_codes<0>(p26, 0x00070007u);
+}
+
+template <>
+__device__ __forceinline__ void pv_unpack<4>(const uint8_t *sa, const uint8_t *sb, uint32_t (&r)[8]) {
+    const uint32_t wa = *reinterpret_cast<const uint32_t *>(sa);
+    const uint32_t wb = *reinterpret_cast<const uint32_t *>(sb);
+    const uint32_t p1 = prmt(wa, wb, 0x5410u);  // codes 0..3 of a | of b
+    const uint32_t p2 = prmt(wa, wb, 0x7632u);  // codes 4..7
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        r[k] = bf16_codes<0>(p1 >> (4 * k), 0x000F000Fu);
+        r[4 + k] = bf16_codes<0>(p2 >> (4 * k), 0x000F000Fu);
+    }
+}
+
+template <>
+__device__ __forceinline__ void pv_unpack<8>(const uint8_t *sa, const uint8_t *sb, uint32_t (&r)[8]) {
+    const uint2 wa = *reinterpret_cast<const uint2 *>(sa);
+    const uint2 wb = *reinterpret_cast<const uint2 *>(sb);
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+        const uint32_t xa = (u < 4) ? wa.x : wa.y, xb = (u < 4) ? wb.x : wb.y;
+        const uint32_t sel = 0x7440u | (u & 3);
+        r[u] = pack_bf16x2(byte_to_f32(xa, sel), byte_to_f32(xb, sel));
+    }
+}
+
+// ------------------------------------------------------------ per-warp ----
+
+template <int NG>
+struct WarpState {
+    float o[NG][4][4];   // O^T tiles: group g, d-tile t; (row gid|gid+8) x (head 2tig|2tig+1)
+    float mt[NG][2];     // min-term partial sums, heads 2tig, 2tig+1
+    float m[2];          // running max (log2 units)
+    float l[2];          // running sum (partial over this lane's rows)
+    uint32_t bq[NG][4][2];  // q as B operand: group, k-step, (b0b1, b2b3)
+    float qsum[NG][2];
+};
+
+// Online-softmax step for one 16-token tile: lg[row][head] are base-2 logits
+// of rows gid, gid+8 and heads 2tig, 2tig+1.  Returns the probabilities in lg.
+template <int NG>
+__device__ __forceinline__ void softmax_step(WarpState<NG> &st, float (&lg)[2][2]) {
+    float alpha[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        float t = fmaxf(lg[0][j], lg[1][j]);
+        t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 4));
+        t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 8));
+        t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 16));
+        const float mnew = fmaxf(st.m[j], t);
+        alpha[j] = exp2f(st.m[j] - mnew);
+        st.m[j] = mnew;
+        lg[0][j] = exp2f(lg[0][j] - mnew);
+        lg[1][j] = exp2f(lg[1][j] - mnew);
+        st.l[j] = st.l[j] * alpha[j] + (lg[0][j] + lg[1][j]);
+    }
+    if (__any_sync(0xFFFFFFFFu, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+#pragma unroll
+            for (int t = 0; t < 4; ++t) {
+                st.o[g][t][0] *= alpha[0];
+                st.o[g][t][1] *= alpha[1];
+                st.o[g][t][2] *= alpha[0];
+                st.o[g][t][3] *= alpha[1];
+            }
+            st.mt[g][0] *= alpha[0];
+            st.mt[g][1] *= alpha[1];
+        }
+    }
+}
+
+// hi/lo bf16 split of a probability-like pair and transpose to B layout
+__device__ __forceinline__ void split_transpose(float a0, float a1, float b0, float b1, uint32_t &bh0,
+                                                uint32_t &bh1, uint32_t &bl0, uint32_t &bl1) {
+    const uint32_t h0 = pack_bf16x2(a0, a1);
+    const uint32_t h1 = pack_bf16x2(b0, b1);
+    const uint32_t l0 = pack_bf16x2(a0 - bf16lo_to_f32(h0), a1 - bf16hi_to_f32(h0));
+    const uint32_t l1 = pack_bf16x2(b0 - bf16lo_to_f32(h1), b1 - bf16hi_to_f32(h1));
+    bh0 = movmatrix_trans(h0);
+    bh1 = movmatrix_trans(h1);
+    bl0 = movmatrix_trans(l0);
+    bl1 = movmatrix_trans(l1);
+}
+
+// One 16-token tile of packed tokens.  Stage layout: K codes [16][RB], V codes
+// [16][RB], K scalemin [16][NG] float2, V scalemin [16][NG] float2.
+template <int B, int NG>
+__device__ __forceinline__ void packed_tile(WarpState<NG> &st, const uint8_t *stage, int n_valid,
+                                            float scale_log2, int gid, int tig) {
+    constexpr int RB = 8 * B * NG;
+    const uint8_t *kc = stage;
+    const uint8_t *vc = stage + 16 * RB;
+    const float2 *ks = reinterpret_cast<const float2 *>(stage + 32 * RB);
+    const float2 *vs = ks + 16 * NG;
+    const int r0 = gid, r1 = gid + 8;
+    const bool v0 = r0 < n_valid, v1 = r1 < n_valid;
+
+    float lg[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        uint32_t a0[8], a1[8];
+        qk_unpack<B>(kc + r0 * RB + g * 8 * B + 2 * B * tig, a0);
+        qk_unpack<B>(kc + r1 * RB + g * 8 * B + 2 * B * tig, a1);
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_bf16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0], st.bq[g][s][1]);
+        const float2 k0 = ks[r0 * NG + g], k1 = ks[r1 * NG + g];
+        lg[0][0] = fmaf(k0.x, acc[0], fmaf(k0.y, st.qsum[g][0], lg[0][0]));
+        lg[0][1] = fmaf(k0.x, acc[1], fmaf(k0.y, st.qsum[g][1], lg[0][1]));
+        lg[1][0] = fmaf(k1.x, acc[2], fmaf(k1.y, st.qsum[g][0], lg[1][0]));
+        lg[1][1] = fmaf(k1.x, acc[3], fmaf(k1.y, st.qsum[g][1], lg[1][1]));
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        lg[0][j] = v0 ? lg[0][j] * scale_log2 : -INFINITY;
+        lg[1][j] = v1 ? lg[1][j] * scale_log2 : -INFINITY;
+    }
+    softmax_step<NG>(st, lg);
+
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        float2 m0 = vs[r0 * NG + g], m1 = vs[r1 * NG + g];
+        if (!v0) m0 = make_float2(0.f, 0.f);
+        if (!v1) m1 = make_float2(0.f, 0.f);
+        st.mt[g][0] = fmaf(lg[0][0], m0.y, fmaf(lg[1][0], m1.y, st.mt[g][0]));
+        st.mt[g][1] = fmaf(lg[0][1], m0.y, fmaf(lg[1][1], m1.y, st.mt[g][1]));
+        uint32_t bh0, bh1, bl0, bl1;
+        split_transpose(lg[0][0] * m0.x, lg[0][1] * m0.x, lg[1][0] * m1.x, lg[1][1] * m1.x, bh0, bh1, bl0, bl1);
+        uint32_t va[8], vb[8];
+        const int off = g * 8 * B + B * gid;
+        pv_unpack<B>(vc + (2 * tig) * RB + off, vc + (2 * tig + 1) * RB + off, va);
+        pv_unpack<B>(vc + (2 * tig + 8) * RB + off, vc + (2 * tig + 9) * RB + off, vb);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            mma_bf16_16816(st.o[g][t], va[2 * t], va[2 * t + 1], vb[2 * t], vb[2 * t + 1], bh0, bh1);
+            mma_bf16_16816(st.o[g][t], va[2 * t], va[2 * t + 1], vb[2 * t], vb[2 * t + 1], bl0, bl1);
+        }
+    }
+}
+
+// Window tile, K half: stage = K rows [16][D] bf16.  Returns base-2 logits.
+template <int NG>
+__device__ __forceinline__ void window_qk(WarpState<NG> &st, const uint8_t *stage, int n_valid,
+                                          float scale_log2, int gid, int tig, float (&lg)[2][2]) {
+    constexpr int D = 64 * NG;
+    const uint16_t *k = reinterpret_cast<const uint16_t *>(stage);
+    const int r0 = gid, r1 = gid + 8;
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        const uint4 *p0 = reinterpret_cast<const uint4 *>(k + r0 * D + 64 * g + 16 * tig);
+        const uint4 *p1 = reinterpret_cast<const uint4 *>(k + r1 * D + 64 * g + 16 * tig);
+        const uint4 x0 = p0[0], x1 = p0[1], y0 = p1[0], y1 = p1[1];
+        const uint32_t a0[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+        const uint32_t a1[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
+#pragma unroll
+        for (int s = 0; s < 4; ++s)
+            mma_bf16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0], st.bq[g][s][1]);
+    }
+    const bool v0 = r0 < n_valid, v1 = r1 < n_valid;
+    lg[0][0] = v0 ? acc[0] * scale_log2 : -INFINITY;
+    lg[0][1] = v0 ? acc[1] * scale_log2 : -INFINITY;
+    lg[1][0] = v1 ? acc[2] * scale_log2 : -INFINITY;
+    lg[1][1] = v1 ? acc[3] * scale_log2 : -INFINITY;
+}
+
+// Window tile, V half: stage = V rows [16][D] bf16; lg holds probabilities.
+template <int NG>
+__device__ __forceinline__ void window_pv(WarpState<NG> &st, const uint8_t *stage, int n_valid,
+                                          const float (&p)[2][2], int gid, int tig) {
+    constexpr int D = 64 * NG;
+    const uint16_t *v = reinterpret_cast<const uint16_t *>(stage);
+    uint32_t bh0, bh1, bl0, bl1;
+    split_transpose(p[0][0], p[0][1], p[1][0], p[1][1], bh0, bh1, bl0, bl1);
+    const int ta = 2 * tig, tb = 2 * tig + 1, tc = 2 * tig + 8, td = 2 * tig + 9;
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        const int col = 64 * g + 8 * gid;
+        uint4 xa = *reinterpret_cast<const uint4 *>(v + ta * D + col);
+        uint4 xb = *reinterpret_cast<const uint4 *>(v + tb * D + col);
+        uint4 xc = *reinterpret_cast<const uint4 *>(v + tc * D + col);
+        uint4 xd = *reinterpret_cast<const uint4 *>(v + td * D + col);
+        // rows past the valid count hold stale bytes: zero them (p is 0 there,
+        // but 0 * NaN would not be)
+        if (ta >= n_valid) xa = make_uint4(0, 0, 0, 0);
+        if (tb >= n_valid) xb = make_uint4(0, 0, 0, 0);
+        if (tc >= n_valid) xc = make_uint4(0, 0, 0, 0);
+        if (td >= n_valid) xd = make_uint4(0, 0, 0, 0);
+        const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w}, wb[4] = {xb.x, xb.y, xb.z, xb.w};
+        const uint32_t wc[4] = {xc.x, xc.y, xc.z, xc.w}, wd[4] = {xd.x, xd.y, xd.z, xd.w};
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const uint32_t a0 = prmt(wa[t], wb[t], 0x5410u), a1 = prmt(wa[t], wb[t], 0x7632u);
+            const uint32_t a2 = prmt(wc[t], wd[t], 0x5410u), a3 = prmt(wc[t], wd[t], 0x7632u);
+            mma_bf16_16816(st.o[g][t], a0, a1, a2, a3, bh0, bh1);
+            mma_bf16_16816(st.o[g][t], a0, a1, a2, a3, bl0, bl1);
+        }
+    }
+}
+
+// ---------------------------------------------------------------- kernel ---
+
+__device__ __forceinline__ uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
+
+template <int NG>
+__global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const __grid_constant__ AttnParams p) {
+    constexpr int D = 64 * NG;
+    extern __shared__ __align__(128) uint8_t smem[];
+    uint16_t *q_s = reinterpret_cast<uint16_t *>(smem);                            // [8][D]
+    float *qsum_s = reinterpret_cast<float *>(smem + 8 * D * 2);                  // [8][NG]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 8 * D * 2 + 8 * NG * 4);  // [4][8]
+    int *flag_s = reinterpret_cast<int *>(bars + kAttnWarps * kMaxStages);
+    uint8_t *rings = smem + ((8 * D * 2 + 8 * NG * 4 + kAttnWarps * kMaxStages * 8 + 16 + 127) & ~127);
+
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int gid = lane >> 2, tig = lane & 3;
+
+    // ---- which unit
+    const int bx = blockIdx.x;
+    int lo = 0, hi = p.n_views - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.views[mid].chunk_begin <= bx) lo = mid; else hi = mid - 1;
+    }
+    const int vi = lo;
+    const AttnView &V = p.views[vi];
+    const int c = bx - V.chunk_begin;
+    const int hk = blockIdx.y, z = blockIdx.z;
+    const int h0 = hk * p.group + z * kHeadsPerCta;
+    const int nh = min(kHeadsPerCta, p.group - z * kHeadsPerCta);
+    const bool is_window = c >= V.n_chunks_packed;
+    const int64_t tok0 = (int64_t)(is_window ? c - V.n_chunks_packed : c) * p.chunk;
+    const int n_tok = (int)min((int64_t)p.chunk, (is_window ? (int64_t)V.n_window : (int64_t)V.n_packed) - tok0);
+    const int n_tiles = (n_tok + kTile - 1) / kTile;
+    const int B = V.bits;
+    const int RB = 8 * B * NG;
+
+    // ---- q (bf16, zero rows past nh), per-group sums, barriers
+    for (int i = tid; i < kHeadsPerCta * D / 8; i += kAttnThreads) {
+        const int j = i / (D / 8), d8 = i % (D / 8);
+        uint4 val = make_uint4(0, 0, 0, 0);
+        if (j < nh) val = reinterpret_cast<const uint4 *>(p.q + ((int64_t)V.view_index * p.n_q_heads + h0 + j) * D)[d8];
+        reinterpret_cast<uint4 *>(q_s)[i] = val;
+    }
+    if (lane == 0) {
+        for (int s = 0; s < kMaxStages; ++s) mbar_init(&bars[warp * kMaxStages + s], 1);
+        fence_mbar_init();
+    }
+    __syncthreads();
+    if (tid < 8 * NG) {
+        const int j = tid / NG, g = tid % NG;
+        float acc = 0.f;
+        for (int d = 0; d < 64; ++d) acc += __uint_as_float((uint32_t)q_s[j * D + 64 * g + d] << 16);
+        qsum_s[j * NG + g] = acc;
+    }
+    __syncthreads();
+
+    WarpState<NG> st;
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+#pragma unroll
+        for (int t = 0; t < 4; ++t)
+#pragma unroll
+            for (int e = 0; e < 4; ++e) st.o[g][t][e] = 0.f;
+        st.mt[g][0] = st.mt[g][1] = 0.f;
+        st.qsum[g][0] = qsum_s[(2 * tig) * NG + g];
+        st.qsum[g][1] = qsum_s[(2 * tig + 1) * NG + g];
+    }
+    st.m[0] = st.m[1] = -INFINITY;
+    st.l[0] = st.l[1] = 0.f;
+
+    // q B-operand fragments: column n = gid, k-slots from the unpack map
+    {
+        const uint16_t *qr = q_s + gid * D;
+        auto qpair = [&](int d0, int d1) -> uint32_t {
+            return (uint32_t)qr[d0] | ((uint32_t)qr[d1] << 16);
+        };
+#pragma unroll
+        for (int g = 0; g < NG; ++g)
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+#pragma unroll
+                for (int j = 0; j < 2; ++j) {
+                    const int r = 2 * s + j;
+                    int e0, e1;
+                    if (is_window) { e0 = 2 * r; e1 = 2 * r + 1; }
+                    else if (B == 2) { e0 = qk_code<2>(r, 0); e1 = qk_code<2>(r, 1); }
+                    else if (B == 3) { e0 = qk_code<3>(r, 0); e1 = qk_code<3>(r, 1); }
+                    else if (B == 4) { e0 = qk_code<4>(r, 0); e1 = qk_code<4>(r, 1); }
+                    else { e0 = qk_code<8>(r, 0); e1 = qk_code<8>(r, 1); }
+                    st.bq[g][s][j] = qpair(64 * g + 16 * tig + e0, 64 * g + 16 * tig + e1);
+                }
+    }
+
+    // ---- per-warp pipeline of bulk copies into this warp's ring
+    uint8_t *ring = rings + (size_t)warp * p.ring_bytes;
+    uint64_t *wbar = bars + warp * kMaxStages;
+    const uint32_t stage_bytes = is_window ? (uint32_t)(kTile * D * 2) : (uint32_t)(32 * RB + 2 * kTile * NG * 8);
+    const int S = min(kMaxStages, (int)(p.ring_bytes / stage_bytes));
+    const int n_my = (warp < n_tiles) ? (n_tiles - warp + kAttnWarps - 1) / kAttnWarps : 0;
+    const int bpt = is_window ? 2 : 1;
+    const int n_blocks = n_my * bpt;
+
+    auto issue = [&](int blk) {
+        const int slot = blk % S;
+        uint8_t *dst = ring + (size_t)slot * stage_bytes;
+        uint64_t *bar = &wbar[slot];
+        const int tile = warp + kAttnWarps * (blk / bpt);
+        const int n = min(kTile, n_tok - kTile * tile);
+        if (!is_window) {
+            const int64_t row = (int64_t)hk * V.cap_packed + tok0 + kTile * tile;
+            const uint32_t bc = round16((uint32_t)(n * RB));
+            const uint32_t bs = round16((uint32_t)(n * NG * 8));
+            mbar_arrive_expect_tx(bar, 2 * bc + 2 * bs);
+            bulk_copy_g2s(dst, V.codes[0] + row * RB, bc, bar);
+            bulk_copy_g2s(dst + 16 * RB, V.codes[1] + row * RB, bc, bar);
+            bulk_copy_g2s(dst + 32 * RB, V.scalemin[0] + row * NG * 2, bs, bar);
+            bulk_copy_g2s(dst + 32 * RB + kTile * NG * 8, V.scalemin[1] + row * NG * 2, bs, bar);
+        } else {
+            const int kv = blk & 1;
+            const uint16_t *base = V.window[kv] + (int64_t)hk * V.cap_window * D;
+            const int logical = (int)tok0 + kTile * tile;
+            const int phys = (V.window_head + logical) % V.cap_window;
+            const int first = min(n, V.cap_window - phys);
+            mbar_arrive_expect_tx(bar, (uint32_t)(n * D * 2));
+            bulk_copy_g2s(dst, base + (int64_t)phys * D, (uint32_t)(first * D * 2), bar);
+            if (n > first) bulk_copy_g2s(dst + first * D * 2, base, (uint32_t)((n - first) * D * 2), bar);
+        }
+    };
+
+    bool failed = false;
+    int issued = 0;
+    if (lane == 0) {
+        for (; issued < min(S, n_blocks); ++issued) issue(issued);
+    }
+    issued = min(S, n_blocks);
+    __syncwarp();
+
+    // warp-uniform: a lane that gives up makes the whole warp give up
+    auto wait_block = [&](int blk) -> bool {
+        const bool ok = mbar_wait_bounded(&wbar[blk % S], (uint32_t)((blk / S) & 1), p.timeout_ns);
+        return __all_sync(0xFFFFFFFFu, ok);
+    };
+    auto release_block = [&](int blk) {
+        __syncwarp();
+        if (blk + S < n_blocks) {
+            if (lane == 0) {
+                fence_proxy_async_shared();
+                issue(blk + S);
+            }
+            issued = blk + S + 1;
+        }
+    };
+
+    int blk = 0;
+    for (int i = 0; i < n_my && !failed; ++i) {
+        const int tile = warp + kAttnWarps * i;
+        const int n_valid = min(kTile, n_tok - kTile * tile);
+        if (!is_window) {
+            if (!wait_block(blk)) { failed = true; break; }
+            const uint8_t *stage = ring + (size_t)(blk % S) * stage_bytes;
+            switch (B) {
+                case 2: packed_tile<2, NG>(st, stage, n_valid, p.scale_log2, gid, tig); break;
+                case 3: packed_tile<3, NG>(st, stage, n_valid, p.scale_log2, gid, tig); break;
+                case 4: packed_tile<4, NG>(st, stage, n_valid, p.scale_log2, gid, tig); break;
+                default: packed_tile<8, NG>(st, stage, n_valid, p.scale_log2, gid, tig); break;
+            }
+            release_block(blk);
+            ++blk;
+        } else {
+            float lg[2][2];
+            if (!wait_block(blk)) { failed = true; break; }
+            window_qk<NG>(st, ring + (size_t)(blk % S) * stage_bytes, n_valid, p.scale_log2, gid, tig, lg);
+            release_block(blk);
+            ++blk;
+            softmax_step<NG>(st, lg);
+            if (!wait_block(blk)) { failed = true; break; }
+            window_pv<NG>(st, ring + (size_t)(blk % S) * stage_bytes, n_valid, lg, gid, tig);
+            release_block(blk);
+            ++blk;
+        }
+    }
+    failed = __any_sync(0xFFFFFFFFu, failed);
+    if (failed) {
+        // let every copy this warp issued land before the CTA can exit
+        for (int b = blk; b < issued; ++b) (void)wait_block(b);
+        if (lane == 0) atomicExch(p.status, 1u);
+    }
+
+    // ---- warp partial -> this warp's ring area (all its copies have landed)
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        float l = st.l[j];
+        l += __shfl_xor_sync(0xFFFFFFFFu, l, 4);
+        l += __shfl_xor_sync(0xFFFFFFFFu, l, 8);
+        l += __shfl_xor_sync(0xFFFFFFFFu, l, 16);
+        st.l[j] = l;
+#pragma unroll
+        for (int g = 0; g < NG; ++g) {
+            float m = st.mt[g][j];
+            m += __shfl_xor_sync(0xFFFFFFFFu, m, 4);
+            m += __shfl_xor_sync(0xFFFFFFFFu, m, 8);
+            m += __shfl_xor_sync(0xFFFFFFFFu, m, 16);
+            st.mt[g][j] = m;
+        }
+    }
+    __syncwarp();
+    float *wpart = reinterpret_cast<float *>(ring);  // m[8], l[8], o[8][D]
+    if (gid == 0) {
+        wpart[2 * tig] = st.m[0];
+        wpart[2 * tig + 1] = st.m[1];
+        wpart[8 + 2 * tig] = st.l[0];
+        wpart[8 + 2 * tig + 1] = st.l[1];
+    }
+    float *wo = wpart + 16;
+#pragma unroll
+    for (int g = 0; g < NG; ++g)
+#pragma unroll
+        for (int t = 0; t < 4; ++t) {
+            const int d0 = 64 * g + 8 * gid + 2 * t;
+            wo[(2 * tig) * D + d0] = st.o[g][t][0] + st.mt[g][0];
+            wo[(2 * tig + 1) * D + d0] = st.o[g][t][1] + st.mt[g][1];
+            wo[(2 * tig) * D + d0 + 1] = st.o[g][t][2] + st.mt[g][0];
+            wo[(2 * tig + 1) * D + d0 + 1] = st.o[g][t][3] + st.mt[g][1];
+        }
+    __syncthreads();
+
+    // ---- merge the 4 warps (fixed order)
+    const bool single = V.n_chunks == 1;
+    const int units_per_view = p.n_kv_heads * p.head_blocks;
+    const int64_t slot = ((int64_t)(V.chunk_begin + c) * p.n_kv_heads + hk) * p.head_blocks + z;
+    float *part = p.partials + slot * (kHeadsPerCta * (D + 2));
+    for (int idx = tid; idx < nh * D; idx += kAttnThreads) {
+        const int j = idx / D, d = idx - j * D;
+        float M = -INFINITY;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w)
+            M = fmaxf(M, reinterpret_cast<const float *>(rings + (size_t)w * p.ring_bytes)[j]);
+        float L = 0.f, O = 0.f;
+#pragma unroll
+        for (int w = 0; w < kAttnWarps; ++w) {
+            const float *wp = reinterpret_cast<const float *>(rings + (size_t)w * p.ring_bytes);
+            const float mw = wp[j];
+            const float e = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+            L = fmaf(e, wp[8 + j], L);
+            O = fmaf(e, wp[16 + j * D + d], O);
+        }
+        if (single) {
+            p.out[((int64_t)V.view_index * p.n_q_heads + h0 + j) * D + d] = O / L;
+        } else {
+            part[j * (D + 2) + d] = O;
+            if (d == 0) {
+                part[j * (D + 2) + D] = M;
+                part[j * (D + 2) + D + 1] = L;
+            }
+        }
+    }
+    if (single) return;
+
+    // ---- last CTA of the unit merges all chunks, in chunk order
+    __threadfence();
+    __syncthreads();
+    uint32_t *counter = p.counters + ((int64_t)vi * units_per_view + hk * p.head_blocks + z);
+    if (tid == 0) {
+        const uint32_t prev = atomicAdd(counter, 1u);
+        flag_s[0] = (prev == (uint32_t)(V.n_chunks - 1)) ? 1 : 0;
+    }
+    __syncthreads();
+    if (!flag_s[0]) return;
+    __threadfence();
+    const int64_t slot0 = ((int64_t)V.chunk_begin * p.n_kv_heads + hk) * p.head_blocks + z;
+    const int64_t slot_stride = (int64_t)p.n_kv_heads * p.head_blocks * (kHeadsPerCta * (D + 2));
+    const float *part0 = p.partials + slot0 * (kHeadsPerCta * (D + 2));
+    for (int idx = tid; idx < nh * D; idx += kAttnThreads) {
+        const int j = idx / D, d = idx - j * D;
+        float M = -INFINITY;
+        for (int cc = 0; cc < V.n_chunks; ++cc) M = fmaxf(M, __ldcg(part0 + cc * slot_stride + j * (D + 2) + D));
+        float L = 0.f, O = 0.f;
+        for (int cc = 0; cc < V.n_chunks; ++cc) {
+            const float *pc = part0 + cc * slot_stride + j * (D + 2);
+            const float e = exp2f(__ldcg(pc + D) - M);
+            L = fmaf(e, __ldcg(pc + D + 1), L);
+            O = fmaf(e, __ldcg(pc + d), O);
+        }
+        p.out[((int64_t)V.view_index * p.n_q_heads + h0 + j) * D + d] = O / L;
+    }
+    if (tid == 0) atomicExch(counter, 0u);
+}
+
+}  // namespace kvq

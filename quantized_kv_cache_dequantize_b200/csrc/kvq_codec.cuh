@@ -1,0 +1,301 @@
+// kvq_codec.cuh -- group-wise affine quantization of bf16 K/V rows into packed
+// b-bit codes with a per-group {scale, min}, and its inverse into bf16.
+//
+// "QKVShare: Quantized KV-Cache Handoff for Multi-Agent On-Device LLMs",
+// Metodologia: quantized KV groups form the handoff card and the receiver
+// rebuilds full-precision past_key_values from them.  "Agent Memory Below the
+// Prompt ...", Abstract: 4-bit format.  "Coordinated Mixed-Precision KV Cache
+// Quantization ...", Abstract: widths 2/3/4 (and 8) per (agent, layer).
+//
+// Both kernels stream HBM: two lanes share one 64-element group (32 elements,
+// 64 bytes of bf16 each), loads and stores are 16-byte vectors, and every
+// result is a bit-exact function of the input (fp32 round-to-nearest steps in
+// the order of the format definition).
+#pragma once
+
+#include <cstdint>
+#include <cuda_bf16.h>
+
+#include "kvq_ptx.cuh"
+
+namespace kvq {
+
+constexpr int kGroup = 64;
+constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: y + magic rounds y to an integer (RNE)
+constexpr uint32_t kRoundMagicBits = 0x4B400000u;
+
+// Quantize one half (32 elements) of a 64-element group held as 16 bf16x2
+// words; the partner half lives in lane ^ 1, which must execute this call in
+// the same instruction stream (full-warp shuffles).  Writes the packed codes
+// of this half (32*B bits = B words, code j at bit j*B) and the group's s, mn.
+template <int B>
+__device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], uint32_t (&packed)[B],
+                                                    float &s_out, float &mn_out) {
+    __nv_bfloat162 lo2 = *reinterpret_cast<const __nv_bfloat162 *>(&x[0]);
+    __nv_bfloat162 hi2 = lo2;
+#pragma unroll
+    for (int i = 1; i < 16; ++i) {
+        const __nv_bfloat162 v = *reinterpret_cast<const __nv_bfloat162 *>(&x[i]);
+        lo2 = __hmin2(lo2, v);
+        hi2 = __hmax2(hi2, v);
+    }
+    const uint32_t lo_bits = *reinterpret_cast<uint32_t *>(&lo2);
+    const uint32_t hi_bits = *reinterpret_cast<uint32_t *>(&hi2);
+    float mn = fminf(bf16lo_to_f32(lo_bits), bf16hi_to_f32(lo_bits));
+    float mx = fmaxf(bf16lo_to_f32(hi_bits), bf16hi_to_f32(hi_bits));
+    mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+    if ((__float_as_uint(mn) << 1) == 0u) mn = 0.0f;  // +0 for either zero
+    if ((__float_as_uint(mx) << 1) == 0u) mx = 0.0f;
+
+    constexpr uint32_t qmax = (1u << B) - 1u;
+    const float s = (mx != mn) ? __fdiv_rn(__fsub_rn(mx, mn), (float)qmax) : 0.0f;
+
+#pragma unroll
+    for (int w = 0; w < B; ++w) packed[w] = 0u;
+
+    if (s != 0.0f) {
+        // Fast path: y = (x - mn) * RN(1/s) lies within 3*2^(B-24) of the
+        // correctly rounded quotient RN((x - mn)/s) (quotients are <= 2^B).
+        // Unless y is within `lim` of a half-integer, both round to the same
+        // integer; near-ties, and any non-finite y (tiny s), take the IEEE
+        // division.  The result is exactly round_half_even(RN((x-mn)/s)).
+        const float r = __frcp_rn(s);
+        const float lim = 0.5f - __uint_as_float((uint32_t)(127 + B - 21) << 23);
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float xf = (i & 1) ? bf16hi_to_f32(x[i >> 1]) : bf16lo_to_f32(x[i >> 1]);
+            const float a = __fsub_rn(xf, mn);
+            const float y = __fmul_rn(a, r);
+            const float t = __fadd_rn(y, kRoundMagic);
+            const float d = __fsub_rn(y, __fsub_rn(t, kRoundMagic));
+            uint32_t c = __float_as_uint(t) - kRoundMagicBits;
+            if (!(fabsf(d) <= lim)) c = __float2uint_rn(__fdiv_rn(a, s));
+            c = min(c, qmax);
+            const int bit = i * B;
+            packed[bit >> 5] |= c << (bit & 31);
+            if ((bit & 31) + B > 32) packed[(bit >> 5) + 1] |= c >> (32 - (bit & 31));
+        }
+    }
+    s_out = s;
+    mn_out = mn;
+}
+
+// Dequantize 32 codes (B words, code j at bit j*B) into 16 bf16x2 words.
+template <int B>
+__device__ __forceinline__ void dequantize_half_group(const uint32_t (&packed)[B], float s, float mn,
+                                                      uint32_t (&y)[16]) {
+    constexpr uint32_t mask = (1u << B) - 1u;
+#pragma unroll
+    for (int i = 0; i < 32; i += 2) {
+        uint32_t c[2];
+#pragma unroll
+        for (int k = 0; k < 2; ++k) {
+            const int bit = (i + k) * B;
+            uint32_t v = packed[bit >> 5] >> (bit & 31);
+            if ((bit & 31) + B > 32) v |= packed[(bit >> 5) + 1] << (32 - (bit & 31));
+            c[k] = v & mask;
+        }
+        // exact small-integer -> float: 2^23 + c, minus 2^23
+        const float c0 = __fsub_rn(__uint_as_float(0x4B000000u | c[0]), 8388608.0f);
+        const float c1 = __fsub_rn(__uint_as_float(0x4B000000u | c[1]), 8388608.0f);
+        y[i >> 1] = pack_bf16x2(__fmaf_rn(c0, s, mn), __fmaf_rn(c1, s, mn));
+    }
+}
+
+struct CodecArgs {
+    const uint16_t *x;       // bf16 (quantize input / dequantize output)
+    int64_t x_head_stride;   // elements
+    int64_t x_tok_stride;    // elements
+    int64_t n_tokens;
+    int32_t n_heads;
+    uint8_t *codes;
+    float *scalemin;
+    int64_t head_cap;        // rows per head in codes/scalemin
+};
+
+// Grid: (blocks per head, n_heads). Each lane pair owns one group; a warp
+// owns 16 consecutive groups of one head per iteration.
+template <int B, int NG>
+__global__ void __launch_bounds__(256) quantize_kernel(CodecArgs a) {
+    constexpr int RB = 8 * B * NG;  // row bytes
+    const int h = blockIdx.y;
+    const int64_t n_groups = a.n_tokens * NG;
+    const int lane = threadIdx.x & 31;
+    const int64_t warp_global = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t warp_stride = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const uint16_t *xh = a.x + (int64_t)h * a.x_head_stride;
+    uint8_t *ch = a.codes + (int64_t)h * a.head_cap * RB;
+    float *sh = a.scalemin + (int64_t)h * a.head_cap * NG * 2;
+
+    for (int64_t base = warp_global * 16; base < n_groups; base += warp_stride * 16) {
+        const int64_t grp = base + (lane >> 1);
+        const int half = lane & 1;
+        const bool active = grp < n_groups;
+        const int64_t t = grp / NG;
+        const int g = (int)(grp - t * NG);
+        uint32_t x[16];
+        if (active) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(xh + t * a.x_tok_stride + g * kGroup + half * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) {
+                const uint4 q = __ldcs(src + v);
+                x[4 * v + 0] = q.x; x[4 * v + 1] = q.y; x[4 * v + 2] = q.z; x[4 * v + 3] = q.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = 0u;
+        }
+        uint32_t packed[B];
+        float s, mn;
+        quantize_half_group<B>(x, packed, s, mn);
+        if (active) {
+            uint8_t *dst = ch + t * RB + g * 8 * B + half * 4 * B;
+            if constexpr (B == 4) {
+                *reinterpret_cast<uint4 *>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            } else if constexpr (B == 8) {
+                reinterpret_cast<uint4 *>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                reinterpret_cast<uint4 *>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+            } else if constexpr (B == 2) {
+                *reinterpret_cast<uint2 *>(dst) = make_uint2(packed[0], packed[1]);
+            } else {
+#pragma unroll
+                for (int w = 0; w < B; ++w) reinterpret_cast<uint32_t *>(dst)[w] = packed[w];
+            }
+            if (half == 0) *reinterpret_cast<float2 *>(sh + (t * NG + g) * 2) = make_float2(s, mn);
+        }
+    }
+}
+
+template <int B, int NG>
+__global__ void __launch_bounds__(256) dequantize_kernel(CodecArgs a) {
+    constexpr int RB = 8 * B * NG;
+    const int h = blockIdx.y;
+    const int64_t n_groups = a.n_tokens * NG;
+    const int lane = threadIdx.x & 31;
+    const int64_t warp_global = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t warp_stride = (int64_t)gridDim.x * (blockDim.x >> 5);
+    uint16_t *yh = const_cast<uint16_t *>(a.x) + (int64_t)h * a.x_head_stride;
+    const uint8_t *ch = a.codes + (int64_t)h * a.head_cap * RB;
+    const float *sh = a.scalemin + (int64_t)h * a.head_cap * NG * 2;
+
+    for (int64_t base = warp_global * 16; base < n_groups; base += warp_stride * 16) {
+        const int64_t grp = base + (lane >> 1);
+        const int half = lane & 1;
+        if (grp >= n_groups) continue;
+        const int64_t t = grp / NG;
+        const int g = (int)(grp - t * NG);
+        const uint8_t *src = ch + t * RB + g * 8 * B + half * 4 * B;
+        uint32_t packed[B];
+        if constexpr (B == 4) {
+            const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(src));
+            packed[0] = q.x; packed[1] = q.y; packed[2] = q.z; packed[3] = q.w;
+        } else if constexpr (B == 8) {
+            const uint4 q0 = __ldcs(reinterpret_cast<const uint4 *>(src));
+            const uint4 q1 = __ldcs(reinterpret_cast<const uint4 *>(src) + 1);
+            packed[0] = q0.x; packed[1] = q0.y; packed[2] = q0.z; packed[3] = q0.w;
+            packed[4] = q1.x; packed[5] = q1.y; packed[6] = q1.z; packed[7] = q1.w;
+        } else if constexpr (B == 2) {
+            const uint2 q = __ldcs(reinterpret_cast<const uint2 *>(src));
+            packed[0] = q.x; packed[1] = q.y;
+        } else {
+#pragma unroll
+            for (int w = 0; w < B; ++w) packed[w] = __ldcs(reinterpret_cast<const uint32_t *>(src) + w);
+        }
+        const float2 sm = __ldcs(reinterpret_cast<const float2 *>(sh + (t * NG + g) * 2));
+        uint32_t y[16];
+        dequantize_half_group<B>(packed, sm.x, sm.y, y);
+        uint4 *dst = reinterpret_cast<uint4 *>(yh + t * a.x_tok_stride + g * kGroup + half * 32);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) __stcs(dst + v, make_uint4(y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]));
+    }
+}
+
+// ------------------------------------------------------------- append ----
+
+// One view's slice of a kvq_append launch, resolved on the host.
+struct AppendView {
+    uint8_t *codes[2];    // K, V
+    float *scalemin[2];
+    uint16_t *window[2];  // bf16 ring [H][cap_window][D] (may be null when cap_window == 0)
+    int64_t cap_packed;
+    int64_t packed_row;   // packed index the flushed token goes to (if flush)
+    int32_t cap_window;
+    int32_t slot;         // ring slot written by the new token (-1: no window)
+    int32_t flush;        // 1: quantize (oldest slot | new token) into packed_row
+    int32_t bits;
+};
+
+constexpr int kAppendMaxViews = 128;
+
+struct AppendArgs {
+    const uint16_t *k_new;  // bf16 [n_views][H][D]
+    const uint16_t *v_new;
+    int32_t n_views;
+    int32_t n_kv_heads;
+    AppendView views[kAppendMaxViews];
+};
+
+// Grid: (n_views, n_kv_heads, 2 = K/V); one warp per block.  Lanes 0..2*NG-1
+// each own half a group of the row being flushed (same arithmetic as the
+// bulk quantize kernel); all lanes then copy the new token into the ring.
+template <int NG>
+__global__ void __launch_bounds__(32) append_kernel(AppendArgs a) {
+    constexpr int D = NG * kGroup;
+    const AppendView &v = a.views[blockIdx.x];
+    const int h = blockIdx.y;
+    const int kv = blockIdx.z;
+    const int lane = threadIdx.x;
+    const uint16_t *newrow = (kv ? a.v_new : a.k_new) + ((int64_t)blockIdx.x * a.n_kv_heads + h) * D;
+    uint16_t *ring = v.window[kv];
+    uint16_t *slotrow = (v.slot >= 0) ? ring + ((int64_t)h * v.cap_window + v.slot) * D : nullptr;
+
+    // 1) quantize the flushed row: the oldest ring token, or the new token if there is no ring
+    if (v.flush) {
+        const uint16_t *src = (v.cap_window > 0) ? slotrow : newrow;
+        const int g = lane >> 1, half = lane & 1;
+        const bool active = g < NG;
+        uint32_t x[16];
+        if (active) {
+            const uint4 *p = reinterpret_cast<const uint4 *>(src + g * kGroup + half * 32);
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+                const uint4 q = p[k];
+                x[4 * k] = q.x; x[4 * k + 1] = q.y; x[4 * k + 2] = q.z; x[4 * k + 3] = q.w;
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 16; ++i) x[i] = 0u;
+        }
+        float s, mn;
+        uint8_t *codes_row = v.codes[kv] + ((int64_t)h * v.cap_packed + v.packed_row) * (8 * v.bits * NG);
+        float *sm_row = v.scalemin[kv] + ((int64_t)h * v.cap_packed + v.packed_row) * NG * 2;
+        switch (v.bits) {
+#define KVQ_APPEND_Q(BB)                                                                         \
+    case BB: {                                                                                   \
+        uint32_t packed[BB];                                                                     \
+        quantize_half_group<BB>(x, packed, s, mn);                                               \
+        if (active) {                                                                            \
+            uint32_t *dst = reinterpret_cast<uint32_t *>(codes_row + g * 8 * BB + half * 4 * BB); \
+            _Pragma("unroll") for (int w = 0; w < BB; ++w) dst[w] = packed[w];                    \
+        }                                                                                        \
+    } break;
+            KVQ_APPEND_Q(2)
+            KVQ_APPEND_Q(3)
+            KVQ_APPEND_Q(4)
+            KVQ_APPEND_Q(8)
+#undef KVQ_APPEND_Q
+            default: s = 0.f; mn = 0.f; break;
+        }
+        if (active && half == 0) *reinterpret_cast<float2 *>(sm_row + g * 2) = make_float2(s, mn);
+    }
+    __syncwarp();
+    // 2) the new token takes its ring slot
+    if (slotrow) {
+        const uint4 *src = reinterpret_cast<const uint4 *>(newrow);
+        uint4 *dst = reinterpret_cast<uint4 *>(slotrow);
+        for (int i = lane; i < D / 8; i += 32) dst[i] = src[i];
+    }
+}
+
+}  // namespace kvq
