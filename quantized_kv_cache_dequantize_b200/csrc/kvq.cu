@@ -39,12 +39,12 @@ int device_sm_count() {
 
 template <int B, int NG>
 void launch_codec(bool quant, const kvq::CodecArgs &a, cudaStream_t st) {
+    // grid-stride over each head's groups; about 8 blocks of 8 warps per SM in total
     const int64_t groups = a.n_tokens * NG;
-    const int64_t warps_needed = (groups + 15) / 16;
-    const int sms = device_sm_count();
-    int64_t blocks = (warps_needed + 7) / 8;  // 8 warps per block
-    const int64_t cap = std::max<int64_t>(1, (int64_t)sms * 8 / std::max(1, a.n_heads));
-    blocks = std::max<int64_t>(1, std::min<int64_t>(blocks, std::max<int64_t>(cap, 4)));
+    const int64_t warp_groups = 16 * (quant ? kvq::kRounds : kvq::kDeqRounds);
+    const int64_t max_blocks = std::max<int64_t>(1, (groups + 8 * warp_groups - 1) / (8 * warp_groups));
+    const int64_t want = ((int64_t)device_sm_count() * 8 + a.n_heads - 1) / a.n_heads;
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(max_blocks, want));
     dim3 grid((unsigned)blocks, (unsigned)a.n_heads);
     if (quant)
         kvq::quantize_kernel<B, NG><<<grid, 256, 0, st>>>(a);
@@ -100,12 +100,16 @@ struct AttnLaunch {
     int total_chunks;
 };
 
+struct ViewChunks {
+    int32_t chunk_packed, chunk_window, n_packed, n_window;  // tokens per chunk, chunk counts
+};
+
 struct AttnPlan {
-    int chunk = 0;
     int ring_bytes = 0;
     size_t smem = 0;
     int head_blocks = 0;
     std::vector<AttnLaunch> launches;
+    std::vector<ViewChunks> chunks;
     size_t counters_off = 0, partials_off = 0, total = 0;
 };
 
@@ -116,7 +120,7 @@ int env_int(const char *name, int dflt) {
     return v > 0 ? (int)v : dflt;
 }
 
-kvq_status validate_views(const kvq_view *views, int32_t n_views, int32_t head_dim, bool need_nonempty) {
+kvq_status validate_views(const kvq_view *views, int32_t n_views, bool need_nonempty) {
     if (!views || n_views <= 0) return KVQ_ERR_INVALID_ARG;
     for (int i = 0; i < n_views; ++i) {
         const kvq_view &v = views[i];
@@ -137,8 +141,99 @@ kvq_status validate_views(const kvq_view *views, int32_t n_views, int32_t head_d
                 return KVQ_ERR_INVALID_ARG;
         }
     }
-    (void)head_dim;
     return KVQ_OK;
+}
+
+int attn_ctas_per_sm(int ng) {
+    switch (ng) {
+        case 1: return kvq::attn_ctas_per_sm<1>();
+        case 2: return kvq::attn_ctas_per_sm<2>();
+        case 3: return kvq::attn_ctas_per_sm<3>();
+        default: return kvq::attn_ctas_per_sm<4>();
+    }
+}
+
+int attn_header_bytes(int ng) {
+    switch (ng) {
+        case 1: return kvq::attn_header_bytes<1>();
+        case 2: return kvq::attn_header_bytes<2>();
+        case 3: return kvq::attn_header_bytes<3>();
+        default: return kvq::attn_header_bytes<4>();
+    }
+}
+
+// Bytes of one unit's packed token (K and V codes + scale/min) and window token.
+int64_t packed_token_bytes(int32_t head_dim, int32_t bits) { return 2 * row_bytes(head_dim, bits) + 16 * (head_dim / 64); }
+int64_t window_token_bytes(int32_t head_dim) { return 4 * (int64_t)head_dim; }
+
+// Chunk the views of one launch so that work items carry about equal bytes
+// and the item count fills the GPU's resident CTA slots in whole waves.
+int64_t chunk_views(const kvq_view *views, int v0, int v1, int64_t units, int32_t head_dim, int64_t slots,
+                    std::vector<ViewChunks> &out) {
+    double total = 0;
+    for (int i = v0; i < v1; ++i)
+        total += (double)units * ((double)views[i].n_packed * packed_token_bytes(head_dim, views[i].bits) +
+                                  (double)views[i].n_window * window_token_bytes(head_dim));
+    auto count = [&](double W, bool store) -> int64_t {
+        int64_t items = 0;
+        for (int i = v0; i < v1; ++i) {
+            const kvq_view &v = views[i];
+            ViewChunks c{16, 16, 0, 0};
+            if (v.n_packed > 0) {
+                const double b = (double)v.n_packed * packed_token_bytes(head_dim, v.bits);
+                int64_t n = std::max<int64_t>(1, (int64_t)std::llround(b / W));
+                int64_t ch = (v.n_packed + n - 1) / n;
+                ch = std::max<int64_t>(128, (ch + 127) / 128 * 128);  // whole 32-token steps for 4 warps
+                c.chunk_packed = (int32_t)ch;
+                c.n_packed = (int32_t)((v.n_packed + ch - 1) / ch);
+            }
+            if (v.n_window > 0) {
+                const double b = (double)v.n_window * window_token_bytes(head_dim);
+                int64_t n = std::max<int64_t>(1, (int64_t)std::llround(b / W));
+                int64_t ch = (v.n_window + n - 1) / n;
+                ch = std::max<int64_t>(64, (ch + 63) / 64 * 64);  // whole 16-token steps for 4 warps
+                c.chunk_window = (int32_t)ch;
+                c.n_window = (int32_t)((v.n_window + ch - 1) / ch);
+            }
+            const int forced = env_int("KVQ_CHUNK_TOKENS", 0);
+            if (forced > 0) {
+                const int ch = std::max(32, forced / 32 * 32);
+                c.chunk_packed = c.chunk_window = ch;
+                c.n_packed = (int32_t)((v.n_packed + ch - 1) / ch);
+                c.n_window = (int32_t)((v.n_window + ch - 1) / ch);
+            }
+            // the in-kernel merge holds at most kMaxChunksPerUnit chunks per unit
+            while (c.n_packed + c.n_window > kvq::kMaxChunksPerUnit) {
+                if (c.n_packed >= c.n_window) {
+                    c.chunk_packed *= 2;
+                    c.n_packed = (int32_t)((v.n_packed + c.chunk_packed - 1) / c.chunk_packed);
+                } else {
+                    c.chunk_window *= 2;
+                    c.n_window = (int32_t)((v.n_window + c.chunk_window - 1) / c.chunk_window);
+                }
+            }
+            items += c.n_packed + c.n_window;
+            if (store) out[i] = c;
+        }
+        return items;
+    };
+    const double kMinItem = 24.0 * 1024, kBigItem = 192.0 * 1024;
+    double W = total / (double)slots;
+    if (W >= kBigItem) {
+        W = kBigItem;  // many waves: the tail is small anyway
+    } else {
+        double chosen = std::max(total / (double)(slots * 8), kMinItem);
+        for (int waves = 1; waves <= 8; ++waves) {
+            const double Ww = total / (double)(slots * waves);
+            if (Ww < kMinItem) break;
+            if (count(Ww, false) * units <= slots * waves) {
+                chosen = Ww;
+                break;
+            }
+        }
+        W = chosen;
+    }
+    return count(W, true);
 }
 
 kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, int32_t n_kv_heads,
@@ -146,57 +241,51 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, 
     if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
     if (n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads || n_kv_heads > 65535)
         return KVQ_ERR_INVALID_ARG;
-    const kvq_status vs = validate_views(views, n_views, head_dim, true);
+    const kvq_status vs = validate_views(views, n_views, true);
     if (vs != KVQ_OK) return vs;
     const int ng = head_dim / 64;
     const int group = n_q_heads / n_kv_heads;
     plan.head_blocks = (group + kvq::kHeadsPerCta - 1) / kvq::kHeadsPerCta;
     if (plan.head_blocks > 65535) return KVQ_ERR_UNSUPPORTED;
+    const int64_t units = (int64_t)n_kv_heads * plan.head_blocks;
 
-    // chunk size: aim for ~4 CTAs per SM over the whole call, in 16-token
-    // tiles, at least 256 tokens so a CTA amortises its set-up
-    int64_t total_tokens = 0;
-    uint32_t stage_max = 0;
+    // shared memory: the CTA's share of the SM at the kernel's target occupancy
+    const int ctas = attn_ctas_per_sm(ng);
+    const int smem_cta = std::min(227 * 1024, (228 * 1024) / ctas - 1024);
+    const int header = attn_header_bytes(ng);
+    uint32_t blk_max = 0;
     for (int i = 0; i < n_views; ++i) {
-        total_tokens += views[i].n_packed + views[i].n_window;
         if (views[i].n_packed > 0)
-            stage_max = std::max<uint32_t>(stage_max, (uint32_t)(32 * row_bytes(head_dim, views[i].bits) + 256 * ng));
-        if (views[i].n_window > 0) stage_max = std::max<uint32_t>(stage_max, (uint32_t)(32 * head_dim));
+            blk_max = std::max<uint32_t>(blk_max, (uint32_t)(64 * row_bytes(head_dim, views[i].bits) + 512 * ng));
+        if (views[i].n_window > 0) blk_max = std::max<uint32_t>(blk_max, (uint32_t)(32 * head_dim));
     }
-    total_tokens *= (int64_t)n_kv_heads * plan.head_blocks;
-    const int64_t target_ctas = (int64_t)device_sm_count() * 4;
-    int64_t chunk = (total_tokens + target_ctas - 1) / target_ctas;
-    chunk = std::max<int64_t>(256, std::min<int64_t>(chunk, 8192));
-    chunk = (chunk + 63) / 64 * 64;
-    plan.chunk = env_int("KVQ_CHUNK_TOKENS", (int)chunk);
-    plan.chunk = std::max(16, plan.chunk / 16 * 16);
-
-    int ring = std::max<int>(16384, (int)(2 * stage_max));
-    ring = std::max(ring, 64 + 32 * head_dim);
-    ring = (ring + 127) / 128 * 128;
+    int ring = (smem_cta - header) / kvq::kAttnWarps / 128 * 128;
+    // a ring holds two blocks, and later the warp's partial; all rings together
+    // hold the unit merge's scratch
+    const uint32_t merge_scratch = (2 * kvq::kMaxChunksPerUnit * kvq::kHeadsPerCta + kvq::kHeadsPerCta) * 4;
+    const int ring_min = (int)std::max<uint32_t>(std::max<uint32_t>(2 * blk_max, (uint32_t)(64 + 32 * head_dim)),
+                                                 (merge_scratch + kvq::kAttnWarps - 1) / kvq::kAttnWarps);
+    if (ring < ring_min) ring = (ring_min + 127) / 128 * 128;  // fewer CTAs per SM, still correct
     plan.ring_bytes = ring;
-    const size_t header = (size_t)((8 * head_dim * 2 + 8 * ng * 4 + kvq::kAttnWarps * kvq::kMaxStages * 8 + 16 + 127) & ~127);
-    plan.smem = header + (size_t)kvq::kAttnWarps * ring;
+    plan.smem = (size_t)header + (size_t)kvq::kAttnWarps * ring;
     if (plan.smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;
 
+    const int64_t slots = (int64_t)device_sm_count() * ctas;
+    plan.chunks.assign(n_views, ViewChunks{16, 16, 0, 0});
     int64_t max_chunks = 0;
     int max_views = 0;
     for (int v0 = 0; v0 < n_views; v0 += kvq::kAttnMaxViews) {
         const int v1 = std::min<int>(n_views, v0 + kvq::kAttnMaxViews);
-        int64_t chunks = 0;
-        for (int i = v0; i < v1; ++i) {
-            chunks += (views[i].n_packed + plan.chunk - 1) / plan.chunk;
-            chunks += (views[i].n_window + plan.chunk - 1) / plan.chunk;
-        }
+        const int64_t chunks = chunk_views(views, v0, v1, units, head_dim, slots, plan.chunks);
         if (chunks > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
         plan.launches.push_back({v0, v1, (int)chunks});
         max_chunks = std::max(max_chunks, chunks);
         max_views = std::max(max_views, v1 - v0);
     }
-    const size_t units = (size_t)max_views * n_kv_heads * plan.head_blocks;
+    const size_t n_units = (size_t)max_views * units;
     plan.counters_off = 256;
-    plan.partials_off = plan.counters_off + (units * 4 + 255) / 256 * 256;
-    const size_t part_floats = (size_t)max_chunks * n_kv_heads * plan.head_blocks * kvq::kHeadsPerCta * (head_dim + 2);
+    plan.partials_off = plan.counters_off + (n_units * 4 + 255) / 256 * 256;
+    const size_t part_floats = (size_t)max_chunks * units * kvq::kHeadsPerCta * (head_dim + 2);
     plan.total = plan.partials_off + part_floats * 4;
     return KVQ_OK;
 }
@@ -207,11 +296,11 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
     static int configured_smem[64] = {0};
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
-    if (dev < 64 && configured_smem[dev] < (int)plan.smem) {
+    if (dev >= 64 || configured_smem[dev] < (int)plan.smem) {
         if (cudaFuncSetAttribute(kvq::decode_attn_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)plan.smem) != cudaSuccess)
             return KVQ_ERR_CUDA;
-        configured_smem[dev] = (int)plan.smem;
+        if (dev < 64) configured_smem[dev] = (int)plan.smem;
     }
     kvq::AttnParams prm;
     std::memset(&prm, 0, sizeof prm);
@@ -226,13 +315,13 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
     prm.n_kv_heads = n_kv_heads;
     prm.group = n_q_heads / n_kv_heads;
     prm.head_blocks = plan.head_blocks;
-    prm.chunk = plan.chunk;
     prm.ring_bytes = plan.ring_bytes;
     for (const AttnLaunch &L : plan.launches) {
         prm.n_views = L.v1 - L.v0;
         int begin = 0;
         for (int i = L.v0; i < L.v1; ++i) {
             const kvq_view &v = views[i];
+            const ViewChunks &c = plan.chunks[i];
             kvq::AttnView &d = prm.views[i - L.v0];
             d.codes[0] = static_cast<const uint8_t *>(v.k_codes);
             d.codes[1] = static_cast<const uint8_t *>(v.v_codes);
@@ -246,8 +335,10 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
             d.cap_window = v.cap_window;
             d.window_head = v.window_head;
             d.bits = v.n_packed > 0 ? v.bits : 4;
-            d.n_chunks_packed = (int32_t)((v.n_packed + plan.chunk - 1) / plan.chunk);
-            d.n_chunks = d.n_chunks_packed + (v.n_window + plan.chunk - 1) / plan.chunk;
+            d.chunk_packed = c.chunk_packed;
+            d.chunk_window = c.chunk_window;
+            d.n_chunks_packed = c.n_packed;
+            d.n_chunks = c.n_packed + c.n_window;
             d.chunk_begin = begin;
             d.view_index = i;
             begin += d.n_chunks;
@@ -294,7 +385,7 @@ KVQ_API kvq_status kvq_append(kvq_view *views, int32_t n_views, int32_t n_kv_hea
                               const void *k_new, const void *v_new, void *stream) {
     if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
     if (n_kv_heads <= 0 || n_kv_heads > 65535) return KVQ_ERR_INVALID_ARG;
-    const kvq_status vs = validate_views(views, n_views, head_dim, false);
+    const kvq_status vs = validate_views(views, n_views, false);
     if (vs != KVQ_OK) return vs;
     if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return KVQ_ERR_INVALID_ARG;
     // first pass: every view must be able to take the token

@@ -42,9 +42,10 @@ namespace kvq {
 constexpr int kAttnWarps = 4;
 constexpr int kAttnThreads = 32 * kAttnWarps;
 constexpr int kTile = 16;
-constexpr int kMaxStages = 8;
+constexpr int kMaxStages = 12;
 constexpr int kHeadsPerCta = 8;
 constexpr int kAttnMaxViews = 96;
+constexpr int kMaxChunksPerUnit = 256;  // merge scratch: 2 * 256 * 8 floats in the ring area
 
 struct AttnView {
     const uint8_t *codes[2];     // K, V packed rows [H_kv][cap][RB]
@@ -56,6 +57,8 @@ struct AttnView {
     int32_t cap_window;
     int32_t window_head;
     int32_t bits;
+    int32_t chunk_packed;        // tokens per packed chunk (multiple of 16)
+    int32_t chunk_window;        // tokens per window chunk (multiple of 16)
     int32_t n_chunks_packed;
     int32_t n_chunks;            // packed + window chunks
     int32_t chunk_begin;         // first chunk index of this view in the launch
@@ -76,8 +79,8 @@ struct AttnParams {
     int32_t n_kv_heads;
     int32_t group;               // n_q_heads / n_kv_heads
     int32_t head_blocks;         // ceil(group / 8)
-    int32_t chunk;               // tokens per chunk, multiple of 16
     int32_t ring_bytes;          // shared-memory ring per warp
+    int32_t pad_;
     AttnView views[kAttnMaxViews];
 };
 
@@ -251,33 +254,48 @@ __device__ __forceinline__ void pv_unpack<8>(const uint8_t *sa, const uint8_t *s
 
 // ------------------------------------------------------------ per-warp ----
 
+// 2^x on the special-function unit (relative error about 2^-22; 2^-inf = 0)
+__device__ __forceinline__ float fast_exp2(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+    return y;
+}
+
 template <int NG>
 struct WarpState {
-    float o[NG][4][4];   // O^T tiles: group g, d-tile t; (row gid|gid+8) x (head 2tig|2tig+1)
-    float mt[NG][2];     // min-term partial sums, heads 2tig, 2tig+1
-    float m[2];          // running max (log2 units)
-    float l[2];          // running sum (partial over this lane's rows)
+    float o[NG][4][4];      // O^T tiles: group g, d-tile t; (row gid|gid+8) x (head 2tig|2tig+1)
+    float mt[NG][2];        // min-term partial sums, heads 2tig, 2tig+1
+    float m[2];             // running max (log2 units), heads 2tig, 2tig+1
+    float l[2];             // running sum (partial over this lane's rows)
     uint32_t bq[NG][4][2];  // q as B operand: group, k-step, (b0b1, b2b3)
-    float qsum[NG][2];
+    float qsum[NG][2];      // sum of q over each group, heads 2tig, 2tig+1
 };
 
-// Online-softmax step for one 16-token tile: lg[row][head] are base-2 logits
-// of rows gid, gid+8 and heads 2tig, 2tig+1.  Returns the probabilities in lg.
-template <int NG>
-__device__ __forceinline__ void softmax_step(WarpState<NG> &st, float (&lg)[2][2]) {
+// Online-softmax step over R row-sets (R = 2: one 16-token tile, rows gid and
+// gid+8; R = 4: two tiles).  lg[r][j] are base-2 logits of this lane's rows
+// for heads 2tig, 2tig+1; they are replaced by the probabilities relative to
+// the new running max.
+template <int NG, int R>
+__device__ __forceinline__ void softmax_step_n(WarpState<NG> &st, float (&lg)[R][2]) {
     float alpha[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-        float t = fmaxf(lg[0][j], lg[1][j]);
+        float t = lg[0][j];
+#pragma unroll
+        for (int r = 1; r < R; ++r) t = fmaxf(t, lg[r][j]);
         t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 4));
         t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 8));
         t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 16));
         const float mnew = fmaxf(st.m[j], t);
-        alpha[j] = exp2f(st.m[j] - mnew);
+        alpha[j] = fast_exp2(st.m[j] - mnew);
         st.m[j] = mnew;
-        lg[0][j] = exp2f(lg[0][j] - mnew);
-        lg[1][j] = exp2f(lg[1][j] - mnew);
-        st.l[j] = st.l[j] * alpha[j] + (lg[0][j] + lg[1][j]);
+        float sum = 0.f;
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            lg[r][j] = fast_exp2(lg[r][j] - mnew);
+            sum += lg[r][j];
+        }
+        st.l[j] = fmaf(st.l[j], alpha[j], sum);
     }
     if (__any_sync(0xFFFFFFFFu, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
 #pragma unroll
@@ -295,7 +313,8 @@ __device__ __forceinline__ void softmax_step(WarpState<NG> &st, float (&lg)[2][2
     }
 }
 
-// hi/lo bf16 split of a probability-like pair and transpose to B layout
+// hi/lo bf16 split of the 16x8 tile (rows gid, gid+8; heads 2tig, 2tig+1)
+// and transpose of both halves to the B-operand layout (tokens along k).
 __device__ __forceinline__ void split_transpose(float a0, float a1, float b0, float b1, uint32_t &bh0,
                                                 uint32_t &bh1, uint32_t &bl0, uint32_t &bl1) {
     const uint32_t h0 = pack_bf16x2(a0, a1);
@@ -308,75 +327,123 @@ __device__ __forceinline__ void split_transpose(float a0, float a1, float b0, fl
     bl1 = movmatrix_trans(l1);
 }
 
-// One 16-token tile of packed tokens.  Stage layout: K codes [16][RB], V codes
-// [16][RB], K scalemin [16][NG] float2, V scalemin [16][NG] float2.
+// QK of one 16-token tile of packed codes: codes rows at `kc` (row stride RB),
+// K scale/min rows at `ks` ([row][NG] float2).  Writes base-2 logits of rows
+// gid, gid+8 (lg0, lg1) for heads 2tig, 2tig+1; rows at or past n_valid are
+// -inf.
 template <int B, int NG>
-__device__ __forceinline__ void packed_tile(WarpState<NG> &st, const uint8_t *stage, int n_valid,
-                                            float scale_log2, int gid, int tig) {
+__device__ __forceinline__ void packed_qk1(const WarpState<NG> &st, const uint8_t *kc, const uint8_t *ks_bytes,
+                                           int n_valid, float scale_log2, int gid, int tig, float (&lg0)[2],
+                                           float (&lg1)[2]) {
     constexpr int RB = 8 * B * NG;
-    const uint8_t *kc = stage;
-    const uint8_t *vc = stage + 16 * RB;
-    const float2 *ks = reinterpret_cast<const float2 *>(stage + 32 * RB);
-    const float2 *vs = ks + 16 * NG;
-    const int r0 = gid, r1 = gid + 8;
-    const bool v0 = r0 < n_valid, v1 = r1 < n_valid;
-
-    float lg[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+    const float2 *sm = reinterpret_cast<const float2 *>(ks_bytes);
+    const uint8_t *row0 = kc + gid * RB + 2 * B * tig;
+    const uint8_t *row1 = row0 + 8 * RB;
+    float l00 = 0.f, l01 = 0.f, l10 = 0.f, l11 = 0.f;
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
         uint32_t a0[8], a1[8];
-        qk_unpack<B>(kc + r0 * RB + g * 8 * B + 2 * B * tig, a0);
-        qk_unpack<B>(kc + r1 * RB + g * 8 * B + 2 * B * tig, a1);
+        qk_unpack<B>(row0 + g * 8 * B, a0);
+        qk_unpack<B>(row1 + g * 8 * B, a1);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int s = 0; s < 4; ++s)
             mma_bf16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0], st.bq[g][s][1]);
-        const float2 k0 = ks[r0 * NG + g], k1 = ks[r1 * NG + g];
-        lg[0][0] = fmaf(k0.x, acc[0], fmaf(k0.y, st.qsum[g][0], lg[0][0]));
-        lg[0][1] = fmaf(k0.x, acc[1], fmaf(k0.y, st.qsum[g][1], lg[0][1]));
-        lg[1][0] = fmaf(k1.x, acc[2], fmaf(k1.y, st.qsum[g][0], lg[1][0]));
-        lg[1][1] = fmaf(k1.x, acc[3], fmaf(k1.y, st.qsum[g][1], lg[1][1]));
+        const float2 k0 = sm[gid * NG + g], k1 = sm[(gid + 8) * NG + g];
+        l00 = fmaf(k0.x, acc[0], fmaf(k0.y, st.qsum[g][0], l00));
+        l01 = fmaf(k0.x, acc[1], fmaf(k0.y, st.qsum[g][1], l01));
+        l10 = fmaf(k1.x, acc[2], fmaf(k1.y, st.qsum[g][0], l10));
+        l11 = fmaf(k1.x, acc[3], fmaf(k1.y, st.qsum[g][1], l11));
     }
-#pragma unroll
-    for (int j = 0; j < 2; ++j) {
-        lg[0][j] = v0 ? lg[0][j] * scale_log2 : -INFINITY;
-        lg[1][j] = v1 ? lg[1][j] * scale_log2 : -INFINITY;
-    }
-    softmax_step<NG>(st, lg);
+    // rows past the valid count hold stale stage bytes: drop them
+    const bool v0 = gid < n_valid, v1 = gid + 8 < n_valid;
+    lg0[0] = v0 ? l00 * scale_log2 : -INFINITY;
+    lg0[1] = v0 ? l01 * scale_log2 : -INFINITY;
+    lg1[0] = v1 ? l10 * scale_log2 : -INFINITY;
+    lg1[1] = v1 ? l11 * scale_log2 : -INFINITY;
+}
 
+// QK of both (full) tiles of a packed block; lg rows: tile A gid, tile A
+// gid+8, tile B gid, tile B gid+8.  The two tiles' MMA chains interleave.
+template <int B, int NG>
+__device__ __forceinline__ void packed_qk2(const WarpState<NG> &st, const uint8_t *blk, float scale_log2, int gid,
+                                           int tig, float (&lg)[4][2]) {
+    constexpr int RB = 8 * B * NG;
+    const float2 *sm = reinterpret_cast<const float2 *>(blk + 4 * kTile * RB);
+    const uint8_t *row0 = blk + gid * RB + 2 * B * tig;
+    float l[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
-        float2 m0 = vs[r0 * NG + g], m1 = vs[r1 * NG + g];
-        if (!v0) m0 = make_float2(0.f, 0.f);
-        if (!v1) m1 = make_float2(0.f, 0.f);
-        st.mt[g][0] = fmaf(lg[0][0], m0.y, fmaf(lg[1][0], m1.y, st.mt[g][0]));
-        st.mt[g][1] = fmaf(lg[0][1], m0.y, fmaf(lg[1][1], m1.y, st.mt[g][1]));
-        uint32_t bh0, bh1, bl0, bl1;
-        split_transpose(lg[0][0] * m0.x, lg[0][1] * m0.x, lg[1][0] * m1.x, lg[1][1] * m1.x, bh0, bh1, bl0, bl1);
-        uint32_t va[8], vb[8];
-        const int off = g * 8 * B + B * gid;
-        pv_unpack<B>(vc + (2 * tig) * RB + off, vc + (2 * tig + 1) * RB + off, va);
-        pv_unpack<B>(vc + (2 * tig + 8) * RB + off, vc + (2 * tig + 9) * RB + off, vb);
 #pragma unroll
-        for (int t = 0; t < 4; ++t) {
-            mma_bf16_16816(st.o[g][t], va[2 * t], va[2 * t + 1], vb[2 * t], vb[2 * t + 1], bh0, bh1);
-            mma_bf16_16816(st.o[g][t], va[2 * t], va[2 * t + 1], vb[2 * t], vb[2 * t + 1], bl0, bl1);
+        for (int tt = 0; tt < 2; ++tt) {
+            uint32_t a0[8], a1[8];
+            qk_unpack<B>(row0 + tt * kTile * RB + g * 8 * B, a0);
+            qk_unpack<B>(row0 + tt * kTile * RB + 8 * RB + g * 8 * B, a1);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+            for (int s = 0; s < 4; ++s)
+                mma_bf16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0],
+                               st.bq[g][s][1]);
+            const float2 k0 = sm[(tt * kTile + gid) * NG + g], k1 = sm[(tt * kTile + gid + 8) * NG + g];
+            l[2 * tt][0] = fmaf(k0.x, acc[0], fmaf(k0.y, st.qsum[g][0], l[2 * tt][0]));
+            l[2 * tt][1] = fmaf(k0.x, acc[1], fmaf(k0.y, st.qsum[g][1], l[2 * tt][1]));
+            l[2 * tt + 1][0] = fmaf(k1.x, acc[2], fmaf(k1.y, st.qsum[g][0], l[2 * tt + 1][0]));
+            l[2 * tt + 1][1] = fmaf(k1.x, acc[3], fmaf(k1.y, st.qsum[g][1], l[2 * tt + 1][1]));
         }
+    }
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        lg[r][0] = l[r][0] * scale_log2;
+        lg[r][1] = l[r][1] * scale_log2;
     }
 }
 
-// Window tile, K half: stage = K rows [16][D] bf16.  Returns base-2 logits.
-template <int NG>
-__device__ __forceinline__ void window_qk(WarpState<NG> &st, const uint8_t *stage, int n_valid,
+// PV of one 16-token tile: V codes rows at `vc` (row stride RB), V scale/min
+// rows at `vs` ([row][NG] float2); p0/p1 are this lane's probabilities of
+// rows gid, gid+8.  FULL == false zeroes the scale/min of rows at or past
+// n_valid (stale stage bytes; p is 0 there but 0 * NaN would not be).
+template <int B, int NG, bool FULL>
+__device__ __forceinline__ void packed_pv(WarpState<NG> &st, const uint8_t *vc, const uint8_t *vs_bytes, int rows,
+                                          int n_valid, const float (&p0)[2], const float (&p1)[2], int gid, int tig) {
+    constexpr int RB = 8 * B * NG;
+    (void)rows;
+    const float2 *sm = reinterpret_cast<const float2 *>(vs_bytes);
+    const uint8_t *ta = vc + (2 * tig) * RB + B * gid;
+    const uint8_t *tb = ta + RB;
+    const uint8_t *tc = ta + 8 * RB;
+    const uint8_t *td = ta + 9 * RB;
+#pragma unroll
+    for (int g = 0; g < NG; ++g) {
+        float2 m0 = sm[gid * NG + g], m1 = sm[(gid + 8) * NG + g];
+        if (!FULL) {
+            if (gid >= n_valid) m0 = make_float2(0.f, 0.f);
+            if (gid + 8 >= n_valid) m1 = make_float2(0.f, 0.f);
+        }
+        st.mt[g][0] = fmaf(p0[0], m0.y, fmaf(p1[0], m1.y, st.mt[g][0]));
+        st.mt[g][1] = fmaf(p0[1], m0.y, fmaf(p1[1], m1.y, st.mt[g][1]));
+        uint32_t bh0, bh1, bl0, bl1;
+        split_transpose(p0[0] * m0.x, p0[1] * m0.x, p1[0] * m1.x, p1[1] * m1.x, bh0, bh1, bl0, bl1);
+        uint32_t va[8], vb[8];
+        pv_unpack<B>(ta + g * 8 * B, tb + g * 8 * B, va);
+        pv_unpack<B>(tc + g * 8 * B, td + g * 8 * B, vb);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) mma_bf16_16816(st.o[g][t], va[2 * t], va[2 * t + 1], vb[2 * t], vb[2 * t + 1], bh0, bh1);
+#pragma unroll
+        for (int t = 0; t < 4; ++t) mma_bf16_16816(st.o[g][t], va[2 * t], va[2 * t + 1], vb[2 * t], vb[2 * t + 1], bl0, bl1);
+    }
+}
+
+// K half of a window tile: block = K rows [16][D] bf16.
+template <int NG, bool FULL>
+__device__ __forceinline__ void window_qk(const WarpState<NG> &st, const uint8_t *blk, int n_valid,
                                           float scale_log2, int gid, int tig, float (&lg)[2][2]) {
     constexpr int D = 64 * NG;
-    const uint16_t *k = reinterpret_cast<const uint16_t *>(stage);
-    const int r0 = gid, r1 = gid + 8;
+    const uint16_t *k = reinterpret_cast<const uint16_t *>(blk);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
-        const uint4 *p0 = reinterpret_cast<const uint4 *>(k + r0 * D + 64 * g + 16 * tig);
-        const uint4 *p1 = reinterpret_cast<const uint4 *>(k + r1 * D + 64 * g + 16 * tig);
+        const uint4 *p0 = reinterpret_cast<const uint4 *>(k + gid * D + 64 * g + 16 * tig);
+        const uint4 *p1 = reinterpret_cast<const uint4 *>(k + (gid + 8) * D + 64 * g + 16 * tig);
         const uint4 x0 = p0[0], x1 = p0[1], y0 = p1[0], y1 = p1[1];
         const uint32_t a0[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
         const uint32_t a1[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
@@ -384,19 +451,22 @@ __device__ __forceinline__ void window_qk(WarpState<NG> &st, const uint8_t *stag
         for (int s = 0; s < 4; ++s)
             mma_bf16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0], st.bq[g][s][1]);
     }
-    const bool v0 = r0 < n_valid, v1 = r1 < n_valid;
-    lg[0][0] = v0 ? acc[0] * scale_log2 : -INFINITY;
-    lg[0][1] = v0 ? acc[1] * scale_log2 : -INFINITY;
-    lg[1][0] = v1 ? acc[2] * scale_log2 : -INFINITY;
-    lg[1][1] = v1 ? acc[3] * scale_log2 : -INFINITY;
+    lg[0][0] = acc[0] * scale_log2;
+    lg[0][1] = acc[1] * scale_log2;
+    lg[1][0] = acc[2] * scale_log2;
+    lg[1][1] = acc[3] * scale_log2;
+    if (!FULL) {
+        if (gid >= n_valid) lg[0][0] = lg[0][1] = -INFINITY;
+        if (gid + 8 >= n_valid) lg[1][0] = lg[1][1] = -INFINITY;
+    }
 }
 
-// Window tile, V half: stage = V rows [16][D] bf16; lg holds probabilities.
-template <int NG>
-__device__ __forceinline__ void window_pv(WarpState<NG> &st, const uint8_t *stage, int n_valid,
+// V half of a window tile: block = V rows [16][D] bf16.
+template <int NG, bool FULL>
+__device__ __forceinline__ void window_pv(WarpState<NG> &st, const uint8_t *blk, int n_valid,
                                           const float (&p)[2][2], int gid, int tig) {
     constexpr int D = 64 * NG;
-    const uint16_t *v = reinterpret_cast<const uint16_t *>(stage);
+    const uint16_t *v = reinterpret_cast<const uint16_t *>(blk);
     uint32_t bh0, bh1, bl0, bl1;
     split_transpose(p[0][0], p[0][1], p[1][0], p[1][1], bh0, bh1, bl0, bl1);
     const int ta = 2 * tig, tb = 2 * tig + 1, tc = 2 * tig + 8, td = 2 * tig + 9;
@@ -407,12 +477,13 @@ __device__ __forceinline__ void window_pv(WarpState<NG> &st, const uint8_t *stag
         uint4 xb = *reinterpret_cast<const uint4 *>(v + tb * D + col);
         uint4 xc = *reinterpret_cast<const uint4 *>(v + tc * D + col);
         uint4 xd = *reinterpret_cast<const uint4 *>(v + td * D + col);
-        // rows past the valid count hold stale bytes: zero them (p is 0 there,
-        // but 0 * NaN would not be)
-        if (ta >= n_valid) xa = make_uint4(0, 0, 0, 0);
-        if (tb >= n_valid) xb = make_uint4(0, 0, 0, 0);
-        if (tc >= n_valid) xc = make_uint4(0, 0, 0, 0);
-        if (td >= n_valid) xd = make_uint4(0, 0, 0, 0);
+        if (!FULL) {
+            // stale rows may hold non-finite bit patterns: zero them (p is 0 there)
+            if (ta >= n_valid) xa = make_uint4(0, 0, 0, 0);
+            if (tb >= n_valid) xb = make_uint4(0, 0, 0, 0);
+            if (tc >= n_valid) xc = make_uint4(0, 0, 0, 0);
+            if (td >= n_valid) xd = make_uint4(0, 0, 0, 0);
+        }
         const uint32_t wa[4] = {xa.x, xa.y, xa.z, xa.w}, wb[4] = {xb.x, xb.y, xb.z, xb.w};
         const uint32_t wc[4] = {xc.x, xc.y, xc.z, xc.w}, wd[4] = {xd.x, xd.y, xd.z, xd.w};
 #pragma unroll
@@ -430,187 +501,232 @@ __device__ __forceinline__ void window_pv(WarpState<NG> &st, const uint8_t *stag
 __device__ __forceinline__ uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
 
 template <int NG>
-__global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const __grid_constant__ AttnParams p) {
+__host__ __device__ constexpr int attn_ctas_per_sm() {
+    return NG <= 2 ? 4 : (NG == 3 ? 3 : 2);
+}
+
+template <int NG>
+__host__ __device__ constexpr int attn_header_bytes() {
+    return (8 * 64 * NG * 2 + kAttnWarps * kMaxStages * 8 + 16 + 127) & ~127;
+}
+
+// One work item: (view, KV head hk, query-head block z, chunk of tokens).
+// The chunk is cut into steps (32 packed tokens, or 16 window tokens); warp w
+// takes steps w, w+4, ...  A packed step is one block holding both halves of
+// two 16-token tiles (K codes, V codes, K scale/min, V scale/min); a window
+// step is two blocks (K rows, then V rows).  Blocks stream through the warp's
+// own ring of S equal slots, each with an mbarrier that counts the bytes of
+// the block's bulk copies; one lane issues the copies and a slot is refilled
+// as soon as the warp has consumed it.
+template <int NG, int B, bool WINDOW>
+__device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V, int vi, int c, int hk, int z,
+                                          uint8_t *smem) {
     constexpr int D = 64 * NG;
-    extern __shared__ __align__(128) uint8_t smem[];
-    uint16_t *q_s = reinterpret_cast<uint16_t *>(smem);                            // [8][D]
-    float *qsum_s = reinterpret_cast<float *>(smem + 8 * D * 2);                  // [8][NG]
-    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 8 * D * 2 + 8 * NG * 4);  // [4][8]
+    constexpr int RB = 8 * B * NG;
+    constexpr int kStepTok = WINDOW ? kTile : 2 * kTile;
+    constexpr int kBlkPerStep = WINDOW ? 2 : 1;
+    // packed block: [K codes 32*RB][V codes 32*RB][K sm 32*NG*8][V sm 32*NG*8]
+    constexpr uint32_t kOffV = 2 * kTile * RB, kOffKs = 4 * kTile * RB, kOffVs = kOffKs + 2 * kTile * NG * 8;
+    constexpr uint32_t kBlk = WINDOW ? (uint32_t)(kTile * D * 2) : (uint32_t)(kOffVs + 2 * kTile * NG * 8);
+    uint16_t *q_s = reinterpret_cast<uint16_t *>(smem);                              // [8][D]
+    uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 8 * D * 2);                // [4][kMaxStages]
     int *flag_s = reinterpret_cast<int *>(bars + kAttnWarps * kMaxStages);
-    uint8_t *rings = smem + ((8 * D * 2 + 8 * NG * 4 + kAttnWarps * kMaxStages * 8 + 16 + 127) & ~127);
+    uint8_t *rings = smem + attn_header_bytes<NG>();
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gid = lane >> 2, tig = lane & 3;
-
-    // ---- which unit
-    const int bx = blockIdx.x;
-    int lo = 0, hi = p.n_views - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (p.views[mid].chunk_begin <= bx) lo = mid; else hi = mid - 1;
-    }
-    const int vi = lo;
-    const AttnView &V = p.views[vi];
-    const int c = bx - V.chunk_begin;
-    const int hk = blockIdx.y, z = blockIdx.z;
     const int h0 = hk * p.group + z * kHeadsPerCta;
     const int nh = min(kHeadsPerCta, p.group - z * kHeadsPerCta);
-    const bool is_window = c >= V.n_chunks_packed;
-    const int64_t tok0 = (int64_t)(is_window ? c - V.n_chunks_packed : c) * p.chunk;
-    const int n_tok = (int)min((int64_t)p.chunk, (is_window ? (int64_t)V.n_window : (int64_t)V.n_packed) - tok0);
-    const int n_tiles = (n_tok + kTile - 1) / kTile;
-    const int B = V.bits;
-    const int RB = 8 * B * NG;
+    const int chunk = WINDOW ? V.chunk_window : V.chunk_packed;
+    const int64_t tok0 = (int64_t)(WINDOW ? c - V.n_chunks_packed : c) * chunk;
+    const int n_tok = (int)min((int64_t)chunk, (WINDOW ? (int64_t)V.n_window : (int64_t)V.n_packed) - tok0);
+    const int n_steps = (n_tok + kStepTok - 1) / kStepTok;
+    const int n_my = (warp < n_steps) ? (n_steps - warp + kAttnWarps - 1) / kAttnWarps : 0;
+    const int n_blocks = kBlkPerStep * n_my;
+    const int S = min(kMaxStages, (int)(p.ring_bytes / kBlk));
+    uint8_t *ring = rings + (size_t)warp * p.ring_bytes;
+    uint64_t *wbar = bars + warp * kMaxStages;
+    constexpr int kAdvTok = kAttnWarps * kStepTok;  // tokens between a warp's steps
 
-    // ---- q (bf16, zero rows past nh), per-group sums, barriers
+    // Copy sources at this warp's first step; incremental from then on (no
+    // integer division on the per-block path).
+    const uint8_t *src_kc = nullptr, *src_vc = nullptr;
+    const float *src_ks = nullptr, *src_vs = nullptr;
+    const uint16_t *win_k = nullptr, *win_v = nullptr;
+    int win_phys = 0;
+    if (!WINDOW) {
+        const int64_t row = (int64_t)hk * V.cap_packed + tok0 + kStepTok * warp;
+        src_kc = V.codes[0] + row * RB;
+        src_vc = V.codes[1] + row * RB;
+        src_ks = V.scalemin[0] + row * NG * 2;
+        src_vs = V.scalemin[1] + row * NG * 2;
+    } else {
+        win_k = V.window[0] + (int64_t)hk * V.cap_window * D;
+        win_v = V.window[1] + (int64_t)hk * V.cap_window * D;
+        win_phys = (int)(((int64_t)V.window_head + tok0 + kStepTok * warp) % V.cap_window);
+    }
+    int issue_blk = 0, issue_slot = 0, issue_left = n_tok - kStepTok * warp;  // lane 0's view
+    auto issue_next = [&]() {
+        uint8_t *dst = ring + (size_t)issue_slot * kBlk;
+        uint64_t *bar = &wbar[issue_slot];
+        const int n = min(kStepTok, issue_left);
+        if (!WINDOW) {
+            const bool full = n == kStepTok;
+            const uint32_t bc = full ? (uint32_t)(kStepTok * RB) : round16((uint32_t)(n * RB));
+            const uint32_t bs = full ? (uint32_t)(kStepTok * NG * 8) : round16((uint32_t)(n * NG * 8));
+            mbar_arrive_expect_tx(bar, 2 * (bc + bs));
+            bulk_copy_g2s(dst, src_kc, bc, bar);
+            bulk_copy_g2s(dst + kOffV, src_vc, bc, bar);
+            bulk_copy_g2s(dst + kOffKs, src_ks, bs, bar);
+            bulk_copy_g2s(dst + kOffVs, src_vs, bs, bar);
+            src_kc += (int64_t)kAdvTok * RB;
+            src_vc += (int64_t)kAdvTok * RB;
+            src_ks += (int64_t)kAdvTok * NG * 2;
+            src_vs += (int64_t)kAdvTok * NG * 2;
+            issue_left -= kAdvTok;
+        } else {
+            const int kv = issue_blk & 1;
+            const uint16_t *base = kv ? win_v : win_k;
+            const int first = min(n, V.cap_window - win_phys);
+            mbar_arrive_expect_tx(bar, (uint32_t)(n * D * 2));
+            bulk_copy_g2s(dst, base + (int64_t)win_phys * D, (uint32_t)(first * D * 2), bar);
+            if (n > first) bulk_copy_g2s(dst + first * D * 2, base, (uint32_t)((n - first) * D * 2), bar);
+            if (kv == 1) {
+                win_phys = (win_phys + kAdvTok) % V.cap_window;
+                issue_left -= kAdvTok;
+            }
+        }
+        ++issue_blk;
+        if (++issue_slot == S) issue_slot = 0;
+    };
+
+    // ---- prologue: barriers, first copies (before anything else waits), q
+    const int n_pro = min(S, n_blocks);
+    if (lane == 0) {
+        for (int s = 0; s < S; ++s) mbar_init(&wbar[s], 1);
+        fence_mbar_init();
+        for (int b = 0; b < n_pro; ++b) issue_next();
+    }
     for (int i = tid; i < kHeadsPerCta * D / 8; i += kAttnThreads) {
-        const int j = i / (D / 8), d8 = i % (D / 8);
+        const int j = i / (D / 8), d8 = i - j * (D / 8);
         uint4 val = make_uint4(0, 0, 0, 0);
         if (j < nh) val = reinterpret_cast<const uint4 *>(p.q + ((int64_t)V.view_index * p.n_q_heads + h0 + j) * D)[d8];
         reinterpret_cast<uint4 *>(q_s)[i] = val;
     }
-    if (lane == 0) {
-        for (int s = 0; s < kMaxStages; ++s) mbar_init(&bars[warp * kMaxStages + s], 1);
-        fence_mbar_init();
-    }
-    __syncthreads();
-    if (tid < 8 * NG) {
-        const int j = tid / NG, g = tid % NG;
-        float acc = 0.f;
-        for (int d = 0; d < 64; ++d) acc += __uint_as_float((uint32_t)q_s[j * D + 64 * g + d] << 16);
-        qsum_s[j * NG + g] = acc;
-    }
     __syncthreads();
 
     WarpState<NG> st;
-#pragma unroll
-    for (int g = 0; g < NG; ++g) {
-#pragma unroll
-        for (int t = 0; t < 4; ++t)
-#pragma unroll
-            for (int e = 0; e < 4; ++e) st.o[g][t][e] = 0.f;
-        st.mt[g][0] = st.mt[g][1] = 0.f;
-        st.qsum[g][0] = qsum_s[(2 * tig) * NG + g];
-        st.qsum[g][1] = qsum_s[(2 * tig + 1) * NG + g];
-    }
-    st.m[0] = st.m[1] = -INFINITY;
-    st.l[0] = st.l[1] = 0.f;
-
-    // q B-operand fragments: column n = gid, k-slots from the unpack map
     {
+        // q as B operand (column n = gid), k-slots from the unpack map; the
+        // per-group sums of q come from the same registers: each lane adds its
+        // 16 elements, lanes of one gid combine, then lanes fetch the sums of
+        // heads 2tig, 2tig+1.
         const uint16_t *qr = q_s + gid * D;
-        auto qpair = [&](int d0, int d1) -> uint32_t {
-            return (uint32_t)qr[d0] | ((uint32_t)qr[d1] << 16);
-        };
 #pragma unroll
-        for (int g = 0; g < NG; ++g)
+        for (int g = 0; g < NG; ++g) {
+            float part = 0.f;
 #pragma unroll
             for (int s = 0; s < 4; ++s)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int r = 2 * s + j;
-                    int e0, e1;
-                    if (is_window) { e0 = 2 * r; e1 = 2 * r + 1; }
-                    else if (B == 2) { e0 = qk_code<2>(r, 0); e1 = qk_code<2>(r, 1); }
-                    else if (B == 3) { e0 = qk_code<3>(r, 0); e1 = qk_code<3>(r, 1); }
-                    else if (B == 4) { e0 = qk_code<4>(r, 0); e1 = qk_code<4>(r, 1); }
-                    else { e0 = qk_code<8>(r, 0); e1 = qk_code<8>(r, 1); }
-                    st.bq[g][s][j] = qpair(64 * g + 16 * tig + e0, 64 * g + 16 * tig + e1);
+                    const int e0 = WINDOW ? 2 * r : qk_code<B>(r, 0);
+                    const int e1 = WINDOW ? 2 * r + 1 : qk_code<B>(r, 1);
+                    const uint32_t w = (uint32_t)qr[64 * g + 16 * tig + e0] | ((uint32_t)qr[64 * g + 16 * tig + e1] << 16);
+                    st.bq[g][s][j] = w;
+                    part += bf16lo_to_f32(w) + bf16hi_to_f32(w);
                 }
-    }
-
-    // ---- per-warp pipeline of bulk copies into this warp's ring
-    uint8_t *ring = rings + (size_t)warp * p.ring_bytes;
-    uint64_t *wbar = bars + warp * kMaxStages;
-    const uint32_t stage_bytes = is_window ? (uint32_t)(kTile * D * 2) : (uint32_t)(32 * RB + 2 * kTile * NG * 8);
-    const int S = min(kMaxStages, (int)(p.ring_bytes / stage_bytes));
-    const int n_my = (warp < n_tiles) ? (n_tiles - warp + kAttnWarps - 1) / kAttnWarps : 0;
-    const int bpt = is_window ? 2 : 1;
-    const int n_blocks = n_my * bpt;
-
-    auto issue = [&](int blk) {
-        const int slot = blk % S;
-        uint8_t *dst = ring + (size_t)slot * stage_bytes;
-        uint64_t *bar = &wbar[slot];
-        const int tile = warp + kAttnWarps * (blk / bpt);
-        const int n = min(kTile, n_tok - kTile * tile);
-        if (!is_window) {
-            const int64_t row = (int64_t)hk * V.cap_packed + tok0 + kTile * tile;
-            const uint32_t bc = round16((uint32_t)(n * RB));
-            const uint32_t bs = round16((uint32_t)(n * NG * 8));
-            mbar_arrive_expect_tx(bar, 2 * bc + 2 * bs);
-            bulk_copy_g2s(dst, V.codes[0] + row * RB, bc, bar);
-            bulk_copy_g2s(dst + 16 * RB, V.codes[1] + row * RB, bc, bar);
-            bulk_copy_g2s(dst + 32 * RB, V.scalemin[0] + row * NG * 2, bs, bar);
-            bulk_copy_g2s(dst + 32 * RB + kTile * NG * 8, V.scalemin[1] + row * NG * 2, bs, bar);
-        } else {
-            const int kv = blk & 1;
-            const uint16_t *base = V.window[kv] + (int64_t)hk * V.cap_window * D;
-            const int logical = (int)tok0 + kTile * tile;
-            const int phys = (V.window_head + logical) % V.cap_window;
-            const int first = min(n, V.cap_window - phys);
-            mbar_arrive_expect_tx(bar, (uint32_t)(n * D * 2));
-            bulk_copy_g2s(dst, base + (int64_t)phys * D, (uint32_t)(first * D * 2), bar);
-            if (n > first) bulk_copy_g2s(dst + first * D * 2, base, (uint32_t)((n - first) * D * 2), bar);
+            part += __shfl_xor_sync(0xFFFFFFFFu, part, 1);
+            part += __shfl_xor_sync(0xFFFFFFFFu, part, 2);
+            st.qsum[g][0] = __shfl_sync(0xFFFFFFFFu, part, 4 * (2 * tig));
+            st.qsum[g][1] = __shfl_sync(0xFFFFFFFFu, part, 4 * (2 * tig + 1));
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) st.o[g][t][e] = 0.f;
+            st.mt[g][0] = st.mt[g][1] = 0.f;
         }
-    };
-
-    bool failed = false;
-    int issued = 0;
-    if (lane == 0) {
-        for (; issued < min(S, n_blocks); ++issued) issue(issued);
+        st.m[0] = st.m[1] = -INFINITY;
+        st.l[0] = st.l[1] = 0.f;
     }
-    issued = min(S, n_blocks);
-    __syncwarp();
 
-    // warp-uniform: a lane that gives up makes the whole warp give up
-    auto wait_block = [&](int blk) -> bool {
-        const bool ok = mbar_wait_bounded(&wbar[blk % S], (uint32_t)((blk / S) & 1), p.timeout_ns);
-        return __all_sync(0xFFFFFFFFu, ok);
+    // consumer position: the current block is in slot `slot`, phase `phase`
+    int slot = 0;
+    uint32_t phase = 0;
+    const uint8_t *stage = ring;
+    int consumed = 0;
+    auto wait_cur = [&]() -> bool {
+        // warp-uniform result: one lane giving up makes the warp give up
+        if (__all_sync(0xFFFFFFFFu, mbar_try_wait(&wbar[slot], phase))) return true;
+        return __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&wbar[slot], phase, p.timeout_ns));
     };
-    auto release_block = [&](int blk) {
+    auto release_cur = [&]() {
         __syncwarp();
-        if (blk + S < n_blocks) {
-            if (lane == 0) {
-                fence_proxy_async_shared();
-                issue(blk + S);
-            }
-            issued = blk + S + 1;
+        if (lane == 0 && consumed + S < n_blocks) {
+            fence_proxy_async_shared();
+            issue_next();
+        }
+        ++consumed;
+        if (++slot == S) {
+            slot = 0;
+            phase ^= 1u;
+            stage = ring;
+        } else {
+            stage += kBlk;
         }
     };
 
-    int blk = 0;
-    for (int i = 0; i < n_my && !failed; ++i) {
-        const int tile = warp + kAttnWarps * i;
-        const int n_valid = min(kTile, n_tok - kTile * tile);
-        if (!is_window) {
-            if (!wait_block(blk)) { failed = true; break; }
-            const uint8_t *stage = ring + (size_t)(blk % S) * stage_bytes;
-            switch (B) {
-                case 2: packed_tile<2, NG>(st, stage, n_valid, p.scale_log2, gid, tig); break;
-                case 3: packed_tile<3, NG>(st, stage, n_valid, p.scale_log2, gid, tig); break;
-                case 4: packed_tile<4, NG>(st, stage, n_valid, p.scale_log2, gid, tig); break;
-                default: packed_tile<8, NG>(st, stage, n_valid, p.scale_log2, gid, tig); break;
+    // ---- main loop
+    bool failed = false;
+    int left = n_tok - kStepTok * warp;
+    for (int i = 0; i < n_my; ++i, left -= kAdvTok) {
+        if (!wait_cur()) { failed = true; break; }
+        if constexpr (!WINDOW) {
+            if (left >= kStepTok) {
+                // two full 16-token tiles, one softmax update over 32 tokens
+                float lg[4][2];
+                packed_qk2<B, NG>(st, stage, p.scale_log2, gid, tig, lg);
+                softmax_step_n<NG, 4>(st, lg);
+                packed_pv<B, NG, true>(st, stage + kOffV, stage + kOffVs, 2 * kTile, 0, lg[0], lg[1], gid, tig);
+                packed_pv<B, NG, true>(st, stage + kOffV + kTile * RB, stage + kOffVs + kTile * NG * 8, 2 * kTile, 0,
+                                       lg[2], lg[3], gid, tig);
+            } else {
+                // the chunk's ragged end: one or two partial tiles
+                float lg[4][2];
+                packed_qk1<B, NG>(st, stage, stage + kOffKs, min(left, kTile), p.scale_log2, gid, tig, lg[0], lg[1]);
+                if (left > kTile)
+                    packed_qk1<B, NG>(st, stage + kTile * RB, stage + kOffKs + kTile * NG * 8, left - kTile,
+                                      p.scale_log2, gid, tig, lg[2], lg[3]);
+                else
+                    lg[2][0] = lg[2][1] = lg[3][0] = lg[3][1] = -INFINITY;
+                softmax_step_n<NG, 4>(st, lg);
+                packed_pv<B, NG, false>(st, stage + kOffV, stage + kOffVs, 2 * kTile, min(left, kTile), lg[0], lg[1],
+                                        gid, tig);
+                if (left > kTile)
+                    packed_pv<B, NG, false>(st, stage + kOffV + kTile * RB, stage + kOffVs + kTile * NG * 8, 2 * kTile,
+                                            left - kTile, lg[2], lg[3], gid, tig);
             }
-            release_block(blk);
-            ++blk;
+            release_cur();
         } else {
+            const int n_valid = min(kTile, left);
             float lg[2][2];
-            if (!wait_block(blk)) { failed = true; break; }
-            window_qk<NG>(st, ring + (size_t)(blk % S) * stage_bytes, n_valid, p.scale_log2, gid, tig, lg);
-            release_block(blk);
-            ++blk;
-            softmax_step<NG>(st, lg);
-            if (!wait_block(blk)) { failed = true; break; }
-            window_pv<NG>(st, ring + (size_t)(blk % S) * stage_bytes, n_valid, lg, gid, tig);
-            release_block(blk);
-            ++blk;
+            if (n_valid == kTile) window_qk<NG, true>(st, stage, n_valid, p.scale_log2, gid, tig, lg);
+            else window_qk<NG, false>(st, stage, n_valid, p.scale_log2, gid, tig, lg);
+            release_cur();
+            softmax_step_n<NG, 2>(st, lg);
+            if (!wait_cur()) { failed = true; break; }
+            if (n_valid == kTile) window_pv<NG, true>(st, stage, n_valid, lg, gid, tig);
+            else window_pv<NG, false>(st, stage, n_valid, lg, gid, tig);
+            release_cur();
         }
     }
-    failed = __any_sync(0xFFFFFFFFu, failed);
     if (failed) {
         // let every copy this warp issued land before the CTA can exit
-        for (int b = blk; b < issued; ++b) (void)wait_block(b);
+        const int issued = __shfl_sync(0xFFFFFFFFu, issue_blk, 0);
+        for (; consumed < issued; ++consumed) {
+            (void)__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&wbar[slot], phase, p.timeout_ns));
+            if (++slot == S) { slot = 0; phase ^= 1u; }
+        }
         if (lane == 0) atomicExch(p.status, 1u);
     }
 
@@ -645,18 +761,18 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const __grid_
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
             const int d0 = 64 * g + 8 * gid + 2 * t;
-            wo[(2 * tig) * D + d0] = st.o[g][t][0] + st.mt[g][0];
-            wo[(2 * tig + 1) * D + d0] = st.o[g][t][1] + st.mt[g][1];
-            wo[(2 * tig) * D + d0 + 1] = st.o[g][t][2] + st.mt[g][0];
-            wo[(2 * tig + 1) * D + d0 + 1] = st.o[g][t][3] + st.mt[g][1];
+            *reinterpret_cast<float2 *>(&wo[(2 * tig) * D + d0]) =
+                make_float2(st.o[g][t][0] + st.mt[g][0], st.o[g][t][2] + st.mt[g][0]);
+            *reinterpret_cast<float2 *>(&wo[(2 * tig + 1) * D + d0]) =
+                make_float2(st.o[g][t][1] + st.mt[g][1], st.o[g][t][3] + st.mt[g][1]);
         }
     __syncthreads();
 
     // ---- merge the 4 warps (fixed order)
     const bool single = V.n_chunks == 1;
     const int units_per_view = p.n_kv_heads * p.head_blocks;
-    const int64_t slot = ((int64_t)(V.chunk_begin + c) * p.n_kv_heads + hk) * p.head_blocks + z;
-    float *part = p.partials + slot * (kHeadsPerCta * (D + 2));
+    const int64_t pslot = ((int64_t)(V.chunk_begin + c) * p.n_kv_heads + hk) * p.head_blocks + z;
+    float *part = p.partials + pslot * (kHeadsPerCta * (D + 2));
     for (int idx = tid; idx < nh * D; idx += kAttnThreads) {
         const int j = idx / D, d = idx - j * D;
         float M = -INFINITY;
@@ -668,7 +784,7 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const __grid_
         for (int w = 0; w < kAttnWarps; ++w) {
             const float *wp = reinterpret_cast<const float *>(rings + (size_t)w * p.ring_bytes);
             const float mw = wp[j];
-            const float e = (mw == -INFINITY) ? 0.f : exp2f(mw - M);
+            const float e = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
             L = fmaf(e, wp[8 + j], L);
             O = fmaf(e, wp[16 + j * D + d], O);
         }
@@ -698,20 +814,78 @@ __global__ void __launch_bounds__(kAttnThreads) decode_attn_kernel(const __grid_
     const int64_t slot0 = ((int64_t)V.chunk_begin * p.n_kv_heads + hk) * p.head_blocks + z;
     const int64_t slot_stride = (int64_t)p.n_kv_heads * p.head_blocks * (kHeadsPerCta * (D + 2));
     const float *part0 = p.partials + slot0 * (kHeadsPerCta * (D + 2));
+    const int n = V.n_chunks;  // <= kMaxChunksPerUnit (host-enforced)
+    // (1) every chunk's (m, l) per head, gathered in one parallel pass
+    float *sm_w = reinterpret_cast<float *>(rings);           // [n][8]: m, then weight
+    float *sm_l = sm_w + kMaxChunksPerUnit * kHeadsPerCta;    // [n][8]: l
+    float *sm_L = sm_l + kMaxChunksPerUnit * kHeadsPerCta;    // [8]: total
+    for (int i = tid; i < n * nh; i += kAttnThreads) {
+        const int cc = i / nh, j = i - cc * nh;
+        const float *pc = part0 + cc * slot_stride + j * (D + 2);
+        sm_w[cc * kHeadsPerCta + j] = __ldcg(pc + D);
+        sm_l[cc * kHeadsPerCta + j] = __ldcg(pc + D + 1);
+    }
+    __syncthreads();
+    // (2) per head: max, weights 2^(m_c - M), total L (warp w owns heads w, w+4)
+    for (int j = warp; j < nh; j += kAttnWarps) {
+        float M = -INFINITY;
+        for (int cc = lane; cc < n; cc += 32) M = fmaxf(M, sm_w[cc * kHeadsPerCta + j]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+        float L = 0.f;
+        for (int cc = lane; cc < n; cc += 32) {
+            const float w = fast_exp2(sm_w[cc * kHeadsPerCta + j] - M);
+            sm_w[cc * kHeadsPerCta + j] = w;
+            L = fmaf(w, sm_l[cc * kHeadsPerCta + j], L);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o);
+        if (lane == 0) sm_L[j] = L;
+    }
+    __syncthreads();
+    // (3) outputs: weighted sum over chunks in chunk order, loads batched 8 deep
     for (int idx = tid; idx < nh * D; idx += kAttnThreads) {
         const int j = idx / D, d = idx - j * D;
-        float M = -INFINITY;
-        for (int cc = 0; cc < V.n_chunks; ++cc) M = fmaxf(M, __ldcg(part0 + cc * slot_stride + j * (D + 2) + D));
-        float L = 0.f, O = 0.f;
-        for (int cc = 0; cc < V.n_chunks; ++cc) {
-            const float *pc = part0 + cc * slot_stride + j * (D + 2);
-            const float e = exp2f(__ldcg(pc + D) - M);
-            L = fmaf(e, __ldcg(pc + D + 1), L);
-            O = fmaf(e, __ldcg(pc + d), O);
+        const float *pj = part0 + j * (D + 2) + d;
+        float O = 0.f;
+        int cc = 0;
+        for (; cc + 8 <= n; cc += 8) {
+            float v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) v[u] = __ldcg(pj + (cc + u) * slot_stride);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) O = fmaf(sm_w[(cc + u) * kHeadsPerCta + j], v[u], O);
         }
-        p.out[((int64_t)V.view_index * p.n_q_heads + h0 + j) * D + d] = O / L;
+        for (; cc < n; ++cc) O = fmaf(sm_w[cc * kHeadsPerCta + j], __ldcg(pj + cc * slot_stride), O);
+        p.out[((int64_t)V.view_index * p.n_q_heads + h0 + j) * D + d] = O / sm_L[j];
     }
     if (tid == 0) atomicExch(counter, 0u);
+}
+
+template <int NG>
+__global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
+    decode_attn_kernel(const __grid_constant__ AttnParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    // ---- which item: view by binary search over chunk ranges
+    const int bx = blockIdx.x;
+    int lo = 0, hi = p.n_views - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.views[mid].chunk_begin <= bx) lo = mid; else hi = mid - 1;
+    }
+    const AttnView &V = p.views[lo];
+    const int c = bx - V.chunk_begin;
+    const int hk = blockIdx.y, z = blockIdx.z;
+    if (c >= V.n_chunks_packed) {
+        attn_item<NG, 4, true>(p, V, lo, c, hk, z, smem);
+    } else {
+        switch (V.bits) {
+            case 2: attn_item<NG, 2, false>(p, V, lo, c, hk, z, smem); break;
+            case 3: attn_item<NG, 3, false>(p, V, lo, c, hk, z, smem); break;
+            case 4: attn_item<NG, 4, false>(p, V, lo, c, hk, z, smem); break;
+            default: attn_item<NG, 8, false>(p, V, lo, c, hk, z, smem); break;
+        }
+    }
 }
 
 }  // namespace kvq

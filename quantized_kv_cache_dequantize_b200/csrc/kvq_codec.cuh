@@ -58,23 +58,36 @@ __device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], uin
         // Fast path: y = (x - mn) * RN(1/s) lies within 3*2^(B-24) of the
         // correctly rounded quotient RN((x - mn)/s) (quotients are <= 2^B).
         // Unless y is within `lim` of a half-integer, both round to the same
-        // integer; near-ties, and any non-finite y (tiny s), take the IEEE
-        // division.  The result is exactly round_half_even(RN((x-mn)/s)).
+        // integer.  If any element of this half is that close, or y is not
+        // finite (tiny s), the whole half is redone with the IEEE division,
+        // so every code is exactly round_half_even(RN((x - mn)/s)).  No clamp
+        // is needed: 0 <= y < 2^B - 1/2 on the fast path.
         const float r = __frcp_rn(s);
         const float lim = 0.5f - __uint_as_float((uint32_t)(127 + B - 21) << 23);
+        bool near_tie = false;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const float xf = (i & 1) ? bf16hi_to_f32(x[i >> 1]) : bf16lo_to_f32(x[i >> 1]);
-            const float a = __fsub_rn(xf, mn);
-            const float y = __fmul_rn(a, r);
+            const float y = __fmul_rn(__fsub_rn(xf, mn), r);
             const float t = __fadd_rn(y, kRoundMagic);
             const float d = __fsub_rn(y, __fsub_rn(t, kRoundMagic));
-            uint32_t c = __float_as_uint(t) - kRoundMagicBits;
-            if (!(fabsf(d) <= lim)) c = __float2uint_rn(__fdiv_rn(a, s));
-            c = min(c, qmax);
+            const uint32_t c = __float_as_uint(t) - kRoundMagicBits;
+            near_tie |= !(fabsf(d) <= lim);
             const int bit = i * B;
-            packed[bit >> 5] |= c << (bit & 31);
-            if ((bit & 31) + B > 32) packed[(bit >> 5) + 1] |= c >> (32 - (bit & 31));
+            packed[bit >> 5] += c << (bit & 31);
+            if ((bit & 31) + B > 32) packed[(bit >> 5) + 1] += c >> (32 - (bit & 31));
+        }
+        if (near_tie) {
+#pragma unroll
+            for (int w = 0; w < B; ++w) packed[w] = 0u;
+#pragma unroll
+            for (int i = 0; i < 32; ++i) {
+                const float xf = (i & 1) ? bf16hi_to_f32(x[i >> 1]) : bf16lo_to_f32(x[i >> 1]);
+                const uint32_t c = min(__float2uint_rn(__fdiv_rn(__fsub_rn(xf, mn), s)), qmax);
+                const int bit = i * B;
+                packed[bit >> 5] += c << (bit & 31);
+                if ((bit & 31) + B > 32) packed[(bit >> 5) + 1] += c >> (32 - (bit & 31));
+            }
         }
     }
     s_out = s;
@@ -114,55 +127,68 @@ struct CodecArgs {
     int64_t head_cap;        // rows per head in codes/scalemin
 };
 
-// Grid: (blocks per head, n_heads). Each lane pair owns one group; a warp
-// owns 16 consecutive groups of one head per iteration.
+// Grid: (blocks per head, n_heads).  Each lane pair owns one group per
+// round; a warp owns 16 consecutive groups of one head per round and runs
+// kRounds rounds per iteration with all loads issued before any compute.
+constexpr int kRounds = 1;       // quantize: rounds per iteration (issue-bound: keep registers low)
+constexpr int kDeqRounds = 4;    // dequantize: rounds per iteration (latency-bound: many loads in flight)
+
 template <int B, int NG>
 __global__ void __launch_bounds__(256) quantize_kernel(CodecArgs a) {
     constexpr int RB = 8 * B * NG;  // row bytes
     const int h = blockIdx.y;
     const int64_t n_groups = a.n_tokens * NG;
     const int lane = threadIdx.x & 31;
+    const int half = lane & 1;
     const int64_t warp_global = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t warp_stride = (int64_t)gridDim.x * (blockDim.x >> 5);
     const uint16_t *xh = a.x + (int64_t)h * a.x_head_stride;
     uint8_t *ch = a.codes + (int64_t)h * a.head_cap * RB;
     float *sh = a.scalemin + (int64_t)h * a.head_cap * NG * 2;
 
-    for (int64_t base = warp_global * 16; base < n_groups; base += warp_stride * 16) {
-        const int64_t grp = base + (lane >> 1);
-        const int half = lane & 1;
-        const bool active = grp < n_groups;
-        const int64_t t = grp / NG;
-        const int g = (int)(grp - t * NG);
-        uint32_t x[16];
-        if (active) {
-            const uint4 *src = reinterpret_cast<const uint4 *>(xh + t * a.x_tok_stride + g * kGroup + half * 32);
+    for (int64_t base = warp_global * 16 * kRounds; base < n_groups; base += warp_stride * 16 * kRounds) {
+        uint32_t x[kRounds][16];
+        int64_t t[kRounds];
+        int g[kRounds];
+        bool active[kRounds];
 #pragma unroll
-            for (int v = 0; v < 4; ++v) {
-                const uint4 q = __ldcs(src + v);
-                x[4 * v + 0] = q.x; x[4 * v + 1] = q.y; x[4 * v + 2] = q.z; x[4 * v + 3] = q.w;
-            }
-        } else {
+        for (int u = 0; u < kRounds; ++u) {
+            const int64_t grp = base + 16 * u + (lane >> 1);
+            active[u] = grp < n_groups;
+            t[u] = grp / NG;
+            g[u] = (int)(grp - t[u] * NG);
+            if (active[u]) {
+                const uint4 *src = reinterpret_cast<const uint4 *>(xh + t[u] * a.x_tok_stride + g[u] * kGroup + half * 32);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) x[i] = 0u;
-        }
-        uint32_t packed[B];
-        float s, mn;
-        quantize_half_group<B>(x, packed, s, mn);
-        if (active) {
-            uint8_t *dst = ch + t * RB + g * 8 * B + half * 4 * B;
-            if constexpr (B == 4) {
-                *reinterpret_cast<uint4 *>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-            } else if constexpr (B == 8) {
-                reinterpret_cast<uint4 *>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                reinterpret_cast<uint4 *>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-            } else if constexpr (B == 2) {
-                *reinterpret_cast<uint2 *>(dst) = make_uint2(packed[0], packed[1]);
+                for (int v = 0; v < 4; ++v) {
+                    const uint4 q = __ldcs(src + v);
+                    x[u][4 * v + 0] = q.x; x[u][4 * v + 1] = q.y; x[u][4 * v + 2] = q.z; x[u][4 * v + 3] = q.w;
+                }
             } else {
 #pragma unroll
-                for (int w = 0; w < B; ++w) reinterpret_cast<uint32_t *>(dst)[w] = packed[w];
+                for (int i = 0; i < 16; ++i) x[u][i] = 0u;
             }
-            if (half == 0) *reinterpret_cast<float2 *>(sh + (t * NG + g) * 2) = make_float2(s, mn);
+        }
+#pragma unroll
+        for (int u = 0; u < kRounds; ++u) {
+            uint32_t packed[B];
+            float s, mn;
+            quantize_half_group<B>(x[u], packed, s, mn);
+            if (active[u]) {
+                uint8_t *dst = ch + t[u] * RB + g[u] * 8 * B + half * 4 * B;
+                if constexpr (B == 4) {
+                    *reinterpret_cast<uint4 *>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                } else if constexpr (B == 8) {
+                    reinterpret_cast<uint4 *>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+                    reinterpret_cast<uint4 *>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+                } else if constexpr (B == 2) {
+                    *reinterpret_cast<uint2 *>(dst) = make_uint2(packed[0], packed[1]);
+                } else {
+#pragma unroll
+                    for (int w = 0; w < B; ++w) reinterpret_cast<uint32_t *>(dst)[w] = packed[w];
+                }
+                if (half == 0) *reinterpret_cast<float2 *>(sh + (t[u] * NG + g[u]) * 2) = make_float2(s, mn);
+            }
         }
     }
 }
@@ -173,41 +199,53 @@ __global__ void __launch_bounds__(256) dequantize_kernel(CodecArgs a) {
     const int h = blockIdx.y;
     const int64_t n_groups = a.n_tokens * NG;
     const int lane = threadIdx.x & 31;
+    const int half = lane & 1;
     const int64_t warp_global = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t warp_stride = (int64_t)gridDim.x * (blockDim.x >> 5);
     uint16_t *yh = const_cast<uint16_t *>(a.x) + (int64_t)h * a.x_head_stride;
     const uint8_t *ch = a.codes + (int64_t)h * a.head_cap * RB;
     const float *sh = a.scalemin + (int64_t)h * a.head_cap * NG * 2;
+    constexpr int kR = kDeqRounds;
 
-    for (int64_t base = warp_global * 16; base < n_groups; base += warp_stride * 16) {
-        const int64_t grp = base + (lane >> 1);
-        const int half = lane & 1;
-        if (grp >= n_groups) continue;
-        const int64_t t = grp / NG;
-        const int g = (int)(grp - t * NG);
-        const uint8_t *src = ch + t * RB + g * 8 * B + half * 4 * B;
-        uint32_t packed[B];
-        if constexpr (B == 4) {
-            const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(src));
-            packed[0] = q.x; packed[1] = q.y; packed[2] = q.z; packed[3] = q.w;
-        } else if constexpr (B == 8) {
-            const uint4 q0 = __ldcs(reinterpret_cast<const uint4 *>(src));
-            const uint4 q1 = __ldcs(reinterpret_cast<const uint4 *>(src) + 1);
-            packed[0] = q0.x; packed[1] = q0.y; packed[2] = q0.z; packed[3] = q0.w;
-            packed[4] = q1.x; packed[5] = q1.y; packed[6] = q1.z; packed[7] = q1.w;
-        } else if constexpr (B == 2) {
-            const uint2 q = __ldcs(reinterpret_cast<const uint2 *>(src));
-            packed[0] = q.x; packed[1] = q.y;
-        } else {
+    for (int64_t base = warp_global * 16 * kR; base < n_groups; base += warp_stride * 16 * kR) {
+        uint32_t packed[kR][B];
+        float2 sm[kR];
+        int64_t t[kR];
+        int g[kR];
 #pragma unroll
-            for (int w = 0; w < B; ++w) packed[w] = __ldcs(reinterpret_cast<const uint32_t *>(src) + w);
+        for (int u = 0; u < kR; ++u) {
+            const int64_t grp = base + 16 * u + (lane >> 1);
+            t[u] = grp / NG;
+            g[u] = (int)(grp - t[u] * NG);
+            if (grp < n_groups) {
+                const uint8_t *src = ch + t[u] * RB + g[u] * 8 * B + half * 4 * B;
+                if constexpr (B == 4) {
+                    const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(src));
+                    packed[u][0] = q.x; packed[u][1] = q.y; packed[u][2] = q.z; packed[u][3] = q.w;
+                } else if constexpr (B == 8) {
+                    const uint4 q0 = __ldcs(reinterpret_cast<const uint4 *>(src));
+                    const uint4 q1 = __ldcs(reinterpret_cast<const uint4 *>(src) + 1);
+                    packed[u][0] = q0.x; packed[u][1] = q0.y; packed[u][2] = q0.z; packed[u][3] = q0.w;
+                    packed[u][4] = q1.x; packed[u][5] = q1.y; packed[u][6] = q1.z; packed[u][7] = q1.w;
+                } else if constexpr (B == 2) {
+                    const uint2 q = __ldcs(reinterpret_cast<const uint2 *>(src));
+                    packed[u][0] = q.x; packed[u][1] = q.y;
+                } else {
+#pragma unroll
+                    for (int w = 0; w < B; ++w) packed[u][w] = __ldcs(reinterpret_cast<const uint32_t *>(src) + w);
+                }
+                sm[u] = __ldcs(reinterpret_cast<const float2 *>(sh + (t[u] * NG + g[u]) * 2));
+            }
         }
-        const float2 sm = __ldcs(reinterpret_cast<const float2 *>(sh + (t * NG + g) * 2));
-        uint32_t y[16];
-        dequantize_half_group<B>(packed, sm.x, sm.y, y);
-        uint4 *dst = reinterpret_cast<uint4 *>(yh + t * a.x_tok_stride + g * kGroup + half * 32);
 #pragma unroll
-        for (int v = 0; v < 4; ++v) __stcs(dst + v, make_uint4(y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]));
+        for (int u = 0; u < kR; ++u) {
+            if (base + 16 * u + (lane >> 1) >= n_groups) continue;
+            uint32_t y[16];
+            dequantize_half_group<B>(packed[u], sm[u].x, sm[u].y, y);
+            uint4 *dst = reinterpret_cast<uint4 *>(yh + t[u] * a.x_tok_stride + g[u] * kGroup + half * 32);
+#pragma unroll
+            for (int v = 0; v < 4; ++v) __stcs(dst + v, make_uint4(y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]));
+        }
     }
 }
 
