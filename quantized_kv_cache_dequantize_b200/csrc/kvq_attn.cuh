@@ -109,23 +109,36 @@ __device__ __forceinline__ uint32_t bf16_codes(uint32_t w, uint32_t mask_at_o) {
     return fma_bf16x2(lop3_and_or(w, mask_at_o, kMagic), kScale, kBias);
 }
 
+// K codes are not normalised: register halves hold 128 + c*2^O as exact bf16
+// (one LOP3), and the B operand carries q*2^-O in the matching slot, so the
+// MMA yields sum q*c + 128 * sum q*2^-O; the second term is a per-(group,
+// head) constant removed in the epilogue.  qk_off<B>(r) is O of register r.
+template <int B>
+__host__ __device__ constexpr int qk_off(int r) {
+    return B == 2 ? (r % 3) * 2 : B == 3 ? (r & 1) * 3 : 0;
+}
+
+__device__ __forceinline__ uint32_t bf16_raw(uint32_t w, uint32_t mask_at_o) {
+    return lop3_and_or(w, mask_at_o, 0x43004300u);  // 128 + (bits under mask), both halves
+}
+
 template <int B>
 __device__ __forceinline__ void qk_unpack(const uint8_t *seg, uint32_t (&r)[8]);
 
 template <>
 __device__ __forceinline__ void qk_unpack<2>(const uint8_t *seg, uint32_t (&r)[8]) {
     // 16 codes x 2 bits = one word; code j at bit 2j.  Low half: codes 0..7,
-    // high half: codes 8..15; register r = (c_r, c_{r+8}).
+    // high half: codes 8..15; register r = (c_r, c_{r+8}) at offset qk_off<2>(r).
     const uint32_t w = *reinterpret_cast<const uint32_t *>(seg);
     const uint32_t w6 = w >> 6, w12 = w >> 12;
-    r[0] = bf16_codes<0>(w, 0x00030003u);
-    r[1] = bf16_codes<2>(w, 0x000C000Cu);
-    r[2] = bf16_codes<4>(w, 0x00300030u);
-    r[3] = bf16_codes<0>(w6, 0x00030003u);
-    r[4] = bf16_codes<2>(w6, 0x000C000Cu);
-    r[5] = bf16_codes<4>(w6, 0x00300030u);
-    r[6] = bf16_codes<0>(w12, 0x00030003u);
-    r[7] = bf16_codes<2>(w12, 0x000C000Cu);
+    r[0] = bf16_raw(w, 0x00030003u);
+    r[1] = bf16_raw(w, 0x000C000Cu);
+    r[2] = bf16_raw(w, 0x00300030u);
+    r[3] = bf16_raw(w6, 0x00030003u);
+    r[4] = bf16_raw(w6, 0x000C000Cu);
+    r[5] = bf16_raw(w6, 0x00300030u);
+    r[6] = bf16_raw(w12, 0x00030003u);
+    r[7] = bf16_raw(w12, 0x000C000Cu);
 }
 
 template <>
@@ -145,8 +158,8 @@ __device__ __forceinline__ void qk_unpack<3>(const uint8_t *seg, uint32_t (&r)[8
         const uint32_t fa = (a == 0) ? lo : __funnelshift_r(lo, hi, a);
         const uint32_t fb = (b < 32) ? __funnelshift_r(lo, hi, b) : (hi >> (b - 32));
         const uint32_t pw = prmt(fa, fb, 0x5410u);
-        r[2 * k] = bf16_codes<0>(pw, 0x00070007u);
-        r[2 * k + 1] = bf16_codes<3>(pw, 0x00380038u);
+        r[2 * k] = bf16_raw(pw, 0x00070007u);
+        r[2 * k + 1] = bf16_raw(pw, 0x00380038u);
     }
 }
 
@@ -157,8 +170,8 @@ __device__ __forceinline__ void qk_unpack<4>(const uint8_t *seg, uint32_t (&r)[8
     const uint2 w = *reinterpret_cast<const uint2 *>(seg);
 #pragma unroll
     for (int k = 0; k < 4; ++k) {
-        r[k] = bf16_codes<0>(w.x >> (4 * k), 0x000F000Fu);
-        r[4 + k] = bf16_codes<0>(w.y >> (4 * k), 0x000F000Fu);
+        r[k] = bf16_raw(w.x >> (4 * k), 0x000F000Fu);
+        r[4 + k] = bf16_raw(w.y >> (4 * k), 0x000F000Fu);
     }
 }
 
@@ -170,7 +183,7 @@ __device__ __forceinline__ float byte_to_f32(uint32_t w, uint32_t sel) {
 
 template <>
 __device__ __forceinline__ void qk_unpack<8>(const uint8_t *seg, uint32_t (&r)[8]) {
-    // 16 bytes; register r = (c_{2r}, c_{2r+1}).
+    // 16 bytes; register r = (c_{2r}, c_{2r+1}) as exact bf16 c (no 128 offset).
     const uint4 w = *reinterpret_cast<const uint4 *>(seg);
     const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -269,6 +282,7 @@ struct WarpState {
     float l[2];             // running sum (partial over this lane's rows)
     uint32_t bq[NG][4][2];  // q as B operand: group, k-step, (b0b1, b2b3)
     float qsum[NG][2];      // sum of q over each group, heads 2tig, 2tig+1
+    float qoff[NG][2];      // -128 * sum of q*2^-O over each group (0 where codes carry no offset)
 };
 
 // Online-softmax step over R row-sets (R = 2: one 16-token tile, rows gid and
@@ -345,7 +359,8 @@ __device__ __forceinline__ void packed_qk1(const WarpState<NG> &st, const uint8_
         uint32_t a0[8], a1[8];
         qk_unpack<B>(row0 + g * 8 * B, a0);
         qk_unpack<B>(row1 + g * 8 * B, a1);
-        float acc[4] = {0.f, 0.f, 0.f, 0.f};
+        // the accumulator starts at the code offset's contribution, -128 sum q*2^-O
+        float acc[4] = {st.qoff[g][0], st.qoff[g][1], st.qoff[g][0], st.qoff[g][1]};
 #pragma unroll
         for (int s = 0; s < 4; ++s)
             mma_bf16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0], st.bq[g][s][1]);
@@ -379,7 +394,7 @@ __device__ __forceinline__ void packed_qk2(const WarpState<NG> &st, const uint8_
             uint32_t a0[8], a1[8];
             qk_unpack<B>(row0 + tt * kTile * RB + g * 8 * B, a0);
             qk_unpack<B>(row0 + tt * kTile * RB + 8 * RB + g * 8 * B, a1);
-            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            float acc[4] = {st.qoff[g][0], st.qoff[g][1], st.qoff[g][0], st.qoff[g][1]};
 #pragma unroll
             for (int s = 0; s < 4; ++s)
                 mma_bf16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0],
@@ -624,7 +639,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         const uint16_t *qr = q_s + gid * D;
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
-            float part = 0.f;
+            float part = 0.f, part_off = 0.f;
 #pragma unroll
             for (int s = 0; s < 4; ++s)
 #pragma unroll
@@ -632,14 +647,23 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
                     const int r = 2 * s + j;
                     const int e0 = WINDOW ? 2 * r : qk_code<B>(r, 0);
                     const int e1 = WINDOW ? 2 * r + 1 : qk_code<B>(r, 1);
-                    const uint32_t w = (uint32_t)qr[64 * g + 16 * tig + e0] | ((uint32_t)qr[64 * g + 16 * tig + e1] << 16);
-                    st.bq[g][s][j] = w;
-                    part += bf16lo_to_f32(w) + bf16hi_to_f32(w);
+                    const float q0 = __uint_as_float((uint32_t)qr[64 * g + 16 * tig + e0] << 16);
+                    const float q1 = __uint_as_float((uint32_t)qr[64 * g + 16 * tig + e1] << 16);
+                    const float sc = (WINDOW || B == 8) ? 1.f : __uint_as_float((uint32_t)(127 - qk_off<B>(r)) << 23);
+                    // q * 2^-O is exact in bf16 (exponent change only)
+                    st.bq[g][s][j] = pack_bf16x2(q0 * sc, q1 * sc);
+                    part += q0 + q1;
+                    part_off += q0 * sc + q1 * sc;
                 }
             part += __shfl_xor_sync(0xFFFFFFFFu, part, 1);
             part += __shfl_xor_sync(0xFFFFFFFFu, part, 2);
+            part_off += __shfl_xor_sync(0xFFFFFFFFu, part_off, 1);
+            part_off += __shfl_xor_sync(0xFFFFFFFFu, part_off, 2);
             st.qsum[g][0] = __shfl_sync(0xFFFFFFFFu, part, 4 * (2 * tig));
             st.qsum[g][1] = __shfl_sync(0xFFFFFFFFu, part, 4 * (2 * tig + 1));
+            const float off_scale = (WINDOW || B == 8) ? 0.f : -128.f;
+            st.qoff[g][0] = off_scale * __shfl_sync(0xFFFFFFFFu, part_off, 4 * (2 * tig));
+            st.qoff[g][1] = off_scale * __shfl_sync(0xFFFFFFFFu, part_off, 4 * (2 * tig + 1));
 #pragma unroll
             for (int t = 0; t < 4; ++t)
 #pragma unroll

@@ -54,17 +54,26 @@ __device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], uin
 #pragma unroll
     for (int w = 0; w < B; ++w) packed[w] = 0u;
 
-    if (s != 0.0f) {
+    if (s != 0.0f && !(s >= 0x1p-100f && s <= 0x1p100f)) {
+        // extreme scales (subnormal ranges): IEEE division for every element
+#pragma unroll
+        for (int i = 0; i < 32; ++i) {
+            const float xf = (i & 1) ? bf16hi_to_f32(x[i >> 1]) : bf16lo_to_f32(x[i >> 1]);
+            const uint32_t c = min(__float2uint_rn(__fdiv_rn(__fsub_rn(xf, mn), s)), qmax);
+            const int bit = i * B;
+            packed[bit >> 5] += c << (bit & 31);
+            if ((bit & 31) + B > 32) packed[(bit >> 5) + 1] += c >> (32 - (bit & 31));
+        }
+    } else if (s != 0.0f) {
         // Fast path: y = (x - mn) * RN(1/s) lies within 3*2^(B-24) of the
-        // correctly rounded quotient RN((x - mn)/s) (quotients are <= 2^B).
-        // Unless y is within `lim` of a half-integer, both round to the same
-        // integer.  If any element of this half is that close, or y is not
-        // finite (tiny s), the whole half is redone with the IEEE division,
-        // so every code is exactly round_half_even(RN((x - mn)/s)).  No clamp
-        // is needed: 0 <= y < 2^B - 1/2 on the fast path.
+        // correctly rounded quotient RN((x - mn)/s) (quotients are <= 2^B), so
+        // unless y is within 2^(B-21) of a half-integer both round to the same
+        // integer (and 0 <= y < 2^B - 1/2: every code is in range).  Elements
+        // closer than that (bf16 grids make exact ties common) are redone
+        // exactly below, without a division.
         const float r = __frcp_rn(s);
         const float lim = 0.5f - __uint_as_float((uint32_t)(127 + B - 21) << 23);
-        bool near_tie = false;
+        uint32_t near = 0u;
 #pragma unroll
         for (int i = 0; i < 32; ++i) {
             const float xf = (i & 1) ? bf16hi_to_f32(x[i >> 1]) : bf16lo_to_f32(x[i >> 1]);
@@ -72,21 +81,44 @@ __device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], uin
             const float t = __fadd_rn(y, kRoundMagic);
             const float d = __fsub_rn(y, __fsub_rn(t, kRoundMagic));
             const uint32_t c = __float_as_uint(t) - kRoundMagicBits;
-            near_tie |= !(fabsf(d) <= lim);
+            near |= (fabsf(d) <= lim) ? 0u : (1u << i);
             const int bit = i * B;
             packed[bit >> 5] += c << (bit & 31);
             if ((bit & 31) + B > 32) packed[(bit >> 5) + 1] += c >> (32 - (bit & 31));
         }
-        if (near_tie) {
+        while (near) {
+            const int i = __ffs(near) - 1;
+            near &= near - 1u;
+            // element i, re-extracted with a compile-time select chain
+            uint32_t w = x[0];
 #pragma unroll
-            for (int w = 0; w < B; ++w) packed[w] = 0u;
+            for (int k = 1; k < 16; ++k) w = ((i >> 1) == k) ? x[k] : w;
+            const float xf = (i & 1) ? bf16hi_to_f32(w) : bf16lo_to_f32(w);
+            const float a = __fsub_rn(xf, mn);
+            const float y = __fmul_rn(a, r);
+            const float t = __fadd_rn(y, kRoundMagic);
+            const float ri = __fsub_rn(t, kRoundMagic);
+            const uint32_t c_fast = __float_as_uint(t) - kRoundMagicBits;
+            // h = the half-integer y is near; e = a - h*s is exact (|e| <
+            // s*2^(B-20) on a grid no finer than ulp(s)/4, i.e. <= B+6
+            // significant bits), so a/s = h + e/s exactly.  RN(a/s) == h iff
+            // |e| <= s*ulp(h)/2 (h has few significant bits, so a tie at that
+            // distance rounds to h); then the code is h rounded half to even,
+            // otherwise the integer on the side of h that e points to.
+            const float h = __fadd_rn(ri, (y >= ri) ? 0.5f : -0.5f);
+            const float e = __fmaf_rn(-h, s, a);
+            const float half_ulp = __uint_as_float((__float_as_uint(h) & 0x7F800000u) - (24u << 23));
+            const uint32_t n = __float_as_uint(__fadd_rn(__fsub_rn(h, 0.5f), kRoundMagic)) - kRoundMagicBits;
+            uint32_t c;
+            if (fabsf(e) <= __fmul_rn(s, half_ulp)) c = n + (n & 1u);
+            else c = (e > 0.0f) ? n + 1u : n;
+            // patch the packed field of element i (XOR: no carries across fields)
+            const uint32_t flip = c ^ c_fast;
+            const int bit = i * B;
 #pragma unroll
-            for (int i = 0; i < 32; ++i) {
-                const float xf = (i & 1) ? bf16hi_to_f32(x[i >> 1]) : bf16lo_to_f32(x[i >> 1]);
-                const uint32_t c = min(__float2uint_rn(__fdiv_rn(__fsub_rn(xf, mn), s)), qmax);
-                const int bit = i * B;
-                packed[bit >> 5] += c << (bit & 31);
-                if ((bit & 31) + B > 32) packed[(bit >> 5) + 1] += c >> (32 - (bit & 31));
+            for (int k = 0; k < B; ++k) {
+                if ((bit >> 5) == k) packed[k] ^= flip << (bit & 31);
+                if (B == 3 && (bit >> 5) + 1 == k && (bit & 31) + B > 32) packed[k] ^= flip >> (32 - (bit & 31));
             }
         }
     }
@@ -131,7 +163,7 @@ struct CodecArgs {
 // round; a warp owns 16 consecutive groups of one head per round and runs
 // kRounds rounds per iteration with all loads issued before any compute.
 constexpr int kRounds = 1;       // quantize: rounds per iteration (issue-bound: keep registers low)
-constexpr int kDeqRounds = 4;    // dequantize: rounds per iteration (latency-bound: many loads in flight)
+constexpr int kDeqRounds = 8;    // dequantize: rounds per iteration (latency-bound: many loads in flight)
 
 template <int B, int NG>
 __global__ void __launch_bounds__(256) quantize_kernel(CodecArgs a) {
