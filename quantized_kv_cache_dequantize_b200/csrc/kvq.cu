@@ -174,28 +174,29 @@ int64_t chunk_views(const kvq_view *views, int v0, int v1, int64_t units, int32_
     for (int i = v0; i < v1; ++i)
         total += (double)units * ((double)views[i].n_packed * packed_token_bytes(head_dim, views[i].bits) +
                                   (double)views[i].n_window * window_token_bytes(head_dim));
-    auto count = [&](double W, bool store) -> int64_t {
+    // items and largest item (bytes) for a target item size W
+    auto count = [&](double W, bool store, double *max_item) -> int64_t {
         int64_t items = 0;
+        double mx = 0;
+        const int forced = env_int("KVQ_CHUNK_TOKENS", 0);
         for (int i = v0; i < v1; ++i) {
             const kvq_view &v = views[i];
             ViewChunks c{16, 16, 0, 0};
+            const double bp = (double)packed_token_bytes(head_dim, v.bits), bw = (double)window_token_bytes(head_dim);
             if (v.n_packed > 0) {
-                const double b = (double)v.n_packed * packed_token_bytes(head_dim, v.bits);
-                int64_t n = std::max<int64_t>(1, (int64_t)std::llround(b / W));
+                int64_t n = std::max<int64_t>(1, (int64_t)std::llround(v.n_packed * bp / W));
                 int64_t ch = (v.n_packed + n - 1) / n;
                 ch = std::max<int64_t>(128, (ch + 127) / 128 * 128);  // whole 32-token steps for 4 warps
                 c.chunk_packed = (int32_t)ch;
                 c.n_packed = (int32_t)((v.n_packed + ch - 1) / ch);
             }
             if (v.n_window > 0) {
-                const double b = (double)v.n_window * window_token_bytes(head_dim);
-                int64_t n = std::max<int64_t>(1, (int64_t)std::llround(b / W));
+                int64_t n = std::max<int64_t>(1, (int64_t)std::llround(v.n_window * bw / W));
                 int64_t ch = (v.n_window + n - 1) / n;
                 ch = std::max<int64_t>(64, (ch + 63) / 64 * 64);  // whole 16-token steps for 4 warps
                 c.chunk_window = (int32_t)ch;
                 c.n_window = (int32_t)((v.n_window + ch - 1) / ch);
             }
-            const int forced = env_int("KVQ_CHUNK_TOKENS", 0);
             if (forced > 0) {
                 const int ch = std::max(32, forced / 32 * 32);
                 c.chunk_packed = c.chunk_window = ch;
@@ -212,28 +213,32 @@ int64_t chunk_views(const kvq_view *views, int v0, int v1, int64_t units, int32_
                     c.n_window = (int32_t)((v.n_window + c.chunk_window - 1) / c.chunk_window);
                 }
             }
+            if (c.n_packed) mx = std::max(mx, std::min<double>(c.chunk_packed, v.n_packed) * bp);
+            if (c.n_window) mx = std::max(mx, std::min<double>(c.chunk_window, v.n_window) * bw);
             items += c.n_packed + c.n_window;
             if (store) out[i] = c;
         }
-        return items;
+        if (max_item) *max_item = mx;
+        return items;  // chunks over the views; each is run once per unit
     };
-    const double kMinItem = 24.0 * 1024, kBigItem = 192.0 * 1024;
-    double W = total / (double)slots;
-    if (W >= kBigItem) {
-        W = kBigItem;  // many waves: the tail is small anyway
-    } else {
-        double chosen = std::max(total / (double)(slots * 8), kMinItem);
-        for (int waves = 1; waves <= 8; ++waves) {
-            const double Ww = total / (double)(slots * waves);
-            if (Ww < kMinItem) break;
-            if (count(Ww, false) * units <= slots * waves) {
-                chosen = Ww;
-                break;
-            }
+    // Pick the item size with the smallest predicted makespan: whole waves of
+    // resident CTAs, each wave as long as its largest item plus a fixed
+    // per-CTA cost (set-up, pipeline fill, merge), in byte-equivalents.
+    const double kMinItem = 16.0 * 1024, kBigItem = 256.0 * 1024, kCtaCost = 24.0 * 1024;
+    double best_W = std::max(kMinItem, std::min(kBigItem, total / (double)slots)), best_cost = 1e300;
+    const double fs[] = {0.6, 0.7, 0.8, 0.9, 1.0, 1.15, 1.3, 1.5, 1.75, 2.0, 2.5, 3.0, 4.0, 5.0, 6.0, 8.0, 12.0, 16.0, 24.0, 32.0};
+    for (double f : fs) {
+        const double W = std::max(kMinItem, std::min(kBigItem, total / ((double)slots * f)));
+        double mx = 0;
+        const int64_t items = count(W, false, &mx) * units;
+        const double waves = (double)((items + slots - 1) / slots);
+        const double cost = waves * (mx + kCtaCost);
+        if (cost < best_cost * 0.999) {
+            best_cost = cost;
+            best_W = W;
         }
-        W = chosen;
     }
-    return count(W, true);
+    return count(best_W, true, nullptr);
 }
 
 kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, int32_t n_kv_heads,

@@ -578,7 +578,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     } else {
         win_k = V.window[0] + (int64_t)hk * V.cap_window * D;
         win_v = V.window[1] + (int64_t)hk * V.cap_window * D;
-        win_phys = (int)(((int64_t)V.window_head + tok0 + kStepTok * warp) % V.cap_window);
+        win_phys = V.cap_window > 0 ? (int)(((int64_t)V.window_head + tok0 + kStepTok * warp) % V.cap_window) : 0;
     }
     int issue_blk = 0, issue_slot = 0, issue_left = n_tok - kStepTok * warp;  // lane 0's view
     auto issue_next = [&]() {
@@ -900,6 +900,7 @@ __global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
     const AttnView &V = p.views[lo];
     const int c = bx - V.chunk_begin;
     const int hk = blockIdx.y, z = blockIdx.z;
+    if (c >= V.n_chunks) return;  // never launched by the host planner; defensive
     if (c >= V.n_chunks_packed) {
         attn_item<NG, 4, true>(p, V, lo, c, hk, z, smem);
     } else {

@@ -25,12 +25,13 @@ constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: y + magic rounds y to
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;
 
 // Quantize one half (32 elements) of a 64-element group held as 16 bf16x2
-// words; the partner half lives in lane ^ 1, which must execute this call in
-// the same instruction stream (full-warp shuffles).  Writes the packed codes
-// of this half (32*B bits = B words, code j at bit j*B) and the group's s, mn.
+// words (also readable at `src`, used only for the rare exact re-check); the
+// partner half lives in lane ^ 1, which must execute this call in the same
+// instruction stream (full-warp shuffles).  Writes the packed codes of this
+// half (32*B bits = B words, code j at bit j*B) and the group's s, mn.
 template <int B>
-__device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], uint32_t (&packed)[B],
-                                                    float &s_out, float &mn_out) {
+__device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], const uint16_t *src,
+                                                    uint32_t (&packed)[B], float &s_out, float &mn_out) {
     __nv_bfloat162 lo2 = *reinterpret_cast<const __nv_bfloat162 *>(&x[0]);
     __nv_bfloat162 hi2 = lo2;
 #pragma unroll
@@ -89,11 +90,9 @@ __device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], uin
         while (near) {
             const int i = __ffs(near) - 1;
             near &= near - 1u;
-            // element i, re-extracted with a compile-time select chain
-            uint32_t w = x[0];
-#pragma unroll
-            for (int k = 1; k < 16; ++k) w = ((i >> 1) == k) ? x[k] : w;
-            const float xf = (i & 1) ? bf16hi_to_f32(w) : bf16lo_to_f32(w);
+            // element i, re-read from memory (a register array indexed at run
+            // time would be demoted to local memory for the whole loop)
+            const float xf = __uint_as_float((uint32_t)src[i] << 16);
             const float a = __fsub_rn(xf, mn);
             const float y = __fmul_rn(a, r);
             const float t = __fadd_rn(y, kRoundMagic);
@@ -205,7 +204,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(CodecArgs a) {
         for (int u = 0; u < kRounds; ++u) {
             uint32_t packed[B];
             float s, mn;
-            quantize_half_group<B>(x[u], packed, s, mn);
+            quantize_half_group<B>(x[u], xh + t[u] * a.x_tok_stride + g[u] * kGroup + half * 32, packed, s, mn);
             if (active[u]) {
                 uint8_t *dst = ch + t[u] * RB + g[u] * 8 * B + half * 4 * B;
                 if constexpr (B == 4) {
@@ -344,7 +343,7 @@ __global__ void __launch_bounds__(32) append_kernel(AppendArgs a) {
 #define KVQ_APPEND_Q(BB)                                                                         \
     case BB: {                                                                                   \
         uint32_t packed[BB];                                                                     \
-        quantize_half_group<BB>(x, packed, s, mn);                                               \
+        quantize_half_group<BB>(x, src + g * kGroup + half * 32, packed, s, mn);                                               \
         if (active) {                                                                            \
             uint32_t *dst = reinterpret_cast<uint32_t *>(codes_row + g * 8 * BB + half * 4 * BB); \
             _Pragma("unroll") for (int w = 0; w < BB; ++w) dst[w] = packed[w];                    \
