@@ -123,35 +123,31 @@ def ev_pair():
     return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
 
 
-def dist_setup(args):
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1:
-        import datetime
-        import torch.distributed as dist
-        backend = "nccl" if torch.cuda.is_available() else "gloo"
-        if torch.cuda.is_available():
-            torch.cuda.set_device(local)
-        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
-    elif torch.cuda.is_available():
-        torch.cuda.set_device(0)
-    return rank, world, local
+def kernel_source_sha():
+    """sha256 of the decode-attention kernel sources (ties ncu counters to a kernel version)."""
+    import hashlib
+    h = hashlib.sha256()
+    for f in ("kvq_attn.cuh", "kvq_ptx.cuh"):
+        with open(os.path.join(ROOT, "quantized_kv_cache_dequantize_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()
 
 
-def max_over_ranks(x: float, world: int) -> float:
-    if world == 1:
-        return x
-    import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda" if torch.cuda.is_available() else "cpu")
-    dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    return float(t.item())
-
-
-def barrier(world):
-    if world > 1:
-        import torch.distributed as dist
-        dist.barrier()
+def profiled_traffic():
+    """DRAM bytes per launch of the per-layer decode-attention kernel from the
+    committed ncu summary, if it was taken on the current kernel source."""
+    path = os.path.join(ROOT, "profiles", "decode_attn_layer_llama8b.md")
+    try:
+        vals = {}
+        for line in open(path):
+            if ":" in line and line.strip().startswith("- "):
+                k, v = line.strip()[2:].split(":", 1)
+                vals[k.strip()] = v.strip().strip("`")
+        if vals.get("kernel_source_sha256") == kernel_source_sha():
+            return float(vals["dram_bytes_per_launch"])
+    except (OSError, KeyError, ValueError):
+        pass
+    return None
 
 
 # ------------------------------------------------------------ oracle timing --
@@ -210,7 +206,7 @@ def run_reference(args, rank, world):
 
 def run_ours(args, rank, world, local):
     import quantized_kv_cache_dequantize_b200 as kvq
-    from quantized_kv_cache_dequantize_b200 import cache as kcache, workloads as wl
+    from quantized_kv_cache_dequantize_b200 import cache as kcache, dist as kdist, workloads as wl
     dev = torch.device("cuda", torch.cuda.current_device())
     peak, peak_kind = peaks()
     extra = {}
@@ -265,7 +261,7 @@ def run_ours(args, rank, world, local):
     for _ in range(args.warmup):
         graph.replay()
     stream.synchronize()
-    barrier(world)
+    kdist.barrier()
     torch.cuda.synchronize()
     e0, e1 = ev_pair()
     with ClockSampler(local) as clk:
@@ -275,11 +271,10 @@ def run_ours(args, rank, world, local):
                 graph.replay()
             e1.record(stream)
         stream.synchronize()
-    barrier(world)
+    kdist.barrier()
     torch.cuda.synchronize()
-    t_step = e0.elapsed_time(e1) / 1e3 / args.steps
-    t_step = max_over_ranks(t_step, world)
-    value = world * bytes_step / t_step / 1e9
+    t_step = kdist.max_over_ranks(e0.elapsed_time(e1) / 1e3 / args.steps)
+    value = kdist.aggregate_throughput(bytes_step, world, t_step) / 1e9
 
     # ---------------- dominant kernel: kvq_decode_attn per layer, timed alone
     attn_layer_bytes = attn_bytes(A, w.n_kv_heads, w.n_q_heads, w.head_dim, w.view_len(0) + 1, w.window, 4)
@@ -337,8 +332,8 @@ def run_ours(args, rank, world, local):
             e2e_step()
         c1.record(stream)
     stream.synchronize()
-    t_e2e = max_over_ranks(c0.elapsed_time(c1) / 1e3 / args.steps, world)
-    e2e_gbs = world * bytes_step / t_e2e / 1e9
+    t_e2e = kdist.max_over_ranks(c0.elapsed_time(c1) / 1e3 / args.steps)
+    e2e_gbs = kdist.aggregate_throughput(bytes_step, world, t_e2e) / 1e9
 
     del pool, ws, ws_all, q, out
     torch.cuda.empty_cache()
@@ -410,7 +405,7 @@ def run_ours(args, rank, world, local):
             "tokens_per_s_per_agent": 1.0 / t_step,
             "hbm_frac": value / world / peak,
             "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
-                         "frac": attn_gbs / peak, "traffic": None,
+                         "frac": attn_gbs / peak, "traffic": profiled_traffic(),
                          "kernel": "decode_attn_kernel<2> (one kvq_decode_attn per layer, 10 views)",
                          "bytes_per_launch": attn_layer_bytes, "launch_us": t_attn * 1e6,
                          "peak_kind": f"{peak_kind} (hbm_gbs)"},
@@ -435,16 +430,15 @@ def main():
     ap.add_argument("--skip-cpu", action="store_true")
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
-    rank, world, local = dist_setup(args)
+    from quantized_kv_cache_dequantize_b200 import dist as kdist
+    rank, world, local = kdist.init_from_env()
     try:
         if args.impl == "reference":
             run_reference(args, rank, world)
         else:
             run_ours(args, rank, world, local)
     finally:
-        if world > 1:
-            import torch.distributed as dist
-            dist.destroy_process_group()
+        kdist.shutdown()
 
 
 if __name__ == "__main__":

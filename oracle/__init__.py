@@ -47,10 +47,29 @@ def build(force: bool = False) -> str:
     return _LIB_PATH
 
 
-def _load():
+class use_library:
+    """Context manager: route every oracle call through another build of
+    kvq_oracle.c (the mutation tests plant mistakes in a copy)."""
+
+    def __init__(self, path: str):
+        self.path = path
+
+    def __enter__(self):
+        global _lib
+        self.saved = _lib
+        _lib = None
+        _load(self.path)
+        return self
+
+    def __exit__(self, *exc):
+        global _lib
+        _lib = self.saved
+
+
+def _load(path: str | None = None):
     global _lib
     if _lib is None:
-        lib = ctypes.CDLL(build())
+        lib = ctypes.CDLL(path or build())
         P = ctypes.c_void_p
         i32, i64, f64 = ctypes.c_int32, ctypes.c_int64, ctypes.c_double
         lib.oracle_quantize_rows.argtypes = [P, i64, i32, i32, P, P]

@@ -90,9 +90,18 @@ __device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], con
         while (near) {
             const int i = __ffs(near) - 1;
             near &= near - 1u;
-            // element i, re-read from memory (a register array indexed at run
-            // time would be demoted to local memory for the whole loop)
-            const float xf = __uint_as_float((uint32_t)src[i] << 16);
+            // element i from the registers by a binary select tree on the bits
+            // of i (stays in registers; no memory round trip)
+            uint32_t t8[8], t4[4], t2[2];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) t8[k] = (i & 16) ? x[k + 8] : x[k];
+#pragma unroll
+            for (int k = 0; k < 4; ++k) t4[k] = (i & 8) ? t8[k + 4] : t8[k];
+#pragma unroll
+            for (int k = 0; k < 2; ++k) t2[k] = (i & 4) ? t4[k + 2] : t4[k];
+            const uint32_t w = (i & 2) ? t2[1] : t2[0];
+            const float xf = (i & 1) ? bf16hi_to_f32(w) : bf16lo_to_f32(w);
+            (void)src;
             const float a = __fsub_rn(xf, mn);
             const float y = __fmul_rn(a, r);
             const float t = __fadd_rn(y, kRoundMagic);

@@ -1,0 +1,71 @@
+"""Small, fixed kernel cases for profilers (ncu) and quick timing.
+
+    python -m quantized_kv_cache_dequantize_b200.profile_cases CASE [--reps N]
+
+CASE:
+  decode-layer   kvq_decode_attn over one layer of the batched decode
+                 workload (10 agents, Llama-3.1-8B shape: 32 q / 8 kv heads,
+                 head_dim 128, 4096 packed 4-bit tokens + 128-token window)
+  decode-8layers the same over 8 layers (80 views) in one call
+  quantize       kvq_quantize of 64 heads x 32768 tokens x 128 (bf16, 512 MiB)
+  dequantize     kvq_dequantize of the same cache
+Each case runs 3 warm-up calls and then --reps timed calls, and prints the
+mean time per call and the algorithmic GB/s.
+"""
+from __future__ import annotations
+
+import argparse
+import sys
+
+import torch
+
+from . import cache as kcache
+from . import workloads as wl
+from . import decode_attn, dequantize, new_workspace, quantize
+
+
+def _time(fn, reps):
+    for _ in range(3):
+        fn()
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
+    e0.record()
+    for _ in range(reps):
+        fn()
+    e1.record()
+    torch.cuda.synchronize()
+    return e0.elapsed_time(e1) / reps / 1e3
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("case", choices=["decode-layer", "decode-8layers", "quantize", "dequantize"])
+    ap.add_argument("--reps", type=int, default=20)
+    a = ap.parse_args(argv)
+    dev = torch.device("cuda:0")
+    if a.case.startswith("decode"):
+        w = wl.decode_llama8b(n_layers=1 if a.case == "decode-layer" else 8)
+        pool = kcache.build_decode(w, dev)
+        q = kcache.decode_queries(w, device=dev)
+        ws = new_workspace(pool.views, w.n_q_heads, device=dev)
+        out = torch.empty((w.n_views, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+        t = _time(lambda: decode_attn(pool.views, q, w.softmax_scale, out=out, workspace=ws), a.reps)
+        rb = w.head_dim // 8 * 4
+        nbytes = w.n_views * (w.n_kv_heads * (w.view_len(0) * (2 * rb + 2 * (w.head_dim // 64) * 8) +
+                                              w.window * 4 * w.head_dim) + w.n_q_heads * w.head_dim * 6)
+    else:
+        H, T, D = 64, 32768, 128
+        g = wl.generator(2, device=dev)
+        x = wl.normal_bf16(g, (H, T, D), dev)
+        codes, sm = quantize(x, 4)
+        y = torch.empty_like(x)
+        nbytes = x.numel() * 2 + codes.numel() + sm.numel() * 4
+        if a.case == "quantize":
+            t = _time(lambda: quantize(x, 4, codes, sm), a.reps)
+        else:
+            t = _time(lambda: dequantize(codes, sm, T, D, 4, out=y), a.reps)
+    print(f"{a.case}: {t * 1e6:.1f} us per call, {nbytes / t / 1e9:.0f} GB/s")
+
+
+if __name__ == "__main__":
+    main(sys.argv[1:])
