@@ -39,17 +39,15 @@ int device_sm_count() {
 
 template <int B, int NG>
 void launch_codec(bool quant, const kvq::CodecArgs &a, cudaStream_t st) {
-    // grid-stride over each head's groups; about 8 blocks of 8 warps per SM in total
-    const int64_t groups = a.n_tokens * NG;
-    const int64_t warp_groups = 16 * (quant ? kvq::kRounds : kvq::kDeqRounds);
-    const int64_t max_blocks = std::max<int64_t>(1, (groups + 8 * warp_groups - 1) / (8 * warp_groups));
-    const int64_t want = ((int64_t)device_sm_count() * 8 + a.n_heads - 1) / a.n_heads;
-    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(max_blocks, want));
-    dim3 grid((unsigned)blocks, (unsigned)a.n_heads);
+    // one flat sweep over (head, group); blocks of 8 warps, a few per SM
+    const int64_t groups = a.n_tokens * NG * a.n_heads;
+    const int64_t per_block = 8 * 16 * (quant ? 1 : kvq::kDeqRounds);
+    const int64_t max_blocks = std::max<int64_t>(1, (groups + per_block - 1) / per_block);
+    const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(max_blocks, (int64_t)device_sm_count() * 8));
     if (quant)
-        kvq::quantize_kernel<B, NG><<<grid, 256, 0, st>>>(a);
+        kvq::quantize_kernel<B, NG><<<(unsigned)blocks, 256, 0, st>>>(a);
     else
-        kvq::dequantize_kernel<B, NG><<<grid, 256, 0, st>>>(a);
+        kvq::dequantize_kernel<B, NG><<<(unsigned)blocks, 256, 0, st>>>(a);
 }
 
 template <int B>

@@ -167,98 +167,98 @@ struct CodecArgs {
     int64_t head_cap;        // rows per head in codes/scalemin
 };
 
-// Grid: (blocks per head, n_heads).  Each lane pair owns one group per
-// round; a warp owns 16 consecutive groups of one head per round and runs
-// kRounds rounds per iteration with all loads issued before any compute.
-constexpr int kRounds = 1;       // quantize: rounds per iteration (issue-bound: keep registers low)
-constexpr int kDeqRounds = 8;    // dequantize: rounds per iteration (latency-bound: many loads in flight)
+// Grid: 1-D, a few blocks per SM.  The (head, group) space is swept in one
+// global, contiguous order: warp w handles groups [16w, 16w+16) of the flat
+// sequence head-major, then jumps by all warps * 16, so concurrent warps touch
+// one narrow window of memory (TLB- and DRAM-page friendly) and every warp's
+// share is balanced across heads.  The (head, group) cursor advances without
+// division.  Each lane pair owns one group.
+constexpr int kDeqRounds = 4;  // dequantize: groups per lane pair per iteration (latency-bound: many loads in flight)
 
-template <int B, int NG>
-__global__ void __launch_bounds__(256) quantize_kernel(CodecArgs a) {
-    constexpr int RB = 8 * B * NG;  // row bytes
-    const int h = blockIdx.y;
-    const int64_t n_groups = a.n_tokens * NG;
-    const int lane = threadIdx.x & 31;
-    const int half = lane & 1;
-    const int64_t warp_global = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int64_t warp_stride = (int64_t)gridDim.x * (blockDim.x >> 5);
-    const uint16_t *xh = a.x + (int64_t)h * a.x_head_stride;
-    uint8_t *ch = a.codes + (int64_t)h * a.head_cap * RB;
-    float *sh = a.scalemin + (int64_t)h * a.head_cap * NG * 2;
+struct SweepCursor {
+    int64_t grp;  // group within the head
+    int h;        // head
+};
 
-    for (int64_t base = warp_global * 16 * kRounds; base < n_groups; base += warp_stride * 16 * kRounds) {
-        uint32_t x[kRounds][16];
-        int64_t t[kRounds];
-        int g[kRounds];
-        bool active[kRounds];
-#pragma unroll
-        for (int u = 0; u < kRounds; ++u) {
-            const int64_t grp = base + 16 * u + (lane >> 1);
-            active[u] = grp < n_groups;
-            t[u] = grp / NG;
-            g[u] = (int)(grp - t[u] * NG);
-            if (active[u]) {
-                const uint4 *src = reinterpret_cast<const uint4 *>(xh + t[u] * a.x_tok_stride + g[u] * kGroup + half * 32);
-#pragma unroll
-                for (int v = 0; v < 4; ++v) {
-                    const uint4 q = __ldcs(src + v);
-                    x[u][4 * v + 0] = q.x; x[u][4 * v + 1] = q.y; x[u][4 * v + 2] = q.z; x[u][4 * v + 3] = q.w;
-                }
-            } else {
-#pragma unroll
-                for (int i = 0; i < 16; ++i) x[u][i] = 0u;
-            }
-        }
-#pragma unroll
-        for (int u = 0; u < kRounds; ++u) {
-            uint32_t packed[B];
-            float s, mn;
-            quantize_half_group<B>(x[u], xh + t[u] * a.x_tok_stride + g[u] * kGroup + half * 32, packed, s, mn);
-            if (active[u]) {
-                uint8_t *dst = ch + t[u] * RB + g[u] * 8 * B + half * 4 * B;
-                if constexpr (B == 4) {
-                    *reinterpret_cast<uint4 *>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                } else if constexpr (B == 8) {
-                    reinterpret_cast<uint4 *>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
-                    reinterpret_cast<uint4 *>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
-                } else if constexpr (B == 2) {
-                    *reinterpret_cast<uint2 *>(dst) = make_uint2(packed[0], packed[1]);
-                } else {
-#pragma unroll
-                    for (int w = 0; w < B; ++w) reinterpret_cast<uint32_t *>(dst)[w] = packed[w];
-                }
-                if (half == 0) *reinterpret_cast<float2 *>(sh + (t[u] * NG + g[u]) * 2) = make_float2(s, mn);
-            }
-        }
+__device__ __forceinline__ void sweep_advance(SweepCursor &c, int64_t step, int64_t n_groups) {
+    c.grp += step;
+    while (c.grp >= n_groups) {
+        c.grp -= n_groups;
+        ++c.h;
     }
 }
 
 template <int B, int NG>
-__global__ void __launch_bounds__(256) dequantize_kernel(CodecArgs a) {
-    constexpr int RB = 8 * B * NG;
-    const int h = blockIdx.y;
+__global__ void __launch_bounds__(256) quantize_kernel(CodecArgs a) {
+    constexpr int RB = 8 * B * NG;  // row bytes
     const int64_t n_groups = a.n_tokens * NG;
     const int lane = threadIdx.x & 31;
     const int half = lane & 1;
     const int64_t warp_global = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
     const int64_t warp_stride = (int64_t)gridDim.x * (blockDim.x >> 5);
-    uint16_t *yh = const_cast<uint16_t *>(a.x) + (int64_t)h * a.x_head_stride;
-    const uint8_t *ch = a.codes + (int64_t)h * a.head_cap * RB;
-    const float *sh = a.scalemin + (int64_t)h * a.head_cap * NG * 2;
-    constexpr int kR = kDeqRounds;
+    SweepCursor cur{0, 0};
+    sweep_advance(cur, warp_global * 16 + (lane >> 1), n_groups);
+    for (; cur.h < a.n_heads; sweep_advance(cur, warp_stride * 16, n_groups)) {
+        const int64_t t = cur.grp / NG;
+        const int g = (int)(cur.grp - t * NG);
+        const uint16_t *src = a.x + (int64_t)cur.h * a.x_head_stride + t * a.x_tok_stride + g * kGroup + half * 32;
+        uint32_t x[16];
+        const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) {
+            const uint4 q = __ldcs(s4 + v);
+            x[4 * v + 0] = q.x; x[4 * v + 1] = q.y; x[4 * v + 2] = q.z; x[4 * v + 3] = q.w;
+        }
+        uint32_t packed[B];
+        float s, mn;
+        quantize_half_group<B>(x, src, packed, s, mn);
+        const int64_t row = (int64_t)cur.h * a.head_cap + t;
+        uint8_t *dst = a.codes + row * RB + g * 8 * B + half * 4 * B;
+        if constexpr (B == 4) {
+            *reinterpret_cast<uint4 *>(dst) = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+        } else if constexpr (B == 8) {
+            reinterpret_cast<uint4 *>(dst)[0] = make_uint4(packed[0], packed[1], packed[2], packed[3]);
+            reinterpret_cast<uint4 *>(dst)[1] = make_uint4(packed[4], packed[5], packed[6], packed[7]);
+        } else if constexpr (B == 2) {
+            *reinterpret_cast<uint2 *>(dst) = make_uint2(packed[0], packed[1]);
+        } else {
+#pragma unroll
+            for (int w = 0; w < B; ++w) reinterpret_cast<uint32_t *>(dst)[w] = packed[w];
+        }
+        if (half == 0) *reinterpret_cast<float2 *>(a.scalemin + (row * NG + g) * 2) = make_float2(s, mn);
+    }
+}
 
-    for (int64_t base = warp_global * 16 * kR; base < n_groups; base += warp_stride * 16 * kR) {
+// Same sweep; each lane pair dequantizes kDeqRounds groups per iteration
+// (all loads first, then compute and streaming stores).
+template <int B, int NG>
+__global__ void __launch_bounds__(256) dequantize_kernel(CodecArgs a) {
+    constexpr int RB = 8 * B * NG;
+    constexpr int kR = kDeqRounds;
+    const int64_t n_groups = a.n_tokens * NG;
+    const int lane = threadIdx.x & 31;
+    const int half = lane & 1;
+    const int64_t warp_global = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    const int64_t warp_stride = (int64_t)gridDim.x * (blockDim.x >> 5);
+    uint16_t *y = const_cast<uint16_t *>(a.x);
+    SweepCursor cur{0, 0};
+    sweep_advance(cur, warp_global * 16 * kR + (lane >> 1), n_groups);
+    while (cur.h < a.n_heads) {
         uint32_t packed[kR][B];
         float2 sm[kR];
         int64_t t[kR];
-        int g[kR];
+        int g[kR], hh[kR];
+        bool ok[kR];
+        SweepCursor c = cur;
 #pragma unroll
         for (int u = 0; u < kR; ++u) {
-            const int64_t grp = base + 16 * u + (lane >> 1);
-            t[u] = grp / NG;
-            g[u] = (int)(grp - t[u] * NG);
-            if (grp < n_groups) {
-                const uint8_t *src = ch + t[u] * RB + g[u] * 8 * B + half * 4 * B;
+            ok[u] = c.h < a.n_heads;
+            hh[u] = c.h;
+            t[u] = c.grp / NG;
+            g[u] = (int)(c.grp - t[u] * NG);
+            if (ok[u]) {
+                const int64_t row = (int64_t)c.h * a.head_cap + t[u];
+                const uint8_t *src = a.codes + row * RB + g[u] * 8 * B + half * 4 * B;
                 if constexpr (B == 4) {
                     const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(src));
                     packed[u][0] = q.x; packed[u][1] = q.y; packed[u][2] = q.z; packed[u][3] = q.w;
@@ -274,18 +274,21 @@ __global__ void __launch_bounds__(256) dequantize_kernel(CodecArgs a) {
 #pragma unroll
                     for (int w = 0; w < B; ++w) packed[u][w] = __ldcs(reinterpret_cast<const uint32_t *>(src) + w);
                 }
-                sm[u] = __ldcs(reinterpret_cast<const float2 *>(sh + (t[u] * NG + g[u]) * 2));
+                sm[u] = __ldcs(reinterpret_cast<const float2 *>(a.scalemin + (row * NG + g[u]) * 2));
             }
+            sweep_advance(c, 16, n_groups);
         }
 #pragma unroll
         for (int u = 0; u < kR; ++u) {
-            if (base + 16 * u + (lane >> 1) >= n_groups) continue;
-            uint32_t y[16];
-            dequantize_half_group<B>(packed[u], sm[u].x, sm[u].y, y);
-            uint4 *dst = reinterpret_cast<uint4 *>(yh + t[u] * a.x_tok_stride + g[u] * kGroup + half * 32);
+            if (!ok[u]) continue;
+            uint32_t yv[16];
+            dequantize_half_group<B>(packed[u], sm[u].x, sm[u].y, yv);
+            uint4 *dst = reinterpret_cast<uint4 *>(y + (int64_t)hh[u] * a.x_head_stride + t[u] * a.x_tok_stride +
+                                                   g[u] * kGroup + half * 32);
 #pragma unroll
-            for (int v = 0; v < 4; ++v) __stcs(dst + v, make_uint4(y[4 * v], y[4 * v + 1], y[4 * v + 2], y[4 * v + 3]));
+            for (int v = 0; v < 4; ++v) __stcs(dst + v, make_uint4(yv[4 * v], yv[4 * v + 1], yv[4 * v + 2], yv[4 * v + 3]));
         }
+        sweep_advance(cur, warp_stride * 16 * kR, n_groups);
     }
 }
 

@@ -9,6 +9,9 @@ CASE:
   decode-8layers the same over 8 layers (80 views) in one call
   quantize       kvq_quantize of 64 heads x 32768 tokens x 128 (bf16, 512 MiB)
   dequantize     kvq_dequantize of the same cache
+  quantize-handoff / dequantize-handoff
+                 the bulk handoff's K cache: 32 layers x 8 kv heads x 32768
+                 tokens x 128 (2 GiB bf16), 1% outlier channels x10
 Each case runs 3 warm-up calls and then --reps timed calls, and prints the
 mean time per call and the algorithmic GB/s.
 """
@@ -39,7 +42,8 @@ def _time(fn, reps):
 
 def main(argv=None):
     ap = argparse.ArgumentParser()
-    ap.add_argument("case", choices=["decode-layer", "decode-8layers", "quantize", "dequantize"])
+    ap.add_argument("case", choices=["decode-layer", "decode-8layers", "quantize", "dequantize", "quantize-handoff",
+                                         "dequantize-handoff"])
     ap.add_argument("--reps", type=int, default=20)
     a = ap.parse_args(argv)
     dev = torch.device("cuda:0")
@@ -54,13 +58,20 @@ def main(argv=None):
         nbytes = w.n_views * (w.n_kv_heads * (w.view_len(0) * (2 * rb + 2 * (w.head_dim // 64) * 8) +
                                               w.window * 4 * w.head_dim) + w.n_q_heads * w.head_dim * 6)
     else:
-        H, T, D = 64, 32768, 128
-        g = wl.generator(2, device=dev)
-        x = wl.normal_bf16(g, (H, T, D), dev)
+        if a.case.endswith("handoff"):
+            hw = wl.handoff_llama8b()
+            H, T, D = hw.n_layers * hw.n_kv_heads, hw.n_tokens, hw.head_dim
+            gm = wl.generator(hw.seed)
+            mask = torch.stack([wl.outlier_mask(gm, hw.n_kv_heads, D, hw.outlier_frac)
+                                for _ in range(hw.n_layers)]).view(H, D)
+            x = wl.normal_bf16(wl.generator(hw.seed, device=dev), (H, T, D), dev, mask)
+        else:
+            H, T, D = 64, 32768, 128
+            x = wl.normal_bf16(wl.generator(2, device=dev), (H, T, D), dev)
         codes, sm = quantize(x, 4)
         y = torch.empty_like(x)
         nbytes = x.numel() * 2 + codes.numel() + sm.numel() * 4
-        if a.case == "quantize":
+        if a.case.startswith("quantize"):
             t = _time(lambda: quantize(x, 4, codes, sm), a.reps)
         else:
             t = _time(lambda: dequantize(codes, sm, T, D, 4, out=y), a.reps)
