@@ -238,7 +238,10 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream()
-    n_launch_per_step = 2 * L
+    # per layer: the append kernel, the attention grid and its split-K
+    # combine grid (every view here has packed and window tokens, so every
+    # unit has more than one chunk and the combine grid is launched)
+    n_launch_per_step = 3 * L
 
     def step():
         for l in range(L):

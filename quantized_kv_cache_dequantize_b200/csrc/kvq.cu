@@ -108,7 +108,7 @@ struct AttnPlan {
     int head_blocks = 0;
     std::vector<AttnLaunch> launches;
     std::vector<ViewChunks> chunks;
-    size_t counters_off = 0, partials_off = 0, total = 0;
+    size_t partials_off = 0, total = 0;
 };
 
 int env_int(const char *name, int dflt) {
@@ -201,7 +201,7 @@ int64_t chunk_views(const kvq_view *views, int v0, int v1, int64_t units, int32_
                 c.n_packed = (int32_t)((v.n_packed + ch - 1) / ch);
                 c.n_window = (int32_t)((v.n_window + ch - 1) / ch);
             }
-            // the in-kernel merge holds at most kMaxChunksPerUnit chunks per unit
+            // the combine grid holds at most kMaxChunksPerUnit chunks per unit
             while (c.n_packed + c.n_window > kvq::kMaxChunksPerUnit) {
                 if (c.n_packed >= c.n_window) {
                     c.chunk_packed *= 2;
@@ -222,7 +222,7 @@ int64_t chunk_views(const kvq_view *views, int v0, int v1, int64_t units, int32_
     // Pick the item size with the smallest predicted makespan: whole waves of
     // resident CTAs, each wave as long as its largest item plus a fixed
     // per-CTA cost (set-up, pipeline fill, merge), in byte-equivalents.
-    const double kMinItem = 16.0 * 1024, kBigItem = 256.0 * 1024, kCtaCost = 24.0 * 1024;
+    const double kMinItem = 16.0 * 1024, kBigItem = 256.0 * 1024, kCtaCost = 96.0 * 1024;
     double best_W = std::max(kMinItem, std::min(kBigItem, total / (double)slots)), best_cost = 1e300;
     const double fs[] = {0.6, 0.7, 0.8, 0.9, 1.0, 1.15, 1.3, 1.5, 1.75, 2.0, 2.5, 3.0, 4.0, 5.0, 6.0, 8.0, 12.0, 16.0, 24.0, 32.0};
     for (double f : fs) {
@@ -263,11 +263,8 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, 
         if (views[i].n_window > 0) blk_max = std::max<uint32_t>(blk_max, (uint32_t)(32 * head_dim));
     }
     int ring = (smem_cta - header) / kvq::kAttnWarps / 128 * 128;
-    // a ring holds two blocks, and later the warp's partial; all rings together
-    // hold the unit merge's scratch
-    const uint32_t merge_scratch = (2 * kvq::kMaxChunksPerUnit * kvq::kHeadsPerCta + kvq::kHeadsPerCta) * 4;
-    const int ring_min = (int)std::max<uint32_t>(std::max<uint32_t>(2 * blk_max, (uint32_t)(64 + 32 * head_dim)),
-                                                 (merge_scratch + kvq::kAttnWarps - 1) / kvq::kAttnWarps);
+    // a ring holds two blocks, and later the warp's partial (m, l, O of 8 heads)
+    const int ring_min = (int)std::max<uint32_t>(2 * blk_max, (uint32_t)(64 + 32 * head_dim));
     if (ring < ring_min) ring = (ring_min + 127) / 128 * 128;  // fewer CTAs per SM, still correct
     plan.ring_bytes = ring;
     plan.smem = (size_t)header + (size_t)kvq::kAttnWarps * ring;
@@ -276,18 +273,14 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, 
     const int64_t slots = (int64_t)device_sm_count() * ctas;
     plan.chunks.assign(n_views, ViewChunks{16, 16, 0, 0});
     int64_t max_chunks = 0;
-    int max_views = 0;
     for (int v0 = 0; v0 < n_views; v0 += kvq::kAttnMaxViews) {
         const int v1 = std::min<int>(n_views, v0 + kvq::kAttnMaxViews);
         const int64_t chunks = chunk_views(views, v0, v1, units, head_dim, slots, plan.chunks);
         if (chunks > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
         plan.launches.push_back({v0, v1, (int)chunks});
         max_chunks = std::max(max_chunks, chunks);
-        max_views = std::max(max_views, v1 - v0);
     }
-    const size_t n_units = (size_t)max_views * units;
-    plan.counters_off = 256;
-    plan.partials_off = plan.counters_off + (n_units * 4 + 255) / 256 * 256;
+    plan.partials_off = 256;  // bytes [0, 4): the device status word
     const size_t part_floats = (size_t)max_chunks * units * kvq::kHeadsPerCta * (head_dim + 2);
     plan.total = plan.partials_off + part_floats * 4;
     return KVQ_OK;
@@ -310,7 +303,6 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
     prm.q = static_cast<const uint16_t *>(q);
     prm.out = out;
     prm.status = reinterpret_cast<uint32_t *>(ws);
-    prm.counters = reinterpret_cast<uint32_t *>(ws + plan.counters_off);
     prm.partials = reinterpret_cast<float *>(ws + plan.partials_off);
     prm.timeout_ns = 2000000000ull;
     prm.scale_log2 = scale * 1.4426950408889634f;
@@ -346,9 +338,27 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
             d.view_index = i;
             begin += d.n_chunks;
         }
-        dim3 grid((unsigned)L.total_chunks, (unsigned)n_kv_heads, (unsigned)plan.head_blocks);
-        kvq::decode_attn_kernel<NG><<<grid, kvq::kAttnThreads, plan.smem, st>>>(prm);
-        if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+        // Both grids carry a programmatic dependency on the preceding work in
+        // the stream: each starts with griddepcontrol.wait, so it reads
+        // nothing before its predecessor has completed, while its launch and
+        // CTA scheduling overlap the predecessor's tail.
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr.val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof cfg);
+        cfg.gridDim = dim3((unsigned)L.total_chunks, (unsigned)n_kv_heads, (unsigned)plan.head_blocks);
+        cfg.blockDim = dim3(kvq::kAttnThreads);
+        cfg.dynamicSmemBytes = plan.smem;
+        cfg.stream = st;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        if (cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG>, prm) != cudaSuccess) return KVQ_ERR_CUDA;
+        if (L.total_chunks > L.v1 - L.v0) {  // some unit has more than one chunk
+            cfg.gridDim = dim3((unsigned)(L.v1 - L.v0), (unsigned)n_kv_heads, (unsigned)plan.head_blocks);
+            cfg.dynamicSmemBytes = 0;
+            if (cudaLaunchKernelEx(&cfg, kvq::combine_kernel<NG>, prm) != cudaSuccess) return KVQ_ERR_CUDA;
+        }
     }
     return KVQ_OK;
 }

@@ -27,9 +27,10 @@
 //        tile is moved from the QK accumulator layout to the B-operand layout
 //        with movmatrix.
 // Window tiles (bf16 K/V) use the same tile loop with the values as operands.
-// Each CTA merges its warps in a fixed order; the last CTA of a unit (an
-// atomic arrival counter, never a spin) merges the chunks in chunk order, so
-// results are bitwise reproducible.
+// Each CTA merges its warps in a fixed order and writes its chunk's partial
+// (m, l, O); a small combine grid, launched with a programmatic dependency,
+// merges each unit's chunks in chunk order, so results are bitwise
+// reproducible and no CTA waits on another.
 #pragma once
 
 #include <cstdint>
@@ -45,7 +46,7 @@ constexpr int kTile = 16;
 constexpr int kMaxStages = 12;
 constexpr int kHeadsPerCta = 8;
 constexpr int kAttnMaxViews = 96;
-constexpr int kMaxChunksPerUnit = 256;  // merge scratch: 2 * 256 * 8 floats in the ring area
+constexpr int kMaxChunksPerUnit = 256;  // combine scratch: 2 * 256 * 8 floats of static shared memory
 
 struct AttnView {
     const uint8_t *codes[2];     // K, V packed rows [H_kv][cap][RB]
@@ -70,7 +71,6 @@ struct AttnParams {
     const uint16_t *q;           // bf16 [n_views_total][Hq][D]
     float *out;                  // fp32 [n_views_total][Hq][D]
     float *partials;             // workspace
-    uint32_t *counters;          // workspace
     uint32_t *status;            // workspace word 0
     uint64_t timeout_ns;
     float scale_log2;            // softmax_scale * log2(e)
@@ -289,6 +289,12 @@ struct WarpState {
 // gid+8; R = 4: two tiles).  lg[r][j] are base-2 logits of this lane's rows
 // for heads 2tig, 2tig+1; they are replaced by the probabilities relative to
 // the new running max.
+// The running max is only moved when a tile exceeds it by more than
+// kLazyMax (log2 units): probabilities relative to a stale max stay below
+// 2^kLazyMax, harmless in fp32 sums and bf16 hi/lo operands, and the O rescale
+// (32+ multiplies) becomes rare instead of firing on most early tiles.
+constexpr float kLazyMax = 8.0f;
+
 template <int NG, int R>
 __device__ __forceinline__ void softmax_step_n(WarpState<NG> &st, float (&lg)[R][2]) {
     float alpha[2];
@@ -300,7 +306,7 @@ __device__ __forceinline__ void softmax_step_n(WarpState<NG> &st, float (&lg)[R]
         t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 4));
         t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 8));
         t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 16));
-        const float mnew = fmaxf(st.m[j], t);
+        const float mnew = (t > st.m[j] + kLazyMax) ? t : st.m[j];
         alpha[j] = fast_exp2(st.m[j] - mnew);
         st.m[j] = mnew;
         float sum = 0.f;
@@ -534,7 +540,7 @@ __host__ __device__ constexpr int attn_header_bytes() {
 // the block's bulk copies; one lane issues the copies and a slot is refilled
 // as soon as the warp has consumed it.
 template <int NG, int B, bool WINDOW>
-__device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V, int vi, int c, int hk, int z,
+__device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V, int c, int hk, int z,
                                           uint8_t *smem) {
     constexpr int D = 64 * NG;
     constexpr int RB = 8 * B * NG;
@@ -545,7 +551,6 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     constexpr uint32_t kBlk = WINDOW ? (uint32_t)(kTile * D * 2) : (uint32_t)(kOffVs + 2 * kTile * NG * 8);
     uint16_t *q_s = reinterpret_cast<uint16_t *>(smem);                              // [8][D]
     uint64_t *bars = reinterpret_cast<uint64_t *>(smem + 8 * D * 2);                // [4][kMaxStages]
-    int *flag_s = reinterpret_cast<int *>(bars + kAttnWarps * kMaxStages);
     uint8_t *rings = smem + attn_header_bytes<NG>();
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -794,7 +799,6 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
 
     // ---- merge the 4 warps (fixed order)
     const bool single = V.n_chunks == 1;
-    const int units_per_view = p.n_kv_heads * p.head_blocks;
     const int64_t pslot = ((int64_t)(V.chunk_begin + c) * p.n_kv_heads + hk) * p.head_blocks + z;
     float *part = p.partials + pslot * (kHeadsPerCta * (D + 2));
     for (int idx = tid; idx < nh * D; idx += kAttnThreads) {
@@ -822,27 +826,60 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             }
         }
     }
-    if (single) return;
+}
 
-    // ---- last CTA of the unit merges all chunks, in chunk order
-    __threadfence();
-    __syncthreads();
-    uint32_t *counter = p.counters + ((int64_t)vi * units_per_view + hk * p.head_blocks + z);
-    if (tid == 0) {
-        const uint32_t prev = atomicAdd(counter, 1u);
-        flag_s[0] = (prev == (uint32_t)(V.n_chunks - 1)) ? 1 : 0;
+template <int NG>
+__global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
+    decode_attn_kernel(const __grid_constant__ AttnParams p) {
+    extern __shared__ __align__(128) uint8_t smem[];
+    pdl_wait();               // inputs may come from the preceding grid
+    pdl_launch_dependents();  // the combine grid may be scheduled as slots free up
+    // ---- which item: view by binary search over chunk ranges
+    const int bx = blockIdx.x;
+    int lo = 0, hi = p.n_views - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (p.views[mid].chunk_begin <= bx) lo = mid; else hi = mid - 1;
     }
-    __syncthreads();
-    if (!flag_s[0]) return;
-    __threadfence();
+    const AttnView &V = p.views[lo];
+    const int c = bx - V.chunk_begin;
+    const int hk = blockIdx.y, z = blockIdx.z;
+    if (c >= V.n_chunks) return;  // never launched by the host planner; defensive
+    if (c >= V.n_chunks_packed) {
+        attn_item<NG, 4, true>(p, V, c, hk, z, smem);
+    } else {
+        switch (V.bits) {
+            case 2: attn_item<NG, 2, false>(p, V, c, hk, z, smem); break;
+            case 3: attn_item<NG, 3, false>(p, V, c, hk, z, smem); break;
+            case 4: attn_item<NG, 4, false>(p, V, c, hk, z, smem); break;
+            default: attn_item<NG, 8, false>(p, V, c, hk, z, smem); break;
+        }
+    }
+}
+
+// Split-K combine: one CTA per (view, KV head, head block) with more than one
+// chunk.  Gathers every chunk's (m, l) per head in one pass, reduces per head
+// with warp shuffles, and sums the chunk partials in chunk order (loads 8
+// deep), so results are bitwise reproducible.  Launched right after the
+// attention grid with a programmatic dependency: it is scheduled while the
+// attention tail runs and waits for that grid's completion before reading.
+template <int NG>
+__global__ void __launch_bounds__(kAttnThreads) combine_kernel(const __grid_constant__ AttnParams p) {
+    constexpr int D = 64 * NG;
+    __shared__ float sm_w[kMaxChunksPerUnit * kHeadsPerCta];  // m, then weight
+    __shared__ float sm_l[kMaxChunksPerUnit * kHeadsPerCta];
+    __shared__ float sm_L[kHeadsPerCta];
+    const int vi = blockIdx.x, hk = blockIdx.y, z = blockIdx.z;
+    const AttnView &V = p.views[vi];
+    const int n = V.n_chunks;
+    if (n <= 1) return;  // single-chunk units were written by the attention grid
+    pdl_wait();
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h0 = hk * p.group + z * kHeadsPerCta;
+    const int nh = min(kHeadsPerCta, p.group - z * kHeadsPerCta);
     const int64_t slot0 = ((int64_t)V.chunk_begin * p.n_kv_heads + hk) * p.head_blocks + z;
     const int64_t slot_stride = (int64_t)p.n_kv_heads * p.head_blocks * (kHeadsPerCta * (D + 2));
     const float *part0 = p.partials + slot0 * (kHeadsPerCta * (D + 2));
-    const int n = V.n_chunks;  // <= kMaxChunksPerUnit (host-enforced)
-    // (1) every chunk's (m, l) per head, gathered in one parallel pass
-    float *sm_w = reinterpret_cast<float *>(rings);           // [n][8]: m, then weight
-    float *sm_l = sm_w + kMaxChunksPerUnit * kHeadsPerCta;    // [n][8]: l
-    float *sm_L = sm_l + kMaxChunksPerUnit * kHeadsPerCta;    // [8]: total
     for (int i = tid; i < n * nh; i += kAttnThreads) {
         const int cc = i / nh, j = i - cc * nh;
         const float *pc = part0 + cc * slot_stride + j * (D + 2);
@@ -850,7 +887,6 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         sm_l[cc * kHeadsPerCta + j] = __ldcg(pc + D + 1);
     }
     __syncthreads();
-    // (2) per head: max, weights 2^(m_c - M), total L (warp w owns heads w, w+4)
     for (int j = warp; j < nh; j += kAttnWarps) {
         float M = -INFINITY;
         for (int cc = lane; cc < n; cc += 32) M = fmaxf(M, sm_w[cc * kHeadsPerCta + j]);
@@ -858,7 +894,8 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
         float L = 0.f;
         for (int cc = lane; cc < n; cc += 32) {
-            const float w = fast_exp2(sm_w[cc * kHeadsPerCta + j] - M);
+            const float mc = sm_w[cc * kHeadsPerCta + j];
+            const float w = (mc == -INFINITY) ? 0.f : fast_exp2(mc - M);
             sm_w[cc * kHeadsPerCta + j] = w;
             L = fmaf(w, sm_l[cc * kHeadsPerCta + j], L);
         }
@@ -867,7 +904,6 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         if (lane == 0) sm_L[j] = L;
     }
     __syncthreads();
-    // (3) outputs: weighted sum over chunks in chunk order, loads batched 8 deep
     for (int idx = tid; idx < nh * D; idx += kAttnThreads) {
         const int j = idx / D, d = idx - j * D;
         const float *pj = part0 + j * (D + 2) + d;
@@ -882,34 +918,6 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         }
         for (; cc < n; ++cc) O = fmaf(sm_w[cc * kHeadsPerCta + j], __ldcg(pj + cc * slot_stride), O);
         p.out[((int64_t)V.view_index * p.n_q_heads + h0 + j) * D + d] = O / sm_L[j];
-    }
-    if (tid == 0) atomicExch(counter, 0u);
-}
-
-template <int NG>
-__global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
-    decode_attn_kernel(const __grid_constant__ AttnParams p) {
-    extern __shared__ __align__(128) uint8_t smem[];
-    // ---- which item: view by binary search over chunk ranges
-    const int bx = blockIdx.x;
-    int lo = 0, hi = p.n_views - 1;
-    while (lo < hi) {
-        const int mid = (lo + hi + 1) >> 1;
-        if (p.views[mid].chunk_begin <= bx) lo = mid; else hi = mid - 1;
-    }
-    const AttnView &V = p.views[lo];
-    const int c = bx - V.chunk_begin;
-    const int hk = blockIdx.y, z = blockIdx.z;
-    if (c >= V.n_chunks) return;  // never launched by the host planner; defensive
-    if (c >= V.n_chunks_packed) {
-        attn_item<NG, 4, true>(p, V, lo, c, hk, z, smem);
-    } else {
-        switch (V.bits) {
-            case 2: attn_item<NG, 2, false>(p, V, lo, c, hk, z, smem); break;
-            case 3: attn_item<NG, 3, false>(p, V, lo, c, hk, z, smem); break;
-            case 4: attn_item<NG, 4, false>(p, V, lo, c, hk, z, smem); break;
-            default: attn_item<NG, 8, false>(p, V, lo, c, hk, z, smem); break;
-        }
     }
 }
 
