@@ -202,6 +202,40 @@ kvq_status kvq_decode_attn(const kvq_view *views, int32_t n_views, int32_t n_q_h
                            float softmax_scale, float *out, void *workspace,
                            size_t workspace_bytes, void *stream);
 
+/* Bytes of the per-device scratch array kvq_decode_attn_noalloc uses. */
+#define KVQ_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
+
+/*
+ * kvq_decode_attn_noalloc -- kvq_decode_attn without a caller-supplied
+ * workspace, allocating no device memory.  None of the source pages has a
+ * counterpart: this is a convenience of the library.
+ *
+ * For callers that cannot allocate device memory at the moment they attend:
+ * a serving loop that has handed all free HBM to its KV-cache pool (any later
+ * cudaMalloc would fail), or a plain C host with no device allocator of its
+ * own to hold a workspace.  The scratch instead comes from one fixed array of
+ * KVQ_NOALLOC_SCRATCH_BYTES per device, compiled into the library.
+ *
+ * Arguments, layouts and results are those of kvq_decode_attn without
+ * workspace / workspace_bytes; the same kernels run on the same plan, so the
+ * result is the same.
+ * Set-up: the first call on a device (with that device current) looks up the
+ * array's device address once; make that first call before any stream
+ * capture.
+ * Each call clears the array's status word on `stream` before its kernels;
+ * the word is not reported back (kvq_decode_attn exposes it).
+ * Errors: KVQ_ERR_CAPACITY, with nothing enqueued, when the views need more
+ * scratch than KVQ_NOALLOC_SCRATCH_BYTES (kvq_decode_attn_workspace_size
+ * gives the need); KVQ_ERR_CUDA if the set-up lookup fails; otherwise as
+ * kvq_decode_attn.
+ * Concurrency: every call on a device shares the one array, so calls that can
+ * overlap on the GPU (different streams, different host threads) race and
+ * corrupt each other's results: keep them in one stream or serialize them.
+ */
+kvq_status kvq_decode_attn_noalloc(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
+                                   int32_t n_kv_heads, int32_t head_dim, const void *q,
+                                   float softmax_scale, float *out, void *stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -10,6 +10,10 @@ Entry points (same names as the C ABI, without the ``kvq_`` prefix):
   quantize, dequantize          -- bf16 rows <-> packed b-bit codes + {s, mn}
   View, append                  -- one (agent, layer) cache; add a decode token
   decode_attn, workspace_size   -- batched split-K attention over many views
+  decode_attn_noalloc           -- the same without a workspace: scratch is a
+                                   fixed per-device array inside the library
+                                   (NOALLOC_SCRATCH_BYTES), for callers that
+                                   cannot allocate device memory when they attend
 """
 from __future__ import annotations
 
@@ -21,9 +25,10 @@ import torch
 from . import workloads  # noqa: F401  (seeded input generators)
 
 __all__ = ["quantize", "dequantize", "View", "append", "decode_attn", "workspace_size",
-           "KvqError", "lib", "row_bytes", "GROUP"]
+           "decode_attn_noalloc", "NOALLOC_SCRATCH_BYTES", "KvqError", "lib", "row_bytes", "GROUP"]
 
 GROUP = 64
+NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024   # KVQ_NOALLOC_SCRATCH_BYTES in kvq.h
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libkvq.so")
 _lib = None
@@ -71,6 +76,8 @@ def lib():
         L.kvq_decode_attn_workspace_size.restype = sz
         L.kvq_decode_attn.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, f32, P, P, sz, P]
         L.kvq_decode_attn.restype = i32
+        L.kvq_decode_attn_noalloc.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, f32, P, P]
+        L.kvq_decode_attn_noalloc.restype = i32
         _lib = L
     return _lib
 
@@ -254,4 +261,20 @@ def decode_attn(views, q: torch.Tensor, softmax_scale: float, out: torch.Tensor 
     _check(lib().kvq_decode_attn(arr, len(views), Hq, views[0].n_kv_heads, D, _ptr(q), float(softmax_scale),
                                  _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
            "kvq_decode_attn")
+    return out
+
+
+def decode_attn_noalloc(views, q: torch.Tensor, softmax_scale: float, out: torch.Tensor, stream=None,
+                        _arr=None) -> torch.Tensor:
+    """kvq_decode_attn_noalloc: like decode_attn, but the library allocates
+    nothing: its scratch is a fixed per-device array of NOALLOC_SCRATCH_BYTES.
+    ``out`` (fp32 [n_views, H_q, D]) must be given, so this call allocates no
+    device memory either.  Calls that may overlap on the GPU race on the one
+    array; the first call on a device should come before any stream capture."""
+    views = list(views)
+    n, Hq, D = q.shape
+    arr = _arr if _arr is not None else _view_array(views)
+    _check(lib().kvq_decode_attn_noalloc(arr, len(views), Hq, views[0].n_kv_heads, D, _ptr(q),
+                                         float(softmax_scale), _ptr(out), _stream(stream)),
+           "kvq_decode_attn_noalloc")
     return out

@@ -7,6 +7,7 @@
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "kvq.h"
@@ -363,6 +364,47 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
     return KVQ_OK;
 }
 
+// ------------------------------------------- fixed scratch (no allocation) ---
+
+// Scratch of kvq_decode_attn_noalloc: one array per device, laid out like a
+// kvq_decode_attn workspace (status word at byte 0, partials from byte 256).
+static __device__ __align__(256) uint8_t g_noalloc_scratch[KVQ_NOALLOC_SCRATCH_BYTES];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mutex;
+void *g_noalloc_ptr[kMaxDevices] = {};
+
+// Device address of the array on the current device, looked up once per device.
+kvq_status noalloc_scratch(void **out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return KVQ_ERR_CUDA;
+    }
+    if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+    if (!g_noalloc_ptr[dev]) {
+        void *p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p || !aligned(p, 256)) {
+            (void)cudaGetLastError();
+            return KVQ_ERR_CUDA;
+        }
+        g_noalloc_ptr[dev] = p;
+    }
+    *out = g_noalloc_ptr[dev];
+    return KVQ_OK;
+}
+
+kvq_status launch_attn(const AttnPlan &plan, const kvq_view *views, int32_t n_q_heads, int32_t n_kv_heads,
+                       int32_t head_dim, const void *q, float scale, float *out, uint8_t *ws, cudaStream_t st) {
+    switch (head_dim / 64) {
+        case 1: return launch_attn_ng<1>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st);
+        case 2: return launch_attn_ng<2>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st);
+        case 3: return launch_attn_ng<3>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st);
+        default: return launch_attn_ng<4>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st);
+    }
+}
+
 }  // namespace
 
 // ================================================================ C ABI ===
@@ -492,4 +534,23 @@ KVQ_API kvq_status kvq_decode_attn(const kvq_view *views, int32_t n_views, int32
         case 3: return launch_attn_ng<3>(plan, views, n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st);
         default: return launch_attn_ng<4>(plan, views, n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st);
     }
+}
+
+KVQ_API kvq_status kvq_decode_attn_noalloc(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
+                                           int32_t n_kv_heads, int32_t head_dim, const void *q, float softmax_scale,
+                                           float *out, void *stream) {
+    AttnPlan plan;
+    const kvq_status ps = plan_attn(views, n_views, n_q_heads, n_kv_heads, head_dim, plan);
+    if (ps != KVQ_OK) return ps;
+    if (!q || !out) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(out, 16)) return KVQ_ERR_INVALID_ARG;
+    if (plan.total > (size_t)KVQ_NOALLOC_SCRATCH_BYTES) return KVQ_ERR_CAPACITY;
+    void *scratch = nullptr;
+    const kvq_status ss = noalloc_scratch(&scratch);
+    if (ss != KVQ_OK) return ss;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    // the status word must start at zero; nothing else is read before written
+    if (cudaMemsetAsync(scratch, 0, sizeof(uint32_t), st) != cudaSuccess) return KVQ_ERR_CUDA;
+    return launch_attn(plan, views, n_q_heads, n_kv_heads, head_dim, q, softmax_scale, out,
+                       static_cast<uint8_t *>(scratch), st);
 }
