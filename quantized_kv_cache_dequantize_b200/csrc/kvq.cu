@@ -19,6 +19,7 @@
 namespace {
 
 constexpr int kAbiVersion = 1;
+constexpr int kMaxDevices = 64;
 
 bool bits_supported(int32_t bits) { return bits == 2 || bits == 3 || bits == 4 || bits == 8; }
 bool head_dim_supported(int32_t d) { return d >= 64 && d <= KVQ_MAX_HEAD_DIM && d % 64 == 0; }
@@ -100,7 +101,7 @@ struct AttnLaunch {
 };
 
 struct ViewChunks {
-    int32_t chunk_packed, chunk_window, n_packed, n_window;  // tokens per chunk, chunk counts
+    int32_t n_packed, n_window;  // chunks of the packed part and of the window
 };
 
 struct AttnPlan {
@@ -165,79 +166,95 @@ int attn_header_bytes(int ng) {
 int64_t packed_token_bytes(int32_t head_dim, int32_t bits) { return 2 * row_bytes(head_dim, bits) + 16 * (head_dim / 64); }
 int64_t window_token_bytes(int32_t head_dim) { return 4 * (int64_t)head_dim; }
 
-// Chunk the views of one launch so that work items carry about equal bytes
-// and the item count fills the GPU's resident CTA slots in whole waves.
-int64_t chunk_views(const kvq_view *views, int v0, int v1, int64_t units, int32_t head_dim, int64_t slots,
-                    std::vector<ViewChunks> &out) {
+// Cost model of a work item, in byte-equivalents: the bytes its tokens bring
+// in plus a fixed per-CTA cost (set-up, pipeline fill, partial merge).  A
+// launch's predicted time is its number of waves times (largest item +
+// per-CTA cost).
+constexpr double kCtaCost = 96.0 * 1024;
+constexpr double kMinItem = 16.0 * 1024, kBigItem = 512.0 * 1024;
+
+// Cost of the largest of n chunks of equal step counts over n_tok tokens.
+double largest_chunk(int64_t n_tok, int step, int64_t n, double tok_cost) {
+    if (n <= 0) return 0.0;
+    const int64_t steps = (n_tok + step - 1) / step;
+    return (double)std::min<int64_t>((steps + n - 1) / n * step, n_tok) * tok_cost;
+}
+
+// Free chunking of the views [v0, v1): each part (packed, window) of a view is
+// cut into chunks of equal step counts (+-1 step) costing about W each, W
+// picked by the smallest predicted time over whole waves of `slots` resident
+// CTAs.  Stores the chunk counts, returns the predicted time; *chunks = the
+// launch's chunk count per unit.
+double plan_free(const kvq_view *views, int v0, int v1, int64_t units, int32_t head_dim, int64_t slots,
+                 std::vector<ViewChunks> &out, int64_t *chunks) {
+    const int forced = env_int("KVQ_CHUNK_TOKENS", 0);  // tests: force a chunk length
     double total = 0;
     for (int i = v0; i < v1; ++i)
         total += (double)units * ((double)views[i].n_packed * packed_token_bytes(head_dim, views[i].bits) +
                                   (double)views[i].n_window * window_token_bytes(head_dim));
-    // items and largest item (bytes) for a target item size W
+    auto split = [&](int64_t n_tok, int step, double tok_cost, double W) -> int64_t {
+        if (n_tok <= 0) return 0;
+        const int64_t steps = (n_tok + step - 1) / step;
+        const int64_t n = forced > 0 ? (n_tok + forced - 1) / forced : std::llround((double)n_tok * tok_cost / W);
+        return std::max<int64_t>(1, std::min<int64_t>(n, steps));
+    };
     auto count = [&](double W, bool store, double *max_item) -> int64_t {
         int64_t items = 0;
         double mx = 0;
-        const int forced = env_int("KVQ_CHUNK_TOKENS", 0);
         for (int i = v0; i < v1; ++i) {
             const kvq_view &v = views[i];
-            ViewChunks c{16, 16, 0, 0};
-            const double bp = (double)packed_token_bytes(head_dim, v.bits), bw = (double)window_token_bytes(head_dim);
-            if (v.n_packed > 0) {
-                int64_t n = std::max<int64_t>(1, (int64_t)std::llround(v.n_packed * bp / W));
-                int64_t ch = (v.n_packed + n - 1) / n;
-                ch = std::max<int64_t>(128, (ch + 127) / 128 * 128);  // whole 32-token steps for 4 warps
-                c.chunk_packed = (int32_t)ch;
-                c.n_packed = (int32_t)((v.n_packed + ch - 1) / ch);
-            }
-            if (v.n_window > 0) {
-                int64_t n = std::max<int64_t>(1, (int64_t)std::llround(v.n_window * bw / W));
-                int64_t ch = (v.n_window + n - 1) / n;
-                ch = std::max<int64_t>(64, (ch + 63) / 64 * 64);  // whole 16-token steps for 4 warps
-                c.chunk_window = (int32_t)ch;
-                c.n_window = (int32_t)((v.n_window + ch - 1) / ch);
-            }
-            if (forced > 0) {
-                const int ch = std::max(32, forced / 32 * 32);
-                c.chunk_packed = c.chunk_window = ch;
-                c.n_packed = (int32_t)((v.n_packed + ch - 1) / ch);
-                c.n_window = (int32_t)((v.n_window + ch - 1) / ch);
-            }
+            const double cp = (double)packed_token_bytes(head_dim, v.bits), cw = (double)window_token_bytes(head_dim);
+            int64_t np = split(v.n_packed, 2 * kvq::kTile, cp, W), nw = split(v.n_window, kvq::kTile, cw, W);
             // the combine grid holds at most kMaxChunksPerUnit chunks per unit
-            while (c.n_packed + c.n_window > kvq::kMaxChunksPerUnit) {
-                if (c.n_packed >= c.n_window) {
-                    c.chunk_packed *= 2;
-                    c.n_packed = (int32_t)((v.n_packed + c.chunk_packed - 1) / c.chunk_packed);
-                } else {
-                    c.chunk_window *= 2;
-                    c.n_window = (int32_t)((v.n_window + c.chunk_window - 1) / c.chunk_window);
-                }
+            while (np + nw > kvq::kMaxChunksPerUnit) {
+                if (np >= nw) np = std::max<int64_t>(1, np * 3 / 4);
+                else nw = std::max<int64_t>(1, nw * 3 / 4);
             }
-            if (c.n_packed) mx = std::max(mx, std::min<double>(c.chunk_packed, v.n_packed) * bp);
-            if (c.n_window) mx = std::max(mx, std::min<double>(c.chunk_window, v.n_window) * bw);
-            items += c.n_packed + c.n_window;
-            if (store) out[i] = c;
+            mx = std::max(mx, std::max(largest_chunk(v.n_packed, 2 * kvq::kTile, np, cp),
+                                       largest_chunk(v.n_window, kvq::kTile, nw, cw)));
+            items += np + nw;
+            if (store) out[i] = ViewChunks{(int32_t)np, (int32_t)nw};
         }
         if (max_item) *max_item = mx;
-        return items;  // chunks over the views; each is run once per unit
+        return items;
     };
-    // Pick the item size with the smallest predicted makespan: whole waves of
-    // resident CTAs, each wave as long as its largest item plus a fixed
-    // per-CTA cost (set-up, pipeline fill, merge), in byte-equivalents.
-    const double kMinItem = 16.0 * 1024, kBigItem = 256.0 * 1024, kCtaCost = 96.0 * 1024;
     double best_W = std::max(kMinItem, std::min(kBigItem, total / (double)slots)), best_cost = 1e300;
-    const double fs[] = {0.6, 0.7, 0.8, 0.9, 1.0, 1.15, 1.3, 1.5, 1.75, 2.0, 2.5, 3.0, 4.0, 5.0, 6.0, 8.0, 12.0, 16.0, 24.0, 32.0};
+    const double fs[] = {0.5, 0.6, 0.7, 0.8, 0.9, 1.0, 1.15, 1.3, 1.5, 1.75, 2.0, 2.5, 3.0, 4.0,
+                         5.0, 6.0, 8.0, 12.0, 16.0, 24.0, 32.0};
     for (double f : fs) {
         const double W = std::max(kMinItem, std::min(kBigItem, total / ((double)slots * f)));
         double mx = 0;
         const int64_t items = count(W, false, &mx) * units;
-        const double waves = (double)((items + slots - 1) / slots);
-        const double cost = waves * (mx + kCtaCost);
+        const double cost = (double)((items + slots - 1) / slots) * (mx + kCtaCost);
         if (cost < best_cost * 0.999) {
             best_cost = cost;
             best_W = W;
         }
     }
-    return count(best_W, true, nullptr);
+    *chunks = count(best_W, true, nullptr);
+    return best_cost;
+}
+
+template <int NG>
+kvq_status ensure_attn_smem(size_t smem) {
+    // the attention kernel's dynamic shared-memory limit, raised once per device
+    static std::mutex mu;
+    static int configured[kMaxDevices] = {0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) {
+        (void)cudaGetLastError();
+        return KVQ_ERR_CUDA;
+    }
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev >= kMaxDevices || configured[dev] < (int)smem) {
+        if (cudaFuncSetAttribute(kvq::decode_attn_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 (int)smem) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return KVQ_ERR_CUDA;
+        }
+        if (dev < kMaxDevices) configured[dev] = (int)smem;
+    }
+    return KVQ_OK;
 }
 
 kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, int32_t n_kv_heads,
@@ -272,11 +289,12 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, 
     if (plan.smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;
 
     const int64_t slots = (int64_t)device_sm_count() * ctas;
-    plan.chunks.assign(n_views, ViewChunks{16, 16, 0, 0});
+    plan.chunks.assign(n_views, ViewChunks{0, 0});
     int64_t max_chunks = 0;
     for (int v0 = 0; v0 < n_views; v0 += kvq::kAttnMaxViews) {
         const int v1 = std::min<int>(n_views, v0 + kvq::kAttnMaxViews);
-        const int64_t chunks = chunk_views(views, v0, v1, units, head_dim, slots, plan.chunks);
+        int64_t chunks = 0;
+        plan_free(views, v0, v1, units, head_dim, slots, plan.chunks, &chunks);
         if (chunks > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
         plan.launches.push_back({v0, v1, (int)chunks});
         max_chunks = std::max(max_chunks, chunks);
@@ -290,15 +308,8 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, 
 template <int NG>
 kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n_q_heads, int32_t n_kv_heads,
                           const void *q, float scale, float *out, uint8_t *ws, cudaStream_t st) {
-    static int configured_smem[64] = {0};
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) return KVQ_ERR_CUDA;
-    if (dev >= 64 || configured_smem[dev] < (int)plan.smem) {
-        if (cudaFuncSetAttribute(kvq::decode_attn_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)plan.smem) != cudaSuccess)
-            return KVQ_ERR_CUDA;
-        if (dev < 64) configured_smem[dev] = (int)plan.smem;
-    }
+    const kvq_status es = ensure_attn_smem<NG>(plan.smem);
+    if (es != KVQ_OK) return es;
     kvq::AttnParams prm;
     std::memset(&prm, 0, sizeof prm);
     prm.q = static_cast<const uint16_t *>(q);
@@ -331,14 +342,16 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
             d.cap_window = v.cap_window;
             d.window_head = v.window_head;
             d.bits = v.n_packed > 0 ? v.bits : 4;
-            d.chunk_packed = c.chunk_packed;
-            d.chunk_window = c.chunk_window;
             d.n_chunks_packed = c.n_packed;
             d.n_chunks = c.n_packed + c.n_window;
             d.chunk_begin = begin;
             d.view_index = i;
             begin += d.n_chunks;
         }
+        // Both grids carry a programmatic dependency on the preceding work in
+        // the stream: each starts with griddepcontrol.wait, so it reads
+        // nothing before its predecessor has completed, while its launch and
+        // CTA scheduling overlap the predecessor's tail.
         // Both grids carry a programmatic dependency on the preceding work in
         // the stream: each starts with griddepcontrol.wait, so it reads
         // nothing before its predecessor has completed, while its launch and
@@ -370,7 +383,6 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
 // kvq_decode_attn workspace (status word at byte 0, partials from byte 256).
 static __device__ __align__(256) uint8_t g_noalloc_scratch[KVQ_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mutex;
 void *g_noalloc_ptr[kMaxDevices] = {};
 

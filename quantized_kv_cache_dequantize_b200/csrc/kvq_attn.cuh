@@ -58,13 +58,10 @@ struct AttnView {
     int32_t cap_window;
     int32_t window_head;
     int32_t bits;
-    int32_t chunk_packed;        // tokens per packed chunk (multiple of 16)
-    int32_t chunk_window;        // tokens per window chunk (multiple of 16)
-    int32_t n_chunks_packed;
-    int32_t n_chunks;            // packed + window chunks
+    int32_t n_chunks_packed;     // the packed part's 32-token steps, split evenly
+    int32_t n_chunks;            // packed + window chunks (window: 16-token steps)
     int32_t chunk_begin;         // first chunk index of this view in the launch
     int32_t view_index;          // row of q / out
-    int32_t pad_;
 };
 
 struct AttnParams {
@@ -557,10 +554,16 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     const int gid = lane >> 2, tig = lane & 3;
     const int h0 = hk * p.group + z * kHeadsPerCta;
     const int nh = min(kHeadsPerCta, p.group - z * kHeadsPerCta);
-    const int chunk = WINDOW ? V.chunk_window : V.chunk_packed;
-    const int64_t tok0 = (int64_t)(WINDOW ? c - V.n_chunks_packed : c) * chunk;
-    const int n_tok = (int)min((int64_t)chunk, (WINDOW ? (int64_t)V.n_window : (int64_t)V.n_packed) - tok0);
-    const int n_steps = (n_tok + kStepTok - 1) / kStepTok;
+    // this chunk's steps: the part's steps split into equal runs (+-1 step)
+    const int n_part = WINDOW ? V.n_window : V.n_packed;
+    const int steps_part = (n_part + kStepTok - 1) / kStepTok;
+    const int chunks_part = WINDOW ? V.n_chunks - V.n_chunks_packed : V.n_chunks_packed;
+    const int ci = WINDOW ? c - V.n_chunks_packed : c;
+    const int s0 = (int)((int64_t)ci * steps_part / chunks_part);
+    const int s1 = (int)((int64_t)(ci + 1) * steps_part / chunks_part);
+    const int64_t tok0 = (int64_t)s0 * kStepTok;
+    const int n_tok = (int)min((int64_t)(s1 - s0) * kStepTok, (int64_t)n_part - tok0);
+    const int n_steps = s1 - s0;
     const int n_my = (warp < n_steps) ? (n_steps - warp + kAttnWarps - 1) / kAttnWarps : 0;
     const int n_blocks = kBlkPerStep * n_my;
     const int S = min(kMaxStages, (int)(p.ring_bytes / kBlk));
@@ -819,10 +822,10 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         if (single) {
             p.out[((int64_t)V.view_index * p.n_q_heads + h0 + j) * D + d] = O / L;
         } else {
-            part[j * (D + 2) + d] = O;
+            part[j * D + d] = O;
             if (d == 0) {
-                part[j * (D + 2) + D] = M;
-                part[j * (D + 2) + D + 1] = L;
+                part[kHeadsPerCta * D + j] = M;
+                part[kHeadsPerCta * D + kHeadsPerCta + j] = L;
             }
         }
     }
@@ -858,14 +861,17 @@ __global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
 }
 
 // Split-K combine: one CTA per (view, KV head, head block) with more than one
-// chunk.  Gathers every chunk's (m, l) per head in one pass, reduces per head
-// with warp shuffles, and sums the chunk partials in chunk order (loads 8
-// deep), so results are bitwise reproducible.  Launched right after the
-// attention grid with a programmatic dependency: it is scheduled while the
-// attention tail runs and waits for that grid's completion before reading.
+// chunk.  A chunk's partial is [O: 8 heads x D][m: 8][l: 8] floats.  The CTA
+// gathers every chunk's (m, l), reduces per head with warp shuffles, then sums
+// the chunks' O in chunk order, 4 elements per thread and 8 chunks per batch
+// of independent loads, so results are bitwise reproducible and the loads of a
+// batch overlap.  Launched right after the attention grid with a programmatic
+// dependency: it is scheduled while the attention tail runs and waits for that
+// grid's completion before reading.
 template <int NG>
 __global__ void __launch_bounds__(kAttnThreads) combine_kernel(const __grid_constant__ AttnParams p) {
     constexpr int D = 64 * NG;
+    constexpr int kSlot = kHeadsPerCta * (D + 2);  // floats per partial
     __shared__ float sm_w[kMaxChunksPerUnit * kHeadsPerCta];  // m, then weight
     __shared__ float sm_l[kMaxChunksPerUnit * kHeadsPerCta];
     __shared__ float sm_L[kHeadsPerCta];
@@ -878,13 +884,13 @@ __global__ void __launch_bounds__(kAttnThreads) combine_kernel(const __grid_cons
     const int h0 = hk * p.group + z * kHeadsPerCta;
     const int nh = min(kHeadsPerCta, p.group - z * kHeadsPerCta);
     const int64_t slot0 = ((int64_t)V.chunk_begin * p.n_kv_heads + hk) * p.head_blocks + z;
-    const int64_t slot_stride = (int64_t)p.n_kv_heads * p.head_blocks * (kHeadsPerCta * (D + 2));
-    const float *part0 = p.partials + slot0 * (kHeadsPerCta * (D + 2));
+    const int64_t stride = (int64_t)p.n_kv_heads * p.head_blocks * kSlot;  // between chunks
+    const float *part0 = p.partials + slot0 * kSlot;
     for (int i = tid; i < n * nh; i += kAttnThreads) {
         const int cc = i / nh, j = i - cc * nh;
-        const float *pc = part0 + cc * slot_stride + j * (D + 2);
-        sm_w[cc * kHeadsPerCta + j] = __ldcg(pc + D);
-        sm_l[cc * kHeadsPerCta + j] = __ldcg(pc + D + 1);
+        const float *pc = part0 + cc * stride + kHeadsPerCta * D;
+        sm_w[cc * kHeadsPerCta + j] = __ldcg(pc + j);
+        sm_l[cc * kHeadsPerCta + j] = __ldcg(pc + kHeadsPerCta + j);
     }
     __syncthreads();
     for (int j = warp; j < nh; j += kAttnWarps) {
@@ -904,20 +910,31 @@ __global__ void __launch_bounds__(kAttnThreads) combine_kernel(const __grid_cons
         if (lane == 0) sm_L[j] = L;
     }
     __syncthreads();
-    for (int idx = tid; idx < nh * D; idx += kAttnThreads) {
-        const int j = idx / D, d = idx - j * D;
-        const float *pj = part0 + j * (D + 2) + d;
-        float O = 0.f;
-        int cc = 0;
-        for (; cc + 8 <= n; cc += 8) {
-            float v[8];
+    const float4 *o4 = reinterpret_cast<const float4 *>(part0);
+    const int64_t stride4 = stride / 4;
+    float4 *out4 = reinterpret_cast<float4 *>(p.out + ((int64_t)V.view_index * p.n_q_heads + h0) * D);
+    for (int f = tid; f < nh * (D / 4); f += kAttnThreads) {
+        const int j = f / (D / 4);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c0 = 0; c0 < n; c0 += 8) {
+            float4 v[8];
+            float w[8];
 #pragma unroll
-            for (int u = 0; u < 8; ++u) v[u] = __ldcg(pj + (cc + u) * slot_stride);
+            for (int u = 0; u < 8; ++u) {
+                const bool ok = c0 + u < n;
+                v[u] = ok ? __ldcg(o4 + (c0 + u) * stride4 + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+                w[u] = ok ? sm_w[(c0 + u) * kHeadsPerCta + j] : 0.f;
+            }
 #pragma unroll
-            for (int u = 0; u < 8; ++u) O = fmaf(sm_w[(cc + u) * kHeadsPerCta + j], v[u], O);
+            for (int u = 0; u < 8; ++u) {
+                acc.x = fmaf(w[u], v[u].x, acc.x);
+                acc.y = fmaf(w[u], v[u].y, acc.y);
+                acc.z = fmaf(w[u], v[u].z, acc.z);
+                acc.w = fmaf(w[u], v[u].w, acc.w);
+            }
         }
-        for (; cc < n; ++cc) O = fmaf(sm_w[cc * kHeadsPerCta + j], __ldcg(pj + cc * slot_stride), O);
-        p.out[((int64_t)V.view_index * p.n_q_heads + h0 + j) * D + d] = O / sm_L[j];
+        const float L = sm_L[j];
+        out4[f] = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
     }
 }
 

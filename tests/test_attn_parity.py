@@ -99,7 +99,6 @@ def test_chunking_changes_only_rounding(cuda_device, monkeypatch):
         for i in range(2):
             assert_close(out[i], ref[i], f"chunk {chunk}")
         outs.append(out)
-    assert not all(np.array_equal(outs[0], o) for o in outs[1:]) or True
 
 
 def test_bitwise_deterministic(cuda_device):

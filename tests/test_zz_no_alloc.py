@@ -59,18 +59,20 @@ def test_two_calls_in_a_row_match_workspace_path(cuda_device):
         assert_close(again[i], ref_a[i], f"noalloc call 3, view {i}")
 
 
-def test_rejects_plans_beyond_the_scratch_array(cuda_device):
-    # 64 views x 32768 packed tokens (8 kv heads, D 128) plan about 43 MiB of
-    # partials: more than the array holds
+def test_rejects_plans_beyond_the_scratch_array(cuda_device, monkeypatch):
+    # 16 views x 32768 packed tokens (8 kv heads, D 128) cut into 128-token
+    # chunks merged through the workspace: about 69 MiB of partials, more than
+    # the array holds
+    monkeypatch.setenv("KVQ_CHUNK_TOKENS", "128")
     views = []
-    for i in range(64):
+    for i in range(16):
         v = kvq.View(8, 128, 4, 32768, 128, device=cuda_device)
         v.set_state(32768, 128)
         views.append(v)
     need = kvq.workspace_size(views, 32)
     assert need > kvq.NOALLOC_SCRATCH_BYTES
-    q = torch.zeros((64, 32, 128), dtype=torch.bfloat16, device=cuda_device)
-    out = torch.full((64, 32, 128), 7.0, dtype=torch.float32, device=cuda_device)
+    q = torch.zeros((16, 32, 128), dtype=torch.bfloat16, device=cuda_device)
+    out = torch.full((16, 32, 128), 7.0, dtype=torch.float32, device=cuda_device)
     with pytest.raises(kvq.KvqError) as e:
         kvq.decode_attn_noalloc(views, q, 1 / math.sqrt(128), out)
     assert e.value.status == kvq.KVQ_ERR_CAPACITY
