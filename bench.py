@@ -4,11 +4,11 @@
 Workload (one step = one decode token for every agent): 10 agents x 32 layers
 in Llama-3.1-8B shape (32 query / 8 KV heads, head_dim 128), each (agent,
 layer) view holding 4096 packed 4-bit tokens plus a full 128-token bf16 recent
-window.  Per layer the step runs kvq_append (the new token enters the window;
-the oldest window token is quantized into the packed part) and then
-kvq_decode_attn over the 10 agents' views of that layer; the 64 calls of a
-step are replayed from one CUDA graph.  The per-step working set (~1.9 GB) is
-far larger than L2, so no flush is needed between steps.
+window.  Per layer the step runs kvq_append_decode_attn over the 10 agents'
+views of that layer: the new token enters the window, the oldest window token
+is quantized into the packed part, and attention runs over the result; the 32
+calls of a step are replayed from one CUDA graph.  The per-step working set
+(~1.9 GB) is far larger than L2, so no flush is needed between steps.
 
 Also measured in the same run: the bulk handoff codec (quantize then
 dequantize one agent's 32-layer x 8-head x 32768-token x 128 K and V cache,
@@ -235,6 +235,8 @@ def run_ours(args, rank, world, local):
     out = torch.empty((L * A, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
     layer_views = [views[l * A:(l + 1) * A] for l in range(L)]
     ws = [kvq.new_workspace(lv, w.n_q_heads, device=dev) for lv in layer_views]
+    ws_step = [torch.zeros(kvq.step_workspace_size(lv, w.n_q_heads), dtype=torch.uint8, device=dev)
+               for lv in layer_views]
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream()
@@ -244,10 +246,11 @@ def run_ours(args, rank, world, local):
     n_launch_per_step = 3 * L
 
     def step():
+        # one decode step per layer: append this token, attend over the result
         for l in range(L):
-            kvq.append(layer_views[l], kn[l * A:(l + 1) * A], vn[l * A:(l + 1) * A], stream=stream)
-            kvq.decode_attn(layer_views[l], q[l * A:(l + 1) * A], w.softmax_scale,
-                            out=out[l * A:(l + 1) * A], workspace=ws[l], stream=stream)
+            kvq.append_decode_attn(layer_views[l], kn[l * A:(l + 1) * A], vn[l * A:(l + 1) * A],
+                                   q[l * A:(l + 1) * A], w.softmax_scale, out=out[l * A:(l + 1) * A],
+                                   workspace=ws_step[l], stream=stream)
 
     # capture one step in a graph; host view counters advance at capture, so
     # the graph replays the same (full-window) append + attend each time
@@ -338,7 +341,7 @@ def run_ours(args, rank, world, local):
     t_e2e = kdist.max_over_ranks(c0.elapsed_time(c1) / 1e3 / args.steps)
     e2e_gbs = kdist.aggregate_throughput(bytes_step, world, t_e2e) / 1e9
 
-    del pool, ws, ws_all, q, out
+    del pool, ws, ws_step, ws_all, q, out
     torch.cuda.empty_cache()
 
     # ---------------- bulk handoff codec (quantize then dequantize), 4-bit
@@ -403,7 +406,7 @@ def run_ours(args, rank, world, local):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": WORKLOAD, "agents_per_gpu": A, "layers": L, "n_q_heads": w.n_q_heads,
                        "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "packed_tokens": w.view_len(0),
-                       "window": w.window, "bits": 4, "calls_per_step": "per layer: kvq_append + kvq_decode_attn",
+                       "window": w.window, "bits": 4, "calls_per_step": "per layer: kvq_append_decode_attn (append, attention and combine grids)",
                        "cuda_graph": True, "l2": "working set per step ~1.9 GB > 126 MB L2, no flush"},
             "tokens_per_s_per_agent": 1.0 / t_step,
             "hbm_frac": value / world / peak,

@@ -202,6 +202,31 @@ kvq_status kvq_decode_attn(const kvq_view *views, int32_t n_views, int32_t n_q_h
                            float softmax_scale, float *out, void *workspace,
                            size_t workspace_bytes, void *stream);
 
+/*
+ * kvq_append_decode_attn -- one decode step over a batch of views: the
+ * effect of kvq_append(views, ..., k_new, v_new) followed by
+ * kvq_decode_attn(views, ...) on the appended views, in one call (CoMixKV,
+ * Abstract: recent states stay native, only flushed blocks are quantized;
+ * Agent Memory, Abstract: attention straight over the quantized caches).
+ *
+ * Arguments as in those two calls; the workspace is sized by
+ * kvq_decode_attn_workspace_size on the views as they will be after the
+ * append (each view's counters advanced by one token).  The attention grid is
+ * launched right behind the append grid and every one of its copies starts at
+ * once except the copy of the block holding a row the append writes (the
+ * flushed packed row, the new window token), which waits for the append grid
+ * first; results and cache contents are the same as with the two calls.
+ * Errors: those of kvq_append (nothing enqueued, no counter changed) and of
+ * kvq_decode_attn's argument checks, all before anything is enqueued;
+ * KVQ_ERR_CUDA if a launch fails (the counters are advanced once the append
+ * is enqueued).
+ */
+kvq_status kvq_append_decode_attn(kvq_view *views, int32_t n_views, int32_t n_q_heads,
+                                  int32_t n_kv_heads, int32_t head_dim, const void *k_new,
+                                  const void *v_new, const void *q, float softmax_scale,
+                                  float *out, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
 /* Bytes of the per-device scratch array kvq_decode_attn_noalloc uses. */
 #define KVQ_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 

@@ -10,6 +10,7 @@ Entry points (same names as the C ABI, without the ``kvq_`` prefix):
   quantize, dequantize          -- bf16 rows <-> packed b-bit codes + {s, mn}
   View, append                  -- one (agent, layer) cache; add a decode token
   decode_attn, workspace_size   -- batched split-K attention over many views
+  append_decode_attn            -- one decode step: append, then attend, in one call
   decode_attn_noalloc           -- the same without a workspace: scratch is a
                                    fixed per-device array inside the library
                                    (NOALLOC_SCRATCH_BYTES), for callers that
@@ -25,7 +26,7 @@ import torch
 from . import workloads  # noqa: F401  (seeded input generators)
 
 __all__ = ["quantize", "dequantize", "View", "append", "decode_attn", "workspace_size",
-           "decode_attn_noalloc", "NOALLOC_SCRATCH_BYTES", "KvqError", "lib", "row_bytes", "GROUP"]
+           "append_decode_attn", "step_workspace_size", "decode_attn_noalloc", "NOALLOC_SCRATCH_BYTES", "KvqError", "lib", "row_bytes", "GROUP"]
 
 GROUP = 64
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024   # KVQ_NOALLOC_SCRATCH_BYTES in kvq.h
@@ -76,6 +77,8 @@ def lib():
         L.kvq_decode_attn_workspace_size.restype = sz
         L.kvq_decode_attn.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, f32, P, P, sz, P]
         L.kvq_decode_attn.restype = i32
+        L.kvq_append_decode_attn.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, P, P, f32, P, P, sz, P]
+        L.kvq_append_decode_attn.restype = i32
         L.kvq_decode_attn_noalloc.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, f32, P, P]
         L.kvq_decode_attn_noalloc.restype = i32
         _lib = L
@@ -261,6 +264,55 @@ def decode_attn(views, q: torch.Tensor, softmax_scale: float, out: torch.Tensor 
     _check(lib().kvq_decode_attn(arr, len(views), Hq, views[0].n_kv_heads, D, _ptr(q), float(softmax_scale),
                                  _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
            "kvq_decode_attn")
+    return out
+
+
+def _advanced(c: CView) -> CView:
+    """A copy of a view's C struct with the counters one append later."""
+    n = CView()
+    ctypes.pointer(n)[0] = c
+    if n.cap_window == 0:
+        n.n_packed += 1
+    elif n.n_window == n.cap_window:
+        n.n_packed += 1
+        n.window_head = (n.window_head + 1) % n.cap_window
+    else:
+        n.n_window += 1
+    return n
+
+
+def step_workspace_size(views, n_q_heads: int) -> int:
+    """Workspace bytes append_decode_attn needs: kvq_decode_attn_workspace_size
+    on the views as they will be after the append."""
+    views = list(views)
+    arr = (CView * len(views))()
+    for i, v in enumerate(views):
+        arr[i] = _advanced(v.c)
+    return int(lib().kvq_decode_attn_workspace_size(arr, len(views), n_q_heads, views[0].n_kv_heads,
+                                                    views[0].head_dim))
+
+
+def append_decode_attn(views, k_new: torch.Tensor, v_new: torch.Tensor, q: torch.Tensor, softmax_scale: float,
+                       out: torch.Tensor | None = None, workspace: torch.Tensor | None = None,
+                       stream=None) -> torch.Tensor:
+    """One decode step (kvq_append_decode_attn): append k_new, v_new (bf16
+    [n_views, H_kv, D]) to the views, then attend with q (bf16 [n_views, H_q,
+    D]) over the appended views; returns fp32 [n_views, H_q, D]."""
+    views = list(views)
+    n, Hq, D = q.shape
+    if workspace is None:
+        # 0 when the step is invalid: the call below then reports why
+        nb = step_workspace_size(views, Hq)
+        workspace = torch.zeros(nb, dtype=torch.uint8, device=q.device) if nb else None
+    if out is None:
+        out = torch.empty((n, Hq, D), dtype=torch.float32, device=q.device)
+    arr = _view_array(views)
+    _check(lib().kvq_append_decode_attn(arr, len(views), Hq, views[0].n_kv_heads, D, _ptr(k_new), _ptr(v_new),
+                                        _ptr(q), float(softmax_scale), _ptr(out), _ptr(workspace),
+                                        workspace.numel() if workspace is not None else 0, _stream(stream)),
+           "kvq_append_decode_attn")
+    for i, v in enumerate(views):
+        v.c.n_packed, v.c.n_window, v.c.window_head = arr[i].n_packed, arr[i].n_window, arr[i].window_head
     return out
 
 

@@ -307,7 +307,8 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, 
 
 template <int NG>
 kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n_q_heads, int32_t n_kv_heads,
-                          const void *q, float scale, float *out, uint8_t *ws, cudaStream_t st) {
+                          const void *q, float scale, float *out, uint8_t *ws, cudaStream_t st,
+                          const int32_t *dep = nullptr) {
     const kvq_status es = ensure_attn_smem<NG>(plan.smem);
     if (es != KVQ_OK) return es;
     kvq::AttnParams prm;
@@ -325,6 +326,9 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
     prm.ring_bytes = plan.ring_bytes;
     for (const AttnLaunch &L : plan.launches) {
         prm.n_views = L.v1 - L.v0;
+        // Right behind a fused append only the first launch skips the entry
+        // wait (later ones follow this call's own grids).
+        prm.fused = (dep != nullptr && L.v0 == 0) ? 1 : 0;
         int begin = 0;
         for (int i = L.v0; i < L.v1; ++i) {
             const kvq_view &v = views[i];
@@ -346,6 +350,8 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
             d.n_chunks = c.n_packed + c.n_window;
             d.chunk_begin = begin;
             d.view_index = i;
+            d.dep_step[0] = prm.fused ? dep[2 * i] : -1;
+            d.dep_step[1] = prm.fused ? dep[2 * i + 1] : -1;
             begin += d.n_chunks;
         }
         // Both grids carry a programmatic dependency on the preceding work in
@@ -375,6 +381,98 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
         }
     }
     return KVQ_OK;
+}
+
+// ------------------------------------------------------------- append ---
+
+kvq_status validate_append(const kvq_view *views, int32_t n_views, int32_t n_kv_heads, int32_t head_dim,
+                           const void *k_new, const void *v_new) {
+    if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
+    if (n_kv_heads <= 0 || n_kv_heads > 65535) return KVQ_ERR_INVALID_ARG;
+    const kvq_status vs = validate_views(views, n_views, false);
+    if (vs != KVQ_OK) return vs;
+    if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return KVQ_ERR_INVALID_ARG;
+    // every view must be able to take the token
+    for (int i = 0; i < n_views; ++i) {
+        const kvq_view &v = views[i];
+        const bool flush = v.cap_window == 0 || v.n_window == v.cap_window;
+        if (flush) {
+            if (!bits_supported(v.bits)) return KVQ_ERR_UNSUPPORTED;
+            if (v.n_packed >= v.cap_packed) return KVQ_ERR_CAPACITY;
+        }
+    }
+    return KVQ_OK;
+}
+
+// Enqueue the append grids (validated arguments); host counters unchanged.
+kvq_status launch_append(const kvq_view *views, int32_t n_views, int32_t n_kv_heads, int32_t head_dim,
+                         const void *k_new, const void *v_new, cudaStream_t st) {
+    const int ng = head_dim / 64;
+    for (int v0 = 0; v0 < n_views; v0 += kvq::kAppendMaxViews) {
+        const int v1 = std::min<int>(n_views, v0 + kvq::kAppendMaxViews);
+        kvq::AppendArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.k_new = static_cast<const uint16_t *>(k_new) + (int64_t)v0 * n_kv_heads * head_dim;
+        a.v_new = static_cast<const uint16_t *>(v_new) + (int64_t)v0 * n_kv_heads * head_dim;
+        a.n_views = v1 - v0;
+        a.n_kv_heads = n_kv_heads;
+        for (int i = v0; i < v1; ++i) {
+            const kvq_view &v = views[i];
+            kvq::AppendView &d = a.views[i - v0];
+            d.codes[0] = static_cast<uint8_t *>(v.k_codes);
+            d.codes[1] = static_cast<uint8_t *>(v.v_codes);
+            d.scalemin[0] = v.k_scalemin;
+            d.scalemin[1] = v.v_scalemin;
+            d.window[0] = static_cast<uint16_t *>(v.k_window);
+            d.window[1] = static_cast<uint16_t *>(v.v_window);
+            d.cap_packed = v.cap_packed;
+            d.cap_window = v.cap_window;
+            d.bits = v.bits;
+            d.packed_row = v.n_packed;
+            if (v.cap_window == 0) {
+                d.flush = 1;
+                d.slot = -1;
+            } else if (v.n_window == v.cap_window) {
+                d.flush = 1;
+                d.slot = v.window_head;
+            } else {
+                d.flush = 0;
+                d.slot = (v.window_head + v.n_window) % v.cap_window;
+            }
+        }
+        // programmatic dependency: the kernel starts with griddepcontrol.wait
+        cudaLaunchAttribute attr;
+        attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr.val.programmaticStreamSerializationAllowed = 1;
+        cudaLaunchConfig_t cfg;
+        std::memset(&cfg, 0, sizeof cfg);
+        cfg.gridDim = dim3((unsigned)(v1 - v0), (unsigned)n_kv_heads, 2);
+        cfg.blockDim = dim3(32);
+        cfg.stream = st;
+        cfg.attrs = &attr;
+        cfg.numAttrs = 1;
+        cudaError_t e;
+        switch (ng) {
+            case 1: e = cudaLaunchKernelEx(&cfg, kvq::append_kernel<1>, a); break;
+            case 2: e = cudaLaunchKernelEx(&cfg, kvq::append_kernel<2>, a); break;
+            case 3: e = cudaLaunchKernelEx(&cfg, kvq::append_kernel<3>, a); break;
+            default: e = cudaLaunchKernelEx(&cfg, kvq::append_kernel<4>, a); break;
+        }
+        if (e != cudaSuccess) return KVQ_ERR_CUDA;
+    }
+    return KVQ_OK;
+}
+
+// A view's counters after one append.
+void advance_view(kvq_view &v) {
+    if (v.cap_window == 0) {
+        v.n_packed += 1;
+    } else if (v.n_window == v.cap_window) {
+        v.n_packed += 1;
+        v.window_head = (v.window_head + 1) % v.cap_window;
+    } else {
+        v.n_window += 1;
+    }
 }
 
 // ------------------------------------------- fixed scratch (no allocation) ---
@@ -450,75 +548,13 @@ KVQ_API kvq_status kvq_dequantize(const void *codes, const float *scalemin, int6
 
 KVQ_API kvq_status kvq_append(kvq_view *views, int32_t n_views, int32_t n_kv_heads, int32_t head_dim,
                               const void *k_new, const void *v_new, void *stream) {
-    if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
-    if (n_kv_heads <= 0 || n_kv_heads > 65535) return KVQ_ERR_INVALID_ARG;
-    const kvq_status vs = validate_views(views, n_views, false);
+    const kvq_status vs = validate_append(views, n_views, n_kv_heads, head_dim, k_new, v_new);
     if (vs != KVQ_OK) return vs;
-    if (!k_new || !v_new || !aligned(k_new, 16) || !aligned(v_new, 16)) return KVQ_ERR_INVALID_ARG;
-    // first pass: every view must be able to take the token
-    for (int i = 0; i < n_views; ++i) {
-        const kvq_view &v = views[i];
-        const bool flush = v.cap_window == 0 || v.n_window == v.cap_window;
-        if (flush) {
-            if (!bits_supported(v.bits)) return KVQ_ERR_UNSUPPORTED;
-            if (v.n_packed >= v.cap_packed) return KVQ_ERR_CAPACITY;
-        }
-    }
-    cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const int ng = head_dim / 64;
-    for (int v0 = 0; v0 < n_views; v0 += kvq::kAppendMaxViews) {
-        const int v1 = std::min<int>(n_views, v0 + kvq::kAppendMaxViews);
-        kvq::AppendArgs a;
-        std::memset(&a, 0, sizeof a);
-        a.k_new = static_cast<const uint16_t *>(k_new) + (int64_t)v0 * n_kv_heads * head_dim;
-        a.v_new = static_cast<const uint16_t *>(v_new) + (int64_t)v0 * n_kv_heads * head_dim;
-        a.n_views = v1 - v0;
-        a.n_kv_heads = n_kv_heads;
-        for (int i = v0; i < v1; ++i) {
-            const kvq_view &v = views[i];
-            kvq::AppendView &d = a.views[i - v0];
-            d.codes[0] = static_cast<uint8_t *>(v.k_codes);
-            d.codes[1] = static_cast<uint8_t *>(v.v_codes);
-            d.scalemin[0] = v.k_scalemin;
-            d.scalemin[1] = v.v_scalemin;
-            d.window[0] = static_cast<uint16_t *>(v.k_window);
-            d.window[1] = static_cast<uint16_t *>(v.v_window);
-            d.cap_packed = v.cap_packed;
-            d.cap_window = v.cap_window;
-            d.bits = v.bits;
-            d.packed_row = v.n_packed;
-            if (v.cap_window == 0) {
-                d.flush = 1;
-                d.slot = -1;
-            } else if (v.n_window == v.cap_window) {
-                d.flush = 1;
-                d.slot = v.window_head;
-            } else {
-                d.flush = 0;
-                d.slot = (v.window_head + v.n_window) % v.cap_window;
-            }
-        }
-        dim3 grid((unsigned)(v1 - v0), (unsigned)n_kv_heads, 2);
-        switch (ng) {
-            case 1: kvq::append_kernel<1><<<grid, 32, 0, st>>>(a); break;
-            case 2: kvq::append_kernel<2><<<grid, 32, 0, st>>>(a); break;
-            case 3: kvq::append_kernel<3><<<grid, 32, 0, st>>>(a); break;
-            default: kvq::append_kernel<4><<<grid, 32, 0, st>>>(a); break;
-        }
-        if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
-    }
+    const kvq_status ls =
+        launch_append(views, n_views, n_kv_heads, head_dim, k_new, v_new, static_cast<cudaStream_t>(stream));
+    if (ls != KVQ_OK) return ls;
     // the launch is enqueued: advance the host-side counters
-    for (int i = 0; i < n_views; ++i) {
-        kvq_view &v = views[i];
-        if (v.cap_window == 0) {
-            v.n_packed += 1;
-        } else if (v.n_window == v.cap_window) {
-            v.n_packed += 1;
-            v.window_head = (v.window_head + 1) % v.cap_window;
-        } else {
-            v.n_window += 1;
-        }
-    }
+    for (int i = 0; i < n_views; ++i) advance_view(views[i]);
     return KVQ_OK;
 }
 
@@ -565,4 +601,40 @@ KVQ_API kvq_status kvq_decode_attn_noalloc(const kvq_view *views, int32_t n_view
     if (cudaMemsetAsync(scratch, 0, sizeof(uint32_t), st) != cudaSuccess) return KVQ_ERR_CUDA;
     return launch_attn(plan, views, n_q_heads, n_kv_heads, head_dim, q, softmax_scale, out,
                        static_cast<uint8_t *>(scratch), st);
+}
+
+KVQ_API kvq_status kvq_append_decode_attn(kvq_view *views, int32_t n_views, int32_t n_q_heads, int32_t n_kv_heads,
+                                          int32_t head_dim, const void *k_new, const void *v_new, const void *q,
+                                          float softmax_scale, float *out, void *workspace, size_t workspace_bytes,
+                                          void *stream) {
+    const kvq_status vs = validate_append(views, n_views, n_kv_heads, head_dim, k_new, v_new);
+    if (vs != KVQ_OK) return vs;
+    // plan the attention over the views as they will be after the append
+    std::vector<kvq_view> post(views, views + n_views);
+    for (kvq_view &v : post) advance_view(v);
+    AttnPlan plan;
+    const kvq_status ps = plan_attn(post.data(), n_views, n_q_heads, n_kv_heads, head_dim, plan);
+    if (ps != KVQ_OK) return ps;
+    if (!q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
+    if (workspace_bytes < plan.total) return KVQ_ERR_INVALID_ARG;
+    // the steps whose rows the append writes: the flushed packed row, the new window token
+    std::vector<int32_t> dep(2 * (size_t)n_views);
+    for (int i = 0; i < n_views; ++i) {
+        const kvq_view &a = views[i], &b = post[i];
+        const bool flush = a.cap_window == 0 || a.n_window == a.cap_window;
+        dep[2 * i] = flush ? (int32_t)((b.n_packed - 1) / (2 * kvq::kTile)) : -1;
+        dep[2 * i + 1] = a.cap_window > 0 ? (b.n_window - 1) / kvq::kTile : -1;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const kvq_status ls = launch_append(views, n_views, n_kv_heads, head_dim, k_new, v_new, st);
+    if (ls != KVQ_OK) return ls;
+    for (int i = 0; i < n_views; ++i) views[i] = post[i];  // enqueued: advance the counters
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    switch (head_dim / 64) {
+        case 1: return launch_attn_ng<1>(plan, post.data(), n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st, dep.data());
+        case 2: return launch_attn_ng<2>(plan, post.data(), n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st, dep.data());
+        case 3: return launch_attn_ng<3>(plan, post.data(), n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st, dep.data());
+        default: return launch_attn_ng<4>(plan, post.data(), n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st, dep.data());
+    }
 }

@@ -62,6 +62,9 @@ struct AttnView {
     int32_t n_chunks;            // packed + window chunks (window: 16-token steps)
     int32_t chunk_begin;         // first chunk index of this view in the launch
     int32_t view_index;          // row of q / out
+    int32_t dep_step[2];         // packed / window step whose rows the preceding append grid
+                                 // writes (-1: none); with AttnParams::fused its copy waits
+                                 // for that grid, every other copy starts at once
 };
 
 struct AttnParams {
@@ -77,7 +80,7 @@ struct AttnParams {
     int32_t group;               // n_q_heads / n_kv_heads
     int32_t head_blocks;         // ceil(group / 8)
     int32_t ring_bytes;          // shared-memory ring per warp
-    int32_t pad_;
+    int32_t fused;               // 1: launched right behind this step's append grid (see dep_step)
     AttnView views[kAttnMaxViews];
 };
 
@@ -289,23 +292,37 @@ struct WarpState {
 // The running max is only moved when a tile exceeds it by more than
 // kLazyMax (log2 units): probabilities relative to a stale max stay below
 // 2^kLazyMax, harmless in fp32 sums and bf16 hi/lo operands, and the O rescale
-// (32+ multiplies) becomes rare instead of firing on most early tiles.
+// (32+ multiplies) becomes rare instead of firing on most early tiles.  One
+// warp vote decides whether any lane's rows exceed it; only then are the
+// per-head maxima reduced across the warp (most tiles skip the shuffles).
 constexpr float kLazyMax = 8.0f;
 
 template <int NG, int R>
 __device__ __forceinline__ void softmax_step_n(WarpState<NG> &st, float (&lg)[R][2]) {
-    float alpha[2];
+    float alpha[2] = {1.f, 1.f};
+    float tl[2];
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
-        float t = lg[0][j];
+        tl[j] = lg[0][j];
 #pragma unroll
-        for (int r = 1; r < R; ++r) t = fmaxf(t, lg[r][j]);
-        t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 4));
-        t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 8));
-        t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 16));
-        const float mnew = (t > st.m[j] + kLazyMax) ? t : st.m[j];
-        alpha[j] = fast_exp2(st.m[j] - mnew);
-        st.m[j] = mnew;
+        for (int r = 1; r < R; ++r) tl[j] = fmaxf(tl[j], lg[r][j]);
+    }
+    const bool move = __any_sync(0xFFFFFFFFu, tl[0] > st.m[0] + kLazyMax || tl[1] > st.m[1] + kLazyMax);
+    if (move) {
+#pragma unroll
+        for (int j = 0; j < 2; ++j) {
+            float t = tl[j];
+            t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 4));
+            t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 8));
+            t = fmaxf(t, __shfl_xor_sync(0xFFFFFFFFu, t, 16));
+            const float mnew = (t > st.m[j] + kLazyMax) ? t : st.m[j];
+            alpha[j] = fast_exp2(st.m[j] - mnew);
+            st.m[j] = mnew;
+        }
+    }
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+        const float mnew = st.m[j];
         float sum = 0.f;
 #pragma unroll
         for (int r = 0; r < R; ++r) {
@@ -314,7 +331,7 @@ __device__ __forceinline__ void softmax_step_n(WarpState<NG> &st, float (&lg)[R]
         }
         st.l[j] = fmaf(st.l[j], alpha[j], sum);
     }
-    if (__any_sync(0xFFFFFFFFu, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
+    if (move && __any_sync(0xFFFFFFFFu, alpha[0] != 1.0f || alpha[1] != 1.0f)) {
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
 #pragma unroll
@@ -589,7 +606,11 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         win_phys = V.cap_window > 0 ? (int)(((int64_t)V.window_head + tok0 + kStepTok * warp) % V.cap_window) : 0;
     }
     int issue_blk = 0, issue_slot = 0, issue_left = n_tok - kStepTok * warp;  // lane 0's view
+    int issue_step = s0 + warp;  // step index within the part
+    const int dep_step = p.fused ? V.dep_step[WINDOW ? 1 : 0] : -1;
     auto issue_next = [&]() {
+        // the block the preceding append grid writes: wait for that grid first
+        if (issue_step == dep_step && (!WINDOW || (issue_blk & 1) == 0)) pdl_wait();
         uint8_t *dst = ring + (size_t)issue_slot * kBlk;
         uint64_t *bar = &wbar[issue_slot];
         const int n = min(kStepTok, issue_left);
@@ -607,6 +628,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             src_ks += (int64_t)kAdvTok * NG * 2;
             src_vs += (int64_t)kAdvTok * NG * 2;
             issue_left -= kAdvTok;
+            issue_step += kAttnWarps;
         } else {
             const int kv = issue_blk & 1;
             const uint16_t *base = kv ? win_v : win_k;
@@ -617,6 +639,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             if (kv == 1) {
                 win_phys = (win_phys + kAdvTok) % V.cap_window;
                 issue_left -= kAdvTok;
+                issue_step += kAttnWarps;
             }
         }
         ++issue_blk;
@@ -633,7 +656,8 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     for (int i = tid; i < kHeadsPerCta * D / 8; i += kAttnThreads) {
         const int j = i / (D / 8), d8 = i - j * (D / 8);
         uint4 val = make_uint4(0, 0, 0, 0);
-        if (j < nh) val = reinterpret_cast<const uint4 *>(p.q + ((int64_t)V.view_index * p.n_q_heads + h0 + j) * D)[d8];
+        // L2 loads: with a fused append this CTA may not have waited for the grids before
+        if (j < nh) val = __ldcg(reinterpret_cast<const uint4 *>(p.q + ((int64_t)V.view_index * p.n_q_heads + h0 + j) * D) + d8);
         reinterpret_cast<uint4 *>(q_s)[i] = val;
     }
     __syncthreads();
@@ -835,7 +859,10 @@ template <int NG>
 __global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
     decode_attn_kernel(const __grid_constant__ AttnParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
-    pdl_wait();               // inputs may come from the preceding grid
+    // Inputs may come from the preceding grid.  Behind a fused append, only
+    // the copies of the blocks the append writes wait for it (see dep_step):
+    // that grid waited for everything before it and then released this one.
+    if (!p.fused) pdl_wait();
     pdl_launch_dependents();  // the combine grid may be scheduled as slots free up
     // ---- which item: view by binary search over chunk ranges
     const int bx = blockIdx.x;
@@ -880,6 +907,7 @@ __global__ void __launch_bounds__(kAttnThreads) combine_kernel(const __grid_cons
     const int n = V.n_chunks;
     if (n <= 1) return;  // single-chunk units were written by the attention grid
     pdl_wait();
+    pdl_launch_dependents();
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h0 = hk * p.group + z * kHeadsPerCta;
     const int nh = min(kHeadsPerCta, p.group - z * kHeadsPerCta);

@@ -323,6 +323,8 @@ struct AppendArgs {
 template <int NG>
 __global__ void __launch_bounds__(32) append_kernel(AppendArgs a) {
     constexpr int D = NG * kGroup;
+    pdl_wait();               // the rows it reads or overwrites may belong to the preceding grid
+    pdl_launch_dependents();  // the attention grid may be scheduled meanwhile (it waits in turn)
     const AppendView &v = a.views[blockIdx.x];
     const int h = blockIdx.y;
     const int kv = blockIdx.z;

@@ -130,3 +130,21 @@ def test_append_capacity_checked_before_launch(L):
     ok_win = (kvq.CView * 1)(cview(n_packed=8, cap_packed=8, n_window=1, cap_window=4,
                                    k_window=0x50000, v_window=0x60000))
     assert L.kvq_append(ok_win, 1, 2, 128, NULL, FAKE, NULL) == kvq.KVQ_ERR_INVALID_ARG  # null k_new
+
+
+def test_fused_step_checks_before_launch(L):
+    # capacity: nothing enqueued, no counter changed
+    full = (kvq.CView * 2)(cview(n_packed=4, cap_packed=8), cview(n_packed=8, cap_packed=8))
+    ws = 1 << 20
+    r = L.kvq_append_decode_attn(full, 2, 8, 2, 128, FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, ws, NULL)
+    assert r == kvq.KVQ_ERR_CAPACITY
+    assert full[0].n_packed == 4 and full[1].n_packed == 8
+    # attention arguments are checked before the append is enqueued
+    ok = (kvq.CView * 1)(cview(n_packed=4, cap_packed=8))
+    assert L.kvq_append_decode_attn(ok, 1, 7, 2, 128, FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, ws, NULL) == \
+        kvq.KVQ_ERR_INVALID_ARG                                                    # Hq % Hkv
+    assert L.kvq_append_decode_attn(ok, 1, 8, 2, 128, FAKE, FAKE, NULL, 0.1, FAKE, FAKE, ws, NULL) == \
+        kvq.KVQ_ERR_INVALID_ARG                                                    # null q
+    assert L.kvq_append_decode_attn(ok, 1, 8, 2, 128, FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, 16, NULL) == \
+        kvq.KVQ_ERR_INVALID_ARG                                                    # workspace too small
+    assert ok[0].n_packed == 4
