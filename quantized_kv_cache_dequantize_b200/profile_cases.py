@@ -12,8 +12,9 @@ CASE:
   quantize-handoff / dequantize-handoff
                  the bulk handoff's K cache: 32 layers x 8 kv heads x 32768
                  tokens x 128 (2 GiB bf16), 1% outlier channels x10
-Each case runs 3 warm-up calls and then --reps timed calls, and prints the
-mean time per call and the algorithmic GB/s.
+Each case runs 3 warm-up calls, captures one call in a CUDA graph, replays
+it once more and then --reps timed times, and prints the mean time per call
+and the algorithmic GB/s.
 """
 from __future__ import annotations
 
@@ -28,15 +29,25 @@ from . import decode_attn, dequantize, new_workspace, quantize
 
 
 def _time(fn, reps):
-    for _ in range(3):
+    """Mean device time of one call: 3 eager warm-up calls, then the call
+    captured in a CUDA graph and replayed `reps` times (host launch cost stays
+    out of the timing)."""
+    st = torch.cuda.Stream()
+    with torch.cuda.stream(st):
+        for _ in range(3):
+            fn()
+    st.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
         fn()
-    torch.cuda.synchronize()
     e0, e1 = torch.cuda.Event(True), torch.cuda.Event(True)
-    e0.record()
-    for _ in range(reps):
-        fn()
-    e1.record()
-    torch.cuda.synchronize()
+    with torch.cuda.stream(st):
+        g.replay()
+        e0.record(st)
+        for _ in range(reps):
+            g.replay()
+        e1.record(st)
+    st.synchronize()
     return e0.elapsed_time(e1) / reps / 1e3
 
 
@@ -53,7 +64,8 @@ def main(argv=None):
         q = kcache.decode_queries(w, device=dev)
         ws = new_workspace(pool.views, w.n_q_heads, device=dev)
         out = torch.empty((w.n_views, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
-        t = _time(lambda: decode_attn(pool.views, q, w.softmax_scale, out=out, workspace=ws), a.reps)
+        t = _time(lambda: decode_attn(pool.views, q, w.softmax_scale, out=out, workspace=ws,
+                                       stream=torch.cuda.current_stream()), a.reps)
         rb = w.head_dim // 8 * 4
         nbytes = w.n_views * (w.n_kv_heads * (w.view_len(0) * (2 * rb + 2 * (w.head_dim // 64) * 8) +
                                               w.window * 4 * w.head_dim) + w.n_q_heads * w.head_dim * 6)
@@ -72,9 +84,9 @@ def main(argv=None):
         y = torch.empty_like(x)
         nbytes = x.numel() * 2 + codes.numel() + sm.numel() * 4
         if a.case.startswith("quantize"):
-            t = _time(lambda: quantize(x, 4, codes, sm), a.reps)
+            t = _time(lambda: quantize(x, 4, codes, sm, stream=torch.cuda.current_stream()), a.reps)
         else:
-            t = _time(lambda: dequantize(codes, sm, T, D, 4, out=y), a.reps)
+            t = _time(lambda: dequantize(codes, sm, T, D, 4, out=y, stream=torch.cuda.current_stream()), a.reps)
     print(f"{a.case}: {t * 1e6:.1f} us per call, {nbytes / t / 1e9:.0f} GB/s")
 
 
