@@ -98,6 +98,7 @@ kvq_status codec(bool quant, const void *x, int64_t hs, int64_t ts, int32_t n_he
 struct AttnLaunch {
     int v0, v1;          // views [v0, v1)
     int total_chunks;
+    int bits;            // the width of every view with packed tokens, 0 if mixed
 };
 
 struct ViewChunks {
@@ -235,7 +236,7 @@ double plan_free(const kvq_view *views, int v0, int v1, int64_t units, int32_t h
     return best_cost;
 }
 
-template <int NG>
+template <int NG, int BSEL>
 kvq_status ensure_attn_smem(size_t smem) {
     // the attention kernel's dynamic shared-memory limit, raised once per device
     static std::mutex mu;
@@ -247,7 +248,7 @@ kvq_status ensure_attn_smem(size_t smem) {
     }
     std::lock_guard<std::mutex> lock(mu);
     if (dev >= kMaxDevices || configured[dev] < (int)smem) {
-        if (cudaFuncSetAttribute(kvq::decode_attn_kernel<NG>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+        if (cudaFuncSetAttribute(kvq::decode_attn_kernel<NG, BSEL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                  (int)smem) != cudaSuccess) {
             (void)cudaGetLastError();
             return KVQ_ERR_CUDA;
@@ -296,7 +297,12 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, 
         int64_t chunks = 0;
         plan_free(views, v0, v1, units, head_dim, slots, plan.chunks, &chunks);
         if (chunks > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
-        plan.launches.push_back({v0, v1, (int)chunks});
+        int bits = -1;  // the launch's common width (views without packed tokens have none)
+        for (int i = v0; i < v1; ++i) {
+            if (views[i].n_packed <= 0) continue;
+            bits = (bits < 0 || bits == views[i].bits) ? views[i].bits : 0;
+        }
+        plan.launches.push_back({v0, v1, (int)chunks, bits < 0 ? 4 : bits});
         max_chunks = std::max(max_chunks, chunks);
     }
     plan.partials_off = 256;  // bytes [0, 4): the device status word
@@ -305,12 +311,40 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, 
     return KVQ_OK;
 }
 
+// The attention grid of one launch: the kernel specialized for its width.
+template <int NG>
+kvq_status launch_attn_grid(int bits, size_t smem, const cudaLaunchConfig_t &cfg, const kvq::AttnParams &prm) {
+    kvq_status es;
+    cudaError_t e;
+    switch (bits) {
+        case 2:
+            if ((es = ensure_attn_smem<NG, 2>(smem)) != KVQ_OK) return es;
+            e = cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, 2>, prm);
+            break;
+        case 3:
+            if ((es = ensure_attn_smem<NG, 3>(smem)) != KVQ_OK) return es;
+            e = cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, 3>, prm);
+            break;
+        case 4:
+            if ((es = ensure_attn_smem<NG, 4>(smem)) != KVQ_OK) return es;
+            e = cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, 4>, prm);
+            break;
+        case 8:
+            if ((es = ensure_attn_smem<NG, 8>(smem)) != KVQ_OK) return es;
+            e = cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, 8>, prm);
+            break;
+        default:
+            if ((es = ensure_attn_smem<NG, 0>(smem)) != KVQ_OK) return es;
+            e = cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, 0>, prm);
+            break;
+    }
+    return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
 template <int NG>
 kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n_q_heads, int32_t n_kv_heads,
                           const void *q, float scale, float *out, uint8_t *ws, cudaStream_t st,
                           const int32_t *dep = nullptr) {
-    const kvq_status es = ensure_attn_smem<NG>(plan.smem);
-    if (es != KVQ_OK) return es;
     kvq::AttnParams prm;
     std::memset(&prm, 0, sizeof prm);
     prm.q = static_cast<const uint16_t *>(q);
@@ -373,7 +407,8 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
         cfg.stream = st;
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
-        if (cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG>, prm) != cudaSuccess) return KVQ_ERR_CUDA;
+        const kvq_status es = launch_attn_grid<NG>(L.bits, plan.smem, cfg, prm);
+        if (es != KVQ_OK) return es;
         if (L.total_chunks > L.v1 - L.v0) {  // some unit has more than one chunk
             cfg.gridDim = dim3((unsigned)(L.v1 - L.v0), (unsigned)n_kv_heads, (unsigned)plan.head_blocks);
             cfg.dynamicSmemBytes = 0;

@@ -605,7 +605,10 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         win_v = V.window[1] + (int64_t)hk * V.cap_window * D;
         win_phys = V.cap_window > 0 ? (int)(((int64_t)V.window_head + tok0 + kStepTok * warp) % V.cap_window) : 0;
     }
-    int issue_blk = 0, issue_slot = 0, issue_left = n_tok - kStepTok * warp;  // lane 0's view
+    // Copy issue: every lane keeps the (warp-uniform) bookkeeping and runs
+    // issue_next; only lane 0's async instructions are predicated on.
+    const bool issuer = lane == 0;
+    int issue_blk = 0, issue_slot = 0, issue_left = n_tok - kStepTok * warp;
     int issue_step = s0 + warp;  // step index within the part
     const int dep_step = p.fused ? V.dep_step[WINDOW ? 1 : 0] : -1;
     auto issue_next = [&]() {
@@ -618,11 +621,11 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             const bool full = n == kStepTok;
             const uint32_t bc = full ? (uint32_t)(kStepTok * RB) : round16((uint32_t)(n * RB));
             const uint32_t bs = full ? (uint32_t)(kStepTok * NG * 8) : round16((uint32_t)(n * NG * 8));
-            mbar_arrive_expect_tx(bar, 2 * (bc + bs));
-            bulk_copy_g2s(dst, src_kc, bc, bar);
-            bulk_copy_g2s(dst + kOffV, src_vc, bc, bar);
-            bulk_copy_g2s(dst + kOffKs, src_ks, bs, bar);
-            bulk_copy_g2s(dst + kOffVs, src_vs, bs, bar);
+            mbar_arrive_expect_tx_if(issuer, bar, 2 * (bc + bs));
+            bulk_copy_g2s_if(issuer, dst, src_kc, bc, bar);
+            bulk_copy_g2s_if(issuer, dst + kOffV, src_vc, bc, bar);
+            bulk_copy_g2s_if(issuer, dst + kOffKs, src_ks, bs, bar);
+            bulk_copy_g2s_if(issuer, dst + kOffVs, src_vs, bs, bar);
             src_kc += (int64_t)kAdvTok * RB;
             src_vc += (int64_t)kAdvTok * RB;
             src_ks += (int64_t)kAdvTok * NG * 2;
@@ -633,9 +636,10 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             const int kv = issue_blk & 1;
             const uint16_t *base = kv ? win_v : win_k;
             const int first = min(n, V.cap_window - win_phys);
-            mbar_arrive_expect_tx(bar, (uint32_t)(n * D * 2));
-            bulk_copy_g2s(dst, base + (int64_t)win_phys * D, (uint32_t)(first * D * 2), bar);
-            if (n > first) bulk_copy_g2s(dst + first * D * 2, base, (uint32_t)((n - first) * D * 2), bar);
+            mbar_arrive_expect_tx_if(issuer, bar, (uint32_t)(n * D * 2));
+            bulk_copy_g2s_if(issuer, dst, base + (int64_t)win_phys * D, (uint32_t)(first * D * 2), bar);
+            if (n > first)
+                bulk_copy_g2s_if(issuer, dst + first * D * 2, base, (uint32_t)((n - first) * D * 2), bar);
             if (kv == 1) {
                 win_phys = (win_phys + kAdvTok) % V.cap_window;
                 issue_left -= kAdvTok;
@@ -651,8 +655,9 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     if (lane == 0) {
         for (int s = 0; s < S; ++s) mbar_init(&wbar[s], 1);
         fence_mbar_init();
-        for (int b = 0; b < n_pro; ++b) issue_next();
     }
+    __syncwarp();
+    for (int b = 0; b < n_pro; ++b) issue_next();
     for (int i = tid; i < kHeadsPerCta * D / 8; i += kAttnThreads) {
         const int j = i / (D / 8), d8 = i - j * (D / 8);
         uint4 val = make_uint4(0, 0, 0, 0);
@@ -718,7 +723,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     };
     auto release_cur = [&]() {
         __syncwarp();
-        if (lane == 0 && consumed + S < n_blocks) {
+        if (consumed + S < n_blocks) {  // warp-uniform
             fence_proxy_async_shared();
             issue_next();
         }
@@ -855,7 +860,13 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     }
 }
 
-template <int NG>
+// BSEL = 2, 3, 4 or 8: every view of the launch that has packed tokens has
+// that width, and only that width's code is compiled in; BSEL = 0: any mix of
+// widths, dispatched per CTA.  Specialized kernels keep the instruction
+// footprint of a launch small: with all four widths compiled into one
+// function, about one instruction fetch in five missed the SM's instruction
+// cache on a uniform 4-bit launch, against one in fifty with 4 bits alone.
+template <int NG, int BSEL>
 __global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
     decode_attn_kernel(const __grid_constant__ AttnParams p) {
     extern __shared__ __align__(128) uint8_t smem[];
@@ -877,6 +888,8 @@ __global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
     if (c >= V.n_chunks) return;  // never launched by the host planner; defensive
     if (c >= V.n_chunks_packed) {
         attn_item<NG, 4, true>(p, V, c, hk, z, smem);
+    } else if constexpr (BSEL != 0) {
+        attn_item<NG, BSEL, false>(p, V, c, hk, z, smem);
     } else {
         switch (V.bits) {
             case 2: attn_item<NG, 2, false>(p, V, c, hk, z, smem); break;

@@ -120,6 +120,31 @@ __device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32
         : "memory");
 }
 
+// Predicated forms, executed by a whole warp with `issue` true in one lane:
+// the warp stays converged (no branch around the async instructions).
+__device__ __forceinline__ void mbar_arrive_expect_tx_if(bool issue, uint64_t *bar, uint32_t bytes) {
+    asm volatile(
+        "{\n"
+        ".reg .pred P;\n"
+        "setp.ne.u32 P, %2, 0;\n"
+        "@P mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n"
+        "}\n" ::"r"(smem_u32(bar)),
+        "r"(bytes), "r"((uint32_t)issue)
+        : "memory");
+}
+
+__device__ __forceinline__ void bulk_copy_g2s_if(bool issue, void *dst, const void *src, uint32_t bytes,
+                                                 uint64_t *bar) {
+    asm volatile(
+        "{\n"
+        ".reg .pred P;\n"
+        "setp.ne.u32 P, %4, 0;\n"
+        "@P cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n"
+        "}\n" ::"r"(smem_u32(dst)),
+        "l"(src), "r"(bytes), "r"(smem_u32(bar)), "r"((uint32_t)issue)
+        : "memory");
+}
+
 // Programmatic dependent launch: wait until the preceding grid in the stream
 // has completed and its memory is visible (a no-op when the launch carried no
 // programmatic dependency), and allow the next grid to be scheduled early.
