@@ -247,8 +247,9 @@ kvq_status kvq_append_decode_attn(kvq_view *views, int32_t n_views, int32_t n_q_
  * Set-up: the first call on a device (with that device current) looks up the
  * array's device address once; make that first call before any stream
  * capture.
- * Each call clears the array's status word on `stream` before its kernels;
- * the word is not reported back (kvq_decode_attn exposes it).
+ * Each call clears the array's status word and arrival counters on `stream`
+ * before its kernels; the status word is not reported back (kvq_decode_attn
+ * exposes it).
  * Errors: KVQ_ERR_CAPACITY, with nothing enqueued, when the views need more
  * scratch than KVQ_NOALLOC_SCRATCH_BYTES (kvq_decode_attn_workspace_size
  * gives the need); KVQ_ERR_CUDA if the set-up lookup fails; otherwise as

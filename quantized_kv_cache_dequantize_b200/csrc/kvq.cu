@@ -111,7 +111,7 @@ struct AttnPlan {
     int head_blocks = 0;
     std::vector<AttnLaunch> launches;
     std::vector<ViewChunks> chunks;
-    size_t partials_off = 0, total = 0;
+    size_t counters_off = 0, partials_off = 0, total = 0;
 };
 
 int env_int(const char *name, int dflt) {
@@ -206,7 +206,7 @@ double plan_free(const kvq_view *views, int v0, int v1, int64_t units, int32_t h
             const kvq_view &v = views[i];
             const double cp = (double)packed_token_bytes(head_dim, v.bits), cw = (double)window_token_bytes(head_dim);
             int64_t np = split(v.n_packed, 2 * kvq::kTile, cp, W), nw = split(v.n_window, kvq::kTile, cw, W);
-            // the combine grid holds at most kMaxChunksPerUnit chunks per unit
+            // the unit combine holds at most kMaxChunksPerUnit chunks per unit
             while (np + nw > kvq::kMaxChunksPerUnit) {
                 if (np >= nw) np = std::max<int64_t>(1, np * 3 / 4);
                 else nw = std::max<int64_t>(1, nw * 3 / 4);
@@ -282,8 +282,11 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, 
         if (views[i].n_window > 0) blk_max = std::max<uint32_t>(blk_max, (uint32_t)(32 * head_dim));
     }
     int ring = (smem_cta - header) / kvq::kAttnWarps / 128 * 128;
-    // a ring holds two blocks, and later the warp's partial (m, l, O of 8 heads)
-    const int ring_min = (int)std::max<uint32_t>(2 * blk_max, (uint32_t)(64 + 32 * head_dim));
+    // a ring holds two blocks, and later the warp's partial (m, l, O of 8
+    // heads); all rings together hold the unit combine's scratch
+    const uint32_t combine_scratch = (2 * kvq::kMaxChunksPerUnit * kvq::kHeadsPerCta + kvq::kHeadsPerCta) * 4;
+    const int ring_min = (int)std::max<uint32_t>(std::max<uint32_t>(2 * blk_max, (uint32_t)(64 + 32 * head_dim)),
+                                                 (combine_scratch + kvq::kAttnWarps - 1) / kvq::kAttnWarps);
     if (ring < ring_min) ring = (ring_min + 127) / 128 * 128;  // fewer CTAs per SM, still correct
     plan.ring_bytes = ring;
     plan.smem = (size_t)header + (size_t)kvq::kAttnWarps * ring;
@@ -305,7 +308,10 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, 
         plan.launches.push_back({v0, v1, (int)chunks, bits < 0 ? 4 : bits});
         max_chunks = std::max(max_chunks, chunks);
     }
-    plan.partials_off = 256;  // bytes [0, 4): the device status word
+    // bytes [0, 4): the device status word; then one arrival counter per unit
+    // of a launch; then the chunk partials
+    plan.counters_off = 256;
+    plan.partials_off = plan.counters_off + ((size_t)kvq::kAttnMaxViews * units * 4 + 255) / 256 * 256;
     const size_t part_floats = (size_t)max_chunks * units * kvq::kHeadsPerCta * (head_dim + 2);
     plan.total = plan.partials_off + part_floats * 4;
     return KVQ_OK;
@@ -350,6 +356,7 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
     prm.q = static_cast<const uint16_t *>(q);
     prm.out = out;
     prm.status = reinterpret_cast<uint32_t *>(ws);
+    prm.counters = reinterpret_cast<uint32_t *>(ws + plan.counters_off);
     prm.partials = reinterpret_cast<float *>(ws + plan.partials_off);
     prm.timeout_ns = 2000000000ull;
     prm.scale_log2 = scale * 1.4426950408889634f;
@@ -388,14 +395,10 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
             d.dep_step[1] = prm.fused ? dep[2 * i + 1] : -1;
             begin += d.n_chunks;
         }
-        // Both grids carry a programmatic dependency on the preceding work in
-        // the stream: each starts with griddepcontrol.wait, so it reads
-        // nothing before its predecessor has completed, while its launch and
-        // CTA scheduling overlap the predecessor's tail.
-        // Both grids carry a programmatic dependency on the preceding work in
-        // the stream: each starts with griddepcontrol.wait, so it reads
-        // nothing before its predecessor has completed, while its launch and
-        // CTA scheduling overlap the predecessor's tail.
+        // The grid carries a programmatic dependency on the preceding work in
+        // the stream: it starts with griddepcontrol.wait, so it reads nothing
+        // before its predecessor has completed, while its launch and CTA
+        // scheduling overlap the predecessor's tail.
         cudaLaunchAttribute attr;
         attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr.val.programmaticStreamSerializationAllowed = 1;
@@ -409,11 +412,6 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
         cfg.numAttrs = 1;
         const kvq_status es = launch_attn_grid<NG>(L.bits, plan.smem, cfg, prm);
         if (es != KVQ_OK) return es;
-        if (L.total_chunks > L.v1 - L.v0) {  // some unit has more than one chunk
-            cfg.gridDim = dim3((unsigned)(L.v1 - L.v0), (unsigned)n_kv_heads, (unsigned)plan.head_blocks);
-            cfg.dynamicSmemBytes = 0;
-            if (cudaLaunchKernelEx(&cfg, kvq::combine_kernel<NG>, prm) != cudaSuccess) return KVQ_ERR_CUDA;
-        }
     }
     return KVQ_OK;
 }
@@ -632,8 +630,9 @@ KVQ_API kvq_status kvq_decode_attn_noalloc(const kvq_view *views, int32_t n_view
     const kvq_status ss = noalloc_scratch(&scratch);
     if (ss != KVQ_OK) return ss;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    // the status word must start at zero; nothing else is read before written
-    if (cudaMemsetAsync(scratch, 0, sizeof(uint32_t), st) != cudaSuccess) return KVQ_ERR_CUDA;
+    // the status word and the arrival counters must start at zero; the
+    // partials are written before they are read
+    if (cudaMemsetAsync(scratch, 0, plan.partials_off, st) != cudaSuccess) return KVQ_ERR_CUDA;
     return launch_attn(plan, views, n_q_heads, n_kv_heads, head_dim, q, softmax_scale, out,
                        static_cast<uint8_t *>(scratch), st);
 }

@@ -28,9 +28,9 @@
 //        with movmatrix.
 // Window tiles (bf16 K/V) use the same tile loop with the values as operands.
 // Each CTA merges its warps in a fixed order and writes its chunk's partial
-// (m, l, O); a small combine grid, launched with a programmatic dependency,
-// merges each unit's chunks in chunk order, so results are bitwise
-// reproducible and no CTA waits on another.
+// (m, l, O); the CTA that finishes a unit's last chunk (an atomic arrival
+// counter, never a wait) merges the unit's chunks in chunk order, so results
+// are bitwise reproducible and no CTA waits on another.
 #pragma once
 
 #include <cstdint>
@@ -46,7 +46,7 @@ constexpr int kTile = 16;
 constexpr int kMaxStages = 12;
 constexpr int kHeadsPerCta = 8;
 constexpr int kAttnMaxViews = 96;
-constexpr int kMaxChunksPerUnit = 256;  // combine scratch: 2 * 256 * 8 floats of static shared memory
+constexpr int kMaxChunksPerUnit = 256;  // combine scratch: 2 * 256 * 8 + 8 floats in the ring area
 
 struct AttnView {
     const uint8_t *codes[2];     // K, V packed rows [H_kv][cap][RB]
@@ -71,6 +71,7 @@ struct AttnParams {
     const uint16_t *q;           // bf16 [n_views_total][Hq][D]
     float *out;                  // fp32 [n_views_total][Hq][D]
     float *partials;             // workspace
+    uint32_t *counters;          // workspace: per unit of the launch, chunks finished
     uint32_t *status;            // workspace word 0
     uint64_t timeout_ns;
     float scale_log2;            // softmax_scale * log2(e)
@@ -545,6 +546,80 @@ __host__ __device__ constexpr int attn_header_bytes() {
     return (8 * 64 * NG * 2 + kAttnWarps * kMaxStages * 8 + 16 + 127) & ~127;
 }
 
+// Split-K combine of one unit (view, KV head, head block) whose n > 1 chunk
+// partials are in the workspace, run by the CTA that finished the unit's last
+// chunk.  A partial is [O: 8 heads x D][m: 8][l: 8] floats.  The CTA gathers
+// every chunk's (m, l), reduces per head with warp shuffles, then sums the
+// chunks' O in chunk order, 4 elements per thread and 8 chunks per batch of
+// independent loads, so results are bitwise reproducible and the loads of a
+// batch overlap.  `scratch` holds 2 * kMaxChunksPerUnit * 8 + 8 floats.
+template <int NG>
+__device__ __forceinline__ void combine_unit(const AttnParams &p, const AttnView &V, int hk, int z,
+                                             float *scratch) {
+    constexpr int D = 64 * NG;
+    constexpr int kSlot = kHeadsPerCta * (D + 2);  // floats per partial
+    float *sm_w = scratch;                                        // m, then weight
+    float *sm_l = scratch + kMaxChunksPerUnit * kHeadsPerCta;
+    float *sm_L = scratch + 2 * kMaxChunksPerUnit * kHeadsPerCta;
+    const int n = V.n_chunks;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int h0 = hk * p.group + z * kHeadsPerCta;
+    const int nh = min(kHeadsPerCta, p.group - z * kHeadsPerCta);
+    const int64_t slot0 = ((int64_t)V.chunk_begin * p.n_kv_heads + hk) * p.head_blocks + z;
+    const int64_t stride = (int64_t)p.n_kv_heads * p.head_blocks * kSlot;  // between chunks
+    const float *part0 = p.partials + slot0 * kSlot;
+    for (int i = tid; i < n * nh; i += kAttnThreads) {
+        const int cc = i / nh, j = i - cc * nh;
+        const float *pc = part0 + cc * stride + kHeadsPerCta * D;
+        sm_w[cc * kHeadsPerCta + j] = __ldcg(pc + j);
+        sm_l[cc * kHeadsPerCta + j] = __ldcg(pc + kHeadsPerCta + j);
+    }
+    __syncthreads();
+    for (int j = warp; j < nh; j += kAttnWarps) {
+        float M = -INFINITY;
+        for (int cc = lane; cc < n; cc += 32) M = fmaxf(M, sm_w[cc * kHeadsPerCta + j]);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
+        float L = 0.f;
+        for (int cc = lane; cc < n; cc += 32) {
+            const float mc = sm_w[cc * kHeadsPerCta + j];
+            const float w = (mc == -INFINITY) ? 0.f : fast_exp2(mc - M);
+            sm_w[cc * kHeadsPerCta + j] = w;
+            L = fmaf(w, sm_l[cc * kHeadsPerCta + j], L);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o);
+        if (lane == 0) sm_L[j] = L;
+    }
+    __syncthreads();
+    const float4 *o4 = reinterpret_cast<const float4 *>(part0);
+    const int64_t stride4 = stride / 4;
+    float4 *out4 = reinterpret_cast<float4 *>(p.out + ((int64_t)V.view_index * p.n_q_heads + h0) * D);
+    for (int f = tid; f < nh * (D / 4); f += kAttnThreads) {
+        const int j = f / (D / 4);
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int c0 = 0; c0 < n; c0 += 8) {
+            float4 v[8];
+            float w[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const bool ok = c0 + u < n;
+                v[u] = ok ? __ldcg(o4 + (c0 + u) * stride4 + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+                w[u] = ok ? sm_w[(c0 + u) * kHeadsPerCta + j] : 0.f;
+            }
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                acc.x = fmaf(w[u], v[u].x, acc.x);
+                acc.y = fmaf(w[u], v[u].y, acc.y);
+                acc.z = fmaf(w[u], v[u].z, acc.z);
+                acc.w = fmaf(w[u], v[u].w, acc.w);
+            }
+        }
+        const float L = sm_L[j];
+        out4[f] = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
+    }
+}
+
 // One work item: (view, KV head hk, query-head block z, chunk of tokens).
 // The chunk is cut into steps (32 packed tokens, or 16 window tokens); warp w
 // takes steps w, w+4, ...  A packed step is one block holding both halves of
@@ -554,7 +629,7 @@ __host__ __device__ constexpr int attn_header_bytes() {
 // the block's bulk copies; one lane issues the copies and a slot is refilled
 // as soon as the warp has consumed it.
 template <int NG, int B, bool WINDOW>
-__device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V, int c, int hk, int z,
+__device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V, int vl, int c, int hk, int z,
                                           uint8_t *smem) {
     constexpr int D = 64 * NG;
     constexpr int RB = 8 * B * NG;
@@ -858,6 +933,24 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             }
         }
     }
+    if (single) return;
+    // ---- the CTA that finishes a unit's last chunk combines the unit (an
+    // arrival counter, never a wait); it resets the counter for the next call
+    int *last_flag = reinterpret_cast<int *>(bars + kAttnWarps * kMaxStages);
+    __threadfence();  // this thread's partial stores, before the arrival below
+    __syncthreads();
+    if (tid == 0) {
+        uint32_t *ctr = p.counters + ((int64_t)vl * p.n_kv_heads + hk) * p.head_blocks + z;
+        const uint32_t before = atomicAdd(ctr, 1u);
+        const bool last = before + 1 == (uint32_t)V.n_chunks;
+        if (last) *ctr = 0u;
+        *last_flag = last ? 1 : 0;
+    }
+    __syncthreads();
+    if (*last_flag) {
+        __threadfence();  // the other chunks' partials, after their arrivals
+        combine_unit<NG>(p, V, hk, z, reinterpret_cast<float *>(rings));
+    }
 }
 
 // BSEL = 2, 3, 4 or 8: every view of the launch that has packed tokens has
@@ -874,7 +967,7 @@ __global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
     // the copies of the blocks the append writes wait for it (see dep_step):
     // that grid waited for everything before it and then released this one.
     if (!p.fused) pdl_wait();
-    pdl_launch_dependents();  // the combine grid may be scheduled as slots free up
+    pdl_launch_dependents();  // the next grid may be scheduled as slots free up (it waits in turn)
     // ---- which item: view by binary search over chunk ranges
     const int bx = blockIdx.x;
     int lo = 0, hi = p.n_views - 1;
@@ -887,95 +980,16 @@ __global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
     const int hk = blockIdx.y, z = blockIdx.z;
     if (c >= V.n_chunks) return;  // never launched by the host planner; defensive
     if (c >= V.n_chunks_packed) {
-        attn_item<NG, 4, true>(p, V, c, hk, z, smem);
+        attn_item<NG, 4, true>(p, V, lo, c, hk, z, smem);
     } else if constexpr (BSEL != 0) {
-        attn_item<NG, BSEL, false>(p, V, c, hk, z, smem);
+        attn_item<NG, BSEL, false>(p, V, lo, c, hk, z, smem);
     } else {
         switch (V.bits) {
-            case 2: attn_item<NG, 2, false>(p, V, c, hk, z, smem); break;
-            case 3: attn_item<NG, 3, false>(p, V, c, hk, z, smem); break;
-            case 4: attn_item<NG, 4, false>(p, V, c, hk, z, smem); break;
-            default: attn_item<NG, 8, false>(p, V, c, hk, z, smem); break;
+            case 2: attn_item<NG, 2, false>(p, V, lo, c, hk, z, smem); break;
+            case 3: attn_item<NG, 3, false>(p, V, lo, c, hk, z, smem); break;
+            case 4: attn_item<NG, 4, false>(p, V, lo, c, hk, z, smem); break;
+            default: attn_item<NG, 8, false>(p, V, lo, c, hk, z, smem); break;
         }
-    }
-}
-
-// Split-K combine: one CTA per (view, KV head, head block) with more than one
-// chunk.  A chunk's partial is [O: 8 heads x D][m: 8][l: 8] floats.  The CTA
-// gathers every chunk's (m, l), reduces per head with warp shuffles, then sums
-// the chunks' O in chunk order, 4 elements per thread and 8 chunks per batch
-// of independent loads, so results are bitwise reproducible and the loads of a
-// batch overlap.  Launched right after the attention grid with a programmatic
-// dependency: it is scheduled while the attention tail runs and waits for that
-// grid's completion before reading.
-template <int NG>
-__global__ void __launch_bounds__(kAttnThreads) combine_kernel(const __grid_constant__ AttnParams p) {
-    constexpr int D = 64 * NG;
-    constexpr int kSlot = kHeadsPerCta * (D + 2);  // floats per partial
-    __shared__ float sm_w[kMaxChunksPerUnit * kHeadsPerCta];  // m, then weight
-    __shared__ float sm_l[kMaxChunksPerUnit * kHeadsPerCta];
-    __shared__ float sm_L[kHeadsPerCta];
-    const int vi = blockIdx.x, hk = blockIdx.y, z = blockIdx.z;
-    const AttnView &V = p.views[vi];
-    const int n = V.n_chunks;
-    if (n <= 1) return;  // single-chunk units were written by the attention grid
-    pdl_wait();
-    pdl_launch_dependents();
-    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int h0 = hk * p.group + z * kHeadsPerCta;
-    const int nh = min(kHeadsPerCta, p.group - z * kHeadsPerCta);
-    const int64_t slot0 = ((int64_t)V.chunk_begin * p.n_kv_heads + hk) * p.head_blocks + z;
-    const int64_t stride = (int64_t)p.n_kv_heads * p.head_blocks * kSlot;  // between chunks
-    const float *part0 = p.partials + slot0 * kSlot;
-    for (int i = tid; i < n * nh; i += kAttnThreads) {
-        const int cc = i / nh, j = i - cc * nh;
-        const float *pc = part0 + cc * stride + kHeadsPerCta * D;
-        sm_w[cc * kHeadsPerCta + j] = __ldcg(pc + j);
-        sm_l[cc * kHeadsPerCta + j] = __ldcg(pc + kHeadsPerCta + j);
-    }
-    __syncthreads();
-    for (int j = warp; j < nh; j += kAttnWarps) {
-        float M = -INFINITY;
-        for (int cc = lane; cc < n; cc += 32) M = fmaxf(M, sm_w[cc * kHeadsPerCta + j]);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xFFFFFFFFu, M, o));
-        float L = 0.f;
-        for (int cc = lane; cc < n; cc += 32) {
-            const float mc = sm_w[cc * kHeadsPerCta + j];
-            const float w = (mc == -INFINITY) ? 0.f : fast_exp2(mc - M);
-            sm_w[cc * kHeadsPerCta + j] = w;
-            L = fmaf(w, sm_l[cc * kHeadsPerCta + j], L);
-        }
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xFFFFFFFFu, L, o);
-        if (lane == 0) sm_L[j] = L;
-    }
-    __syncthreads();
-    const float4 *o4 = reinterpret_cast<const float4 *>(part0);
-    const int64_t stride4 = stride / 4;
-    float4 *out4 = reinterpret_cast<float4 *>(p.out + ((int64_t)V.view_index * p.n_q_heads + h0) * D);
-    for (int f = tid; f < nh * (D / 4); f += kAttnThreads) {
-        const int j = f / (D / 4);
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int c0 = 0; c0 < n; c0 += 8) {
-            float4 v[8];
-            float w[8];
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                const bool ok = c0 + u < n;
-                v[u] = ok ? __ldcg(o4 + (c0 + u) * stride4 + f) : make_float4(0.f, 0.f, 0.f, 0.f);
-                w[u] = ok ? sm_w[(c0 + u) * kHeadsPerCta + j] : 0.f;
-            }
-#pragma unroll
-            for (int u = 0; u < 8; ++u) {
-                acc.x = fmaf(w[u], v[u].x, acc.x);
-                acc.y = fmaf(w[u], v[u].y, acc.y);
-                acc.z = fmaf(w[u], v[u].z, acc.z);
-                acc.w = fmaf(w[u], v[u].w, acc.w);
-            }
-        }
-        const float L = sm_L[j];
-        out4[f] = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
     }
 }
 
