@@ -240,10 +240,9 @@ def run_ours(args, rank, world, local):
     torch.cuda.synchronize()
 
     stream = torch.cuda.Stream()
-    # per layer: the append kernel, the attention grid and its split-K
-    # combine grid (every view here has packed and window tokens, so every
-    # unit has more than one chunk and the combine grid is launched)
-    n_launch_per_step = 3 * L
+    # per layer: the append grid and the attention grid (whose last CTA per
+    # unit does the split-K combine)
+    n_launch_per_step = 2 * L
 
     def step():
         # one decode step per layer: append this token, attend over the result
@@ -282,9 +281,9 @@ def run_ours(args, rank, world, local):
     t_step = kdist.max_over_ranks(e0.elapsed_time(e1) / 1e3 / args.steps)
     value = kdist.aggregate_throughput(bytes_step, world, t_step) / 1e9
 
-    # ---------------- dominant kernel: kvq_decode_attn per layer (attention
-    # grid + its split-K combine grid), the 32 layers' calls replayed from one
-    # CUDA graph so that host launch cost stays out of the device timing
+    # ---------------- dominant kernel: kvq_decode_attn per layer (one
+    # attention grid, split-K combine included), the 32 layers' calls replayed
+    # from one CUDA graph so that host launch cost stays out of the device timing
     attn_layer_bytes = attn_bytes(A, w.n_kv_heads, w.n_q_heads, w.head_dim, w.view_len(0) + 1, w.window, 4)
 
     def attn_layers():
@@ -424,13 +423,13 @@ def run_ours(args, rank, world, local):
             "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
             "config": {"workload": WORKLOAD, "agents_per_gpu": A, "layers": L, "n_q_heads": w.n_q_heads,
                        "n_kv_heads": w.n_kv_heads, "head_dim": w.head_dim, "packed_tokens": w.view_len(0),
-                       "window": w.window, "bits": 4, "calls_per_step": "per layer: kvq_append_decode_attn (append, attention and combine grids)",
+                       "window": w.window, "bits": 4, "calls_per_step": "per layer: kvq_append_decode_attn (append grid + attention grid)",
                        "cuda_graph": True, "l2": "working set per step ~1.9 GB > 126 MB L2, no flush"},
             "tokens_per_s_per_agent": 1.0 / t_step,
             "hbm_frac": value / world / peak,
             "roofline": {"bound": "hbm", "achieved": attn_gbs, "peak": peak, "unit": "GB/s",
                          "frac": attn_gbs / peak, "traffic": profiled_traffic(),
-                         "kernel": "kvq_decode_attn per layer, 10 views: decode_attn_kernel<2> + combine_kernel<2>",
+                         "kernel": "decode_attn_kernel<2, 4>: one kvq_decode_attn per layer, 10 views",
                          "bytes_per_launch": attn_layer_bytes, "launch_us": t_attn * 1e6,
                          "peak_kind": f"{peak_kind} (hbm_gbs)"},
             "all_views_one_call": {"gbs": all_gbs, "frac": all_gbs / peak, "ms": t_all * 1e3},
