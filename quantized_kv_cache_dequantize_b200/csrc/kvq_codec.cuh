@@ -229,66 +229,90 @@ __global__ void __launch_bounds__(256) quantize_kernel(CodecArgs a) {
     }
 }
 
-// Same sweep; each lane pair dequantizes kDeqRounds groups per iteration
-// (all loads first, then compute and streaming stores).
+// Same sweep; each lane pair dequantizes kDeqRounds groups per iteration.
+// Software-pipelined: the codes and scale/min of the next iteration are
+// loaded before this iteration's groups are converted and stored, so the load
+// latency overlaps the (3x larger) store stream.
+template <int B>
+struct DeqSet {
+    uint32_t packed[kDeqRounds][B];
+    float2 sm[kDeqRounds];
+    int64_t t[kDeqRounds];
+    int g[kDeqRounds], hh[kDeqRounds];
+    bool ok[kDeqRounds];
+};
+
+template <int B, int NG>
+__device__ __forceinline__ void deq_load(const CodecArgs &a, SweepCursor c, int half, int64_t n_groups, DeqSet<B> &d) {
+    constexpr int RB = 8 * B * NG;
+#pragma unroll
+    for (int u = 0; u < kDeqRounds; ++u) {
+        d.ok[u] = c.h < a.n_heads;
+        d.hh[u] = c.h;
+        d.t[u] = c.grp / NG;
+        d.g[u] = (int)(c.grp - d.t[u] * NG);
+        if (d.ok[u]) {
+            const int64_t row = (int64_t)c.h * a.head_cap + d.t[u];
+            const uint8_t *src = a.codes + row * RB + d.g[u] * 8 * B + half * 4 * B;
+            if constexpr (B == 4) {
+                const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(src));
+                d.packed[u][0] = q.x; d.packed[u][1] = q.y; d.packed[u][2] = q.z; d.packed[u][3] = q.w;
+            } else if constexpr (B == 8) {
+                const uint4 q0 = __ldcs(reinterpret_cast<const uint4 *>(src));
+                const uint4 q1 = __ldcs(reinterpret_cast<const uint4 *>(src) + 1);
+                d.packed[u][0] = q0.x; d.packed[u][1] = q0.y; d.packed[u][2] = q0.z; d.packed[u][3] = q0.w;
+                d.packed[u][4] = q1.x; d.packed[u][5] = q1.y; d.packed[u][6] = q1.z; d.packed[u][7] = q1.w;
+            } else if constexpr (B == 2) {
+                const uint2 q = __ldcs(reinterpret_cast<const uint2 *>(src));
+                d.packed[u][0] = q.x; d.packed[u][1] = q.y;
+            } else {
+#pragma unroll
+                for (int w = 0; w < B; ++w) d.packed[u][w] = __ldcs(reinterpret_cast<const uint32_t *>(src) + w);
+            }
+            d.sm[u] = __ldcs(reinterpret_cast<const float2 *>(a.scalemin + (row * NG + d.g[u]) * 2));
+        }
+        sweep_advance(c, 16, n_groups);
+    }
+}
+
+template <int B>
+__device__ __forceinline__ void deq_store(const CodecArgs &a, int half, const DeqSet<B> &d) {
+    uint16_t *y = const_cast<uint16_t *>(a.x);
+#pragma unroll
+    for (int u = 0; u < kDeqRounds; ++u) {
+        if (!d.ok[u]) continue;
+        uint32_t yv[16];
+        dequantize_half_group<B>(d.packed[u], d.sm[u].x, d.sm[u].y, yv);
+        uint4 *dst = reinterpret_cast<uint4 *>(y + (int64_t)d.hh[u] * a.x_head_stride + d.t[u] * a.x_tok_stride +
+                                               d.g[u] * kGroup + half * 32);
+#pragma unroll
+        for (int v = 0; v < 4; ++v) __stcs(dst + v, make_uint4(yv[4 * v], yv[4 * v + 1], yv[4 * v + 2], yv[4 * v + 3]));
+    }
+}
+
 template <int B, int NG>
 __global__ void __launch_bounds__(256) dequantize_kernel(CodecArgs a) {
-    constexpr int RB = 8 * B * NG;
-    constexpr int kR = kDeqRounds;
     const int64_t n_groups = a.n_tokens * NG;
     const int lane = threadIdx.x & 31;
     const int half = lane & 1;
     const int64_t warp_global = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int64_t warp_stride = (int64_t)gridDim.x * (blockDim.x >> 5);
-    uint16_t *y = const_cast<uint16_t *>(a.x);
+    const int64_t step = (int64_t)gridDim.x * (blockDim.x >> 5) * 16 * kDeqRounds;
     SweepCursor cur{0, 0};
-    sweep_advance(cur, warp_global * 16 * kR + (lane >> 1), n_groups);
-    while (cur.h < a.n_heads) {
-        uint32_t packed[kR][B];
-        float2 sm[kR];
-        int64_t t[kR];
-        int g[kR], hh[kR];
-        bool ok[kR];
-        SweepCursor c = cur;
-#pragma unroll
-        for (int u = 0; u < kR; ++u) {
-            ok[u] = c.h < a.n_heads;
-            hh[u] = c.h;
-            t[u] = c.grp / NG;
-            g[u] = (int)(c.grp - t[u] * NG);
-            if (ok[u]) {
-                const int64_t row = (int64_t)c.h * a.head_cap + t[u];
-                const uint8_t *src = a.codes + row * RB + g[u] * 8 * B + half * 4 * B;
-                if constexpr (B == 4) {
-                    const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(src));
-                    packed[u][0] = q.x; packed[u][1] = q.y; packed[u][2] = q.z; packed[u][3] = q.w;
-                } else if constexpr (B == 8) {
-                    const uint4 q0 = __ldcs(reinterpret_cast<const uint4 *>(src));
-                    const uint4 q1 = __ldcs(reinterpret_cast<const uint4 *>(src) + 1);
-                    packed[u][0] = q0.x; packed[u][1] = q0.y; packed[u][2] = q0.z; packed[u][3] = q0.w;
-                    packed[u][4] = q1.x; packed[u][5] = q1.y; packed[u][6] = q1.z; packed[u][7] = q1.w;
-                } else if constexpr (B == 2) {
-                    const uint2 q = __ldcs(reinterpret_cast<const uint2 *>(src));
-                    packed[u][0] = q.x; packed[u][1] = q.y;
-                } else {
-#pragma unroll
-                    for (int w = 0; w < B; ++w) packed[u][w] = __ldcs(reinterpret_cast<const uint32_t *>(src) + w);
-                }
-                sm[u] = __ldcs(reinterpret_cast<const float2 *>(a.scalemin + (row * NG + g[u]) * 2));
-            }
-            sweep_advance(c, 16, n_groups);
-        }
-#pragma unroll
-        for (int u = 0; u < kR; ++u) {
-            if (!ok[u]) continue;
-            uint32_t yv[16];
-            dequantize_half_group<B>(packed[u], sm[u].x, sm[u].y, yv);
-            uint4 *dst = reinterpret_cast<uint4 *>(y + (int64_t)hh[u] * a.x_head_stride + t[u] * a.x_tok_stride +
-                                                   g[u] * kGroup + half * 32);
-#pragma unroll
-            for (int v = 0; v < 4; ++v) __stcs(dst + v, make_uint4(yv[4 * v], yv[4 * v + 1], yv[4 * v + 2], yv[4 * v + 3]));
-        }
-        sweep_advance(cur, warp_stride * 16 * kR, n_groups);
+    sweep_advance(cur, warp_global * 16 * kDeqRounds + (lane >> 1), n_groups);
+    if (cur.h >= a.n_heads) return;
+    DeqSet<B> d0, d1;
+    deq_load<B, NG>(a, cur, half, n_groups, d0);
+    while (true) {
+        sweep_advance(cur, step, n_groups);
+        const bool more = cur.h < a.n_heads;
+        if (more) deq_load<B, NG>(a, cur, half, n_groups, d1);
+        deq_store<B>(a, half, d0);
+        if (!more) break;
+        sweep_advance(cur, step, n_groups);
+        const bool more2 = cur.h < a.n_heads;
+        if (more2) deq_load<B, NG>(a, cur, half, n_groups, d0);
+        deq_store<B>(a, half, d1);
+        if (!more2) break;
     }
 }
 
