@@ -113,8 +113,10 @@ class ClockSampler:
             for name, val in zip(names, r[5:9]):
                 if val.strip().lower().startswith("active"):
                     reasons.add(name)
+        pw = [float(r[3]) for r in rows if r[3].strip().replace(".", "").isdigit()]
         return {"sm_mhz": float(np.median(sm)) if sm else None, "sm_max_mhz": mx,
-                "reasons": sorted(reasons), "samples": len(rows)}
+                "reasons": sorted(reasons), "samples": len(rows),
+                "power_w": float(np.median(pw)) if pw else None}
 
 
 # ------------------------------------------------------------------ helpers --
@@ -380,7 +382,7 @@ def run_ours(args, rank, world, local):
         n_el = 2 * H * hw.n_tokens * hw.head_dim
         codec_bytes = n_el * 2 + 2 * (kc.numel() + ks.numel() * 4)
         qt, dt = [], []
-        with torch.cuda.stream(stream):
+        with ClockSampler(local) as codec_clk, torch.cuda.stream(stream):
             for it in range(args.warmup + args.steps):
                 a0, a1, a2 = torch.cuda.Event(True), torch.cuda.Event(True), torch.cuda.Event(True)
                 a0.record(stream)
@@ -393,7 +395,7 @@ def run_ours(args, rank, world, local):
                 if it >= args.warmup:
                     qt.append((a0, a1))
                     dt.append((a1, a2))
-        stream.synchronize()
+            stream.synchronize()
         tq = float(np.mean([x.elapsed_time(y) for x, y in qt])) / 1e3
         td = float(np.mean([x.elapsed_time(y) for x, y in dt])) / 1e3
         codec = {"workload": "bulk cache handoff, Llama-3.1-8B shape: 32 layers x 8 kv heads x 32768 tokens x "
@@ -402,7 +404,8 @@ def run_ours(args, rank, world, local):
                  "quantize_gbs": codec_bytes / tq / 1e9, "quantize_ms": tq * 1e3,
                  "quantize_frac": codec_bytes / tq / 1e9 / peak,
                  "dequantize_gbs": codec_bytes / td / 1e9, "dequantize_ms": td * 1e3,
-                 "dequantize_frac": codec_bytes / td / 1e9 / peak}
+                 "dequantize_frac": codec_bytes / td / 1e9 / peak,
+                 "clocks": codec_clk.summary()}
         del kx, vx, kc, vc, ks, vs, ky, vy
         torch.cuda.empty_cache()
 
