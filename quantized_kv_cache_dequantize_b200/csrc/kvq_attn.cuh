@@ -548,11 +548,13 @@ __host__ __device__ constexpr int attn_header_bytes() {
 
 // Split-K combine of one unit (view, KV head, head block) whose n > 1 chunk
 // partials are in the workspace, run by the CTA that finished the unit's last
-// chunk.  A partial is [O: 8 heads x D][m: 8][l: 8] floats.  The CTA gathers
+// chunk.  A partial is [O: 8 heads x D][m: 8][l: 8] floats.  Up to 8 chunks:
+// every thread loads all chunks' (m, l) of its head and O of its 4 outputs in
+// one round and merges them in chunk order.  More chunks: the CTA gathers
 // every chunk's (m, l), reduces per head with warp shuffles, then sums the
 // chunks' O in chunk order, 4 elements per thread and 8 chunks per batch of
-// independent loads, so results are bitwise reproducible and the loads of a
-// batch overlap.  `scratch` holds 2 * kMaxChunksPerUnit * 8 + 8 floats.
+// independent loads.  Fixed orders throughout: results are bitwise
+// reproducible.  `scratch` holds 2 * kMaxChunksPerUnit * 8 + 8 floats.
 template <int NG>
 __device__ __forceinline__ void combine_unit(const AttnParams &p, const AttnView &V, int hk, int z,
                                              float *scratch) {
@@ -568,6 +570,41 @@ __device__ __forceinline__ void combine_unit(const AttnParams &p, const AttnView
     const int64_t slot0 = ((int64_t)V.chunk_begin * p.n_kv_heads + hk) * p.head_blocks + z;
     const int64_t stride = (int64_t)p.n_kv_heads * p.head_blocks * kSlot;  // between chunks
     const float *part0 = p.partials + slot0 * kSlot;
+    float4 *out4 = reinterpret_cast<float4 *>(p.out + ((int64_t)V.view_index * p.n_q_heads + h0) * D);
+    if (n <= 8) {
+        // one round of loads: each thread fetches every chunk's (m, l) of its
+        // head and O of its 4 outputs at once, then merges in chunk order
+        const float4 *o4 = reinterpret_cast<const float4 *>(part0);
+        for (int f = tid; f < nh * (D / 4); f += kAttnThreads) {
+            const int j = f / (D / 4);
+            float m[8], l[8];
+            float4 v[8];
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const bool ok = u < n;
+                const float *pc = part0 + u * stride + kHeadsPerCta * D;
+                m[u] = ok ? __ldcg(pc + j) : -INFINITY;
+                l[u] = ok ? __ldcg(pc + kHeadsPerCta + j) : 0.f;
+                v[u] = ok ? __ldcg(o4 + u * (stride / 4) + f) : make_float4(0.f, 0.f, 0.f, 0.f);
+            }
+            float M = m[0];
+#pragma unroll
+            for (int u = 1; u < 8; ++u) M = fmaxf(M, m[u]);
+            float L = 0.f;
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int u = 0; u < 8; ++u) {
+                const float w = (m[u] == -INFINITY) ? 0.f : fast_exp2(m[u] - M);
+                L = fmaf(w, l[u], L);
+                acc.x = fmaf(w, v[u].x, acc.x);
+                acc.y = fmaf(w, v[u].y, acc.y);
+                acc.z = fmaf(w, v[u].z, acc.z);
+                acc.w = fmaf(w, v[u].w, acc.w);
+            }
+            out4[f] = make_float4(acc.x / L, acc.y / L, acc.z / L, acc.w / L);
+        }
+        return;
+    }
     for (int i = tid; i < n * nh; i += kAttnThreads) {
         const int cc = i / nh, j = i - cc * nh;
         const float *pc = part0 + cc * stride + kHeadsPerCta * D;
@@ -594,7 +631,6 @@ __device__ __forceinline__ void combine_unit(const AttnParams &p, const AttnView
     __syncthreads();
     const float4 *o4 = reinterpret_cast<const float4 *>(part0);
     const int64_t stride4 = stride / 4;
-    float4 *out4 = reinterpret_cast<float4 *>(p.out + ((int64_t)V.view_index * p.n_q_heads + h0) * D);
     for (int f = tid; f < nh * (D / 4); f += kAttnThreads) {
         const int j = f / (D / 4);
         float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
