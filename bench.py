@@ -333,30 +333,66 @@ def run_ours(args, rank, world, local):
     t_all = b0.elapsed_time(b1) / 1e3 / args.steps
     all_gbs = attn_bytes(L * A, w.n_kv_heads, w.n_q_heads, w.head_dim, w.view_len(0) + 1, w.window, 4) / t_all / 1e9
 
-    # ---------------- end to end through the public API with host buffers
+    # ---------------- end to end through the public API with host buffers.
+    # Every step copies its q and new K/V in from pinned host memory and its
+    # output back out.  The copies run on a second stream, double-buffered
+    # through device staging tensors, so the next step's inputs arrive and the
+    # previous step's output leaves while a step computes (a serving loop's
+    # pipelining); the timed region spans the first input copy to the last
+    # output copy.
     q_h = q.cpu().pin_memory()
     kn_h, vn_h = kn.cpu().pin_memory(), vn.cpu().pin_memory()
-    out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    out_h = [torch.empty(out.shape, dtype=out.dtype).pin_memory() for _ in range(2)]
     h2d = q_h.numel() * 2 + kn_h.numel() * 2 + vn_h.numel() * 2
-    d2h = out_h.numel() * 4
+    d2h = out.numel() * 4
+    stage_in = [(torch.empty_like(q), torch.empty_like(kn), torch.empty_like(vn)) for _ in range(2)]
+    stage_out = [torch.empty_like(out) for _ in range(2)]
+    cstream = torch.cuda.Stream()
+    in_ready = [torch.cuda.Event() for _ in range(2)]   # host -> stage b landed
+    in_free = [torch.cuda.Event() for _ in range(2)]    # stage b copied into the step's inputs
+    out_ready = [torch.cuda.Event() for _ in range(2)]  # step output copied into stage b
+    out_free = [torch.cuda.Event() for _ in range(2)]   # stage b read back to the host
 
-    def e2e_step():
-        q.copy_(q_h, non_blocking=True)
-        kn.copy_(kn_h, non_blocking=True)
-        vn.copy_(vn_h, non_blocking=True)
-        graph.replay()
-        out_h.copy_(out, non_blocking=True)
+    def copy_in(b):
+        cstream.wait_event(in_free[b])
+        with torch.cuda.stream(cstream):
+            for dst, src in zip(stage_in[b], (q_h, kn_h, vn_h)):
+                dst.copy_(src, non_blocking=True)
+            in_ready[b].record(cstream)
 
-    with torch.cuda.stream(stream):
-        for _ in range(args.warmup):
-            e2e_step()
-        stream.synchronize()
-        c0, c1 = ev_pair()
-        c0.record(stream)
-        for _ in range(args.steps):
-            e2e_step()
-        c1.record(stream)
-    stream.synchronize()
+    def e2e_run(n):
+        for b in range(2):
+            in_free[b].record(stream)
+            out_free[b].record(cstream)
+        t0, t1 = ev_pair()
+        t0.record(cstream)
+        copy_in(0)
+        for i in range(n):
+            b = i % 2
+            stream.wait_event(in_ready[b])
+            with torch.cuda.stream(stream):
+                for dst, src in zip((q, kn, vn), stage_in[b]):
+                    dst.copy_(src)
+                in_free[b].record(stream)
+            if i + 1 < n:
+                copy_in(1 - b)
+            with torch.cuda.stream(stream):
+                graph.replay()
+                stream.wait_event(out_free[b])
+                stage_out[b].copy_(out)
+                out_ready[b].record(stream)
+            cstream.wait_event(out_ready[b])
+            with torch.cuda.stream(cstream):
+                out_h[b].copy_(stage_out[b], non_blocking=True)
+                out_free[b].record(cstream)
+        stream.wait_stream(cstream)
+        t1.record(stream)
+        return t0, t1
+
+    e2e_run(args.warmup)
+    torch.cuda.synchronize()
+    c0, c1 = e2e_run(args.steps)
+    torch.cuda.synchronize()
     t_e2e = kdist.max_over_ranks(c0.elapsed_time(c1) / 1e3 / args.steps)
     e2e_gbs = kdist.aggregate_throughput(bytes_step, world, t_e2e) / 1e9
 
@@ -439,7 +475,9 @@ def run_ours(args, rank, world, local):
             "codec": codec,
             "cpu_baseline": cpu,
             "e2e": {"value": e2e_gbs, "unit": "GB/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-                    "ms_per_step": t_e2e * 1e3},
+                    "ms_per_step": t_e2e * 1e3,
+                    "copies": "pinned host <-> device every step, on a second stream, double-buffered and "
+                              "overlapped with the neighbouring steps' compute"},
             "gpu_launches": n_launch_per_step * args.steps,
             "clocks": clocks,
         }
