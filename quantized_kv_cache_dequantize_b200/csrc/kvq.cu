@@ -96,9 +96,10 @@ kvq_status codec(bool quant, const void *x, int64_t hs, int64_t ts, int32_t n_he
 // ------------------------------------------------------ decode planning ---
 
 struct AttnLaunch {
-    int v0, v1;          // views [v0, v1)
+    int v0, v1;          // views order[v0 .. v1) of the plan
     int total_chunks;
-    int bits;            // the width of every view with packed tokens, 0 if mixed
+    int bits;            // the width of every view of the launch with packed tokens
+    size_t counters_off, partials_off;  // this launch's workspace regions
 };
 
 struct ViewChunks {
@@ -109,9 +110,10 @@ struct AttnPlan {
     int ring_bytes = 0;
     size_t smem = 0;
     int head_blocks = 0;
+    std::vector<int> order;  // views grouped by width (stable), as the launches take them
     std::vector<AttnLaunch> launches;
     std::vector<ViewChunks> chunks;
-    size_t counters_off = 0, partials_off = 0, total = 0;
+    size_t zero_bytes = 0, total = 0;
 };
 
 int env_int(const char *name, int dflt) {
@@ -181,18 +183,20 @@ double largest_chunk(int64_t n_tok, int step, int64_t n, double tok_cost) {
     return (double)std::min<int64_t>((steps + n - 1) / n * step, n_tok) * tok_cost;
 }
 
-// Free chunking of the views [v0, v1): each part (packed, window) of a view is
-// cut into chunks of equal step counts (+-1 step) costing about W each, W
-// picked by the smallest predicted time over whole waves of `slots` resident
-// CTAs.  Stores the chunk counts, returns the predicted time; *chunks = the
-// launch's chunk count per unit.
-double plan_free(const kvq_view *views, int v0, int v1, int64_t units, int32_t head_dim, int64_t slots,
+// Free chunking of the views idx[0 .. n): each part (packed, window) of a
+// view is cut into chunks of equal step counts (+-1 step) costing about W
+// each, W picked by the smallest predicted time over whole waves of `slots`
+// resident CTAs.  Stores the chunk counts, returns the predicted time;
+// *chunks = the launch's chunk count per unit.
+double plan_free(const kvq_view *views, const int *idx, int n_idx, int64_t units, int32_t head_dim, int64_t slots,
                  std::vector<ViewChunks> &out, int64_t *chunks) {
     const int forced = env_int("KVQ_CHUNK_TOKENS", 0);  // tests: force a chunk length
     double total = 0;
-    for (int i = v0; i < v1; ++i)
-        total += (double)units * ((double)views[i].n_packed * packed_token_bytes(head_dim, views[i].bits) +
-                                  (double)views[i].n_window * window_token_bytes(head_dim));
+    for (int k = 0; k < n_idx; ++k) {
+        const kvq_view &v = views[idx[k]];
+        total += (double)units * ((double)v.n_packed * packed_token_bytes(head_dim, v.bits) +
+                                  (double)v.n_window * window_token_bytes(head_dim));
+    }
     auto split = [&](int64_t n_tok, int step, double tok_cost, double W) -> int64_t {
         if (n_tok <= 0) return 0;
         const int64_t steps = (n_tok + step - 1) / step;
@@ -202,7 +206,8 @@ double plan_free(const kvq_view *views, int v0, int v1, int64_t units, int32_t h
     auto count = [&](double W, bool store, double *max_item) -> int64_t {
         int64_t items = 0;
         double mx = 0;
-        for (int i = v0; i < v1; ++i) {
+        for (int k = 0; k < n_idx; ++k) {
+            const int i = idx[k];
             const kvq_view &v = views[i];
             const double cp = (double)packed_token_bytes(head_dim, v.bits), cw = (double)window_token_bytes(head_dim);
             int64_t np = split(v.n_packed, 2 * kvq::kTile, cp, W), nw = split(v.n_window, kvq::kTile, cw, W);
@@ -294,26 +299,49 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, 
 
     const int64_t slots = (int64_t)device_sm_count() * ctas;
     plan.chunks.assign(n_views, ViewChunks{0, 0});
-    int64_t max_chunks = 0;
-    for (int v0 = 0; v0 < n_views; v0 += kvq::kAttnMaxViews) {
-        const int v1 = std::min<int>(n_views, v0 + kvq::kAttnMaxViews);
-        int64_t chunks = 0;
-        plan_free(views, v0, v1, units, head_dim, slots, plan.chunks, &chunks);
-        if (chunks > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
-        int bits = -1;  // the launch's common width (views without packed tokens have none)
-        for (int i = v0; i < v1; ++i) {
-            if (views[i].n_packed <= 0) continue;
-            bits = (bits < 0 || bits == views[i].bits) ? views[i].bits : 0;
+    // Views grouped by width (stable; views without packed tokens join the
+    // first width), at most kAttnMaxViews per launch: each launch then runs
+    // the kernel built for its width alone.  All launches of a call run
+    // concurrently, each on its own workspace regions, so each is planned for
+    // its byte share of the GPU.
+    int first_bits = 4;
+    for (int i = 0; i < n_views; ++i)
+        if (views[i].n_packed > 0) { first_bits = views[i].bits; break; }
+    auto key = [&](int i) { return views[i].n_packed > 0 ? views[i].bits : first_bits; };
+    plan.order.resize(n_views);
+    for (int i = 0; i < n_views; ++i) plan.order[i] = i;
+    std::stable_sort(plan.order.begin(), plan.order.end(), [&](int a, int b) { return key(a) < key(b); });
+    double bytes_all = 0;
+    for (int i = 0; i < n_views; ++i)
+        bytes_all += (double)views[i].n_packed * packed_token_bytes(head_dim, views[i].bits) +
+                     (double)views[i].n_window * window_token_bytes(head_dim);
+    size_t off = 256;  // bytes [0, 4): the device status word
+    for (int v0 = 0; v0 < n_views;) {
+        int v1 = v0 + 1;
+        while (v1 < n_views && v1 - v0 < kvq::kAttnMaxViews && key(plan.order[v1]) == key(plan.order[v0])) ++v1;
+        double bytes = 0;
+        for (int k = v0; k < v1; ++k) {
+            const kvq_view &v = views[plan.order[k]];
+            bytes += (double)v.n_packed * packed_token_bytes(head_dim, v.bits) +
+                     (double)v.n_window * window_token_bytes(head_dim);
         }
-        plan.launches.push_back({v0, v1, (int)chunks, bits < 0 ? 4 : bits});
-        max_chunks = std::max(max_chunks, chunks);
+        const int64_t share = std::max<int64_t>(
+            1, (int64_t)std::llround((double)slots * (bytes_all > 0 ? bytes / bytes_all : 1.0)));
+        int64_t chunks = 0;
+        plan_free(views, plan.order.data() + v0, v1 - v0, units, head_dim, share, plan.chunks, &chunks);
+        if (chunks > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
+        AttnLaunch L{v0, v1, (int)chunks, key(plan.order[v0]), 0, 0};
+        L.counters_off = off;  // one arrival counter per unit of the launch
+        off += ((size_t)(v1 - v0) * units * 4 + 255) / 256 * 256;
+        plan.launches.push_back(L);
+        v0 = v1;
     }
-    // bytes [0, 4): the device status word; then one arrival counter per unit
-    // of a launch; then the chunk partials
-    plan.counters_off = 256;
-    plan.partials_off = plan.counters_off + ((size_t)kvq::kAttnMaxViews * units * 4 + 255) / 256 * 256;
-    const size_t part_floats = (size_t)max_chunks * units * kvq::kHeadsPerCta * (head_dim + 2);
-    plan.total = plan.partials_off + part_floats * 4;
+    plan.zero_bytes = off;  // status word and counters: the part that must start at zero
+    for (AttnLaunch &L : plan.launches) {
+        L.partials_off = off;
+        off += ((size_t)L.total_chunks * units * kvq::kHeadsPerCta * (head_dim + 2) * 4 + 255) / 256 * 256;
+    }
+    plan.total = off;
     return KVQ_OK;
 }
 
@@ -335,13 +363,9 @@ kvq_status launch_attn_grid(int bits, size_t smem, const cudaLaunchConfig_t &cfg
             if ((es = ensure_attn_smem<NG, 4>(smem)) != KVQ_OK) return es;
             e = cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, 4>, prm);
             break;
-        case 8:
+        default:
             if ((es = ensure_attn_smem<NG, 8>(smem)) != KVQ_OK) return es;
             e = cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, 8>, prm);
-            break;
-        default:
-            if ((es = ensure_attn_smem<NG, 0>(smem)) != KVQ_OK) return es;
-            e = cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, 0>, prm);
             break;
     }
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
@@ -356,8 +380,6 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
     prm.q = static_cast<const uint16_t *>(q);
     prm.out = out;
     prm.status = reinterpret_cast<uint32_t *>(ws);
-    prm.counters = reinterpret_cast<uint32_t *>(ws + plan.counters_off);
-    prm.partials = reinterpret_cast<float *>(ws + plan.partials_off);
     prm.timeout_ns = 2000000000ull;
     prm.scale_log2 = scale * 1.4426950408889634f;
     prm.n_q_heads = n_q_heads;
@@ -367,14 +389,22 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
     prm.ring_bytes = plan.ring_bytes;
     for (const AttnLaunch &L : plan.launches) {
         prm.n_views = L.v1 - L.v0;
-        // Right behind a fused append only the first launch skips the entry
-        // wait (later ones follow this call's own grids).
-        prm.fused = (dep != nullptr && L.v0 == 0) ? 1 : 0;
+        prm.counters = reinterpret_cast<uint32_t *>(ws + L.counters_off);
+        prm.partials = reinterpret_cast<float *>(ws + L.partials_off);
+        // The first launch waits for the preceding work at entry (behind a
+        // fused append: only its blocks that read appended rows wait).  Later
+        // launches of the call start as soon as the one before has released
+        // them, so all run concurrently on their own workspace regions; each
+        // waits for its predecessor before it exits, so the call's last grid
+        // completes after all of them.
+        prm.fused = dep != nullptr ? 1 : 0;
+        prm.chain = L.v0 > 0 ? 1 : 0;
         int begin = 0;
-        for (int i = L.v0; i < L.v1; ++i) {
+        for (int k = L.v0; k < L.v1; ++k) {
+            const int i = plan.order[k];
             const kvq_view &v = views[i];
             const ViewChunks &c = plan.chunks[i];
-            kvq::AttnView &d = prm.views[i - L.v0];
+            kvq::AttnView &d = prm.views[k - L.v0];
             d.codes[0] = static_cast<const uint8_t *>(v.k_codes);
             d.codes[1] = static_cast<const uint8_t *>(v.v_codes);
             d.scalemin[0] = v.k_scalemin;
@@ -632,7 +662,7 @@ KVQ_API kvq_status kvq_decode_attn_noalloc(const kvq_view *views, int32_t n_view
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     // the status word and the arrival counters must start at zero; the
     // partials are written before they are read
-    if (cudaMemsetAsync(scratch, 0, plan.partials_off, st) != cudaSuccess) return KVQ_ERR_CUDA;
+    if (cudaMemsetAsync(scratch, 0, plan.zero_bytes, st) != cudaSuccess) return KVQ_ERR_CUDA;
     return launch_attn(plan, views, n_q_heads, n_kv_heads, head_dim, q, softmax_scale, out,
                        static_cast<uint8_t *>(scratch), st);
 }

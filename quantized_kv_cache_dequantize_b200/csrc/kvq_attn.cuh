@@ -82,6 +82,7 @@ struct AttnParams {
     int32_t head_blocks;         // ceil(group / 8)
     int32_t ring_bytes;          // shared-memory ring per warp
     int32_t fused;               // 1: launched right behind this step's append grid (see dep_step)
+    int32_t chain;               // 1: a later launch of a call: no wait at entry, wait before exit
     AttnView views[kAttnMaxViews];
 };
 
@@ -990,19 +991,17 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
 }
 
 // BSEL = 2, 3, 4 or 8: every view of the launch that has packed tokens has
-// that width, and only that width's code is compiled in; BSEL = 0: any mix of
-// widths, dispatched per CTA.  Specialized kernels keep the instruction
-// footprint of a launch small: with all four widths compiled into one
-// function, about one instruction fetch in five missed the SM's instruction
-// cache on a uniform 4-bit launch, against one in fifty with 4 bits alone.
+// that width, and only that width's code is compiled into the kernel (the
+// host groups the views of a call by width, one launch per group).  With all
+// four widths compiled into one function, about one instruction fetch in
+// five missed the SM's instruction cache, against one in fifty for one width.
 template <int NG, int BSEL>
-__global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
-    decode_attn_kernel(const __grid_constant__ AttnParams p) {
-    extern __shared__ __align__(128) uint8_t smem[];
+__device__ __forceinline__ void decode_attn_body(const AttnParams &p, uint8_t *smem) {
     // Inputs may come from the preceding grid.  Behind a fused append, only
     // the copies of the blocks the append writes wait for it (see dep_step):
     // that grid waited for everything before it and then released this one.
-    if (!p.fused) pdl_wait();
+    // A later launch of a call starts once the one before has released it.
+    if (!p.fused && !p.chain) pdl_wait();
     pdl_launch_dependents();  // the next grid may be scheduled as slots free up (it waits in turn)
     // ---- which item: view by binary search over chunk ranges
     const int bx = blockIdx.x;
@@ -1015,18 +1014,19 @@ __global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
     const int c = bx - V.chunk_begin;
     const int hk = blockIdx.y, z = blockIdx.z;
     if (c >= V.n_chunks) return;  // never launched by the host planner; defensive
-    if (c >= V.n_chunks_packed) {
-        attn_item<NG, 4, true>(p, V, lo, c, hk, z, smem);
-    } else if constexpr (BSEL != 0) {
-        attn_item<NG, BSEL, false>(p, V, lo, c, hk, z, smem);
-    } else {
-        switch (V.bits) {
-            case 2: attn_item<NG, 2, false>(p, V, lo, c, hk, z, smem); break;
-            case 3: attn_item<NG, 3, false>(p, V, lo, c, hk, z, smem); break;
-            case 4: attn_item<NG, 4, false>(p, V, lo, c, hk, z, smem); break;
-            default: attn_item<NG, 8, false>(p, V, lo, c, hk, z, smem); break;
-        }
-    }
+    if (c >= V.n_chunks_packed) attn_item<NG, 4, true>(p, V, lo, c, hk, z, smem);
+    else attn_item<NG, BSEL, false>(p, V, lo, c, hk, z, smem);
+}
+
+template <int NG, int BSEL>
+__global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
+    decode_attn_kernel(const __grid_constant__ AttnParams p) {
+    static_assert(BSEL == 2 || BSEL == 3 || BSEL == 4 || BSEL == 8, "width");
+    extern __shared__ __align__(128) uint8_t smem[];
+    decode_attn_body<NG, BSEL>(p, smem);
+    // a later launch of a call completes only after the one before it, so
+    // the call's last grid completes after all of them
+    if (p.chain) pdl_wait();
 }
 
 }  // namespace kvq
