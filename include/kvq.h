@@ -227,6 +227,74 @@ kvq_status kvq_append_decode_attn(kvq_view *views, int32_t n_views, int32_t n_q_
                                   float *out, void *workspace, size_t workspace_bytes,
                                   void *stream);
 
+/*
+ * CacheCard -- one contiguous artifact holding several views' caches, for
+ * handing them to another agent or process and for persistence
+ * (QKVShare, Metodologia: the CacheCard packs the quantized KV groups, their
+ * width assignment and metadata -- sequence length, model id, position
+ * offset; Agent Memory, Abstract: per-agent 4-bit caches persisted and
+ * reloaded straight into attention).
+ *
+ * Layout (little-endian; version 1):
+ *   [0, 64)          header: "KVQCARD1", u32 version, u32 n_views,
+ *                    u32 n_kv_heads, u32 head_dim, u64 model_id,
+ *                    u64 total_bytes, 24 bytes zero
+ *   [64, 64+64*n)    per view: u32 bits, u32 n_window, u64 n_packed,
+ *                    i64 position_offset, u64 data_offset, u64 data_bytes,
+ *                    u64 seq_len (= n_packed + n_window), 16 bytes zero
+ *   per view, at data_offset (256-byte aligned), six 16-byte-aligned
+ *   sections: K codes [H][n_packed][row_bytes], V codes, K scale/min
+ *   [H][n_packed][head_dim/64][2] fp32, V scale/min, K window
+ *   [H][n_window][head_dim] bf16 oldest first, V window.
+ * Only the used rows travel: a card is independent of the views' capacities
+ * and of where their rings start.
+ */
+
+/* Bytes of the card of these views (0 when the arguments are invalid). */
+size_t kvq_card_bytes(const kvq_view *views, int32_t n_views, int32_t n_kv_heads,
+                      int32_t head_dim);
+
+/*
+ * kvq_card_pack -- write the card of n_views views into DEVICE memory `card`
+ * (256-byte aligned, at least kvq_card_bytes bytes), on `stream`; copy it to
+ * the host with cudaMemcpyAsync for transfer or storage.
+ *  model_id           stored in the header as given (the caller's tag).
+ *  position_offsets   HOST array of n_views positions of each view's first
+ *                     token, or NULL for zeros.
+ */
+kvq_status kvq_card_pack(const kvq_view *views, int32_t n_views, int32_t n_kv_heads,
+                         int32_t head_dim, uint64_t model_id, const int64_t *position_offsets,
+                         void *card, size_t card_bytes, void *stream);
+
+/*
+ * kvq_card_read_header / kvq_card_view_info -- read a card held in HOST
+ * memory (validated: magic, version, sizes, and every offset where the
+ * layout puts it).  Any output pointer may be NULL.  Use them to allocate
+ * views that can take the card: each view's bits must match the card's and
+ * its capacities must hold n_packed and n_window.
+ */
+kvq_status kvq_card_read_header(const void *card_host, size_t card_bytes, int32_t *n_views,
+                                int32_t *n_kv_heads, int32_t *head_dim, uint64_t *model_id);
+kvq_status kvq_card_view_info(const void *card_host, size_t card_bytes, int32_t index,
+                              int32_t *bits, int64_t *n_packed, int32_t *n_window,
+                              int64_t *position_offset);
+
+/*
+ * kvq_card_unpack -- restore a card into n_views views.  The card's bytes
+ * are given twice: `card_host` (HOST copy, parsed and validated here) and
+ * `card` (DEVICE copy of the same bytes, 256-byte aligned, read by the
+ * kernel).  The views' buffers receive the used rows; their counters are set
+ * from the card (n_packed, n_window; window_head = 0: the window lands in
+ * ring slots 0..n_window-1).
+ * Errors (nothing enqueued, no view changed): KVQ_ERR_INVALID_ARG for a card
+ * that fails validation, counts that differ from the card's, or a view whose
+ * bits differ from its record; KVQ_ERR_CAPACITY when a view cannot hold its
+ * record's tokens.
+ */
+kvq_status kvq_card_unpack(const void *card_host, const void *card, size_t card_bytes,
+                           kvq_view *views, int32_t n_views, int32_t n_kv_heads,
+                           int32_t head_dim, void *stream);
+
 /* Bytes of the per-device scratch array kvq_decode_attn_noalloc uses. */
 #define KVQ_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 

@@ -11,6 +11,8 @@ Entry points (same names as the C ABI, without the ``kvq_`` prefix):
   View, append                  -- one (agent, layer) cache; add a decode token
   decode_attn, workspace_size   -- batched split-K attention over many views
   append_decode_attn            -- one decode step: append, then attend, in one call
+  card_pack, card_unpack, ...   -- CacheCard: several views' caches as one
+                                   artifact (transfer, save_card / load_card)
   decode_attn_noalloc           -- the same without a workspace: scratch is a
                                    fixed per-device array inside the library
                                    (NOALLOC_SCRATCH_BYTES), for callers that
@@ -26,7 +28,8 @@ import torch
 from . import workloads  # noqa: F401  (seeded input generators)
 
 __all__ = ["quantize", "dequantize", "View", "append", "decode_attn", "workspace_size",
-           "append_decode_attn", "step_workspace_size", "decode_attn_noalloc", "NOALLOC_SCRATCH_BYTES", "KvqError", "lib", "row_bytes", "GROUP"]
+           "append_decode_attn", "step_workspace_size", "decode_attn_noalloc",
+           "card_bytes", "card_pack", "card_info", "card_unpack", "views_for_card", "save_card", "load_card", "NOALLOC_SCRATCH_BYTES", "KvqError", "lib", "row_bytes", "GROUP"]
 
 GROUP = 64
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024   # KVQ_NOALLOC_SCRATCH_BYTES in kvq.h
@@ -79,6 +82,17 @@ def lib():
         L.kvq_decode_attn.restype = i32
         L.kvq_append_decode_attn.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, P, P, f32, P, P, sz, P]
         L.kvq_append_decode_attn.restype = i32
+        u64 = ctypes.c_uint64
+        L.kvq_card_bytes.argtypes = [ctypes.POINTER(CView), i32, i32, i32]
+        L.kvq_card_bytes.restype = sz
+        L.kvq_card_pack.argtypes = [ctypes.POINTER(CView), i32, i32, i32, u64, P, P, sz, P]
+        L.kvq_card_pack.restype = i32
+        L.kvq_card_read_header.argtypes = [P, sz, P, P, P, P]
+        L.kvq_card_read_header.restype = i32
+        L.kvq_card_view_info.argtypes = [P, sz, i32, P, P, P, P]
+        L.kvq_card_view_info.restype = i32
+        L.kvq_card_unpack.argtypes = [P, P, sz, ctypes.POINTER(CView), i32, i32, i32, P]
+        L.kvq_card_unpack.restype = i32
         L.kvq_decode_attn_noalloc.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, f32, P, P]
         L.kvq_decode_attn_noalloc.restype = i32
         _lib = L
@@ -330,3 +344,92 @@ def decode_attn_noalloc(views, q: torch.Tensor, softmax_scale: float, out: torch
                                          float(softmax_scale), _ptr(out), _stream(stream)),
            "kvq_decode_attn_noalloc")
     return out
+
+
+# ---------------------------------------------------------- CacheCard -----
+
+def card_bytes(views) -> int:
+    views = list(views)
+    return int(lib().kvq_card_bytes(_view_array(views), len(views), views[0].n_kv_heads, views[0].head_dim))
+
+
+def card_pack(views, model_id: int = 0, position_offsets=None, out: torch.Tensor | None = None,
+              stream=None) -> torch.Tensor:
+    """kvq_card_pack: the card of these views as a DEVICE uint8 tensor."""
+    views = list(views)
+    n = card_bytes(views)
+    if n == 0:
+        raise KvqError(KVQ_ERR_INVALID_ARG, "kvq_card_bytes")
+    dev = views[0].k_codes.device
+    if out is None:
+        out = torch.empty(n, dtype=torch.uint8, device=dev)
+    pos = None
+    if position_offsets is not None:
+        pos = (ctypes.c_int64 * len(views))(*[int(x) for x in position_offsets])
+    _check(lib().kvq_card_pack(_view_array(views), len(views), views[0].n_kv_heads, views[0].head_dim,
+                               int(model_id), ctypes.cast(pos, ctypes.c_void_p) if pos is not None else None,
+                               _ptr(out), out.numel(), _stream(stream)), "kvq_card_pack")
+    return out
+
+
+def card_info(card_host: torch.Tensor) -> dict:
+    """Header and per-view records of a card held in host memory."""
+    if card_host.is_cuda:
+        raise ValueError("card_info reads a host copy of the card")
+    card_host = card_host.contiguous()
+    nv, hk, d = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32()
+    mid = ctypes.c_uint64()
+    _check(lib().kvq_card_read_header(_ptr(card_host), card_host.numel(), ctypes.byref(nv), ctypes.byref(hk),
+                                      ctypes.byref(d), ctypes.byref(mid)), "kvq_card_read_header")
+    recs = []
+    for i in range(nv.value):
+        b, w = ctypes.c_int32(), ctypes.c_int32()
+        p, off = ctypes.c_int64(), ctypes.c_int64()
+        _check(lib().kvq_card_view_info(_ptr(card_host), card_host.numel(), i, ctypes.byref(b), ctypes.byref(p),
+                                        ctypes.byref(w), ctypes.byref(off)), "kvq_card_view_info")
+        recs.append(dict(bits=b.value, n_packed=p.value, n_window=w.value, position_offset=off.value))
+    return dict(n_views=nv.value, n_kv_heads=hk.value, head_dim=d.value, model_id=mid.value, views=recs)
+
+
+def views_for_card(card_host: torch.Tensor, cap_window: int | None = None, extra_packed: int = 0,
+                   device="cuda") -> list:
+    """Fresh views that can take the card: each view's width from its record,
+    capacity for its tokens (plus extra_packed rows; window capacity
+    cap_window, default the record's n_window)."""
+    info = card_info(card_host)
+    out = []
+    for r in info["views"]:
+        W = r["n_window"] if cap_window is None else cap_window
+        out.append(View(info["n_kv_heads"], info["head_dim"], r["bits"], max(2, r["n_packed"] + extra_packed), W,
+                        device=device))
+    return out
+
+
+def card_unpack(card_host: torch.Tensor, views, card: torch.Tensor | None = None, stream=None):
+    """kvq_card_unpack: restore the card into views (uploads the host copy
+    when no device copy is given)."""
+    views = list(views)
+    card_host = card_host.contiguous()
+    if card is None:
+        # upload on the stream the kernel runs on
+        s = stream if stream is not None else torch.cuda.current_stream(views[0].k_codes.device)
+        with torch.cuda.stream(s):
+            card = card_host.to(views[0].k_codes.device, non_blocking=True)
+    arr = _view_array(views)
+    _check(lib().kvq_card_unpack(_ptr(card_host), _ptr(card), card_host.numel(), arr, len(views),
+                                 views[0].n_kv_heads, views[0].head_dim, _stream(stream)), "kvq_card_unpack")
+    for i, v in enumerate(views):
+        v.c.n_packed, v.c.n_window, v.c.window_head = arr[i].n_packed, arr[i].n_window, arr[i].window_head
+    return views
+
+
+def save_card(path: str, card: torch.Tensor):
+    """Write a card (device or host tensor) to a file, byte for byte."""
+    card.detach().cpu().numpy().tofile(path)
+
+
+def load_card(path: str, pin: bool = True) -> torch.Tensor:
+    """Read a card file into a host uint8 tensor (pinned for fast upload)."""
+    import numpy as np
+    t = torch.from_numpy(np.fromfile(path, dtype=np.uint8))
+    return t.pin_memory() if pin and torch.cuda.is_available() else t

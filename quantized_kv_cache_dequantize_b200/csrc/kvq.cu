@@ -12,6 +12,7 @@
 
 #include "kvq.h"
 #include "kvq_attn.cuh"
+#include "kvq_card.cuh"
 #include "kvq_codec.cuh"
 
 #define KVQ_API extern "C" __attribute__((visibility("default")))
@@ -538,6 +539,132 @@ void advance_view(kvq_view &v) {
     }
 }
 
+// ------------------------------------------------------------ CacheCard ---
+
+size_t align_up(size_t x, size_t a) { return (x + a - 1) / a * a; }
+
+// Byte layout of a card for these per-view (bits, n_packed, n_window).
+struct CardLayout {
+    size_t total = 0;
+    std::vector<uint64_t> data_off, data_bytes;
+    std::vector<std::vector<uint64_t>> sect;  // six section offsets per view
+};
+
+void card_layout(int32_t n_views, int32_t n_kv_heads, int32_t head_dim, const int32_t *bits, const int64_t *n_packed,
+                 const int32_t *n_window, CardLayout &L) {
+    const int ng = head_dim / 64;
+    size_t off = align_up(sizeof(kvq::CardHeader) + sizeof(kvq::CardView) * (size_t)n_views, 256);
+    L.data_off.resize(n_views);
+    L.data_bytes.resize(n_views);
+    L.sect.assign(n_views, std::vector<uint64_t>(6, 0));
+    for (int i = 0; i < n_views; ++i) {
+        const size_t codes = n_packed[i] > 0 ? (size_t)n_kv_heads * n_packed[i] * row_bytes(head_dim, bits[i]) : 0;
+        const size_t sm = (size_t)n_kv_heads * (size_t)std::max<int64_t>(n_packed[i], 0) * ng * 8;
+        const size_t win = (size_t)n_kv_heads * (size_t)std::max(n_window[i], 0) * head_dim * 2;
+        const size_t sizes[6] = {codes, codes, sm, sm, win, win};
+        L.data_off[i] = off;
+        for (int k = 0; k < 6; ++k) {
+            L.sect[i][k] = off;
+            off = align_up(off + sizes[k], 16);
+        }
+        L.data_bytes[i] = off - L.data_off[i];
+        off = align_up(off, 256);
+    }
+    L.total = off;
+}
+
+void card_layout_of_views(const kvq_view *views, int32_t n_views, int32_t n_kv_heads, int32_t head_dim,
+                          CardLayout &L) {
+    std::vector<int32_t> b(n_views), w(n_views);
+    std::vector<int64_t> p(n_views);
+    for (int i = 0; i < n_views; ++i) {
+        b[i] = views[i].bits;
+        p[i] = views[i].n_packed;
+        w[i] = views[i].n_window;
+    }
+    card_layout(n_views, n_kv_heads, head_dim, b.data(), p.data(), w.data(), L);
+}
+
+kvq_status card_launch(bool pack, const kvq_view *views, int32_t n_views, int32_t n_kv_heads, int32_t head_dim,
+                       const CardLayout &L, const kvq::CardHeader *header, const int64_t *position_offsets,
+                       uint8_t *card, cudaStream_t st) {
+    for (int v0 = 0; v0 < n_views; v0 += kvq::kCardMaxViews) {
+        const int v1 = std::min<int>(n_views, v0 + kvq::kCardMaxViews);
+        kvq::CardArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.card = card;
+        a.n_views = v1 - v0;
+        a.n_kv_heads = n_kv_heads;
+        a.head_dim = head_dim;
+        a.write_header = (pack && v0 == 0) ? 1 : 0;
+        if (header) a.header = *header;
+        a.records_off = sizeof(kvq::CardHeader) + sizeof(kvq::CardView) * (uint64_t)v0;
+        for (int i = v0; i < v1; ++i) {
+            const kvq_view &v = views[i];
+            kvq::CardSide &d = a.views[i - v0];
+            d.codes[0] = static_cast<uint8_t *>(v.k_codes);
+            d.codes[1] = static_cast<uint8_t *>(v.v_codes);
+            d.scalemin[0] = v.k_scalemin;
+            d.scalemin[1] = v.v_scalemin;
+            d.window[0] = static_cast<uint16_t *>(v.k_window);
+            d.window[1] = static_cast<uint16_t *>(v.v_window);
+            d.cap_packed = v.cap_packed;
+            d.n_packed = v.n_packed;
+            d.cap_window = v.cap_window;
+            d.n_window = v.n_window;
+            d.window_head = pack ? v.window_head : 0;
+            d.row_bytes = v.n_packed > 0 ? (int32_t)row_bytes(head_dim, v.bits) : 0;
+            for (int k = 0; k < 6; ++k) d.sect_off[k] = L.sect[i][k];
+            d.record.bits = (uint32_t)v.bits;
+            d.record.n_window = (uint32_t)v.n_window;
+            d.record.n_packed = (uint64_t)v.n_packed;
+            d.record.position_offset = position_offsets ? position_offsets[i] : 0;
+            d.record.data_offset = L.data_off[i];
+            d.record.data_bytes = L.data_bytes[i];
+            d.record.seq_len = (uint64_t)v.n_packed + (uint64_t)v.n_window;
+        }
+        const dim3 grid((unsigned)(v1 - v0), (unsigned)n_kv_heads, 6);
+        if (pack) kvq::card_kernel<true><<<grid, 256, 0, st>>>(a);
+        else kvq::card_kernel<false><<<grid, 256, 0, st>>>(a);
+        if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+    }
+    return KVQ_OK;
+}
+
+// Validate a card held in host memory; fills its header and records.
+kvq_status card_parse(const void *card_host, size_t card_bytes, kvq::CardHeader &h,
+                      std::vector<kvq::CardView> &recs) {
+    if (!card_host || card_bytes < sizeof(kvq::CardHeader)) return KVQ_ERR_INVALID_ARG;
+    std::memcpy(&h, card_host, sizeof h);
+    if (std::memcmp(h.magic, "KVQCARD1", 8) != 0 || h.version != kvq::kCardVersion) return KVQ_ERR_INVALID_ARG;
+    if (!head_dim_supported((int32_t)h.head_dim)) return KVQ_ERR_UNSUPPORTED;
+    if (h.n_views == 0 || h.n_views > (1u << 24) || h.n_kv_heads == 0 || h.n_kv_heads > 65535)
+        return KVQ_ERR_INVALID_ARG;
+    const size_t rec_end = sizeof(kvq::CardHeader) + sizeof(kvq::CardView) * (size_t)h.n_views;
+    if (h.total_bytes > card_bytes || rec_end > h.total_bytes) return KVQ_ERR_INVALID_ARG;
+    recs.resize(h.n_views);
+    std::memcpy(recs.data(), static_cast<const uint8_t *>(card_host) + sizeof(kvq::CardHeader),
+                sizeof(kvq::CardView) * (size_t)h.n_views);
+    std::vector<int32_t> b(h.n_views), w(h.n_views);
+    std::vector<int64_t> p(h.n_views);
+    for (uint32_t i = 0; i < h.n_views; ++i) {
+        const kvq::CardView &r = recs[i];
+        if (r.n_packed > (uint64_t)INT32_MAX || r.n_window > (uint32_t)INT32_MAX) return KVQ_ERR_INVALID_ARG;
+        if (r.n_packed > 0 && !bits_supported((int32_t)r.bits)) return KVQ_ERR_UNSUPPORTED;
+        if (r.seq_len != r.n_packed + r.n_window) return KVQ_ERR_INVALID_ARG;
+        b[i] = (int32_t)r.bits;
+        p[i] = (int64_t)r.n_packed;
+        w[i] = (int32_t)r.n_window;
+    }
+    // the data must sit exactly where this version's layout puts it
+    CardLayout L;
+    card_layout((int32_t)h.n_views, (int32_t)h.n_kv_heads, (int32_t)h.head_dim, b.data(), p.data(), w.data(), L);
+    if (L.total != h.total_bytes) return KVQ_ERR_INVALID_ARG;
+    for (uint32_t i = 0; i < h.n_views; ++i)
+        if (recs[i].data_offset != L.data_off[i] || recs[i].data_bytes != L.data_bytes[i]) return KVQ_ERR_INVALID_ARG;
+    return KVQ_OK;
+}
+
 // ------------------------------------------- fixed scratch (no allocation) ---
 
 // Scratch of kvq_decode_attn_noalloc: one array per device, laid out like a
@@ -701,4 +828,96 @@ KVQ_API kvq_status kvq_append_decode_attn(kvq_view *views, int32_t n_views, int3
         case 3: return launch_attn_ng<3>(plan, post.data(), n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st, dep.data());
         default: return launch_attn_ng<4>(plan, post.data(), n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st, dep.data());
     }
+}
+
+KVQ_API size_t kvq_card_bytes(const kvq_view *views, int32_t n_views, int32_t n_kv_heads, int32_t head_dim) {
+    if (!head_dim_supported(head_dim) || n_kv_heads <= 0 || n_kv_heads > 65535) return 0;
+    if (validate_views(views, n_views, false) != KVQ_OK) return 0;
+    CardLayout L;
+    card_layout_of_views(views, n_views, n_kv_heads, head_dim, L);
+    return L.total;
+}
+
+KVQ_API kvq_status kvq_card_pack(const kvq_view *views, int32_t n_views, int32_t n_kv_heads, int32_t head_dim,
+                                 uint64_t model_id, const int64_t *position_offsets, void *card, size_t card_bytes,
+                                 void *stream) {
+    if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
+    if (n_kv_heads <= 0 || n_kv_heads > 65535) return KVQ_ERR_INVALID_ARG;
+    const kvq_status vs = validate_views(views, n_views, false);
+    if (vs != KVQ_OK) return vs;
+    if (!card || !aligned(card, 256)) return KVQ_ERR_INVALID_ARG;
+    CardLayout L;
+    card_layout_of_views(views, n_views, n_kv_heads, head_dim, L);
+    if (card_bytes < L.total) return KVQ_ERR_INVALID_ARG;
+    kvq::CardHeader h;
+    std::memset(&h, 0, sizeof h);
+    std::memcpy(h.magic, "KVQCARD1", 8);
+    h.version = kvq::kCardVersion;
+    h.n_views = (uint32_t)n_views;
+    h.n_kv_heads = (uint32_t)n_kv_heads;
+    h.head_dim = (uint32_t)head_dim;
+    h.model_id = model_id;
+    h.total_bytes = L.total;
+    return card_launch(true, views, n_views, n_kv_heads, head_dim, L, &h, position_offsets,
+                       static_cast<uint8_t *>(card), static_cast<cudaStream_t>(stream));
+}
+
+KVQ_API kvq_status kvq_card_read_header(const void *card_host, size_t card_bytes, int32_t *n_views,
+                                        int32_t *n_kv_heads, int32_t *head_dim, uint64_t *model_id) {
+    kvq::CardHeader h;
+    std::vector<kvq::CardView> recs;
+    const kvq_status ps = card_parse(card_host, card_bytes, h, recs);
+    if (ps != KVQ_OK) return ps;
+    if (n_views) *n_views = (int32_t)h.n_views;
+    if (n_kv_heads) *n_kv_heads = (int32_t)h.n_kv_heads;
+    if (head_dim) *head_dim = (int32_t)h.head_dim;
+    if (model_id) *model_id = h.model_id;
+    return KVQ_OK;
+}
+
+KVQ_API kvq_status kvq_card_view_info(const void *card_host, size_t card_bytes, int32_t index, int32_t *bits,
+                                      int64_t *n_packed, int32_t *n_window, int64_t *position_offset) {
+    kvq::CardHeader h;
+    std::vector<kvq::CardView> recs;
+    const kvq_status ps = card_parse(card_host, card_bytes, h, recs);
+    if (ps != KVQ_OK) return ps;
+    if (index < 0 || (uint32_t)index >= h.n_views) return KVQ_ERR_INVALID_ARG;
+    const kvq::CardView &r = recs[index];
+    if (bits) *bits = (int32_t)r.bits;
+    if (n_packed) *n_packed = (int64_t)r.n_packed;
+    if (n_window) *n_window = (int32_t)r.n_window;
+    if (position_offset) *position_offset = r.position_offset;
+    return KVQ_OK;
+}
+
+KVQ_API kvq_status kvq_card_unpack(const void *card_host, const void *card, size_t card_bytes, kvq_view *views,
+                                   int32_t n_views, int32_t n_kv_heads, int32_t head_dim, void *stream) {
+    kvq::CardHeader h;
+    std::vector<kvq::CardView> recs;
+    const kvq_status ps = card_parse(card_host, card_bytes, h, recs);
+    if (ps != KVQ_OK) return ps;
+    if (!card || !aligned(card, 256)) return KVQ_ERR_INVALID_ARG;
+    if (n_views != (int32_t)h.n_views || n_kv_heads != (int32_t)h.n_kv_heads || head_dim != (int32_t)h.head_dim)
+        return KVQ_ERR_INVALID_ARG;
+    // the views as they will be: the card's counts, window from slot 0
+    std::vector<kvq_view> post(views, views + n_views);
+    for (int i = 0; i < n_views; ++i) {
+        const kvq::CardView &r = recs[i];
+        kvq_view &v = post[i];
+        if (r.n_packed > 0 && v.bits != (int32_t)r.bits) return KVQ_ERR_INVALID_ARG;  // rows are laid out per width
+        if ((int64_t)r.n_packed > v.cap_packed || (int32_t)r.n_window > v.cap_window) return KVQ_ERR_CAPACITY;
+        v.n_packed = (int64_t)r.n_packed;
+        v.n_window = (int32_t)r.n_window;
+        v.window_head = 0;
+    }
+    const kvq_status vs = validate_views(post.data(), n_views, false);
+    if (vs != KVQ_OK) return vs;
+    CardLayout L;
+    card_layout_of_views(post.data(), n_views, n_kv_heads, head_dim, L);
+    const kvq_status ls = card_launch(false, post.data(), n_views, n_kv_heads, head_dim, L, nullptr, nullptr,
+                                      const_cast<uint8_t *>(static_cast<const uint8_t *>(card)),
+                                      static_cast<cudaStream_t>(stream));
+    if (ls != KVQ_OK) return ls;
+    for (int i = 0; i < n_views; ++i) views[i] = post[i];
+    return KVQ_OK;
 }
