@@ -623,7 +623,22 @@ kvq_status card_launch(bool pack, const kvq_view *views, int32_t n_views, int32_
             d.record.data_bytes = L.data_bytes[i];
             d.record.seq_len = (uint64_t)v.n_packed + (uint64_t)v.n_window;
         }
-        const dim3 grid((unsigned)(v1 - v0), (unsigned)n_kv_heads, 6);
+        // one CTA per piece of every (view, section), views in order
+        uint64_t ctas = 0;
+        for (int i = v0; i < v1; ++i) {
+            const kvq_view &v = views[i];
+            const int64_t rows[6] = {v.n_packed, v.n_packed, v.n_packed, v.n_packed, v.n_window, v.n_window};
+            const int64_t row[6] = {a.views[i - v0].row_bytes, a.views[i - v0].row_bytes, (int64_t)(head_dim / 64) * 8,
+                                    (int64_t)(head_dim / 64) * 8, (int64_t)head_dim * 2, (int64_t)head_dim * 2};
+            for (int k = 0; k < 6; ++k) {
+                a.entry_cta[(i - v0) * 6 + k] = (uint32_t)ctas;
+                if (rows[k] > 0) ctas += (uint64_t)n_kv_heads * (uint64_t)kvq::card_pieces_per_head(rows[k], row[k]);
+            }
+        }
+        if (ctas > (uint64_t)INT32_MAX) return KVQ_ERR_INVALID_ARG;
+        a.entry_cta[(v1 - v0) * 6] = (uint32_t)ctas;
+        const unsigned grid = (unsigned)std::max<uint64_t>(ctas, pack ? 1 : 0);
+        if (grid == 0) continue;
         if (pack) kvq::card_kernel<true><<<grid, 256, 0, st>>>(a);
         else kvq::card_kernel<false><<<grid, 256, 0, st>>>(a);
         if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;

@@ -64,6 +64,20 @@ struct CardSide {
     CardView record;          // written by pack
 };
 
+// Sections are cut into pieces of whole rows of one KV head, about
+// kCardPieceBytes each; one CTA copies one piece.  Host and kernel both derive
+// a section's piece count from its row size with these two functions.
+constexpr int64_t kCardPieceBytes = 32 * 1024;
+constexpr int kCardSections = 6;
+
+__host__ __device__ inline int64_t card_piece_rows(int64_t row) {
+    return row >= kCardPieceBytes ? 1 : kCardPieceBytes / row;
+}
+__host__ __device__ inline int64_t card_pieces_per_head(int64_t rows, int64_t row) {
+    const int64_t r = card_piece_rows(row);
+    return (rows + r - 1) / r;
+}
+
 struct CardArgs {
     uint8_t *card;            // device card image
     int32_t n_views;
@@ -72,52 +86,87 @@ struct CardArgs {
     int32_t write_header;     // pack: this launch also writes the card header
     CardHeader header;
     uint64_t records_off;     // card offset of this launch's first record
+    // first CTA of each (view, section) entry, entry = view * 6 + section;
+    // entry_cta[6 * n_views] is the number of copying CTAs
+    uint32_t entry_cta[kCardMaxViews * kCardSections + 1];
     CardSide views[kCardMaxViews];
 };
 
-// Copy n bytes (multiple of 8, both ends 8-byte aligned) with one CTA.
-__device__ __forceinline__ void cta_copy8(uint8_t *dst, const uint8_t *src, int64_t n) {
-    const uint2 *s = reinterpret_cast<const uint2 *>(src);
-    uint2 *d = reinterpret_cast<uint2 *>(dst);
-    const int64_t n8 = n >> 3;
-    for (int64_t i = threadIdx.x; i < n8; i += blockDim.x) __stcs(d + i, __ldcs(s + i));
+// Copy n bytes from src to dst with one CTA, T-sized accesses (n and both
+// addresses multiples of sizeof(T)); four loads in flight per thread.
+template <typename T>
+__device__ __forceinline__ void cta_copy(uint8_t *dst, const uint8_t *src, int64_t n) {
+    const T *s = reinterpret_cast<const T *>(src);
+    T *d = reinterpret_cast<T *>(dst);
+    const int64_t nv = n / (int64_t)sizeof(T), bd = blockDim.x;
+    int64_t i = threadIdx.x;
+    for (; i + 3 * bd < nv; i += 4 * bd) {
+        const T a0 = __ldcs(s + i), a1 = __ldcs(s + i + bd), a2 = __ldcs(s + i + 2 * bd), a3 = __ldcs(s + i + 3 * bd);
+        __stcs(d + i, a0);
+        __stcs(d + i + bd, a1);
+        __stcs(d + i + 2 * bd, a2);
+        __stcs(d + i + 3 * bd, a3);
+    }
+    for (; i < nv; i += bd) __stcs(d + i, __ldcs(s + i));
 }
 
-// Grid (view, KV head, section).  PACK: views -> card; otherwise card -> views
-// (the window lands in slots 0 .. n_window-1).
+// Every row size is a multiple of 8 bytes; 16-byte accesses when both ends
+// allow them.
+__device__ __forceinline__ void cta_copy_rows(uint8_t *dst, const uint8_t *src, int64_t n) {
+    if (((reinterpret_cast<uintptr_t>(dst) | reinterpret_cast<uintptr_t>(src) | (uintptr_t)n) & 15) == 0)
+        cta_copy<uint4>(dst, src, n);
+    else
+        cta_copy<uint2>(dst, src, n);
+}
+
+// One CTA per piece.  PACK: views -> card (CTA 0 also writes this launch's
+// records and, on the first launch, the header); otherwise card -> views, the
+// window landing in slots 0 .. n_window-1.
 template <bool PACK>
-__global__ void __launch_bounds__(256) card_kernel(const __grid_constant__ CardArgs a) {
-    const CardSide &v = a.views[blockIdx.x];
-    const int h = blockIdx.y, sect = blockIdx.z;
-    const int D = a.head_dim, NG = D / 64;
-    if (PACK && threadIdx.x == 0 && h == 0 && sect == 0) {
-        reinterpret_cast<CardView *>(a.card + a.records_off)[blockIdx.x] = v.record;
-        if (a.write_header && blockIdx.x == 0) *reinterpret_cast<CardHeader *>(a.card) = a.header;
+__global__ void __launch_bounds__(256, 4) card_kernel(const __grid_constant__ CardArgs a) {
+    if (PACK && blockIdx.x == 0) {
+        CardView *rec = reinterpret_cast<CardView *>(a.card + a.records_off);
+        for (int i = threadIdx.x; i < a.n_views; i += blockDim.x) rec[i] = a.views[i].record;
+        if (a.write_header && threadIdx.x == 0) *reinterpret_cast<CardHeader *>(a.card) = a.header;
     }
-    const int kv = sect & 1;
-    if (sect < 4) {
-        // packed rows of head h: contiguous in the view and in the card
-        const bool codes = sect < 2;
-        const int64_t row = codes ? v.row_bytes : (int64_t)NG * 8;
-        const int64_t n = v.n_packed * row;
-        uint8_t *view_p = codes ? v.codes[kv] + (int64_t)h * v.cap_packed * row
-                                : reinterpret_cast<uint8_t *>(v.scalemin[kv]) + (int64_t)h * v.cap_packed * row;
-        uint8_t *card_p = a.card + v.sect_off[sect] + (int64_t)h * n;
-        if (PACK) cta_copy8(card_p, view_p, n);
-        else cta_copy8(view_p, card_p, n);
+    const uint32_t cta = blockIdx.x;
+    const int n_entries = a.n_views * kCardSections;
+    if (cta >= a.entry_cta[n_entries]) return;
+    // the entry holding this CTA: the last one whose first CTA is <= cta
+    int lo = 0, hi = n_entries - 1;
+    while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (a.entry_cta[mid] <= cta) lo = mid;
+        else hi = mid - 1;
+    }
+    const CardSide &v = a.views[lo / kCardSections];
+    const int sect = lo % kCardSections, kv = sect & 1;
+    const int D = a.head_dim;
+    const bool window = sect >= 4;
+    const int64_t row = sect < 2 ? v.row_bytes : sect < 4 ? (int64_t)(D / 64) * 8 : (int64_t)D * 2;
+    const int64_t rows = window ? v.n_window : v.n_packed;
+    const int64_t pph = card_pieces_per_head(rows, row);
+    const int64_t local = cta - a.entry_cta[lo];
+    const int64_t h = local / pph, r0 = (local % pph) * card_piece_rows(row);
+    const int64_t r1 = min(rows, r0 + card_piece_rows(row));
+    uint8_t *card_p = a.card + v.sect_off[sect] + (h * rows + r0) * row;
+    if (!window) {
+        uint8_t *base = sect < 2 ? v.codes[kv] : reinterpret_cast<uint8_t *>(v.scalemin[kv]);
+        uint8_t *view_p = base + (h * v.cap_packed + r0) * row;
+        if (PACK) cta_copy_rows(card_p, view_p, (r1 - r0) * row);
+        else cta_copy_rows(view_p, card_p, (r1 - r0) * row);
     } else {
-        // window rows of head h: the ring's logical order (two pieces when it wraps)
-        if (v.n_window == 0) return;
-        const int64_t row = (int64_t)D * 2;
-        uint8_t *ring = reinterpret_cast<uint8_t *>(v.window[kv]) + (int64_t)h * v.cap_window * row;
-        uint8_t *card_p = a.card + v.sect_off[sect] + (int64_t)h * v.n_window * row;
-        const int first = min(v.n_window, v.cap_window - v.window_head);
+        // logical rows r0..r1 of the ring: slots (window_head + r) mod cap, at
+        // most two contiguous runs
+        uint8_t *ring = reinterpret_cast<uint8_t *>(v.window[kv]) + h * v.cap_window * row;
+        const int64_t s0 = (v.window_head + r0) % v.cap_window;
+        const int64_t first = min(r1 - r0, (int64_t)v.cap_window - s0);
         if (PACK) {
-            cta_copy8(card_p, ring + (int64_t)v.window_head * row, first * row);
-            if (first < v.n_window) cta_copy8(card_p + first * row, ring, (v.n_window - first) * row);
+            cta_copy_rows(card_p, ring + s0 * row, first * row);
+            if (first < r1 - r0) cta_copy_rows(card_p + first * row, ring, (r1 - r0 - first) * row);
         } else {
-            cta_copy8(ring + (int64_t)v.window_head * row, card_p, first * row);
-            if (first < v.n_window) cta_copy8(ring, card_p + first * row, (v.n_window - first) * row);
+            cta_copy_rows(ring + s0 * row, card_p, first * row);
+            if (first < r1 - r0) cta_copy_rows(ring, card_p + first * row, (r1 - r0 - first) * row);
         }
     }
 }

@@ -12,6 +12,14 @@ CASE:
   quantize-handoff / dequantize-handoff
                  the bulk handoff's K cache: 32 layers x 8 kv heads x 32768
                  tokens x 128 (2 GiB bf16), 1% outlier channels x10
+  card-pack / card-unpack
+                 kvq_card_pack of one agent's whole cache in Llama-3.1-8B
+                 shape (32 layers x 8 kv heads, 32640 packed 4-bit tokens +
+                 a full 128-token window), and kvq_card_unpack of that card
+                 into fresh views
+  card-pack-decode
+                 kvq_card_pack of every view of the batched decode workload
+                 (10 agents x 32 layers, 4096 packed + 128 window)
 Each case runs 3 warm-up calls, captures one call in a CUDA graph, replays
 it once more and then --reps timed times, and prints the mean time per call
 and the algorithmic GB/s.
@@ -25,7 +33,7 @@ import torch
 
 from . import cache as kcache
 from . import workloads as wl
-from . import decode_attn, dequantize, new_workspace, quantize
+from . import card_info, card_pack, card_unpack, decode_attn, dequantize, new_workspace, quantize, views_for_card
 
 
 def _time(fn, reps):
@@ -54,11 +62,26 @@ def _time(fn, reps):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["decode-layer", "decode-8layers", "quantize", "dequantize", "quantize-handoff",
-                                         "dequantize-handoff"])
+                                         "dequantize-handoff", "card-pack", "card-unpack", "card-pack-decode"])
     ap.add_argument("--reps", type=int, default=20)
     a = ap.parse_args(argv)
     dev = torch.device("cuda:0")
-    if a.case.startswith("decode"):
+    if a.case.startswith("card"):
+        w = (wl.decode_llama8b(n_agents=1, length=32768 - 128) if a.case != "card-pack-decode"
+             else wl.decode_llama8b())
+        pool = kcache.build_decode(w, dev)
+        card = card_pack(pool.views)
+        host = card.cpu()
+        # bytes moved: every section read once and written once
+        H, D = w.n_kv_heads, w.head_dim
+        nbytes = 2 * sum(2 * H * (r["n_packed"] * (D * r["bits"] // 8 + D // 64 * 8) + r["n_window"] * D * 2)
+                         for r in card_info(host)["views"])
+        if a.case == "card-unpack":
+            fresh = views_for_card(host, device=dev)
+            t = _time(lambda: card_unpack(host, fresh, card=card, stream=torch.cuda.current_stream()), a.reps)
+        else:
+            t = _time(lambda: card_pack(pool.views, out=card, stream=torch.cuda.current_stream()), a.reps)
+    elif a.case.startswith("decode"):
         w = wl.decode_llama8b(n_layers=1 if a.case == "decode-layer" else 8)
         pool = kcache.build_decode(w, dev)
         q = kcache.decode_queries(w, device=dev)
