@@ -193,6 +193,60 @@ def decode_attn(q: np.ndarray, bits: int,
     return (out, probs) if want_probs else out
 
 
+def _bf16_to_f64(bits_u16: np.ndarray) -> np.ndarray:
+    """bf16 bit patterns -> their exact fp64 values (a bf16 is the top half of an fp32)."""
+    return (_c(bits_u16, np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+def decode_attn_segments(q: np.ndarray, segments, softmax_scale: float) -> np.ndarray:
+    """Decode attention of one sequence whose tokens are held by several
+    segments, each with its own width, in fp64.
+
+    Sources: "Coordinated Mixed-Precision KV Cache Quantization ..." (Abstract:
+    only newly quantized blocks take a new allocation, old ones keep theirs)
+    and "QKVShare ..." (Metodologia: per-token widths {2, 4, 8, FP16}).
+    Reading: the sequence's cache is the union of its segments' (key, value)
+    pairs, the packed ones attended as their exact affine values mn + s*c and
+    the window ones as bf16; softmax attention depends on that set only, not on
+    where each pair sits.  So this is textbook softmax attention over the
+    segments' rows concatenated: logits = scale * K q, p = softmax(logits),
+    out = p V, with query head h reading KV head h // (Hq / Hkv).
+
+    q: uint16 bf16 [H_q][D].  segments: list of dicts with "bits" and any of
+    k_codes/v_codes (uint8 [H_kv][n_p][rb]), k_sm/v_sm (float32
+    [H_kv][n_p][D/64][2]), k_win/v_win (uint16 bf16 [H_kv][n_w][D], oldest
+    first); missing or zero-length parts hold no tokens.  Returns float64
+    [H_q][D].
+    """
+    q = _c(q, np.uint16)
+    Hq, D = q.shape
+    ks, vs = [], []
+    for seg in segments:
+        kc = seg.get("k_codes")
+        if kc is not None and kc.shape[1] > 0:
+            ks.append(affine(kc, seg["k_sm"], D, seg["bits"]))
+            vs.append(affine(seg["v_codes"], seg["v_sm"], D, seg["bits"]))
+        kw = seg.get("k_win")
+        if kw is not None and kw.shape[1] > 0:
+            ks.append(_bf16_to_f64(kw))
+            vs.append(_bf16_to_f64(seg["v_win"]))
+    if not ks:
+        raise ValueError("empty sequence")
+    k = np.concatenate(ks, axis=1)
+    v = np.concatenate(vs, axis=1)
+    Hkv = k.shape[0]
+    if Hq % Hkv:
+        raise ValueError("n_q_heads must be a multiple of n_kv_heads")
+    G = Hq // Hkv
+    qd = _bf16_to_f64(q)
+    out = np.zeros((Hq, D), np.float64)
+    for h in range(Hq):
+        logits = softmax_scale * (k[h // G] @ qd[h])
+        w = np.exp(logits - logits.max())
+        out[h] = (w / w.sum()) @ v[h // G]
+    return out
+
+
 class WindowModel:
     """Bookkeeping model of one view's token placement under appends.
 

@@ -407,6 +407,77 @@ def test_key_and_value_roles_are_not_swapped():
     assert kp.shape[1] == 1
 
 
+# ------------------------------------------- sequences of several views ---
+
+def seg_of(view, rows=None, window=True, bits=None):
+    """A segment dict holding the packed rows `rows` (a slice) of a view and,
+    optionally, its window."""
+    rows = slice(0, view["k_codes"].shape[1]) if rows is None else rows
+    seg = dict(bits=view["bits"] if bits is None else bits)
+    for key in ("k_codes", "k_sm", "v_codes", "v_sm"):
+        seg[key] = view[key][:, rows]
+    if window:
+        seg["k_win"], seg["v_win"] = view["k_win"], view["v_win"]
+    return seg
+
+
+def test_one_segment_is_the_view_attention():
+    view = make_view(21, n_p=45, n_w=6)
+    got = oracle.decode_attn_segments(view["q"], [seg_of(view)], 1 / 8)
+    np.testing.assert_allclose(got, run(view, 1 / 8), rtol=1e-13, atol=1e-14)
+
+
+@pytest.mark.parametrize("cut", [1, 17, 44])
+def test_view_split_into_segments_changes_nothing(cut):
+    # the packed rows cut in two segments (the window with the second): the
+    # union of tokens is the view's, so is the attention
+    view = make_view(22, n_p=45, n_w=6)
+    segs = [seg_of(view, slice(0, cut), window=False), seg_of(view, slice(cut, 45))]
+    got = oracle.decode_attn_segments(view["q"], segs, 1 / 8)
+    np.testing.assert_allclose(got, run(view, 1 / 8), rtol=1e-12, atol=1e-13)
+    # and the window as a segment of its own, listed first
+    only_win = dict(bits=4, k_win=view["k_win"], v_win=view["v_win"])
+    segs = [only_win, seg_of(view, slice(0, cut), window=False), seg_of(view, slice(cut, 45), window=False)]
+    np.testing.assert_allclose(oracle.decode_attn_segments(view["q"], segs, 1 / 8), run(view, 1 / 8),
+                               rtol=1e-12, atol=1e-13)
+
+
+def test_segments_of_different_widths_match_brute_force_and_order():
+    # three widths and a bf16-only segment; textbook softmax over all rows
+    from scipy.special import softmax
+    views = [make_view(30 + b, n_p=20 + 3 * b, n_w=0 if b != 8 else 5, bits=b) for b in (2, 3, 8)]
+    q = views[0]["q"]
+    segs = [seg_of(v, window=v["k_win"].shape[1] > 0) for v in views]
+    got = oracle.decode_attn_segments(q, segs, 0.15)
+    ks, vs = zip(*[dense_kv(v) for v in views])
+    k, v = np.concatenate(ks, axis=1), np.concatenate(vs, axis=1)
+    qd = bf16_to_f64(q)
+    for h in range(4):
+        p = softmax(0.15 * (k[h // 2] @ qd[h]))
+        np.testing.assert_allclose(got[h], p @ v[h // 2], rtol=1e-12, atol=1e-13)
+    rev = oracle.decode_attn_segments(q, segs[::-1], 0.15)
+    np.testing.assert_allclose(rev, got, rtol=1e-12, atol=1e-13)
+    # a dropped segment changes the result
+    assert not np.allclose(oracle.decode_attn_segments(q, segs[:2], 0.15), got, atol=1e-6)
+
+
+def test_identical_keys_over_segments_give_mean_of_all_values():
+    # every key zero (code 0, s = mn = 0) in every segment: all logits equal,
+    # so the output is the plain mean of all segments' values
+    views = [make_view(40 + b, n_p=11 + b, n_w=3, bits=b) for b in (2, 4)]
+    segs = []
+    for v in views:
+        seg = seg_of(v)
+        seg["k_codes"] = np.zeros_like(seg["k_codes"])
+        seg["k_sm"] = np.zeros_like(seg["k_sm"])
+        seg["k_win"] = np.zeros_like(seg["k_win"])
+        segs.append(seg)
+    got = oracle.decode_attn_segments(views[0]["q"], segs, 0.3)
+    vals = np.concatenate([dense_kv(v)[1] for v in views], axis=1)
+    for h in range(4):
+        np.testing.assert_allclose(got[h], vals[h // 2].mean(axis=0), rtol=1e-12, atol=1e-13)
+
+
 # --------------------------------------------------------- window model ---
 
 @pytest.mark.parametrize("W", [0, 1, 4, 7])
