@@ -203,6 +203,56 @@ kvq_status kvq_decode_attn(const kvq_view *views, int32_t n_views, int32_t n_q_h
                            size_t workspace_bytes, void *stream);
 
 /*
+ * Sequences made of several views (segments).  A sequence's cache may be held
+ * by more than one view, each with its own width: blocks flushed before and
+ * after a change of the layer's width (CoMixKV, Abstract: only newly quantized
+ * blocks take the new allocation, old ones are not requantized), or tokens of
+ * one sequence kept at different widths by importance (QKVShare, Metodologia:
+ * per-token widths {2, 4, 8, FP16}; FP16 tokens are a view with a window only).
+ * Softmax attention does not depend on the order of the (key, value) pairs,
+ * so the sequence's output is attention over the union of its views' tokens.
+ *
+ * KVQ_MAX_SEGMENTS: views holding tokens, per sequence.
+ */
+#define KVQ_MAX_SEGMENTS 64
+
+/*
+ * kvq_decode_attn_seq_workspace_size -- scratch bytes kvq_decode_attn_seq
+ * needs for these views and sequences; 0 if the arguments are invalid.
+ */
+size_t kvq_decode_attn_seq_workspace_size(const kvq_view *views, int32_t n_views,
+                                          const int32_t *seq_begin, int32_t n_seqs,
+                                          int32_t n_q_heads, int32_t n_kv_heads,
+                                          int32_t head_dim);
+
+/*
+ * kvq_decode_attn_seq -- kvq_decode_attn over sequences of views.
+ *
+ *  views      HOST array of n_views views; a view may be empty (no tokens).
+ *  seq_begin  HOST int32 [n_seqs + 1]: sequence s is views seq_begin[s] ..
+ *             seq_begin[s+1]-1.  seq_begin[0] == 0, seq_begin[n_seqs] ==
+ *             n_views, strictly increasing; every sequence holds >= 1 token
+ *             and at most KVQ_MAX_SEGMENTS non-empty views.  Views of any
+ *             widths may share a sequence.
+ *  q          bf16 [n_seqs][n_q_heads][head_dim] device array, 16-B aligned.
+ *  out        float [n_seqs][n_q_heads][head_dim], 16-B aligned: attention of
+ *             q[s] over the tokens of all views of sequence s.
+ *  workspace  at least kvq_decode_attn_seq_workspace_size(...) bytes, 256-B
+ *             aligned, zero-filled before first use (left ready for the next
+ *             call, as with kvq_decode_attn).
+ * Deterministic, like kvq_decode_attn: partials merge in view order, then
+ * chunk order.  With seq_begin = {0, 1, ..., n_views} the result is bitwise
+ * that of kvq_decode_attn.
+ * Errors: KVQ_ERR_INVALID_ARG for a malformed seq_begin or an empty sequence,
+ * KVQ_ERR_UNSUPPORTED for more than KVQ_MAX_SEGMENTS non-empty views in a
+ * sequence; otherwise as kvq_decode_attn.  Nothing is enqueued on error.
+ */
+kvq_status kvq_decode_attn_seq(const kvq_view *views, int32_t n_views, const int32_t *seq_begin,
+                               int32_t n_seqs, int32_t n_q_heads, int32_t n_kv_heads,
+                               int32_t head_dim, const void *q, float softmax_scale, float *out,
+                               void *workspace, size_t workspace_bytes, void *stream);
+
+/*
  * kvq_append_decode_attn -- one decode step over a batch of views: the
  * effect of kvq_append(views, ..., k_new, v_new) followed by
  * kvq_decode_attn(views, ...) on the appended views, in one call (CoMixKV,

@@ -10,6 +10,9 @@ Entry points (same names as the C ABI, without the ``kvq_`` prefix):
   quantize, dequantize          -- bf16 rows <-> packed b-bit codes + {s, mn}
   View, append                  -- one (agent, layer) cache; add a decode token
   decode_attn, workspace_size   -- batched split-K attention over many views
+  decode_attn_seq               -- the same over sequences held by several views
+                                   (segments) of any widths; View.new_segment
+                                   starts a segment at a new width
   append_decode_attn            -- one decode step: append, then attend, in one call
   card_pack, card_unpack, ...   -- CacheCard: several views' caches as one
                                    artifact (transfer, save_card / load_card)
@@ -28,11 +31,13 @@ import torch
 from . import workloads  # noqa: F401  (seeded input generators)
 
 __all__ = ["quantize", "dequantize", "View", "append", "decode_attn", "workspace_size",
-           "append_decode_attn", "step_workspace_size", "decode_attn_noalloc",
+           "append_decode_attn", "step_workspace_size", "decode_attn_noalloc", "decode_attn_seq",
+           "seq_workspace_size", "new_seq_workspace", "MAX_SEGMENTS",
            "card_bytes", "card_pack", "card_info", "card_unpack", "views_for_card", "save_card", "load_card", "NOALLOC_SCRATCH_BYTES", "KvqError", "lib", "row_bytes", "GROUP"]
 
 GROUP = 64
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024   # KVQ_NOALLOC_SCRATCH_BYTES in kvq.h
+MAX_SEGMENTS = 64                          # KVQ_MAX_SEGMENTS in kvq.h
 _HERE = os.path.dirname(os.path.abspath(__file__))
 _LIB_PATH = os.path.join(_HERE, "libkvq.so")
 _lib = None
@@ -80,6 +85,10 @@ def lib():
         L.kvq_decode_attn_workspace_size.restype = sz
         L.kvq_decode_attn.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, f32, P, P, sz, P]
         L.kvq_decode_attn.restype = i32
+        L.kvq_decode_attn_seq_workspace_size.argtypes = [ctypes.POINTER(CView), i32, P, i32, i32, i32, i32]
+        L.kvq_decode_attn_seq_workspace_size.restype = sz
+        L.kvq_decode_attn_seq.argtypes = [ctypes.POINTER(CView), i32, P, i32, i32, i32, i32, P, f32, P, P, sz, P]
+        L.kvq_decode_attn_seq.restype = i32
         L.kvq_append_decode_attn.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, P, P, f32, P, P, sz, P]
         L.kvq_append_decode_attn.restype = i32
         u64 = ctypes.c_uint64
@@ -213,6 +222,23 @@ class View:
         if bits is not None:
             self.c.bits = self.bits = bits
 
+    def new_segment(self, bits: int, cap_packed: int, device=None) -> "View":
+        """Continue this cache at another width without requantizing it: a new
+        view of width ``bits`` with room for ``cap_packed`` packed rows takes
+        over this view's window ring (the same memory, the same tokens), so
+        later flushes are quantized at the new width.  This view keeps its
+        packed rows and gives up its window (cap_window 0).  Attend to both
+        with decode_attn_seq; append to the new one."""
+        dev = self.k_codes.device if device is None else device
+        t = dict(k_window=self.k_window, v_window=self.v_window)
+        seg = View(self.n_kv_heads, self.head_dim, bits, cap_packed, self.c.cap_window, device=dev, tensors=t)
+        seg.c.n_window, seg.c.window_head = self.c.n_window, self.c.window_head
+        self.c.n_window = self.c.window_head = self.c.cap_window = 0
+        self.k_window = self.k_window[:, :0]
+        self.v_window = self.v_window[:, :0]
+        self._sync_ptrs()
+        return seg
+
     def fill_packed(self, k: torch.Tensor, v: torch.Tensor, stream=None):
         """Quantize bf16 K/V [H, T, D] into packed rows [0, T) (prefill handoff)."""
         T = k.shape[1]
@@ -278,6 +304,43 @@ def decode_attn(views, q: torch.Tensor, softmax_scale: float, out: torch.Tensor 
     _check(lib().kvq_decode_attn(arr, len(views), Hq, views[0].n_kv_heads, D, _ptr(q), float(softmax_scale),
                                  _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
            "kvq_decode_attn")
+    return out
+
+
+def _seq_array(seq_begin):
+    sb = [int(x) for x in seq_begin]
+    return (ctypes.c_int32 * len(sb))(*sb), len(sb) - 1
+
+
+def seq_workspace_size(views, seq_begin, n_q_heads: int) -> int:
+    """kvq_decode_attn_seq_workspace_size (0 if the arguments are invalid)."""
+    views = list(views)
+    sb, n_seqs = _seq_array(seq_begin)
+    return int(lib().kvq_decode_attn_seq_workspace_size(_view_array(views), len(views), sb, n_seqs, n_q_heads,
+                                                        views[0].n_kv_heads, views[0].head_dim))
+
+
+def new_seq_workspace(views, seq_begin, n_q_heads: int, device="cuda") -> torch.Tensor:
+    n = seq_workspace_size(views, seq_begin, n_q_heads)
+    if n == 0:
+        raise KvqError(KVQ_ERR_INVALID_ARG, "kvq_decode_attn_seq_workspace_size")
+    return torch.zeros(n, dtype=torch.uint8, device=device)
+
+
+def decode_attn_seq(views, seq_begin, q: torch.Tensor, softmax_scale: float, out: torch.Tensor | None = None,
+                    workspace: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """kvq_decode_attn_seq: sequence s is views seq_begin[s] .. seq_begin[s+1]-1.
+    q: bf16 [n_seqs, H_q, D] -> fp32 [n_seqs, H_q, D]."""
+    views = list(views)
+    n, Hq, D = q.shape
+    sb, n_seqs = _seq_array(seq_begin)
+    if workspace is None:
+        workspace = new_seq_workspace(views, seq_begin, Hq, device=q.device)
+    if out is None:
+        out = torch.empty((n, Hq, D), dtype=torch.float32, device=q.device)
+    _check(lib().kvq_decode_attn_seq(_view_array(views), len(views), sb, n_seqs, Hq, views[0].n_kv_heads, D,
+                                     _ptr(q), float(softmax_scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                     _stream(stream)), "kvq_decode_attn_seq")
     return out
 
 

@@ -100,7 +100,6 @@ struct AttnLaunch {
     int v0, v1;          // views order[v0 .. v1) of the plan
     int total_chunks;
     int bits;            // the width of every view of the launch with packed tokens
-    size_t counters_off, partials_off;  // this launch's workspace regions
 };
 
 struct ViewChunks {
@@ -111,9 +110,12 @@ struct AttnPlan {
     int ring_bytes = 0;
     size_t smem = 0;
     int head_blocks = 0;
-    std::vector<int> order;  // views grouped by width (stable), as the launches take them
+    std::vector<int> order;  // views with tokens, grouped by width (stable), as the launches take them
     std::vector<AttnLaunch> launches;
     std::vector<ViewChunks> chunks;
+    std::vector<int32_t> seq_of, part_begin;        // per view: its sequence, partial slot of its chunk 0
+    std::vector<int32_t> seq_part_begin, seq_chunks;  // per sequence
+    size_t counters_off = 0, partials_off = 0;
     size_t zero_bytes = 0, total = 0;
 };
 
@@ -264,13 +266,35 @@ kvq_status ensure_attn_smem(size_t smem) {
     return KVQ_OK;
 }
 
-kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, int32_t n_kv_heads,
-                     int32_t head_dim, AttnPlan &plan) {
+// seq_begin == nullptr: every view is a sequence of its own (and must hold a
+// token).  Otherwise sequence s is views seq_begin[s] .. seq_begin[s+1]-1, its
+// tokens the concatenation of theirs; empty views are allowed and skipped.
+kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_begin, int32_t n_seqs,
+                     int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, AttnPlan &plan) {
     if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
     if (n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads || n_kv_heads > 65535)
         return KVQ_ERR_INVALID_ARG;
-    const kvq_status vs = validate_views(views, n_views, true);
+    const kvq_status vs = validate_views(views, n_views, seq_begin == nullptr);
     if (vs != KVQ_OK) return vs;
+    plan.seq_of.assign(n_views, 0);
+    if (!seq_begin) {
+        n_seqs = n_views;
+        for (int i = 0; i < n_views; ++i) plan.seq_of[i] = i;
+    } else {
+        if (n_seqs <= 0 || seq_begin[0] != 0 || seq_begin[n_seqs] != n_views) return KVQ_ERR_INVALID_ARG;
+        for (int s = 0; s < n_seqs; ++s) {
+            if (seq_begin[s + 1] <= seq_begin[s]) return KVQ_ERR_INVALID_ARG;
+            int64_t tokens = 0;
+            int used = 0;
+            for (int i = seq_begin[s]; i < seq_begin[s + 1]; ++i) {
+                plan.seq_of[i] = s;
+                tokens += views[i].n_packed + views[i].n_window;
+                used += views[i].n_packed + views[i].n_window > 0 ? 1 : 0;
+            }
+            if (tokens <= 0) return KVQ_ERR_INVALID_ARG;
+            if (used > KVQ_MAX_SEGMENTS) return KVQ_ERR_UNSUPPORTED;
+        }
+    }
     const int ng = head_dim / 64;
     const int group = n_q_heads / n_kv_heads;
     plan.head_blocks = (group + kvq::kHeadsPerCta - 1) / kvq::kHeadsPerCta;
@@ -309,17 +333,18 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, 
     for (int i = 0; i < n_views; ++i)
         if (views[i].n_packed > 0) { first_bits = views[i].bits; break; }
     auto key = [&](int i) { return views[i].n_packed > 0 ? views[i].bits : first_bits; };
-    plan.order.resize(n_views);
-    for (int i = 0; i < n_views; ++i) plan.order[i] = i;
+    plan.order.clear();
+    for (int i = 0; i < n_views; ++i)
+        if (views[i].n_packed + views[i].n_window > 0) plan.order.push_back(i);
+    const int n_used = (int)plan.order.size();
     std::stable_sort(plan.order.begin(), plan.order.end(), [&](int a, int b) { return key(a) < key(b); });
     double bytes_all = 0;
     for (int i = 0; i < n_views; ++i)
         bytes_all += (double)views[i].n_packed * packed_token_bytes(head_dim, views[i].bits) +
                      (double)views[i].n_window * window_token_bytes(head_dim);
-    size_t off = 256;  // bytes [0, 4): the device status word
-    for (int v0 = 0; v0 < n_views;) {
+    for (int v0 = 0; v0 < n_used;) {
         int v1 = v0 + 1;
-        while (v1 < n_views && v1 - v0 < kvq::kAttnMaxViews && key(plan.order[v1]) == key(plan.order[v0])) ++v1;
+        while (v1 < n_used && v1 - v0 < kvq::kAttnMaxViews && key(plan.order[v1]) == key(plan.order[v0])) ++v1;
         double bytes = 0;
         for (int k = v0; k < v1; ++k) {
             const kvq_view &v = views[plan.order[k]];
@@ -331,17 +356,55 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads, 
         int64_t chunks = 0;
         plan_free(views, plan.order.data() + v0, v1 - v0, units, head_dim, share, plan.chunks, &chunks);
         if (chunks > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
-        AttnLaunch L{v0, v1, (int)chunks, key(plan.order[v0]), 0, 0};
-        L.counters_off = off;  // one arrival counter per unit of the launch
-        off += ((size_t)(v1 - v0) * units * 4 + 255) / 256 * 256;
-        plan.launches.push_back(L);
+        plan.launches.push_back(AttnLaunch{v0, v1, (int)chunks, key(plan.order[v0])});
         v0 = v1;
     }
-    plan.zero_bytes = off;  // status word and counters: the part that must start at zero
-    for (AttnLaunch &L : plan.launches) {
-        L.partials_off = off;
-        off += ((size_t)L.total_chunks * units * kvq::kHeadsPerCta * (head_dim + 2) * 4 + 255) / 256 * 256;
+    // A sequence's unit combine holds at most kMaxChunksPerUnit chunks: trim
+    // the largest parts of the sequences above that.
+    const int32_t *sb = seq_begin;
+    auto seq_first = [&](int s) { return sb ? sb[s] : s; };
+    auto seq_end = [&](int s) { return sb ? sb[s + 1] : s + 1; };
+    for (int s = 0; s < n_seqs; ++s) {
+        for (;;) {
+            int64_t total = 0;
+            int32_t *big = nullptr;
+            for (int i = seq_first(s); i < seq_end(s); ++i) {
+                ViewChunks &c = plan.chunks[i];
+                total += c.n_packed + c.n_window;
+                if (!big || c.n_packed > *big) big = &c.n_packed;
+                if (c.n_window > *big) big = &c.n_window;
+            }
+            if (total <= kvq::kMaxChunksPerUnit) break;
+            *big = std::max<int32_t>(1, *big * 3 / 4);
+        }
     }
+    for (AttnLaunch &L : plan.launches) {
+        int64_t chunks = 0;
+        for (int k = L.v0; k < L.v1; ++k)
+            chunks += plan.chunks[plan.order[k]].n_packed + plan.chunks[plan.order[k]].n_window;
+        L.total_chunks = (int)chunks;
+    }
+    // partial slots: sequences in order, each one's views in order, each
+    // view's chunks in order (the order the unit combine merges them in)
+    plan.part_begin.assign(n_views, 0);
+    plan.seq_part_begin.assign(n_seqs, 0);
+    plan.seq_chunks.assign(n_seqs, 0);
+    int64_t slot = 0;
+    for (int s = 0; s < n_seqs; ++s) {
+        plan.seq_part_begin[s] = (int32_t)slot;
+        for (int i = seq_first(s); i < seq_end(s); ++i) {
+            plan.part_begin[i] = (int32_t)slot;
+            slot += plan.chunks[i].n_packed + plan.chunks[i].n_window;
+        }
+        plan.seq_chunks[s] = (int32_t)(slot - plan.seq_part_begin[s]);
+        if (slot > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
+    }
+    size_t off = 256;  // bytes [0, 4): the device status word
+    plan.counters_off = off;  // one arrival counter per (sequence, KV head, head block)
+    off += ((size_t)n_seqs * units * 4 + 255) / 256 * 256;
+    plan.zero_bytes = off;  // status word and counters: the part that must start at zero
+    plan.partials_off = off;
+    off += ((size_t)slot * units * kvq::kHeadsPerCta * (head_dim + 2) * 4 + 255) / 256 * 256;
     plan.total = off;
     return KVQ_OK;
 }
@@ -388,10 +451,10 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
     prm.group = n_q_heads / n_kv_heads;
     prm.head_blocks = plan.head_blocks;
     prm.ring_bytes = plan.ring_bytes;
+    prm.counters = reinterpret_cast<uint32_t *>(ws + plan.counters_off);
+    prm.partials = reinterpret_cast<float *>(ws + plan.partials_off);
     for (const AttnLaunch &L : plan.launches) {
         prm.n_views = L.v1 - L.v0;
-        prm.counters = reinterpret_cast<uint32_t *>(ws + L.counters_off);
-        prm.partials = reinterpret_cast<float *>(ws + L.partials_off);
         // The first launch waits for the preceding work at entry (behind a
         // fused append: only its blocks that read appended rows wait).  Later
         // launches of the call start as soon as the one before has released
@@ -399,7 +462,7 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
         // waits for its predecessor before it exits, so the call's last grid
         // completes after all of them.
         prm.fused = dep != nullptr ? 1 : 0;
-        prm.chain = L.v0 > 0 ? 1 : 0;
+        prm.chain = &L != &plan.launches[0] ? 1 : 0;
         int begin = 0;
         for (int k = L.v0; k < L.v1; ++k) {
             const int i = plan.order[k];
@@ -421,7 +484,10 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
             d.n_chunks_packed = c.n_packed;
             d.n_chunks = c.n_packed + c.n_window;
             d.chunk_begin = begin;
-            d.view_index = i;
+            d.seq_index = plan.seq_of[i];
+            d.part_begin = plan.part_begin[i];
+            d.seq_part_begin = plan.seq_part_begin[plan.seq_of[i]];
+            d.seq_chunks = plan.seq_chunks[plan.seq_of[i]];
             d.dep_step[0] = prm.fused ? dep[2 * i] : -1;
             d.dep_step[1] = prm.fused ? dep[2 * i + 1] : -1;
             begin += d.n_chunks;
@@ -766,7 +832,7 @@ KVQ_API kvq_status kvq_append(kvq_view *views, int32_t n_views, int32_t n_kv_hea
 KVQ_API size_t kvq_decode_attn_workspace_size(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
                                               int32_t n_kv_heads, int32_t head_dim) {
     AttnPlan plan;
-    if (plan_attn(views, n_views, n_q_heads, n_kv_heads, head_dim, plan) != KVQ_OK) return 0;
+    if (plan_attn(views, n_views, nullptr, 0, n_q_heads, n_kv_heads, head_dim, plan) != KVQ_OK) return 0;
     return plan.total;
 }
 
@@ -774,7 +840,7 @@ KVQ_API kvq_status kvq_decode_attn(const kvq_view *views, int32_t n_views, int32
                                    int32_t head_dim, const void *q, float softmax_scale, float *out, void *workspace,
                                    size_t workspace_bytes, void *stream) {
     AttnPlan plan;
-    const kvq_status ps = plan_attn(views, n_views, n_q_heads, n_kv_heads, head_dim, plan);
+    const kvq_status ps = plan_attn(views, n_views, nullptr, 0, n_q_heads, n_kv_heads, head_dim, plan);
     if (ps != KVQ_OK) return ps;
     if (!q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
@@ -789,11 +855,35 @@ KVQ_API kvq_status kvq_decode_attn(const kvq_view *views, int32_t n_views, int32
     }
 }
 
+KVQ_API size_t kvq_decode_attn_seq_workspace_size(const kvq_view *views, int32_t n_views, const int32_t *seq_begin,
+                                                  int32_t n_seqs, int32_t n_q_heads, int32_t n_kv_heads,
+                                                  int32_t head_dim) {
+    if (!seq_begin) return 0;
+    AttnPlan plan;
+    if (plan_attn(views, n_views, seq_begin, n_seqs, n_q_heads, n_kv_heads, head_dim, plan) != KVQ_OK) return 0;
+    return plan.total;
+}
+
+KVQ_API kvq_status kvq_decode_attn_seq(const kvq_view *views, int32_t n_views, const int32_t *seq_begin,
+                                       int32_t n_seqs, int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim,
+                                       const void *q, float softmax_scale, float *out, void *workspace,
+                                       size_t workspace_bytes, void *stream) {
+    if (!seq_begin) return KVQ_ERR_INVALID_ARG;
+    AttnPlan plan;
+    const kvq_status ps = plan_attn(views, n_views, seq_begin, n_seqs, n_q_heads, n_kv_heads, head_dim, plan);
+    if (ps != KVQ_OK) return ps;
+    if (!q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
+    if (workspace_bytes < plan.total) return KVQ_ERR_INVALID_ARG;
+    return launch_attn(plan, views, n_q_heads, n_kv_heads, head_dim, q, softmax_scale, out,
+                       static_cast<uint8_t *>(workspace), static_cast<cudaStream_t>(stream));
+}
+
 KVQ_API kvq_status kvq_decode_attn_noalloc(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
                                            int32_t n_kv_heads, int32_t head_dim, const void *q, float softmax_scale,
                                            float *out, void *stream) {
     AttnPlan plan;
-    const kvq_status ps = plan_attn(views, n_views, n_q_heads, n_kv_heads, head_dim, plan);
+    const kvq_status ps = plan_attn(views, n_views, nullptr, 0, n_q_heads, n_kv_heads, head_dim, plan);
     if (ps != KVQ_OK) return ps;
     if (!q || !out) return KVQ_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(out, 16)) return KVQ_ERR_INVALID_ARG;
@@ -819,7 +909,7 @@ KVQ_API kvq_status kvq_append_decode_attn(kvq_view *views, int32_t n_views, int3
     std::vector<kvq_view> post(views, views + n_views);
     for (kvq_view &v : post) advance_view(v);
     AttnPlan plan;
-    const kvq_status ps = plan_attn(post.data(), n_views, n_q_heads, n_kv_heads, head_dim, plan);
+    const kvq_status ps = plan_attn(post.data(), n_views, nullptr, 0, n_q_heads, n_kv_heads, head_dim, plan);
     if (ps != KVQ_OK) return ps;
     if (!q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;

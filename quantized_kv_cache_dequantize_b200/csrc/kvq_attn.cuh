@@ -61,17 +61,20 @@ struct AttnView {
     int32_t n_chunks_packed;     // the packed part's 32-token steps, split evenly
     int32_t n_chunks;            // packed + window chunks (window: 16-token steps)
     int32_t chunk_begin;         // first chunk index of this view in the launch
-    int32_t view_index;          // row of q / out
+    int32_t seq_index;           // its sequence: row of q / out, arrival counter
+    int32_t part_begin;          // partial slot of the view's chunk 0 (call-wide)
+    int32_t seq_part_begin;      // partial slot of the sequence's first chunk
+    int32_t seq_chunks;          // chunks of the whole sequence (all its views)
     int32_t dep_step[2];         // packed / window step whose rows the preceding append grid
                                  // writes (-1: none); with AttnParams::fused its copy waits
                                  // for that grid, every other copy starts at once
 };
 
 struct AttnParams {
-    const uint16_t *q;           // bf16 [n_views_total][Hq][D]
-    float *out;                  // fp32 [n_views_total][Hq][D]
-    float *partials;             // workspace
-    uint32_t *counters;          // workspace: per unit of the launch, chunks finished
+    const uint16_t *q;           // bf16 [n_seqs][Hq][D]
+    float *out;                  // fp32 [n_seqs][Hq][D]
+    float *partials;             // workspace: chunk partials of the whole call
+    uint32_t *counters;          // workspace: per (sequence, KV head, head block), chunks finished
     uint32_t *status;            // workspace word 0
     uint64_t timeout_ns;
     float scale_log2;            // softmax_scale * log2(e)
@@ -547,8 +550,9 @@ __host__ __device__ constexpr int attn_header_bytes() {
     return (8 * 64 * NG * 2 + kAttnWarps * kMaxStages * 8 + 16 + 127) & ~127;
 }
 
-// Split-K combine of one unit (view, KV head, head block) whose n > 1 chunk
-// partials are in the workspace, run by the CTA that finished the unit's last
+// Split-K combine of one unit (sequence, KV head, head block) whose n > 1
+// chunk partials are in the workspace (the chunks of all the sequence's views,
+// in view order, contiguous), run by the CTA that finished the unit's last
 // chunk.  A partial is [O: 8 heads x D][m: 8][l: 8] floats.  Up to 8 chunks:
 // every thread loads all chunks' (m, l) of its head and O of its 4 outputs in
 // one round and merges them in chunk order.  More chunks: the CTA gathers
@@ -564,14 +568,14 @@ __device__ __forceinline__ void combine_unit(const AttnParams &p, const AttnView
     float *sm_w = scratch;                                        // m, then weight
     float *sm_l = scratch + kMaxChunksPerUnit * kHeadsPerCta;
     float *sm_L = scratch + 2 * kMaxChunksPerUnit * kHeadsPerCta;
-    const int n = V.n_chunks;
+    const int n = V.seq_chunks;
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int h0 = hk * p.group + z * kHeadsPerCta;
     const int nh = min(kHeadsPerCta, p.group - z * kHeadsPerCta);
-    const int64_t slot0 = ((int64_t)V.chunk_begin * p.n_kv_heads + hk) * p.head_blocks + z;
+    const int64_t slot0 = ((int64_t)V.seq_part_begin * p.n_kv_heads + hk) * p.head_blocks + z;
     const int64_t stride = (int64_t)p.n_kv_heads * p.head_blocks * kSlot;  // between chunks
     const float *part0 = p.partials + slot0 * kSlot;
-    float4 *out4 = reinterpret_cast<float4 *>(p.out + ((int64_t)V.view_index * p.n_q_heads + h0) * D);
+    float4 *out4 = reinterpret_cast<float4 *>(p.out + ((int64_t)V.seq_index * p.n_q_heads + h0) * D);
     if (n <= 8) {
         // one round of loads: each thread fetches every chunk's (m, l) of its
         // head and O of its 4 outputs at once, then merges in chunk order
@@ -666,7 +670,7 @@ __device__ __forceinline__ void combine_unit(const AttnParams &p, const AttnView
 // the block's bulk copies; one lane issues the copies and a slot is refilled
 // as soon as the warp has consumed it.
 template <int NG, int B, bool WINDOW>
-__device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V, int vl, int c, int hk, int z,
+__device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V, int c, int hk, int z,
                                           uint8_t *smem) {
     constexpr int D = 64 * NG;
     constexpr int RB = 8 * B * NG;
@@ -774,7 +778,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         const int j = i / (D / 8), d8 = i - j * (D / 8);
         uint4 val = make_uint4(0, 0, 0, 0);
         // L2 loads: with a fused append this CTA may not have waited for the grids before
-        if (j < nh) val = __ldcg(reinterpret_cast<const uint4 *>(p.q + ((int64_t)V.view_index * p.n_q_heads + h0 + j) * D) + d8);
+        if (j < nh) val = __ldcg(reinterpret_cast<const uint4 *>(p.q + ((int64_t)V.seq_index * p.n_q_heads + h0 + j) * D) + d8);
         reinterpret_cast<uint4 *>(q_s)[i] = val;
     }
     __syncthreads();
@@ -942,8 +946,8 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     __syncthreads();
 
     // ---- merge the 4 warps (fixed order)
-    const bool single = V.n_chunks == 1;
-    const int64_t pslot = ((int64_t)(V.chunk_begin + c) * p.n_kv_heads + hk) * p.head_blocks + z;
+    const bool single = V.seq_chunks == 1;
+    const int64_t pslot = ((int64_t)(V.part_begin + c) * p.n_kv_heads + hk) * p.head_blocks + z;
     float *part = p.partials + pslot * (kHeadsPerCta * (D + 2));
     for (int idx = tid; idx < nh * D; idx += kAttnThreads) {
         const int j = idx / D, d = idx - j * D;
@@ -961,7 +965,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             O = fmaf(e, wp[16 + j * D + d], O);
         }
         if (single) {
-            p.out[((int64_t)V.view_index * p.n_q_heads + h0 + j) * D + d] = O / L;
+            p.out[((int64_t)V.seq_index * p.n_q_heads + h0 + j) * D + d] = O / L;
         } else {
             part[j * D + d] = O;
             if (d == 0) {
@@ -977,9 +981,9 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     __threadfence();  // this thread's partial stores, before the arrival below
     __syncthreads();
     if (tid == 0) {
-        uint32_t *ctr = p.counters + ((int64_t)vl * p.n_kv_heads + hk) * p.head_blocks + z;
+        uint32_t *ctr = p.counters + ((int64_t)V.seq_index * p.n_kv_heads + hk) * p.head_blocks + z;
         const uint32_t before = atomicAdd(ctr, 1u);
-        const bool last = before + 1 == (uint32_t)V.n_chunks;
+        const bool last = before + 1 == (uint32_t)V.seq_chunks;
         if (last) *ctr = 0u;
         *last_flag = last ? 1 : 0;
     }
@@ -1014,8 +1018,8 @@ __device__ __forceinline__ void decode_attn_body(const AttnParams &p, uint8_t *s
     const int c = bx - V.chunk_begin;
     const int hk = blockIdx.y, z = blockIdx.z;
     if (c >= V.n_chunks) return;  // never launched by the host planner; defensive
-    if (c >= V.n_chunks_packed) attn_item<NG, 4, true>(p, V, lo, c, hk, z, smem);
-    else attn_item<NG, BSEL, false>(p, V, lo, c, hk, z, smem);
+    if (c >= V.n_chunks_packed) attn_item<NG, 4, true>(p, V, c, hk, z, smem);
+    else attn_item<NG, BSEL, false>(p, V, c, hk, z, smem);
 }
 
 template <int NG, int BSEL>

@@ -114,6 +114,41 @@ def test_decode_attn_validation(L):
     assert L.kvq_decode_attn(win, 1, 8, 2, 128, FAKE, 0.1, FAKE, FAKE, ws, NULL) == kvq.KVQ_ERR_INVALID_ARG
 
 
+def test_decode_attn_seq_validation(L):
+    def sb(*xs):
+        return (ctypes.c_int32 * len(xs))(*xs)
+
+    views = (kvq.CView * 4)(cview(), cview(bits=2, n_packed=0), cview(bits=8), cview(bits=3))
+    ws = L.kvq_decode_attn_seq_workspace_size(views, 4, sb(0, 3, 4), 2, 8, 2, 128)
+    assert ws > 0
+    # one view per sequence needs the same scratch as kvq_decode_attn
+    one = (kvq.CView * 2)(cview(), cview(bits=8))
+    assert L.kvq_decode_attn_seq_workspace_size(one, 2, sb(0, 1, 2), 2, 8, 2, 128) == \
+        L.kvq_decode_attn_workspace_size(one, 2, 8, 2, 128)
+    for bad in [sb(1, 3, 4), sb(0, 3, 3), sb(0, 4, 4), sb(0, 0, 4), sb(0, 3, 5)]:
+        assert L.kvq_decode_attn_seq_workspace_size(views, 4, bad, 2, 8, 2, 128) == 0
+        assert L.kvq_decode_attn_seq(views, 4, bad, 2, 8, 2, 128, FAKE, 0.1, FAKE, FAKE, ws, NULL) == \
+            kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_decode_attn_seq(views, 4, NULL, 2, 8, 2, 128, FAKE, 0.1, FAKE, FAKE, ws, NULL) == \
+        kvq.KVQ_ERR_INVALID_ARG
+    # a sequence whose views hold no token
+    empty = (kvq.CView * 2)(cview(), cview(n_packed=0))
+    assert L.kvq_decode_attn_seq(empty, 2, sb(0, 1, 2), 2, 8, 2, 128, FAKE, 0.1, FAKE, FAKE, ws, NULL) == \
+        kvq.KVQ_ERR_INVALID_ARG
+    # too many non-empty segments in one sequence
+    n = kvq.MAX_SEGMENTS + 1
+    many = (kvq.CView * n)(*[cview() for _ in range(n)])
+    assert L.kvq_decode_attn_seq(many, n, sb(0, n), 1, 8, 2, 128, FAKE, 0.1, FAKE, FAKE, 1 << 30, NULL) == \
+        kvq.KVQ_ERR_UNSUPPORTED
+    ok = (kvq.CView * (n - 1))(*[cview() for _ in range(n - 1)])
+    assert L.kvq_decode_attn_seq_workspace_size(ok, n - 1, sb(0, n - 1), 1, 8, 2, 128) > 0
+    # workspace too small, unaligned q
+    assert L.kvq_decode_attn_seq(views, 4, sb(0, 3, 4), 2, 8, 2, 128, FAKE, 0.1, FAKE, FAKE, ws - 1, NULL) == \
+        kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_decode_attn_seq(views, 4, sb(0, 3, 4), 2, 8, 2, 128, ctypes.c_void_p(0x10008), 0.1, FAKE, FAKE,
+                                 ws, NULL) == kvq.KVQ_ERR_INVALID_ARG
+
+
 def test_workspace_grows_with_views(L):
     one = (kvq.CView * 1)(cview(n_packed=4096, cap_packed=4096))
     many = (kvq.CView * 200)(*[cview(n_packed=4096, cap_packed=4096) for _ in range(200)])
