@@ -247,6 +247,60 @@ def decode_attn_segments(q: np.ndarray, segments, softmax_scale: float) -> np.nd
     return out
 
 
+def sparse_decode_attn(q: np.ndarray, bits: int, k_codes, k_sm, v_codes, v_sm, k_win, v_win,
+                       softmax_scale: float, top_k: int):
+    """Top-K sparse decode attention over one view, in fp64.
+
+    Source: "Reasoning-Aware Error-Bounded KV-Cache Compression and Sparse
+    Attention for Long-Context LLMs" (Metodologia C, dynamic sparse decode
+    attention: the top-K entries by a query-aware score form the active set,
+    the others stay in the cache unused for this step).  Readings: the score
+    of a packed token for a KV head is its instantaneous query-key
+    compatibility, the largest logit softmax_scale * q_h . k over the query
+    heads h of that KV head's group (the page's utility terms need attention
+    history and a reasoning-phase signal, which the decode step does not
+    have); the K highest-scoring packed tokens are selected per KV head, equal
+    scores going to the lower token index; the bf16 recent window is always
+    active (recent states are kept native and never evicted).  Attention is
+    then plain softmax attention over the active tokens.
+
+    Arguments as decode_attn, plus top_k >= 1.  Returns (out float64 [H_q][D],
+    selected: list over KV heads of ascending packed-token index arrays).
+    """
+    q = _c(q, np.uint16)
+    Hq, D = q.shape
+    n_p = 0 if k_codes is None else k_codes.shape[1]
+    n_w = 0 if k_win is None else k_win.shape[1]
+    if n_p + n_w == 0 or top_k < 1:
+        raise ValueError("empty view or top_k < 1")
+    Hkv = (k_codes if n_p else k_win).shape[0]
+    G = Hq // Hkv
+    qd = _bf16_to_f64(q)
+    kp = affine(k_codes, k_sm, D, bits) if n_p else np.zeros((Hkv, 0, D))
+    vp = affine(v_codes, v_sm, D, bits) if n_p else np.zeros((Hkv, 0, D))
+    kw = _bf16_to_f64(k_win) if n_w else np.zeros((Hkv, 0, D))
+    vw = _bf16_to_f64(v_win) if n_w else np.zeros((Hkv, 0, D))
+    out = np.zeros((Hq, D), np.float64)
+    selected = []
+    for hk in range(Hkv):
+        heads = range(hk * G, (hk + 1) * G)
+        if n_p:
+            score = np.max(np.stack([softmax_scale * (kp[hk] @ qd[h]) for h in heads]), axis=0)
+            # descending score, ties to the lower index (stable sort of -score)
+            order = np.argsort(-score, kind="stable")
+            sel = np.sort(order[:min(top_k, n_p)])
+        else:
+            sel = np.zeros(0, np.int64)
+        selected.append(sel)
+        k = np.concatenate([kp[hk][sel], kw[hk]], axis=0)
+        v = np.concatenate([vp[hk][sel], vw[hk]], axis=0)
+        for h in heads:
+            logits = softmax_scale * (k @ qd[h])
+            w = np.exp(logits - logits.max())
+            out[h] = (w / w.sum()) @ v
+    return out, selected
+
+
 class WindowModel:
     """Bookkeeping model of one view's token placement under appends.
 

@@ -478,6 +478,84 @@ def test_identical_keys_over_segments_give_mean_of_all_values():
         np.testing.assert_allclose(got[h], vals[h // 2].mean(axis=0), rtol=1e-12, atol=1e-13)
 
 
+# ------------------------------------------------- top-K sparse decode ---
+
+def run_sparse(view, scale, top_k):
+    return oracle.sparse_decode_attn(view["q"], view["bits"], view["k_codes"], view["k_sm"], view["v_codes"],
+                                     view["v_sm"], view["k_win"], view["v_win"], scale, top_k)
+
+
+@pytest.mark.parametrize("top_k", [45, 46, 1000])
+def test_sparse_with_every_token_selected_is_dense(top_k):
+    view = make_view(50, n_p=45, n_w=6)
+    out, sel = run_sparse(view, 1 / 8, top_k)
+    np.testing.assert_allclose(out, run(view, 1 / 8), rtol=1e-12, atol=1e-13)
+    assert all(np.array_equal(s, np.arange(45)) for s in sel)
+
+
+@pytest.mark.parametrize("bits,top_k", [(2, 1), (4, 5), (4, 20), (8, 33), (3, 44)])
+def test_sparse_error_within_discarded_mass_bound(bits, top_k):
+    # RECAS (Metodologia B): with ||v|| <= V_max for every token and delta the
+    # full attention's mass on the tokens left out, ||o - o'|| <= 2 V_max delta
+    view = make_view(51 + bits, Hq=8, Hkv=2, n_p=45, n_w=6, bits=bits)
+    dense, probs = run(view, 0.3, probs=True)
+    sparse, sel = run_sparse(view, 0.3, top_k)
+    _, v = dense_kv(view)
+    G = 4
+    for h in range(8):
+        hk = h // G
+        left_out = np.setdiff1d(np.arange(45), sel[hk])
+        delta = probs[h][left_out].sum()
+        vmax = np.sqrt((v[hk] ** 2).sum(axis=1)).max()
+        err = np.sqrt(((dense[h] - sparse[h]) ** 2).sum())
+        assert err <= 2 * vmax * delta * (1 + 1e-9) + 1e-12
+        assert len(sel[hk]) == top_k
+
+
+def test_sparse_selects_a_planted_key_and_attends_it_with_the_window():
+    # one packed key far more aligned with q than all others: with K = 1 it is
+    # the selection, and the output is attention over it and the window only
+    view = make_view(60, Hq=2, Hkv=1, n_p=30, n_w=4, bits=8)
+    q = np.zeros((2, 64), np.uint16)
+    q[:, 0] = 0x3F80                                   # q = e_0 (bf16 1.0)
+    view["q"] = q
+    codes = view["k_codes"].copy()
+    sm = view["k_sm"].copy()
+    sm[0, 17, 0] = (1.0, 0.0)                          # token 17: k_0 = code (s = 1, mn = 0)
+    codes[0, 17, 0] = 255
+    view["k_codes"], view["k_sm"] = codes, sm
+    out, sel = run_sparse(view, 1.0, 1)
+    assert list(sel[0]) == [17]
+    k, v = dense_kv(view)
+    rows = [17] + list(range(30, 34))
+    logits = k[0][rows] @ bf16_to_f64(q[0])
+    p = np.exp(logits - logits.max())
+    p /= p.sum()
+    np.testing.assert_allclose(out[0], p @ v[0][rows], rtol=1e-12, atol=1e-13)
+
+
+def test_sparse_score_takes_the_group_maximum_and_ties_go_low():
+    # two query heads share the KV head; a token liked by either is selected;
+    # among equal scores the lower index wins
+    view = make_view(61, Hq=2, Hkv=1, n_p=10, n_w=0, bits=8)
+    q = np.zeros((2, 64), np.uint16)
+    q[0, 0] = 0x3F80
+    q[1, 1] = 0x3F80
+    view["q"] = q
+    codes = np.zeros_like(view["k_codes"])
+    sm = np.zeros_like(view["k_sm"])
+    sm[0, :, 0, 0] = 1.0                               # s = 1, mn = 0: k = codes
+    codes[0, 3, 0] = 200                               # head 0 likes token 3
+    codes[0, 7, 1] = 150                               # head 1 likes token 7
+    codes[0, 5, 1] = 100                               # and token 5 less
+    codes[0, 8, 0] = 100                               # token 8 ties with token 5
+    view["k_codes"], view["k_sm"] = codes, sm
+    assert list(run_sparse(view, 1.0, 2)[1][0]) == [3, 7]
+    assert list(run_sparse(view, 1.0, 3)[1][0]) == [3, 5, 7]
+    assert list(run_sparse(view, 1.0, 4)[1][0]) == [3, 5, 7, 8]
+    assert list(run_sparse(view, 1.0, 5)[1][0]) == [0, 3, 5, 7, 8]
+
+
 # --------------------------------------------------------- window model ---
 
 @pytest.mark.parametrize("W", [0, 1, 4, 7])
