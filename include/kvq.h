@@ -253,6 +253,49 @@ kvq_status kvq_decode_attn_seq(const kvq_view *views, int32_t n_views, const int
                                void *workspace, size_t workspace_bytes, void *stream);
 
 /*
+ * kvq_sparse_decode_attn -- top-K sparse decode attention over packed caches
+ * ("Reasoning-Aware Error-Bounded KV-Cache Compression and Sparse Attention
+ * for Long-Context LLMs", Metodologia C: a query-aware score picks the K
+ * entries that attend this step; the others stay in the cache).
+ *
+ * For every view and KV head hk:
+ *   score(t) = max over the query heads h of hk's group of
+ *              softmax_scale * (q_h . k_t), k_t = mn + s*c exactly, for each
+ *              packed token t;
+ *   the top_k packed tokens by score are selected (equal scores: the lower
+ *   token index first; all of them when n_packed <= top_k);
+ *   out[h] = softmax attention of q_h over the selected packed tokens and
+ *   all of the view's bf16 window tokens (the recent window is always active).
+ * With top_k >= n_packed the result is that of kvq_decode_attn (within
+ * rounding).  When the full attention puts mass delta on the packed tokens
+ * left out and every value vector has norm <= V_max, the output moves by at
+ * most 2 * V_max * delta (ibid., Metodologia B).
+ *
+ *  views, n_q_heads, n_kv_heads, head_dim, q, softmax_scale, out
+ *             as kvq_decode_attn.
+ *  top_k      >= 1, packed tokens selected per (view, KV head).
+ *  selected   NULL, or int32 [n_views][n_kv_heads][top_k] device array that
+ *             receives the selected packed-token indices, ascending, padded
+ *             with -1 when a view has fewer than top_k packed tokens.
+ *  workspace  at least kvq_sparse_decode_attn_workspace_size(...) bytes,
+ *             256-B aligned, zero-filled before first use; the first bytes
+ *             are left ready for the next call with the same views, heads and
+ *             top_k, while the sizes of the views change.
+ * Scores are fp32; the attention is that of kvq_decode_attn over per-head
+ * compact views (the selected rows gathered into the workspace).
+ * Errors: as kvq_decode_attn, and KVQ_ERR_INVALID_ARG for top_k < 1.
+ */
+size_t kvq_sparse_decode_attn_workspace_size(const kvq_view *views, int32_t n_views,
+                                             int32_t n_q_heads, int32_t n_kv_heads,
+                                             int32_t head_dim, int32_t top_k);
+
+kvq_status kvq_sparse_decode_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
+                                  int32_t n_kv_heads, int32_t head_dim, const void *q,
+                                  float softmax_scale, int32_t top_k, float *out,
+                                  int32_t *selected, void *workspace, size_t workspace_bytes,
+                                  void *stream);
+
+/*
  * kvq_append_decode_attn -- one decode step over a batch of views: the
  * effect of kvq_append(views, ..., k_new, v_new) followed by
  * kvq_decode_attn(views, ...) on the appended views, in one call (CoMixKV,

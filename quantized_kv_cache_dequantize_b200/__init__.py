@@ -10,6 +10,9 @@ Entry points (same names as the C ABI, without the ``kvq_`` prefix):
   quantize, dequantize          -- bf16 rows <-> packed b-bit codes + {s, mn}
   View, append                  -- one (agent, layer) cache; add a decode token
   decode_attn, workspace_size   -- batched split-K attention over many views
+  sparse_decode_attn            -- top-K sparse decode: the K best packed tokens
+                                   per (view, KV head) by query score, plus the
+                                   bf16 window
   decode_attn_seq               -- the same over sequences held by several views
                                    (segments) of any widths; View.new_segment
                                    starts a segment at a new width
@@ -32,7 +35,8 @@ from . import workloads  # noqa: F401  (seeded input generators)
 
 __all__ = ["quantize", "dequantize", "View", "append", "decode_attn", "workspace_size",
            "append_decode_attn", "step_workspace_size", "decode_attn_noalloc", "decode_attn_seq",
-           "seq_workspace_size", "new_seq_workspace", "MAX_SEGMENTS",
+           "seq_workspace_size", "new_seq_workspace", "MAX_SEGMENTS", "sparse_decode_attn",
+           "sparse_workspace_size",
            "card_bytes", "card_pack", "card_info", "card_unpack", "views_for_card", "save_card", "load_card", "NOALLOC_SCRATCH_BYTES", "KvqError", "lib", "row_bytes", "GROUP"]
 
 GROUP = 64
@@ -89,6 +93,11 @@ def lib():
         L.kvq_decode_attn_seq_workspace_size.restype = sz
         L.kvq_decode_attn_seq.argtypes = [ctypes.POINTER(CView), i32, P, i32, i32, i32, i32, P, f32, P, P, sz, P]
         L.kvq_decode_attn_seq.restype = i32
+        L.kvq_sparse_decode_attn_workspace_size.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, i32]
+        L.kvq_sparse_decode_attn_workspace_size.restype = sz
+        L.kvq_sparse_decode_attn.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, f32, i32, P, P, P, sz,
+                                             P]
+        L.kvq_sparse_decode_attn.restype = i32
         L.kvq_append_decode_attn.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, P, P, f32, P, P, sz, P]
         L.kvq_append_decode_attn.restype = i32
         u64 = ctypes.c_uint64
@@ -342,6 +351,33 @@ def decode_attn_seq(views, seq_begin, q: torch.Tensor, softmax_scale: float, out
                                      _ptr(q), float(softmax_scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                      _stream(stream)), "kvq_decode_attn_seq")
     return out
+
+
+def sparse_workspace_size(views, n_q_heads: int, top_k: int) -> int:
+    """kvq_sparse_decode_attn_workspace_size (0 if the arguments are invalid)."""
+    views = list(views)
+    return int(lib().kvq_sparse_decode_attn_workspace_size(_view_array(views), len(views), n_q_heads,
+                                                           views[0].n_kv_heads, views[0].head_dim, int(top_k)))
+
+
+def sparse_decode_attn(views, q: torch.Tensor, softmax_scale: float, top_k: int, out: torch.Tensor | None = None,
+                       selected: torch.Tensor | None = None, workspace: torch.Tensor | None = None, stream=None):
+    """kvq_sparse_decode_attn.  q: bf16 [n_views, H_q, D]; returns (out fp32
+    [n_views, H_q, D], selected int32 [n_views, H_kv, top_k] or None)."""
+    views = list(views)
+    n, Hq, D = q.shape
+    if workspace is None:
+        nb = sparse_workspace_size(views, Hq, top_k)
+        if nb == 0:
+            raise KvqError(KVQ_ERR_INVALID_ARG, "kvq_sparse_decode_attn_workspace_size")
+        workspace = torch.zeros(nb, dtype=torch.uint8, device=q.device)
+    if out is None:
+        out = torch.empty((n, Hq, D), dtype=torch.float32, device=q.device)
+    _check(lib().kvq_sparse_decode_attn(_view_array(views), len(views), Hq, views[0].n_kv_heads, D, _ptr(q),
+                                        float(softmax_scale), int(top_k), _ptr(out),
+                                        _ptr(selected) if selected is not None else None, _ptr(workspace),
+                                        workspace.numel(), _stream(stream)), "kvq_sparse_decode_attn")
+    return out, selected
 
 
 def _advanced(c: CView) -> CView:

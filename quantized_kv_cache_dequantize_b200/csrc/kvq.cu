@@ -14,6 +14,7 @@
 #include "kvq_attn.cuh"
 #include "kvq_card.cuh"
 #include "kvq_codec.cuh"
+#include "kvq_sparse.cuh"
 
 #define KVQ_API extern "C" __attribute__((visibility("default")))
 
@@ -786,6 +787,232 @@ kvq_status launch_attn(const AttnPlan &plan, const kvq_view *views, int32_t n_q_
     }
 }
 
+// ------------------------------------------------------ sparse decode ---
+
+// Top-K sparse decode: every (view, KV head) becomes a compact view of its own
+// (one KV head, the group's query heads): its K selected packed rows, gathered
+// into the workspace (or the view's own rows when it has no more than K), and
+// the view's bf16 window for that head, read in place.  Workspace: the
+// attention's region first (its zero part stays at offset 0 from call to
+// call), then scores, selections and compact rows.
+struct SparsePlan {
+    std::vector<kvq_view> compact;     // [n_views * H_kv]
+    std::vector<int64_t> score_off;    // per view, floats from scores_off; -1: no scoring
+    std::vector<size_t> rows_off;      // per view, bytes from compact_off (views with n_packed > K)
+    AttnPlan attn;
+    size_t scores_off = 0, sel_off = 0, compact_off = 0, total = 0;
+};
+
+kvq_status plan_sparse(const kvq_view *views, int32_t n_views, int32_t n_q_heads, int32_t n_kv_heads,
+                       int32_t head_dim, int32_t top_k, uint8_t *ws, SparsePlan &sp) {
+    if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
+    if (n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads || n_kv_heads > 65535)
+        return KVQ_ERR_INVALID_ARG;
+    if (top_k < 1 || top_k > (1 << 24)) return KVQ_ERR_INVALID_ARG;
+    const kvq_status vs = validate_views(views, n_views, true);
+    if (vs != KVQ_OK) return vs;
+    const int ng = head_dim / 64, group = n_q_heads / n_kv_heads;
+    const int64_t kc = top_k + (top_k & 1);
+    sp.score_off.assign(n_views, -1);
+    sp.rows_off.assign(n_views, 0);
+    int64_t n_scores = 0;
+    size_t rows = 0;
+    for (int i = 0; i < n_views; ++i) {
+        const kvq_view &v = views[i];
+        if (v.n_packed <= top_k) continue;
+        sp.score_off[i] = n_scores;
+        n_scores += (int64_t)n_kv_heads * v.n_packed;
+        sp.rows_off[i] = rows;
+        rows += 2 * align_up((size_t)n_kv_heads * kc * row_bytes(head_dim, v.bits), 256) +
+                2 * align_up((size_t)n_kv_heads * kc * ng * 8, 256);
+    }
+    // compact views; gathered rows get their addresses once the layout is known
+    uint8_t *const fake = reinterpret_cast<uint8_t *>(uintptr_t(1) << 20);  // aligned, for planning only
+    sp.compact.assign((size_t)n_views * n_kv_heads, kvq_view{});
+    for (int i = 0; i < n_views; ++i) {
+        const kvq_view &v = views[i];
+        const int64_t rb = row_bytes(head_dim, v.bits);
+        for (int hk = 0; hk < n_kv_heads; ++hk) {
+            kvq_view &c = sp.compact[(size_t)i * n_kv_heads + hk];
+            c.bits = v.bits;
+            c.n_window = v.n_window;
+            c.cap_window = v.cap_window;
+            c.window_head = v.window_head;
+            if (v.cap_window > 0) {
+                const size_t w = (size_t)hk * v.cap_window * head_dim * 2;
+                c.k_window = static_cast<uint8_t *>(v.k_window) + w;
+                c.v_window = static_cast<uint8_t *>(v.v_window) + w;
+            }
+            c.n_packed = std::min<int64_t>(v.n_packed, top_k);
+            if (v.n_packed <= top_k) {  // every packed row: the view's own, in place
+                c.cap_packed = v.cap_packed;
+                if (v.cap_packed > 0) {
+                    c.k_codes = static_cast<uint8_t *>(v.k_codes) + (size_t)hk * v.cap_packed * rb;
+                    c.v_codes = static_cast<uint8_t *>(v.v_codes) + (size_t)hk * v.cap_packed * rb;
+                    c.k_scalemin = v.k_scalemin + (size_t)hk * v.cap_packed * ng * 2;
+                    c.v_scalemin = v.v_scalemin + (size_t)hk * v.cap_packed * ng * 2;
+                }
+            } else {
+                c.cap_packed = kc;
+                c.k_codes = c.v_codes = fake;
+                c.k_scalemin = c.v_scalemin = reinterpret_cast<float *>(fake);
+            }
+        }
+    }
+    const kvq_status ps = plan_attn(sp.compact.data(), n_views * n_kv_heads, nullptr, 0, group, 1, head_dim, sp.attn);
+    if (ps != KVQ_OK) return ps;
+    size_t off = align_up(sp.attn.total, 256);
+    sp.scores_off = off;
+    off = align_up(off + (size_t)n_scores * 4, 256);
+    sp.sel_off = off;
+    off = align_up(off + (size_t)n_views * n_kv_heads * top_k * 4, 256);
+    sp.compact_off = off;
+    sp.total = off + rows;
+    if (!ws) return KVQ_OK;
+    for (int i = 0; i < n_views; ++i) {
+        const kvq_view &v = views[i];
+        if (v.n_packed <= top_k) continue;
+        const size_t cb = align_up((size_t)n_kv_heads * kc * row_bytes(head_dim, v.bits), 256);
+        const size_t sb = align_up((size_t)n_kv_heads * kc * ng * 8, 256);
+        uint8_t *base = ws + sp.compact_off + sp.rows_off[i];
+        for (int hk = 0; hk < n_kv_heads; ++hk) {
+            kvq_view &c = sp.compact[(size_t)i * n_kv_heads + hk];
+            const size_t h_codes = (size_t)hk * kc * row_bytes(head_dim, v.bits), h_sm = (size_t)hk * kc * ng * 8;
+            c.k_codes = base + h_codes;
+            c.v_codes = base + cb + h_codes;
+            c.k_scalemin = reinterpret_cast<float *>(base + 2 * cb + h_sm);
+            c.v_scalemin = reinterpret_cast<float *>(base + 2 * cb + sb + h_sm);
+        }
+    }
+    return KVQ_OK;
+}
+
+template <int NG, int B>
+kvq_status launch_score_grid(const kvq::ScoreArgs &a, unsigned ctas, size_t smem, cudaStream_t st) {
+    if (smem > 48 * 1024 &&
+        cudaFuncSetAttribute(kvq::score_kernel<NG, B>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+            cudaSuccess) {
+        (void)cudaGetLastError();
+        return KVQ_ERR_UNSUPPORTED;
+    }
+    kvq::score_kernel<NG, B><<<ctas, kvq::kScoreTok, smem, st>>>(a);
+    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
+template <int NG>
+kvq_status launch_score_ng(int bits, const kvq::ScoreArgs &a, unsigned ctas, size_t smem, cudaStream_t st) {
+    switch (bits) {
+        case 2: return launch_score_grid<NG, 2>(a, ctas, smem, st);
+        case 3: return launch_score_grid<NG, 3>(a, ctas, smem, st);
+        case 4: return launch_score_grid<NG, 4>(a, ctas, smem, st);
+        default: return launch_score_grid<NG, 8>(a, ctas, smem, st);
+    }
+}
+
+kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_views, int32_t n_q_heads,
+                         int32_t n_kv_heads, int32_t head_dim, const void *q, float scale, int32_t top_k, float *out,
+                         int32_t *sel, uint8_t *ws, cudaStream_t st) {
+    const int ng = head_dim / 64, group = n_q_heads / n_kv_heads;
+    float *scores = reinterpret_cast<float *>(ws + sp.scores_off);
+    // 1. scores of the views with more than K packed tokens, one launch per width group
+    std::vector<int> scored;
+    for (int i = 0; i < n_views; ++i)
+        if (sp.score_off[i] >= 0) scored.push_back(i);
+    std::stable_sort(scored.begin(), scored.end(), [&](int x, int y) { return views[x].bits < views[y].bits; });
+    const size_t smem = (size_t)group * head_dim * 4 + (size_t)group * ng * 4;
+    if (smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;
+    for (size_t v0 = 0; v0 < scored.size();) {
+        size_t v1 = v0 + 1;
+        while (v1 < scored.size() && v1 - v0 < (size_t)kvq::kSparseMaxViews &&
+               views[scored[v1]].bits == views[scored[v0]].bits)
+            ++v1;
+        kvq::ScoreArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.q = static_cast<const uint16_t *>(q);
+        a.scores = scores;
+        a.scale = scale;
+        a.n_views = (int)(v1 - v0);
+        a.n_q_heads = n_q_heads;
+        a.group = group;
+        int64_t ctas = 0;
+        for (size_t k = v0; k < v1; ++k) {
+            const int i = scored[k];
+            const kvq_view &v = views[i];
+            kvq::ScoreView &d = a.views[k - v0];
+            d.k_codes = static_cast<const uint8_t *>(v.k_codes);
+            d.k_sm = v.k_scalemin;
+            d.cap_packed = v.cap_packed;
+            d.score_off = sp.score_off[i];
+            d.n_packed = (int32_t)v.n_packed;
+            d.blocks = (int32_t)((v.n_packed + kvq::kScoreTok - 1) / kvq::kScoreTok);
+            d.cta_begin = (int32_t)ctas;
+            d.q_row = i;
+            ctas += (int64_t)n_kv_heads * d.blocks;
+        }
+        if (ctas > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
+        kvq_status es;
+        switch (ng) {
+            case 1: es = launch_score_ng<1>(views[scored[v0]].bits, a, (unsigned)ctas, smem, st); break;
+            case 2: es = launch_score_ng<2>(views[scored[v0]].bits, a, (unsigned)ctas, smem, st); break;
+            case 3: es = launch_score_ng<3>(views[scored[v0]].bits, a, (unsigned)ctas, smem, st); break;
+            default: es = launch_score_ng<4>(views[scored[v0]].bits, a, (unsigned)ctas, smem, st); break;
+        }
+        if (es != KVQ_OK) return es;
+        v0 = v1;
+    }
+    // 2. selections of every view
+    for (int v0 = 0; v0 < n_views; v0 += kvq::kSparseMaxViews) {
+        const int v1 = std::min<int>(n_views, v0 + kvq::kSparseMaxViews);
+        kvq::SelectArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.scores = scores;
+        a.sel = sel;
+        a.top_k = top_k;
+        a.n_kv_heads = n_kv_heads;
+        for (int i = v0; i < v1; ++i) {
+            a.views[i - v0].score_off = std::max<int64_t>(sp.score_off[i], 0);
+            a.views[i - v0].n_packed = (int32_t)views[i].n_packed;
+            a.views[i - v0].out_row = i;
+        }
+        kvq::select_kernel<<<dim3((unsigned)(v1 - v0), (unsigned)n_kv_heads), kvq::kSelectThreads, 0, st>>>(a);
+        if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+    }
+    // 3. gather the selected rows of the scored views
+    for (size_t v0 = 0; v0 < scored.size(); v0 += kvq::kSparseMaxViews) {
+        const size_t v1 = std::min(scored.size(), v0 + (size_t)kvq::kSparseMaxViews);
+        kvq::GatherArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.sel = sel;
+        a.top_k = top_k;
+        a.n_kv_heads = n_kv_heads;
+        a.sm_bytes = ng * 8;
+        for (size_t k = v0; k < v1; ++k) {
+            const int i = scored[k];
+            const kvq_view &v = views[i];
+            const kvq_view &c0 = sp.compact[(size_t)i * n_kv_heads];  // head 0 of the compact rows
+            kvq::GatherView &d = a.views[k - v0];
+            d.codes[0] = static_cast<const uint8_t *>(v.k_codes);
+            d.codes[1] = static_cast<const uint8_t *>(v.v_codes);
+            d.sm[0] = v.k_scalemin;
+            d.sm[1] = v.v_scalemin;
+            d.dst_codes[0] = static_cast<uint8_t *>(c0.k_codes);
+            d.dst_codes[1] = static_cast<uint8_t *>(c0.v_codes);
+            d.dst_sm[0] = c0.k_scalemin;
+            d.dst_sm[1] = c0.v_scalemin;
+            d.cap_packed = v.cap_packed;
+            d.cap_compact = c0.cap_packed;
+            d.row_bytes = (int32_t)row_bytes(head_dim, v.bits);
+            d.sel_row = i;
+        }
+        const dim3 grid((unsigned)(v1 - v0), (unsigned)n_kv_heads,
+                        (unsigned)((top_k + kvq::kGatherRows - 1) / kvq::kGatherRows));
+        kvq::gather_kernel<<<grid, 256, 0, st>>>(a);
+        if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+    }
+    // 4. attention over the compact views: one KV head each, the group's query heads
+    return launch_attn(sp.attn, sp.compact.data(), group, 1, head_dim, q, scale, out, ws, st);
+}
+
 }  // namespace
 
 // ================================================================ C ABI ===
@@ -933,6 +1160,31 @@ KVQ_API kvq_status kvq_append_decode_attn(kvq_view *views, int32_t n_views, int3
         case 3: return launch_attn_ng<3>(plan, post.data(), n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st, dep.data());
         default: return launch_attn_ng<4>(plan, post.data(), n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st, dep.data());
     }
+}
+
+KVQ_API size_t kvq_sparse_decode_attn_workspace_size(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
+                                                     int32_t n_kv_heads, int32_t head_dim, int32_t top_k) {
+    SparsePlan sp;
+    if (plan_sparse(views, n_views, n_q_heads, n_kv_heads, head_dim, top_k, nullptr, sp) != KVQ_OK) return 0;
+    return sp.total;
+}
+
+KVQ_API kvq_status kvq_sparse_decode_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
+                                          int32_t n_kv_heads, int32_t head_dim, const void *q, float softmax_scale,
+                                          int32_t top_k, float *out, int32_t *selected, void *workspace,
+                                          size_t workspace_bytes, void *stream) {
+    SparsePlan sp;
+    const kvq_status ps = plan_sparse(views, n_views, n_q_heads, n_kv_heads, head_dim, top_k, nullptr, sp);
+    if (ps != KVQ_OK) return ps;
+    if (!q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
+    if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
+    if (selected && !aligned(selected, 4)) return KVQ_ERR_INVALID_ARG;
+    if (workspace_bytes < sp.total) return KVQ_ERR_INVALID_ARG;
+    uint8_t *ws = static_cast<uint8_t *>(workspace);
+    plan_sparse(views, n_views, n_q_heads, n_kv_heads, head_dim, top_k, ws, sp);  // now with the row addresses
+    int32_t *sel = selected ? selected : reinterpret_cast<int32_t *>(ws + sp.sel_off);
+    return launch_sparse(sp, views, n_views, n_q_heads, n_kv_heads, head_dim, q, softmax_scale, top_k, out, sel, ws,
+                         static_cast<cudaStream_t>(stream));
 }
 
 KVQ_API size_t kvq_card_bytes(const kvq_view *views, int32_t n_views, int32_t n_kv_heads, int32_t head_dim) {

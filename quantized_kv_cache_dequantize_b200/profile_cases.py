@@ -17,6 +17,12 @@ CASE:
                  shape (32 layers x 8 kv heads, 32640 packed 4-bit tokens +
                  a full 128-token window), and kvq_card_unpack of that card
                  into fresh views
+  sparse-layer / sparse-8layers
+                 kvq_sparse_decode_attn (top_k 512 of the 4096 packed tokens per
+                 view and KV head, + the 128-token window) over the layer(s)
+                 of decode-layer / decode-8layers; GB/s counts the bytes the
+                 path must read: all packed K and scale/min (scoring), the
+                 selected V rows and scale/min, the window, q and out
   card-pack-decode
                  kvq_card_pack of every view of the batched decode workload
                  (10 agents x 32 layers, 4096 packed + 128 window)
@@ -33,7 +39,8 @@ import torch
 
 from . import cache as kcache
 from . import workloads as wl
-from . import card_info, card_pack, card_unpack, decode_attn, dequantize, new_workspace, quantize, views_for_card
+from . import (card_info, card_pack, card_unpack, decode_attn, dequantize, new_workspace, quantize,
+               sparse_decode_attn, sparse_workspace_size, views_for_card)
 
 
 def _time(fn, reps):
@@ -62,7 +69,8 @@ def _time(fn, reps):
 def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["decode-layer", "decode-8layers", "quantize", "dequantize", "quantize-handoff",
-                                         "dequantize-handoff", "card-pack", "card-unpack", "card-pack-decode"])
+                                         "dequantize-handoff", "card-pack", "card-unpack", "card-pack-decode", "sparse-layer",
+                                         "sparse-8layers"])
     ap.add_argument("--reps", type=int, default=20)
     a = ap.parse_args(argv)
     dev = torch.device("cuda:0")
@@ -81,6 +89,19 @@ def main(argv=None):
             t = _time(lambda: card_unpack(host, fresh, card=card, stream=torch.cuda.current_stream()), a.reps)
         else:
             t = _time(lambda: card_pack(pool.views, out=card, stream=torch.cuda.current_stream()), a.reps)
+    elif a.case.startswith("sparse"):
+        w = wl.decode_llama8b(n_layers=1 if a.case == "sparse-layer" else 8)
+        top_k = 512
+        pool = kcache.build_decode(w, dev)
+        q = kcache.decode_queries(w, device=dev)
+        ws = torch.zeros(sparse_workspace_size(pool.views, w.n_q_heads, top_k), dtype=torch.uint8, device=dev)
+        out = torch.empty((w.n_views, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+        t = _time(lambda: sparse_decode_attn(pool.views, q, w.softmax_scale, top_k, out=out, workspace=ws,
+                                             stream=torch.cuda.current_stream()), a.reps)
+        rb, ng = w.head_dim // 8 * 4, w.head_dim // 64
+        n_p = w.view_len(0)
+        nbytes = w.n_views * (w.n_kv_heads * (n_p * (rb + ng * 8) + top_k * (rb + ng * 8) + w.window * 4 * w.head_dim)
+                              + w.n_q_heads * w.head_dim * 6)
     elif a.case.startswith("decode"):
         w = wl.decode_llama8b(n_layers=1 if a.case == "decode-layer" else 8)
         pool = kcache.build_decode(w, dev)

@@ -44,13 +44,13 @@ class Case:
     q_bits: np.ndarray | None = None
 
 
-def build_case(n_q_heads, n_kv_heads, head_dim, specs, q_seed=99, device="cuda") -> Case:
+def build_case(n_q_heads, n_kv_heads, head_dim, specs, q_seed=99, device="cuda", extra_packed=0) -> Case:
     case = Case(n_q_heads, n_kv_heads, head_dim, list(specs))
     for s in specs:
         g = wl.generator(s.seed)
         mask = wl.outlier_mask(g, n_kv_heads, head_dim, s.outlier_frac, first4=s.first4)
         k, v = wl.kv_pair(g, n_kv_heads, s.n_packed + s.n_window, head_dim, mask)
-        view = kvq.View(n_kv_heads, head_dim, s.bits, max(s.n_packed, 2), s.cap_window, device=device)
+        view = kvq.View(n_kv_heads, head_dim, s.bits, max(s.n_packed + extra_packed, 2), s.cap_window, device=device)
         if s.n_packed:
             view.fill_packed(k[:, :s.n_packed].to(device), v[:, :s.n_packed].to(device))
         if s.cap_window:

@@ -149,6 +149,28 @@ def test_decode_attn_seq_validation(L):
                                  ws, NULL) == kvq.KVQ_ERR_INVALID_ARG
 
 
+def test_sparse_decode_attn_validation(L):
+    views = (kvq.CView * 2)(cview(n_packed=4096, cap_packed=4096), cview(bits=2, n_packed=16))
+    ws = L.kvq_sparse_decode_attn_workspace_size(views, 2, 8, 2, 128, 64)
+    assert ws >= 2 * 4096 * 4 + 2 * 2 * 64 * 4  # at least the scores and the selections
+    assert L.kvq_sparse_decode_attn_workspace_size(views, 2, 8, 2, 128, 0) == 0
+    assert L.kvq_sparse_decode_attn_workspace_size(views, 2, 7, 2, 128, 64) == 0
+    # top_k above every view's packed count: no scores and no gathered rows
+    big = L.kvq_sparse_decode_attn_workspace_size(views, 2, 8, 2, 128, 5000)
+    assert 0 < big
+    call = lambda **kw: L.kvq_sparse_decode_attn(
+        kw.get("views", views), 2, 8, 2, 128, kw.get("q", FAKE), 0.1, kw.get("k", 64), FAKE, kw.get("sel", NULL),
+        FAKE, kw.get("ws", ws), NULL)
+    assert call(k=0) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(ws=ws - 1) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(q=NULL) == kvq.KVQ_ERR_INVALID_ARG
+    assert call(sel=ctypes.c_void_p(0x10002)) == kvq.KVQ_ERR_INVALID_ARG
+    bad = (kvq.CView * 2)(cview(bits=5), cview())
+    assert call(views=bad) == kvq.KVQ_ERR_UNSUPPORTED
+    empty = (kvq.CView * 2)(cview(), cview(n_packed=0))
+    assert call(views=empty) == kvq.KVQ_ERR_INVALID_ARG
+
+
 def test_workspace_grows_with_views(L):
     one = (kvq.CView * 1)(cview(n_packed=4096, cap_packed=4096))
     many = (kvq.CView * 200)(*[cview(n_packed=4096, cap_packed=4096) for _ in range(200)])
