@@ -245,9 +245,9 @@ double plan_free(const kvq_view *views, const int *idx, int n_idx, int64_t units
     return best_cost;
 }
 
-template <int NG, int BSEL>
+template <int NG, int BSEL, bool SCORE = false>
 kvq_status ensure_attn_smem(size_t smem) {
-    // the attention kernel's dynamic shared-memory limit, raised once per device
+    // the attention (or score) kernel's dynamic shared-memory limit, raised once per device
     static std::mutex mu;
     static int configured[kMaxDevices] = {0};
     int dev = 0;
@@ -257,8 +257,8 @@ kvq_status ensure_attn_smem(size_t smem) {
     }
     std::lock_guard<std::mutex> lock(mu);
     if (dev >= kMaxDevices || configured[dev] < (int)smem) {
-        if (cudaFuncSetAttribute(kvq::decode_attn_kernel<NG, BSEL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 (int)smem) != cudaSuccess) {
+        if (cudaFuncSetAttribute(SCORE ? kvq::score_attn_kernel<NG, BSEL> : kvq::decode_attn_kernel<NG, BSEL>,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
             (void)cudaGetLastError();
             return KVQ_ERR_CUDA;
         }
@@ -270,8 +270,11 @@ kvq_status ensure_attn_smem(size_t smem) {
 // seq_begin == nullptr: every view is a sequence of its own (and must hold a
 // token).  Otherwise sequence s is views seq_begin[s] .. seq_begin[s+1]-1, its
 // tokens the concatenation of theirs; empty views are allowed and skipped.
+// allow_empty (internal callers): sequences without tokens are planned as
+// nothing at all.
 kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_begin, int32_t n_seqs,
-                     int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, AttnPlan &plan) {
+                     int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, AttnPlan &plan,
+                     bool allow_empty = false) {
     if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
     if (n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads || n_kv_heads > 65535)
         return KVQ_ERR_INVALID_ARG;
@@ -292,7 +295,7 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
                 tokens += views[i].n_packed + views[i].n_window;
                 used += views[i].n_packed + views[i].n_window > 0 ? 1 : 0;
             }
-            if (tokens <= 0) return KVQ_ERR_INVALID_ARG;
+            if (tokens <= 0 && !allow_empty) return KVQ_ERR_INVALID_ARG;
             if (used > KVQ_MAX_SEGMENTS) return KVQ_ERR_UNSUPPORTED;
         }
     }
@@ -410,36 +413,33 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
     return KVQ_OK;
 }
 
-// The attention grid of one launch: the kernel specialized for its width.
-template <int NG>
-kvq_status launch_attn_grid(int bits, size_t smem, const cudaLaunchConfig_t &cfg, const kvq::AttnParams &prm) {
-    kvq_status es;
-    cudaError_t e;
-    switch (bits) {
-        case 2:
-            if ((es = ensure_attn_smem<NG, 2>(smem)) != KVQ_OK) return es;
-            e = cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, 2>, prm);
-            break;
-        case 3:
-            if ((es = ensure_attn_smem<NG, 3>(smem)) != KVQ_OK) return es;
-            e = cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, 3>, prm);
-            break;
-        case 4:
-            if ((es = ensure_attn_smem<NG, 4>(smem)) != KVQ_OK) return es;
-            e = cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, 4>, prm);
-            break;
-        default:
-            if ((es = ensure_attn_smem<NG, 8>(smem)) != KVQ_OK) return es;
-            e = cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, 8>, prm);
-            break;
-    }
+// The attention grid of one launch: the kernel specialized for its width
+// (or its score-only variant).
+template <int NG, int BSEL, bool SCORE>
+kvq_status launch_attn_width(size_t smem, const cudaLaunchConfig_t &cfg, const kvq::AttnParams &prm) {
+    const kvq_status es = ensure_attn_smem<NG, BSEL, SCORE>(smem);
+    if (es != KVQ_OK) return es;
+    const cudaError_t e = SCORE ? cudaLaunchKernelEx(&cfg, kvq::score_attn_kernel<NG, BSEL>, prm)
+                                : cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, BSEL>, prm);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
+template <int NG, bool SCORE>
+kvq_status launch_attn_grid(int bits, size_t smem, const cudaLaunchConfig_t &cfg, const kvq::AttnParams &prm) {
+    switch (bits) {
+        case 2: return launch_attn_width<NG, 2, SCORE>(smem, cfg, prm);
+        case 3: return launch_attn_width<NG, 3, SCORE>(smem, cfg, prm);
+        case 4: return launch_attn_width<NG, 4, SCORE>(smem, cfg, prm);
+        default: return launch_attn_width<NG, 8, SCORE>(smem, cfg, prm);
+    }
+}
+
+// scores != nullptr: the score-only grids (views without windows, one head
+// block), each view's scores at scores + score_off[view]
 template <int NG>
 kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n_q_heads, int32_t n_kv_heads,
                           const void *q, float scale, float *out, uint8_t *ws, cudaStream_t st,
-                          const int32_t *dep = nullptr) {
+                          const int32_t *dep = nullptr, float *scores = nullptr, const int64_t *score_off = nullptr) {
     kvq::AttnParams prm;
     std::memset(&prm, 0, sizeof prm);
     prm.q = static_cast<const uint16_t *>(q);
@@ -491,6 +491,7 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
             d.seq_chunks = plan.seq_chunks[plan.seq_of[i]];
             d.dep_step[0] = prm.fused ? dep[2 * i] : -1;
             d.dep_step[1] = prm.fused ? dep[2 * i + 1] : -1;
+            d.score_off = scores ? score_off[i] : 0;
             begin += d.n_chunks;
         }
         // The grid carries a programmatic dependency on the preceding work in
@@ -508,7 +509,9 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
         cfg.stream = st;
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
-        const kvq_status es = launch_attn_grid<NG>(L.bits, plan.smem, cfg, prm);
+        prm.scores = scores;
+        const kvq_status es = scores ? launch_attn_grid<NG, true>(L.bits, plan.smem, cfg, prm)
+                                     : launch_attn_grid<NG, false>(L.bits, plan.smem, cfg, prm);
         if (es != KVQ_OK) return es;
     }
     return KVQ_OK;
@@ -805,6 +808,7 @@ struct SparsePlan {
 
 kvq_status plan_sparse(const kvq_view *views, int32_t n_views, int32_t n_q_heads, int32_t n_kv_heads,
                        int32_t head_dim, int32_t top_k, uint8_t *ws, SparsePlan &sp) {
+    sp = SparsePlan();
     if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
     if (n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads || n_kv_heads > 65535)
         return KVQ_ERR_INVALID_ARG;
@@ -887,6 +891,25 @@ kvq_status plan_sparse(const kvq_view *views, int32_t n_views, int32_t n_q_heads
     return KVQ_OK;
 }
 
+// A launch with a programmatic dependency on the preceding work in the stream
+// (the kernel starts with griddepcontrol.wait).
+template <typename Args>
+kvq_status launch_pdl(void (*kernel)(Args), dim3 grid, unsigned block, size_t smem, cudaStream_t st,
+                      const Args &a) {
+    cudaLaunchAttribute attr;
+    attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr.val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = &attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, kernel, a) == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
 template <int NG, int B>
 kvq_status launch_score_grid(const kvq::ScoreArgs &a, unsigned ctas, size_t smem, cudaStream_t st) {
     if (smem > 48 * 1024 &&
@@ -895,8 +918,7 @@ kvq_status launch_score_grid(const kvq::ScoreArgs &a, unsigned ctas, size_t smem
         (void)cudaGetLastError();
         return KVQ_ERR_UNSUPPORTED;
     }
-    kvq::score_kernel<NG, B><<<ctas, kvq::kScoreTok, smem, st>>>(a);
-    return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+    return launch_pdl(kvq::score_kernel<NG, B>, dim3(ctas), kvq::kScoreTok, smem, st, a);
 }
 
 template <int NG>
@@ -914,10 +936,40 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
                          int32_t *sel, uint8_t *ws, cudaStream_t st) {
     const int ng = head_dim / 64, group = n_q_heads / n_kv_heads;
     float *scores = reinterpret_cast<float *>(ws + sp.scores_off);
-    // 1. scores of the views with more than K packed tokens, one launch per width group
+    // 1. scores of the views with more than K packed tokens.  A group of at
+    // most 8 query heads: the attention grid's QK path (tensor cores) over the
+    // packed parts, scores in base-2 logit units (the order is that of the
+    // logits); wider groups: the SIMT score kernel.
     std::vector<int> scored;
     for (int i = 0; i < n_views; ++i)
         if (sp.score_off[i] >= 0) scored.push_back(i);
+    if (group <= kvq::kHeadsPerCta && !scored.empty()) {
+        // every view its own sequence (q row = view index); views not scored
+        // are left empty, windows are left out
+        std::vector<kvq_view> packed(views, views + n_views);
+        std::vector<int32_t> seq(n_views + 1);
+        for (int i = 0; i < n_views; ++i) {
+            kvq_view &v = packed[i];
+            v.n_window = v.cap_window = v.window_head = 0;
+            v.k_window = v.v_window = nullptr;
+            if (sp.score_off[i] < 0) v.n_packed = 0;
+            seq[i] = i;
+        }
+        seq[n_views] = n_views;
+        AttnPlan splan;
+        const kvq_status ps =
+            plan_attn(packed.data(), n_views, seq.data(), n_views, n_q_heads, n_kv_heads, head_dim, splan, true);
+        if (ps != KVQ_OK) return ps;
+        kvq_status es;
+        switch (ng) {
+            case 1: es = launch_attn_ng<1>(splan, packed.data(), n_q_heads, n_kv_heads, q, scale, nullptr, ws, st, nullptr, scores, sp.score_off.data()); break;
+            case 2: es = launch_attn_ng<2>(splan, packed.data(), n_q_heads, n_kv_heads, q, scale, nullptr, ws, st, nullptr, scores, sp.score_off.data()); break;
+            case 3: es = launch_attn_ng<3>(splan, packed.data(), n_q_heads, n_kv_heads, q, scale, nullptr, ws, st, nullptr, scores, sp.score_off.data()); break;
+            default: es = launch_attn_ng<4>(splan, packed.data(), n_q_heads, n_kv_heads, q, scale, nullptr, ws, st, nullptr, scores, sp.score_off.data()); break;
+        }
+        if (es != KVQ_OK) return es;
+        scored.clear();  // nothing left for the SIMT kernel
+    }
     std::stable_sort(scored.begin(), scored.end(), [&](int x, int y) { return views[x].bits < views[y].bits; });
     const size_t smem = (size_t)group * head_dim * 4 + (size_t)group * ng * 4;
     if (smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;
@@ -944,7 +996,8 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
             d.cap_packed = v.cap_packed;
             d.score_off = sp.score_off[i];
             d.n_packed = (int32_t)v.n_packed;
-            d.blocks = (int32_t)((v.n_packed + kvq::kScoreTok - 1) / kvq::kScoreTok);
+            d.blocks = (int32_t)((v.n_packed + kvq::kScoreTok * kvq::kScoreBlocks - 1) /
+                                 (kvq::kScoreTok * kvq::kScoreBlocks));
             d.cta_begin = (int32_t)ctas;
             d.q_row = i;
             ctas += (int64_t)n_kv_heads * d.blocks;
@@ -960,7 +1013,8 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
         if (es != KVQ_OK) return es;
         v0 = v1;
     }
-    // 2. selections of every view
+    // 2. selections of every view; the views with more than K packed tokens
+    // also copy their selected rows into the compact views
     for (int v0 = 0; v0 < n_views; v0 += kvq::kSparseMaxViews) {
         const int v1 = std::min<int>(n_views, v0 + kvq::kSparseMaxViews);
         kvq::SelectArgs a;
@@ -969,28 +1023,16 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
         a.sel = sel;
         a.top_k = top_k;
         a.n_kv_heads = n_kv_heads;
-        for (int i = v0; i < v1; ++i) {
-            a.views[i - v0].score_off = std::max<int64_t>(sp.score_off[i], 0);
-            a.views[i - v0].n_packed = (int32_t)views[i].n_packed;
-            a.views[i - v0].out_row = i;
-        }
-        kvq::select_kernel<<<dim3((unsigned)(v1 - v0), (unsigned)n_kv_heads), kvq::kSelectThreads, 0, st>>>(a);
-        if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
-    }
-    // 3. gather the selected rows of the scored views
-    for (size_t v0 = 0; v0 < scored.size(); v0 += kvq::kSparseMaxViews) {
-        const size_t v1 = std::min(scored.size(), v0 + (size_t)kvq::kSparseMaxViews);
-        kvq::GatherArgs a;
-        std::memset(&a, 0, sizeof a);
-        a.sel = sel;
-        a.top_k = top_k;
-        a.n_kv_heads = n_kv_heads;
         a.sm_bytes = ng * 8;
-        for (size_t k = v0; k < v1; ++k) {
-            const int i = scored[k];
+        size_t smem = 0;
+        for (int i = v0; i < v1; ++i) {
             const kvq_view &v = views[i];
+            kvq::SelectView &d = a.views[i - v0];
+            d.score_off = std::max<int64_t>(sp.score_off[i], 0);
+            d.n_packed = (int32_t)v.n_packed;
+            d.out_row = i;
+            if (sp.score_off[i] < 0) continue;
             const kvq_view &c0 = sp.compact[(size_t)i * n_kv_heads];  // head 0 of the compact rows
-            kvq::GatherView &d = a.views[k - v0];
             d.codes[0] = static_cast<const uint8_t *>(v.k_codes);
             d.codes[1] = static_cast<const uint8_t *>(v.v_codes);
             d.sm[0] = v.k_scalemin;
@@ -1002,12 +1044,17 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
             d.cap_packed = v.cap_packed;
             d.cap_compact = c0.cap_packed;
             d.row_bytes = (int32_t)row_bytes(head_dim, v.bits);
-            d.sel_row = i;
+            d.staged = v.n_packed <= kvq::kSelectStageMax ? 1 : 0;
+            if (d.staged) smem = std::max(smem, (size_t)v.n_packed * 4);
         }
-        const dim3 grid((unsigned)(v1 - v0), (unsigned)n_kv_heads,
-                        (unsigned)((top_k + kvq::kGatherRows - 1) / kvq::kGatherRows));
-        kvq::gather_kernel<<<grid, 256, 0, st>>>(a);
-        if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+        if (smem > 48 * 1024 && cudaFuncSetAttribute(kvq::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                     (int)smem) != cudaSuccess) {
+            (void)cudaGetLastError();
+            return KVQ_ERR_CUDA;
+        }
+        const kvq_status es = launch_pdl(kvq::select_kernel, dim3((unsigned)(v1 - v0), (unsigned)n_kv_heads),
+                                         kvq::kSelectThreads, smem, st, a);
+        if (es != KVQ_OK) return es;
     }
     // 4. attention over the compact views: one KV head each, the group's query heads
     return launch_attn(sp.attn, sp.compact.data(), group, 1, head_dim, q, scale, out, ws, st);

@@ -68,6 +68,7 @@ struct AttnView {
     int32_t dep_step[2];         // packed / window step whose rows the preceding append grid
                                  // writes (-1: none); with AttnParams::fused its copy waits
                                  // for that grid, every other copy starts at once
+    int64_t score_off;           // score grids: float offset of the view's head-0 scores
 };
 
 struct AttnParams {
@@ -86,6 +87,7 @@ struct AttnParams {
     int32_t ring_bytes;          // shared-memory ring per warp
     int32_t fused;               // 1: launched right behind this step's append grid (see dep_step)
     int32_t chain;               // 1: a later launch of a call: no wait at entry, wait before exit
+    float *scores;               // score grids: [view][H_kv][n_packed] largest logit of the CTA's heads
     AttnView views[kAttnMaxViews];
 };
 
@@ -669,7 +671,10 @@ __device__ __forceinline__ void combine_unit(const AttnParams &p, const AttnView
 // own ring of S equal slots, each with an mbarrier that counts the bytes of
 // the block's bulk copies; one lane issues the copies and a slot is refilled
 // as soon as the warp has consumed it.
-template <int NG, int B, bool WINDOW>
+// SCORE: the packed part's K rows only (no V copies, no softmax, no PV): each
+// token's largest logit over the CTA's query heads (base-2 units, scale_log2
+// applied) goes to p.scores; no partials, no combine.
+template <int NG, int B, bool WINDOW, bool SCORE = false>
 __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V, int c, int hk, int z,
                                           uint8_t *smem) {
     constexpr int D = 64 * NG;
@@ -737,11 +742,11 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             const bool full = n == kStepTok;
             const uint32_t bc = full ? (uint32_t)(kStepTok * RB) : round16((uint32_t)(n * RB));
             const uint32_t bs = full ? (uint32_t)(kStepTok * NG * 8) : round16((uint32_t)(n * NG * 8));
-            mbar_arrive_expect_tx_if(issuer, bar, 2 * (bc + bs));
+            mbar_arrive_expect_tx_if(issuer, bar, SCORE ? bc + bs : 2 * (bc + bs));
             bulk_copy_g2s_if(issuer, dst, src_kc, bc, bar);
-            bulk_copy_g2s_if(issuer, dst + kOffV, src_vc, bc, bar);
+            if (!SCORE) bulk_copy_g2s_if(issuer, dst + kOffV, src_vc, bc, bar);
             bulk_copy_g2s_if(issuer, dst + kOffKs, src_ks, bs, bar);
-            bulk_copy_g2s_if(issuer, dst + kOffVs, src_vs, bs, bar);
+            if (!SCORE) bulk_copy_g2s_if(issuer, dst + kOffVs, src_vs, bs, bar);
             src_kc += (int64_t)kAdvTok * RB;
             src_vc += (int64_t)kAdvTok * RB;
             src_ks += (int64_t)kAdvTok * NG * 2;
@@ -858,6 +863,30 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     int left = n_tok - kStepTok * warp;
     for (int i = 0; i < n_my; ++i, left -= kAdvTok) {
         if (!wait_cur()) { failed = true; break; }
+        if constexpr (SCORE && !WINDOW) {
+            float lg[4][2];
+            if (left >= kStepTok) {
+                packed_qk2<B, NG>(st, stage, p.scale_log2, gid, tig, lg);
+            } else {
+                packed_qk1<B, NG>(st, stage, stage + kOffKs, min(left, kTile), p.scale_log2, gid, tig, lg[0], lg[1]);
+                if (left > kTile)
+                    packed_qk1<B, NG>(st, stage + kTile * RB, stage + kOffKs + kTile * NG * 8, left - kTile,
+                                      p.scale_log2, gid, tig, lg[2], lg[3]);
+            }
+            release_cur();
+            // largest logit over the CTA's heads (2 per lane, 8 per quad)
+            float *dst = p.scores + V.score_off + (int64_t)hk * V.n_packed + tok0 +
+                         (int64_t)kStepTok * (warp + i * kAttnWarps);
+#pragma unroll
+            for (int r = 0; r < 4; ++r) {
+                float m = fmaxf(2 * tig < nh ? lg[r][0] : -INFINITY, 2 * tig + 1 < nh ? lg[r][1] : -INFINITY);
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                const int row = (r >> 1) * kTile + gid + (r & 1) * 8;
+                if (tig == 0 && row < left) dst[row] = m;
+            }
+            continue;
+        }
         if constexpr (!WINDOW) {
             if (left >= kStepTok) {
                 // two full 16-token tiles, one softmax update over 32 tokens
@@ -906,6 +935,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         }
         if (lane == 0) atomicExch(p.status, 1u);
     }
+    if constexpr (SCORE) return;
 
     // ---- warp partial -> this warp's ring area (all its copies have landed)
 #pragma unroll
@@ -999,7 +1029,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
 // host groups the views of a call by width, one launch per group).  With all
 // four widths compiled into one function, about one instruction fetch in
 // five missed the SM's instruction cache, against one in fifty for one width.
-template <int NG, int BSEL>
+template <int NG, int BSEL, bool SCORE = false>
 __device__ __forceinline__ void decode_attn_body(const AttnParams &p, uint8_t *smem) {
     // Inputs may come from the preceding grid.  Behind a fused append, only
     // the copies of the blocks the append writes wait for it (see dep_step):
@@ -1018,8 +1048,12 @@ __device__ __forceinline__ void decode_attn_body(const AttnParams &p, uint8_t *s
     const int c = bx - V.chunk_begin;
     const int hk = blockIdx.y, z = blockIdx.z;
     if (c >= V.n_chunks) return;  // never launched by the host planner; defensive
-    if (c >= V.n_chunks_packed) attn_item<NG, 4, true>(p, V, c, hk, z, smem);
-    else attn_item<NG, BSEL, false>(p, V, c, hk, z, smem);
+    if constexpr (SCORE) {
+        if (c < V.n_chunks_packed) attn_item<NG, BSEL, false, true>(p, V, c, hk, z, smem);
+    } else {
+        if (c >= V.n_chunks_packed) attn_item<NG, 4, true>(p, V, c, hk, z, smem);
+        else attn_item<NG, BSEL, false>(p, V, c, hk, z, smem);
+    }
 }
 
 template <int NG, int BSEL>
@@ -1030,6 +1064,17 @@ __global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
     decode_attn_body<NG, BSEL>(p, smem);
     // a later launch of a call completes only after the one before it, so
     // the call's last grid completes after all of them
+    if (p.chain) pdl_wait();
+}
+
+// Scores of packed tokens for the top-K selection: the attention grid's QK
+// path alone over views without windows, one query-head block per KV head.
+template <int NG, int BSEL>
+__global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
+    score_attn_kernel(const __grid_constant__ AttnParams p) {
+    static_assert(BSEL == 2 || BSEL == 3 || BSEL == 4 || BSEL == 8, "width");
+    extern __shared__ __align__(128) uint8_t smem[];
+    decode_attn_body<NG, BSEL, true>(p, smem);
     if (p.chain) pdl_wait();
 }
 

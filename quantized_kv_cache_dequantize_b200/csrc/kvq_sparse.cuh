@@ -1,6 +1,6 @@
 // kvq_sparse.cuh -- top-K sparse decode attention over the packed cache:
 // score every packed token against the query group, select the K best per
-// (view, KV head), gather their rows into a compact per-head view; the
+// (view, KV head) and gather their rows into a compact per-head view; the
 // attention kernel then runs over the compact rows plus the bf16 window.
 //
 // "Reasoning-Aware Error-Bounded KV-Cache Compression and Sparse Attention
@@ -14,13 +14,17 @@
 
 #include <cstdint>
 
+#include "kvq_ptx.cuh"
+
 namespace kvq {
 
-constexpr int kSparseMaxViews = 96;  // views per score / select / gather launch
-constexpr int kScoreTok = 128;       // tokens per score CTA, one per thread
+constexpr int kSparseMaxViews = 96;  // views per score / select launch
+constexpr int kScoreTok = 128;       // threads of a score CTA, one token each at a time
+constexpr int kScoreBlocks = 4;      // blocks of kScoreTok tokens per score CTA
 constexpr int kScoreHeads = 8;       // query heads per register batch
 constexpr int kSelectThreads = 512;
-constexpr int kGatherRows = 32;      // selected rows per gather CTA
+constexpr int kSelectStageMax = 45056;  // keys a select CTA stages in shared memory (176 KiB)
+constexpr int kSelectIdxMax = 4096;     // selections a select CTA also keeps in shared memory
 
 struct ScoreView {
     const uint8_t *k_codes;   // [H_kv][cap][RB]
@@ -28,7 +32,7 @@ struct ScoreView {
     int64_t cap_packed;
     int64_t score_off;        // float offset of head 0's scores; head hk at + hk * n_packed
     int32_t n_packed;
-    int32_t blocks;           // token blocks of kScoreTok per head
+    int32_t blocks;           // score CTAs per head (kScoreBlocks * kScoreTok tokens each)
     int32_t cta_begin;        // first CTA of this view in the launch
     int32_t q_row;            // row of q: [q_row][H_q][D]
 };
@@ -43,15 +47,20 @@ struct ScoreArgs {
     ScoreView views[kSparseMaxViews];
 };
 
-// One thread per packed token: the token's K codes are unpacked group by
-// group into exact floats, dotted with each query head's 64 q values (fp32,
-// fixed order), scaled by s and offset by mn times the q group sum.
+// One thread per packed token, kScoreBlocks blocks of kScoreTok tokens per
+// CTA: the token's K codes are unpacked 16 at a time into exact floats and
+// dotted with each query head's q values (fp32, fixed order); per group the
+// sum is scaled by s and offset by mn times the q group sum.
 template <int NG, int B>
 __global__ void __launch_bounds__(kScoreTok) score_kernel(const __grid_constant__ ScoreArgs a) {
     constexpr int D = 64 * NG;
     constexpr int RB = 8 * B * NG;
     extern __shared__ __align__(16) float score_smem[];
-    const int bx = blockIdx.x, tid = threadIdx.x;
+    // q and the cache may come from the preceding grid; the next stage may be
+    // scheduled as slots free up (it waits for this grid in turn)
+    pdl_wait();
+    pdl_launch_dependents();
+    const int bx = blockIdx.x, tid = threadIdx.x, lane = tid & 31;
     int lo = 0, hi = a.n_views - 1;
     while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -59,73 +68,100 @@ __global__ void __launch_bounds__(kScoreTok) score_kernel(const __grid_constant_
     }
     const ScoreView &v = a.views[lo];
     const int local = bx - v.cta_begin;
-    const int hk = local / v.blocks, tb = local - hk * v.blocks;
+    const int hk = local / v.blocks, tb0 = (local - hk * v.blocks) * kScoreBlocks;
     const int G = a.group;
     float *qs = score_smem;          // [G][D]
     float *qsum = qs + G * D;        // [G][NG]
     const uint16_t *qp = a.q + ((int64_t)v.q_row * a.n_q_heads + (int64_t)hk * G) * D;
-    for (int i = tid; i < G * D; i += kScoreTok) qs[i] = __uint_as_float((uint32_t)qp[i] << 16);
-    __syncthreads();
-    for (int i = tid; i < G * NG; i += kScoreTok) {
-        const float *x = qs + (i / NG) * D + (i % NG) * 64;
-        float t = 0.f;
-        for (int j = 0; j < 64; ++j) t += x[j];
-        qsum[i] = t;
-    }
-    __syncthreads();
-    const int t = tb * kScoreTok + tid;
-    if (t >= v.n_packed) return;
-    const uint8_t *row = v.k_codes + ((int64_t)hk * v.cap_packed + t) * RB;
-    const float2 *smr = reinterpret_cast<const float2 *>(v.k_sm + ((int64_t)hk * v.cap_packed + t) * NG * 2);
-    float best = -INFINITY;
-    for (int h0 = 0; h0 < G; h0 += kScoreHeads) {
-        float l[kScoreHeads];
+    // q to fp32, and each (head, group) sum of 64 values: 4 values per lane,
+    // then 16 lanes by shuffles (fixed order)
+    for (int i0 = 0; i0 < G * D; i0 += 4 * kScoreTok) {
+        const int i = i0 + 4 * tid;
+        float x[4] = {0.f, 0.f, 0.f, 0.f};
+        if (i < G * D) {
 #pragma unroll
-        for (int h = 0; h < kScoreHeads; ++h) l[h] = 0.f;
-#pragma unroll 1
-        for (int g = 0; g < NG; ++g) {
-            // the group's 64 codes: 8*B bytes, LSB-first little-endian
-            uint64_t w[B];
-#pragma unroll
-            for (int i = 0; i < B; ++i) w[i] = __ldg(reinterpret_cast<const unsigned long long *>(row + g * 8 * B) + i);
-            float cf[64];
-#pragma unroll
-            for (int j = 0; j < 64; ++j) {
-                const int bit = j * B, wi = bit >> 6, sh = bit & 63;
-                uint32_t c = (uint32_t)(w[wi] >> sh);
-                if (sh + B > 64) c |= (uint32_t)(w[wi + 1] << (64 - sh));
-                c &= (1u << B) - 1u;
-                cf[j] = __uint_as_float(0x4B000000u | c) - 8388608.0f;  // exact: c < 2^23
-            }
-            const float2 sm = __ldg(smr + g);
-#pragma unroll
-            for (int h = 0; h < kScoreHeads; ++h) {
-                if (h0 + h < G) {
-                    const float4 *q4 = reinterpret_cast<const float4 *>(qs + (h0 + h) * D + g * 64);
-                    float acc = 0.f;
-#pragma unroll
-                    for (int j = 0; j < 16; ++j) {
-                        const float4 x = q4[j];
-                        acc = fmaf(x.x, cf[4 * j], acc);
-                        acc = fmaf(x.y, cf[4 * j + 1], acc);
-                        acc = fmaf(x.z, cf[4 * j + 2], acc);
-                        acc = fmaf(x.w, cf[4 * j + 3], acc);
-                    }
-                    l[h] = fmaf(sm.x, acc, fmaf(sm.y, qsum[(h0 + h) * NG + g], l[h]));
-                }
+            for (int j = 0; j < 4; ++j) {
+                x[j] = __uint_as_float((uint32_t)qp[i + j] << 16);
+                qs[i + j] = x[j];
             }
         }
+        float t = (x[0] + x[1]) + (x[2] + x[3]);
 #pragma unroll
-        for (int h = 0; h < kScoreHeads; ++h)
-            if (h0 + h < G) best = fmaxf(best, a.scale * l[h]);
+        for (int o = 1; o < 16; o <<= 1) t += __shfl_xor_sync(0xFFFFFFFFu, t, o);
+        if ((lane & 15) == 0 && i < G * D) qsum[i / 64] = t;
     }
-    a.scores[v.score_off + (int64_t)hk * v.n_packed + t] = best;
+    __syncthreads();
+    for (int tb = tb0; tb < tb0 + kScoreBlocks; ++tb) {
+        const int t = tb * kScoreTok + tid;
+        if (t >= v.n_packed) break;
+        const uint8_t *row = v.k_codes + ((int64_t)hk * v.cap_packed + t) * RB;
+        const float2 *smr = reinterpret_cast<const float2 *>(v.k_sm + ((int64_t)hk * v.cap_packed + t) * NG * 2);
+        float best = -INFINITY;
+        for (int h0 = 0; h0 < G; h0 += kScoreHeads) {
+            float l[kScoreHeads];
+#pragma unroll
+            for (int h = 0; h < kScoreHeads; ++h) l[h] = 0.f;
+#pragma unroll 1
+            for (int g = 0; g < NG; ++g) {
+                // the group's 64 codes: 8*B bytes, LSB-first little-endian
+                uint64_t w[B];
+#pragma unroll
+                for (int i = 0; i < B; ++i)
+                    w[i] = __ldg(reinterpret_cast<const unsigned long long *>(row + g * 8 * B) + i);
+                float acc[kScoreHeads];
+#pragma unroll
+                for (int h = 0; h < kScoreHeads; ++h) acc[h] = 0.f;
+#pragma unroll
+                for (int c0 = 0; c0 < 64; c0 += 16) {
+                    float cf[16];
+#pragma unroll
+                    for (int j = 0; j < 16; ++j) {
+                        const int bit = (c0 + j) * B, wi = bit >> 6, sh = bit & 63;
+                        uint32_t c = (uint32_t)(w[wi] >> sh);
+                        if (sh + B > 64) c |= (uint32_t)(w[wi + 1] << (64 - sh));
+                        c &= (1u << B) - 1u;
+                        cf[j] = __uint_as_float(0x4B000000u | c) - 8388608.0f;  // exact: c < 2^23
+                    }
+#pragma unroll
+                    for (int h = 0; h < kScoreHeads; ++h) {
+                        if (h0 + h < G) {
+                            const float4 *q4 = reinterpret_cast<const float4 *>(qs + (h0 + h) * D + g * 64 + c0);
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const float4 x = q4[j];
+                                acc[h] = fmaf(x.x, cf[4 * j], acc[h]);
+                                acc[h] = fmaf(x.y, cf[4 * j + 1], acc[h]);
+                                acc[h] = fmaf(x.z, cf[4 * j + 2], acc[h]);
+                                acc[h] = fmaf(x.w, cf[4 * j + 3], acc[h]);
+                            }
+                        }
+                    }
+                }
+                const float2 sm = __ldg(smr + g);
+#pragma unroll
+                for (int h = 0; h < kScoreHeads; ++h)
+                    if (h0 + h < G) l[h] = fmaf(sm.x, acc[h], fmaf(sm.y, qsum[(h0 + h) * NG + g], l[h]));
+            }
+#pragma unroll
+            for (int h = 0; h < kScoreHeads; ++h)
+                if (h0 + h < G) best = fmaxf(best, a.scale * l[h]);
+        }
+        a.scores[v.score_off + (int64_t)hk * v.n_packed + t] = best;
+    }
 }
 
 struct SelectView {
     int64_t score_off;        // as ScoreView::score_off
-    int32_t n_packed;         // n_packed <= top_k: every token, no scores read
+    int32_t n_packed;         // n_packed <= top_k: every token, no scores read, no rows copied
     int32_t out_row;          // row of the selection: [out_row][H_kv][top_k]
+    const uint8_t *codes[2];  // source K, V codes [H_kv][cap][RB]
+    const float *sm[2];       // source K, V scale/min [H_kv][cap][NG][2]
+    uint8_t *dst_codes[2];    // compact [H_kv][cap_c][RB]
+    float *dst_sm[2];         // compact [H_kv][cap_c][NG][2]
+    int64_t cap_packed;
+    int64_t cap_compact;
+    int32_t row_bytes;
+    int32_t staged;           // 1: the head's keys fit the launch's shared-memory stage
 };
 
 struct SelectArgs {
@@ -133,6 +169,7 @@ struct SelectArgs {
     int32_t *sel;             // int32 [n_views][H_kv][top_k], ascending, -1 padded
     int32_t top_k;
     int32_t n_kv_heads;
+    int32_t sm_bytes;         // scale/min bytes per row: (D/64) * 8
     SelectView views[kSparseMaxViews];
 };
 
@@ -142,41 +179,19 @@ __device__ __forceinline__ uint32_t order_key(float f) {
     return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
 }
 
-// Exclusive prefix sum over the block's threads (kSelectThreads), in thread order.
-__device__ __forceinline__ uint32_t block_excl_scan(uint32_t x, uint32_t *warp_tot) {
-    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-    uint32_t inc = x;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-        const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, inc, o);
-        if (lane >= o) inc += y;
-    }
-    if (lane == 31) warp_tot[warp] = inc;
-    __syncthreads();
-    if (warp == 0) {
-        uint32_t t = lane < kSelectThreads / 32 ? warp_tot[lane] : 0u;
-        uint32_t ti = t;
-#pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, ti, o);
-            if (lane >= o) ti += y;
-        }
-        if (lane < kSelectThreads / 32) warp_tot[lane] = ti - t;
-    }
-    __syncthreads();
-    const uint32_t r = warp_tot[warp] + inc - x;
-    __syncthreads();  // warp_tot is reused by the next scan
-    return r;
-}
-
 // One CTA per (view, KV head): radix select of the K largest scores (four
-// 8-bit digit passes from the top), then an ordered compaction that writes
-// the selected indices in ascending order, equal scores at the threshold
-// taken from the lowest index up.
+// 8-bit digit passes from the top, over keys staged in shared memory when
+// they fit), an ordered compaction that writes the selected indices in
+// ascending order (equal scores at the threshold taken from the lowest index
+// up), then the copy of the selected packed rows (K and V codes and
+// scale/min) to consecutive rows of the compact view.
 __global__ void __launch_bounds__(kSelectThreads) select_kernel(const __grid_constant__ SelectArgs a) {
+    extern __shared__ uint32_t skeys[];
     __shared__ uint32_t hist[256];
-    __shared__ uint32_t warp_tot[kSelectThreads / 32];
+    __shared__ int32_t sidx[kSelectIdxMax];
     __shared__ uint32_t pick[2];
+    pdl_wait();  // the scores of the preceding grid
+    pdl_launch_dependents();
     const SelectView &v = a.views[blockIdx.x];
     const int hk = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
     const int n = v.n_packed, K = a.top_k;
@@ -186,13 +201,36 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const __grid_con
         return;
     }
     const float *sc = a.scores + v.score_off + (int64_t)hk * n;
+    const bool staged = v.staged != 0;
+    if (staged) {
+        // eight loads in flight per thread
+        for (int i0 = tid; i0 < n; i0 += 8 * kSelectThreads) {
+            float x[8];
+#pragma unroll
+            for (int j = 0; j < 8; ++j) x[j] = i0 + j * kSelectThreads < n ? __ldcg(sc + i0 + j * kSelectThreads) : 0.f;
+#pragma unroll
+            for (int j = 0; j < 8; ++j)
+                if (i0 + j * kSelectThreads < n) skeys[i0 + j * kSelectThreads] = order_key(x[j]);
+        }
+        __syncthreads();
+    }
+    auto key_at = [&](int i) { return staged ? skeys[i] : order_key(sc[i]); };
     uint32_t prefix = 0, mask = 0, remaining = (uint32_t)K;
     for (int shift = 24; shift >= 0; shift -= 8) {
         for (int i = tid; i < 256; i += kSelectThreads) hist[i] = 0u;
         __syncthreads();
-        for (int i = tid; i < n; i += kSelectThreads) {
-            const uint32_t k = order_key(sc[i]);
-            if ((k & mask) == prefix) atomicAdd(&hist[(k >> shift) & 255u], 1u);
+        // scores cluster in few bins (the top digit holds the sign and most of
+        // the exponent): lanes with the same bin add once, with their count
+        for (int i0 = 0; i0 < n; i0 += kSelectThreads) {
+            const int i = i0 + tid;
+            const uint32_t k = i < n ? key_at(i) : 0u;
+            const bool in = i < n && (k & mask) == prefix;
+            const uint32_t bin = (k >> shift) & 255u;
+            const uint32_t act = __ballot_sync(0xFFFFFFFFu, in);
+            if (in) {
+                const uint32_t peers = __match_any_sync(act, bin);
+                if (lane == __ffs(peers) - 1) atomicAdd(&hist[bin], (uint32_t)__popc(peers));
+            }
         }
         __syncthreads();
         if (tid < 32) {
@@ -228,63 +266,66 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const __grid_con
         remaining -= pick[1];
         __syncthreads();
     }
-    // keys above the threshold key `prefix`, and the first `remaining` equal to it
-    const int per = (n + kSelectThreads - 1) / kSelectThreads;
-    const int b0 = min(n, tid * per), b1 = min(n, b0 + per);
+    // keys above the threshold key `prefix`, and the first `remaining` equal
+    // to it.  Warp w owns one contiguous segment of the keys and walks it 32
+    // keys at a time (lane = key): counts first, then positions from ballots.
+    const int warp = tid >> 5;
+    constexpr int kWarps = kSelectThreads / 32;
+    const int seg = (n + kWarps - 1) / kWarps;
+    const int w0 = min(n, warp * seg), w1 = min(n, w0 + seg);
     uint32_t gt = 0, eq = 0;
-    for (int i = b0; i < b1; ++i) {
-        const uint32_t k = order_key(sc[i]);
-        gt += k > prefix;
-        eq += k == prefix;
+    for (int i0 = w0; i0 < w1; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t k = i < w1 ? key_at(i) : 0u;
+        gt += __popc(__ballot_sync(0xFFFFFFFFu, i < w1 && k > prefix));
+        eq += __popc(__ballot_sync(0xFFFFFFFFu, i < w1 && k == prefix));
     }
-    const uint32_t eq_before = block_excl_scan(eq, warp_tot);
-    const uint32_t take = eq_before >= remaining ? 0u : min(eq, remaining - eq_before);
-    uint32_t pos = block_excl_scan(gt + take, warp_tot);
-    uint32_t taken = 0;
-    for (int i = b0; i < b1; ++i) {
-        const uint32_t k = order_key(sc[i]);
-        if (k > prefix || (k == prefix && taken < take)) {
-            out[pos++] = i;
-            if (k == prefix) ++taken;
+    if (lane == 0) {
+        hist[warp] = gt;
+        hist[kWarps + warp] = eq;
+    }
+    __syncthreads();
+    if (tid == 0) {
+        // per warp: the equal keys it takes and its first output position
+        uint32_t eq_before = 0, pos = 0;
+        for (int w = 0; w < kWarps; ++w) {
+            const uint32_t e = hist[kWarps + w];
+            const uint32_t take = eq_before >= remaining ? 0u : min(e, remaining - eq_before);
+            hist[2 * kWarps + w] = take;
+            hist[3 * kWarps + w] = pos;
+            pos += hist[w] + take;
+            eq_before += e;
         }
     }
-}
-
-struct GatherView {
-    const uint8_t *codes[2];  // source K, V codes [H_kv][cap][RB]
-    const float *sm[2];       // source K, V scale/min [H_kv][cap][NG][2]
-    uint8_t *dst_codes[2];    // compact [H_kv][cap_c][RB]
-    float *dst_sm[2];         // compact [H_kv][cap_c][NG][2]
-    int64_t cap_packed;
-    int64_t cap_compact;
-    int32_t row_bytes;
-    int32_t sel_row;
-};
-
-struct GatherArgs {
-    const int32_t *sel;       // [n_views][H_kv][top_k]
-    int32_t top_k;
-    int32_t n_kv_heads;
-    int32_t sm_bytes;         // scale/min bytes per row: (D/64) * 8
-    GatherView views[kSparseMaxViews];
-};
-
-// Grid (view, KV head, block of kGatherRows selections): copy the selected
-// packed rows (K and V codes and scale/min) to consecutive compact rows, 8
-// bytes per thread and access.
-__global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ GatherArgs a) {
-    const GatherView &v = a.views[blockIdx.x];
-    const int hk = blockIdx.y;
-    const int r0 = blockIdx.z * kGatherRows;
-    const int rows = min(kGatherRows, a.top_k - r0);
-    const int32_t *sel = a.sel + ((int64_t)v.sel_row * a.n_kv_heads + hk) * a.top_k + r0;
+    __syncthreads();
+    const bool keep = K <= kSelectIdxMax;  // the selection also stays in shared memory
+    {
+        const uint32_t take = hist[2 * kWarps + warp];
+        uint32_t pos = hist[3 * kWarps + warp], taken = 0;
+        const uint32_t below = (1u << lane) - 1u;
+        for (int i0 = w0; i0 < w1; i0 += 32) {
+            const int i = i0 + lane;
+            const uint32_t k = i < w1 ? key_at(i) : 0u;
+            const uint32_t eqm = __ballot_sync(0xFFFFFFFFu, i < w1 && k == prefix);
+            const bool pick_me = i < w1 && (k > prefix || (k == prefix && taken + __popc(eqm & below) < take));
+            const uint32_t pm = __ballot_sync(0xFFFFFFFFu, pick_me);
+            if (pick_me) {
+                const uint32_t at = pos + __popc(pm & below);
+                if (keep) sidx[at] = i;
+                out[at] = i;
+            }
+            pos += __popc(pm);
+            taken += min((uint32_t)__popc(eqm), take - min(take, taken));
+        }
+    }
+    __syncthreads();  // the CTA's selection writes, before it reads them back
+    // the selected rows, in selection order, 8 bytes per thread and access,
+    // eight loads in flight per thread
     const int wc = v.row_bytes / 8, ws = a.sm_bytes / 8, W = 2 * wc + 2 * ws;
-    for (int i = threadIdx.x; i < rows * W; i += blockDim.x) {
+    auto word = [&](int i, const uint2 *&src, uint2 *&dst) {
         const int r = i / W, w = i - r * W;
-        const int64_t src_row = (int64_t)hk * v.cap_packed + sel[r];
-        const int64_t dst_row = (int64_t)hk * v.cap_compact + r0 + r;
-        const uint2 *src;
-        uint2 *dst;
+        const int64_t src_row = (int64_t)hk * v.cap_packed + (keep ? sidx[r] : out[r]);
+        const int64_t dst_row = (int64_t)hk * v.cap_compact + r;
         if (w < 2 * wc) {
             const int kv = w >= wc, x = w - kv * wc;
             src = reinterpret_cast<const uint2 *>(v.codes[kv] + src_row * v.row_bytes) + x;
@@ -294,7 +335,21 @@ __global__ void __launch_bounds__(256) gather_kernel(const __grid_constant__ Gat
             src = reinterpret_cast<const uint2 *>(reinterpret_cast<const uint8_t *>(v.sm[kv]) + src_row * a.sm_bytes) + x;
             dst = reinterpret_cast<uint2 *>(reinterpret_cast<uint8_t *>(v.dst_sm[kv]) + dst_row * a.sm_bytes) + x;
         }
-        *dst = __ldg(src);
+    };
+    const int total = K * W;
+    for (int i0 = tid; i0 < total; i0 += 8 * kSelectThreads) {
+        const uint2 *src[8];
+        uint2 *dst[8];
+        uint2 val[8];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (i0 + j * kSelectThreads < total) word(i0 + j * kSelectThreads, src[j], dst[j]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (i0 + j * kSelectThreads < total) val[j] = __ldg(src[j]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (i0 + j * kSelectThreads < total) *dst[j] = val[j];
     }
 }
 

@@ -17,12 +17,15 @@ CASE:
                  shape (32 layers x 8 kv heads, 32640 packed 4-bit tokens +
                  a full 128-token window), and kvq_card_unpack of that card
                  into fresh views
-  sparse-layer / sparse-8layers
-                 kvq_sparse_decode_attn (top_k 512 of the 4096 packed tokens per
-                 view and KV head, + the 128-token window) over the layer(s)
-                 of decode-layer / decode-8layers; GB/s counts the bytes the
-                 path must read: all packed K and scale/min (scoring), the
-                 selected V rows and scale/min, the window, q and out
+  decode-long    kvq_decode_attn over one layer of 10 agents with 32768
+                 packed tokens each (+ 128-token window), Llama-3.1-8B shape
+  sparse-layer / sparse-8layers / sparse-long
+                 kvq_sparse_decode_attn over the views of decode-layer,
+                 decode-8layers (top_k 512 of 4096 packed tokens per view and
+                 KV head) and decode-long (top_k 2048 of 32768), + the window;
+                 GB/s counts the bytes the path must read: all packed K codes
+                 and scale/min (scoring), the selected rows' V codes and
+                 scale/min, the window, q and out
   card-pack-decode
                  kvq_card_pack of every view of the batched decode workload
                  (10 agents x 32 layers, 4096 packed + 128 window)
@@ -70,7 +73,7 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["decode-layer", "decode-8layers", "quantize", "dequantize", "quantize-handoff",
                                          "dequantize-handoff", "card-pack", "card-unpack", "card-pack-decode", "sparse-layer",
-                                         "sparse-8layers"])
+                                         "sparse-8layers", "decode-long", "sparse-long"])
     ap.add_argument("--reps", type=int, default=20)
     a = ap.parse_args(argv)
     dev = torch.device("cuda:0")
@@ -90,8 +93,9 @@ def main(argv=None):
         else:
             t = _time(lambda: card_pack(pool.views, out=card, stream=torch.cuda.current_stream()), a.reps)
     elif a.case.startswith("sparse"):
-        w = wl.decode_llama8b(n_layers=1 if a.case == "sparse-layer" else 8)
-        top_k = 512
+        long = a.case == "sparse-long"
+        w = wl.decode_llama8b(n_layers=8 if a.case == "sparse-8layers" else 1, length=32768 if long else 4096)
+        top_k = 2048 if long else 512
         pool = kcache.build_decode(w, dev)
         q = kcache.decode_queries(w, device=dev)
         ws = torch.zeros(sparse_workspace_size(pool.views, w.n_q_heads, top_k), dtype=torch.uint8, device=dev)
@@ -103,7 +107,8 @@ def main(argv=None):
         nbytes = w.n_views * (w.n_kv_heads * (n_p * (rb + ng * 8) + top_k * (rb + ng * 8) + w.window * 4 * w.head_dim)
                               + w.n_q_heads * w.head_dim * 6)
     elif a.case.startswith("decode"):
-        w = wl.decode_llama8b(n_layers=1 if a.case == "decode-layer" else 8)
+        w = wl.decode_llama8b(n_layers=8 if a.case == "decode-8layers" else 1,
+                              length=32768 if a.case == "decode-long" else 4096)
         pool = kcache.build_decode(w, dev)
         q = kcache.decode_queries(w, device=dev)
         ws = new_workspace(pool.views, w.n_q_heads, device=dev)

@@ -86,7 +86,10 @@ def test_sparse_llama_shape_small(cuda_device):
     check(case, scale, k, "llama")
 
 
-@pytest.mark.parametrize("bits,D,hq,hkv", [(2, 64, 2, 2), (3, 128, 8, 2), (8, 256, 16, 8), (4, 64, 64, 8)])
+# groups of up to 8 query heads score on the attention grid's tensor-core QK
+# path, wider ones (32 / 2) on the SIMT score kernel
+@pytest.mark.parametrize("bits,D,hq,hkv", [(2, 64, 2, 2), (3, 128, 8, 2), (8, 256, 16, 8), (4, 64, 64, 8),
+                                           (4, 128, 32, 2)])
 def test_sparse_widths_shapes_groups(cuda_device, bits, D, hq, hkv):
     specs = [ViewSpec(300, 8, 8, bits, head=3, seed=300 + bits), ViewSpec(129, 0, 0, bits, seed=301 + bits),
              ViewSpec(0, 5, 8, bits, head=6, seed=302 + bits)]
