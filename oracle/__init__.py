@@ -301,6 +301,109 @@ def sparse_decode_attn(q: np.ndarray, bits: int, k_codes, k_sm, v_codes, v_sm, k
     return out, selected
 
 
+def width_sensitivity(q: np.ndarray, k_win: np.ndarray, v_win: np.ndarray, softmax_scale: float) -> float:
+    """Sensitivity S of one view to the width of its next quantized blocks, in
+    fp64: quantizing at b bits is expected to move the attention output by at
+    most about S / (2^b - 1).
+
+    Source: "Coordinated Mixed-Precision KV Cache Quantization ..." (Abstract:
+    sensitivity from a local attention-error bound on recent queries, keys and
+    values, with no calibration data and no trial quantization).  The page
+    prints no formula; this is the first-order bound that the format gives.
+    A group of range R quantized at b bits moves each element by at most
+    s/2 = R / (2 (2^b - 1)).  For KV head hk, over its recent (window) tokens:
+      R_k[g], R_v[g] = the largest group range of K, V in group g;
+      V_max = the largest ||v_t||_2;
+      Delta = scale * max over the group's query heads h of
+              sum_g ||q_h[g]||_1 * R_k[g] / 2          (logit shift * (2^b - 1));
+      E_v = sqrt(sum_g 64 * (R_v[g] / 2)^2)            (value shift * (2^b - 1)).
+    A logit shift of at most delta moves the softmax by at most e^(2 delta) - 1
+    in L1, so the output moves by at most V_max (e^(2 Delta/(2^b-1)) - 1) +
+    E_v / (2^b - 1); to first order that is S / (2^b - 1) with
+    S = 2 V_max Delta + E_v.  The view's S is the largest over its KV heads;
+    0 without recent tokens.
+
+    q: uint16 bf16 [H_q][D]; k_win, v_win: uint16 bf16 [H_kv][n_w][D].
+    Returns (S, Delta, E_v, V_max) with the last three per KV head.
+    """
+    q = _bf16_to_f64(q)
+    k = _bf16_to_f64(k_win)
+    v = _bf16_to_f64(v_win)
+    Hq, D = q.shape
+    Hkv, n_w = k.shape[:2]
+    G, NG = Hq // Hkv, D // GROUP
+    S, deltas, evs, vmaxs = 0.0, [], [], []
+    for hk in range(Hkv):
+        if n_w == 0:
+            deltas.append(0.0); evs.append(0.0); vmaxs.append(0.0)
+            continue
+        kg = k[hk].reshape(n_w, NG, GROUP)
+        vg = v[hk].reshape(n_w, NG, GROUP)
+        rk = (kg.max(axis=2) - kg.min(axis=2)).max(axis=0)
+        rv = (vg.max(axis=2) - vg.min(axis=2)).max(axis=0)
+        vmax = np.sqrt((v[hk] ** 2).sum(axis=1)).max()
+        l1 = np.abs(q[hk * G:(hk + 1) * G].reshape(G, NG, GROUP)).sum(axis=2)
+        delta = softmax_scale * (l1 * rk / 2).sum(axis=1).max()
+        ev = np.sqrt((64 * (rv / 2) ** 2).sum())
+        deltas.append(delta); evs.append(ev); vmaxs.append(vmax)
+        S = max(S, 2 * vmax * delta + ev)
+    return S, deltas, evs, vmaxs
+
+
+WIDTHS = (8, 4, 3, 2)
+
+
+def allocate_widths(sens, capacity, n_kv_heads: int, head_dim: int, budget_bytes: int, units: int = 4096):
+    """Joint width allocation under a shared byte budget.
+
+    Source: "Coordinated Mixed-Precision KV Cache Quantization ..." (Abstract:
+    a shared controller combines the sensitivity scores with the remaining
+    quantizable capacity and byte-level storage costs to minimize total
+    estimated error).  Reading: view v, given width b, stores its capacity_v
+    tokens still to be quantized at 2 * n_kv_heads * (head_dim*b/8 +
+    (head_dim/64)*8) bytes each and contributes sens_v / (2^b - 1) to the
+    total estimated error.  The budget is cut into `units` equal units (a
+    unit is ceil(budget / units) bytes) and each option's cost is rounded up
+    to whole units, so a chosen allocation never exceeds the budget; among
+    allocations within it the total error is minimal (dynamic programming
+    over views and units).  Equal totals keep the earlier choice in the
+    order 8, 4, 3, 2 bits of the earlier view.  Returns (bits per view,
+    total error), or None when even all-2-bit does not fit.
+    """
+    n = len(sens)
+    unit = -(-int(budget_bytes) // units) if budget_bytes > 0 else 1
+    cap_units = int(budget_bytes) // unit
+    INF = float("inf")
+    best = np.full(cap_units + 1, INF)        # best[u]: least error of the views so far using exactly u units
+    best[0] = 0.0
+    choice = np.zeros((n, cap_units + 1), np.int8)
+    for i in range(n):
+        new = np.full(cap_units + 1, INF)
+        pick = np.zeros(cap_units + 1, np.int8)
+        for j, b in enumerate(WIDTHS):
+            cost = -(-(int(capacity[i]) * 2 * n_kv_heads * (head_dim * b // 8 + head_dim // 64 * 8)) // unit)
+            err = float(sens[i]) / (2 ** b - 1)
+            for u in range(cost, cap_units + 1):
+                cand = best[u - cost] + err
+                if cand < new[u]:
+                    new[u] = cand
+                    pick[u] = j
+        best = new
+        choice[i] = pick
+    # the least total error over every budget use; the smallest such use
+    u = int(np.argmin(best))
+    if best[u] == INF:
+        return None
+    total = float(best[u])
+    bits = [0] * n
+    for i in range(n - 1, -1, -1):
+        j = int(choice[i][u])
+        bits[i] = WIDTHS[j]
+        cost = -(-(int(capacity[i]) * 2 * n_kv_heads * (head_dim * WIDTHS[j] // 8 + head_dim // 64 * 8)) // unit)
+        u -= cost
+    return bits, total
+
+
 class WindowModel:
     """Bookkeeping model of one view's token placement under appends.
 

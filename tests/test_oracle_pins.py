@@ -556,6 +556,91 @@ def test_sparse_score_takes_the_group_maximum_and_ties_go_low():
     assert list(run_sparse(view, 1.0, 5)[1][0]) == [0, 3, 5, 7, 8]
 
 
+# ------------------------------------------------ width allocation ---
+
+@pytest.mark.parametrize("bits", [2, 3, 4, 8])
+def test_sensitivity_bounds_the_error_of_quantizing_recent_tokens(bits):
+    # quantize a view's recent K and V at `bits` (oracle quantizer) and attend
+    # with the same q: the output moves by no more than the bound the
+    # sensitivity is built from, V_max (e^(2 Delta/(2^b-1)) - 1) + E_v/(2^b-1)
+    for seed in range(3):
+        g = wl.generator(80 + seed)
+        Hq, Hkv, D, n = 8, 2, 128, 48
+        mask = wl.outlier_mask(g, Hkv, D, 0.02)
+        k, v = wl.kv_pair(g, Hkv, n, D, mask)
+        q = wl.bf16_bits(wl.normal_bf16(g, (Hq, D)))
+        kb, vb = wl.bf16_bits(k), wl.bf16_bits(v)
+        scale = 1 / np.sqrt(D)
+        S, deltas, evs, vmaxs = oracle.width_sensitivity(q, kb, vb, scale)
+        exact = oracle.decode_attn(q, bits, None, None, None, None, kb, vb, scale)
+        kc, ks = oracle.quantize(kb, bits)
+        vc, vs = oracle.quantize(vb, bits)
+        quant = oracle.decode_attn(q, bits, kc, ks, vc, vs, None, None, scale)
+        m = 2 ** bits - 1
+        for h in range(Hq):
+            hk = h // (Hq // Hkv)
+            err = np.sqrt(((exact[h] - quant[h]) ** 2).sum())
+            bound = vmaxs[hk] * np.expm1(2 * deltas[hk] / m) + evs[hk] / m
+            assert err <= bound * (1 + 1e-6) + 1e-9, (bits, seed, h, err, bound)
+            assert err > 0
+        assert S == max(2 * vm * d + e for vm, d, e in zip(vmaxs, deltas, evs))
+
+
+def test_sensitivity_of_a_constant_window_is_zero():
+    # every group constant: ranges 0, nothing to lose at any width
+    k = np.full((2, 5, 64), 0x3F80, np.uint16)
+    v = np.full((2, 5, 64), 0xC000, np.uint16)
+    q = wl.bf16_bits(wl.normal_bf16(wl.generator(5), (4, 64)))
+    assert oracle.width_sensitivity(q, k, v, 0.125)[0] == 0.0
+    assert oracle.width_sensitivity(q, k[:, :0], v[:, :0], 0.125)[0] == 0.0
+
+
+def brute_force_allocation(sens, cap, H, D, budget, units):
+    import itertools
+    unit = -(-budget // units)
+    best = None
+    for combo in itertools.product(oracle.WIDTHS, repeat=len(sens)):
+        used = sum(-(-(c * 2 * H * (D * b // 8 + D // 64 * 8)) // unit) for c, b in zip(cap, combo))
+        if used > budget // unit:
+            continue
+        err = sum(s / (2 ** b - 1) for s, b in zip(sens, combo))
+        if best is None or err < best[1] - 1e-12:
+            best = (list(combo), err)
+    return best
+
+
+@pytest.mark.parametrize("seed", range(6))
+def test_allocation_matches_brute_force(seed):
+    rng = np.random.default_rng(seed)
+    n = int(rng.integers(1, 6))
+    sens = rng.exponential(1.0, n)
+    cap = rng.integers(100, 5000, n)
+    H, D = 2, 128
+    lo = sum(c * 2 * H * (D * 2 // 8 + D // 64 * 8) for c in cap)
+    hi = sum(c * 2 * H * (D * 8 // 8 + D // 64 * 8) for c in cap)
+    for budget in (int(lo * 1.02), int((lo + hi) / 2), int(hi * 0.9), hi + 1000):
+        got = oracle.allocate_widths(sens, cap, H, D, budget, units=256)
+        want = brute_force_allocation(sens, cap, H, D, budget, 256)
+        assert got is not None and want is not None
+        assert abs(got[1] - want[1]) <= 1e-12 * max(1.0, want[1]), (seed, budget, got, want)
+
+
+def test_allocation_extremes():
+    sens, cap, H, D = [3.0, 1.0, 0.5], [1000, 2000, 500], 8, 128
+    per = lambda b: 2 * H * (D * b // 8 + D // 64 * 8)
+    everything = sum(c * per(8) for c in cap)
+    assert oracle.allocate_widths(sens, cap, H, D, everything * 2)[0] == [8, 8, 8]
+    floor = sum(c * per(2) for c in cap)
+    assert oracle.allocate_widths(sens, cap, H, D, floor - 1) is None
+    # more budget never gives a larger total error
+    errs = [oracle.allocate_widths(sens, cap, H, D, int(floor * f))[1] for f in (1.05, 1.5, 2.0, 3.0, 4.0)]
+    assert all(a >= b for a, b in zip(errs, errs[1:]))
+    # the most sensitive view is never given fewer bits than a less sensitive
+    # one of the same size
+    bits, _ = oracle.allocate_widths([5.0, 1.0], [1000, 1000], H, D, int(1000 * (per(8) + per(2)) * 1.01))
+    assert bits[0] >= bits[1]
+
+
 # --------------------------------------------------------- window model ---
 
 @pytest.mark.parametrize("W", [0, 1, 4, 7])
