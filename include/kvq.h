@@ -296,6 +296,54 @@ kvq_status kvq_sparse_decode_attn(const kvq_view *views, int32_t n_views, int32_
                                   void *stream);
 
 /*
+ * Width allocation across agents and layers under a shared byte budget
+ * ("Coordinated Mixed-Precision KV Cache Quantization for Efficient LLM-based
+ * Multi-agent Systems", Abstract: sensitivity from a local attention-error
+ * bound on recent queries, keys and values; a shared controller minimizing
+ * the total estimated error under byte-level storage costs; the widths apply
+ * to newly quantized blocks only).  The page prints no formula; the bound
+ * below is the first-order one the group-wise affine format gives.
+ *
+ * kvq_width_sensitivity -- per view, S such that quantizing its blocks at b
+ * bits is expected to move the attention output by at most about
+ * S / (2^b - 1).  Over the view's window tokens and per KV head: R_k[g],
+ * R_v[g] the largest K, V range of 64-element group g, V_max the largest
+ * value norm; Delta = softmax_scale * max over the head's query heads h of
+ * sum_g |q_h[g]|_1 * R_k[g] / 2; E_v = sqrt(sum_g 64 * (R_v[g] / 2)^2);
+ * S = 2 * V_max * Delta + E_v, the largest over KV heads (0 without window
+ * tokens).  fp32.
+ *  views      HOST array; only the window part is read.
+ *  q          bf16 [n_views][n_q_heads][head_dim] device array, 16-B aligned
+ *             (the most recent query of each view).
+ *  sens       float [n_views] device array (written).
+ * Errors: as kvq_decode_attn's argument checks; nothing is enqueued on error.
+ */
+kvq_status kvq_width_sensitivity(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
+                                 int32_t n_kv_heads, int32_t head_dim, const void *q,
+                                 float softmax_scale, float *sens, void *stream);
+
+/*
+ * kvq_allocate_widths -- host only.  Chooses bits[i] in {2, 3, 4, 8} for each
+ * view to minimize sum_i sens[i] / (2^bits[i] - 1) subject to
+ * sum_i cost_i(bits[i]) <= budget_bytes, where cost_i(b) = capacity[i] *
+ * 2 * n_kv_heads * (head_dim*b/8 + (head_dim/64)*8) bytes, the storage of the
+ * capacity[i] tokens the view has still to quantize.  The budget is cut into
+ * `units` units of ceil(budget_bytes / units) bytes and costs are rounded up
+ * to whole units, so the result never exceeds the budget; over those
+ * allocations the total is minimal (dynamic programming, O(n_views * units)).
+ * Equal totals keep the wider width of the earlier view.
+ *  sens       HOST float [n_views], >= 0 and finite.
+ *  capacity   HOST int64 [n_views], >= 0.
+ *  bits       HOST int32 [n_views] (written).
+ *  total_error  NULL or HOST double (written): the minimal total.
+ * Errors: KVQ_ERR_CAPACITY if even 2 bits everywhere does not fit;
+ * KVQ_ERR_INVALID_ARG for bad arguments (units outside [1, 2^20]).
+ */
+kvq_status kvq_allocate_widths(const float *sens, const int64_t *capacity, int32_t n_views,
+                               int32_t n_kv_heads, int32_t head_dim, uint64_t budget_bytes,
+                               int32_t units, int32_t *bits, double *total_error);
+
+/*
  * kvq_append_decode_attn -- one decode step over a batch of views: the
  * effect of kvq_append(views, ..., k_new, v_new) followed by
  * kvq_decode_attn(views, ...) on the appended views, in one call (CoMixKV,

@@ -17,6 +17,10 @@ Entry points (same names as the C ABI, without the ``kvq_`` prefix):
                                    (segments) of any widths; View.new_segment
                                    starts a segment at a new width
   append_decode_attn            -- one decode step: append, then attend, in one call
+  width_sensitivity, allocate_widths
+                                -- per-view sensitivity to the width from the
+                                   recent window and query; exact width choice
+                                   under a shared byte budget
   card_pack, card_unpack, ...   -- CacheCard: several views' caches as one
                                    artifact (transfer, save_card / load_card)
   decode_attn_noalloc           -- the same without a workspace: scratch is a
@@ -36,7 +40,7 @@ from . import workloads  # noqa: F401  (seeded input generators)
 __all__ = ["quantize", "dequantize", "View", "append", "decode_attn", "workspace_size",
            "append_decode_attn", "step_workspace_size", "decode_attn_noalloc", "decode_attn_seq",
            "seq_workspace_size", "new_seq_workspace", "MAX_SEGMENTS", "sparse_decode_attn",
-           "sparse_workspace_size",
+           "sparse_workspace_size", "width_sensitivity", "allocate_widths",
            "card_bytes", "card_pack", "card_info", "card_unpack", "views_for_card", "save_card", "load_card", "NOALLOC_SCRATCH_BYTES", "KvqError", "lib", "row_bytes", "GROUP"]
 
 GROUP = 64
@@ -98,6 +102,10 @@ def lib():
         L.kvq_sparse_decode_attn.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, f32, i32, P, P, P, sz,
                                              P]
         L.kvq_sparse_decode_attn.restype = i32
+        L.kvq_width_sensitivity.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, f32, P, P]
+        L.kvq_width_sensitivity.restype = i32
+        L.kvq_allocate_widths.argtypes = [P, P, i32, i32, i32, ctypes.c_uint64, i32, P, P]
+        L.kvq_allocate_widths.restype = i32
         L.kvq_append_decode_attn.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, P, P, f32, P, P, sz, P]
         L.kvq_append_decode_attn.restype = i32
         u64 = ctypes.c_uint64
@@ -378,6 +386,30 @@ def sparse_decode_attn(views, q: torch.Tensor, softmax_scale: float, top_k: int,
                                         _ptr(selected) if selected is not None else None, _ptr(workspace),
                                         workspace.numel(), _stream(stream)), "kvq_sparse_decode_attn")
     return out, selected
+
+
+def width_sensitivity(views, q: torch.Tensor, softmax_scale: float, out: torch.Tensor | None = None,
+                      stream=None) -> torch.Tensor:
+    """kvq_width_sensitivity: q bf16 [n_views, H_q, D] -> fp32 [n_views] (device)."""
+    views = list(views)
+    n, Hq, D = q.shape
+    if out is None:
+        out = torch.empty(n, dtype=torch.float32, device=q.device)
+    _check(lib().kvq_width_sensitivity(_view_array(views), len(views), Hq, views[0].n_kv_heads, D, _ptr(q),
+                                       float(softmax_scale), _ptr(out), _stream(stream)), "kvq_width_sensitivity")
+    return out
+
+
+def allocate_widths(sens, capacity, n_kv_heads: int, head_dim: int, budget_bytes: int, units: int = 4096):
+    """kvq_allocate_widths (host): returns (bits list, total estimated error)."""
+    import numpy as np
+    s = np.ascontiguousarray(np.asarray(sens, dtype=np.float32))
+    c = np.ascontiguousarray(np.asarray(capacity, dtype=np.int64))
+    bits = np.zeros(len(s), dtype=np.int32)
+    total = ctypes.c_double()
+    _check(lib().kvq_allocate_widths(s.ctypes.data, c.ctypes.data, len(s), n_kv_heads, head_dim, int(budget_bytes),
+                                     int(units), bits.ctypes.data, ctypes.byref(total)), "kvq_allocate_widths")
+    return [int(b) for b in bits], total.value
 
 
 def _advanced(c: CView) -> CView:

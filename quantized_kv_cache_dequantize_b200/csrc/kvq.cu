@@ -4,6 +4,8 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cmath>
+#include <limits>
 #include <cstdint>
 #include <cstdlib>
 #include <cstring>
@@ -11,6 +13,7 @@
 #include <vector>
 
 #include "kvq.h"
+#include "kvq_alloc.cuh"
 #include "kvq_attn.cuh"
 #include "kvq_card.cuh"
 #include "kvq_codec.cuh"
@@ -1232,6 +1235,97 @@ KVQ_API kvq_status kvq_sparse_decode_attn(const kvq_view *views, int32_t n_views
     int32_t *sel = selected ? selected : reinterpret_cast<int32_t *>(ws + sp.sel_off);
     return launch_sparse(sp, views, n_views, n_q_heads, n_kv_heads, head_dim, q, softmax_scale, top_k, out, sel, ws,
                          static_cast<cudaStream_t>(stream));
+}
+
+KVQ_API kvq_status kvq_width_sensitivity(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
+                                         int32_t n_kv_heads, int32_t head_dim, const void *q, float softmax_scale,
+                                         float *sens, void *stream) {
+    if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
+    if (n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads || n_kv_heads > 65535)
+        return KVQ_ERR_INVALID_ARG;
+    const kvq_status vs = validate_views(views, n_views, false);
+    if (vs != KVQ_OK) return vs;
+    if (!q || !sens || !aligned(q, 16) || !aligned(sens, 4)) return KVQ_ERR_INVALID_ARG;
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    for (int v0 = 0; v0 < n_views; v0 += kvq::kSensMaxViews) {
+        const int v1 = std::min<int>(n_views, v0 + kvq::kSensMaxViews);
+        kvq::SensArgs a;
+        std::memset(&a, 0, sizeof a);
+        a.q = static_cast<const uint16_t *>(q);
+        a.sens = sens;
+        a.scale = softmax_scale;
+        a.n_q_heads = n_q_heads;
+        a.n_kv_heads = n_kv_heads;
+        a.group = n_q_heads / n_kv_heads;
+        for (int i = v0; i < v1; ++i) {
+            kvq::SensView &d = a.views[i - v0];
+            d.k_window = static_cast<const uint16_t *>(views[i].k_window);
+            d.v_window = static_cast<const uint16_t *>(views[i].v_window);
+            d.cap_window = views[i].cap_window;
+            d.n_window = views[i].n_window;
+            d.window_head = views[i].window_head;
+            d.row = i;
+        }
+        const unsigned grid = (unsigned)(v1 - v0);
+        switch (head_dim / 64) {
+            case 1: kvq::sensitivity_kernel<1><<<grid, 32 * kvq::kSensWarps, 0, st>>>(a); break;
+            case 2: kvq::sensitivity_kernel<2><<<grid, 32 * kvq::kSensWarps, 0, st>>>(a); break;
+            case 3: kvq::sensitivity_kernel<3><<<grid, 32 * kvq::kSensWarps, 0, st>>>(a); break;
+            default: kvq::sensitivity_kernel<4><<<grid, 32 * kvq::kSensWarps, 0, st>>>(a); break;
+        }
+        if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+    }
+    return KVQ_OK;
+}
+
+KVQ_API kvq_status kvq_allocate_widths(const float *sens, const int64_t *capacity, int32_t n_views, int32_t n_kv_heads,
+                                       int32_t head_dim, uint64_t budget_bytes, int32_t units, int32_t *bits,
+                                       double *total_error) {
+    if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
+    if (!sens || !capacity || !bits || n_views <= 0 || n_kv_heads <= 0 || n_kv_heads > 65535) return KVQ_ERR_INVALID_ARG;
+    if (units < 1 || units > (1 << 20)) return KVQ_ERR_INVALID_ARG;
+    static const int kWidths[4] = {8, 4, 3, 2};  // equal totals keep the earlier (wider) choice
+    for (int i = 0; i < n_views; ++i)
+        if (capacity[i] < 0 || capacity[i] > ((int64_t)1 << 40) || !(sens[i] >= 0.f) || std::isinf(sens[i]))
+            return KVQ_ERR_INVALID_ARG;
+    const uint64_t unit = budget_bytes > 0 ? (budget_bytes + (uint64_t)units - 1) / (uint64_t)units : 1;
+    const size_t cap_units = (size_t)(budget_bytes / unit);
+    const double inf = std::numeric_limits<double>::infinity();
+    std::vector<double> best(cap_units + 1, inf), next(cap_units + 1);
+    std::vector<int8_t> choice((size_t)n_views * (cap_units + 1), 0);
+    std::vector<uint64_t> cost((size_t)n_views * 4);
+    best[0] = 0.0;
+    for (int i = 0; i < n_views; ++i) {
+        std::fill(next.begin(), next.end(), inf);
+        int8_t *pick = choice.data() + (size_t)i * (cap_units + 1);
+        for (int j = 0; j < 4; ++j) {
+            const int b = kWidths[j];
+            const uint64_t bytes = (uint64_t)capacity[i] * 2u * (uint64_t)n_kv_heads *
+                                   (uint64_t)(head_dim * b / 8 + head_dim / 64 * 8);
+            const uint64_t c = (bytes + unit - 1) / unit;
+            cost[(size_t)i * 4 + j] = c;
+            const double err = (double)sens[i] / (double)((1 << b) - 1);
+            for (size_t u = (size_t)std::min<uint64_t>(c, cap_units + 1); u <= cap_units; ++u) {
+                const double cand = best[u - c] + err;
+                if (cand < next[u]) {
+                    next[u] = cand;
+                    pick[u] = (int8_t)j;
+                }
+            }
+        }
+        best.swap(next);
+    }
+    size_t u = 0;
+    for (size_t k = 1; k <= cap_units; ++k)
+        if (best[k] < best[u]) u = k;
+    if (best[u] == inf) return KVQ_ERR_CAPACITY;
+    if (total_error) *total_error = best[u];
+    for (int i = n_views - 1; i >= 0; --i) {
+        const int j = choice[(size_t)i * (cap_units + 1) + u];
+        bits[i] = kWidths[j];
+        u -= (size_t)cost[(size_t)i * 4 + j];
+    }
+    return KVQ_OK;
 }
 
 KVQ_API size_t kvq_card_bytes(const kvq_view *views, int32_t n_views, int32_t n_kv_heads, int32_t head_dim) {
