@@ -15,7 +15,7 @@ from test_append import setup_views
 pytestmark = pytest.mark.gpu
 
 H, D, HQ = 4, 128, 8
-CONFIGS = [(4, 8, 300, 8, 3, 400), (2, 8, 0, 5, 5, 64), (3, 0, 77, 0, 0, 96), (8, 16, 33, 16, 15, 64),
+VIEW_CASES = [(4, 8, 300, 8, 3, 400), (2, 8, 0, 5, 5, 64), (3, 0, 77, 0, 0, 96), (8, 16, 33, 16, 15, 64),
            (4, 1, 1, 1, 0, 40)]
 
 
@@ -47,7 +47,7 @@ def section(card, rec, k, H, D):
 
 
 def test_card_matches_oracle_and_restores_exactly(cuda_device, tmp_path):
-    views, models, tk, tv = setup_views(CONFIGS, H, D, cuda_device)
+    views, models, tk, tv = setup_views(VIEW_CASES, H, D, cuda_device)
     advance(views, models, tk, tv, 11, seed=515)
     positions = [3, 0, 1000, 7, -1]
     card = kvq.card_pack(views, model_id=0x5151, position_offsets=positions)
@@ -106,7 +106,7 @@ def test_card_matches_oracle_and_restores_exactly(cuda_device, tmp_path):
 
 
 def test_card_unpack_rejects_mismatched_views(cuda_device):
-    views, _, _, _ = setup_views(CONFIGS[:2], H, D, cuda_device)
+    views, _, _, _ = setup_views(VIEW_CASES[:2], H, D, cuda_device)
     host = kvq.card_pack(views).cpu()
     wrong = [kvq.View(H, D, 3, 400, 8, device=cuda_device), kvq.View(H, D, 2, 64, 8, device=cuda_device)]
     with pytest.raises(kvq.KvqError) as e:

@@ -64,3 +64,80 @@ def test_pins_catch_mutation(name, tmp_path):
             except (AssertionError, ValueError):
                 caught.append(fn.__name__)
     assert caught, f"no pin caught: {name}"
+
+
+# ---- the oracle's numpy functions (sequences, top-K, width allocation):
+# each case rewrites one line of one function's source, runs the mutant in
+# the oracle module's namespace, and checks that a pin fails against it
+
+import inspect
+
+PY_MUTATIONS = {
+    "segments: window rows dropped": (
+        "decode_attn_segments", "            ks.append(_bf16_to_f64(kw))\n            vs.append(_bf16_to_f64(seg[\"v_win\"]))",
+        "            pass"),
+    "segments: values taken from the key codes": (
+        "decode_attn_segments", "vs.append(affine(seg[\"v_codes\"], seg[\"v_sm\"], D, seg[\"bits\"]))",
+        "vs.append(affine(kc, seg[\"k_sm\"], D, seg[\"bits\"]))"),
+    "segments: only the first segment attended": (
+        "decode_attn_segments", "    for seg in segments:", "    for seg in segments[:1]:"),
+    "top-K: score from the group's first query head only": (
+        "sparse_decode_attn", "for h in heads]), axis=0)", "for h in heads][:1]), axis=0)"),
+    "top-K: ties to the higher index": (
+        "sparse_decode_attn", "order = np.argsort(-score, kind=\"stable\")",
+        "order = (n_p - 1 - np.argsort(-score[::-1], kind=\"stable\"))"),
+    "top-K: window left out of the active set": (
+        "sparse_decode_attn", "k = np.concatenate([kp[hk][sel], kw[hk]], axis=0)",
+        "k = np.concatenate([kp[hk][sel], kw[hk][:0]], axis=0)"),
+    "top-K: one token too many": (
+        "sparse_decode_attn", "sel = np.sort(order[:min(top_k, n_p)])", "sel = np.sort(order[:min(top_k + 1, n_p)])"),
+    "sensitivity: value term dropped": (
+        "width_sensitivity", "ev = np.sqrt((64 * (rv / 2) ** 2).sum())", "ev = 0.0"),
+    "sensitivity: key ranges halved twice": (
+        "width_sensitivity", "delta = softmax_scale * (l1 * rk / 2).sum(axis=1).max()",
+        "delta = softmax_scale * (l1 * rk / 4).sum(axis=1).max()"),
+    "sensitivity: group ranges from the first token only": (
+        "width_sensitivity", "rk = (kg.max(axis=2) - kg.min(axis=2)).max(axis=0)",
+        "rk = (kg.max(axis=2) - kg.min(axis=2))[0]"),
+    "allocation: error per width with 2^b instead of 2^b - 1": (
+        "allocate_widths", "err = float(sens[i]) / (2 ** b - 1)", "err = float(sens[i]) / (2 ** b)"),
+    "allocation: costs rounded down": (
+        "allocate_widths", "            cost = -(-(int(capacity[i]) * 2 * n_kv_heads * (head_dim * b // 8 + head_dim // 64 * 8)) // unit)",
+        "            cost = (int(capacity[i]) * 2 * n_kv_heads * (head_dim * b // 8 + head_dim // 64 * 8)) // unit"),
+    "allocation: scale/min bytes left out of the cost": (
+        "allocate_widths", "            cost = -(-(int(capacity[i]) * 2 * n_kv_heads * (head_dim * b // 8 + head_dim // 64 * 8)) // unit)",
+        "            cost = -(-(int(capacity[i]) * 2 * n_kv_heads * (head_dim * b // 8)) // unit)"),
+}
+
+PY_CHECKS = {
+    "decode_attn_segments": [(pins.test_one_segment_is_the_view_attention, {}),
+                             (pins.test_view_split_into_segments_changes_nothing, dict(cut=17)),
+                             (pins.test_segments_of_different_widths_match_brute_force_and_order, {}),
+                             (pins.test_identical_keys_over_segments_give_mean_of_all_values, {})],
+    "sparse_decode_attn": [(pins.test_sparse_with_every_token_selected_is_dense, dict(top_k=45)),
+                           (pins.test_sparse_error_within_discarded_mass_bound, dict(bits=4, top_k=5)),
+                           (pins.test_sparse_selects_a_planted_key_and_attends_it_with_the_window, {}),
+                           (pins.test_sparse_score_takes_the_group_maximum_and_ties_go_low, {})],
+    "width_sensitivity": [(pins.test_sensitivity_bounds_the_error_of_quantizing_recent_tokens, dict(bits=b))
+                          for b in (2, 3, 4, 8)] + [(pins.test_sensitivity_of_a_constant_window_is_zero, {}),
+                                                    (pins.test_sensitivity_closed_form, {})],
+    "allocate_widths": [(pins.test_allocation_matches_brute_force, dict(seed=s)) for s in range(6)] +
+                       [(pins.test_allocation_extremes, {})],
+}
+
+
+@pytest.mark.parametrize("name", sorted(PY_MUTATIONS))
+def test_pins_catch_python_oracle_mutation(name, monkeypatch):
+    fn, old, new = PY_MUTATIONS[name]
+    src = inspect.getsource(getattr(oracle, fn))
+    assert src.count(old) == 1, f"mutation anchor not found: {old}"
+    ns = dict(vars(oracle))
+    exec(compile(src.replace(old, new), f"<mutant {fn}>", "exec"), ns)
+    monkeypatch.setattr(oracle, fn, ns[fn])
+    caught = []
+    for check, kw in PY_CHECKS[fn]:
+        try:
+            check(**kw)
+        except Exception:  # noqa: BLE001  (a failing pin is what we want)
+            caught.append(check.__name__)
+    assert caught, f"no pin caught: {name}"

@@ -586,6 +586,37 @@ def test_sensitivity_bounds_the_error_of_quantizing_recent_tokens(bits):
         assert S == max(2 * vm * d + e for vm, d, e in zip(vmaxs, deltas, evs))
 
 
+def test_sensitivity_closed_form():
+    # one KV head, one query head, head_dim 64, two recent tokens worked by
+    # hand: K ranges 2 (token 1's last channel is 2, the rest 0), q all ones
+    # (|q|_1 = 64), scale 1/8: Delta = 1/8 * 64 * 2/2 = 8.  V: token 1 is
+    # 3 e_0, so R_v = 3, V_max = 3, E_v = sqrt(64 * 1.5^2) = 12.
+    # S = 2 * 3 * 8 + 12 = 60.
+    bf = lambda x: (np.asarray(x, np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    k = np.zeros((1, 2, 64), np.float32)
+    k[0, 1, 63] = 2.0
+    v = np.zeros((1, 2, 64), np.float32)
+    v[0, 1, 0] = 3.0
+    q = np.ones((1, 64), np.float32)
+    S, deltas, evs, vmaxs = oracle.width_sensitivity(bf(q), bf(k), bf(v), 0.125)
+    assert (S, deltas[0], evs[0], vmaxs[0]) == (60.0, 8.0, 12.0, 3.0)
+    # two query heads on the KV head: Delta takes the larger one; a second
+    # group (head_dim 128) adds its own range terms
+    k2 = np.zeros((1, 2, 128), np.float32)
+    k2[0, 1, 63] = 2.0
+    k2[0, 0, 100] = -1.0                      # group 1 range 1
+    v2 = np.zeros((1, 2, 128), np.float32)
+    v2[0, 1, 0] = 3.0
+    v2[0, 0, 127] = 4.0                       # group 1 range 4; ||v_0|| = 4
+    q2 = np.zeros((2, 128), np.float32)
+    q2[0, :64] = 1.0                          # head 0: |q[0]|_1 = 64, |q[1]|_1 = 0
+    q2[1, 64:] = 2.0                          # head 1: |q[1]|_1 = 128
+    S, deltas, evs, vmaxs = oracle.width_sensitivity(bf(q2), bf(k2), bf(v2), 0.125)
+    # Delta = 1/8 * max(64 * 2/2, 128 * 1/2) = 8; E_v = sqrt(64 * (1.5^2 + 2^2)) = 20
+    assert (deltas[0], evs[0], vmaxs[0]) == (8.0, 20.0, 4.0)
+    assert S == 2 * 4.0 * 8.0 + 20.0
+
+
 def test_sensitivity_of_a_constant_window_is_zero():
     # every group constant: ranges 0, nothing to lose at any width
     k = np.full((2, 5, 64), 0x3F80, np.uint16)
