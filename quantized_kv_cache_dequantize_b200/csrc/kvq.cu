@@ -783,13 +783,16 @@ kvq_status noalloc_scratch(void **out) {
     return KVQ_OK;
 }
 
+// The attention (or score) grids of a plan, for the view's head_dim; dep and
+// scores/score_off as launch_attn_ng.
 kvq_status launch_attn(const AttnPlan &plan, const kvq_view *views, int32_t n_q_heads, int32_t n_kv_heads,
-                       int32_t head_dim, const void *q, float scale, float *out, uint8_t *ws, cudaStream_t st) {
+                       int32_t head_dim, const void *q, float scale, float *out, uint8_t *ws, cudaStream_t st,
+                       const int32_t *dep = nullptr, float *scores = nullptr, const int64_t *score_off = nullptr) {
     switch (head_dim / 64) {
-        case 1: return launch_attn_ng<1>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st);
-        case 2: return launch_attn_ng<2>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st);
-        case 3: return launch_attn_ng<3>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st);
-        default: return launch_attn_ng<4>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st);
+        case 1: return launch_attn_ng<1>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off);
+        case 2: return launch_attn_ng<2>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off);
+        case 3: return launch_attn_ng<3>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off);
+        default: return launch_attn_ng<4>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off);
     }
 }
 
@@ -963,13 +966,8 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
         const kvq_status ps =
             plan_attn(packed.data(), n_views, seq.data(), n_views, n_q_heads, n_kv_heads, head_dim, splan, true);
         if (ps != KVQ_OK) return ps;
-        kvq_status es;
-        switch (ng) {
-            case 1: es = launch_attn_ng<1>(splan, packed.data(), n_q_heads, n_kv_heads, q, scale, nullptr, ws, st, nullptr, scores, sp.score_off.data()); break;
-            case 2: es = launch_attn_ng<2>(splan, packed.data(), n_q_heads, n_kv_heads, q, scale, nullptr, ws, st, nullptr, scores, sp.score_off.data()); break;
-            case 3: es = launch_attn_ng<3>(splan, packed.data(), n_q_heads, n_kv_heads, q, scale, nullptr, ws, st, nullptr, scores, sp.score_off.data()); break;
-            default: es = launch_attn_ng<4>(splan, packed.data(), n_q_heads, n_kv_heads, q, scale, nullptr, ws, st, nullptr, scores, sp.score_off.data()); break;
-        }
+        const kvq_status es = launch_attn(splan, packed.data(), n_q_heads, n_kv_heads, head_dim, q, scale, nullptr,
+                                          ws, st, nullptr, scores, sp.score_off.data());
         if (es != KVQ_OK) return es;
         scored.clear();  // nothing left for the SIMT kernel
     }
@@ -1124,12 +1122,7 @@ KVQ_API kvq_status kvq_decode_attn(const kvq_view *views, int32_t n_views, int32
     if (workspace_bytes < plan.total) return KVQ_ERR_INVALID_ARG;
     cudaStream_t st = static_cast<cudaStream_t>(stream);
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    switch (head_dim / 64) {
-        case 1: return launch_attn_ng<1>(plan, views, n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st);
-        case 2: return launch_attn_ng<2>(plan, views, n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st);
-        case 3: return launch_attn_ng<3>(plan, views, n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st);
-        default: return launch_attn_ng<4>(plan, views, n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st);
-    }
+    return launch_attn(plan, views, n_q_heads, n_kv_heads, head_dim, q, softmax_scale, out, ws, st);
 }
 
 KVQ_API size_t kvq_decode_attn_seq_workspace_size(const kvq_view *views, int32_t n_views, const int32_t *seq_begin,
@@ -1204,12 +1197,7 @@ KVQ_API kvq_status kvq_append_decode_attn(kvq_view *views, int32_t n_views, int3
     if (ls != KVQ_OK) return ls;
     for (int i = 0; i < n_views; ++i) views[i] = post[i];  // enqueued: advance the counters
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    switch (head_dim / 64) {
-        case 1: return launch_attn_ng<1>(plan, post.data(), n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st, dep.data());
-        case 2: return launch_attn_ng<2>(plan, post.data(), n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st, dep.data());
-        case 3: return launch_attn_ng<3>(plan, post.data(), n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st, dep.data());
-        default: return launch_attn_ng<4>(plan, post.data(), n_q_heads, n_kv_heads, q, softmax_scale, out, ws, st, dep.data());
-    }
+    return launch_attn(plan, post.data(), n_q_heads, n_kv_heads, head_dim, q, softmax_scale, out, ws, st, dep.data());
 }
 
 KVQ_API size_t kvq_sparse_decode_attn_workspace_size(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
