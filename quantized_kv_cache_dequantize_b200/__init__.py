@@ -37,11 +37,12 @@ import torch
 
 from . import workloads  # noqa: F401  (seeded input generators)
 
-__all__ = ["quantize", "dequantize", "View", "append", "decode_attn", "workspace_size",
-           "append_decode_attn", "step_workspace_size", "decode_attn_noalloc", "decode_attn_seq",
-           "seq_workspace_size", "new_seq_workspace", "MAX_SEGMENTS", "sparse_decode_attn",
-           "sparse_workspace_size", "width_sensitivity", "allocate_widths",
-           "card_bytes", "card_pack", "card_info", "card_unpack", "views_for_card", "save_card", "load_card", "NOALLOC_SCRATCH_BYTES", "KvqError", "lib", "row_bytes", "GROUP"]
+__all__ = ["quantize", "dequantize", "View", "append", "decode_attn", "workspace_size", "append_decode_attn",
+           "step_workspace_size", "decode_attn_noalloc", "decode_attn_seq", "seq_workspace_size",
+           "new_seq_workspace", "MAX_SEGMENTS", "sparse_decode_attn", "sparse_workspace_size",
+           "width_sensitivity", "allocate_widths", "card_bytes", "card_pack", "card_info", "card_unpack",
+           "views_for_card", "save_card", "load_card", "NOALLOC_SCRATCH_BYTES", "KvqError", "lib",
+           "row_bytes", "GROUP"]
 
 GROUP = 64
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024   # KVQ_NOALLOC_SCRATCH_BYTES in kvq.h
