@@ -118,3 +118,34 @@ def test_unpack_checks_views_before_launch(L):
     assert r == kvq.KVQ_ERR_CAPACITY and arr[0].n_packed == 0          # packed capacity; view untouched
     r, arr = unpack([cview(4, 0, 64, 0, 4), cview(2, 0, 10, 0, 0)])
     assert r == kvq.KVQ_ERR_CAPACITY                                    # window capacity
+
+
+def test_random_corruption_never_crashes_the_parser(L):
+    # a card read from a file is untrusted input: random bytes in the header
+    # and records, and random truncations, give a status (or a valid reading),
+    # never a read outside the buffer
+    rng = np.random.default_rng(7)
+    good = make_card(4, 128, [(4, 300, 16), (2, 0, 7), (8, 33, 0)], model_id=3, positions=[1, 2, 3])
+    meta = 64 + 64 * 3
+    outcomes = set()
+    for trial in range(3000):
+        card = good.copy()
+        if trial % 3 == 0:
+            card = card[:int(rng.integers(0, len(card)))].copy()
+        for _ in range(int(rng.integers(1, 4))):
+            if len(card) == 0:
+                break
+            i = int(rng.integers(0, min(meta, len(card))))
+            card[i] = rng.integers(0, 256)
+        p = card.ctypes.data_as(ctypes.c_void_p) if len(card) else ctypes.c_void_p(0)
+        n, hk, d, mid = ctypes.c_int32(), ctypes.c_int32(), ctypes.c_int32(), ctypes.c_uint64()
+        st = L.kvq_card_read_header(p, len(card), ctypes.byref(n), ctypes.byref(hk), ctypes.byref(d),
+                                    ctypes.byref(mid))
+        outcomes.add(st)
+        if st == kvq.KVQ_OK:
+            for i in range(n.value):
+                b, w = ctypes.c_int32(), ctypes.c_int32()
+                np_, off = ctypes.c_int64(), ctypes.c_int64()
+                assert L.kvq_card_view_info(p, len(card), i, ctypes.byref(b), ctypes.byref(np_), ctypes.byref(w),
+                                            ctypes.byref(off)) == kvq.KVQ_OK
+    assert kvq.KVQ_ERR_INVALID_ARG in outcomes and kvq.KVQ_OK in outcomes
