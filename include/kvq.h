@@ -337,7 +337,9 @@ kvq_status kvq_width_sensitivity(const kvq_view *views, int32_t n_views, int32_t
  *  bits       HOST int32 [n_views] (written).
  *  total_error  NULL or HOST double (written): the minimal total.
  * Errors: KVQ_ERR_CAPACITY if even 2 bits everywhere does not fit;
- * KVQ_ERR_INVALID_ARG for bad arguments (units outside [1, 2^20]).
+ * KVQ_ERR_INVALID_ARG for bad arguments (units outside [1, 2^20]);
+ * KVQ_ERR_UNSUPPORTED when n_views * (units + 1) exceeds 2^30 (the host
+ * memory of the back-pointers).
  */
 kvq_status kvq_allocate_widths(const float *sens, const int64_t *capacity, int32_t n_views,
                                int32_t n_kv_heads, int32_t head_dim, uint64_t budget_bytes,

@@ -1278,6 +1278,8 @@ KVQ_API kvq_status kvq_allocate_widths(const float *sens, const int64_t *capacit
             return KVQ_ERR_INVALID_ARG;
     const uint64_t unit = budget_bytes > 0 ? (budget_bytes + (uint64_t)units - 1) / (uint64_t)units : 1;
     const size_t cap_units = (size_t)(budget_bytes / unit);
+    // the back-pointers take one byte per (view, unit): at most 1 GiB
+    if ((uint64_t)n_views * (uint64_t)(cap_units + 1) > (1ull << 30)) return KVQ_ERR_UNSUPPORTED;
     const double inf = std::numeric_limits<double>::infinity();
     std::vector<double> best(cap_units + 1, inf), next(cap_units + 1);
     std::vector<int8_t> choice((size_t)n_views * (cap_units + 1), 0);

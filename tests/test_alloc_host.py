@@ -55,3 +55,10 @@ def test_allocation_budget_extremes_and_errors():
     # are rounded up to whole units, so an exact fit needs a little slack)
     bits, _ = kvq.allocate_widths([1.0, 1.0], [0, 1000], H, D, int(1000 * per(2) * 1.01))
     assert bits == [8, 2]
+
+
+def test_allocation_refuses_oversized_tables():
+    n = 2048
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.allocate_widths(np.ones(n, np.float32), np.full(n, 1000), 8, 128, 10 ** 12, units=1 << 20)
+    assert e.value.status == kvq.KVQ_ERR_UNSUPPORTED
