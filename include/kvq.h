@@ -132,7 +132,10 @@ kvq_status kvq_dequantize(const void *codes, const float *scalemin, int64_t in_h
  *                          (may be NULL when cap_window == 0).
  * The sequence a query attends is packed tokens 0..n_packed-1, then window
  * tokens oldest to newest.
+ * Every call takes at most KVQ_MAX_VIEWS views (KVQ_ERR_INVALID_ARG beyond).
  */
+#define KVQ_MAX_VIEWS (1 << 22)
+
 typedef struct kvq_view {
     int32_t bits;
     int32_t n_window;

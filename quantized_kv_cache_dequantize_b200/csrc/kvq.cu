@@ -131,7 +131,7 @@ int env_int(const char *name, int dflt) {
 }
 
 kvq_status validate_views(const kvq_view *views, int32_t n_views, bool need_nonempty) {
-    if (!views || n_views <= 0) return KVQ_ERR_INVALID_ARG;
+    if (!views || n_views <= 0 || n_views > KVQ_MAX_VIEWS) return KVQ_ERR_INVALID_ARG;
     for (int i = 0; i < n_views; ++i) {
         const kvq_view &v = views[i];
         if (v.n_packed < 0 || v.cap_packed < v.n_packed || (v.cap_packed & 1)) return KVQ_ERR_INVALID_ARG;

@@ -205,3 +205,11 @@ def test_fused_step_checks_before_launch(L):
     assert L.kvq_append_decode_attn(ok, 1, 8, 2, 128, FAKE, FAKE, FAKE, 0.1, FAKE, FAKE, 16, NULL) == \
         kvq.KVQ_ERR_INVALID_ARG                                                    # workspace too small
     assert ok[0].n_packed == 4
+
+
+def test_view_count_is_bounded(L):
+    # the bound is checked before the views are read
+    one = (kvq.CView * 1)(cview())
+    assert L.kvq_decode_attn(one, (1 << 22) + 1, 8, 2, 128, FAKE, 0.1, FAKE, FAKE, 1 << 30, NULL) == \
+        kvq.KVQ_ERR_INVALID_ARG
+    assert L.kvq_decode_attn_workspace_size(one, (1 << 22) + 1, 8, 2, 128) == 0
