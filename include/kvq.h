@@ -15,7 +15,15 @@
  *    LLM-based Multi-agent Systems", Abstract: each (agent, layer) has its own
  *    width, recent states keep native precision, and only newly quantized
  *    blocks take a width while older blocks stay as they are (kvq_view.bits,
- *    the bf16 recent window, kvq_append).
+ *    the bf16 recent window, kvq_append); the widths come from a sensitivity
+ *    bound and a budgeted allocation (kvq_width_sensitivity,
+ *    kvq_allocate_widths), and a sequence may span views of several widths
+ *    (kvq_decode_attn_seq).
+ *  - QKVShare, Metodologia: the CacheCard artifact that carries the quantized
+ *    groups and their metadata (kvq_card_*).
+ *  - "Reasoning-Aware Error-Bounded KV-Cache Compression and Sparse Attention
+ *    for Long-Context LLMs", Metodologia C: top-K sparse decode attention
+ *    (kvq_sparse_decode_attn).
  *
  * Quantization format (the pages leave it open; this is the library's
  * definition):
@@ -68,7 +76,8 @@ typedef enum kvq_status {
     KVQ_OK = 0,
     KVQ_ERR_INVALID_ARG = 1, /* null/misaligned pointer, bad size or stride */
     KVQ_ERR_UNSUPPORTED = 2, /* bits not in {2,3,4,8}, head_dim not 64..256 step 64 */
-    KVQ_ERR_CAPACITY = 3,    /* an append would write past cap_packed */
+    KVQ_ERR_CAPACITY = 3,    /* a capacity is exceeded: an append past cap_packed, a card
+                                into smaller views, a scratch or a byte budget too small */
     KVQ_ERR_CUDA = 4         /* a kernel launch or device query failed */
 } kvq_status;
 
