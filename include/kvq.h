@@ -450,6 +450,31 @@ kvq_status kvq_card_unpack(const void *card_host, const void *card, size_t card_
                            kvq_view *views, int32_t n_views, int32_t n_kv_heads,
                            int32_t head_dim, void *stream);
 
+/*
+ * kvq_debug_build -- 1 in the debug build of the library (libkvq_debug.so,
+ * compiled with -DKVQ_DEBUG), 0 in the normal one.  No counterpart in the
+ * pages: a test aid in place of a sanitizer.  In the debug build every kernel
+ * checks the global addresses it computes against the extents of the buffers
+ * they belong to (a view head's packed rows, its window ring, q, out, the
+ * workspace, the card image, the score and selection arrays); a failed check
+ * sets a bit in one device word and the access is skipped, so nothing traps.
+ */
+int32_t kvq_debug_build(void);
+
+/*
+ * kvq_debug_flags -- copy the debug build's flags word of the current device
+ * into `flags` (4-byte aligned; device memory or host memory the copy engine
+ * can reach, pinned for an asynchronous copy), enqueued on `stream`, then
+ * clear the word when `clear` is nonzero.  Stream-ordered: the word holds the
+ * failed checks of the kernels enqueued before this call (bit 0 packed-row
+ * copies, 1 window copies, 2 shared-memory stages, 3 q/out/scores, 4
+ * workspace, 5 codec, 6 append, 7 card, 8 scores, 9 selections, 10
+ * sensitivity).  Errors: KVQ_ERR_UNSUPPORTED in the normal build,
+ * KVQ_ERR_INVALID_ARG for a null or misaligned `flags`, KVQ_ERR_CUDA when
+ * the copy cannot be enqueued.
+ */
+kvq_status kvq_debug_flags(uint32_t *flags, int32_t clear, void *stream);
+
 /* Bytes of the per-device scratch array kvq_decode_attn_noalloc uses. */
 #define KVQ_NOALLOC_SCRATCH_BYTES (32u * 1024u * 1024u)
 
@@ -467,15 +492,18 @@ kvq_status kvq_card_unpack(const void *card_host, const void *card, size_t card_
  * Arguments, layouts and results are those of kvq_decode_attn without
  * workspace / workspace_bytes; the same kernels run on the same plan, so the
  * result is the same.
- * Set-up: the first call on a device (with that device current) looks up the
- * array's device address once; make that first call before any stream
- * capture.
+ * Set-up: every call looks up the array's device address on the current
+ * device (a host-side runtime query, no device work), so a device reset or a
+ * re-created primary context never leaves a stale address in use.  The first
+ * call on a device also loads the library's device code there; make that
+ * first call before any stream capture.
  * Each call clears the array's status word and arrival counters on `stream`
- * before its kernels; the status word is not reported back (kvq_decode_attn
- * exposes it).
+ * before its kernels.  The status word (0, or 1 when a bounded copy wait gave
+ * up and the outputs of that call are not valid) can be read back with
+ * kvq_decode_attn_noalloc_status before the next call clears it.
  * Errors: KVQ_ERR_CAPACITY, with nothing enqueued, when the views need more
  * scratch than KVQ_NOALLOC_SCRATCH_BYTES (kvq_decode_attn_workspace_size
- * gives the need); KVQ_ERR_CUDA if the set-up lookup fails; otherwise as
+ * gives the need); KVQ_ERR_CUDA if the address lookup fails; otherwise as
  * kvq_decode_attn.
  * Concurrency: every call on a device shares the one array, so calls that can
  * overlap on the GPU (different streams, different host threads) race and
@@ -484,6 +512,20 @@ kvq_status kvq_card_unpack(const void *card_host, const void *card, size_t card_
 kvq_status kvq_decode_attn_noalloc(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
                                    int32_t n_kv_heads, int32_t head_dim, const void *q,
                                    float softmax_scale, float *out, void *stream);
+
+/*
+ * kvq_decode_attn_noalloc_status -- copy the status word of the current
+ * device's scratch array into `status` (4-byte aligned; device memory, or
+ * host memory the copy engine can reach: pinned host memory keeps the copy
+ * asynchronous), enqueued on `stream`.  Stream-ordered: it reads the word as
+ * the kvq_decode_attn_noalloc call enqueued before it on that stream left it,
+ * and a later call clears the word again.  0: the outputs are valid; 1: a
+ * bounded copy wait gave up, the outputs of that call are not valid.  Like
+ * kvq_decode_attn_noalloc it allocates nothing; no counterpart in the pages.
+ * Errors: KVQ_ERR_INVALID_ARG for a null or misaligned `status`,
+ * KVQ_ERR_CUDA when the address lookup or the copy cannot be enqueued.
+ */
+kvq_status kvq_decode_attn_noalloc_status(uint32_t *status, void *stream);
 
 #ifdef __cplusplus
 }

@@ -38,17 +38,19 @@ import torch
 from . import workloads  # noqa: F401  (seeded input generators)
 
 __all__ = ["quantize", "dequantize", "View", "append", "decode_attn", "workspace_size", "append_decode_attn",
-           "step_workspace_size", "decode_attn_noalloc", "decode_attn_seq", "seq_workspace_size",
+           "step_workspace_size", "decode_attn_noalloc", "decode_attn_noalloc_status", "decode_attn_seq", "seq_workspace_size",
            "new_seq_workspace", "MAX_SEGMENTS", "sparse_decode_attn", "sparse_workspace_size",
            "width_sensitivity", "allocate_widths", "card_bytes", "card_pack", "card_info", "card_unpack",
-           "views_for_card", "save_card", "load_card", "NOALLOC_SCRATCH_BYTES", "KvqError", "lib",
+           "views_for_card", "save_card", "load_card", "NOALLOC_SCRATCH_BYTES", "KvqError", "lib", "debug_flags",
            "row_bytes", "GROUP"]
 
 GROUP = 64
 NOALLOC_SCRATCH_BYTES = 32 * 1024 * 1024   # KVQ_NOALLOC_SCRATCH_BYTES in kvq.h
 MAX_SEGMENTS = 64                          # KVQ_MAX_SEGMENTS in kvq.h
 _HERE = os.path.dirname(os.path.abspath(__file__))
-_LIB_PATH = os.path.join(_HERE, "libkvq.so")
+# KVQ_DEBUG=1 in the environment selects the debug build (device bounds
+# checks recorded in a flags word, see debug_flags); read once, at first use
+_LIB_PATH = os.path.join(_HERE, "libkvq_debug.so" if os.environ.get("KVQ_DEBUG") == "1" else "libkvq.so")
 _lib = None
 
 KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_CAPACITY, KVQ_ERR_CUDA = range(5)
@@ -122,6 +124,12 @@ def lib():
         L.kvq_card_unpack.restype = i32
         L.kvq_decode_attn_noalloc.argtypes = [ctypes.POINTER(CView), i32, i32, i32, i32, P, f32, P, P]
         L.kvq_decode_attn_noalloc.restype = i32
+        L.kvq_decode_attn_noalloc_status.argtypes = [P, P]
+        L.kvq_decode_attn_noalloc_status.restype = i32
+        L.kvq_debug_build.argtypes = []
+        L.kvq_debug_build.restype = i32
+        L.kvq_debug_flags.argtypes = [P, i32, P]
+        L.kvq_debug_flags.restype = i32
         _lib = L
     return _lib
 
@@ -143,6 +151,77 @@ def _check(status: int, where: str):
 
 def _ptr(t):
     return ctypes.c_void_p(t.data_ptr()) if t is not None else ctypes.c_void_p(0)
+
+
+def _views_device(views):
+    return views[0].k_codes.device
+
+
+def _check_tensor(name, t, dtype, shape, device):
+    """A tensor the C call reads or writes as a dense array: dtype, shape,
+    contiguity and device must match, since the library sees only a pointer."""
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, the views are on {device}")
+
+
+def _require_cuda(dev):
+    """Last of the checks: the views (and so every tensor checked against
+    them) must be in device memory."""
+    if dev.type != "cuda":
+        raise ValueError(f"the views and tensors must be CUDA tensors, not {dev}")
+
+
+def _check_views(views):
+    """The views of one call share n_kv_heads and head_dim (the C ABI takes them once)."""
+    if not views:
+        raise ValueError("at least one view is needed")
+    H, D = views[0].n_kv_heads, views[0].head_dim
+    dev = _views_device(views)
+    for v in views:
+        if v.n_kv_heads != H or v.head_dim != D:
+            raise ValueError("all views of a call must have the same n_kv_heads and head_dim")
+        if v.k_codes.device != dev:
+            raise ValueError("all views of a call must be on one device")
+    return H, D, dev
+
+
+def _check_q(views, q, n_rows):
+    """q: bf16 [n_rows, H_q, D] with H_q a multiple of the views' n_kv_heads."""
+    H, D, dev = _check_views(views)
+    if not isinstance(q, torch.Tensor) or q.dim() != 3:
+        raise ValueError("q must be a 3-d tensor [rows, H_q, D]")
+    Hq = q.shape[1]
+    if Hq <= 0 or Hq % H:
+        raise ValueError(f"q has {Hq} query heads, not a multiple of n_kv_heads {H}")
+    _check_tensor("q", q, torch.bfloat16, (n_rows, Hq, D), dev)
+    return Hq, D, dev
+
+
+def _check_out(out, n_rows, Hq, D, dev):
+    _check_tensor("out", out, torch.float32, (n_rows, Hq, D), dev)
+
+
+def _check_new_tokens(views, k_new, v_new):
+    H, D, dev = _check_views(views)
+    _check_tensor("k_new", k_new, torch.bfloat16, (len(views), H, D), dev)
+    _check_tensor("v_new", v_new, torch.bfloat16, (len(views), H, D), dev)
+
+
+def _check_workspace(ws, dev):
+    if ws is None:
+        return
+    if not isinstance(ws, torch.Tensor) or ws.dtype != torch.uint8 or ws.dim() != 1 or not ws.is_contiguous():
+        raise ValueError("workspace must be a contiguous 1-d uint8 tensor")
+    if ws.device != dev:
+        raise ValueError(f"workspace is on {ws.device}, the views are on {dev}")
 
 
 # -------------------------------------------------------------- codec -----
@@ -286,8 +365,10 @@ def _view_array(views):
 def append(views, k_new: torch.Tensor, v_new: torch.Tensor, stream=None):
     """Append one token per view: k_new, v_new bf16 [n_views, H_kv, D]."""
     views = list(views)
+    _check_new_tokens(views, k_new, v_new)
     arr = _view_array(views)
     H, D = views[0].n_kv_heads, views[0].head_dim
+    _require_cuda(views[0].k_codes.device)
     _check(lib().kvq_append(arr, len(views), H, D, _ptr(k_new), _ptr(v_new), _stream(stream)),
            "kvq_append")
     for i, v in enumerate(views):
@@ -313,12 +394,16 @@ def decode_attn(views, q: torch.Tensor, softmax_scale: float, out: torch.Tensor 
                 workspace: torch.Tensor | None = None, stream=None, _arr=None) -> torch.Tensor:
     """q: bf16 [n_views, H_q, D] -> fp32 [n_views, H_q, D]."""
     views = list(views)
-    n, Hq, D = q.shape
+    Hq, D, dev = _check_q(views, q, len(views))
+    n = len(views)
     arr = _arr if _arr is not None else _view_array(views)
     if workspace is None:
         workspace = new_workspace(views, Hq, device=q.device)
+    _check_workspace(workspace, dev)
     if out is None:
         out = torch.empty((n, Hq, D), dtype=torch.float32, device=q.device)
+    _check_out(out, n, Hq, D, dev)
+    _require_cuda(dev)
     _check(lib().kvq_decode_attn(arr, len(views), Hq, views[0].n_kv_heads, D, _ptr(q), float(softmax_scale),
                                  _ptr(out), _ptr(workspace), workspace.numel(), _stream(stream)),
            "kvq_decode_attn")
@@ -350,12 +435,16 @@ def decode_attn_seq(views, seq_begin, q: torch.Tensor, softmax_scale: float, out
     """kvq_decode_attn_seq: sequence s is views seq_begin[s] .. seq_begin[s+1]-1.
     q: bf16 [n_seqs, H_q, D] -> fp32 [n_seqs, H_q, D]."""
     views = list(views)
-    n, Hq, D = q.shape
     sb, n_seqs = _seq_array(seq_begin)
+    Hq, D, dev = _check_q(views, q, n_seqs)
+    n = n_seqs
     if workspace is None:
         workspace = new_seq_workspace(views, seq_begin, Hq, device=q.device)
+    _check_workspace(workspace, dev)
     if out is None:
         out = torch.empty((n, Hq, D), dtype=torch.float32, device=q.device)
+    _check_out(out, n, Hq, D, dev)
+    _require_cuda(dev)
     _check(lib().kvq_decode_attn_seq(_view_array(views), len(views), sb, n_seqs, Hq, views[0].n_kv_heads, D,
                                      _ptr(q), float(softmax_scale), _ptr(out), _ptr(workspace), workspace.numel(),
                                      _stream(stream)), "kvq_decode_attn_seq")
@@ -374,14 +463,20 @@ def sparse_decode_attn(views, q: torch.Tensor, softmax_scale: float, top_k: int,
     """kvq_sparse_decode_attn.  q: bf16 [n_views, H_q, D]; returns (out fp32
     [n_views, H_q, D], selected int32 [n_views, H_kv, top_k] or None)."""
     views = list(views)
-    n, Hq, D = q.shape
+    Hq, D, dev = _check_q(views, q, len(views))
+    n = len(views)
     if workspace is None:
         nb = sparse_workspace_size(views, Hq, top_k)
         if nb == 0:
             raise KvqError(KVQ_ERR_INVALID_ARG, "kvq_sparse_decode_attn_workspace_size")
         workspace = torch.zeros(nb, dtype=torch.uint8, device=q.device)
+    _check_workspace(workspace, dev)
     if out is None:
         out = torch.empty((n, Hq, D), dtype=torch.float32, device=q.device)
+    _check_out(out, n, Hq, D, dev)
+    if selected is not None:
+        _check_tensor("selected", selected, torch.int32, (n, views[0].n_kv_heads, int(top_k)), dev)
+    _require_cuda(dev)
     _check(lib().kvq_sparse_decode_attn(_view_array(views), len(views), Hq, views[0].n_kv_heads, D, _ptr(q),
                                         float(softmax_scale), int(top_k), _ptr(out),
                                         _ptr(selected) if selected is not None else None, _ptr(workspace),
@@ -393,9 +488,12 @@ def width_sensitivity(views, q: torch.Tensor, softmax_scale: float, out: torch.T
                       stream=None) -> torch.Tensor:
     """kvq_width_sensitivity: q bf16 [n_views, H_q, D] -> fp32 [n_views] (device)."""
     views = list(views)
-    n, Hq, D = q.shape
+    Hq, D, dev = _check_q(views, q, len(views))
+    n = len(views)
     if out is None:
         out = torch.empty(n, dtype=torch.float32, device=q.device)
+    _check_tensor("out", out, torch.float32, (n,), dev)
+    _require_cuda(dev)
     _check(lib().kvq_width_sensitivity(_view_array(views), len(views), Hq, views[0].n_kv_heads, D, _ptr(q),
                                        float(softmax_scale), _ptr(out), _stream(stream)), "kvq_width_sensitivity")
     return out
@@ -445,14 +543,19 @@ def append_decode_attn(views, k_new: torch.Tensor, v_new: torch.Tensor, q: torch
     [n_views, H_kv, D]) to the views, then attend with q (bf16 [n_views, H_q,
     D]) over the appended views; returns fp32 [n_views, H_q, D]."""
     views = list(views)
-    n, Hq, D = q.shape
+    Hq, D, dev = _check_q(views, q, len(views))
+    _check_new_tokens(views, k_new, v_new)
+    n = len(views)
     if workspace is None:
         # 0 when the step is invalid: the call below then reports why
         nb = step_workspace_size(views, Hq)
         workspace = torch.zeros(nb, dtype=torch.uint8, device=q.device) if nb else None
+    _check_workspace(workspace, dev)
     if out is None:
         out = torch.empty((n, Hq, D), dtype=torch.float32, device=q.device)
+    _check_out(out, n, Hq, D, dev)
     arr = _view_array(views)
+    _require_cuda(dev)
     _check(lib().kvq_append_decode_attn(arr, len(views), Hq, views[0].n_kv_heads, D, _ptr(k_new), _ptr(v_new),
                                         _ptr(q), float(softmax_scale), _ptr(out), _ptr(workspace),
                                         workspace.numel() if workspace is not None else 0, _stream(stream)),
@@ -470,11 +573,39 @@ def decode_attn_noalloc(views, q: torch.Tensor, softmax_scale: float, out: torch
     device memory either.  Calls that may overlap on the GPU race on the one
     array; the first call on a device should come before any stream capture."""
     views = list(views)
-    n, Hq, D = q.shape
+    Hq, D, dev = _check_q(views, q, len(views))
+    _check_out(out, len(views), Hq, D, dev)
     arr = _arr if _arr is not None else _view_array(views)
+    _require_cuda(dev)
     _check(lib().kvq_decode_attn_noalloc(arr, len(views), Hq, views[0].n_kv_heads, D, _ptr(q),
                                          float(softmax_scale), _ptr(out), _stream(stream)),
            "kvq_decode_attn_noalloc")
+    return out
+
+
+def debug_flags(clear: bool = True, stream=None) -> int:
+    """The debug build's flags word (0: every device bounds check passed;
+    one bit per kernel family otherwise), read after the work enqueued on
+    ``stream`` so far, and cleared when ``clear``.  Synchronizes the stream.
+    Raises KvqError (KVQ_ERR_UNSUPPORTED) in the normal build."""
+    out = torch.zeros(1, dtype=torch.int32).pin_memory()
+    _check(lib().kvq_debug_flags(_ptr(out), 1 if clear else 0, _stream(stream)), "kvq_debug_flags")
+    (stream if stream is not None else torch.cuda.current_stream()).synchronize()
+    return int(out.item()) & 0xFFFFFFFF
+
+
+def decode_attn_noalloc_status(out: torch.Tensor | None = None, stream=None) -> torch.Tensor:
+    """kvq_decode_attn_noalloc_status: the status word the last
+    decode_attn_noalloc call enqueued on ``stream`` left in the scratch array
+    (0: outputs valid; 1: a bounded copy wait gave up), copied into ``out``
+    (an int32 tensor of one element: device, or pinned host memory; a new
+    pinned host tensor when None).  Stream-ordered: synchronize the stream
+    before reading a host tensor."""
+    if out is None:
+        out = torch.zeros(1, dtype=torch.int32).pin_memory()
+    if out.dtype != torch.int32 or out.numel() != 1 or not out.is_contiguous():
+        raise ValueError("out must be a contiguous int32 tensor of one element")
+    _check(lib().kvq_decode_attn_noalloc_status(_ptr(out), _stream(stream)), "kvq_decode_attn_noalloc_status")
     return out
 
 

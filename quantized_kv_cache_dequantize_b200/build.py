@@ -1,9 +1,13 @@
-"""Build libkvq.so in-tree with nvcc for sm_100a.
+"""Build libkvq.so (and its debug build, libkvq_debug.so) in-tree with nvcc
+for sm_100a.
 
-    python -m quantized_kv_cache_dequantize_b200.build [--verbose]
+    python -m quantized_kv_cache_dequantize_b200.build [--verbose] [--debug-only]
 
-The shared library is written next to this file so that it travels with the
-source tree; it exports only the extern "C" entry points of include/kvq.h.
+The shared libraries are written next to this file so that they travel with
+the source tree; they export only the extern "C" entry points of
+include/kvq.h.  The debug build is compiled with -DKVQ_DEBUG: its kernels
+check every global address they compute and record failures in a flags word
+(kvq_debug_flags) instead of touching memory out of bounds.
 """
 from __future__ import annotations
 
@@ -16,6 +20,7 @@ ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB = os.path.join(HERE, "libkvq.so")
+DEBUG_LIB = os.path.join(HERE, "libkvq_debug.so")
 SOURCES = [os.path.join(CSRC, "kvq.cu")]
 DEPS = SOURCES + [os.path.join(CSRC, f) for f in os.listdir(CSRC) if f.endswith((".cuh", ".h"))] + [
     os.path.join(INCLUDE, "kvq.h")]
@@ -37,24 +42,41 @@ def nvcc() -> str:
     return cand if os.path.exists(cand) else "nvcc"
 
 
-def up_to_date() -> bool:
-    if not os.path.exists(LIB):
+def up_to_date(lib: str = LIB) -> bool:
+    if not os.path.exists(lib):
         return False
-    t = os.path.getmtime(LIB)
+    t = os.path.getmtime(lib)
     return all(os.path.getmtime(p) <= t for p in DEPS)
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and up_to_date():
-        return LIB
-    tmp = LIB + f".tmp{os.getpid()}"
+def _command(lib: str, tmp: str, verbose: bool):
     cmd = [nvcc(), *NVCC_FLAGS, "-I", INCLUDE, "-I", CSRC, "-o", tmp, *SOURCES, "-lcudart"]
+    if lib == DEBUG_LIB:
+        cmd.insert(1, "-DKVQ_DEBUG")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
-    subprocess.run(cmd, check=True)
-    os.replace(tmp, LIB)
-    return LIB
+    return cmd
+
+
+def build(force: bool = False, verbose: bool = False, debug: bool | None = None) -> str:
+    """Compile what is out of date: the normal library (debug False), the
+    debug build (debug True), or both at once (debug None, the default: two
+    nvcc processes side by side).  Returns the normal library's path (the
+    debug one's when debug is True)."""
+    libs = [LIB, DEBUG_LIB] if debug is None else [DEBUG_LIB if debug else LIB]
+    todo = [lib for lib in libs if force or not up_to_date(lib)]
+    procs = []
+    for lib in todo:
+        tmp = lib + f".tmp{os.getpid()}"
+        procs.append((lib, tmp, subprocess.Popen(_command(lib, tmp, verbose))))
+    failed = [lib for lib, tmp, pr in procs if pr.wait() != 0]
+    if failed:
+        raise subprocess.CalledProcessError(1, f"nvcc ({', '.join(os.path.basename(f) for f in failed)})")
+    for lib, tmp, _ in procs:
+        os.replace(tmp, lib)
+    return DEBUG_LIB if debug else LIB
 
 
 if __name__ == "__main__":
-    print(build(force=True, verbose="--verbose" in sys.argv))
+    only_debug = "--debug-only" in sys.argv
+    print(build(force=True, verbose="--verbose" in sys.argv, debug=True if only_debug else None))

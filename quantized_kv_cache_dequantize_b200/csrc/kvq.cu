@@ -46,10 +46,12 @@ int device_sm_count() {
 
 template <int B, int NG>
 void launch_codec(bool quant, const kvq::CodecArgs &a, cudaStream_t st) {
-    // one flat sweep over (head, group); blocks of 8 warps, a few per SM
-    const int64_t groups = a.n_tokens * NG * a.n_heads;
-    const int64_t per_block = 8 * 16 * (quant ? 1 : kvq::kDeqRounds);
-    const int64_t max_blocks = std::max<int64_t>(1, (groups + per_block - 1) / per_block);
+    // one flat sweep over the rows of all heads; blocks of 8 warps, a few per
+    // SM.  Quantize: 16 groups per warp at a time; dequantize: kDeqUnroll
+    // units of RPU rows per warp at a time.
+    const int64_t rows = a.n_tokens * a.n_heads;
+    const int64_t per_block = quant ? 8 * 16 / NG : 8 * kvq::kDeqUnroll * kvq::DeqShape<NG>::RPU;
+    const int64_t max_blocks = std::max<int64_t>(1, (rows + per_block - 1) / per_block);
     const int64_t blocks = std::max<int64_t>(1, std::min<int64_t>(max_blocks, (int64_t)device_sm_count() * 8));
     if (quant)
         kvq::quantize_kernel<B, NG><<<(unsigned)blocks, 256, 0, st>>>(a);
@@ -121,6 +123,7 @@ struct AttnPlan {
     std::vector<int32_t> seq_part_begin, seq_chunks;  // per sequence
     size_t counters_off = 0, partials_off = 0;
     size_t zero_bytes = 0, total = 0;
+    int64_t n_slots = 0;                            // partial slots of the call (every unit)
 };
 
 int env_int(const char *name, int dflt) {
@@ -406,6 +409,7 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
         plan.seq_chunks[s] = (int32_t)(slot - plan.seq_part_begin[s]);
         if (slot > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
     }
+    plan.n_slots = slot * units;
     size_t off = 256;  // bytes [0, 4): the device status word
     plan.counters_off = off;  // one arrival counter per (sequence, KV head, head block)
     off += ((size_t)n_seqs * units * 4 + 255) / 256 * 256;
@@ -442,9 +446,13 @@ kvq_status launch_attn_grid(int bits, size_t smem, const cudaLaunchConfig_t &cfg
 template <int NG>
 kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n_q_heads, int32_t n_kv_heads,
                           const void *q, float scale, float *out, uint8_t *ws, cudaStream_t st,
-                          const int32_t *dep = nullptr, float *scores = nullptr, const int64_t *score_off = nullptr) {
+                          const int32_t *dep = nullptr, float *scores = nullptr, const int64_t *score_off = nullptr,
+                          bool prefetch = true, int64_t n_scores = 0) {
     kvq::AttnParams prm;
     std::memset(&prm, 0, sizeof prm);
+    prm.n_seqs = (int32_t)plan.seq_chunks.size();
+    prm.n_part_slots = plan.n_slots;
+    prm.n_scores = n_scores;
     prm.q = static_cast<const uint16_t *>(q);
     prm.out = out;
     prm.status = reinterpret_cast<uint32_t *>(ws);
@@ -459,14 +467,16 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
     prm.partials = reinterpret_cast<float *>(ws + plan.partials_off);
     for (const AttnLaunch &L : plan.launches) {
         prm.n_views = L.v1 - L.v0;
-        // The first launch waits for the preceding work at entry (behind a
-        // fused append: only its blocks that read appended rows wait).  Later
-        // launches of the call start as soon as the one before has released
-        // them, so all run concurrently on their own workspace regions; each
-        // waits for its predecessor before it exits, so the call's last grid
-        // completes after all of them.
-        prm.fused = dep != nullptr ? 1 : 0;
+        // The first launch fills its first ring stages, then waits for the
+        // preceding work (behind a fused append, the blocks holding appended
+        // rows are copied only after that wait) and releases the next launch.
+        // Later launches of the call start as soon as the one before has
+        // released them, so all run concurrently on their own workspace
+        // regions; each waits for its predecessor before it exits, so the
+        // call's last grid completes after all of them.
         prm.chain = &L != &plan.launches[0] ? 1 : 0;
+        prm.fused = (dep != nullptr && !prm.chain) ? 1 : 0;
+        prm.prefetch = prefetch ? 1 : 0;
         int begin = 0;
         for (int k = L.v0; k < L.v1; ++k) {
             const int i = plan.order[k];
@@ -498,9 +508,9 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
             begin += d.n_chunks;
         }
         // The grid carries a programmatic dependency on the preceding work in
-        // the stream: it starts with griddepcontrol.wait, so it reads nothing
-        // before its predecessor has completed, while its launch and CTA
-        // scheduling overlap the predecessor's tail.
+        // the stream: before griddepcontrol.wait it only copies packed rows
+        // and windows (prefetch), so its launch, CTA scheduling and first
+        // copies overlap the predecessor's tail.
         cudaLaunchAttribute attr;
         attr.id = cudaLaunchAttributeProgrammaticStreamSerialization;
         attr.val.programmaticStreamSerializationAllowed = 1;
@@ -543,7 +553,7 @@ kvq_status validate_append(const kvq_view *views, int32_t n_views, int32_t n_kv_
 
 // Enqueue the append grids (validated arguments); host counters unchanged.
 kvq_status launch_append(const kvq_view *views, int32_t n_views, int32_t n_kv_heads, int32_t head_dim,
-                         const void *k_new, const void *v_new, cudaStream_t st) {
+                         const void *k_new, const void *v_new, cudaStream_t st, bool early = false) {
     const int ng = head_dim / 64;
     for (int v0 = 0; v0 < n_views; v0 += kvq::kAppendMaxViews) {
         const int v1 = std::min<int>(n_views, v0 + kvq::kAppendMaxViews);
@@ -553,6 +563,7 @@ kvq_status launch_append(const kvq_view *views, int32_t n_views, int32_t n_kv_he
         a.v_new = static_cast<const uint16_t *>(v_new) + (int64_t)v0 * n_kv_heads * head_dim;
         a.n_views = v1 - v0;
         a.n_kv_heads = n_kv_heads;
+        a.early = early ? 1 : 0;
         for (int i = v0; i < v1; ++i) {
             const kvq_view &v = views[i];
             kvq::AppendView &d = a.views[i - v0];
@@ -666,6 +677,7 @@ kvq_status card_launch(bool pack, const kvq_view *views, int32_t n_views, int32_
         kvq::CardArgs a;
         std::memset(&a, 0, sizeof a);
         a.card = card;
+        a.card_bytes = L.total;
         a.n_views = v1 - v0;
         a.n_kv_heads = n_kv_heads;
         a.head_dim = head_dim;
@@ -759,27 +771,17 @@ kvq_status card_parse(const void *card_host, size_t card_bytes, kvq::CardHeader 
 // kvq_decode_attn workspace (status word at byte 0, partials from byte 256).
 static __device__ __align__(256) uint8_t g_noalloc_scratch[KVQ_NOALLOC_SCRATCH_BYTES];
 
-std::mutex g_noalloc_mutex;
-void *g_noalloc_ptr[kMaxDevices] = {};
-
-// Device address of the array on the current device, looked up once per device.
+// Device address of the array on the current device.  It is looked up on
+// every call (a host-side query of the runtime, no device work), so a reset
+// or re-created primary context never leaves a stale address behind; the
+// first lookup on a device also loads the library's device code there.
 kvq_status noalloc_scratch(void **out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess) {
+    void *p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p || !aligned(p, 256)) {
         (void)cudaGetLastError();
         return KVQ_ERR_CUDA;
     }
-    if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
-    std::lock_guard<std::mutex> lock(g_noalloc_mutex);
-    if (!g_noalloc_ptr[dev]) {
-        void *p = nullptr;
-        if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p || !aligned(p, 256)) {
-            (void)cudaGetLastError();
-            return KVQ_ERR_CUDA;
-        }
-        g_noalloc_ptr[dev] = p;
-    }
-    *out = g_noalloc_ptr[dev];
+    *out = p;
     return KVQ_OK;
 }
 
@@ -787,12 +789,13 @@ kvq_status noalloc_scratch(void **out) {
 // scores/score_off as launch_attn_ng.
 kvq_status launch_attn(const AttnPlan &plan, const kvq_view *views, int32_t n_q_heads, int32_t n_kv_heads,
                        int32_t head_dim, const void *q, float scale, float *out, uint8_t *ws, cudaStream_t st,
-                       const int32_t *dep = nullptr, float *scores = nullptr, const int64_t *score_off = nullptr) {
+                       const int32_t *dep = nullptr, float *scores = nullptr, const int64_t *score_off = nullptr,
+                       bool prefetch = true, int64_t n_scores = 0) {
     switch (head_dim / 64) {
-        case 1: return launch_attn_ng<1>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off);
-        case 2: return launch_attn_ng<2>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off);
-        case 3: return launch_attn_ng<3>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off);
-        default: return launch_attn_ng<4>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off);
+        case 1: return launch_attn_ng<1>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off, prefetch, n_scores);
+        case 2: return launch_attn_ng<2>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off, prefetch, n_scores);
+        case 3: return launch_attn_ng<3>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off, prefetch, n_scores);
+        default: return launch_attn_ng<4>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off, prefetch, n_scores);
     }
 }
 
@@ -967,7 +970,8 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
             plan_attn(packed.data(), n_views, seq.data(), n_views, n_q_heads, n_kv_heads, head_dim, splan, true);
         if (ps != KVQ_OK) return ps;
         const kvq_status es = launch_attn(splan, packed.data(), n_q_heads, n_kv_heads, head_dim, q, scale, nullptr,
-                                          ws, st, nullptr, scores, sp.score_off.data());
+                                          ws, st, nullptr, scores, sp.score_off.data(), true,
+                                          (int64_t)((sp.sel_off - sp.scores_off) / sizeof(float)));
         if (es != KVQ_OK) return es;
         scored.clear();  // nothing left for the SIMT kernel
     }
@@ -983,6 +987,7 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
         std::memset(&a, 0, sizeof a);
         a.q = static_cast<const uint16_t *>(q);
         a.scores = scores;
+        a.n_scores = (int64_t)((sp.sel_off - sp.scores_off) / sizeof(float));
         a.scale = scale;
         a.n_views = (int)(v1 - v0);
         a.n_q_heads = n_q_heads;
@@ -1022,6 +1027,8 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
         std::memset(&a, 0, sizeof a);
         a.scores = scores;
         a.sel = sel;
+        a.n_scores = (int64_t)((sp.sel_off - sp.scores_off) / sizeof(float));
+        a.n_sel_rows = n_views;
         a.top_k = top_k;
         a.n_kv_heads = n_kv_heads;
         a.sm_bytes = ng * 8;
@@ -1057,8 +1064,11 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
                                          kvq::kSelectThreads, smem, st, a);
         if (es != KVQ_OK) return es;
     }
-    // 4. attention over the compact views: one KV head each, the group's query heads
-    return launch_attn(sp.attn, sp.compact.data(), group, 1, head_dim, q, scale, out, ws, st);
+    // 4. attention over the compact views: one KV head each, the group's query
+    // heads; the select grid writes the compact rows, so no copy starts
+    // before the dependency wait
+    return launch_attn(sp.attn, sp.compact.data(), group, 1, head_dim, q, scale, out, ws, st, nullptr, nullptr,
+                       nullptr, false);
 }
 
 }  // namespace
@@ -1077,6 +1087,37 @@ KVQ_API const char *kvq_status_string(int32_t status) {
 }
 
 KVQ_API int32_t kvq_abi_version(void) { return kAbiVersion; }
+
+KVQ_API int32_t kvq_debug_build(void) {
+#ifdef KVQ_DEBUG
+    return 1;
+#else
+    return 0;
+#endif
+}
+
+KVQ_API kvq_status kvq_debug_flags(uint32_t *flags, int32_t clear, void *stream) {
+#ifdef KVQ_DEBUG
+    if (!flags || !aligned(flags, 4)) return KVQ_ERR_INVALID_ARG;
+    void *word = nullptr;
+    if (cudaGetSymbolAddress(&word, kvq::g_debug_flags) != cudaSuccess || !word) {
+        (void)cudaGetLastError();
+        return KVQ_ERR_CUDA;
+    }
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    if (cudaMemcpyAsync(flags, word, sizeof(uint32_t), cudaMemcpyDefault, st) != cudaSuccess ||
+        (clear && cudaMemsetAsync(word, 0, sizeof(uint32_t), st) != cudaSuccess)) {
+        (void)cudaGetLastError();
+        return KVQ_ERR_CUDA;
+    }
+    return KVQ_OK;
+#else
+    (void)flags;
+    (void)clear;
+    (void)stream;
+    return KVQ_ERR_UNSUPPORTED;
+#endif
+}
 
 KVQ_API kvq_status kvq_quantize(const void *x, int64_t x_head_stride, int64_t x_tok_stride, int32_t n_heads,
                                 int64_t n_tokens, int32_t head_dim, int32_t bits, void *codes, float *scalemin,
@@ -1169,6 +1210,21 @@ KVQ_API kvq_status kvq_decode_attn_noalloc(const kvq_view *views, int32_t n_view
                        static_cast<uint8_t *>(scratch), st);
 }
 
+KVQ_API kvq_status kvq_decode_attn_noalloc_status(uint32_t *status, void *stream) {
+    if (!status || !aligned(status, 4)) return KVQ_ERR_INVALID_ARG;
+    void *scratch = nullptr;
+    const kvq_status ss = noalloc_scratch(&scratch);
+    if (ss != KVQ_OK) return ss;
+    // stream-ordered: the word as the last call enqueued before this one on
+    // the stream left it
+    if (cudaMemcpyAsync(status, scratch, sizeof(uint32_t), cudaMemcpyDefault, static_cast<cudaStream_t>(stream)) !=
+        cudaSuccess) {
+        (void)cudaGetLastError();
+        return KVQ_ERR_CUDA;
+    }
+    return KVQ_OK;
+}
+
 KVQ_API kvq_status kvq_append_decode_attn(kvq_view *views, int32_t n_views, int32_t n_q_heads, int32_t n_kv_heads,
                                           int32_t head_dim, const void *k_new, const void *v_new, const void *q,
                                           float softmax_scale, float *out, void *workspace, size_t workspace_bytes,
@@ -1193,7 +1249,7 @@ KVQ_API kvq_status kvq_append_decode_attn(kvq_view *views, int32_t n_views, int3
         dep[2 * i + 1] = a.cap_window > 0 ? (b.n_window - 1) / kvq::kTile : -1;
     }
     cudaStream_t st = static_cast<cudaStream_t>(stream);
-    const kvq_status ls = launch_append(views, n_views, n_kv_heads, head_dim, k_new, v_new, st);
+    const kvq_status ls = launch_append(views, n_views, n_kv_heads, head_dim, k_new, v_new, st, true);
     if (ls != KVQ_OK) return ls;
     for (int i = 0; i < n_views; ++i) views[i] = post[i];  // enqueued: advance the counters
     uint8_t *ws = static_cast<uint8_t *>(workspace);
@@ -1241,6 +1297,7 @@ KVQ_API kvq_status kvq_width_sensitivity(const kvq_view *views, int32_t n_views,
         std::memset(&a, 0, sizeof a);
         a.q = static_cast<const uint16_t *>(q);
         a.sens = sens;
+        a.n_rows = n_views;
         a.scale = softmax_scale;
         a.n_q_heads = n_q_heads;
         a.n_kv_heads = n_kv_heads;
@@ -1276,7 +1333,10 @@ KVQ_API kvq_status kvq_allocate_widths(const float *sens, const int64_t *capacit
     for (int i = 0; i < n_views; ++i)
         if (capacity[i] < 0 || capacity[i] > ((int64_t)1 << 40) || !(sens[i] >= 0.f) || std::isinf(sens[i]))
             return KVQ_ERR_INVALID_ARG;
-    const uint64_t unit = budget_bytes > 0 ? (budget_bytes + (uint64_t)units - 1) / (uint64_t)units : 1;
+    // ceil(budget / units) without forming budget + units - 1, which wraps
+    // for budgets near 2^64
+    const uint64_t unit = budget_bytes > 0 ? budget_bytes / (uint64_t)units + (budget_bytes % (uint64_t)units != 0)
+                                           : 1;
     const size_t cap_units = (size_t)(budget_bytes / unit);
     // the back-pointers take one byte per (view, unit): at most 1 GiB
     if ((uint64_t)n_views * (uint64_t)(cap_units + 1) > (1ull << 30)) return KVQ_ERR_UNSUPPORTED;
@@ -1290,9 +1350,13 @@ KVQ_API kvq_status kvq_allocate_widths(const float *sens, const int64_t *capacit
         int8_t *pick = choice.data() + (size_t)i * (cap_units + 1);
         for (int j = 0; j < 4; ++j) {
             const int b = kWidths[j];
-            const uint64_t bytes = (uint64_t)capacity[i] * 2u * (uint64_t)n_kv_heads *
-                                   (uint64_t)(head_dim * b / 8 + head_dim / 64 * 8);
-            const uint64_t c = (bytes + unit - 1) / unit;
+            // up to 2^40 * 2 * 65535 * 288 bytes: wider than 64 bits, so in
+            // 128-bit arithmetic; a cost above the whole budget is simply not
+            // affordable (cap_units + 1 units)
+            const unsigned __int128 bytes = (unsigned __int128)capacity[i] * 2u * (unsigned __int128)n_kv_heads *
+                                            (unsigned __int128)(head_dim * b / 8 + head_dim / 64 * 8);
+            const unsigned __int128 c128 = (bytes + unit - 1) / unit;
+            const uint64_t c = c128 > (unsigned __int128)cap_units ? (uint64_t)cap_units + 1 : (uint64_t)c128;
             cost[(size_t)i * 4 + j] = c;
             const double err = (double)sens[i] / (double)((1 << b) - 1);
             for (size_t u = (size_t)std::min<uint64_t>(c, cap_units + 1); u <= cap_units; ++u) {

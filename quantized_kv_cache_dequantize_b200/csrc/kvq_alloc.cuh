@@ -16,6 +16,8 @@
 
 #include <cstdint>
 
+#include "kvq_debug.cuh"
+
 namespace kvq {
 
 constexpr int kSensMaxViews = 96;  // views per launch
@@ -33,6 +35,7 @@ struct SensView {
 struct SensArgs {
     const uint16_t *q;
     float *sens;
+    int32_t n_rows;            // rows of q and sens (the debug build's checks)
     float scale;
     int32_t n_q_heads;
     int32_t n_kv_heads;
@@ -65,6 +68,11 @@ __global__ void __launch_bounds__(32 * kSensWarps) sensitivity_kernel(const __gr
     const SensView &v = a.views[blockIdx.x];
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int G = a.group;
+    // the view's row and its window ring (debug build; uniform over the CTA)
+    if (!dcheck(v.row >= 0 && v.row < a.n_rows && v.n_window <= v.cap_window && v.window_head >= 0 &&
+                    (v.n_window == 0 || v.window_head < v.cap_window),
+                kDbgSens))
+        return;
     float S = 0.f;
     for (int hk = 0; hk < a.n_kv_heads; ++hk) {
         float rk[NG], rv[NG], vm2 = 0.f;

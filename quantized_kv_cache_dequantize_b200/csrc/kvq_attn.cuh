@@ -36,6 +36,7 @@
 #include <cstdint>
 #include <cuda_bf16.h>
 
+#include "kvq_debug.cuh"
 #include "kvq_ptx.cuh"
 
 namespace kvq {
@@ -87,7 +88,13 @@ struct AttnParams {
     int32_t ring_bytes;          // shared-memory ring per warp
     int32_t fused;               // 1: launched right behind this step's append grid (see dep_step)
     int32_t chain;               // 1: a later launch of a call: no wait at entry, wait before exit
+    int32_t prefetch;            // 1: no grid that may still run before this one writes the packed
+                                 // rows or windows (dep_step blocks aside), so the first ring
+                                 // stages are filled before the dependency wait
     float *scores;               // score grids: [view][H_kv][n_packed] largest logit of the CTA's heads
+    int64_t n_part_slots;        // extents for the debug build's checks: partial slots of the call,
+    int64_t n_scores;            // floats of the score array,
+    int32_t n_seqs;              // rows of q and out
     AttnView views[kAttnMaxViews];
 };
 
@@ -578,6 +585,12 @@ __device__ __forceinline__ void combine_unit(const AttnParams &p, const AttnView
     const int64_t stride = (int64_t)p.n_kv_heads * p.head_blocks * kSlot;  // between chunks
     const float *part0 = p.partials + slot0 * kSlot;
     float4 *out4 = reinterpret_cast<float4 *>(p.out + ((int64_t)V.seq_index * p.n_q_heads + h0) * D);
+    // the unit's chunk slots and output rows (debug build)
+    if (!dcheck(n >= 1 && n <= kMaxChunksPerUnit && slot0 >= 0 &&
+                    slot0 + (int64_t)(n - 1) * p.n_kv_heads * p.head_blocks < p.n_part_slots,
+                kDbgAttnWorkspace) ||
+        !dcheck(V.seq_index < p.n_seqs && h0 + nh <= p.n_q_heads, kDbgAttnIo))
+        return;
     if (n <= 8) {
         // one round of loads: each thread fetches every chunk's (m, l) of its
         // head and O of its 4 outputs at once, then merges in chunk order
@@ -738,15 +751,26 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         uint8_t *dst = ring + (size_t)issue_slot * kBlk;
         uint64_t *bar = &wbar[issue_slot];
         const int n = min(kStepTok, issue_left);
+        const bool stage_ok = dcheck((size_t)(issue_slot + 1) * kBlk <= (size_t)p.ring_bytes, kDbgAttnStage);
         if (!WINDOW) {
             const bool full = n == kStepTok;
             const uint32_t bc = full ? (uint32_t)(kStepTok * RB) : round16((uint32_t)(n * RB));
             const uint32_t bs = full ? (uint32_t)(kStepTok * NG * 8) : round16((uint32_t)(n * NG * 8));
-            mbar_arrive_expect_tx_if(issuer, bar, SCORE ? bc + bs : 2 * (bc + bs));
-            bulk_copy_g2s_if(issuer, dst, src_kc, bc, bar);
-            if (!SCORE) bulk_copy_g2s_if(issuer, dst + kOffV, src_vc, bc, bar);
-            bulk_copy_g2s_if(issuer, dst + kOffKs, src_ks, bs, bar);
-            if (!SCORE) bulk_copy_g2s_if(issuer, dst + kOffVs, src_vs, bs, bar);
+            // the copies stay inside the view's rows of this head (debug build)
+            const int64_t hrows = (int64_t)hk * V.cap_packed;
+            const bool ok = stage_ok &&
+                            dcheck(n > 0 && within(src_kc, bc, V.codes[0] + hrows * RB, V.cap_packed * RB) &&
+                                       within(src_ks, bs, V.scalemin[0] + hrows * NG * 2, V.cap_packed * NG * 8) &&
+                                       (SCORE || (within(src_vc, bc, V.codes[1] + hrows * RB, V.cap_packed * RB) &&
+                                                  within(src_vs, bs, V.scalemin[1] + hrows * NG * 2,
+                                                         V.cap_packed * NG * 8))),
+                                   kDbgAttnPacked);
+            // a refused block completes its barrier without bytes (its stage is garbage)
+            mbar_arrive_expect_tx_if(issuer, bar, !ok ? 0u : SCORE ? bc + bs : 2 * (bc + bs));
+            bulk_copy_g2s_if(issuer && ok, dst, src_kc, bc, bar);
+            if (!SCORE) bulk_copy_g2s_if(issuer && ok, dst + kOffV, src_vc, bc, bar);
+            bulk_copy_g2s_if(issuer && ok, dst + kOffKs, src_ks, bs, bar);
+            if (!SCORE) bulk_copy_g2s_if(issuer && ok, dst + kOffVs, src_vs, bs, bar);
             src_kc += (int64_t)kAdvTok * RB;
             src_vc += (int64_t)kAdvTok * RB;
             src_ks += (int64_t)kAdvTok * NG * 2;
@@ -757,10 +781,12 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             const int kv = issue_blk & 1;
             const uint16_t *base = kv ? win_v : win_k;
             const int first = min(n, V.cap_window - win_phys);
-            mbar_arrive_expect_tx_if(issuer, bar, (uint32_t)(n * D * 2));
-            bulk_copy_g2s_if(issuer, dst, base + (int64_t)win_phys * D, (uint32_t)(first * D * 2), bar);
+            const bool ok = stage_ok && dcheck(n > 0 && win_phys >= 0 && first > 0 && n - first <= V.cap_window,
+                                               kDbgAttnWindow);
+            mbar_arrive_expect_tx_if(issuer, bar, ok ? (uint32_t)(n * D * 2) : 0u);
+            bulk_copy_g2s_if(issuer && ok, dst, base + (int64_t)win_phys * D, (uint32_t)(first * D * 2), bar);
             if (n > first)
-                bulk_copy_g2s_if(issuer, dst + first * D * 2, base, (uint32_t)((n - first) * D * 2), bar);
+                bulk_copy_g2s_if(issuer && ok, dst + first * D * 2, base, (uint32_t)((n - first) * D * 2), bar);
             if (kv == 1) {
                 win_phys = (win_phys + kAdvTok) % V.cap_window;
                 issue_left -= kAdvTok;
@@ -771,19 +797,29 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         if (++issue_slot == S) issue_slot = 0;
     };
 
-    // ---- prologue: barriers, first copies (before anything else waits), q
+    // ---- prologue: barriers and the first copies, then the dependency wait
+    // (q, the partials, the counters and out belong to the stream's order),
+    // then q.  The packed rows and windows of the layer do not depend on the
+    // grid before (prefetch; the blocks an append of the same step writes
+    // wait inside issue_next), so their first ring stages are already in
+    // flight while that grid drains.
     const int n_pro = min(S, n_blocks);
+    if (!p.chain && !p.prefetch) pdl_wait();
     if (lane == 0) {
         for (int s = 0; s < S; ++s) mbar_init(&wbar[s], 1);
         fence_mbar_init();
     }
     __syncwarp();
     for (int b = 0; b < n_pro; ++b) issue_next();
+    if (!p.chain) {
+        pdl_wait();
+        pdl_launch_dependents();  // the next grid may be scheduled as slots free up (it waits in turn)
+    }
     for (int i = tid; i < kHeadsPerCta * D / 8; i += kAttnThreads) {
         const int j = i / (D / 8), d8 = i - j * (D / 8);
         uint4 val = make_uint4(0, 0, 0, 0);
-        // L2 loads: with a fused append this CTA may not have waited for the grids before
-        if (j < nh) val = __ldcg(reinterpret_cast<const uint4 *>(p.q + ((int64_t)V.seq_index * p.n_q_heads + h0 + j) * D) + d8);
+        if (j < nh && dcheck(V.seq_index < p.n_seqs && h0 + j < p.n_q_heads, kDbgAttnIo))
+            val = __ldcg(reinterpret_cast<const uint4 *>(p.q + ((int64_t)V.seq_index * p.n_q_heads + h0 + j) * D) + d8);
         reinterpret_cast<uint4 *>(q_s)[i] = val;
     }
     __syncthreads();
@@ -875,15 +911,16 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             }
             release_cur();
             // largest logit over the CTA's heads (2 per lane, 8 per quad)
-            float *dst = p.scores + V.score_off + (int64_t)hk * V.n_packed + tok0 +
-                         (int64_t)kStepTok * (warp + i * kAttnWarps);
+            const int64_t dst_i = V.score_off + (int64_t)hk * V.n_packed + tok0 + (int64_t)kStepTok * (warp + i * kAttnWarps);
+            float *dst = p.scores + dst_i;
 #pragma unroll
             for (int r = 0; r < 4; ++r) {
                 float m = fmaxf(2 * tig < nh ? lg[r][0] : -INFINITY, 2 * tig + 1 < nh ? lg[r][1] : -INFINITY);
                 m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
                 m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
                 const int row = (r >> 1) * kTile + gid + (r & 1) * 8;
-                if (tig == 0 && row < left) dst[row] = m;
+                if (tig == 0 && row < left && dcheck(dst_i + row >= 0 && dst_i + row < p.n_scores, kDbgAttnIo))
+                    dst[row] = m;
             }
             continue;
         }
@@ -979,7 +1016,9 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     const bool single = V.seq_chunks == 1;
     const int64_t pslot = ((int64_t)(V.part_begin + c) * p.n_kv_heads + hk) * p.head_blocks + z;
     float *part = p.partials + pslot * (kHeadsPerCta * (D + 2));
-    for (int idx = tid; idx < nh * D; idx += kAttnThreads) {
+    const bool io_ok = single ? dcheck(V.seq_index < p.n_seqs && h0 + nh <= p.n_q_heads, kDbgAttnIo)
+                              : dcheck(pslot >= 0 && pslot < p.n_part_slots, kDbgAttnWorkspace);
+    for (int idx = io_ok ? tid : nh * D; idx < nh * D; idx += kAttnThreads) {
         const int j = idx / D, d = idx - j * D;
         float M = -INFINITY;
 #pragma unroll
@@ -1011,10 +1050,14 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     __threadfence();  // this thread's partial stores, before the arrival below
     __syncthreads();
     if (tid == 0) {
-        uint32_t *ctr = p.counters + ((int64_t)V.seq_index * p.n_kv_heads + hk) * p.head_blocks + z;
-        const uint32_t before = atomicAdd(ctr, 1u);
-        const bool last = before + 1 == (uint32_t)V.seq_chunks;
-        if (last) *ctr = 0u;
+        const int64_t ci = ((int64_t)V.seq_index * p.n_kv_heads + hk) * p.head_blocks + z;
+        bool last = false;
+        if (dcheck(ci >= 0 && ci < (int64_t)p.n_seqs * p.n_kv_heads * p.head_blocks, kDbgAttnWorkspace)) {
+            uint32_t *ctr = p.counters + ci;
+            const uint32_t before = atomicAdd(ctr, 1u);
+            last = before + 1 == (uint32_t)V.seq_chunks;
+            if (last) *ctr = 0u;
+        }
         *last_flag = last ? 1 : 0;
     }
     __syncthreads();
@@ -1031,12 +1074,12 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
 // five missed the SM's instruction cache, against one in fifty for one width.
 template <int NG, int BSEL, bool SCORE = false>
 __device__ __forceinline__ void decode_attn_body(const AttnParams &p, uint8_t *smem) {
-    // Inputs may come from the preceding grid.  Behind a fused append, only
-    // the copies of the blocks the append writes wait for it (see dep_step):
-    // that grid waited for everything before it and then released this one.
-    // A later launch of a call starts once the one before has released it.
-    if (!p.fused && !p.chain) pdl_wait();
-    pdl_launch_dependents();  // the next grid may be scheduled as slots free up (it waits in turn)
+    // The first launch of a call waits for the preceding grid inside the
+    // item, after its first copies (see attn_item) and releases the next grid
+    // right after that wait.  A later launch of a call is released by the one
+    // before it once that one has waited, so it needs no wait at entry and
+    // releases the next grid at once.
+    if (p.chain) pdl_launch_dependents();
     // ---- which item: view by binary search over chunk ranges
     const int bx = blockIdx.x;
     int lo = 0, hi = p.n_views - 1;

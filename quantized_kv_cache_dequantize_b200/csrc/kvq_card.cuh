@@ -20,6 +20,8 @@
 
 #include <cstdint>
 
+#include "kvq_debug.cuh"
+
 namespace kvq {
 
 constexpr int kCardMaxViews = 96;  // views per pack/unpack launch
@@ -80,6 +82,7 @@ __host__ __device__ inline int64_t card_pieces_per_head(int64_t rows, int64_t ro
 
 struct CardArgs {
     uint8_t *card;            // device card image
+    uint64_t card_bytes;      // its size (the debug build's checks)
     int32_t n_views;
     int32_t n_kv_heads;
     int32_t head_dim;
@@ -150,6 +153,12 @@ __global__ void __launch_bounds__(256, 4) card_kernel(const __grid_constant__ Ca
     const int64_t h = local / pph, r0 = (local % pph) * card_piece_rows(row);
     const int64_t r1 = min(rows, r0 + card_piece_rows(row));
     uint8_t *card_p = a.card + v.sect_off[sect] + (h * rows + r0) * row;
+    // the piece lies in the card and in the view's rows or ring (debug build)
+    if (!dcheck(h < a.n_kv_heads && r0 >= 0 && r0 <= r1 &&
+                    v.sect_off[sect] + (uint64_t)((h * rows + r1) * row) <= a.card_bytes &&
+                    (window ? r1 <= v.cap_window : r1 <= v.cap_packed),
+                kDbgCard))
+        return;
     if (!window) {
         uint8_t *base = sect < 2 ? v.codes[kv] : reinterpret_cast<uint8_t *>(v.scalemin[kv]);
         uint8_t *view_p = base + (h * v.cap_packed + r0) * row;

@@ -15,7 +15,9 @@
 
 #include <cstdint>
 #include <cuda_bf16.h>
+#include <type_traits>
 
+#include "kvq_debug.cuh"
 #include "kvq_ptx.cuh"
 
 namespace kvq {
@@ -23,6 +25,21 @@ namespace kvq {
 constexpr int kGroup = 64;
 constexpr float kRoundMagic = 12582912.0f;  // 1.5 * 2^23: y + magic rounds y to an integer (RNE)
 constexpr uint32_t kRoundMagicBits = 0x4B400000u;
+
+// The packed words of 32 fields that all hold kRoundMagicBits (field j at bit
+// j*B, mod 2^32): the fast path packs the magic sums' raw bits, 0x4B400000 +
+// c, and removes this constant once per word (shifts and sums are linear mod
+// 2^32, and c < 2^22 never carries into the magic bits).
+template <int B>
+__host__ __device__ constexpr uint32_t magic_pack_word(int w) {
+    uint32_t acc = 0;
+    for (int i = 0; i < 32; ++i) {
+        const int bit = i * B;
+        if ((bit >> 5) == w) acc += kRoundMagicBits << (bit & 31);
+        if ((bit & 31) + B > 32 && (bit >> 5) + 1 == w) acc += kRoundMagicBits >> (32 - (bit & 31));
+    }
+    return acc;
+}
 
 // Quantize one half (32 elements) of a 64-element group held as 16 bf16x2
 // words (also readable at `src`, used only for the rare exact re-check); the
@@ -66,27 +83,41 @@ __device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], con
             if ((bit & 31) + B > 32) packed[(bit >> 5) + 1] += c >> (32 - (bit & 31));
         }
     } else if (s != 0.0f) {
-        // Fast path: y = (x - mn) * RN(1/s) lies within 3*2^(B-24) of the
-        // correctly rounded quotient RN((x - mn)/s) (quotients are <= 2^B), so
-        // unless y is within 2^(B-21) of a half-integer both round to the same
-        // integer (and 0 <= y < 2^B - 1/2: every code is in range).  Elements
+        // Fast path: y = fma(x, r, -RN(mn*r)) with r = RN(1/s) lies within
+        // 2^(B-23) + |mn*r|*2^-24 of the quotient (x - mn)/s (quotients are
+        // <= 2^B), so unless y is within 2^(B-21) + |mn*r|*2^-21 of a
+        // half-integer it rounds to the same integer as the correctly rounded
+        // quotient RN((x - mn)/s) (and every code is in range).  Elements
         // closer than that (bf16 grids make exact ties common) are redone
         // exactly below, without a division.
+        // A group whose min is large against its scale (|mn*r| >= 2^(B+2))
+        // takes y = (x - mn) * r instead (within 3*2^(B-24) of the quotient;
+        // window 2^(B-21)), which keeps y > -1/2 there.
         const float r = __frcp_rn(s);
-        const float lim = 0.5f - __uint_as_float((uint32_t)(127 + B - 21) << 23);
+        const float mr = __fmul_rn(mn, r);
+        const bool fma_ok = fabsf(mr) < __uint_as_float((uint32_t)(127 + B + 2) << 23);
+        const float lim = __fsub_rn(0.5f - __uint_as_float((uint32_t)(127 + B - 21) << 23),
+                                    fma_ok ? __fmul_rn(fabsf(mr), 0x1p-21f) : 0.0f);
         uint32_t near = 0u;
+        auto fast = [&](auto use_fma) {
 #pragma unroll
-        for (int i = 0; i < 32; ++i) {
-            const float xf = (i & 1) ? bf16hi_to_f32(x[i >> 1]) : bf16lo_to_f32(x[i >> 1]);
-            const float y = __fmul_rn(__fsub_rn(xf, mn), r);
-            const float t = __fadd_rn(y, kRoundMagic);
-            const float d = __fsub_rn(y, __fsub_rn(t, kRoundMagic));
-            const uint32_t c = __float_as_uint(t) - kRoundMagicBits;
-            near |= (fabsf(d) <= lim) ? 0u : (1u << i);
-            const int bit = i * B;
-            packed[bit >> 5] += c << (bit & 31);
-            if ((bit & 31) + B > 32) packed[(bit >> 5) + 1] += c >> (32 - (bit & 31));
-        }
+            for (int i = 0; i < 32; ++i) {
+                const float xf = (i & 1) ? bf16hi_to_f32(x[i >> 1]) : bf16lo_to_f32(x[i >> 1]);
+                const float y = use_fma ? __fmaf_rn(xf, r, -mr) : __fmul_rn(__fsub_rn(xf, mn), r);
+                const float t = __fadd_rn(y, kRoundMagic);
+                const float d = __fsub_rn(y, __fsub_rn(t, kRoundMagic));
+                near |= (fabsf(d) <= lim) ? 0u : (1u << i);
+                // the magic sum's bits, 0x4B400000 + c; the constant goes below
+                const uint32_t tb = __float_as_uint(t);
+                const int bit = i * B;
+                packed[bit >> 5] += tb << (bit & 31);
+                if ((bit & 31) + B > 32) packed[(bit >> 5) + 1] += tb >> (32 - (bit & 31));
+            }
+        };
+        if (fma_ok) fast(std::true_type{});
+        else fast(std::false_type{});
+#pragma unroll
+        for (int w = 0; w < B; ++w) packed[w] -= magic_pack_word<B>(w);
         while (near) {
             const int i = __ffs(near) - 1;
             near &= near - 1u;
@@ -103,7 +134,9 @@ __device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], con
             const float xf = (i & 1) ? bf16hi_to_f32(w) : bf16lo_to_f32(w);
             (void)src;
             const float a = __fsub_rn(xf, mn);
-            const float y = __fmul_rn(a, r);
+            // the code the fast path packed (the same arithmetic), and the
+            // half-integer the quotient is near
+            const float y = fma_ok ? __fmaf_rn(xf, r, -mr) : __fmul_rn(a, r);
             const float t = __fadd_rn(y, kRoundMagic);
             const float ri = __fsub_rn(t, kRoundMagic);
             const uint32_t c_fast = __float_as_uint(t) - kRoundMagicBits;
@@ -173,8 +206,6 @@ struct CodecArgs {
 // one narrow window of memory (TLB- and DRAM-page friendly) and every warp's
 // share is balanced across heads.  The (head, group) cursor advances without
 // division.  Each lane pair owns one group.
-constexpr int kDeqRounds = 4;  // dequantize: groups per lane pair per iteration (latency-bound: many loads in flight)
-
 struct SweepCursor {
     int64_t grp;  // group within the head
     int h;        // head
@@ -202,16 +233,21 @@ __global__ void __launch_bounds__(256) quantize_kernel(CodecArgs a) {
         const int64_t t = cur.grp / NG;
         const int g = (int)(cur.grp - t * NG);
         const uint16_t *src = a.x + (int64_t)cur.h * a.x_head_stride + t * a.x_tok_stride + g * kGroup + half * 32;
+        // the row is one of the input's and of the outputs' (debug build); a
+        // refused row is neither read nor written, and its lanes still take
+        // part in the pair's shuffles
+        const bool ok = dcheck(t < a.n_tokens && t < a.head_cap && cur.h < a.n_heads, kDbgCodec);
         uint32_t x[16];
         const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-            const uint4 q = __ldcs(s4 + v);
+            const uint4 q = ok ? __ldcs(s4 + v) : make_uint4(0, 0, 0, 0);
             x[4 * v + 0] = q.x; x[4 * v + 1] = q.y; x[4 * v + 2] = q.z; x[4 * v + 3] = q.w;
         }
         uint32_t packed[B];
         float s, mn;
         quantize_half_group<B>(x, src, packed, s, mn);
+        if (!ok) continue;
         const int64_t row = (int64_t)cur.h * a.head_cap + t;
         uint8_t *dst = a.codes + row * RB + g * 8 * B + half * 4 * B;
         if constexpr (B == 4) {
@@ -229,90 +265,121 @@ __global__ void __launch_bounds__(256) quantize_kernel(CodecArgs a) {
     }
 }
 
-// Same sweep; each lane pair dequantizes kDeqRounds groups per iteration.
-// Software-pipelined: the codes and scale/min of the next iteration are
-// loaded before this iteration's groups are converted and stored, so the load
-// latency overlaps the (3x larger) store stream.
-template <int B>
-struct DeqSet {
-    uint32_t packed[kDeqRounds][B];
-    float2 sm[kDeqRounds];
-    int64_t t[kDeqRounds];
-    int g[kDeqRounds], hh[kDeqRounds];
-    bool ok[kDeqRounds];
+// Dequantize: the rows of all heads form one flat sequence (head-major).  A
+// warp unit is RPU consecutive rows, 32*CPL chunks of 8 elements; lane l owns
+// chunks l, l + 32, ... of its unit, so each warp load of codes and each
+// 16-byte store of a warp covers consecutive bytes (one 512-byte store when
+// the output rows are contiguous).  kDeqUnroll units per iteration: all their
+// loads are issued before the first conversion and store.
+constexpr int kDeqUnroll = 4;
+
+template <int NG>
+struct DeqShape {
+    static constexpr int CPR = 8 * NG;           // 8-element chunks per row
+    static constexpr int CPL = NG == 3 ? 3 : 1;  // chunks per lane per unit
+    static constexpr int RPU = 32 * CPL / CPR;   // rows per unit: 4, 2, 4, 1
 };
 
-template <int B, int NG>
-__device__ __forceinline__ void deq_load(const CodecArgs &a, SweepCursor c, int half, int64_t n_groups, DeqSet<B> &d) {
-    constexpr int RB = 8 * B * NG;
-#pragma unroll
-    for (int u = 0; u < kDeqRounds; ++u) {
-        d.ok[u] = c.h < a.n_heads;
-        d.hh[u] = c.h;
-        d.t[u] = c.grp / NG;
-        d.g[u] = (int)(c.grp - d.t[u] * NG);
-        if (d.ok[u]) {
-            const int64_t row = (int64_t)c.h * a.head_cap + d.t[u];
-            const uint8_t *src = a.codes + row * RB + d.g[u] * 8 * B + half * 4 * B;
-            if constexpr (B == 4) {
-                const uint4 q = __ldcs(reinterpret_cast<const uint4 *>(src));
-                d.packed[u][0] = q.x; d.packed[u][1] = q.y; d.packed[u][2] = q.z; d.packed[u][3] = q.w;
-            } else if constexpr (B == 8) {
-                const uint4 q0 = __ldcs(reinterpret_cast<const uint4 *>(src));
-                const uint4 q1 = __ldcs(reinterpret_cast<const uint4 *>(src) + 1);
-                d.packed[u][0] = q0.x; d.packed[u][1] = q0.y; d.packed[u][2] = q0.z; d.packed[u][3] = q0.w;
-                d.packed[u][4] = q1.x; d.packed[u][5] = q1.y; d.packed[u][6] = q1.z; d.packed[u][7] = q1.w;
-            } else if constexpr (B == 2) {
-                const uint2 q = __ldcs(reinterpret_cast<const uint2 *>(src));
-                d.packed[u][0] = q.x; d.packed[u][1] = q.y;
-            } else {
-#pragma unroll
-                for (int w = 0; w < B; ++w) d.packed[u][w] = __ldcs(reinterpret_cast<const uint32_t *>(src) + w);
-            }
-            d.sm[u] = __ldcs(reinterpret_cast<const float2 *>(a.scalemin + (row * NG + d.g[u]) * 2));
-        }
-        sweep_advance(c, 16, n_groups);
+// The 8 codes of chunk d8 of a row (B bytes at byte d8*B, code j at bit B*j):
+// in .x (and .y for B = 8), read with aligned loads that stay inside the row.
+template <int B>
+__device__ __forceinline__ uint2 load_chunk_codes(const uint8_t *row, int d8) {
+    if constexpr (B == 8) {
+        return __ldcs(reinterpret_cast<const uint2 *>(row) + d8);
+    } else if constexpr (B == 4) {
+        return make_uint2(__ldcs(reinterpret_cast<const uint32_t *>(row) + d8), 0u);
+    } else if constexpr (B == 2) {
+        return make_uint2(__ldcs(reinterpret_cast<const unsigned short *>(row) + d8), 0u);
+    } else {
+        // 3 bytes at any byte offset: the aligned word holding the first, and
+        // the next one only when the bytes run into it (it then still lies
+        // inside the row: rows are 8-byte multiples)
+        const int off = 3 * d8, w = off & ~3, sh = 8 * (off & 3);
+        const uint32_t x = __ldcs(reinterpret_cast<const uint32_t *>(row + w));
+        if ((off & 3) < 2) return make_uint2(x >> sh, 0u);
+        const uint32_t y = __ldcs(reinterpret_cast<const uint32_t *>(row + w + 4));
+        return make_uint2(__funnelshift_r(x, y, sh), 0u);
     }
 }
 
+// 8 codes -> 8 bf16 values bf16_rne(fmaf(c, s, mn)), as one 16-byte vector.
 template <int B>
-__device__ __forceinline__ void deq_store(const CodecArgs &a, int half, const DeqSet<B> &d) {
-    uint16_t *y = const_cast<uint16_t *>(a.x);
+__device__ __forceinline__ uint4 dequant_chunk(uint2 w, float s, float mn) {
+    constexpr uint32_t mask = (1u << B) - 1u;
+    uint32_t y[4];
 #pragma unroll
-    for (int u = 0; u < kDeqRounds; ++u) {
-        if (!d.ok[u]) continue;
-        uint32_t yv[16];
-        dequantize_half_group<B>(d.packed[u], d.sm[u].x, d.sm[u].y, yv);
-        uint4 *dst = reinterpret_cast<uint4 *>(y + (int64_t)d.hh[u] * a.x_head_stride + d.t[u] * a.x_tok_stride +
-                                               d.g[u] * kGroup + half * 32);
+    for (int j = 0; j < 4; ++j) {
+        float c[2];
 #pragma unroll
-        for (int v = 0; v < 4; ++v) __stcs(dst + v, make_uint4(yv[4 * v], yv[4 * v + 1], yv[4 * v + 2], yv[4 * v + 3]));
+        for (int e = 0; e < 2; ++e) {
+            const int i = 2 * j + e;
+            const uint32_t code = (B == 8) ? ((i < 4 ? w.x : w.y) >> (8 * (i & 3))) & 255u : (w.x >> (B * i)) & mask;
+            // exact small integer -> float: 2^23 + c, minus 2^23
+            c[e] = __fsub_rn(__uint_as_float(0x4B000000u | code), 8388608.0f);
+        }
+        y[j] = pack_bf16x2(__fmaf_rn(c[0], s, mn), __fmaf_rn(c[1], s, mn));
     }
+    return make_uint4(y[0], y[1], y[2], y[3]);
 }
 
 template <int B, int NG>
 __global__ void __launch_bounds__(256) dequantize_kernel(CodecArgs a) {
-    const int64_t n_groups = a.n_tokens * NG;
+    using S = DeqShape<NG>;
+    constexpr int RB = 8 * B * NG;
     const int lane = threadIdx.x & 31;
-    const int half = lane & 1;
-    const int64_t warp_global = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
-    const int64_t step = (int64_t)gridDim.x * (blockDim.x >> 5) * 16 * kDeqRounds;
-    SweepCursor cur{0, 0};
-    sweep_advance(cur, warp_global * 16 * kDeqRounds + (lane >> 1), n_groups);
-    if (cur.h >= a.n_heads) return;
-    DeqSet<B> d0, d1;
-    deq_load<B, NG>(a, cur, half, n_groups, d0);
-    while (true) {
-        sweep_advance(cur, step, n_groups);
-        const bool more = cur.h < a.n_heads;
-        if (more) deq_load<B, NG>(a, cur, half, n_groups, d1);
-        deq_store<B>(a, half, d0);
-        if (!more) break;
-        sweep_advance(cur, step, n_groups);
-        const bool more2 = cur.h < a.n_heads;
-        if (more2) deq_load<B, NG>(a, cur, half, n_groups, d0);
-        deq_store<B>(a, half, d1);
-        if (!more2) break;
+    const int64_t warps = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t warp = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5);
+    // rows between a lane's consecutive units, split into whole heads and tokens
+    const int64_t step = warps * S::RPU;
+    const int64_t step_h = step / a.n_tokens, step_t = step - step_h * a.n_tokens;
+    // one (head, token) cursor per chunk the lane owns in a unit
+    int64_t h[S::CPL], t[S::CPL];
+    int d8[S::CPL];
+#pragma unroll
+    for (int k = 0; k < S::CPL; ++k) {
+        const int uc = 32 * k + lane;
+        d8[k] = uc % S::CPR;
+        const int64_t r = warp * S::RPU + uc / S::CPR;
+        h[k] = r / a.n_tokens;
+        t[k] = r - h[k] * a.n_tokens;
+    }
+    uint16_t *yout = const_cast<uint16_t *>(a.x);
+    while (h[0] < a.n_heads || (S::CPL > 1 && h[S::CPL - 1] < a.n_heads)) {
+        uint2 cw[kDeqUnroll][S::CPL];
+        float2 sm[kDeqUnroll][S::CPL];
+        int64_t hh[kDeqUnroll][S::CPL], tt[kDeqUnroll][S::CPL];
+#pragma unroll
+        for (int u = 0; u < kDeqUnroll; ++u) {
+#pragma unroll
+            for (int k = 0; k < S::CPL; ++k) {
+                hh[u][k] = h[k];
+                tt[u][k] = t[k];
+                if (h[k] < a.n_heads && dcheck(t[k] < a.n_tokens && t[k] < a.head_cap, kDbgCodec)) {
+                    const int64_t row = h[k] * a.head_cap + t[k];
+                    cw[u][k] = load_chunk_codes<B>(a.codes + row * RB, d8[k]);
+                    sm[u][k] = __ldcs(reinterpret_cast<const float2 *>(a.scalemin + (row * NG + d8[k] / 8) * 2));
+                } else {
+                    hh[u][k] = a.n_heads;  // nothing to store
+                }
+                t[k] += step_t;
+                h[k] += step_h;
+                if (t[k] >= a.n_tokens) {
+                    t[k] -= a.n_tokens;
+                    ++h[k];
+                }
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < kDeqUnroll; ++u) {
+#pragma unroll
+            for (int k = 0; k < S::CPL; ++k) {
+                if (hh[u][k] >= a.n_heads) continue;
+                const uint4 v = dequant_chunk<B>(cw[u][k], sm[u][k].x, sm[u][k].y);
+                __stcs(reinterpret_cast<uint4 *>(yout + hh[u][k] * a.x_head_stride + tt[u][k] * a.x_tok_stride +
+                                                 d8[k] * 8),
+                       v);
+            }
+        }
     }
 }
 
@@ -338,6 +405,7 @@ struct AppendArgs {
     const uint16_t *v_new;
     int32_t n_views;
     int32_t n_kv_heads;
+    int32_t early;          // 1: release the next grid (this step's attention) before waiting
     AppendView views[kAppendMaxViews];
 };
 
@@ -347,12 +415,23 @@ struct AppendArgs {
 template <int NG>
 __global__ void __launch_bounds__(32) append_kernel(AppendArgs a) {
     constexpr int D = NG * kGroup;
-    pdl_wait();               // the rows it reads or overwrites may belong to the preceding grid
-    pdl_launch_dependents();  // the attention grid may be scheduled meanwhile (it waits in turn)
+    // The next grid is released before the wait only when it is this step's
+    // attention grid, which knows the rows written here and waits before
+    // reading them.  Any other grid after a plain append starts when the
+    // append has completed.
+    if (a.early) pdl_launch_dependents();
+    pdl_wait();  // the rows it reads or overwrites may belong to the preceding grid
     const AppendView &v = a.views[blockIdx.x];
     const int h = blockIdx.y;
     const int kv = blockIdx.z;
     const int lane = threadIdx.x;
+    // the view, the packed row and the ring slot exist (debug build; uniform
+    // over the warp, so a refused block returns whole)
+    if (!dcheck((int)blockIdx.x < a.n_views && h < a.n_kv_heads &&
+                    (!v.flush || (v.packed_row >= 0 && v.packed_row < v.cap_packed)) &&
+                    (v.slot < 0 || v.slot < v.cap_window) && (v.flush || v.slot >= 0),
+                kDbgAppend))
+        return;
     const uint16_t *newrow = (kv ? a.v_new : a.k_new) + ((int64_t)blockIdx.x * a.n_kv_heads + h) * D;
     uint16_t *ring = v.window[kv];
     uint16_t *slotrow = (v.slot >= 0) ? ring + ((int64_t)h * v.cap_window + v.slot) * D : nullptr;

@@ -14,6 +14,7 @@
 
 #include <cstdint>
 
+#include "kvq_debug.cuh"
 #include "kvq_ptx.cuh"
 
 namespace kvq {
@@ -40,6 +41,7 @@ struct ScoreView {
 struct ScoreArgs {
     const uint16_t *q;        // bf16 [n_views][H_q][D]
     float *scores;
+    int64_t n_scores;         // floats of the score array (the debug build's checks)
     float scale;
     int32_t n_views;
     int32_t n_q_heads;
@@ -94,6 +96,8 @@ __global__ void __launch_bounds__(kScoreTok) score_kernel(const __grid_constant_
     for (int tb = tb0; tb < tb0 + kScoreBlocks; ++tb) {
         const int t = tb * kScoreTok + tid;
         if (t >= v.n_packed) break;
+        const int64_t si = v.score_off + (int64_t)hk * v.n_packed + t;
+        if (!dcheck(t < v.cap_packed && si >= 0 && si < a.n_scores, kDbgScore)) break;
         const uint8_t *row = v.k_codes + ((int64_t)hk * v.cap_packed + t) * RB;
         const float2 *smr = reinterpret_cast<const float2 *>(v.k_sm + ((int64_t)hk * v.cap_packed + t) * NG * 2);
         float best = -INFINITY;
@@ -146,7 +150,7 @@ __global__ void __launch_bounds__(kScoreTok) score_kernel(const __grid_constant_
             for (int h = 0; h < kScoreHeads; ++h)
                 if (h0 + h < G) best = fmaxf(best, a.scale * l[h]);
         }
-        a.scores[v.score_off + (int64_t)hk * v.n_packed + t] = best;
+        a.scores[si] = best;
     }
 }
 
@@ -167,6 +171,8 @@ struct SelectView {
 struct SelectArgs {
     const float *scores;
     int32_t *sel;             // int32 [n_views][H_kv][top_k], ascending, -1 padded
+    int64_t n_scores;         // floats of the score array,
+    int32_t n_sel_rows;       // rows of sel (the debug build's checks)
     int32_t top_k;
     int32_t n_kv_heads;
     int32_t sm_bytes;         // scale/min bytes per row: (D/64) * 8
@@ -196,6 +202,13 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const __grid_con
     const int hk = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
     const int n = v.n_packed, K = a.top_k;
     int32_t *out = a.sel + ((int64_t)v.out_row * a.n_kv_heads + hk) * K;
+    // the selection row, the head's scores and its compact rows exist (debug
+    // build; uniform over the CTA, so a refused CTA returns whole)
+    if (!dcheck(v.out_row >= 0 && v.out_row < a.n_sel_rows && hk < a.n_kv_heads &&
+                    (n <= K || (v.score_off >= 0 && v.score_off + (int64_t)(hk + 1) * n <= a.n_scores &&
+                                n <= v.cap_packed && K <= v.cap_compact)),
+                kDbgSelect))
+        return;
     if (n <= K) {
         for (int i = tid; i < K; i += kSelectThreads) out[i] = i < n ? i : -1;
         return;

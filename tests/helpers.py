@@ -97,3 +97,52 @@ def assert_close(out, ref, what=""):
     assert np.all(np.isfinite(out)), f"{what}: non-finite output"
     assert mx <= ATOL and rel <= RTOL_L2, f"{what}: max_abs {mx:.3e} (<= {ATOL}), rel_l2 {rel:.3e} (<= {RTOL_L2})"
     return mx, rel
+
+
+def host_threads() -> int:
+    import os
+    return max(1, len(os.sched_getaffinity(0)))
+
+
+class OracleRunner:
+    """Runs oracle checks on host threads (the C oracle releases the GIL in
+    ctypes calls) while the main thread prepares the next inputs.  submit()
+    takes a function returning None (pass) or a failure message; at most
+    `depth` checks are in flight, which bounds the host memory they hold."""
+
+    def __init__(self, depth: int | None = None):
+        from concurrent.futures import ThreadPoolExecutor
+        self.n = host_threads()
+        self.pool = ThreadPoolExecutor(self.n)
+        self.depth = depth or 2 * self.n
+        self.pending = []
+        self.failures = []
+        self.done = 0
+
+    def _drain(self, keep: int):
+        while len(self.pending) > keep:
+            f = self.pending.pop(0)
+            msg = f.result()
+            self.done += 1
+            if msg:
+                self.failures.append(msg)
+
+    def submit(self, fn, *args):
+        self._drain(self.depth - 1)
+        self.pending.append(self.pool.submit(fn, *args))
+
+    def finish(self):
+        self._drain(0)
+        self.pool.shutdown()
+        assert not self.failures, f"{len(self.failures)} of {self.done} checks failed; first: {self.failures[:3]}"
+        return self.done
+
+
+def close_msg(out, ref, what):
+    """None if out is within the attention tolerance of ref, else a message."""
+    if not np.all(np.isfinite(out)):
+        return f"{what}: non-finite output"
+    mx, rel = compare(out, ref)
+    if mx <= ATOL and rel <= RTOL_L2:
+        return None
+    return f"{what}: max_abs {mx:.3e} (<= {ATOL}), rel_l2 {rel:.3e} (<= {RTOL_L2})"

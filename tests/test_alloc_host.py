@@ -62,3 +62,23 @@ def test_allocation_refuses_oversized_tables():
     with pytest.raises(kvq.KvqError) as e:
         kvq.allocate_widths(np.ones(n, np.float32), np.full(n, 1000), 8, 128, 10 ** 12, units=1 << 20)
     assert e.value.status == kvq.KVQ_ERR_UNSUPPORTED
+
+
+def test_allocation_costs_wider_than_64_bits():
+    # at the argument limits a width's byte cost, 2^40 tokens x 2 x 65535 heads
+    # x 288 bytes at 8 bits and head_dim 256, needs more than 64 bits: it must
+    # come out unaffordable, not wrap around to a small cost that fits the
+    # budget (wrapped, 8 bits would cost about 934 of 4096 units here)
+    H, D = 65535, 256
+    per = lambda b: 2 * H * (D * b // 8 + D // 64 * 8)
+    cap = [1 << 40]
+    assert cap[0] * per(8) >= 1 << 64 > cap[0] * per(2)
+    budget = (1 << 64) - 1
+    want = oracle.allocate_widths([1.0], cap, H, D, budget, units=4096)
+    got = kvq.allocate_widths([1.0], cap, H, D, budget, units=4096)
+    assert got[0] == want[0] and got[1] == want[1]
+    assert got[0] == [2]
+    # below the 2-bit cost nothing fits
+    with pytest.raises(kvq.KvqError) as e:
+        kvq.allocate_widths([1.0], cap, H, D, cap[0] * per(2) - 1, units=4096)
+    assert e.value.status == kvq.KVQ_ERR_CAPACITY

@@ -102,7 +102,9 @@ def test_card_matches_oracle_and_restores_exactly(cuda_device, tmp_path):
         a = kvq.append_decode_attn(views, kn, vn, q, 0.1)
         b = kvq.append_decode_attn(again, kn, vn, q, 0.1)
         torch.cuda.synchronize()
-        torch.testing.assert_close(a, b, rtol=0, atol=1e-6)
+        # the same plan (counts and widths agree; only capacities and ring
+        # slots differ) on the same kernels: bitwise the originals' outputs
+        assert torch.equal(a, b)
 
 
 def test_card_unpack_rejects_mismatched_views(cuda_device):

@@ -1,12 +1,14 @@
 """kvq_decode_attn_noalloc against kvq_decode_attn, through the C ABI.
 
 The no-allocation variant takes its scratch from a fixed per-device array in
-the library instead of a caller workspace.  Two calls in a row (different view
-sets, so the second reuses scratch the first one wrote) must each match
-kvq_decode_attn on the same inputs within the attention tolerance; a call whose
-plan needs more than the array holds is refused with KVQ_ERR_CAPACITY before
-anything is enqueued.  This file sorts last so that it also runs after every
-other GPU test in the same process.
+the library instead of a caller workspace.  It runs the same plan on the same
+kernels as kvq_decode_attn, so two calls in a row (different view sets, so the
+second reuses scratch the first one wrote) must each give bitwise the outputs
+of kvq_decode_attn on the same inputs (and therefore lie within the attention
+tolerance of it); the scratch's status word reads 0 after each call.  A call
+whose plan needs more than the array holds is refused with KVQ_ERR_CAPACITY
+before anything is enqueued.  This file sorts last so that it also runs after
+every other GPU test in the same process.
 """
 import math
 
@@ -24,7 +26,9 @@ def _noalloc(case, scale):
     out = torch.empty((len(case.views), case.n_q_heads, case.head_dim), dtype=torch.float32,
                       device=case.q.device)
     kvq.decode_attn_noalloc(case.views, case.q, scale, out)
+    status = kvq.decode_attn_noalloc_status()
     torch.cuda.synchronize()
+    assert int(status.item()) == 0, "a bounded copy wait gave up"
     return out.cpu().numpy().astype(np.float64)
 
 
@@ -53,10 +57,13 @@ def test_two_calls_in_a_row_match_workspace_path(cuda_device):
         assert_close(got_a[i], ref_a[i], f"noalloc call 1, view {i}")
     for i in range(len(b.views)):
         assert_close(got_b[i], ref_b[i], f"noalloc call 2, view {i}")
+    # the same plan on the same kernels: bitwise the workspace path's outputs
+    assert np.array_equal(got_a, ref_a) and np.array_equal(got_b, ref_b)
     # and once more on the first set, after the second call overwrote the scratch
     again = _noalloc(a, sa)
     for i in range(len(a.views)):
         assert_close(again[i], ref_a[i], f"noalloc call 3, view {i}")
+    assert np.array_equal(again, ref_a)
 
 
 def test_rejects_plans_beyond_the_scratch_array(cuda_device, monkeypatch):
