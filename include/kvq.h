@@ -208,6 +208,16 @@ size_t kvq_decode_attn_workspace_size(const kvq_view *views, int32_t n_views, in
  * The result is deterministic: the same inputs on the same device give the
  * same bits (no floating-point atomics; partial results merge in a fixed
  * order).
+ * Stream order: the attention grid is launched with programmatic stream
+ * serialization.  It starts copying the views' packed rows and windows into
+ * shared memory before it waits for the preceding kernel of the stream, and
+ * reads q, writes out and touches the workspace only after that wait; it
+ * lets the next kernel start once it has waited.  Every library call that
+ * writes packed rows or windows (kvq_append, kvq_quantize, kvq_card_unpack)
+ * lets a following kernel start only when it has completed, and so does any
+ * kernel launched without programmatic serialization.  A caller's own kernel
+ * that writes a view's rows and calls griddepcontrol.launch_dependents
+ * before those writes must not be the kernel right before this call.
  */
 kvq_status kvq_decode_attn(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
                            int32_t n_kv_heads, int32_t head_dim, const void *q,
@@ -366,11 +376,13 @@ kvq_status kvq_allocate_widths(const float *sens, const int64_t *capacity, int32
  *
  * Arguments as in those two calls; the workspace is sized by
  * kvq_decode_attn_workspace_size on the views as they will be after the
- * append (each view's counters advanced by one token).  The attention grid is
- * launched right behind the append grid and every one of its copies starts at
- * once except the copy of the block holding a row the append writes (the
- * flushed packed row, the new window token), which waits for the append grid
- * first; results and cache contents are the same as with the two calls.
+ * append (each view's counters advanced by one token).  The append grid lets
+ * the attention grid start before it waits for the preceding kernel itself,
+ * so the attention grid's copies of packed rows and windows overlap the
+ * previous step's tail (a previous layer's attention, say); only the copy of
+ * the block holding a row the append writes (the flushed packed row, the new
+ * window token) waits for the append grid first.  Results and cache contents
+ * are the same as with the two calls.
  * Errors: those of kvq_append (nothing enqueued, no counter changed) and of
  * kvq_decode_attn's argument checks, all before anything is enqueued;
  * KVQ_ERR_CUDA if a launch fails (the counters are advanced once the append

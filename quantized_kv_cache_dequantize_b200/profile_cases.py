@@ -29,6 +29,13 @@ CASE:
   card-pack-decode
                  kvq_card_pack of every view of the batched decode workload
                  (10 agents x 32 layers, 4096 packed + 128 window)
+  gemma-layer    kvq_decode_attn over one layer of the variable-length decode
+                 workload in Gemma-3-12B shape (6 agents, 16 q / 8 kv heads,
+                 head_dim 256, 4K-32K packed 4-bit tokens + 256-token window)
+  qwen-layer     kvq_decode_attn over one layer of the mixed-precision decode
+                 workload in Qwen3-32B shape (8 agents, 64 q / 8 kv heads,
+                 head_dim 128, 8K-16K packed tokens at the layer's widths
+                 {2, 3, 4, 8} + 128-token window)
 Each case runs 3 warm-up calls, captures one call in a CUDA graph, replays
 it once more and then --reps timed times, and prints the mean time per call
 and the algorithmic GB/s.
@@ -73,7 +80,7 @@ def main(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("case", choices=["decode-layer", "decode-8layers", "quantize", "dequantize", "quantize-handoff",
                                          "dequantize-handoff", "card-pack", "card-unpack", "card-pack-decode", "sparse-layer",
-                                         "sparse-8layers", "decode-long", "sparse-long"])
+                                         "sparse-8layers", "decode-long", "sparse-long", "gemma-layer", "qwen-layer"])
     ap.add_argument("--reps", type=int, default=20)
     a = ap.parse_args(argv)
     dev = torch.device("cuda:0")
@@ -106,6 +113,21 @@ def main(argv=None):
         n_p = w.view_len(0)
         nbytes = w.n_views * (w.n_kv_heads * (n_p * (rb + ng * 8) + top_k * (rb + ng * 8) + w.window * 4 * w.head_dim)
                               + w.n_q_heads * w.head_dim * 6)
+    elif a.case in ("gemma-layer", "qwen-layer"):
+        w = wl.varlen_gemma12b(n_layers=1) if a.case == "gemma-layer" else wl.mixed_qwen32b(n_layers=1)
+        if a.case == "qwen-layer":
+            # the first layer's widths of the 8 x 64 workload (its seeded allocation)
+            full = wl.mixed_qwen32b()
+            w = type(w)(**{**w.__dict__, "bits": tuple(full.view_bits(ag, 0) for ag in range(full.n_agents))})
+        pool = kcache.build_decode(w, dev)
+        q = kcache.decode_queries(w, device=dev)
+        ws = new_workspace(pool.views, w.n_q_heads, device=dev)
+        out = torch.empty((w.n_views, w.n_q_heads, w.head_dim), dtype=torch.float32, device=dev)
+        t = _time(lambda: decode_attn(pool.views, q, w.softmax_scale, out=out, workspace=ws,
+                                       stream=torch.cuda.current_stream()), a.reps)
+        D = w.head_dim
+        nbytes = sum(w.n_kv_heads * (w.view_len(ag) * (2 * D // 8 * w.view_bits(ag, 0) + 2 * (D // 64) * 8) +
+                                     w.window * 4 * D) + w.n_q_heads * D * 6 for ag in range(w.n_agents))
     elif a.case.startswith("decode"):
         w = wl.decode_llama8b(n_layers=8 if a.case == "decode-8layers" else 1,
                               length=32768 if a.case == "decode-long" else 4096)
