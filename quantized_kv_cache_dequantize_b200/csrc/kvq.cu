@@ -105,7 +105,8 @@ kvq_status codec(bool quant, const void *x, int64_t hs, int64_t ts, int32_t n_he
 struct AttnLaunch {
     int v0, v1;          // views order[v0 .. v1) of the plan
     int total_chunks;
-    int bits;            // the width of every view of the launch with packed tokens
+    int bits;            // the width of every view of the launch with packed tokens (0: several,
+                         // the all-widths kernel)
 };
 
 struct ViewChunks {
@@ -263,8 +264,14 @@ kvq_status ensure_attn_smem(size_t smem) {
     }
     std::lock_guard<std::mutex> lock(mu);
     if (dev >= kMaxDevices || configured[dev] < (int)smem) {
-        if (cudaFuncSetAttribute(SCORE ? kvq::score_attn_kernel<NG, BSEL> : kvq::decode_attn_kernel<NG, BSEL>,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) != cudaSuccess) {
+        cudaError_t e;
+        if constexpr (SCORE)
+            e = cudaFuncSetAttribute(kvq::score_attn_kernel<NG, BSEL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem);
+        else
+            e = cudaFuncSetAttribute(kvq::decode_attn_kernel<NG, BSEL>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     (int)smem);
+        if (e != cudaSuccess) {
             (void)cudaGetLastError();
             return KVQ_ERR_CUDA;
         }
@@ -280,7 +287,7 @@ kvq_status ensure_attn_smem(size_t smem) {
 // nothing at all.
 kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_begin, int32_t n_seqs,
                      int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, AttnPlan &plan,
-                     bool allow_empty = false) {
+                     bool allow_empty = false, bool one_width = false) {
     if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
     if (n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads || n_kv_heads > 65535)
         return KVQ_ERR_INVALID_ARG;
@@ -352,9 +359,17 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
     for (int i = 0; i < n_views; ++i)
         bytes_all += (double)views[i].n_packed * packed_token_bytes(head_dim, views[i].bits) +
                      (double)views[i].n_window * window_token_bytes(head_dim);
+    // A call of several widths whose views fit one launch runs as one grid
+    // of the all-widths kernel (unless one_width: the score grids, or
+    // KVQ_WIDTH_SPLIT=1, keep one launch per width).
+    bool mixed = false;
+    for (int k = 1; k < n_used; ++k) mixed |= key(plan.order[k]) != key(plan.order[0]);
+    const bool merge = mixed && !one_width && n_used <= kvq::kAttnMaxViews && env_int("KVQ_WIDTH_SPLIT", 0) == 0;
     for (int v0 = 0; v0 < n_used;) {
         int v1 = v0 + 1;
-        while (v1 < n_used && v1 - v0 < kvq::kAttnMaxViews && key(plan.order[v1]) == key(plan.order[v0])) ++v1;
+        while (v1 < n_used && v1 - v0 < kvq::kAttnMaxViews &&
+               (merge || key(plan.order[v1]) == key(plan.order[v0])))
+            ++v1;
         double bytes = 0;
         for (int k = v0; k < v1; ++k) {
             const kvq_view &v = views[plan.order[k]];
@@ -366,7 +381,7 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
         int64_t chunks = 0;
         plan_free(views, plan.order.data() + v0, v1 - v0, units, head_dim, share, plan.chunks, &chunks);
         if (chunks > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
-        plan.launches.push_back(AttnLaunch{v0, v1, (int)chunks, key(plan.order[v0])});
+        plan.launches.push_back(AttnLaunch{v0, v1, (int)chunks, merge ? 0 : key(plan.order[v0])});
         v0 = v1;
     }
     // A sequence's unit combine holds at most kMaxChunksPerUnit chunks: trim
@@ -426,14 +441,16 @@ template <int NG, int BSEL, bool SCORE>
 kvq_status launch_attn_width(size_t smem, const cudaLaunchConfig_t &cfg, const kvq::AttnParams &prm) {
     const kvq_status es = ensure_attn_smem<NG, BSEL, SCORE>(smem);
     if (es != KVQ_OK) return es;
-    const cudaError_t e = SCORE ? cudaLaunchKernelEx(&cfg, kvq::score_attn_kernel<NG, BSEL>, prm)
-                                : cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, BSEL>, prm);
+    cudaError_t e;
+    if constexpr (SCORE) e = cudaLaunchKernelEx(&cfg, kvq::score_attn_kernel<NG, BSEL>, prm);
+    else e = cudaLaunchKernelEx(&cfg, kvq::decode_attn_kernel<NG, BSEL>, prm);
     return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
 template <int NG, bool SCORE>
 kvq_status launch_attn_grid(int bits, size_t smem, const cudaLaunchConfig_t &cfg, const kvq::AttnParams &prm) {
     switch (bits) {
+        case 0: if constexpr (!SCORE) return launch_attn_width<NG, 0, false>(smem, cfg, prm); else return KVQ_ERR_UNSUPPORTED;
         case 2: return launch_attn_width<NG, 2, SCORE>(smem, cfg, prm);
         case 3: return launch_attn_width<NG, 3, SCORE>(smem, cfg, prm);
         case 4: return launch_attn_width<NG, 4, SCORE>(smem, cfg, prm);
@@ -967,7 +984,7 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
         seq[n_views] = n_views;
         AttnPlan splan;
         const kvq_status ps =
-            plan_attn(packed.data(), n_views, seq.data(), n_views, n_q_heads, n_kv_heads, head_dim, splan, true);
+            plan_attn(packed.data(), n_views, seq.data(), n_views, n_q_heads, n_kv_heads, head_dim, splan, true, true);
         if (ps != KVQ_OK) return ps;
         const kvq_status es = launch_attn(splan, packed.data(), n_q_heads, n_kv_heads, head_dim, q, scale, nullptr,
                                           ws, st, nullptr, scores, sp.score_off.data(), true,

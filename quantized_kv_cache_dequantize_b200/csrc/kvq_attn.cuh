@@ -100,135 +100,122 @@ struct AttnParams {
 
 // ------------------------------------------------------- code unpacking ---
 //
+// Codes enter the tensor cores as fp16 subnormals: a b-bit code moved, with
+// LOP3/PRMT only, to bit offset o (o + b <= 10) of a 16-bit half whose
+// exponent field is zero is the fp16 value c * 2^(o - 24), exactly.  The MMA
+// multiplies it exactly with an fp16 operand and accumulates in fp32, so no
+// conversion instruction and no offset constant is needed; the weight 2^o
+// is compensated in the other operand (QK: in q) or in the output rows (PV).
+//
 // QK operand: lane (gid, tig) holds, for one token row and one group, the 16
 // codes [16*tig, 16*tig + 16) of the group (2*B bytes at byte 2*B*tig).  They
-// become 8 bf16x2 registers r = 0..7; register r holds codes
-// (qk_code<B>(r, 0), qk_code<B>(r, 1)) in its (low, high) halves and feeds
-// k-step r/2, half r%2 of the group's four m16n8k16 steps.  The same map
-// places q in the B operand, so the dot product sums matching elements.
+// become 8 registers r = 0..7; half e of register r holds code qk_code<B>(r, e)
+// at bit qk_off<B>(r, e), and register r feeds k-step r/2, half r%2 of the
+// group's four m16n8k16 steps.  The same map places q (times 2^-offset) in the
+// B operand, so the dot product sums matching elements.
 
 template <int B>
 __host__ __device__ constexpr int qk_code(int r, int e) {
-    return B == 2 ? r + 8 * e : B == 3 ? r + 8 * e : B == 4 ? ((r < 4 ? r : r + 4) + 4 * e) : 2 * r + e;
+    return B == 4 ? 8 * (r / 4) + (r % 4) + 4 * e
+         : B == 8 ? 4 * (r / 2) + (r & 1) + 2 * e
+         : B == 2 ? r + 8 * e
+                  : (r == 7 ? 7 + e : r + 9 * e);
 }
 
-// (bits at offset o in each 16-bit half) -> exact bf16 integers c, 2 per word
-template <int O>
-__device__ __forceinline__ uint32_t bf16_codes(uint32_t w, uint32_t mask_at_o) {
-    // 128 + c*2^O  ->  c   (exact: (128 + c 2^O) * 2^-O - 128 * 2^-O)
-    constexpr uint32_t kMagic = 0x43004300u;  // 128.0 in both halves
-    constexpr uint32_t kScale = (O == 0) ? 0x3F803F80u : (O == 2) ? 0x3E803E80u : (O == 3) ? 0x3E003E00u : 0x3D803D80u;
-    constexpr uint32_t kBias = (O == 0) ? 0xC300C300u : (O == 2) ? 0xC200C200u : (O == 3) ? 0xC180C180u : 0xC100C100u;
-    static_assert(O == 0 || O == 2 || O == 3 || O == 4, "offset");
-    return fma_bf16x2(lop3_and_or(w, mask_at_o, kMagic), kScale, kBias);
-}
-
-// K codes are not normalised: register halves hold 128 + c*2^O as exact bf16
-// (one LOP3), and the B operand carries q*2^-O in the matching slot, so the
-// MMA yields sum q*c + 128 * sum q*2^-O; the second term is a per-(group,
-// head) constant removed in the epilogue.  qk_off<B>(r) is O of register r.
 template <int B>
-__host__ __device__ constexpr int qk_off(int r) {
-    return B == 2 ? (r % 3) * 2 : B == 3 ? (r & 1) * 3 : 0;
-}
-
-__device__ __forceinline__ uint32_t bf16_raw(uint32_t w, uint32_t mask_at_o) {
-    return lop3_and_or(w, mask_at_o, 0x43004300u);  // 128 + (bits under mask), both halves
+__host__ __device__ constexpr int qk_off(int r, int e) {
+    return B == 4 ? 4 * (r & 1)
+         : B == 8 ? 0
+         : B == 2 ? (r < 5 ? 2 * r : 2 * (r - 3))
+                  : (r == 7 ? (e ? 6 : 3) : 3 * (r % 3));
 }
 
 template <int B>
 __device__ __forceinline__ void qk_unpack(const uint8_t *seg, uint32_t (&r)[8]);
 
 template <>
+__device__ __forceinline__ void qk_unpack<4>(const uint8_t *seg, uint32_t (&r)[8]) {
+    // two words of 8 nibbles; per word: nibbles (0,4) and (1,5) in place at
+    // offsets 0 and 4, bytes 1 and 3 moved down for nibbles (2,6) and (3,7)
+    const uint2 w = *reinterpret_cast<const uint2 *>(seg);
+#pragma unroll
+    for (int k = 0; k < 2; ++k) {
+        const uint32_t wk = k ? w.y : w.x;
+        const uint32_t x = prmt(wk, 0u, 0x4341u);
+        r[4 * k + 0] = wk & 0x000F000Fu;
+        r[4 * k + 1] = wk & 0x00F000F0u;
+        r[4 * k + 2] = x & 0x000F000Fu;
+        r[4 * k + 3] = x & 0x00F000F0u;
+    }
+}
+
+template <>
+__device__ __forceinline__ void qk_unpack<8>(const uint8_t *seg, uint32_t (&r)[8]) {
+    // four words of 4 bytes: bytes (0,2) in place, bytes (1,3) moved down
+    // (the zero second source clears the high bytes)
+    const uint4 w = *reinterpret_cast<const uint4 *>(seg);
+    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        r[2 * k] = ws[k] & 0x00FF00FFu;
+        r[2 * k + 1] = prmt(ws[k], 0u, 0x4341u);
+    }
+}
+
+template <>
 __device__ __forceinline__ void qk_unpack<2>(const uint8_t *seg, uint32_t (&r)[8]) {
-    // 16 codes x 2 bits = one word; code j at bit 2j.  Low half: codes 0..7,
-    // high half: codes 8..15; register r = (c_r, c_{r+8}) at offset qk_off<2>(r).
+    // one word, code j at bit 2j (halves: codes 0..7 and 8..15): codes 0..4 of
+    // each half in place at offsets 0..8, codes 5..7 at offsets 4..8 after >> 6
     const uint32_t w = *reinterpret_cast<const uint32_t *>(seg);
-    const uint32_t w6 = w >> 6, w12 = w >> 12;
-    r[0] = bf16_raw(w, 0x00030003u);
-    r[1] = bf16_raw(w, 0x000C000Cu);
-    r[2] = bf16_raw(w, 0x00300030u);
-    r[3] = bf16_raw(w6, 0x00030003u);
-    r[4] = bf16_raw(w6, 0x000C000Cu);
-    r[5] = bf16_raw(w6, 0x00300030u);
-    r[6] = bf16_raw(w12, 0x00030003u);
-    r[7] = bf16_raw(w12, 0x000C000Cu);
+    const uint32_t y = w >> 6;
+    r[0] = w & 0x00030003u;
+    r[1] = w & 0x000C000Cu;
+    r[2] = w & 0x00300030u;
+    r[3] = w & 0x00C000C0u;
+    r[4] = w & 0x03000300u;
+    r[5] = y & 0x00300030u;
+    r[6] = y & 0x00C000C0u;
+    r[7] = y & 0x03000300u;
 }
 
 template <>
 __device__ __forceinline__ void qk_unpack<3>(const uint8_t *seg, uint32_t (&r)[8]) {
-    // 16 codes x 3 bits = 6 bytes at a 2-byte-aligned address; code j at bit
-    // 3j.  Register 2k+e = (c_{2k+e}, c_{2k+8+e}): the 16-bit windows at bits
-    // 6k and 6k+24 are paired into one word, codes at offsets 0 and 3.
+    // 16 codes x 3 bits = 6 bytes at a 2-byte-aligned address, code j at bit
+    // 3j.  16-bit windows at bits 9k hold codes 3k..3k+2 at offsets 0, 3, 6;
+    // windows k and k+3 are paired into one word.
     const uintptr_t addr = reinterpret_cast<uintptr_t>(seg);
     const uint32_t *wp = reinterpret_cast<const uint32_t *>(addr & ~uintptr_t(3));
     const uint32_t sh = (uint32_t)(addr & 3u) * 8u;  // 0 or 16
     const uint32_t w0 = wp[0], w1 = wp[1];
     const uint32_t lo = __funnelshift_r(w0, w1, sh);  // bits 0..31 of the segment
-    const uint32_t hi = w1 >> sh;                     // bits 32..47 (low 16 bits valid)
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        const int a = 6 * k, b = 6 * k + 24;
-        const uint32_t fa = (a == 0) ? lo : __funnelshift_r(lo, hi, a);
-        const uint32_t fb = (b < 32) ? __funnelshift_r(lo, hi, b) : (hi >> (b - 32));
-        const uint32_t pw = prmt(fa, fb, 0x5410u);
-        r[2 * k] = bf16_raw(pw, 0x00070007u);
-        r[2 * k + 1] = bf16_raw(pw, 0x00380038u);
-    }
+    const uint32_t hi = w1 >> sh;                     // bits 32..47 (above: not used)
+    const uint32_t p0 = prmt(lo, __funnelshift_r(lo, hi, 27), 0x5410u);            // codes 0..2 | 9..11
+    const uint32_t x9 = __funnelshift_r(lo, hi, 9);
+    const uint32_t p1 = prmt(x9, hi >> 4, 0x5410u);                                  // codes 3..5 | 12..14
+    const uint32_t x18 = __funnelshift_r(lo, hi, 18);
+    const uint32_t p2 = prmt(x18, hi >> 13, 0x5410u);                                // codes 6..8 | 15
+    r[0] = p0 & 0x00070007u;
+    r[1] = p0 & 0x00380038u;
+    r[2] = p0 & 0x01C001C0u;
+    r[3] = p1 & 0x00070007u;
+    r[4] = p1 & 0x00380038u;
+    r[5] = p1 & 0x01C001C0u;
+    r[6] = p2 & 0x00070007u;
+    r[7] = prmt(x18, x18, 0x1010u) & 0x01C00038u;  // codes 7 (offset 3) | 8 (offset 6)
 }
 
-template <>
-__device__ __forceinline__ void qk_unpack<4>(const uint8_t *seg, uint32_t (&r)[8]) {
-    // 16 codes x 4 bits = 2 words; register k = (c_k, c_{k+4}) from word 0,
-    // register 4+k = (c_{8+k}, c_{12+k}) from word 1.
-    const uint2 w = *reinterpret_cast<const uint2 *>(seg);
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        r[k] = bf16_raw(w.x >> (4 * k), 0x000F000Fu);
-        r[4 + k] = bf16_raw(w.y >> (4 * k), 0x000F000Fu);
-    }
-}
-
-__device__ __forceinline__ float byte_to_f32(uint32_t w, uint32_t sel) {
-    // prmt places the selected byte under exponent 2^23; subtracting 2^23
-    // leaves the byte's value exactly.
-    return __fsub_rn(__uint_as_float(prmt(w, 0x4B000000u, sel)), 8388608.0f);
-}
-
-template <>
-__device__ __forceinline__ void qk_unpack<8>(const uint8_t *seg, uint32_t (&r)[8]) {
-    // 16 bytes; register r = (c_{2r}, c_{2r+1}) as exact bf16 c (no 128 offset).
-    const uint4 w = *reinterpret_cast<const uint4 *>(seg);
-    const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
-#pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        r[2 * k] = pack_bf16x2(byte_to_f32(ws[k], 0x7440u), byte_to_f32(ws[k], 0x7441u));
-        r[2 * k + 1] = pack_bf16x2(byte_to_f32(ws[k], 0x7442u), byte_to_f32(ws[k], 0x7443u));
-    }
-}
-
-// PV operand: lane (gid, tig) holds, for two tokens a and b and one group, the
-// 8 codes [8*gid, 8*gid + 8) (B bytes at byte B*gid); register u = 0..7 holds
-// (code u of token a, code u of token b).
+// PV operand: O^T rows d, columns heads; the A fragment pairs two tokens per
+// register.  Lane (gid, tig) loads, for tokens 2tig, 2tig+1, 2tig+8, 2tig+9 of
+// a 16-token tile, the 8 codes d = 8*gid .. 8*gid+7 of the group (B bytes at
+// byte B*gid).  d-tile t's row gid is d = 8*gid + 2t, its row gid+8 is
+// d = 8*gid + 2t + 1; their codes sit at bit pv_off<B>(t, odd) of fp16
+// subnormals, so output row d accumulates 2^(pv_off - 24) times its value.
 template <int B>
-__device__ __forceinline__ void pv_unpack(const uint8_t *sa, const uint8_t *sb, uint32_t (&r)[8]);
-
-template <>
-__device__ __forceinline__ void pv_unpack<2>(const uint8_t *sa, const uint8_t *sb, uint32_t (&r)[8]) {
-    // 2 bytes per token at a 2-byte-aligned address
-    const uintptr_t a = reinterpret_cast<uintptr_t>(sa);
-    const uint32_t wa = *reinterpret_cast<const uint32_t *>(a & ~uintptr_t(3));
-    const uint32_t wb = *reinterpret_cast<const uint32_t *>(reinterpret_cast<uintptr_t>(sb) & ~uintptr_t(3));
-    const uint32_t p = prmt(wa, wb, (a & 2u) ? 0x7632u : 0x5410u);
-    const uint32_t p6 = p >> 6, p12 = p >> 12;
-    r[0] = bf16_codes<0>(p, 0x00030003u);
-    r[1] = bf16_codes<2>(p, 0x000C000Cu);
-    r[2] = bf16_codes<4>(p, 0x00300030u);
-    r[3] = bf16_codes<0>(p6, 0x00030003u);
-    r[4] = bf16_codes<2>(p6, 0x000C000Cu);
-    r[5] = bf16_codes<4>(p6, 0x00300030u);
-    r[6] = bf16_codes<0>(p12, 0x00030003u);
-    r[7] = bf16_codes<2>(p12, 0x000C000Cu);
+__host__ __device__ constexpr int pv_off(int t, int odd) {
+    return B == 4 ? 4 * odd
+         : B == 8 ? 0
+         : B == 2 ? (odd ? (t == 0 ? 2 : t == 1 ? 6 : t == 2 ? 4 : 8) : (t == 0 ? 0 : t == 1 ? 4 : t == 2 ? 8 : 6))
+                  : (odd ? (t == 0 ? 3 : t == 1 ? 0 : t == 2 ? 0 : 6) : (t == 0 ? 0 : t == 1 ? 6 : 3));
 }
 
 __device__ __forceinline__ uint32_t load24(const uint8_t *s) {
@@ -238,44 +225,57 @@ __device__ __forceinline__ uint32_t load24(const uint8_t *s) {
     return __funnelshift_r(wp[0], wp[1], (uint32_t)(a & 3u) * 8u);
 }
 
-template <>
-__device__ __forceinline__ void pv_unpack<3>(const uint8_t *sa, const uint8_t *sb, uint32_t (&r)[8]) {
-    const uint32_t xa = load24(sa), xb = load24(sb);
-    const uint32_t p1 = prmt(xa, xb, 0x5410u);               // codes 0..4 (+bit 15) of a | of b
-    const uint32_t p2 = prmt(xa >> 15, xb >> 15, 0x5410u);   // codes 5..7
-    const uint32_t p16 = p1 >> 6, p112 = p1 >> 12, p26 = p2 >> 6;
-    r[0] = bf16_codes<0>(p1, 0x00070007u);
-    r[1] = bf16_codes<3>(p1, 0x00380038u);
-    r[2] = bf16_codes<0>(p16, 0x00070007u);
-    r[3] = bf16_codes<3>(p16, 0x00380038u);
-    r[4] = bf16_codes<0>(p112, 0x00070007u);
-    r[5] = bf16_codes<0>(p2, 0x00070007u);
-    r[6] = bf16_codes<3>(p2, 0x00380038u);
-    r[7] = bf16_codes<0>(p26, 0x00070007u);
+// The 8 codes of one token row for this lane (see above), low bits.
+template <int B>
+__device__ __forceinline__ uint2 pv_row(const uint8_t *s) {
+    if constexpr (B == 8) return *reinterpret_cast<const uint2 *>(s);
+    else if constexpr (B == 4) return make_uint2(*reinterpret_cast<const uint32_t *>(s), 0u);
+    else if constexpr (B == 2) return make_uint2(*reinterpret_cast<const uint16_t *>(s), 0u);
+    else return make_uint2(load24(s), 0u);
 }
 
-template <>
-__device__ __forceinline__ void pv_unpack<4>(const uint8_t *sa, const uint8_t *sb, uint32_t (&r)[8]) {
-    const uint32_t wa = *reinterpret_cast<const uint32_t *>(sa);
-    const uint32_t wb = *reinterpret_cast<const uint32_t *>(sb);
-    const uint32_t p1 = prmt(wa, wb, 0x5410u);  // codes 0..3 of a | of b
-    const uint32_t p2 = prmt(wa, wb, 0x7632u);  // codes 4..7
+// Registers of d-tile t for the token pair (a, b): x[0] = row gid (even d),
+// x[1] = row gid+8 (odd d).
+template <int B>
+__device__ __forceinline__ void pv_pair(uint2 a, uint2 b, uint32_t (&x)[4][2]) {
+    if constexpr (B == 4) {
 #pragma unroll
-    for (int k = 0; k < 4; ++k) {
-        r[k] = bf16_codes<0>(p1 >> (4 * k), 0x000F000Fu);
-        r[4 + k] = bf16_codes<0>(p2 >> (4 * k), 0x000F000Fu);
-    }
-}
-
-template <>
-__device__ __forceinline__ void pv_unpack<8>(const uint8_t *sa, const uint8_t *sb, uint32_t (&r)[8]) {
-    const uint2 wa = *reinterpret_cast<const uint2 *>(sa);
-    const uint2 wb = *reinterpret_cast<const uint2 *>(sb);
+        for (int t = 0; t < 4; ++t) {
+            const uint32_t p = prmt(a.x, b.x, (uint32_t)(t | ((4 + t) << 8)));  // byte t of a | of b
+            x[t][0] = p & 0x000F000Fu;
+            x[t][1] = p & 0x00F000F0u;
+        }
+    } else if constexpr (B == 8) {
 #pragma unroll
-    for (int u = 0; u < 8; ++u) {
-        const uint32_t xa = (u < 4) ? wa.x : wa.y, xb = (u < 4) ? wb.x : wb.y;
-        const uint32_t sel = 0x7440u | (u & 3);
-        r[u] = pack_bf16x2(byte_to_f32(xa, sel), byte_to_f32(xb, sel));
+        for (int t = 0; t < 4; ++t) {
+            const uint32_t sa = t < 2 ? a.x : a.y, sb = t < 2 ? b.x : b.y;
+            const uint32_t k = (uint32_t)(2 * t) & 3u;
+            x[t][0] = prmt(sa, sb, k | ((4u + k) << 8)) & 0x00FF00FFu;
+            x[t][1] = prmt(sa, sb, (k + 1u) | ((5u + k) << 8)) & 0x00FF00FFu;
+        }
+    } else if constexpr (B == 2) {
+        const uint32_t p = prmt(a.x, b.x, 0x5410u);  // the 16 bits of a | of b
+        const uint32_t y = p >> 6;
+        x[0][0] = p & 0x00030003u;
+        x[0][1] = p & 0x000C000Cu;
+        x[1][0] = p & 0x00300030u;
+        x[1][1] = p & 0x00C000C0u;
+        x[2][0] = p & 0x03000300u;
+        x[2][1] = y & 0x00300030u;
+        x[3][0] = y & 0x00C000C0u;
+        x[3][1] = y & 0x03000300u;
+    } else {
+        const uint32_t p = prmt(a.x, b.x, 0x5410u);                // codes 0..4 of a | of b
+        const uint32_t y = p >> 9;                                  // codes 3, 4 at offsets 0, 3
+        const uint32_t q = prmt(a.x >> 15, b.x >> 15, 0x5410u);    // codes 5..7 at offsets 0, 3, 6
+        x[0][0] = p & 0x00070007u;
+        x[0][1] = p & 0x00380038u;
+        x[1][0] = p & 0x01C001C0u;
+        x[1][1] = y & 0x00070007u;
+        x[2][0] = y & 0x00380038u;
+        x[2][1] = q & 0x00070007u;
+        x[3][0] = q & 0x00380038u;
+        x[3][1] = q & 0x01C001C0u;
     }
 }
 
@@ -294,9 +294,10 @@ struct WarpState {
     float mt[NG][2];        // min-term partial sums, heads 2tig, 2tig+1
     float m[2];             // running max (log2 units), heads 2tig, 2tig+1
     float l[2];             // running sum (partial over this lane's rows)
-    uint32_t bq[NG][4][2];  // q as B operand: group, k-step, (b0b1, b2b3)
-    float qsum[NG][2];      // sum of q over each group, heads 2tig, 2tig+1
-    float qoff[NG][2];      // -128 * sum of q*2^-O over each group (0 where codes carry no offset)
+    uint32_t bq[NG][4][2];  // q as B operand: group, k-step, (b0b1, b2b3); fp16 (packed items) or bf16 (window)
+    float qsum[NG][2];      // packed items: sum of q over each group / 2^(10 + eq), heads 2tig, 2tig+1
+    float pscale;           // packed items: p*s enters the PV MMA times pscale (a power of two) ...
+    float plimit;           // ... chosen so that p*s*pscale < 2^15 while V scales stay below plimit
 };
 
 // Online-softmax step over R row-sets (R = 2: one 16-token tile, rows gid and
@@ -376,12 +377,14 @@ __device__ __forceinline__ void split_transpose(float a0, float a1, float b0, fl
 }
 
 // QK of one 16-token tile of packed codes: codes rows at `kc` (row stride RB),
-// K scale/min rows at `ks` ([row][NG] float2).  Writes base-2 logits of rows
-// gid, gid+8 (lg0, lg1) for heads 2tig, 2tig+1; rows at or past n_valid are
-// -inf.
+// K scale/min rows at `ks` ([row][NG] float2).  The fp16 MMA accumulates
+// sum_d c_d q_d 2^(-10-eq) per group exactly scaled, so the group's logit is
+// s*acc + mn*qsum (qsum carries the same factor) and `scale` (softmax scale *
+// log2 e * 2^(10+eq)) turns the sum into base-2 logits.  Writes rows gid,
+// gid+8 (lg0, lg1) for heads 2tig, 2tig+1; rows at or past n_valid are -inf.
 template <int B, int NG>
 __device__ __forceinline__ void packed_qk1(const WarpState<NG> &st, const uint8_t *kc, const uint8_t *ks_bytes,
-                                           int n_valid, float scale_log2, int gid, int tig, float (&lg0)[2],
+                                           int n_valid, float scale, int gid, int tig, float (&lg0)[2],
                                            float (&lg1)[2]) {
     constexpr int RB = 8 * B * NG;
     const float2 *sm = reinterpret_cast<const float2 *>(ks_bytes);
@@ -393,11 +396,10 @@ __device__ __forceinline__ void packed_qk1(const WarpState<NG> &st, const uint8_
         uint32_t a0[8], a1[8];
         qk_unpack<B>(row0 + g * 8 * B, a0);
         qk_unpack<B>(row1 + g * 8 * B, a1);
-        // the accumulator starts at the code offset's contribution, -128 sum q*2^-O
-        float acc[4] = {st.qoff[g][0], st.qoff[g][1], st.qoff[g][0], st.qoff[g][1]};
+        float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int s = 0; s < 4; ++s)
-            mma_bf16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0], st.bq[g][s][1]);
+            mma_f16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0], st.bq[g][s][1]);
         const float2 k0 = sm[gid * NG + g], k1 = sm[(gid + 8) * NG + g];
         l00 = fmaf(k0.x, acc[0], fmaf(k0.y, st.qsum[g][0], l00));
         l01 = fmaf(k0.x, acc[1], fmaf(k0.y, st.qsum[g][1], l01));
@@ -406,16 +408,16 @@ __device__ __forceinline__ void packed_qk1(const WarpState<NG> &st, const uint8_
     }
     // rows past the valid count hold stale stage bytes: drop them
     const bool v0 = gid < n_valid, v1 = gid + 8 < n_valid;
-    lg0[0] = v0 ? l00 * scale_log2 : -INFINITY;
-    lg0[1] = v0 ? l01 * scale_log2 : -INFINITY;
-    lg1[0] = v1 ? l10 * scale_log2 : -INFINITY;
-    lg1[1] = v1 ? l11 * scale_log2 : -INFINITY;
+    lg0[0] = v0 ? l00 * scale : -INFINITY;
+    lg0[1] = v0 ? l01 * scale : -INFINITY;
+    lg1[0] = v1 ? l10 * scale : -INFINITY;
+    lg1[1] = v1 ? l11 * scale : -INFINITY;
 }
 
 // QK of both (full) tiles of a packed block; lg rows: tile A gid, tile A
 // gid+8, tile B gid, tile B gid+8.  The two tiles' MMA chains interleave.
 template <int B, int NG>
-__device__ __forceinline__ void packed_qk2(const WarpState<NG> &st, const uint8_t *blk, float scale_log2, int gid,
+__device__ __forceinline__ void packed_qk2(const WarpState<NG> &st, const uint8_t *blk, float scale, int gid,
                                            int tig, float (&lg)[4][2]) {
     constexpr int RB = 8 * B * NG;
     const float2 *sm = reinterpret_cast<const float2 *>(blk + 4 * kTile * RB);
@@ -428,11 +430,11 @@ __device__ __forceinline__ void packed_qk2(const WarpState<NG> &st, const uint8_
             uint32_t a0[8], a1[8];
             qk_unpack<B>(row0 + tt * kTile * RB + g * 8 * B, a0);
             qk_unpack<B>(row0 + tt * kTile * RB + 8 * RB + g * 8 * B, a1);
-            float acc[4] = {st.qoff[g][0], st.qoff[g][1], st.qoff[g][0], st.qoff[g][1]};
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                mma_bf16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0],
-                               st.bq[g][s][1]);
+                mma_f16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0],
+                              st.bq[g][s][1]);
             const float2 k0 = sm[(tt * kTile + gid) * NG + g], k1 = sm[(tt * kTile + gid + 8) * NG + g];
             l[2 * tt][0] = fmaf(k0.x, acc[0], fmaf(k0.y, st.qsum[g][0], l[2 * tt][0]));
             l[2 * tt][1] = fmaf(k0.x, acc[1], fmaf(k0.y, st.qsum[g][1], l[2 * tt][1]));
@@ -442,25 +444,67 @@ __device__ __forceinline__ void packed_qk2(const WarpState<NG> &st, const uint8_
     }
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
-        lg[r][0] = l[r][0] * scale_log2;
-        lg[r][1] = l[r][1] * scale_log2;
+        lg[r][0] = l[r][0] * scale;
+        lg[r][1] = l[r][1] * scale;
     }
+}
+
+// Before the PV of a packed block: V scales of up to `rows` rows of the block
+// (sm rows [row][NG] float2) against the warp's limit.  p (<= 2^8 under the
+// lazy max) times s times pscale must stay below the fp16 range; when a scale
+// reaches plimit, pscale drops to 2^(6 - floor(log2 s_max)) and the O
+// accumulators (in p*s*pscale units) follow.  One warp reduction per block.
+template <int NG>
+__device__ __forceinline__ void track_pscale(WarpState<NG> &st, const uint8_t *vs_bytes, int rows, int gid) {
+    const float2 *sm = reinterpret_cast<const float2 *>(vs_bytes);
+    float mx = 0.f;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+        const int row = gid + 8 * q;  // rows gid, gid+8 of both tiles
+        if (row < rows) {
+#pragma unroll
+            for (int g = 0; g < NG; ++g) mx = fmaxf(mx, sm[row * NG + g].x);
+        }
+    }
+    // scales are >= 0: their bit patterns order like the values
+    const uint32_t wmax = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mx));
+    if (__uint_as_float(wmax) >= st.plimit) {
+        const int ex = max(-100, min(120, (int)(max(wmax, 0x0D800000u) >> 23) - 127));  // floor(log2 s_max)
+        const float ps = __uint_as_float((uint32_t)(127 + 6 - ex) << 23);
+        const float f = ps / st.pscale;  // a power of two: exact
+#pragma unroll
+        for (int g = 0; g < NG; ++g)
+#pragma unroll
+            for (int t = 0; t < 4; ++t)
+#pragma unroll
+                for (int e = 0; e < 4; ++e) st.o[g][t][e] *= f;
+        st.pscale = ps;
+        st.plimit = __uint_as_float((uint32_t)(127 + ex + 1) << 23);
+    }
+}
+
+// hi/lo split of x for two fp16 terms: hi keeps 11 significant bits (exact
+// in fp16 in its normal range), lo = x - hi is exact in fp32 and rounds once
+// in fp16, so hi + lo carries x to about 2^-22.
+__device__ __forceinline__ void split_f16(float x, float &hi, float &lo) {
+    hi = __uint_as_float(__float_as_uint(x) & 0xFFFFE000u);
+    lo = x - hi;
 }
 
 // PV of one 16-token tile: V codes rows at `vc` (row stride RB), V scale/min
 // rows at `vs` ([row][NG] float2); p0/p1 are this lane's probabilities of
-// rows gid, gid+8.  FULL == false zeroes the scale/min of rows at or past
-// n_valid (stale stage bytes; p is 0 there but 0 * NaN would not be).
+// rows gid, gid+8.  O^T[d][h] += codes^T[d][t] . (p s pscale)[t][h] on the
+// fp16 tensor cores (codes as exact subnormals, p*s*pscale as a hi + lo pair
+// of fp16 terms, relative error about 2^-22), plus the min term
+// sum_t p_t mn_t per group in fp32.  FULL == false zeroes the scale/min of
+// rows at or past n_valid (stale stage bytes; p is 0 there but 0 * NaN would
+// not be).
 template <int B, int NG, bool FULL>
-__device__ __forceinline__ void packed_pv(WarpState<NG> &st, const uint8_t *vc, const uint8_t *vs_bytes, int rows,
+__device__ __forceinline__ void packed_pv(WarpState<NG> &st, const uint8_t *vc, const uint8_t *vs_bytes,
                                           int n_valid, const float (&p0)[2], const float (&p1)[2], int gid, int tig) {
     constexpr int RB = 8 * B * NG;
-    (void)rows;
     const float2 *sm = reinterpret_cast<const float2 *>(vs_bytes);
     const uint8_t *ta = vc + (2 * tig) * RB + B * gid;
-    const uint8_t *tb = ta + RB;
-    const uint8_t *tc = ta + 8 * RB;
-    const uint8_t *td = ta + 9 * RB;
 #pragma unroll
     for (int g = 0; g < NG; ++g) {
         float2 m0 = sm[gid * NG + g], m1 = sm[(gid + 8) * NG + g];
@@ -470,15 +514,25 @@ __device__ __forceinline__ void packed_pv(WarpState<NG> &st, const uint8_t *vc, 
         }
         st.mt[g][0] = fmaf(p0[0], m0.y, fmaf(p1[0], m1.y, st.mt[g][0]));
         st.mt[g][1] = fmaf(p0[1], m0.y, fmaf(p1[1], m1.y, st.mt[g][1]));
-        uint32_t bh0, bh1, bl0, bl1;
-        split_transpose(p0[0] * m0.x, p0[1] * m0.x, p1[0] * m1.x, p1[1] * m1.x, bh0, bh1, bl0, bl1);
-        uint32_t va[8], vb[8];
-        pv_unpack<B>(ta + g * 8 * B, tb + g * 8 * B, va);
-        pv_unpack<B>(tc + g * 8 * B, td + g * 8 * B, vb);
+        const float s0 = m0.x * st.pscale, s1 = m1.x * st.pscale;
+        // (p s pscale) of rows gid, gid+8 (heads 2tig, 2tig+1) as hi + lo,
+        // moved to the B-operand layout (tokens along k)
+        float h[4], l[4];
+        split_f16(p0[0] * s0, h[0], l[0]);
+        split_f16(p0[1] * s0, h[1], l[1]);
+        split_f16(p1[0] * s1, h[2], l[2]);
+        split_f16(p1[1] * s1, h[3], l[3]);
+        const uint32_t bh0 = movmatrix_trans(pack_f16x2(h[0], h[1]));
+        const uint32_t bh1 = movmatrix_trans(pack_f16x2(h[2], h[3]));
+        const uint32_t bl0 = movmatrix_trans(pack_f16x2(l[0], l[1]));
+        const uint32_t bl1 = movmatrix_trans(pack_f16x2(l[2], l[3]));
+        uint32_t xab[4][2], xcd[4][2];
+        pv_pair<B>(pv_row<B>(ta + g * 8 * B), pv_row<B>(ta + RB + g * 8 * B), xab);
+        pv_pair<B>(pv_row<B>(ta + 8 * RB + g * 8 * B), pv_row<B>(ta + 9 * RB + g * 8 * B), xcd);
 #pragma unroll
-        for (int t = 0; t < 4; ++t) mma_bf16_16816(st.o[g][t], va[2 * t], va[2 * t + 1], vb[2 * t], vb[2 * t + 1], bh0, bh1);
+        for (int t = 0; t < 4; ++t) mma_f16_16816(st.o[g][t], xab[t][0], xab[t][1], xcd[t][0], xcd[t][1], bh0, bh1);
 #pragma unroll
-        for (int t = 0; t < 4; ++t) mma_bf16_16816(st.o[g][t], va[2 * t], va[2 * t + 1], vb[2 * t], vb[2 * t + 1], bl0, bl1);
+        for (int t = 0; t < 4; ++t) mma_f16_16816(st.o[g][t], xab[t][0], xab[t][1], xcd[t][0], xcd[t][1], bl0, bl1);
     }
 }
 
@@ -825,39 +879,55 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     __syncthreads();
 
     WarpState<NG> st;
+    // base-2 logits per unit of the QK accumulators (window items: bf16 q
+    // as it is; packed items: the factor q was scaled by, see below)
+    float qk_scale = p.scale_log2;
     {
         // q as B operand (column n = gid), k-slots from the unpack map; the
-        // per-group sums of q come from the same registers: each lane adds its
+        // per-group sums of q come from the same values: each lane adds its
         // 16 elements, lanes of one gid combine, then lanes fetch the sums of
         // heads 2tig, 2tig+1.
         const uint16_t *qr = q_s + gid * D;
+        auto qf = [&](int g, int k) { return __uint_as_float((uint32_t)qr[64 * g + 16 * tig + k] << 16); };
+        // packed items: q * 2^(14 - off - eq) in fp16, with 2^eq > max|q| over
+        // the CTA's heads (every warp sees all of them), so that |B| < 2^14
+        // and the products with the codes' 2^(off - 24) carry 2^(-10 - eq)
+        int eq = 0;
+        if (!WINDOW) {
+            float mx = 0.f;
+#pragma unroll
+            for (int g = 0; g < NG; ++g)
+#pragma unroll
+                for (int k = 0; k < 16; ++k) mx = fmaxf(mx, fabsf(qf(g, k)));
+            const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mx));
+            eq = wm == 0u ? 0 : max(-100, min(110, (int)(wm >> 23) - 126));
+            qk_scale = p.scale_log2 * __uint_as_float((uint32_t)(127 + 10 + eq) << 23);
+        }
 #pragma unroll
         for (int g = 0; g < NG; ++g) {
-            float part = 0.f, part_off = 0.f;
+            float part = 0.f;
 #pragma unroll
             for (int s = 0; s < 4; ++s)
 #pragma unroll
                 for (int j = 0; j < 2; ++j) {
                     const int r = 2 * s + j;
-                    const int e0 = WINDOW ? 2 * r : qk_code<B>(r, 0);
-                    const int e1 = WINDOW ? 2 * r + 1 : qk_code<B>(r, 1);
-                    const float q0 = __uint_as_float((uint32_t)qr[64 * g + 16 * tig + e0] << 16);
-                    const float q1 = __uint_as_float((uint32_t)qr[64 * g + 16 * tig + e1] << 16);
-                    const float sc = (WINDOW || B == 8) ? 1.f : __uint_as_float((uint32_t)(127 - qk_off<B>(r)) << 23);
-                    // q * 2^-O is exact in bf16 (exponent change only)
-                    st.bq[g][s][j] = pack_bf16x2(q0 * sc, q1 * sc);
+                    const float q0 = qf(g, WINDOW ? 2 * r : qk_code<B>(r, 0));
+                    const float q1 = qf(g, WINDOW ? 2 * r + 1 : qk_code<B>(r, 1));
+                    if (WINDOW) {
+                        st.bq[g][s][j] = pack_bf16x2(q0, q1);
+                    } else {
+                        // exact: a power-of-two scaling of a bf16 value (fp16 normal range)
+                        const float c0 = __uint_as_float((uint32_t)(127 + 14 - qk_off<B>(r, 0) - eq) << 23);
+                        const float c1 = __uint_as_float((uint32_t)(127 + 14 - qk_off<B>(r, 1) - eq) << 23);
+                        st.bq[g][s][j] = pack_f16x2(q0 * c0, q1 * c1);
+                    }
                     part += q0 + q1;
-                    part_off += q0 * sc + q1 * sc;
                 }
             part += __shfl_xor_sync(0xFFFFFFFFu, part, 1);
             part += __shfl_xor_sync(0xFFFFFFFFu, part, 2);
-            part_off += __shfl_xor_sync(0xFFFFFFFFu, part_off, 1);
-            part_off += __shfl_xor_sync(0xFFFFFFFFu, part_off, 2);
-            st.qsum[g][0] = __shfl_sync(0xFFFFFFFFu, part, 4 * (2 * tig));
-            st.qsum[g][1] = __shfl_sync(0xFFFFFFFFu, part, 4 * (2 * tig + 1));
-            const float off_scale = (WINDOW || B == 8) ? 0.f : -128.f;
-            st.qoff[g][0] = off_scale * __shfl_sync(0xFFFFFFFFu, part_off, 4 * (2 * tig));
-            st.qoff[g][1] = off_scale * __shfl_sync(0xFFFFFFFFu, part_off, 4 * (2 * tig + 1));
+            const float qs = WINDOW ? 1.f : __uint_as_float((uint32_t)(127 - 10 - eq) << 23);
+            st.qsum[g][0] = qs * __shfl_sync(0xFFFFFFFFu, part, 4 * (2 * tig));
+            st.qsum[g][1] = qs * __shfl_sync(0xFFFFFFFFu, part, 4 * (2 * tig + 1));
 #pragma unroll
             for (int t = 0; t < 4; ++t)
 #pragma unroll
@@ -866,6 +936,8 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         }
         st.m[0] = st.m[1] = -INFINITY;
         st.l[0] = st.l[1] = 0.f;
+        st.pscale = 1.f;
+        st.plimit = 0.f;  // the first packed block sets pscale
     }
 
     // consumer position: the current block is in slot `slot`, phase `phase`
@@ -902,12 +974,12 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         if constexpr (SCORE && !WINDOW) {
             float lg[4][2];
             if (left >= kStepTok) {
-                packed_qk2<B, NG>(st, stage, p.scale_log2, gid, tig, lg);
+                packed_qk2<B, NG>(st, stage, qk_scale, gid, tig, lg);
             } else {
-                packed_qk1<B, NG>(st, stage, stage + kOffKs, min(left, kTile), p.scale_log2, gid, tig, lg[0], lg[1]);
+                packed_qk1<B, NG>(st, stage, stage + kOffKs, min(left, kTile), qk_scale, gid, tig, lg[0], lg[1]);
                 if (left > kTile)
                     packed_qk1<B, NG>(st, stage + kTile * RB, stage + kOffKs + kTile * NG * 8, left - kTile,
-                                      p.scale_log2, gid, tig, lg[2], lg[3]);
+                                      qk_scale, gid, tig, lg[2], lg[3]);
             }
             release_cur();
             // largest logit over the CTA's heads (2 per lane, 8 per quad)
@@ -928,33 +1000,34 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             if (left >= kStepTok) {
                 // two full 16-token tiles, one softmax update over 32 tokens
                 float lg[4][2];
-                packed_qk2<B, NG>(st, stage, p.scale_log2, gid, tig, lg);
+                packed_qk2<B, NG>(st, stage, qk_scale, gid, tig, lg);
                 softmax_step_n<NG, 4>(st, lg);
-                packed_pv<B, NG, true>(st, stage + kOffV, stage + kOffVs, 2 * kTile, 0, lg[0], lg[1], gid, tig);
-                packed_pv<B, NG, true>(st, stage + kOffV + kTile * RB, stage + kOffVs + kTile * NG * 8, 2 * kTile, 0,
-                                       lg[2], lg[3], gid, tig);
+                track_pscale<NG>(st, stage + kOffVs, 2 * kTile, gid);
+                packed_pv<B, NG, true>(st, stage + kOffV, stage + kOffVs, 0, lg[0], lg[1], gid, tig);
+                packed_pv<B, NG, true>(st, stage + kOffV + kTile * RB, stage + kOffVs + kTile * NG * 8, 0, lg[2],
+                                       lg[3], gid, tig);
             } else {
                 // the chunk's ragged end: one or two partial tiles
                 float lg[4][2];
-                packed_qk1<B, NG>(st, stage, stage + kOffKs, min(left, kTile), p.scale_log2, gid, tig, lg[0], lg[1]);
+                packed_qk1<B, NG>(st, stage, stage + kOffKs, min(left, kTile), qk_scale, gid, tig, lg[0], lg[1]);
                 if (left > kTile)
                     packed_qk1<B, NG>(st, stage + kTile * RB, stage + kOffKs + kTile * NG * 8, left - kTile,
-                                      p.scale_log2, gid, tig, lg[2], lg[3]);
+                                      qk_scale, gid, tig, lg[2], lg[3]);
                 else
                     lg[2][0] = lg[2][1] = lg[3][0] = lg[3][1] = -INFINITY;
                 softmax_step_n<NG, 4>(st, lg);
-                packed_pv<B, NG, false>(st, stage + kOffV, stage + kOffVs, 2 * kTile, min(left, kTile), lg[0], lg[1],
-                                        gid, tig);
+                track_pscale<NG>(st, stage + kOffVs, min(left, 2 * kTile), gid);  // the block's valid rows
+                packed_pv<B, NG, false>(st, stage + kOffV, stage + kOffVs, min(left, kTile), lg[0], lg[1], gid, tig);
                 if (left > kTile)
-                    packed_pv<B, NG, false>(st, stage + kOffV + kTile * RB, stage + kOffVs + kTile * NG * 8, 2 * kTile,
+                    packed_pv<B, NG, false>(st, stage + kOffV + kTile * RB, stage + kOffVs + kTile * NG * 8,
                                             left - kTile, lg[2], lg[3], gid, tig);
             }
             release_cur();
         } else {
             const int n_valid = min(kTile, left);
             float lg[2][2];
-            if (n_valid == kTile) window_qk<NG, true>(st, stage, n_valid, p.scale_log2, gid, tig, lg);
-            else window_qk<NG, false>(st, stage, n_valid, p.scale_log2, gid, tig, lg);
+            if (n_valid == kTile) window_qk<NG, true>(st, stage, n_valid, qk_scale, gid, tig, lg);
+            else window_qk<NG, false>(st, stage, n_valid, qk_scale, gid, tig, lg);
             release_cur();
             softmax_step_n<NG, 2>(st, lg);
             if (!wait_cur()) { failed = true; break; }
@@ -1000,15 +1073,19 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         wpart[8 + 2 * tig + 1] = st.l[1];
     }
     float *wo = wpart + 16;
+    // packed items: O row d accumulated 2^(pv_off - 24) * pscale times its value
+    const float inv_ps = 1.f / st.pscale;  // a power of two: exact
 #pragma unroll
     for (int g = 0; g < NG; ++g)
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
             const int d0 = 64 * g + 8 * gid + 2 * t;
+            const float fe = WINDOW ? 1.f : inv_ps * __uint_as_float((uint32_t)(127 + 24 - pv_off<B>(t, 0)) << 23);
+            const float fo = WINDOW ? 1.f : inv_ps * __uint_as_float((uint32_t)(127 + 24 - pv_off<B>(t, 1)) << 23);
             *reinterpret_cast<float2 *>(&wo[(2 * tig) * D + d0]) =
-                make_float2(st.o[g][t][0] + st.mt[g][0], st.o[g][t][2] + st.mt[g][0]);
+                make_float2(fmaf(st.o[g][t][0], fe, st.mt[g][0]), fmaf(st.o[g][t][2], fo, st.mt[g][0]));
             *reinterpret_cast<float2 *>(&wo[(2 * tig + 1) * D + d0]) =
-                make_float2(st.o[g][t][1] + st.mt[g][1], st.o[g][t][3] + st.mt[g][1]);
+                make_float2(fmaf(st.o[g][t][1], fe, st.mt[g][1]), fmaf(st.o[g][t][3], fo, st.mt[g][1]));
         }
     __syncthreads();
 
@@ -1069,9 +1146,10 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
 
 // BSEL = 2, 3, 4 or 8: every view of the launch that has packed tokens has
 // that width, and only that width's code is compiled into the kernel (the
-// host groups the views of a call by width, one launch per group).  With all
-// four widths compiled into one function, about one instruction fetch in
-// five missed the SM's instruction cache, against one in fifty for one width.
+// host groups the views of a call by width, one launch per group).  BSEL = 0:
+// all four widths in one kernel, dispatched per CTA; the host uses it for a
+// call of several widths that fits one launch, saving the separate launches'
+// fill and drain at the cost of instruction-cache reach.
 template <int NG, int BSEL, bool SCORE = false>
 __device__ __forceinline__ void decode_attn_body(const AttnParams &p, uint8_t *smem) {
     // The first launch of a call waits for the preceding grid inside the
@@ -1093,16 +1171,25 @@ __device__ __forceinline__ void decode_attn_body(const AttnParams &p, uint8_t *s
     if (c >= V.n_chunks) return;  // never launched by the host planner; defensive
     if constexpr (SCORE) {
         if (c < V.n_chunks_packed) attn_item<NG, BSEL, false, true>(p, V, c, hk, z, smem);
+    } else if constexpr (BSEL == 0) {
+        // every width in one grid: the CTA's view picks the code path (the
+        // host orders views by width, so neighbouring CTAs share one)
+        if (c >= V.n_chunks_packed) attn_item<NG, 4, true>(p, V, c, hk, z, smem);
+        else if (V.bits == 2) attn_item<NG, 2, false>(p, V, c, hk, z, smem);
+        else if (V.bits == 3) attn_item<NG, 3, false>(p, V, c, hk, z, smem);
+        else if (V.bits == 4) attn_item<NG, 4, false>(p, V, c, hk, z, smem);
+        else attn_item<NG, 8, false>(p, V, c, hk, z, smem);
     } else {
         if (c >= V.n_chunks_packed) attn_item<NG, 4, true>(p, V, c, hk, z, smem);
         else attn_item<NG, BSEL, false>(p, V, c, hk, z, smem);
     }
 }
 
+// BSEL = 0: views of any width in one launch (see decode_attn_body).
 template <int NG, int BSEL>
 __global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
     decode_attn_kernel(const __grid_constant__ AttnParams p) {
-    static_assert(BSEL == 2 || BSEL == 3 || BSEL == 4 || BSEL == 8, "width");
+    static_assert(BSEL == 0 || BSEL == 2 || BSEL == 3 || BSEL == 4 || BSEL == 8, "width");
     extern __shared__ __align__(128) uint8_t smem[];
     decode_attn_body<NG, BSEL>(p, smem);
     // a later launch of a call completes only after the one before it, so

@@ -40,7 +40,8 @@ def main():
     # attention: mixed widths, windows, GQA 4, a window-only view, forced chunks
     scale = 1 / np.sqrt(128)
     case = build_case(8, 2, 128, [ViewSpec(300, 16, 16, 4, head=3, seed=1), ViewSpec(97, 0, 0, 2, seed=2),
-                                  ViewSpec(0, 5, 8, 3, head=6, seed=3), ViewSpec(513, 8, 8, 8, head=1, seed=4)])
+                                  ViewSpec(0, 5, 8, 3, head=6, seed=3), ViewSpec(513, 8, 8, 8, head=1, seed=4)],
+                      extra_packed=8)  # room for the decode steps below
     out = kvq.decode_attn(case.views, case.q, scale)
     torch.cuda.synchronize()
     got = out.cpu().numpy().astype(np.float64)
