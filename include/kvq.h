@@ -378,11 +378,13 @@ kvq_status kvq_allocate_widths(const float *sens, const int64_t *capacity, int32
  * kvq_decode_attn_workspace_size on the views as they will be after the
  * append (each view's counters advanced by one token).  The append grid lets
  * the attention grid start before it waits for the preceding kernel itself,
- * so the attention grid's copies of packed rows and windows overlap the
- * previous step's tail (a previous layer's attention, say); only the copy of
- * the block holding a row the append writes (the flushed packed row, the new
- * window token) waits for the append grid first.  Results and cache contents
- * are the same as with the two calls.
+ * and reads k_new, v_new and the windows' oldest tokens and quantizes before
+ * that wait (only its stores follow it); so the attention grid's copies of
+ * packed rows and windows overlap the previous step's tail (a previous
+ * layer's attention, say), and only the copy of the block holding a row the
+ * append writes (the flushed packed row, the new window token) waits for the
+ * append grid.  The stream contract of kvq_decode_attn extends to k_new and
+ * v_new.  Results and cache contents are the same as with the two calls.
  * Errors: those of kvq_append (nothing enqueued, no counter changed) and of
  * kvq_decode_attn's argument checks, all before anything is enqueued;
  * KVQ_ERR_CUDA if a launch fails (the counters are advanced once the append

@@ -105,8 +105,7 @@ kvq_status codec(bool quant, const void *x, int64_t hs, int64_t ts, int32_t n_he
 struct AttnLaunch {
     int v0, v1;          // views order[v0 .. v1) of the plan
     int total_chunks;
-    int bits;            // the width of every view of the launch with packed tokens (0: several,
-                         // the all-widths kernel)
+    int bits;            // the width of every view of the launch with packed tokens
 };
 
 struct ViewChunks {
@@ -164,6 +163,15 @@ int attn_ctas_per_sm(int ng) {
         case 2: return kvq::attn_ctas_per_sm<2>();
         case 3: return kvq::attn_ctas_per_sm<3>();
         default: return kvq::attn_ctas_per_sm<4>();
+    }
+}
+
+int attn_team_warps(int ng) {
+    switch (ng) {
+        case 1: return kvq::attn_team_warps<1>();
+        case 2: return kvq::attn_team_warps<2>();
+        case 3: return kvq::attn_team_warps<3>();
+        default: return kvq::attn_team_warps<4>();
     }
 }
 
@@ -287,7 +295,7 @@ kvq_status ensure_attn_smem(size_t smem) {
 // nothing at all.
 kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_begin, int32_t n_seqs,
                      int32_t n_q_heads, int32_t n_kv_heads, int32_t head_dim, AttnPlan &plan,
-                     bool allow_empty = false, bool one_width = false) {
+                     bool allow_empty = false) {
     if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
     if (n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads || n_kv_heads > 65535)
         return KVQ_ERR_INVALID_ARG;
@@ -329,11 +337,14 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
         if (views[i].n_window > 0) blk_max = std::max<uint32_t>(blk_max, (uint32_t)(32 * head_dim));
     }
     int ring = (smem_cta - header) / kvq::kAttnWarps / 128 * 128;
-    // a ring holds two blocks, and later the warp's partial (m, l, O of 8
-    // heads); all rings together hold the unit combine's scratch
+    // a team's ring (its warps' rings together) holds two blocks, and later
+    // the team's partial (m, l, O of 8 heads); all rings together hold the
+    // unit combine's scratch
+    const uint32_t tw = (uint32_t)attn_team_warps(ng);
     const uint32_t combine_scratch = (2 * kvq::kMaxChunksPerUnit * kvq::kHeadsPerCta + kvq::kHeadsPerCta) * 4;
-    const int ring_min = (int)std::max<uint32_t>(std::max<uint32_t>(2 * blk_max, (uint32_t)(64 + 32 * head_dim)),
-                                                 (combine_scratch + kvq::kAttnWarps - 1) / kvq::kAttnWarps);
+    const int ring_min =
+        (int)std::max<uint32_t>(std::max<uint32_t>((2 * blk_max + tw - 1) / tw, (64 + 32 * (uint32_t)head_dim + tw - 1) / tw),
+                                (combine_scratch + kvq::kAttnWarps - 1) / kvq::kAttnWarps);
     if (ring < ring_min) ring = (ring_min + 127) / 128 * 128;  // fewer CTAs per SM, still correct
     plan.ring_bytes = ring;
     plan.smem = (size_t)header + (size_t)kvq::kAttnWarps * ring;
@@ -359,17 +370,9 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
     for (int i = 0; i < n_views; ++i)
         bytes_all += (double)views[i].n_packed * packed_token_bytes(head_dim, views[i].bits) +
                      (double)views[i].n_window * window_token_bytes(head_dim);
-    // A call of several widths whose views fit one launch runs as one grid
-    // of the all-widths kernel (unless one_width: the score grids, or
-    // KVQ_WIDTH_SPLIT=1, keep one launch per width).
-    bool mixed = false;
-    for (int k = 1; k < n_used; ++k) mixed |= key(plan.order[k]) != key(plan.order[0]);
-    const bool merge = mixed && !one_width && n_used <= kvq::kAttnMaxViews && env_int("KVQ_WIDTH_SPLIT", 0) == 0;
     for (int v0 = 0; v0 < n_used;) {
         int v1 = v0 + 1;
-        while (v1 < n_used && v1 - v0 < kvq::kAttnMaxViews &&
-               (merge || key(plan.order[v1]) == key(plan.order[v0])))
-            ++v1;
+        while (v1 < n_used && v1 - v0 < kvq::kAttnMaxViews && key(plan.order[v1]) == key(plan.order[v0])) ++v1;
         double bytes = 0;
         for (int k = v0; k < v1; ++k) {
             const kvq_view &v = views[plan.order[k]];
@@ -381,7 +384,7 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
         int64_t chunks = 0;
         plan_free(views, plan.order.data() + v0, v1 - v0, units, head_dim, share, plan.chunks, &chunks);
         if (chunks > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
-        plan.launches.push_back(AttnLaunch{v0, v1, (int)chunks, merge ? 0 : key(plan.order[v0])});
+        plan.launches.push_back(AttnLaunch{v0, v1, (int)chunks, key(plan.order[v0])});
         v0 = v1;
     }
     // A sequence's unit combine holds at most kMaxChunksPerUnit chunks: trim
@@ -450,7 +453,6 @@ kvq_status launch_attn_width(size_t smem, const cudaLaunchConfig_t &cfg, const k
 template <int NG, bool SCORE>
 kvq_status launch_attn_grid(int bits, size_t smem, const cudaLaunchConfig_t &cfg, const kvq::AttnParams &prm) {
     switch (bits) {
-        case 0: if constexpr (!SCORE) return launch_attn_width<NG, 0, false>(smem, cfg, prm); else return KVQ_ERR_UNSUPPORTED;
         case 2: return launch_attn_width<NG, 2, SCORE>(smem, cfg, prm);
         case 3: return launch_attn_width<NG, 3, SCORE>(smem, cfg, prm);
         case 4: return launch_attn_width<NG, 4, SCORE>(smem, cfg, prm);
@@ -984,7 +986,7 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
         seq[n_views] = n_views;
         AttnPlan splan;
         const kvq_status ps =
-            plan_attn(packed.data(), n_views, seq.data(), n_views, n_q_heads, n_kv_heads, head_dim, splan, true, true);
+            plan_attn(packed.data(), n_views, seq.data(), n_views, n_q_heads, n_kv_heads, head_dim, splan, true);
         if (ps != KVQ_OK) return ps;
         const kvq_status es = launch_attn(splan, packed.data(), n_q_heads, n_kv_heads, head_dim, q, scale, nullptr,
                                           ws, st, nullptr, scores, sp.score_off.data(), true,

@@ -377,54 +377,56 @@ __device__ __forceinline__ void split_transpose(float a0, float a1, float b0, fl
 }
 
 // QK of one 16-token tile of packed codes: codes rows at `kc` (row stride RB),
-// K scale/min rows at `ks` ([row][NG] float2).  The fp16 MMA accumulates
-// sum_d c_d q_d 2^(-10-eq) per group exactly scaled, so the group's logit is
-// s*acc + mn*qsum (qsum carries the same factor) and `scale` (softmax scale *
-// log2 e * 2^(10+eq)) turns the sum into base-2 logits.  Writes rows gid,
-// gid+8 (lg0, lg1) for heads 2tig, 2tig+1; rows at or past n_valid are -inf.
-template <int B, int NG>
-__device__ __forceinline__ void packed_qk1(const WarpState<NG> &st, const uint8_t *kc, const uint8_t *ks_bytes,
-                                           int n_valid, float scale, int gid, int tig, float (&lg0)[2],
-                                           float (&lg1)[2]) {
+// K scale/min rows at `ks` ([row][NG] float2), over the warp's groups g0 ..
+// g0+NGW-1.  The fp16 MMA accumulates sum_d c_d q_d 2^(-10-eq) per group
+// exactly scaled, so the group's contribution is s*acc + mn*qsum (qsum carries
+// the same factor).  Writes the raw sums of rows gid, gid+8 (l[0], l[1]) for
+// heads 2tig, 2tig+1; the caller adds a team partner's groups, scales to
+// base-2 logits and masks rows past the valid count.
+template <int B, int NG, int NGW>
+__device__ __forceinline__ void packed_qk_tile(const WarpState<NGW> &st, const uint8_t *kc, const uint8_t *ks_bytes,
+                                               int gid, int tig, int g0, float (&l)[2][2]) {
     constexpr int RB = 8 * B * NG;
     const float2 *sm = reinterpret_cast<const float2 *>(ks_bytes);
     const uint8_t *row0 = kc + gid * RB + 2 * B * tig;
     const uint8_t *row1 = row0 + 8 * RB;
     float l00 = 0.f, l01 = 0.f, l10 = 0.f, l11 = 0.f;
 #pragma unroll
-    for (int g = 0; g < NG; ++g) {
+    for (int gg = 0; gg < NGW; ++gg) {
+        const int g = g0 + gg;
         uint32_t a0[8], a1[8];
         qk_unpack<B>(row0 + g * 8 * B, a0);
         qk_unpack<B>(row1 + g * 8 * B, a1);
         float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
         for (int s = 0; s < 4; ++s)
-            mma_f16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0], st.bq[g][s][1]);
+            mma_f16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[gg][s][0], st.bq[gg][s][1]);
         const float2 k0 = sm[gid * NG + g], k1 = sm[(gid + 8) * NG + g];
-        l00 = fmaf(k0.x, acc[0], fmaf(k0.y, st.qsum[g][0], l00));
-        l01 = fmaf(k0.x, acc[1], fmaf(k0.y, st.qsum[g][1], l01));
-        l10 = fmaf(k1.x, acc[2], fmaf(k1.y, st.qsum[g][0], l10));
-        l11 = fmaf(k1.x, acc[3], fmaf(k1.y, st.qsum[g][1], l11));
+        l00 = fmaf(k0.x, acc[0], fmaf(k0.y, st.qsum[gg][0], l00));
+        l01 = fmaf(k0.x, acc[1], fmaf(k0.y, st.qsum[gg][1], l01));
+        l10 = fmaf(k1.x, acc[2], fmaf(k1.y, st.qsum[gg][0], l10));
+        l11 = fmaf(k1.x, acc[3], fmaf(k1.y, st.qsum[gg][1], l11));
     }
-    // rows past the valid count hold stale stage bytes: drop them
-    const bool v0 = gid < n_valid, v1 = gid + 8 < n_valid;
-    lg0[0] = v0 ? l00 * scale : -INFINITY;
-    lg0[1] = v0 ? l01 * scale : -INFINITY;
-    lg1[0] = v1 ? l10 * scale : -INFINITY;
-    lg1[1] = v1 ? l11 * scale : -INFINITY;
+    l[0][0] = l00;
+    l[0][1] = l01;
+    l[1][0] = l10;
+    l[1][1] = l11;
 }
 
-// QK of both (full) tiles of a packed block; lg rows: tile A gid, tile A
-// gid+8, tile B gid, tile B gid+8.  The two tiles' MMA chains interleave.
-template <int B, int NG>
-__device__ __forceinline__ void packed_qk2(const WarpState<NG> &st, const uint8_t *blk, float scale, int gid,
-                                           int tig, float (&lg)[4][2]) {
+// QK of both (full) tiles of a packed block, raw sums; l rows: tile A gid,
+// tile A gid+8, tile B gid, tile B gid+8.  The two tiles' MMA chains
+// interleave.
+template <int B, int NG, int NGW>
+__device__ __forceinline__ void packed_qk_block(const WarpState<NGW> &st, const uint8_t *blk, int gid, int tig, int g0,
+                                                float (&l)[4][2]) {
     constexpr int RB = 8 * B * NG;
     const float2 *sm = reinterpret_cast<const float2 *>(blk + 4 * kTile * RB);
     const uint8_t *row0 = blk + gid * RB + 2 * B * tig;
-    float l[4][2] = {{0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}, {0.f, 0.f}};
 #pragma unroll
-    for (int g = 0; g < NG; ++g) {
+    for (int r = 0; r < 4; ++r) l[r][0] = l[r][1] = 0.f;
+#pragma unroll
+    for (int gg = 0; gg < NGW; ++gg) {
+        const int g = g0 + gg;
 #pragma unroll
         for (int tt = 0; tt < 2; ++tt) {
             uint32_t a0[8], a1[8];
@@ -433,19 +435,14 @@ __device__ __forceinline__ void packed_qk2(const WarpState<NG> &st, const uint8_
             float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
             for (int s = 0; s < 4; ++s)
-                mma_f16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0],
-                              st.bq[g][s][1]);
+                mma_f16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[gg][s][0],
+                              st.bq[gg][s][1]);
             const float2 k0 = sm[(tt * kTile + gid) * NG + g], k1 = sm[(tt * kTile + gid + 8) * NG + g];
-            l[2 * tt][0] = fmaf(k0.x, acc[0], fmaf(k0.y, st.qsum[g][0], l[2 * tt][0]));
-            l[2 * tt][1] = fmaf(k0.x, acc[1], fmaf(k0.y, st.qsum[g][1], l[2 * tt][1]));
-            l[2 * tt + 1][0] = fmaf(k1.x, acc[2], fmaf(k1.y, st.qsum[g][0], l[2 * tt + 1][0]));
-            l[2 * tt + 1][1] = fmaf(k1.x, acc[3], fmaf(k1.y, st.qsum[g][1], l[2 * tt + 1][1]));
+            l[2 * tt][0] = fmaf(k0.x, acc[0], fmaf(k0.y, st.qsum[gg][0], l[2 * tt][0]));
+            l[2 * tt][1] = fmaf(k0.x, acc[1], fmaf(k0.y, st.qsum[gg][1], l[2 * tt][1]));
+            l[2 * tt + 1][0] = fmaf(k1.x, acc[2], fmaf(k1.y, st.qsum[gg][0], l[2 * tt + 1][0]));
+            l[2 * tt + 1][1] = fmaf(k1.x, acc[3], fmaf(k1.y, st.qsum[gg][1], l[2 * tt + 1][1]));
         }
-    }
-#pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        lg[r][0] = l[r][0] * scale;
-        lg[r][1] = l[r][1] * scale;
     }
 }
 
@@ -454,8 +451,8 @@ __device__ __forceinline__ void packed_qk2(const WarpState<NG> &st, const uint8_
 // lazy max) times s times pscale must stay below the fp16 range; when a scale
 // reaches plimit, pscale drops to 2^(6 - floor(log2 s_max)) and the O
 // accumulators (in p*s*pscale units) follow.  One warp reduction per block.
-template <int NG>
-__device__ __forceinline__ void track_pscale(WarpState<NG> &st, const uint8_t *vs_bytes, int rows, int gid) {
+template <int NG, int NGW>
+__device__ __forceinline__ void track_pscale(WarpState<NGW> &st, const uint8_t *vs_bytes, int rows, int gid, int g0) {
     const float2 *sm = reinterpret_cast<const float2 *>(vs_bytes);
     float mx = 0.f;
 #pragma unroll
@@ -463,7 +460,7 @@ __device__ __forceinline__ void track_pscale(WarpState<NG> &st, const uint8_t *v
         const int row = gid + 8 * q;  // rows gid, gid+8 of both tiles
         if (row < rows) {
 #pragma unroll
-            for (int g = 0; g < NG; ++g) mx = fmaxf(mx, sm[row * NG + g].x);
+            for (int gg = 0; gg < NGW; ++gg) mx = fmaxf(mx, sm[row * NG + g0 + gg].x);
         }
     }
     // scales are >= 0: their bit patterns order like the values
@@ -473,7 +470,7 @@ __device__ __forceinline__ void track_pscale(WarpState<NG> &st, const uint8_t *v
         const float ps = __uint_as_float((uint32_t)(127 + 6 - ex) << 23);
         const float f = ps / st.pscale;  // a power of two: exact
 #pragma unroll
-        for (int g = 0; g < NG; ++g)
+        for (int g = 0; g < NGW; ++g)
 #pragma unroll
             for (int t = 0; t < 4; ++t)
 #pragma unroll
@@ -491,60 +488,91 @@ __device__ __forceinline__ void split_f16(float x, float &hi, float &lo) {
     lo = x - hi;
 }
 
-// PV of one 16-token tile: V codes rows at `vc` (row stride RB), V scale/min
-// rows at `vs` ([row][NG] float2); p0/p1 are this lane's probabilities of
-// rows gid, gid+8.  O^T[d][h] += codes^T[d][t] . (p s pscale)[t][h] on the
-// fp16 tensor cores (codes as exact subnormals, p*s*pscale as a hi + lo pair
-// of fp16 terms, relative error about 2^-22), plus the min term
-// sum_t p_t mn_t per group in fp32.  FULL == false zeroes the scale/min of
-// rows at or past n_valid (stale stage bytes; p is 0 there but 0 * NaN would
-// not be).
-template <int B, int NG, bool FULL>
-__device__ __forceinline__ void packed_pv(WarpState<NG> &st, const uint8_t *vc, const uint8_t *vs_bytes,
-                                          int n_valid, const float (&p0)[2], const float (&p1)[2], int gid, int tig) {
+// O += a block's PV sums (one d-tile).  The tensor cores add an MMA's
+// products to its fp32 accumulator after aligning them to the largest term
+// and dropping the bits below, so chaining thousands of tiles through O
+// (whose code terms are all >= 0) loses a little at every MMA, always
+// downward; at 32K tokens in one chunk that came to about 2e-2 relative in
+// the output, where the code and min terms cancel.  Each block's MMAs start
+// from zero instead and O takes the block sum in round-to-nearest fp32 adds:
+// the error no longer grows with the tokens a warp accumulates.
+__device__ __forceinline__ void add_block(float (&o)[4], const float (&acc)[4]) {
+#pragma unroll
+    for (int e = 0; e < 4; ++e) o[e] += acc[e];
+}
+
+// PV of one packed block (two 16-token tiles): V codes rows at `vc` (row
+// stride RB), V scale/min rows at `vs` ([row][NG] float2); p[2tt], p[2tt+1]
+// are this lane's probabilities of tile tt's rows gid, gid+8.
+// O^T[d][h] += codes^T[d][t] . (p s pscale)[t][h] on the fp16 tensor cores
+// (codes as exact subnormals, p*s*pscale as a hi + lo pair of fp16 terms,
+// relative error about 2^-22), group by group, both tiles into one zeroed
+// accumulator that joins O through add_block; plus the min term
+// sum_t p_t mn_t per group in fp32.  FULL == false: only the first n_valid
+// rows hold tokens; a tile past them is skipped, and the scale/min of rows
+// at or past n_valid are zeroed (stale stage bytes; p is 0 there but 0 * NaN
+// would not be).
+template <int B, int NG, int NGW, bool FULL>
+__device__ __forceinline__ void packed_pv_block(WarpState<NGW> &st, const uint8_t *vc, const uint8_t *vs_bytes,
+                                                int n_valid, const float (&p)[4][2], int gid, int tig, int g0) {
     constexpr int RB = 8 * B * NG;
     const float2 *sm = reinterpret_cast<const float2 *>(vs_bytes);
     const uint8_t *ta = vc + (2 * tig) * RB + B * gid;
 #pragma unroll
-    for (int g = 0; g < NG; ++g) {
-        float2 m0 = sm[gid * NG + g], m1 = sm[(gid + 8) * NG + g];
-        if (!FULL) {
-            if (gid >= n_valid) m0 = make_float2(0.f, 0.f);
-            if (gid + 8 >= n_valid) m1 = make_float2(0.f, 0.f);
+    for (int gg = 0; gg < NGW; ++gg) {
+        const int g = g0 + gg;
+        float acc[4][4] = {};
+#pragma unroll
+        for (int tt = 0; tt < 2; ++tt) {
+            if (!FULL && tt * kTile >= n_valid) break;  // warp-uniform
+            const int r0 = tt * kTile + gid;
+            float2 m0 = sm[r0 * NG + g], m1 = sm[(r0 + 8) * NG + g];
+            if (!FULL) {
+                if (r0 >= n_valid) m0 = make_float2(0.f, 0.f);
+                if (r0 + 8 >= n_valid) m1 = make_float2(0.f, 0.f);
+            }
+            const float(&p0)[2] = p[2 * tt];
+            const float(&p1)[2] = p[2 * tt + 1];
+            st.mt[gg][0] = fmaf(p0[0], m0.y, fmaf(p1[0], m1.y, st.mt[gg][0]));
+            st.mt[gg][1] = fmaf(p0[1], m0.y, fmaf(p1[1], m1.y, st.mt[gg][1]));
+            const float s0 = m0.x * st.pscale, s1 = m1.x * st.pscale;
+            // (p s pscale) of rows gid, gid+8 (heads 2tig, 2tig+1) as hi + lo,
+            // moved to the B-operand layout (tokens along k)
+            float h[4], l[4];
+            split_f16(p0[0] * s0, h[0], l[0]);
+            split_f16(p0[1] * s0, h[1], l[1]);
+            split_f16(p1[0] * s1, h[2], l[2]);
+            split_f16(p1[1] * s1, h[3], l[3]);
+            const uint32_t bh0 = movmatrix_trans(pack_f16x2(h[0], h[1]));
+            const uint32_t bh1 = movmatrix_trans(pack_f16x2(h[2], h[3]));
+            const uint32_t bl0 = movmatrix_trans(pack_f16x2(l[0], l[1]));
+            const uint32_t bl1 = movmatrix_trans(pack_f16x2(l[2], l[3]));
+            const uint8_t *tr = ta + tt * kTile * RB + g * 8 * B;
+            uint32_t xab[4][2], xcd[4][2];
+            pv_pair<B>(pv_row<B>(tr), pv_row<B>(tr + RB), xab);
+            pv_pair<B>(pv_row<B>(tr + 8 * RB), pv_row<B>(tr + 9 * RB), xcd);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) mma_f16_16816(acc[t], xab[t][0], xab[t][1], xcd[t][0], xcd[t][1], bh0, bh1);
+#pragma unroll
+            for (int t = 0; t < 4; ++t) mma_f16_16816(acc[t], xab[t][0], xab[t][1], xcd[t][0], xcd[t][1], bl0, bl1);
         }
-        st.mt[g][0] = fmaf(p0[0], m0.y, fmaf(p1[0], m1.y, st.mt[g][0]));
-        st.mt[g][1] = fmaf(p0[1], m0.y, fmaf(p1[1], m1.y, st.mt[g][1]));
-        const float s0 = m0.x * st.pscale, s1 = m1.x * st.pscale;
-        // (p s pscale) of rows gid, gid+8 (heads 2tig, 2tig+1) as hi + lo,
-        // moved to the B-operand layout (tokens along k)
-        float h[4], l[4];
-        split_f16(p0[0] * s0, h[0], l[0]);
-        split_f16(p0[1] * s0, h[1], l[1]);
-        split_f16(p1[0] * s1, h[2], l[2]);
-        split_f16(p1[1] * s1, h[3], l[3]);
-        const uint32_t bh0 = movmatrix_trans(pack_f16x2(h[0], h[1]));
-        const uint32_t bh1 = movmatrix_trans(pack_f16x2(h[2], h[3]));
-        const uint32_t bl0 = movmatrix_trans(pack_f16x2(l[0], l[1]));
-        const uint32_t bl1 = movmatrix_trans(pack_f16x2(l[2], l[3]));
-        uint32_t xab[4][2], xcd[4][2];
-        pv_pair<B>(pv_row<B>(ta + g * 8 * B), pv_row<B>(ta + RB + g * 8 * B), xab);
-        pv_pair<B>(pv_row<B>(ta + 8 * RB + g * 8 * B), pv_row<B>(ta + 9 * RB + g * 8 * B), xcd);
 #pragma unroll
-        for (int t = 0; t < 4; ++t) mma_f16_16816(st.o[g][t], xab[t][0], xab[t][1], xcd[t][0], xcd[t][1], bh0, bh1);
-#pragma unroll
-        for (int t = 0; t < 4; ++t) mma_f16_16816(st.o[g][t], xab[t][0], xab[t][1], xcd[t][0], xcd[t][1], bl0, bl1);
+        for (int t = 0; t < 4; ++t) add_block(st.o[gg][t], acc[t]);
     }
 }
 
-// K half of a window tile: block = K rows [16][D] bf16.
-template <int NG, bool FULL>
-__device__ __forceinline__ void window_qk(const WarpState<NG> &st, const uint8_t *blk, int n_valid,
-                                          float scale_log2, int gid, int tig, float (&lg)[2][2]) {
+// K half of a window tile: block = K rows [16][D] bf16, over the warp's
+// groups g0 .. g0+NGW-1; raw sums of rows gid, gid+8 (l[0], l[1]) for heads
+// 2tig, 2tig+1 (the caller adds a team partner's groups, scales and masks).
+template <int NG, int NGW>
+__device__ __forceinline__ void window_qk(const WarpState<NGW> &st, const uint8_t *blk, int gid, int tig, int g0,
+                                          float (&l)[2][2]) {
     constexpr int D = 64 * NG;
     const uint16_t *k = reinterpret_cast<const uint16_t *>(blk);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-    for (int g = 0; g < NG; ++g) {
+    for (int gg = 0; gg < NGW; ++gg) {
+        const int g = g0 + gg;
         const uint4 *p0 = reinterpret_cast<const uint4 *>(k + gid * D + 64 * g + 16 * tig);
         const uint4 *p1 = reinterpret_cast<const uint4 *>(k + (gid + 8) * D + 64 * g + 16 * tig);
         const uint4 x0 = p0[0], x1 = p0[1], y0 = p1[0], y1 = p1[1];
@@ -552,30 +580,26 @@ __device__ __forceinline__ void window_qk(const WarpState<NG> &st, const uint8_t
         const uint32_t a1[8] = {y0.x, y0.y, y0.z, y0.w, y1.x, y1.y, y1.z, y1.w};
 #pragma unroll
         for (int s = 0; s < 4; ++s)
-            mma_bf16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[g][s][0], st.bq[g][s][1]);
+            mma_bf16_16816(acc, a0[2 * s], a1[2 * s], a0[2 * s + 1], a1[2 * s + 1], st.bq[gg][s][0], st.bq[gg][s][1]);
     }
-    lg[0][0] = acc[0] * scale_log2;
-    lg[0][1] = acc[1] * scale_log2;
-    lg[1][0] = acc[2] * scale_log2;
-    lg[1][1] = acc[3] * scale_log2;
-    if (!FULL) {
-        if (gid >= n_valid) lg[0][0] = lg[0][1] = -INFINITY;
-        if (gid + 8 >= n_valid) lg[1][0] = lg[1][1] = -INFINITY;
-    }
+    l[0][0] = acc[0];
+    l[0][1] = acc[1];
+    l[1][0] = acc[2];
+    l[1][1] = acc[3];
 }
 
-// V half of a window tile: block = V rows [16][D] bf16.
-template <int NG, bool FULL>
-__device__ __forceinline__ void window_pv(WarpState<NG> &st, const uint8_t *blk, int n_valid,
-                                          const float (&p)[2][2], int gid, int tig) {
+// V half of a window tile: block = V rows [16][D] bf16, the warp's groups.
+template <int NG, int NGW, bool FULL>
+__device__ __forceinline__ void window_pv(WarpState<NGW> &st, const uint8_t *blk, int n_valid,
+                                          const float (&p)[2][2], int gid, int tig, int g0) {
     constexpr int D = 64 * NG;
     const uint16_t *v = reinterpret_cast<const uint16_t *>(blk);
     uint32_t bh0, bh1, bl0, bl1;
     split_transpose(p[0][0], p[0][1], p[1][0], p[1][1], bh0, bh1, bl0, bl1);
     const int ta = 2 * tig, tb = 2 * tig + 1, tc = 2 * tig + 8, td = 2 * tig + 9;
 #pragma unroll
-    for (int g = 0; g < NG; ++g) {
-        const int col = 64 * g + 8 * gid;
+    for (int gg = 0; gg < NGW; ++gg) {
+        const int col = 64 * (g0 + gg) + 8 * gid;
         uint4 xa = *reinterpret_cast<const uint4 *>(v + ta * D + col);
         uint4 xb = *reinterpret_cast<const uint4 *>(v + tb * D + col);
         uint4 xc = *reinterpret_cast<const uint4 *>(v + tc * D + col);
@@ -593,24 +617,93 @@ __device__ __forceinline__ void window_pv(WarpState<NG> &st, const uint8_t *blk,
         for (int t = 0; t < 4; ++t) {
             const uint32_t a0 = prmt(wa[t], wb[t], 0x5410u), a1 = prmt(wa[t], wb[t], 0x7632u);
             const uint32_t a2 = prmt(wc[t], wd[t], 0x5410u), a3 = prmt(wc[t], wd[t], 0x7632u);
-            mma_bf16_16816(st.o[g][t], a0, a1, a2, a3, bh0, bh1);
-            mma_bf16_16816(st.o[g][t], a0, a1, a2, a3, bl0, bl1);
+            float acc[4] = {0.f, 0.f, 0.f, 0.f};
+            mma_bf16_16816(acc, a0, a1, a2, a3, bh0, bh1);
+            mma_bf16_16816(acc, a0, a1, a2, a3, bl0, bl1);
+            add_block(st.o[gg][t], acc);
         }
     }
+}
+
+// Named barrier 1 + team for the two warps (64 threads) of a team, with the
+// id as an immediate.
+__device__ __forceinline__ void team_bar(int team) {
+    if (team == 0) asm volatile("bar.sync 1, 64;\n" ::: "memory");
+    else asm volatile("bar.sync 2, 64;\n" ::: "memory");
+}
+
+// Two warps of a team hold halves of head_dim: each has summed the QK terms
+// of its groups; this adds the partner's (addition commutes, so both warps
+// hold the same sums) and ANDs the two warps' copy-wait results.  xb: the
+// team's exchange area, [2 parities][2 halves][32 lanes][8 floats] then
+// [2 parities][2 halves] flags; alternating parities keep a write from racing
+// the partner's read of the block before.  `bar` is the team's named barrier.
+template <int R>
+__device__ __forceinline__ bool team_add(float (&l)[R][2], float *xb, int parity, int half, int lane, int bar,
+                                         bool ok) {
+    static_assert(R == 2 || R == 4, "rows");
+    float4 *mine = reinterpret_cast<float4 *>(xb + ((parity * 2 + half) * 32 + lane) * 8);
+    const float4 *theirs = reinterpret_cast<const float4 *>(xb + ((parity * 2 + (half ^ 1)) * 32 + lane) * 8);
+    int *flags = reinterpret_cast<int *>(xb + 2 * 2 * 32 * 8);
+    mine[0] = make_float4(l[0][0], l[0][1], l[1][0], l[1][1]);
+    if (R == 4) mine[1] = make_float4(l[R - 2][0], l[R - 2][1], l[R - 1][0], l[R - 1][1]);
+    if (lane == 0) flags[parity * 2 + half] = ok ? 1 : 0;
+    team_bar(bar - 1);
+    const float4 a = theirs[0];
+    l[0][0] += a.x;
+    l[0][1] += a.y;
+    l[1][0] += a.z;
+    l[1][1] += a.w;
+    if (R == 4) {
+        const float4 b = theirs[1];
+        l[R - 2][0] += b.x;
+        l[R - 2][1] += b.y;
+        l[R - 1][0] += b.z;
+        l[R - 1][1] += b.w;
+    }
+    return ok && flags[parity * 2 + (half ^ 1)] != 0;
+}
+
+// The two warps' copy-wait results ANDed at the team barrier (flags after
+// team_add's, same parity scheme).
+__device__ __forceinline__ bool team_and(bool ok, float *xb, int parity, int half, int lane, int bar) {
+    int *flags = reinterpret_cast<int *>(xb + 2 * 2 * 32 * 8) + 4;
+    if (lane == 0) flags[parity * 2 + half] = ok ? 1 : 0;
+    team_bar(bar - 1);
+    return ok && flags[parity * 2 + (half ^ 1)] != 0;
 }
 
 // ---------------------------------------------------------------- kernel ---
 
 __device__ __forceinline__ uint32_t round16(uint32_t x) { return (x + 15u) & ~15u; }
 
+// Warps per team: a team streams one sequence of steps through one ring and
+// its warps split head_dim (head_dim 256: two warps of 128 each, so that a
+// warp's accumulators and q operands stay within 128 registers).
+template <int NG>
+__host__ __device__ constexpr int attn_team_warps() {
+    return NG == 4 ? 2 : 1;
+}
+
 template <int NG>
 __host__ __device__ constexpr int attn_ctas_per_sm() {
-    return NG <= 2 ? 4 : (NG == 3 ? 3 : 2);
+    return NG == 3 ? 3 : 4;
+}
+
+// per team: [2 parities][2 halves][32 lanes][8 floats] of QK sums, then two
+// sets of [2 parities][2 halves] flags
+constexpr int kXchgFloats = 2 * 2 * 32 * 8 + 8;
+
+template <int NG>
+__host__ __device__ constexpr int attn_xchg_offset() {
+    return (8 * 64 * NG * 2 + kAttnWarps * kMaxStages * 8 + 16 + 15) & ~15;
 }
 
 template <int NG>
 __host__ __device__ constexpr int attn_header_bytes() {
-    return (8 * 64 * NG * 2 + kAttnWarps * kMaxStages * 8 + 16 + 127) & ~127;
+    return (attn_xchg_offset<NG>() +
+            (attn_team_warps<NG>() > 1 ? kAttnWarps / attn_team_warps<NG>() * kXchgFloats * 4 : 0) + 127) &
+           ~127;
 }
 
 // Split-K combine of one unit (sequence, KV head, head block) whose n > 1
@@ -731,13 +824,18 @@ __device__ __forceinline__ void combine_unit(const AttnParams &p, const AttnView
 }
 
 // One work item: (view, KV head hk, query-head block z, chunk of tokens).
-// The chunk is cut into steps (32 packed tokens, or 16 window tokens); warp w
-// takes steps w, w+4, ...  A packed step is one block holding both halves of
-// two 16-token tiles (K codes, V codes, K scale/min, V scale/min); a window
-// step is two blocks (K rows, then V rows).  Blocks stream through the warp's
-// own ring of S equal slots, each with an mbarrier that counts the bytes of
-// the block's bulk copies; one lane issues the copies and a slot is refilled
-// as soon as the warp has consumed it.
+// The chunk is cut into steps (32 packed tokens, or 16 window tokens).  The
+// CTA's warps form T = 4 / TW teams of TW warps; team t takes steps t, t+T,
+// ...  A packed step is one block holding both halves of two 16-token tiles
+// (K codes, V codes, K scale/min, V scale/min); a window step is two blocks
+// (K rows, then V rows).  Blocks stream through the team's own ring of S
+// equal slots, each with an mbarrier that counts the bytes of the block's
+// bulk copies; lane 0 of the team's first warp issues them.  With TW = 1 a
+// slot is refilled as soon as the warp has consumed it.  With TW = 2 the two
+// warps split the head's groups: each computes the QK sums of its groups,
+// they add each other's through shared memory at a named barrier (team_add),
+// both run the same softmax, and each does the PV of its groups; a slot is
+// refilled at that barrier, once both warps are past the block it held.
 // SCORE: the packed part's K rows only (no V copies, no softmax, no PV): each
 // token's largest logit over the CTA's query heads (base-2 units, scale_log2
 // applied) goes to p.scores; no partials, no combine.
@@ -746,6 +844,9 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
                                           uint8_t *smem) {
     constexpr int D = 64 * NG;
     constexpr int RB = 8 * B * NG;
+    constexpr int TW = attn_team_warps<NG>();
+    constexpr int T = kAttnWarps / TW;    // teams per CTA
+    constexpr int NGW = NG / TW;          // groups per warp
     constexpr int kStepTok = WINDOW ? kTile : 2 * kTile;
     constexpr int kBlkPerStep = WINDOW ? 2 : 1;
     // packed block: [K codes 32*RB][V codes 32*RB][K sm 32*NG*8][V sm 32*NG*8]
@@ -757,6 +858,8 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
 
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int gid = lane >> 2, tig = lane & 3;
+    const int team = warp / TW, half = warp % TW, g0 = half * NGW;
+    float *xb = reinterpret_cast<float *>(smem + attn_xchg_offset<NG>()) + team * kXchgFloats;
     const int h0 = hk * p.group + z * kHeadsPerCta;
     const int nh = min(kHeadsPerCta, p.group - z * kHeadsPerCta);
     // this chunk's steps: the part's steps split into equal runs (+-1 step)
@@ -769,21 +872,22 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     const int64_t tok0 = (int64_t)s0 * kStepTok;
     const int n_tok = (int)min((int64_t)(s1 - s0) * kStepTok, (int64_t)n_part - tok0);
     const int n_steps = s1 - s0;
-    const int n_my = (warp < n_steps) ? (n_steps - warp + kAttnWarps - 1) / kAttnWarps : 0;
+    const int n_my = (team < n_steps) ? (n_steps - team + T - 1) / T : 0;
     const int n_blocks = kBlkPerStep * n_my;
-    const int S = min(kMaxStages, (int)(p.ring_bytes / kBlk));
-    uint8_t *ring = rings + (size_t)warp * p.ring_bytes;
-    uint64_t *wbar = bars + warp * kMaxStages;
-    constexpr int kAdvTok = kAttnWarps * kStepTok;  // tokens between a warp's steps
+    const int team_ring = TW * p.ring_bytes;
+    const int S = min(kMaxStages, (int)(team_ring / kBlk));
+    uint8_t *ring = rings + (size_t)team * team_ring;
+    uint64_t *wbar = bars + team * kMaxStages;
+    constexpr int kAdvTok = T * kStepTok;  // tokens between a team's steps
 
-    // Copy sources at this warp's first step; incremental from then on (no
+    // Copy sources at this team's first step; incremental from then on (no
     // integer division on the per-block path).
     const uint8_t *src_kc = nullptr, *src_vc = nullptr;
     const float *src_ks = nullptr, *src_vs = nullptr;
     const uint16_t *win_k = nullptr, *win_v = nullptr;
     int win_phys = 0;
     if (!WINDOW) {
-        const int64_t row = (int64_t)hk * V.cap_packed + tok0 + kStepTok * warp;
+        const int64_t row = (int64_t)hk * V.cap_packed + tok0 + kStepTok * team;
         src_kc = V.codes[0] + row * RB;
         src_vc = V.codes[1] + row * RB;
         src_ks = V.scalemin[0] + row * NG * 2;
@@ -791,13 +895,14 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     } else {
         win_k = V.window[0] + (int64_t)hk * V.cap_window * D;
         win_v = V.window[1] + (int64_t)hk * V.cap_window * D;
-        win_phys = V.cap_window > 0 ? (int)(((int64_t)V.window_head + tok0 + kStepTok * warp) % V.cap_window) : 0;
+        win_phys = V.cap_window > 0 ? (int)(((int64_t)V.window_head + tok0 + kStepTok * team) % V.cap_window) : 0;
     }
-    // Copy issue: every lane keeps the (warp-uniform) bookkeeping and runs
-    // issue_next; only lane 0's async instructions are predicated on.
-    const bool issuer = lane == 0;
-    int issue_blk = 0, issue_slot = 0, issue_left = n_tok - kStepTok * warp;
-    int issue_step = s0 + warp;  // step index within the part
+    // Copy issue: every lane of the team's first warp keeps the (warp-uniform)
+    // bookkeeping and runs issue_next; only its lane 0's async instructions are
+    // predicated on.
+    const bool issuer = lane == 0 && half == 0;
+    int issue_blk = 0, issue_slot = 0, issue_left = n_tok - kStepTok * team;
+    int issue_step = s0 + team;  // step index within the part
     const int dep_step = p.fused ? V.dep_step[WINDOW ? 1 : 0] : -1;
     auto issue_next = [&]() {
         // the block the preceding append grid writes: wait for that grid first
@@ -805,7 +910,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         uint8_t *dst = ring + (size_t)issue_slot * kBlk;
         uint64_t *bar = &wbar[issue_slot];
         const int n = min(kStepTok, issue_left);
-        const bool stage_ok = dcheck((size_t)(issue_slot + 1) * kBlk <= (size_t)p.ring_bytes, kDbgAttnStage);
+        const bool stage_ok = dcheck((size_t)(issue_slot + 1) * kBlk <= (size_t)team_ring, kDbgAttnStage);
         if (!WINDOW) {
             const bool full = n == kStepTok;
             const uint32_t bc = full ? (uint32_t)(kStepTok * RB) : round16((uint32_t)(n * RB));
@@ -830,7 +935,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             src_ks += (int64_t)kAdvTok * NG * 2;
             src_vs += (int64_t)kAdvTok * NG * 2;
             issue_left -= kAdvTok;
-            issue_step += kAttnWarps;
+            issue_step += T;
         } else {
             const int kv = issue_blk & 1;
             const uint16_t *base = kv ? win_v : win_k;
@@ -844,7 +949,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             if (kv == 1) {
                 win_phys = (win_phys + kAdvTok) % V.cap_window;
                 issue_left -= kAdvTok;
-                issue_step += kAttnWarps;
+                issue_step += T;
             }
         }
         ++issue_blk;
@@ -859,12 +964,14 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     // flight while that grid drains.
     const int n_pro = min(S, n_blocks);
     if (!p.chain && !p.prefetch) pdl_wait();
-    if (lane == 0) {
-        for (int s = 0; s < S; ++s) mbar_init(&wbar[s], 1);
-        fence_mbar_init();
+    if (half == 0) {
+        if (lane == 0) {
+            for (int s = 0; s < S; ++s) mbar_init(&wbar[s], 1);
+            fence_mbar_init();
+        }
+        __syncwarp();
+        for (int b = 0; b < n_pro; ++b) issue_next();
     }
-    __syncwarp();
-    for (int b = 0; b < n_pro; ++b) issue_next();
     if (!p.chain) {
         pdl_wait();
         pdl_launch_dependents();  // the next grid may be scheduled as slots free up (it waits in turn)
@@ -876,35 +983,36 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             val = __ldcg(reinterpret_cast<const uint4 *>(p.q + ((int64_t)V.seq_index * p.n_q_heads + h0 + j) * D) + d8);
         reinterpret_cast<uint4 *>(q_s)[i] = val;
     }
-    __syncthreads();
+    __syncthreads();  // also publishes the barriers' initialization to the team's other warp
 
-    WarpState<NG> st;
+    WarpState<NGW> st;
     // base-2 logits per unit of the QK accumulators (window items: bf16 q
     // as it is; packed items: the factor q was scaled by, see below)
     float qk_scale = p.scale_log2;
     {
-        // q as B operand (column n = gid), k-slots from the unpack map; the
-        // per-group sums of q come from the same values: each lane adds its
-        // 16 elements, lanes of one gid combine, then lanes fetch the sums of
-        // heads 2tig, 2tig+1.
+        // q as B operand (column n = gid) for the warp's groups, k-slots from
+        // the unpack map; the per-group sums of q come from the same values:
+        // each lane adds its 16 elements, lanes of one gid combine, then lanes
+        // fetch the sums of heads 2tig, 2tig+1.
         const uint16_t *qr = q_s + gid * D;
         auto qf = [&](int g, int k) { return __uint_as_float((uint32_t)qr[64 * g + 16 * tig + k] << 16); };
         // packed items: q * 2^(14 - off - eq) in fp16, with 2^eq > max|q| over
-        // the CTA's heads (every warp sees all of them), so that |B| < 2^14
-        // and the products with the codes' 2^(off - 24) carry 2^(-10 - eq)
+        // the CTA's heads and this warp's groups, so that |B| < 2^14 and the
+        // products with the codes' 2^(off - 24) carry 2^(-10 - eq)
         int eq = 0;
         if (!WINDOW) {
             float mx = 0.f;
 #pragma unroll
-            for (int g = 0; g < NG; ++g)
+            for (int gg = 0; gg < NGW; ++gg)
 #pragma unroll
-                for (int k = 0; k < 16; ++k) mx = fmaxf(mx, fabsf(qf(g, k)));
+                for (int k = 0; k < 16; ++k) mx = fmaxf(mx, fabsf(qf(g0 + gg, k)));
             const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, __float_as_uint(mx));
             eq = wm == 0u ? 0 : max(-100, min(110, (int)(wm >> 23) - 126));
             qk_scale = p.scale_log2 * __uint_as_float((uint32_t)(127 + 10 + eq) << 23);
         }
 #pragma unroll
-        for (int g = 0; g < NG; ++g) {
+        for (int gg = 0; gg < NGW; ++gg) {
+            const int g = g0 + gg;
             float part = 0.f;
 #pragma unroll
             for (int s = 0; s < 4; ++s)
@@ -914,31 +1022,34 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
                     const float q0 = qf(g, WINDOW ? 2 * r : qk_code<B>(r, 0));
                     const float q1 = qf(g, WINDOW ? 2 * r + 1 : qk_code<B>(r, 1));
                     if (WINDOW) {
-                        st.bq[g][s][j] = pack_bf16x2(q0, q1);
+                        st.bq[gg][s][j] = pack_bf16x2(q0, q1);
                     } else {
                         // exact: a power-of-two scaling of a bf16 value (fp16 normal range)
                         const float c0 = __uint_as_float((uint32_t)(127 + 14 - qk_off<B>(r, 0) - eq) << 23);
                         const float c1 = __uint_as_float((uint32_t)(127 + 14 - qk_off<B>(r, 1) - eq) << 23);
-                        st.bq[g][s][j] = pack_f16x2(q0 * c0, q1 * c1);
+                        st.bq[gg][s][j] = pack_f16x2(q0 * c0, q1 * c1);
                     }
                     part += q0 + q1;
                 }
             part += __shfl_xor_sync(0xFFFFFFFFu, part, 1);
             part += __shfl_xor_sync(0xFFFFFFFFu, part, 2);
             const float qs = WINDOW ? 1.f : __uint_as_float((uint32_t)(127 - 10 - eq) << 23);
-            st.qsum[g][0] = qs * __shfl_sync(0xFFFFFFFFu, part, 4 * (2 * tig));
-            st.qsum[g][1] = qs * __shfl_sync(0xFFFFFFFFu, part, 4 * (2 * tig + 1));
+            st.qsum[gg][0] = qs * __shfl_sync(0xFFFFFFFFu, part, 4 * (2 * tig));
+            st.qsum[gg][1] = qs * __shfl_sync(0xFFFFFFFFu, part, 4 * (2 * tig + 1));
 #pragma unroll
             for (int t = 0; t < 4; ++t)
 #pragma unroll
-                for (int e = 0; e < 4; ++e) st.o[g][t][e] = 0.f;
-            st.mt[g][0] = st.mt[g][1] = 0.f;
+                for (int e = 0; e < 4; ++e) st.o[gg][t][e] = 0.f;
+            st.mt[gg][0] = st.mt[gg][1] = 0.f;
         }
         st.m[0] = st.m[1] = -INFINITY;
         st.l[0] = st.l[1] = 0.f;
         st.pscale = 1.f;
         st.plimit = 0.f;  // the first packed block sets pscale
     }
+    // the two warps of a team use different logit scales (eq) only inside
+    // their QK sums; those are added in logit units
+    float team_scale = qk_scale;
 
     // consumer position: the current block is in slot `slot`, phase `phase`
     int slot = 0;
@@ -950,12 +1061,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         if (__all_sync(0xFFFFFFFFu, mbar_try_wait(&wbar[slot], phase))) return true;
         return __all_sync(0xFFFFFFFFu, mbar_wait_bounded(&wbar[slot], phase, p.timeout_ns));
     };
-    auto release_cur = [&]() {
-        __syncwarp();
-        if (consumed + S < n_blocks) {  // warp-uniform
-            fence_proxy_async_shared();
-            issue_next();
-        }
+    auto advance_cur = [&]() {
         ++consumed;
         if (++slot == S) {
             slot = 0;
@@ -965,89 +1071,140 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             stage += kBlk;
         }
     };
+    // TW = 1: a consumed slot is refilled at once
+    auto release_cur = [&]() {
+        if (TW == 1) {
+            __syncwarp();
+            if (consumed + S < n_blocks) {  // warp-uniform
+                fence_proxy_async_shared();
+                issue_next();
+            }
+        }
+        advance_cur();
+    };
+    // TW = 2, at the team barrier: blocks [0, both) are done in both warps
+    auto refill_team = [&](int both) {
+        if (TW == 2 && half == 0) {
+            bool fenced = false;
+            while (issue_blk < n_blocks && issue_blk < both + S) {
+                if (!fenced) {
+                    fence_proxy_async_shared();
+                    fenced = true;
+                }
+                issue_next();
+            }
+        }
+    };
+    // QK sums of the warp's groups -> logits of the team's heads: the
+    // partner's groups added (TW = 2), scale, rows past `valid` masked
+    auto finish_qk = [&](auto &l, int i, bool ok, int valid) -> bool {
+        constexpr int R = sizeof(l) / sizeof(l[0]);
+        if constexpr (TW == 2) {
+            // the partner's sums carry its own eq: bring them to logit units first
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                l[r][0] *= team_scale;
+                l[r][1] *= team_scale;
+            }
+            ok = team_add<R>(l, xb, i & 1, half, lane, 1 + team, ok);
+        } else {
+#pragma unroll
+            for (int r = 0; r < R; ++r) {
+                l[r][0] *= team_scale;
+                l[r][1] *= team_scale;
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < R; ++r) {
+            const int row = (r >> 1) * kTile + gid + (r & 1) * 8;
+            if (row >= valid) l[r][0] = l[r][1] = -INFINITY;
+        }
+        return ok;
+    };
 
     // ---- main loop
     bool failed = false;
-    int left = n_tok - kStepTok * warp;
+    int left = n_tok - kStepTok * team;
     for (int i = 0; i < n_my; ++i, left -= kAdvTok) {
-        if (!wait_cur()) { failed = true; break; }
-        if constexpr (SCORE && !WINDOW) {
+        const bool ok = wait_cur();
+        if (TW == 1 && !ok) { failed = true; break; }
+        // TW = 2: a failed wait still takes part in the team barrier below,
+        // so that both warps leave the loop together
+        if constexpr (!WINDOW) {
             float lg[4][2];
             if (left >= kStepTok) {
-                packed_qk2<B, NG>(st, stage, qk_scale, gid, tig, lg);
+                packed_qk_block<B, NG, NGW>(st, stage, gid, tig, g0, lg);
             } else {
-                packed_qk1<B, NG>(st, stage, stage + kOffKs, min(left, kTile), qk_scale, gid, tig, lg[0], lg[1]);
+                float a[2][2], b[2][2] = {{0.f, 0.f}, {0.f, 0.f}};
+                packed_qk_tile<B, NG, NGW>(st, stage, stage + kOffKs, gid, tig, g0, a);
                 if (left > kTile)
-                    packed_qk1<B, NG>(st, stage + kTile * RB, stage + kOffKs + kTile * NG * 8, left - kTile,
-                                      qk_scale, gid, tig, lg[2], lg[3]);
+                    packed_qk_tile<B, NG, NGW>(st, stage + kTile * RB, stage + kOffKs + kTile * NG * 8, gid, tig, g0,
+                                               b);
+                lg[0][0] = a[0][0]; lg[0][1] = a[0][1]; lg[1][0] = a[1][0]; lg[1][1] = a[1][1];
+                lg[2][0] = b[0][0]; lg[2][1] = b[0][1]; lg[3][0] = b[1][0]; lg[3][1] = b[1][1];
             }
-            release_cur();
-            // largest logit over the CTA's heads (2 per lane, 8 per quad)
-            const int64_t dst_i = V.score_off + (int64_t)hk * V.n_packed + tok0 + (int64_t)kStepTok * (warp + i * kAttnWarps);
-            float *dst = p.scores + dst_i;
+            if (!finish_qk(lg, i, ok, min(left, kStepTok))) { failed = true; break; }
+            refill_team(i);  // TW = 2: the blocks before this one are done in both warps
+            if constexpr (SCORE) {
+                release_cur();
+                // largest logit over the CTA's heads (2 per lane, 8 per quad)
+                const int64_t dst_i = V.score_off + (int64_t)hk * V.n_packed + tok0 + (int64_t)kStepTok * (team + i * T);
+                float *dst = p.scores + dst_i;
 #pragma unroll
-            for (int r = 0; r < 4; ++r) {
-                float m = fmaxf(2 * tig < nh ? lg[r][0] : -INFINITY, 2 * tig + 1 < nh ? lg[r][1] : -INFINITY);
-                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-                m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-                const int row = (r >> 1) * kTile + gid + (r & 1) * 8;
-                if (tig == 0 && row < left && dcheck(dst_i + row >= 0 && dst_i + row < p.n_scores, kDbgAttnIo))
-                    dst[row] = m;
+                for (int r = 0; r < 4; ++r) {
+                    float m = fmaxf(2 * tig < nh ? lg[r][0] : -INFINITY, 2 * tig + 1 < nh ? lg[r][1] : -INFINITY);
+                    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                    m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                    const int row = (r >> 1) * kTile + gid + (r & 1) * 8;
+                    if (half == 0 && tig == 0 && row < left &&
+                        dcheck(dst_i + row >= 0 && dst_i + row < p.n_scores, kDbgAttnIo))
+                        dst[row] = m;
+                }
+                continue;
             }
-            continue;
-        }
-        if constexpr (!WINDOW) {
+            softmax_step_n<NGW, 4>(st, lg);
             if (left >= kStepTok) {
                 // two full 16-token tiles, one softmax update over 32 tokens
-                float lg[4][2];
-                packed_qk2<B, NG>(st, stage, qk_scale, gid, tig, lg);
-                softmax_step_n<NG, 4>(st, lg);
-                track_pscale<NG>(st, stage + kOffVs, 2 * kTile, gid);
-                packed_pv<B, NG, true>(st, stage + kOffV, stage + kOffVs, 0, lg[0], lg[1], gid, tig);
-                packed_pv<B, NG, true>(st, stage + kOffV + kTile * RB, stage + kOffVs + kTile * NG * 8, 0, lg[2],
-                                       lg[3], gid, tig);
+                track_pscale<NG, NGW>(st, stage + kOffVs, 2 * kTile, gid, g0);
+                packed_pv_block<B, NG, NGW, true>(st, stage + kOffV, stage + kOffVs, 2 * kTile, lg, gid, tig, g0);
             } else {
                 // the chunk's ragged end: one or two partial tiles
-                float lg[4][2];
-                packed_qk1<B, NG>(st, stage, stage + kOffKs, min(left, kTile), qk_scale, gid, tig, lg[0], lg[1]);
-                if (left > kTile)
-                    packed_qk1<B, NG>(st, stage + kTile * RB, stage + kOffKs + kTile * NG * 8, left - kTile,
-                                      qk_scale, gid, tig, lg[2], lg[3]);
-                else
-                    lg[2][0] = lg[2][1] = lg[3][0] = lg[3][1] = -INFINITY;
-                softmax_step_n<NG, 4>(st, lg);
-                track_pscale<NG>(st, stage + kOffVs, min(left, 2 * kTile), gid);  // the block's valid rows
-                packed_pv<B, NG, false>(st, stage + kOffV, stage + kOffVs, min(left, kTile), lg[0], lg[1], gid, tig);
-                if (left > kTile)
-                    packed_pv<B, NG, false>(st, stage + kOffV + kTile * RB, stage + kOffVs + kTile * NG * 8,
-                                            left - kTile, lg[2], lg[3], gid, tig);
+                const int n_valid = min(left, 2 * kTile);
+                track_pscale<NG, NGW>(st, stage + kOffVs, n_valid, gid, g0);  // the block's valid rows
+                packed_pv_block<B, NG, NGW, false>(st, stage + kOffV, stage + kOffVs, n_valid, lg, gid, tig, g0);
             }
             release_cur();
         } else {
             const int n_valid = min(kTile, left);
             float lg[2][2];
-            if (n_valid == kTile) window_qk<NG, true>(st, stage, n_valid, qk_scale, gid, tig, lg);
-            else window_qk<NG, false>(st, stage, n_valid, qk_scale, gid, tig, lg);
+            window_qk<NG, NGW>(st, stage, gid, tig, g0, lg);
+            if (!finish_qk(lg, i, ok, n_valid)) { failed = true; break; }
             release_cur();
-            softmax_step_n<NG, 2>(st, lg);
-            if (!wait_cur()) { failed = true; break; }
-            if (n_valid == kTile) window_pv<NG, true>(st, stage, n_valid, lg, gid, tig);
-            else window_pv<NG, false>(st, stage, n_valid, lg, gid, tig);
+            refill_team(2 * i + 1);  // TW = 2: up to this step's K block, done in both warps
+            softmax_step_n<NGW, 2>(st, lg);
+            bool vok = wait_cur();
+            if constexpr (TW == 2) vok = team_and(vok, xb, i & 1, half, lane, 1 + team);
+            if (!vok) { failed = true; break; }
+            if (n_valid == kTile) window_pv<NG, NGW, true>(st, stage, n_valid, lg, gid, tig, g0);
+            else window_pv<NG, NGW, false>(st, stage, n_valid, lg, gid, tig, g0);
             release_cur();
         }
     }
     if (failed) {
-        // let every copy this warp issued land before the CTA can exit
-        const int issued = __shfl_sync(0xFFFFFFFFu, issue_blk, 0);
-        for (; consumed < issued; ++consumed) {
-            (void)__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&wbar[slot], phase, p.timeout_ns));
-            if (++slot == S) { slot = 0; phase ^= 1u; }
+        // let every copy this team issued land before the CTA can exit
+        if (half == 0) {
+            const int issued = __shfl_sync(0xFFFFFFFFu, issue_blk, 0);
+            for (; consumed < issued; ++consumed) {
+                (void)__all_sync(0xFFFFFFFFu, mbar_wait_bounded(&wbar[slot], phase, p.timeout_ns));
+                if (++slot == S) { slot = 0; phase ^= 1u; }
+            }
         }
         if (lane == 0) atomicExch(p.status, 1u);
     }
     if constexpr (SCORE) return;
 
-    // ---- warp partial -> this warp's ring area (all its copies have landed)
+    // ---- team partial -> the team's ring area (all its copies have landed):
+    // m and l from the team's first warp, each warp's groups of O
 #pragma unroll
     for (int j = 0; j < 2; ++j) {
         float l = st.l[j];
@@ -1056,7 +1213,7 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         l += __shfl_xor_sync(0xFFFFFFFFu, l, 16);
         st.l[j] = l;
 #pragma unroll
-        for (int g = 0; g < NG; ++g) {
+        for (int g = 0; g < NGW; ++g) {
             float m = st.mt[g][j];
             m += __shfl_xor_sync(0xFFFFFFFFu, m, 4);
             m += __shfl_xor_sync(0xFFFFFFFFu, m, 8);
@@ -1064,9 +1221,10 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
             st.mt[g][j] = m;
         }
     }
+    if (TW == 2) team_bar(team);  // both warps past the ring
     __syncwarp();
     float *wpart = reinterpret_cast<float *>(ring);  // m[8], l[8], o[8][D]
-    if (gid == 0) {
+    if (gid == 0 && half == 0) {
         wpart[2 * tig] = st.m[0];
         wpart[2 * tig + 1] = st.m[1];
         wpart[8 + 2 * tig] = st.l[0];
@@ -1076,20 +1234,20 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     // packed items: O row d accumulated 2^(pv_off - 24) * pscale times its value
     const float inv_ps = 1.f / st.pscale;  // a power of two: exact
 #pragma unroll
-    for (int g = 0; g < NG; ++g)
+    for (int gg = 0; gg < NGW; ++gg)
 #pragma unroll
         for (int t = 0; t < 4; ++t) {
-            const int d0 = 64 * g + 8 * gid + 2 * t;
+            const int d0 = 64 * (g0 + gg) + 8 * gid + 2 * t;
             const float fe = WINDOW ? 1.f : inv_ps * __uint_as_float((uint32_t)(127 + 24 - pv_off<B>(t, 0)) << 23);
             const float fo = WINDOW ? 1.f : inv_ps * __uint_as_float((uint32_t)(127 + 24 - pv_off<B>(t, 1)) << 23);
             *reinterpret_cast<float2 *>(&wo[(2 * tig) * D + d0]) =
-                make_float2(fmaf(st.o[g][t][0], fe, st.mt[g][0]), fmaf(st.o[g][t][2], fo, st.mt[g][0]));
+                make_float2(fmaf(st.o[gg][t][0], fe, st.mt[gg][0]), fmaf(st.o[gg][t][2], fo, st.mt[gg][0]));
             *reinterpret_cast<float2 *>(&wo[(2 * tig + 1) * D + d0]) =
-                make_float2(fmaf(st.o[g][t][1], fe, st.mt[g][1]), fmaf(st.o[g][t][3], fo, st.mt[g][1]));
+                make_float2(fmaf(st.o[gg][t][1], fe, st.mt[gg][1]), fmaf(st.o[gg][t][3], fo, st.mt[gg][1]));
         }
     __syncthreads();
 
-    // ---- merge the 4 warps (fixed order)
+    // ---- merge the T teams (fixed order)
     const bool single = V.seq_chunks == 1;
     const int64_t pslot = ((int64_t)(V.part_begin + c) * p.n_kv_heads + hk) * p.head_blocks + z;
     float *part = p.partials + pslot * (kHeadsPerCta * (D + 2));
@@ -1099,12 +1257,12 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         const int j = idx / D, d = idx - j * D;
         float M = -INFINITY;
 #pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w)
-            M = fmaxf(M, reinterpret_cast<const float *>(rings + (size_t)w * p.ring_bytes)[j]);
+        for (int w = 0; w < T; ++w)
+            M = fmaxf(M, reinterpret_cast<const float *>(rings + (size_t)w * team_ring)[j]);
         float L = 0.f, O = 0.f;
 #pragma unroll
-        for (int w = 0; w < kAttnWarps; ++w) {
-            const float *wp = reinterpret_cast<const float *>(rings + (size_t)w * p.ring_bytes);
+        for (int w = 0; w < T; ++w) {
+            const float *wp = reinterpret_cast<const float *>(rings + (size_t)w * team_ring);
             const float mw = wp[j];
             const float e = (mw == -INFINITY) ? 0.f : fast_exp2(mw - M);
             L = fmaf(e, wp[8 + j], L);
@@ -1146,10 +1304,11 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
 
 // BSEL = 2, 3, 4 or 8: every view of the launch that has packed tokens has
 // that width, and only that width's code is compiled into the kernel (the
-// host groups the views of a call by width, one launch per group).  BSEL = 0:
-// all four widths in one kernel, dispatched per CTA; the host uses it for a
-// call of several widths that fits one launch, saving the separate launches'
-// fill and drain at the cost of instruction-cache reach.
+// host groups the views of a call by width, one launch per group).  With all
+// four widths compiled into one kernel and dispatched per CTA, the Qwen3-32B
+// layer (8 views, up to four widths) took 72 us against 64 us for the
+// per-width launches (more spills, one fetch in five missing the
+// instruction cache).
 template <int NG, int BSEL, bool SCORE = false>
 __device__ __forceinline__ void decode_attn_body(const AttnParams &p, uint8_t *smem) {
     // The first launch of a call waits for the preceding grid inside the
@@ -1171,25 +1330,16 @@ __device__ __forceinline__ void decode_attn_body(const AttnParams &p, uint8_t *s
     if (c >= V.n_chunks) return;  // never launched by the host planner; defensive
     if constexpr (SCORE) {
         if (c < V.n_chunks_packed) attn_item<NG, BSEL, false, true>(p, V, c, hk, z, smem);
-    } else if constexpr (BSEL == 0) {
-        // every width in one grid: the CTA's view picks the code path (the
-        // host orders views by width, so neighbouring CTAs share one)
-        if (c >= V.n_chunks_packed) attn_item<NG, 4, true>(p, V, c, hk, z, smem);
-        else if (V.bits == 2) attn_item<NG, 2, false>(p, V, c, hk, z, smem);
-        else if (V.bits == 3) attn_item<NG, 3, false>(p, V, c, hk, z, smem);
-        else if (V.bits == 4) attn_item<NG, 4, false>(p, V, c, hk, z, smem);
-        else attn_item<NG, 8, false>(p, V, c, hk, z, smem);
     } else {
         if (c >= V.n_chunks_packed) attn_item<NG, 4, true>(p, V, c, hk, z, smem);
         else attn_item<NG, BSEL, false>(p, V, c, hk, z, smem);
     }
 }
 
-// BSEL = 0: views of any width in one launch (see decode_attn_body).
 template <int NG, int BSEL>
 __global__ void __launch_bounds__(kAttnThreads, attn_ctas_per_sm<NG>())
     decode_attn_kernel(const __grid_constant__ AttnParams p) {
-    static_assert(BSEL == 0 || BSEL == 2 || BSEL == 3 || BSEL == 4 || BSEL == 8, "width");
+    static_assert(BSEL == 2 || BSEL == 3 || BSEL == 4 || BSEL == 8, "width");
     extern __shared__ __align__(128) uint8_t smem[];
     decode_attn_body<NG, BSEL>(p, smem);
     // a later launch of a call completes only after the one before it, so

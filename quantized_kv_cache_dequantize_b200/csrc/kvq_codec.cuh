@@ -412,6 +412,11 @@ struct AppendArgs {
 // Grid: (n_views, n_kv_heads, 2 = K/V); one warp per block.  Lanes 0..2*NG-1
 // each own half a group of the row being flushed (same arithmetic as the
 // bulk quantize kernel); all lanes then copy the new token into the ring.
+// In a decode step (early) the loads and the quantization run before the
+// dependency wait: the rows read (the ring's oldest token, the new token) are
+// not written by the grid before, which only reads this layer's cache or
+// none of it, so only the stores wait and the append adds little to the
+// step.  A plain append waits first.
 template <int NG>
 __global__ void __launch_bounds__(32) append_kernel(AppendArgs a) {
     constexpr int D = NG * kGroup;
@@ -420,7 +425,7 @@ __global__ void __launch_bounds__(32) append_kernel(AppendArgs a) {
     // reading them.  Any other grid after a plain append starts when the
     // append has completed.
     if (a.early) pdl_launch_dependents();
-    pdl_wait();  // the rows it reads or overwrites may belong to the preceding grid
+    else pdl_wait();  // the rows it reads or overwrites may belong to the preceding grid
     const AppendView &v = a.views[blockIdx.x];
     const int h = blockIdx.y;
     const int kv = blockIdx.z;
@@ -430,17 +435,21 @@ __global__ void __launch_bounds__(32) append_kernel(AppendArgs a) {
     if (!dcheck((int)blockIdx.x < a.n_views && h < a.n_kv_heads &&
                     (!v.flush || (v.packed_row >= 0 && v.packed_row < v.cap_packed)) &&
                     (v.slot < 0 || v.slot < v.cap_window) && (v.flush || v.slot >= 0),
-                kDbgAppend))
+                kDbgAppend)) {
+        if (a.early) pdl_wait();
         return;
+    }
     const uint16_t *newrow = (kv ? a.v_new : a.k_new) + ((int64_t)blockIdx.x * a.n_kv_heads + h) * D;
     uint16_t *ring = v.window[kv];
     uint16_t *slotrow = (v.slot >= 0) ? ring + ((int64_t)h * v.cap_window + v.slot) * D : nullptr;
 
     // 1) quantize the flushed row: the oldest ring token, or the new token if there is no ring
+    const int g = lane >> 1, half = lane & 1;
+    const bool active = g < NG;
+    uint32_t packed[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+    float s = 0.f, mn = 0.f;
     if (v.flush) {
         const uint16_t *src = (v.cap_window > 0) ? slotrow : newrow;
-        const int g = lane >> 1, half = lane & 1;
-        const bool active = g < NG;
         uint32_t x[16];
         if (active) {
             const uint4 *p = reinterpret_cast<const uint4 *>(src + g * kGroup + half * 32);
@@ -453,35 +462,39 @@ __global__ void __launch_bounds__(32) append_kernel(AppendArgs a) {
 #pragma unroll
             for (int i = 0; i < 16; ++i) x[i] = 0u;
         }
-        float s, mn;
-        uint8_t *codes_row = v.codes[kv] + ((int64_t)h * v.cap_packed + v.packed_row) * (8 * v.bits * NG);
-        float *sm_row = v.scalemin[kv] + ((int64_t)h * v.cap_packed + v.packed_row) * NG * 2;
         switch (v.bits) {
-#define KVQ_APPEND_Q(BB)                                                                         \
-    case BB: {                                                                                   \
-        uint32_t packed[BB];                                                                     \
-        quantize_half_group<BB>(x, src + g * kGroup + half * 32, packed, s, mn);                                               \
-        if (active) {                                                                            \
-            uint32_t *dst = reinterpret_cast<uint32_t *>(codes_row + g * 8 * BB + half * 4 * BB); \
-            _Pragma("unroll") for (int w = 0; w < BB; ++w) dst[w] = packed[w];                    \
-        }                                                                                        \
+#define KVQ_APPEND_Q(BB)                                                          \
+    case BB: {                                                                    \
+        uint32_t pk[BB];                                                          \
+        quantize_half_group<BB>(x, src + g * kGroup + half * 32, pk, s, mn);      \
+        _Pragma("unroll") for (int w = 0; w < BB; ++w) packed[w] = pk[w];         \
     } break;
             KVQ_APPEND_Q(2)
             KVQ_APPEND_Q(3)
             KVQ_APPEND_Q(4)
             KVQ_APPEND_Q(8)
 #undef KVQ_APPEND_Q
-            default: s = 0.f; mn = 0.f; break;
+            default: break;
         }
-        if (active && half == 0) *reinterpret_cast<float2 *>(sm_row + g * 2) = make_float2(s, mn);
     }
-    __syncwarp();
-    // 2) the new token takes its ring slot
-    if (slotrow) {
-        const uint4 *src = reinterpret_cast<const uint4 *>(newrow);
-        uint4 *dst = reinterpret_cast<uint4 *>(slotrow);
-        for (int i = lane; i < D / 8; i += 32) dst[i] = src[i];
+    // 2) the new token, for its ring slot (D/8 <= 32 vectors: one per lane)
+    uint4 nv = make_uint4(0, 0, 0, 0);
+    if (slotrow && lane < D / 8) nv = reinterpret_cast<const uint4 *>(newrow)[lane];
+    __syncwarp();  // every lane has read the ring's oldest token before any lane overwrites it
+
+    if (a.early) pdl_wait();  // the stores: after the preceding grid, which may still read this layer
+    if (v.flush && active) {
+        uint8_t *codes_row = v.codes[kv] + ((int64_t)h * v.cap_packed + v.packed_row) * (8 * v.bits * NG);
+        uint32_t *dst = reinterpret_cast<uint32_t *>(codes_row + g * 8 * v.bits + half * 4 * v.bits);
+#pragma unroll
+        for (int w = 0; w < 8; ++w)
+            if (w < v.bits) dst[w] = packed[w];
+        if (half == 0) {
+            float *sm_row = v.scalemin[kv] + ((int64_t)h * v.cap_packed + v.packed_row) * NG * 2;
+            *reinterpret_cast<float2 *>(sm_row + g * 2) = make_float2(s, mn);
+        }
     }
+    if (slotrow && lane < D / 8) reinterpret_cast<uint4 *>(slotrow)[lane] = nv;
 }
 
 }  // namespace kvq

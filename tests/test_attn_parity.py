@@ -101,6 +101,22 @@ def test_chunking_changes_only_rounding(cuda_device, monkeypatch):
         outs.append(out)
 
 
+@pytest.mark.parametrize("D,bits", [(256, 4), (128, 8), (128, 2), (64, 3)])
+def test_long_single_chunk(cuda_device, monkeypatch, D, bits):
+    """32768 packed tokens forced into ONE chunk, so one warp (or team) sweeps
+    the whole view: the error must not grow with the tokens a warp
+    accumulates.  A PV accumulator chained through every tile's MMA drops low
+    bits at each tile, always downward, and fails here (about 4e-2 relative L2
+    at head_dim 256)."""
+    hq, hkv = (16, 8) if D == 256 else (8, 2)
+    specs = [ViewSpec(32768, 64, 64, bits, head=5, seed=90 + bits, outlier_frac=0.01)]
+    case = build_case(hq, hkv, D, specs, q_seed=14)
+    monkeypatch.setenv("KVQ_CHUNK_TOKENS", "32768")
+    scale = 1 / math.sqrt(D)
+    out = run_gpu(case, scale)
+    assert_close(out[0], oracle_view(case, 0, scale), f"one chunk, D {D}, {bits} bits")
+
+
 def test_bitwise_deterministic(cuda_device):
     specs = [ViewSpec(5000, 128, 128, 4, head=3, seed=60), ViewSpec(777, 100, 128, 3, head=120, seed=61)]
     case = build_case(32, 8, 128, specs, q_seed=12)
