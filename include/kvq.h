@@ -303,8 +303,9 @@ kvq_status kvq_decode_attn_seq(const kvq_view *views, int32_t n_views, const int
  *             256-B aligned, zero-filled before first use; the first bytes
  *             are left ready for the next call with the same views, heads and
  *             top_k, while the sizes of the views change.
- * Scores are fp32; the attention is that of kvq_decode_attn over per-head
- * compact views (the selected rows gathered into the workspace).
+ * Scores are fp32; the attention is that of kvq_decode_attn over one view
+ * per (view, KV head) whose packed part is the selected rows, read in place
+ * through the selection list (in `selected` or the workspace).
  * Errors: as kvq_decode_attn, and KVQ_ERR_INVALID_ARG for top_k < 1.
  */
 size_t kvq_sparse_decode_attn_workspace_size(const kvq_view *views, int32_t n_views,

@@ -466,7 +466,7 @@ template <int NG>
 kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n_q_heads, int32_t n_kv_heads,
                           const void *q, float scale, float *out, uint8_t *ws, cudaStream_t st,
                           const int32_t *dep = nullptr, float *scores = nullptr, const int64_t *score_off = nullptr,
-                          bool prefetch = true, int64_t n_scores = 0) {
+                          bool prefetch = true, int64_t n_scores = 0, const int32_t *const *gather = nullptr) {
     kvq::AttnParams prm;
     std::memset(&prm, 0, sizeof prm);
     prm.n_seqs = (int32_t)plan.seq_chunks.size();
@@ -524,6 +524,7 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
             d.dep_step[0] = prm.fused ? dep[2 * i] : -1;
             d.dep_step[1] = prm.fused ? dep[2 * i + 1] : -1;
             d.score_off = scores ? score_off[i] : 0;
+            d.gather = gather ? gather[i] : nullptr;
             begin += d.n_chunks;
         }
         // The grid carries a programmatic dependency on the preceding work in
@@ -809,33 +810,32 @@ kvq_status noalloc_scratch(void **out) {
 kvq_status launch_attn(const AttnPlan &plan, const kvq_view *views, int32_t n_q_heads, int32_t n_kv_heads,
                        int32_t head_dim, const void *q, float scale, float *out, uint8_t *ws, cudaStream_t st,
                        const int32_t *dep = nullptr, float *scores = nullptr, const int64_t *score_off = nullptr,
-                       bool prefetch = true, int64_t n_scores = 0) {
+                       bool prefetch = true, int64_t n_scores = 0, const int32_t *const *gather = nullptr) {
     switch (head_dim / 64) {
-        case 1: return launch_attn_ng<1>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off, prefetch, n_scores);
-        case 2: return launch_attn_ng<2>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off, prefetch, n_scores);
-        case 3: return launch_attn_ng<3>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off, prefetch, n_scores);
-        default: return launch_attn_ng<4>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off, prefetch, n_scores);
+        case 1: return launch_attn_ng<1>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off, prefetch, n_scores, gather);
+        case 2: return launch_attn_ng<2>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off, prefetch, n_scores, gather);
+        case 3: return launch_attn_ng<3>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off, prefetch, n_scores, gather);
+        default: return launch_attn_ng<4>(plan, views, n_q_heads, n_kv_heads, q, scale, out, ws, st, dep, scores, score_off, prefetch, n_scores, gather);
     }
 }
 
 // ------------------------------------------------------ sparse decode ---
 
-// Top-K sparse decode: every (view, KV head) becomes a compact view of its own
-// (one KV head, the group's query heads): its K selected packed rows, gathered
-// into the workspace (or the view's own rows when it has no more than K), and
-// the view's bf16 window for that head, read in place.  Workspace: the
-// attention's region first (its zero part stays at offset 0 from call to
-// call), then scores, selections and compact rows.
+// Top-K sparse decode: every (view, KV head) becomes a view of its own (one
+// KV head, the group's query heads): its packed part is the K selected rows,
+// read in place through the selection list (gather), or every packed row
+// when the view has no more than K; its window is the view's bf16 window for
+// that head.  Workspace: the attention's region first (its zero part stays
+// at offset 0 from call to call), then scores and selections.
 struct SparsePlan {
-    std::vector<kvq_view> compact;     // [n_views * H_kv]
+    std::vector<kvq_view> compact;     // [n_views * H_kv]: per (view, KV head)
     std::vector<int64_t> score_off;    // per view, floats from scores_off; -1: no scoring
-    std::vector<size_t> rows_off;      // per view, bytes from compact_off (views with n_packed > K)
     AttnPlan attn;
-    size_t scores_off = 0, sel_off = 0, compact_off = 0, total = 0;
+    size_t scores_off = 0, sel_off = 0, total = 0;
 };
 
 kvq_status plan_sparse(const kvq_view *views, int32_t n_views, int32_t n_q_heads, int32_t n_kv_heads,
-                       int32_t head_dim, int32_t top_k, uint8_t *ws, SparsePlan &sp) {
+                       int32_t head_dim, int32_t top_k, SparsePlan &sp) {
     sp = SparsePlan();
     if (!head_dim_supported(head_dim)) return KVQ_ERR_UNSUPPORTED;
     if (n_kv_heads <= 0 || n_q_heads <= 0 || n_q_heads % n_kv_heads || n_kv_heads > 65535)
@@ -844,22 +844,14 @@ kvq_status plan_sparse(const kvq_view *views, int32_t n_views, int32_t n_q_heads
     const kvq_status vs = validate_views(views, n_views, true);
     if (vs != KVQ_OK) return vs;
     const int ng = head_dim / 64, group = n_q_heads / n_kv_heads;
-    const int64_t kc = top_k + (top_k & 1);
     sp.score_off.assign(n_views, -1);
-    sp.rows_off.assign(n_views, 0);
     int64_t n_scores = 0;
-    size_t rows = 0;
     for (int i = 0; i < n_views; ++i) {
         const kvq_view &v = views[i];
         if (v.n_packed <= top_k) continue;
         sp.score_off[i] = n_scores;
         n_scores += (int64_t)n_kv_heads * v.n_packed;
-        sp.rows_off[i] = rows;
-        rows += 2 * align_up((size_t)n_kv_heads * kc * row_bytes(head_dim, v.bits), 256) +
-                2 * align_up((size_t)n_kv_heads * kc * ng * 8, 256);
     }
-    // compact views; gathered rows get their addresses once the layout is known
-    uint8_t *const fake = reinterpret_cast<uint8_t *>(uintptr_t(1) << 20);  // aligned, for planning only
     sp.compact.assign((size_t)n_views * n_kv_heads, kvq_view{});
     for (int i = 0; i < n_views; ++i) {
         const kvq_view &v = views[i];
@@ -875,19 +867,14 @@ kvq_status plan_sparse(const kvq_view *views, int32_t n_views, int32_t n_q_heads
                 c.k_window = static_cast<uint8_t *>(v.k_window) + w;
                 c.v_window = static_cast<uint8_t *>(v.v_window) + w;
             }
+            // the head's own rows, every one or the selected ones
             c.n_packed = std::min<int64_t>(v.n_packed, top_k);
-            if (v.n_packed <= top_k) {  // every packed row: the view's own, in place
-                c.cap_packed = v.cap_packed;
-                if (v.cap_packed > 0) {
-                    c.k_codes = static_cast<uint8_t *>(v.k_codes) + (size_t)hk * v.cap_packed * rb;
-                    c.v_codes = static_cast<uint8_t *>(v.v_codes) + (size_t)hk * v.cap_packed * rb;
-                    c.k_scalemin = v.k_scalemin + (size_t)hk * v.cap_packed * ng * 2;
-                    c.v_scalemin = v.v_scalemin + (size_t)hk * v.cap_packed * ng * 2;
-                }
-            } else {
-                c.cap_packed = kc;
-                c.k_codes = c.v_codes = fake;
-                c.k_scalemin = c.v_scalemin = reinterpret_cast<float *>(fake);
+            c.cap_packed = v.cap_packed;
+            if (v.cap_packed > 0) {
+                c.k_codes = static_cast<uint8_t *>(v.k_codes) + (size_t)hk * v.cap_packed * rb;
+                c.v_codes = static_cast<uint8_t *>(v.v_codes) + (size_t)hk * v.cap_packed * rb;
+                c.k_scalemin = v.k_scalemin + (size_t)hk * v.cap_packed * ng * 2;
+                c.v_scalemin = v.v_scalemin + (size_t)hk * v.cap_packed * ng * 2;
             }
         }
     }
@@ -897,25 +884,7 @@ kvq_status plan_sparse(const kvq_view *views, int32_t n_views, int32_t n_q_heads
     sp.scores_off = off;
     off = align_up(off + (size_t)n_scores * 4, 256);
     sp.sel_off = off;
-    off = align_up(off + (size_t)n_views * n_kv_heads * top_k * 4, 256);
-    sp.compact_off = off;
-    sp.total = off + rows;
-    if (!ws) return KVQ_OK;
-    for (int i = 0; i < n_views; ++i) {
-        const kvq_view &v = views[i];
-        if (v.n_packed <= top_k) continue;
-        const size_t cb = align_up((size_t)n_kv_heads * kc * row_bytes(head_dim, v.bits), 256);
-        const size_t sb = align_up((size_t)n_kv_heads * kc * ng * 8, 256);
-        uint8_t *base = ws + sp.compact_off + sp.rows_off[i];
-        for (int hk = 0; hk < n_kv_heads; ++hk) {
-            kvq_view &c = sp.compact[(size_t)i * n_kv_heads + hk];
-            const size_t h_codes = (size_t)hk * kc * row_bytes(head_dim, v.bits), h_sm = (size_t)hk * kc * ng * 8;
-            c.k_codes = base + h_codes;
-            c.v_codes = base + cb + h_codes;
-            c.k_scalemin = reinterpret_cast<float *>(base + 2 * cb + h_sm);
-            c.v_scalemin = reinterpret_cast<float *>(base + 2 * cb + sb + h_sm);
-        }
-    }
+    sp.total = align_up(off + (size_t)n_views * n_kv_heads * top_k * 4, 256);
     return KVQ_OK;
 }
 
@@ -1038,56 +1007,73 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
         if (es != KVQ_OK) return es;
         v0 = v1;
     }
-    // 2. selections of every view; the views with more than K packed tokens
-    // also copy their selected rows into the compact views
-    for (int v0 = 0; v0 < n_views; v0 += kvq::kSparseMaxViews) {
-        const int v1 = std::min<int>(n_views, v0 + kvq::kSparseMaxViews);
-        kvq::SelectArgs a;
-        std::memset(&a, 0, sizeof a);
-        a.scores = scores;
-        a.sel = sel;
-        a.n_scores = (int64_t)((sp.sel_off - sp.scores_off) / sizeof(float));
-        a.n_sel_rows = n_views;
-        a.top_k = top_k;
-        a.n_kv_heads = n_kv_heads;
-        a.sm_bytes = ng * 8;
-        size_t smem = 0;
-        for (int i = v0; i < v1; ++i) {
-            const kvq_view &v = views[i];
-            kvq::SelectView &d = a.views[i - v0];
-            d.score_off = std::max<int64_t>(sp.score_off[i], 0);
-            d.n_packed = (int32_t)v.n_packed;
-            d.out_row = i;
-            if (sp.score_off[i] < 0) continue;
-            const kvq_view &c0 = sp.compact[(size_t)i * n_kv_heads];  // head 0 of the compact rows
-            d.codes[0] = static_cast<const uint8_t *>(v.k_codes);
-            d.codes[1] = static_cast<const uint8_t *>(v.v_codes);
-            d.sm[0] = v.k_scalemin;
-            d.sm[1] = v.v_scalemin;
-            d.dst_codes[0] = static_cast<uint8_t *>(c0.k_codes);
-            d.dst_codes[1] = static_cast<uint8_t *>(c0.v_codes);
-            d.dst_sm[0] = c0.k_scalemin;
-            d.dst_sm[1] = c0.v_scalemin;
-            d.cap_packed = v.cap_packed;
-            d.cap_compact = c0.cap_packed;
-            d.row_bytes = (int32_t)row_bytes(head_dim, v.bits);
-            d.staged = v.n_packed <= kvq::kSelectStageMax ? 1 : 0;
-            if (d.staged) smem = std::max(smem, (size_t)v.n_packed * 4);
+    // 2. selections of every view (ascending row indices): views of up to
+    // 32768 packed tokens on select_fast_kernel, longer ones on
+    // select_kernel (keys staged in shared memory or read from the scores)
+    for (int large = 0; large < 2; ++large) {
+        std::vector<int> idx;
+        for (int i = 0; i < n_views; ++i)
+            if ((views[i].n_packed > kvq::kSelFastMax) == (large != 0)) idx.push_back(i);
+        for (size_t v0 = 0; v0 < idx.size(); v0 += kvq::kSparseMaxViews) {
+            const size_t v1 = std::min(idx.size(), v0 + kvq::kSparseMaxViews);
+            kvq::SelectArgs a;
+            std::memset(&a, 0, sizeof a);
+            a.scores = scores;
+            a.sel = sel;
+            a.n_scores = (int64_t)((sp.sel_off - sp.scores_off) / sizeof(float));
+            a.n_sel_rows = n_views;
+            a.top_k = top_k;
+            a.n_kv_heads = n_kv_heads;
+            size_t smem = 0;
+            int64_t max_n = 0;
+            for (size_t k = v0; k < v1; ++k) {
+                const int i = idx[k];
+                const kvq_view &v = views[i];
+                kvq::SelectView &d = a.views[k - v0];
+                d.score_off = std::max<int64_t>(sp.score_off[i], 0);
+                d.n_packed = (int32_t)v.n_packed;
+                d.out_row = i;
+                if (sp.score_off[i] < 0) continue;
+                max_n = std::max<int64_t>(max_n, v.n_packed);
+                d.staged = v.n_packed <= kvq::kSelectStageMax ? 1 : 0;
+                if (d.staged) smem = std::max(smem, (size_t)v.n_packed * 4);
+            }
+            const dim3 grid((unsigned)(v1 - v0), (unsigned)n_kv_heads);
+            kvq_status es;
+            if (!large) {
+                const size_t keys = (size_t)max_n * 4;
+                if (keys > 48 * 1024 && cudaFuncSetAttribute(kvq::select_fast_kernel<1024>,
+                                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                             (int)keys) != cudaSuccess) {
+                    (void)cudaGetLastError();
+                    return KVQ_ERR_CUDA;
+                }
+                // (latency-bound: more warps beat fewer keys per warp, also for
+                // short views)
+                es = launch_pdl(kvq::select_fast_kernel<1024>, grid, 1024, keys, st, a);
+            } else {
+                if (smem > 48 * 1024 &&
+                    cudaFuncSetAttribute(kvq::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+                        cudaSuccess) {
+                    (void)cudaGetLastError();
+                    return KVQ_ERR_CUDA;
+                }
+                es = launch_pdl(kvq::select_kernel, grid, kvq::kSelectThreads, smem, st, a);
+            }
+            if (es != KVQ_OK) return es;
         }
-        if (smem > 48 * 1024 && cudaFuncSetAttribute(kvq::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                     (int)smem) != cudaSuccess) {
-            (void)cudaGetLastError();
-            return KVQ_ERR_CUDA;
-        }
-        const kvq_status es = launch_pdl(kvq::select_kernel, dim3((unsigned)(v1 - v0), (unsigned)n_kv_heads),
-                                         kvq::kSelectThreads, smem, st, a);
-        if (es != KVQ_OK) return es;
     }
-    // 4. attention over the compact views: one KV head each, the group's query
-    // heads; the select grid writes the compact rows, so no copy starts
-    // before the dependency wait
+    // 3. attention over the per-head views: one KV head each, the group's
+    // query heads; a view with more than K packed rows reads the selected
+    // ones through its selection list, which the select grid writes, so no
+    // copy starts before the dependency wait
+    std::vector<const int32_t *> gather((size_t)n_views * n_kv_heads, nullptr);
+    for (int i = 0; i < n_views; ++i)
+        if (sp.score_off[i] >= 0)
+            for (int hk = 0; hk < n_kv_heads; ++hk)
+                gather[(size_t)i * n_kv_heads + hk] = sel + ((int64_t)i * n_kv_heads + hk) * top_k;
     return launch_attn(sp.attn, sp.compact.data(), group, 1, head_dim, q, scale, out, ws, st, nullptr, nullptr,
-                       nullptr, false);
+                       nullptr, false, 0, gather.data());
 }
 
 }  // namespace
@@ -1278,7 +1264,7 @@ KVQ_API kvq_status kvq_append_decode_attn(kvq_view *views, int32_t n_views, int3
 KVQ_API size_t kvq_sparse_decode_attn_workspace_size(const kvq_view *views, int32_t n_views, int32_t n_q_heads,
                                                      int32_t n_kv_heads, int32_t head_dim, int32_t top_k) {
     SparsePlan sp;
-    if (plan_sparse(views, n_views, n_q_heads, n_kv_heads, head_dim, top_k, nullptr, sp) != KVQ_OK) return 0;
+    if (plan_sparse(views, n_views, n_q_heads, n_kv_heads, head_dim, top_k, sp) != KVQ_OK) return 0;
     return sp.total;
 }
 
@@ -1287,14 +1273,13 @@ KVQ_API kvq_status kvq_sparse_decode_attn(const kvq_view *views, int32_t n_views
                                           int32_t top_k, float *out, int32_t *selected, void *workspace,
                                           size_t workspace_bytes, void *stream) {
     SparsePlan sp;
-    const kvq_status ps = plan_sparse(views, n_views, n_q_heads, n_kv_heads, head_dim, top_k, nullptr, sp);
+    const kvq_status ps = plan_sparse(views, n_views, n_q_heads, n_kv_heads, head_dim, top_k, sp);
     if (ps != KVQ_OK) return ps;
     if (!q || !out || !workspace) return KVQ_ERR_INVALID_ARG;
     if (!aligned(q, 16) || !aligned(out, 16) || !aligned(workspace, 256)) return KVQ_ERR_INVALID_ARG;
     if (selected && !aligned(selected, 4)) return KVQ_ERR_INVALID_ARG;
     if (workspace_bytes < sp.total) return KVQ_ERR_INVALID_ARG;
     uint8_t *ws = static_cast<uint8_t *>(workspace);
-    plan_sparse(views, n_views, n_q_heads, n_kv_heads, head_dim, top_k, ws, sp);  // now with the row addresses
     int32_t *sel = selected ? selected : reinterpret_cast<int32_t *>(ws + sp.sel_off);
     return launch_sparse(sp, views, n_views, n_q_heads, n_kv_heads, head_dim, q, softmax_scale, top_k, out, sel, ws,
                          static_cast<cudaStream_t>(stream));

@@ -70,6 +70,8 @@ struct AttnView {
                                  // writes (-1: none); with AttnParams::fused its copy waits
                                  // for that grid, every other copy starts at once
     int64_t score_off;           // score grids: float offset of the view's head-0 scores
+    const int32_t *gather;       // packed position j holds row gather[j] of the head's rows
+                                 // (written by the preceding grid); nullptr: row j
 };
 
 struct AttnParams {
@@ -823,6 +825,17 @@ __device__ __forceinline__ void combine_unit(const AttnParams &p, const AttnView
     }
 }
 
+// BYTES (a multiple of 8) from src to dst as cp.async pieces: 16 bytes when
+// BYTES is a multiple of 16, else 8 (both addresses aligned to the piece).
+template <int BYTES>
+__device__ __forceinline__ void cp_async_row(uint8_t *dst, const uint8_t *src) {
+    constexpr int P = BYTES % 16 == 0 ? 16 : 8;
+    // both addresses aligned to the piece (debug build; a refused row is skipped)
+    if (!dcheck((((uintptr_t)dst | (uintptr_t)src) & (P - 1)) == 0, kDbgAttnPacked)) return;
+#pragma unroll
+    for (int i = 0; i < BYTES / P; ++i) cp_async<P>(dst + i * P, src + i * P);
+}
+
 // One work item: (view, KV head hk, query-head block z, chunk of tokens).
 // The chunk is cut into steps (32 packed tokens, or 16 window tokens).  The
 // CTA's warps form T = 4 / TW teams of TW warps; team t takes steps t, t+T,
@@ -903,6 +916,10 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     const bool issuer = lane == 0 && half == 0;
     int issue_blk = 0, issue_slot = 0, issue_left = n_tok - kStepTok * team;
     int issue_step = s0 + team;  // step index within the part
+    // gathered packed rows: position of the next block's first row in the
+    // gather list; lane r of the issuing warp copies row r of a block
+    const int32_t *gather = (WINDOW || SCORE) ? nullptr : V.gather;
+    int64_t issue_pos = tok0 + kStepTok * team;
     const int dep_step = p.fused ? V.dep_step[WINDOW ? 1 : 0] : -1;
     auto issue_next = [&]() {
         // the block the preceding append grid writes: wait for that grid first
@@ -911,7 +928,29 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
         uint64_t *bar = &wbar[issue_slot];
         const int n = min(kStepTok, issue_left);
         const bool stage_ok = dcheck((size_t)(issue_slot + 1) * kBlk <= (size_t)team_ring, kDbgAttnStage);
-        if (!WINDOW) {
+        if (!WINDOW && gather != nullptr) {
+            // K and V codes and scale/min of up to 32 selected rows, one row
+            // per lane; the slot's barrier counts one arrival per lane, made
+            // once that lane's copies have landed (rows past n stay stale
+            // and are masked like a ragged tail)
+            if (stage_ok && lane < n) {
+                const int64_t pos = issue_pos + lane;
+                const int32_t row = dcheck(pos < V.n_packed, kDbgAttnPacked) ? __ldcg(gather + pos) : -1;
+                if (dcheck(row >= 0 && row < V.cap_packed, kDbgAttnPacked)) {
+                    const int64_t r = (int64_t)hk * V.cap_packed + row;
+                    cp_async_row<RB>(dst + lane * RB, V.codes[0] + r * RB);
+                    cp_async_row<RB>(dst + kOffV + lane * RB, V.codes[1] + r * RB);
+                    cp_async_row<NG * 8>(dst + kOffKs + lane * NG * 8,
+                                         reinterpret_cast<const uint8_t *>(V.scalemin[0] + r * NG * 2));
+                    cp_async_row<NG * 8>(dst + kOffVs + lane * NG * 8,
+                                         reinterpret_cast<const uint8_t *>(V.scalemin[1] + r * NG * 2));
+                }
+            }
+            cp_async_mbar_arrive(bar);
+            issue_pos += kAdvTok;
+            issue_left -= kAdvTok;
+            issue_step += T;
+        } else if (!WINDOW) {
             const bool full = n == kStepTok;
             const uint32_t bc = full ? (uint32_t)(kStepTok * RB) : round16((uint32_t)(n * RB));
             const uint32_t bs = full ? (uint32_t)(kStepTok * NG * 8) : round16((uint32_t)(n * NG * 8));
@@ -963,10 +1002,10 @@ __device__ __forceinline__ void attn_item(const AttnParams &p, const AttnView &V
     // wait inside issue_next), so their first ring stages are already in
     // flight while that grid drains.
     const int n_pro = min(S, n_blocks);
-    if (!p.chain && !p.prefetch) pdl_wait();
+    if (!p.chain && (!p.prefetch || gather != nullptr)) pdl_wait();  // a gather list comes from the grid before
     if (half == 0) {
         if (lane == 0) {
-            for (int s = 0; s < S; ++s) mbar_init(&wbar[s], 1);
+            for (int s = 0; s < S; ++s) mbar_init(&wbar[s], gather != nullptr ? 32u : 1u);
             fence_mbar_init();
         }
         __syncwarp();

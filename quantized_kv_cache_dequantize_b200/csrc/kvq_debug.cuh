@@ -24,7 +24,7 @@ enum DebugBit : uint32_t {
     kDbgAppend = 1u << 6,         // append rows or ring slots outside the view
     kDbgCard = 1u << 7,           // card pieces outside the card or the views
     kDbgScore = 1u << 8,          // score kernel rows or scores outside their arrays
-    kDbgSelect = 1u << 9,         // selections or compact rows outside their arrays
+    kDbgSelect = 1u << 9,         // selections or scores outside their arrays
     kDbgSens = 1u << 10,          // sensitivity window rows outside the ring
 };
 

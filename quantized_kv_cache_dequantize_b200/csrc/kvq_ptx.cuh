@@ -163,6 +163,25 @@ __device__ __forceinline__ void bulk_copy_g2s_if(bool issue, void *dst, const vo
         : "memory");
 }
 
+// Per-thread asynchronous copy global -> shared of 8 or 16 bytes (both
+// addresses aligned to the size).  Their completion reaches an mbarrier
+// through cp_async_mbar_arrive.
+template <int BYTES>
+__device__ __forceinline__ void cp_async(void *dst, const void *src) {
+    static_assert(BYTES == 8 || BYTES == 16, "cp.async size");
+    if constexpr (BYTES == 16)
+        asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+    else
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+// One arrival on `bar`, made once every cp.async this thread issued before
+// it has landed.  The arrival is counted in the barrier's initial count
+// (noinc), so a barrier fed this way by n threads is initialised with n.
+__device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {
+    asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(smem_u32(bar)) : "memory");
+}
+
 // Programmatic dependent launch: wait until the preceding grid in the stream
 // has completed and its memory is visible (a no-op when the launch carried no
 // programmatic dependency), and allow the next grid to be scheduled early.

@@ -1,7 +1,7 @@
 // kvq_sparse.cuh -- top-K sparse decode attention over the packed cache:
 // score every packed token against the query group, select the K best per
-// (view, KV head) and gather their rows into a compact per-head view; the
-// attention kernel then runs over the compact rows plus the bf16 window.
+// (view, KV head) as a list of ascending row indices; the attention kernel
+// then reads those rows through the list, plus the bf16 window.
 //
 // "Reasoning-Aware Error-Bounded KV-Cache Compression and Sparse Attention
 // for Long-Context LLMs", Metodologia C (dynamic sparse decode attention: the
@@ -25,7 +25,8 @@ constexpr int kScoreBlocks = 4;      // blocks of kScoreTok tokens per score CTA
 constexpr int kScoreHeads = 8;       // query heads per register batch
 constexpr int kSelectThreads = 512;
 constexpr int kSelectStageMax = 45056;  // keys a select CTA stages in shared memory (176 KiB)
-constexpr int kSelectIdxMax = 4096;     // selections a select CTA also keeps in shared memory
+constexpr int kSelFastMax = 32768;      // select_fast_kernel: views of up to 32 keys per thread
+constexpr int kSelBins = 2048;          // histogram bins of a select_fast_kernel pass
 
 struct ScoreView {
     const uint8_t *k_codes;   // [H_kv][cap][RB]
@@ -156,15 +157,8 @@ __global__ void __launch_bounds__(kScoreTok) score_kernel(const __grid_constant_
 
 struct SelectView {
     int64_t score_off;        // as ScoreView::score_off
-    int32_t n_packed;         // n_packed <= top_k: every token, no scores read, no rows copied
+    int32_t n_packed;         // n_packed <= top_k: every token, no scores read
     int32_t out_row;          // row of the selection: [out_row][H_kv][top_k]
-    const uint8_t *codes[2];  // source K, V codes [H_kv][cap][RB]
-    const float *sm[2];       // source K, V scale/min [H_kv][cap][NG][2]
-    uint8_t *dst_codes[2];    // compact [H_kv][cap_c][RB]
-    float *dst_sm[2];         // compact [H_kv][cap_c][NG][2]
-    int64_t cap_packed;
-    int64_t cap_compact;
-    int32_t row_bytes;
     int32_t staged;           // 1: the head's keys fit the launch's shared-memory stage
 };
 
@@ -175,7 +169,6 @@ struct SelectArgs {
     int32_t n_sel_rows;       // rows of sel (the debug build's checks)
     int32_t top_k;
     int32_t n_kv_heads;
-    int32_t sm_bytes;         // scale/min bytes per row: (D/64) * 8
     SelectView views[kSparseMaxViews];
 };
 
@@ -189,12 +182,10 @@ __device__ __forceinline__ uint32_t order_key(float f) {
 // 8-bit digit passes from the top, over keys staged in shared memory when
 // they fit), an ordered compaction that writes the selected indices in
 // ascending order (equal scores at the threshold taken from the lowest index
-// up), then the copy of the selected packed rows (K and V codes and
-// scale/min) to consecutive rows of the compact view.
+// up).  The attention grid reads the selected rows through that list.
 __global__ void __launch_bounds__(kSelectThreads) select_kernel(const __grid_constant__ SelectArgs a) {
     extern __shared__ uint32_t skeys[];
     __shared__ uint32_t hist[256];
-    __shared__ int32_t sidx[kSelectIdxMax];
     __shared__ uint32_t pick[2];
     pdl_wait();  // the scores of the preceding grid
     pdl_launch_dependents();
@@ -202,11 +193,10 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const __grid_con
     const int hk = blockIdx.y, tid = threadIdx.x, lane = tid & 31;
     const int n = v.n_packed, K = a.top_k;
     int32_t *out = a.sel + ((int64_t)v.out_row * a.n_kv_heads + hk) * K;
-    // the selection row, the head's scores and its compact rows exist (debug
+    // the selection row and the head's scores exist (debug
     // build; uniform over the CTA, so a refused CTA returns whole)
     if (!dcheck(v.out_row >= 0 && v.out_row < a.n_sel_rows && hk < a.n_kv_heads &&
-                    (n <= K || (v.score_off >= 0 && v.score_off + (int64_t)(hk + 1) * n <= a.n_scores &&
-                                n <= v.cap_packed && K <= v.cap_compact)),
+                    (n <= K || (v.score_off >= 0 && v.score_off + (int64_t)(hk + 1) * n <= a.n_scores)),
                 kDbgSelect))
         return;
     if (n <= K) {
@@ -311,7 +301,6 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const __grid_con
         }
     }
     __syncthreads();
-    const bool keep = K <= kSelectIdxMax;  // the selection also stays in shared memory
     {
         const uint32_t take = hist[2 * kWarps + warp];
         uint32_t pos = hist[3 * kWarps + warp], taken = 0;
@@ -322,47 +311,285 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const __grid_con
             const uint32_t eqm = __ballot_sync(0xFFFFFFFFu, i < w1 && k == prefix);
             const bool pick_me = i < w1 && (k > prefix || (k == prefix && taken + __popc(eqm & below) < take));
             const uint32_t pm = __ballot_sync(0xFFFFFFFFu, pick_me);
-            if (pick_me) {
-                const uint32_t at = pos + __popc(pm & below);
-                if (keep) sidx[at] = i;
-                out[at] = i;
-            }
+            if (pick_me) out[pos + __popc(pm & below)] = i;
             pos += __popc(pm);
             taken += min((uint32_t)__popc(eqm), take - min(take, taken));
         }
     }
-    __syncthreads();  // the CTA's selection writes, before it reads them back
-    // the selected rows, in selection order, 8 bytes per thread and access,
-    // eight loads in flight per thread
-    const int wc = v.row_bytes / 8, ws = a.sm_bytes / 8, W = 2 * wc + 2 * ws;
-    auto word = [&](int i, const uint2 *&src, uint2 *&dst) {
-        const int r = i / W, w = i - r * W;
-        const int64_t src_row = (int64_t)hk * v.cap_packed + (keep ? sidx[r] : out[r]);
-        const int64_t dst_row = (int64_t)hk * v.cap_compact + r;
-        if (w < 2 * wc) {
-            const int kv = w >= wc, x = w - kv * wc;
-            src = reinterpret_cast<const uint2 *>(v.codes[kv] + src_row * v.row_bytes) + x;
-            dst = reinterpret_cast<uint2 *>(v.dst_codes[kv] + dst_row * v.row_bytes) + x;
-        } else {
-            const int y = w - 2 * wc, kv = y >= ws, x = y - kv * ws;
-            src = reinterpret_cast<const uint2 *>(reinterpret_cast<const uint8_t *>(v.sm[kv]) + src_row * a.sm_bytes) + x;
-            dst = reinterpret_cast<uint2 *>(reinterpret_cast<uint8_t *>(v.dst_sm[kv]) + dst_row * a.sm_bytes) + x;
+}
+
+// ---- select with a float-range first pass (views of up to 32768 tokens)
+
+// Inverse of order_key.
+__device__ __forceinline__ float key_float(uint32_t k) {
+    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Bin of order key k among kSelBins equal-width bins over [lo, lo + kSelBins
+// / scl], keys below and above the range in the end bins: monotone in the
+// key's float value, computed without contraction so that every use agrees.
+__device__ __forceinline__ uint32_t float_bin(uint32_t k, float lo, float scl) {
+    const float y = __fmul_rn(__fsub_rn(key_float(k), lo), scl);
+    return y <= 0.f ? 0u : min((uint32_t)(kSelBins - 1), (uint32_t)y);
+}
+
+// One CTA of THREADS per (view, KV head) with 32 * THREADS packed tokens at
+// most.  Keys (order keys of the scores) are staged in shared memory; thread
+// t owns keys t, t + kSelFastThreads, ... and marks which of them are still
+// candidates in one register.  The K-th largest key T comes from histogram
+// passes over the candidates: first kSelBins equal-width bins over the
+// scores' float range (scores spread evenly there, so the counters rarely
+// collide), then 11-bit digits of the candidates' keys below the bits they
+// all share.  The keys in the bins above the boundary bin are taken; those
+// in it stay candidates.  Each warp then walks one contiguous segment of the
+// keys and writes every key above T and the first (by index) of those equal
+// to T in ascending order.
+template <int THREADS>
+__global__ void __launch_bounds__(THREADS) select_fast_kernel(const __grid_constant__ SelectArgs a) {
+    static_assert(THREADS >= 64 && THREADS <= 1024 && kSelBins % THREADS == 0, "threads");
+    constexpr int kSelFastThreads = THREADS;
+    extern __shared__ uint32_t fkeys[];
+    __shared__ uint32_t hist[kSelBins];
+    __shared__ uint32_t red[5 * 32];
+    __shared__ uint32_t pick[2];
+    constexpr int kWarps = THREADS / 32;
+    constexpr int kKeys = 32;                         // keys per thread at most
+    constexpr int kBpt = kSelBins / THREADS;          // bins per thread of the boundary search
+    pdl_wait();  // the scores of the preceding grid
+    pdl_launch_dependents();
+    const SelectView &v = a.views[blockIdx.x];
+    const int hk = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const int n = v.n_packed, K = a.top_k;
+    int32_t *out = a.sel + ((int64_t)v.out_row * a.n_kv_heads + hk) * K;
+    // the selection row and the head's scores exist, and the keys fit (debug
+    // build; uniform over the CTA, so a refused CTA returns whole)
+    if (!dcheck(v.out_row >= 0 && v.out_row < a.n_sel_rows && hk < a.n_kv_heads &&
+                    (n <= K || (v.score_off >= 0 && v.score_off + (int64_t)(hk + 1) * n <= a.n_scores &&
+                                n <= kKeys * THREADS)),
+                kDbgSelect))
+        return;
+    if (n <= K) {
+        for (int i = tid; i < K; i += kSelFastThreads) out[i] = i < n ? i : -1;
+        return;
+    }
+    const float *sc = a.scores + v.score_off + (int64_t)hk * n;
+    const int nk = tid < n ? (n - tid + kSelFastThreads - 1) / kSelFastThreads : 0;  // keys of this thread
+    uint32_t cand = 0;  // bit j: key tid + j * kSelFastThreads is a candidate
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+    float s1 = 0.f, s2 = 0.f;  // sum and sum of squares of the finite scores
+#pragma unroll 8
+    for (int j = 0; j < kKeys; ++j) {
+        const int i = tid + j * kSelFastThreads;
+        if (i < n) {
+            const float x = __ldcg(sc + i);
+            const uint32_t k = order_key(x);
+            fkeys[i] = k;
+            cand |= 1u << j;
+            mn = min(mn, k);
+            mx = max(mx, k);
+            if (isfinite(x)) {
+                s1 += x;
+                s2 = fmaf(x, x, s2);
+            }
         }
-    };
-    const int total = K * W;
-    for (int i0 = tid; i0 < total; i0 += 8 * kSelectThreads) {
-        const uint2 *src[8];
-        uint2 *dst[8];
-        uint2 val[8];
+    }
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (i0 + j * kSelectThreads < total) word(i0 + j * kSelectThreads, src[j], dst[j]);
+    for (int o = 16; o > 0; o >>= 1) {
+        s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
+        s2 += __shfl_xor_sync(0xFFFFFFFFu, s2, o);
+    }
+    if (lane == 0) {
+        reinterpret_cast<float *>(red)[96 + warp] = s1;
+        reinterpret_cast<float *>(red)[128 + warp] = s2;
+    }
+    __syncthreads();
+    s1 = lane < kWarps ? reinterpret_cast<const float *>(red)[96 + lane] : 0.f;
+    s2 = lane < kWarps ? reinterpret_cast<const float *>(red)[128 + lane] : 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (i0 + j * kSelectThreads < total) val[j] = __ldg(src[j]);
+    for (int o = 16; o > 0; o >>= 1) {
+        s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
+        s2 += __shfl_xor_sync(0xFFFFFFFFu, s2, o);
+    }
+    // the first pass's range: mean +- 6 standard deviations within [min, max]
+    // (any range gives the exact selection: scores outside it fall into the
+    // end bins; a range that leaves out a few outliers keeps the bins where
+    // the K-th score lies from collapsing into one)
+    const float mean = s1 / (float)n, sd = sqrtf(fmaxf(s2 / (float)n - mean * mean, 0.f));
+    uint32_t rem = (uint32_t)K;
+    bool first = true, done = false, failed = false;
+    // at most one float pass and three digit passes; the bound and the
+    // boundary check only guard against a broken count
+    for (int pass = 0; pass < 5; ++pass) {
+        // block-wide min and max of the candidates (shuffles, then warp 0's
+        // partials in shared memory)
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-            if (i0 + j * kSelectThreads < total) *dst[j] = val[j];
+        for (int o = 16; o > 0; o >>= 1) {
+            mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+            mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        }
+        if (lane == 0) {
+            red[warp] = mn;
+            red[32 + warp] = mx;
+        }
+        __syncthreads();
+        mn = lane < kWarps ? red[lane] : 0xFFFFFFFFu;
+        mx = lane < kWarps ? red[32 + lane] : 0u;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
+            mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
+        }
+        if (mn == mx) {  // the candidates are all T (uniform)
+            done = true;
+            break;
+        }
+        // this pass's bins: the float range on the first pass when its ends
+        // are finite and distinct, else 11-bit digits below the shared bits
+        // (every candidate finite: the smallest and largest are)
+        const bool ends_finite = isfinite(key_float(mn)) && isfinite(key_float(mx));
+        float lo = key_float(mn), hi = key_float(mx);
+        if (first && ends_finite && isfinite(mean) && isfinite(sd) && sd > 0.f) {
+            lo = fmaxf(lo, mean - 6.f * sd);
+            hi = fminf(hi, mean + 6.f * sd);
+        }
+        const float span = hi - lo;
+        const float scl = (float)kSelBins / span;
+        const bool use_float = first && ends_finite && isfinite(span) && span > 0.f && isfinite(scl);
+        first = false;
+        const int top_bit = 31 - __clz(mn ^ mx);
+        const int shift = top_bit > 10 ? top_bit - 10 : 0;
+        for (int i = tid; i < kSelBins; i += kSelFastThreads) hist[i] = 0u;
+        if (tid == 0) {
+            pick[0] = 0xFFFFFFFFu;  // stays so if no bin holds the boundary
+            pick[1] = 0u;
+        }
+        __syncthreads();
+        // the candidates: on the first pass every key of the thread (an
+        // unrolled loop, several in flight), later the set bits
+        if (pass == 0) {
+#pragma unroll 8
+            for (int j = 0; j < nk; ++j) {
+                const uint32_t k = fkeys[tid + j * kSelFastThreads];
+                const uint32_t b = use_float ? float_bin(k, lo, scl) : (k >> shift) & (uint32_t)(kSelBins - 1);
+                atomicAdd(&hist[b], 1u);
+            }
+        } else {
+            for (uint32_t cb = cand; cb != 0u; cb &= cb - 1u) {
+                const int j = __ffs(cb) - 1;
+                const uint32_t k = fkeys[tid + j * kSelFastThreads];
+                const uint32_t b = use_float ? float_bin(k, lo, scl) : (k >> shift) & (uint32_t)(kSelBins - 1);
+                atomicAdd(&hist[b], 1u);
+            }
+        }
+        __syncthreads();
+        // boundary bin: thread t sums bins kSelBins - (t+1)*kBpt .. kSelBins
+        // - t*kBpt - 1 (the highest bins first), one block scan of the sums
+        const int top = kSelBins - tid * kBpt;
+        uint32_t c = 0;
+#pragma unroll
+        for (int i = 1; i <= kBpt; ++i) c += hist[top - i];
+        uint32_t inc = c;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+            if (lane >= o) inc += y;
+        }
+        if (lane == 31) red[64 + warp] = inc;
+        __syncthreads();
+        uint32_t wtot = lane < kWarps ? red[64 + lane] : 0u, winc = wtot;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, winc, o);
+            if (lane >= o) winc += y;
+        }
+        uint32_t above = __shfl_sync(0xFFFFFFFFu, winc - wtot, warp) + inc - c;
+        if (above < rem && rem <= above + c) {
+#pragma unroll
+            for (int i = 1; i <= kBpt; ++i) {
+                const uint32_t h = hist[top - i];
+                if (above + h >= rem) {
+                    pick[0] = (uint32_t)(top - i);
+                    pick[1] = above;
+                    break;
+                }
+                above += h;
+            }
+        }
+        __syncthreads();
+        const uint32_t pb = pick[0], pabove = pick[1];
+        if (pb >= (uint32_t)kSelBins) {
+            failed = true;
+            break;
+        }
+        rem -= pabove;
+        mn = 0xFFFFFFFFu;
+        mx = 0u;
+        if (pass == 0) {
+#pragma unroll 8
+            for (int j = 0; j < nk; ++j) {
+                const uint32_t k = fkeys[tid + j * kSelFastThreads];
+                const uint32_t b = use_float ? float_bin(k, lo, scl) : (k >> shift) & (uint32_t)(kSelBins - 1);
+                if (b != pb) {
+                    cand &= ~(1u << j);
+                } else {
+                    mn = min(mn, k);
+                    mx = max(mx, k);
+                }
+            }
+        } else {
+            for (uint32_t cb = cand; cb != 0u; cb &= cb - 1u) {
+                const int j = __ffs(cb) - 1;
+                const uint32_t k = fkeys[tid + j * kSelFastThreads];
+                const uint32_t b = use_float ? float_bin(k, lo, scl) : (k >> shift) & (uint32_t)(kSelBins - 1);
+                if (b != pb) {
+                    cand &= ~(1u << j);
+                } else {
+                    mn = min(mn, k);
+                    mx = max(mx, k);
+                }
+            }
+        }
+        __syncthreads();  // red, hist and pick are rewritten by the next pass
+    }
+    if (!dcheck(done && !failed && rem >= 1u && rem <= (uint32_t)K, kDbgSelect) || !done || failed) {
+        for (int i = tid; i < K; i += kSelFastThreads) out[i] = -1;
+        return;
+    }
+    const uint32_t T = mn;  // rem keys equal to T remain to be taken
+    // ordered compaction: warp w walks keys [w0, w1), 32 at a time
+    const int seg = (n + kWarps - 1) / kWarps;
+    const int w0 = min(n, warp * seg), w1 = min(n, w0 + seg);
+    uint32_t gt = 0, eq = 0;
+    for (int i0 = w0; i0 < w1; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t k = i < w1 ? fkeys[i] : 0u;
+        gt += __popc(__ballot_sync(0xFFFFFFFFu, i < w1 && k > T));
+        eq += __popc(__ballot_sync(0xFFFFFFFFu, i < w1 && k == T));
+    }
+    if (lane == 0) {
+        red[96 + warp] = gt;
+        red[128 + warp] = eq;
+    }
+    __syncthreads();
+    // this warp's first output position and the equal keys it takes
+    uint32_t g_before = 0, e_before = 0;
+    for (int w = 0; w < warp; ++w) {
+        g_before += red[96 + w];
+        e_before += red[128 + w];
+    }
+    const uint32_t take = e_before >= rem ? 0u : min(eq, rem - e_before);
+    uint32_t pos = g_before + min(e_before, rem), taken = 0;
+    const uint32_t below = (1u << lane) - 1u;
+    for (int i0 = w0; i0 < w1; i0 += 32) {
+        const int i = i0 + lane;
+        const uint32_t k = i < w1 ? fkeys[i] : 0u;
+        const uint32_t eqm = __ballot_sync(0xFFFFFFFFu, i < w1 && k == T);
+        const bool pick_me = i < w1 && (k > T || (k == T && taken + __popc(eqm & below) < take));
+        const uint32_t pm = __ballot_sync(0xFFFFFFFFu, pick_me);
+        const uint32_t at = pos + __popc(pm & below);
+        if (pick_me && dcheck(at < (uint32_t)K, kDbgSelect)) out[at] = i;
+        pos += __popc(pm);
+        taken += min((uint32_t)__popc(eqm), take - min(take, taken));
     }
 }
 

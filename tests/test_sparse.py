@@ -200,3 +200,68 @@ def test_sparse_many_views_and_workspace_reuse_while_growing(cuda_device):
             h["v"] = np.concatenate([h["v"], wl.bf16_bits(vn[i])[:, None]], axis=1)
             s.n_packed += 1  # the window was full: its oldest token moved to the packed part
         torch.cuda.synchronize()
+
+
+def test_sparse_long_views_both_select_paths(cuda_device):
+    # 32768 packed tokens (keys in registers, 1024 threads), 40000 (keys
+    # staged in shared memory) and 5000 (256 threads), top_k in the
+    # thousands
+    specs = [ViewSpec(32768, 16, 16, 4, head=2, seed=810), ViewSpec(40000, 16, 16, 4, head=0, seed=811),
+             ViewSpec(5000, 0, 0, 2, seed=812)]
+    case = build_case(8, 2, 128, specs, q_seed=21)
+    scale = 1 / np.sqrt(128)
+    k = pick_top_k(case, scale, range(1500, 2400, 7))
+    check(case, scale, k, "long views")
+
+
+def dup_case(n_packed, n_window, bits, D, hq, hkv, block, copies, seed):
+    """One view whose first `block` packed tokens repeat `copies` times in
+    aligned blocks (equal K and V rows, so equal scores on both sides)."""
+    g = wl.generator(seed)
+    mask = wl.outlier_mask(g, hkv, D, 0.0)
+    k, v = wl.kv_pair(g, hkv, n_packed + n_window, D, mask)
+    for m in range(1, copies):
+        k[:, m * block:(m + 1) * block] = k[:, :block]
+        v[:, m * block:(m + 1) * block] = v[:, :block]
+    view = kvq.View(hkv, D, bits, n_packed + 2, n_window, device="cuda")
+    view.fill_packed(k[:, :n_packed].cuda(), v[:, :n_packed].cuda())
+    view.fill_window(k[:, n_packed:].cuda(), v[:, n_packed:].cuda(), head=0)
+    gq = wl.generator(seed + 1)
+    q = wl.normal_bf16(gq, (1, hq, D))
+    from helpers import Case
+    return Case(hq, hkv, D, [ViewSpec(n_packed, n_window, n_window, bits, seed=seed)], [view], q.cuda(),
+                [dict(k=wl.bf16_bits(k), v=wl.bf16_bits(v))], wl.bf16_bits(q))
+
+
+def test_sparse_exact_ties_take_lowest_indices(cuda_device):
+    # 8 copies of a 32-token block: the K-th score falls inside a group of 8
+    # equal scores for at least one KV head, where the tie rule (lowest index
+    # first) decides; the other heads have a clear gap at K
+    for n, seed in ((4096, 830), (20000, 831)):
+        case = dup_case(n, 16, 4, 128, 8, 2, 32, 8, seed)
+        scale = 1 / np.sqrt(128)
+        sc = oracle_scores(case, 0, scale)
+        chosen = None
+        for k in range(64, n - 64):
+            inside, ok = False, True
+            for s in sc:
+                srt = np.sort(s)[::-1]
+                if srt[k - 1] - srt[k] >= GAP:
+                    continue
+                if srt[k - 1] != srt[k]:
+                    ok = False
+                    break
+                # an exact tie group [lo, hi) around rank k, clear of its neighbours
+                lo = k - 1
+                while lo > 0 and srt[lo - 1] == srt[k]:
+                    lo -= 1
+                hi = k
+                while hi < len(srt) and srt[hi] == srt[k]:
+                    hi += 1
+                ok &= (lo == 0 or srt[lo - 1] - srt[k] >= GAP) and (hi == len(srt) or srt[k] - srt[hi] >= GAP)
+                inside = True
+            if ok and inside:
+                chosen = k
+                break
+        assert chosen is not None, "no top_k inside a tie group"
+        check(case, scale, chosen, f"ties n {n}")
