@@ -188,8 +188,22 @@ int attn_header_bytes(int ng) {
 int64_t packed_token_bytes(int32_t head_dim, int32_t bits) { return 2 * row_bytes(head_dim, bits) + 16 * (head_dim / 64); }
 int64_t window_token_bytes(int32_t head_dim) { return 4 * (int64_t)head_dim; }
 
-// Cost model of a work item, in byte-equivalents: the bytes its tokens bring
-// in plus a fixed per-CTA cost (set-up, pipeline fill, partial merge).  A
+// Planner cost of a packed token, in byte-equivalents: its bytes, or a floor
+// for its arithmetic (unpacking, MMAs and the affine fold do not shrink with
+// the width), whichever is more.  Without the floor a 2-bit token looks 40 %
+// cheaper than a 4-bit one, and a mixed-width call gives its narrow views
+// too few CTAs.  The floor, 80 bytes per 64-dim group, is the largest that
+// leaves the 4-bit plans as they were: Qwen3-32B-shape layer 82.1 -> 72.0
+// us; Llama-3.1-8B and Gemma-3-12B layers unchanged (120 and more moved the
+// Gemma plan off its best, 74 -> 80 us).
+constexpr double kTokComputePerGroup = 80.0;
+double packed_token_cost(int32_t head_dim, int32_t bits) {
+    return std::max((double)packed_token_bytes(head_dim, bits), kTokComputePerGroup * (head_dim / 64));
+}
+
+// Cost model of a work item, in byte-equivalents: its tokens' costs (packed:
+// packed_token_cost; window: bytes) plus a fixed per-CTA cost (set-up,
+// pipeline fill, partial merge).  A
 // launch's predicted time is its number of waves times (largest item +
 // per-CTA cost).
 constexpr double kCtaCost = 96.0 * 1024;
@@ -213,7 +227,7 @@ double plan_free(const kvq_view *views, const int *idx, int n_idx, int64_t units
     double total = 0;
     for (int k = 0; k < n_idx; ++k) {
         const kvq_view &v = views[idx[k]];
-        total += (double)units * ((double)v.n_packed * packed_token_bytes(head_dim, v.bits) +
+        total += (double)units * ((double)v.n_packed * packed_token_cost(head_dim, v.bits) +
                                   (double)v.n_window * window_token_bytes(head_dim));
     }
     auto split = [&](int64_t n_tok, int step, double tok_cost, double W) -> int64_t {
@@ -228,7 +242,7 @@ double plan_free(const kvq_view *views, const int *idx, int n_idx, int64_t units
         for (int k = 0; k < n_idx; ++k) {
             const int i = idx[k];
             const kvq_view &v = views[i];
-            const double cp = (double)packed_token_bytes(head_dim, v.bits), cw = (double)window_token_bytes(head_dim);
+            const double cp = packed_token_cost(head_dim, v.bits), cw = (double)window_token_bytes(head_dim);
             int64_t np = split(v.n_packed, 2 * kvq::kTile, cp, W), nw = split(v.n_window, kvq::kTile, cw, W);
             // the unit combine holds at most kMaxChunksPerUnit chunks per unit
             while (np + nw > kvq::kMaxChunksPerUnit) {
@@ -368,7 +382,7 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
     std::stable_sort(plan.order.begin(), plan.order.end(), [&](int a, int b) { return key(a) < key(b); });
     double bytes_all = 0;
     for (int i = 0; i < n_views; ++i)
-        bytes_all += (double)views[i].n_packed * packed_token_bytes(head_dim, views[i].bits) +
+        bytes_all += (double)views[i].n_packed * packed_token_cost(head_dim, views[i].bits) +
                      (double)views[i].n_window * window_token_bytes(head_dim);
     for (int v0 = 0; v0 < n_used;) {
         int v1 = v0 + 1;
@@ -376,7 +390,7 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
         double bytes = 0;
         for (int k = v0; k < v1; ++k) {
             const kvq_view &v = views[plan.order[k]];
-            bytes += (double)v.n_packed * packed_token_bytes(head_dim, v.bits) +
+            bytes += (double)v.n_packed * packed_token_cost(head_dim, v.bits) +
                      (double)v.n_window * window_token_bytes(head_dim);
         }
         const int64_t share = std::max<int64_t>(
