@@ -106,6 +106,8 @@ struct AttnLaunch {
     int v0, v1;          // views order[v0 .. v1) of the plan
     int total_chunks;
     int bits;            // the width of every view of the launch with packed tokens
+    int ring_bytes = 0;  // per warp, and the launch's dynamic shared memory:
+    size_t smem = 0;     // sized for this launch's own blocks
 };
 
 struct ViewChunks {
@@ -344,25 +346,32 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
     const int ctas = attn_ctas_per_sm(ng);
     const int smem_cta = std::min(227 * 1024, (228 * 1024) / ctas - 1024);
     const int header = attn_header_bytes(ng);
-    uint32_t blk_max = 0;
-    for (int i = 0; i < n_views; ++i) {
-        if (views[i].n_packed > 0)
-            blk_max = std::max<uint32_t>(blk_max, (uint32_t)(64 * row_bytes(head_dim, views[i].bits) + 512 * ng));
-        if (views[i].n_window > 0) blk_max = std::max<uint32_t>(blk_max, (uint32_t)(32 * head_dim));
-    }
-    int ring = (smem_cta - header) / kvq::kAttnWarps / 128 * 128;
-    // a team's ring (its warps' rings together) holds two blocks, and later
-    // the team's partial (m, l, O of 8 heads); all rings together hold the
-    // unit combine's scratch
+    const int ring_fit = (smem_cta - header) / kvq::kAttnWarps / 128 * 128;
+    // Ring and shared memory of a launch over views[order[v0 .. v1)]: a
+    // team's ring (its warps' rings together) holds two of the launch's
+    // largest blocks, and later the team's partial (m, l, O of 8 heads); all
+    // rings together hold the unit combine's scratch.  Per launch, so that a
+    // mixed-width call's 8-bit blocks do not take the narrower launches'
+    // CTAs per SM.
     const uint32_t tw = (uint32_t)attn_team_warps(ng);
     const uint32_t combine_scratch = (2 * kvq::kMaxChunksPerUnit * kvq::kHeadsPerCta + kvq::kHeadsPerCta) * 4;
-    const int ring_min =
-        (int)std::max<uint32_t>(std::max<uint32_t>((2 * blk_max + tw - 1) / tw, (64 + 32 * (uint32_t)head_dim + tw - 1) / tw),
-                                (combine_scratch + kvq::kAttnWarps - 1) / kvq::kAttnWarps);
-    if (ring < ring_min) ring = (ring_min + 127) / 128 * 128;  // fewer CTAs per SM, still correct
-    plan.ring_bytes = ring;
-    plan.smem = (size_t)header + (size_t)kvq::kAttnWarps * ring;
-    if (plan.smem > 227 * 1024) return KVQ_ERR_UNSUPPORTED;
+    auto size_launch = [&](AttnLaunch &L) -> bool {
+        uint32_t blk_max = 0;
+        for (int k = L.v0; k < L.v1; ++k) {
+            const kvq_view &v = views[plan.order[k]];
+            if (v.n_packed > 0)
+                blk_max = std::max<uint32_t>(blk_max, (uint32_t)(64 * row_bytes(head_dim, v.bits) + 512 * ng));
+            if (v.n_window > 0) blk_max = std::max<uint32_t>(blk_max, (uint32_t)(32 * head_dim));
+        }
+        const int ring_min = (int)std::max<uint32_t>(
+            std::max<uint32_t>((2 * blk_max + tw - 1) / tw, (64 + 32 * (uint32_t)head_dim + tw - 1) / tw),
+            (combine_scratch + kvq::kAttnWarps - 1) / kvq::kAttnWarps);
+        int ring = ring_fit;
+        if (ring < ring_min) ring = (ring_min + 127) / 128 * 128;  // fewer CTAs per SM, still correct
+        L.ring_bytes = ring;
+        L.smem = (size_t)header + (size_t)kvq::kAttnWarps * ring;
+        return L.smem <= 227 * 1024;
+    };
 
     const int64_t slots = (int64_t)device_sm_count() * ctas;
     plan.chunks.assign(n_views, ViewChunks{0, 0});
@@ -398,7 +407,11 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
         int64_t chunks = 0;
         plan_free(views, plan.order.data() + v0, v1 - v0, units, head_dim, share, plan.chunks, &chunks);
         if (chunks > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
-        plan.launches.push_back(AttnLaunch{v0, v1, (int)chunks, key(plan.order[v0])});
+        AttnLaunch L{v0, v1, (int)chunks, key(plan.order[v0])};
+        if (!size_launch(L)) return KVQ_ERR_UNSUPPORTED;
+        plan.ring_bytes = std::max(plan.ring_bytes, L.ring_bytes);
+        plan.smem = std::max(plan.smem, L.smem);
+        plan.launches.push_back(L);
         v0 = v1;
     }
     // A sequence's unit combine holds at most kMaxChunksPerUnit chunks: trim
@@ -495,7 +508,7 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
     prm.n_kv_heads = n_kv_heads;
     prm.group = n_q_heads / n_kv_heads;
     prm.head_blocks = plan.head_blocks;
-    prm.ring_bytes = plan.ring_bytes;
+
     prm.counters = reinterpret_cast<uint32_t *>(ws + plan.counters_off);
     prm.partials = reinterpret_cast<float *>(ws + plan.partials_off);
     for (const AttnLaunch &L : plan.launches) {
@@ -552,13 +565,14 @@ kvq_status launch_attn_ng(const AttnPlan &plan, const kvq_view *views, int32_t n
         std::memset(&cfg, 0, sizeof cfg);
         cfg.gridDim = dim3((unsigned)L.total_chunks, (unsigned)n_kv_heads, (unsigned)plan.head_blocks);
         cfg.blockDim = dim3(kvq::kAttnThreads);
-        cfg.dynamicSmemBytes = plan.smem;
+        cfg.dynamicSmemBytes = L.smem;
+        prm.ring_bytes = L.ring_bytes;
         cfg.stream = st;
         cfg.attrs = &attr;
         cfg.numAttrs = 1;
         prm.scores = scores;
-        const kvq_status es = scores ? launch_attn_grid<NG, true>(L.bits, plan.smem, cfg, prm)
-                                     : launch_attn_grid<NG, false>(L.bits, plan.smem, cfg, prm);
+        const kvq_status es = scores ? launch_attn_grid<NG, true>(L.bits, L.smem, cfg, prm)
+                                     : launch_attn_grid<NG, false>(L.bits, L.smem, cfg, prm);
         if (es != KVQ_OK) return es;
     }
     return KVQ_OK;
