@@ -105,9 +105,12 @@ def test_sparse_llama_shape_small(cuda_device):
 
 
 # groups of up to 8 query heads score on the attention grid's tensor-core QK
-# path, wider ones (32 / 2) on the SIMT score kernel
+# path, wider ones (32 / 2) on the SIMT score kernel; the gathered rows are
+# copied in 16-byte pieces, or 8-byte ones where a row is not a 16-byte
+# multiple (3-bit codes at head_dim 64 and 192, scale/min rows of head_dim 64
+# and 192)
 @pytest.mark.parametrize("bits,D,hq,hkv", [(2, 64, 2, 2), (3, 128, 8, 2), (8, 256, 16, 8), (4, 64, 64, 8),
-                                           (4, 128, 32, 2)])
+                                           (4, 128, 32, 2), (3, 64, 4, 2), (3, 192, 6, 2), (4, 192, 8, 4)])
 def test_sparse_widths_shapes_groups(cuda_device, bits, D, hq, hkv):
     specs = [ViewSpec(300, 8, 8, bits, head=3, seed=300 + bits), ViewSpec(129, 0, 0, bits, seed=301 + bits),
              ViewSpec(0, 5, 8, bits, head=6, seed=302 + bits)]
