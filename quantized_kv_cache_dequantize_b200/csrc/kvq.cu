@@ -393,6 +393,14 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
     for (int i = 0; i < n_views; ++i)
         bytes_all += (double)views[i].n_packed * packed_token_cost(head_dim, views[i].bits) +
                      (double)views[i].n_window * window_token_bytes(head_dim);
+    // A call of several width launches is planned for 5/4 of the resident
+    // slots: the launches run side by side, and smaller items let them share
+    // the SMs more evenly (Qwen3-32B-shape layer, widths 2/3/4/8: 68.5 vs
+    // 73.0 us).  A single-width call keeps whole waves of its own (planned
+    // for 5/4, the Gemma-3-12B and Llama-3.1-8B layers lost 20-25 %).
+    bool mixed = false;
+    for (int k = 1; k < n_used; ++k) mixed |= key(plan.order[k]) != key(plan.order[0]);
+    const int64_t plan_slots = mixed ? slots * 5 / 4 : slots;
     for (int v0 = 0; v0 < n_used;) {
         int v1 = v0 + 1;
         while (v1 < n_used && v1 - v0 < kvq::kAttnMaxViews && key(plan.order[v1]) == key(plan.order[v0])) ++v1;
@@ -403,7 +411,7 @@ kvq_status plan_attn(const kvq_view *views, int32_t n_views, const int32_t *seq_
                      (double)v.n_window * window_token_bytes(head_dim);
         }
         const int64_t share = std::max<int64_t>(
-            1, (int64_t)std::llround((double)slots * (bytes_all > 0 ? bytes / bytes_all : 1.0)));
+            1, (int64_t)std::llround((double)plan_slots * (bytes_all > 0 ? bytes / bytes_all : 1.0)));
         int64_t chunks = 0;
         plan_free(views, plan.order.data() + v0, v1 - v0, units, head_dim, share, plan.chunks, &chunks);
         if (chunks > INT32_MAX) return KVQ_ERR_UNSUPPORTED;
