@@ -42,7 +42,8 @@ __host__ __device__ constexpr uint32_t magic_pack_word(int w) {
 }
 
 // Quantize one half (32 elements) of a 64-element group held as 16 bf16x2
-// words (also readable at `src`, used only for the rare exact re-check); the
+// words (also readable at `src`, read again only for the exact re-check of
+// near-tie elements); the
 // partner half lives in lane ^ 1, which must execute this call in the same
 // instruction stream (full-warp shuffles).  Writes the packed codes of this
 // half (32*B bits = B words, code j at bit j*B) and the group's s, mn.
@@ -121,18 +122,11 @@ __device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], con
         while (near) {
             const int i = __ffs(near) - 1;
             near &= near - 1u;
-            // element i from the registers by a binary select tree on the bits
-            // of i (stays in registers; no memory round trip)
-            uint32_t t8[8], t4[4], t2[2];
-#pragma unroll
-            for (int k = 0; k < 8; ++k) t8[k] = (i & 16) ? x[k + 8] : x[k];
-#pragma unroll
-            for (int k = 0; k < 4; ++k) t4[k] = (i & 8) ? t8[k + 4] : t8[k];
-#pragma unroll
-            for (int k = 0; k < 2; ++k) t2[k] = (i & 4) ? t4[k + 2] : t4[k];
-            const uint32_t w = (i & 2) ? t2[1] : t2[0];
-            const float xf = (i & 1) ? bf16hi_to_f32(w) : bf16lo_to_f32(w);
-            (void)src;
+            // element i again from memory: the lane has just read the row, so
+            // it is a cache hit, and one load costs the integer pipe (the
+            // kernel's bound) less than a select tree over the 16 registers
+            // (handoff K cache: 628.5 vs 637.7 us)
+            const float xf = __uint_as_float((uint32_t)__ldg(src + i) << 16);
             const float a = __fsub_rn(xf, mn);
             // the code the fast path packed (the same arithmetic), and the
             // half-integer the quotient is near
