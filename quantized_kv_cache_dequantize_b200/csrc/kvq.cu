@@ -943,6 +943,28 @@ kvq_status launch_pdl(void (*kernel)(Args), dim3 grid, unsigned block, size_t sm
     return cudaLaunchKernelEx(&cfg, kernel, a) == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
+// The same with thread-block clusters of `cluster` CTAs along x.
+template <typename Args>
+kvq_status launch_pdl_cluster(void (*kernel)(Args), dim3 grid, unsigned block, unsigned cluster, size_t smem,
+                              cudaStream_t st, const Args &a) {
+    cudaLaunchAttribute attr[2];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    attr[1].id = cudaLaunchAttributeClusterDimension;
+    attr[1].val.clusterDim.x = cluster;
+    attr[1].val.clusterDim.y = 1;
+    attr[1].val.clusterDim.z = 1;
+    cudaLaunchConfig_t cfg;
+    std::memset(&cfg, 0, sizeof cfg);
+    cfg.gridDim = grid;
+    cfg.blockDim = dim3(block);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = st;
+    cfg.attrs = attr;
+    cfg.numAttrs = 2;
+    return cudaLaunchKernelEx(&cfg, kernel, a) == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
 template <int NG, int B>
 kvq_status launch_score_grid(const kvq::ScoreArgs &a, unsigned ctas, size_t smem, cudaStream_t st) {
     if (smem > 48 * 1024 &&
@@ -1044,7 +1066,7 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
         v0 = v1;
     }
     // 2. selections of every view (ascending row indices): views of up to
-    // 32768 packed tokens on select_fast_kernel, longer ones on
+    // kSelFastMax packed tokens on select_cluster_kernel, longer ones on
     // select_kernel (keys staged in shared memory or read from the scores)
     for (int large = 0; large < 2; ++large) {
         std::vector<int> idx;
@@ -1074,26 +1096,43 @@ kvq_status launch_sparse(const SparsePlan &sp, const kvq_view *views, int32_t n_
                 d.staged = v.n_packed <= kvq::kSelectStageMax ? 1 : 0;
                 if (d.staged) smem = std::max(smem, (size_t)v.n_packed * 4);
             }
-            const dim3 grid((unsigned)(v1 - v0), (unsigned)n_kv_heads);
             kvq_status es;
             if (!large) {
-                const size_t keys = (size_t)max_n * 4;
-                if (keys > 48 * 1024 && cudaFuncSetAttribute(kvq::select_fast_kernel<1024>,
-                                                             cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                                             (int)keys) != cudaSuccess) {
+                // `cl` CTAs per (view, KV head), a thread-block cluster when
+                // more than one: the fewest that leave a lane at most 32 keys
+                // (KVQ_SELECT_CLUSTER = 2 or 4 asks for more)
+                constexpr int64_t T = kvq::kSelClusterThreads;
+                int cl = 1;
+                const int forced = env_int("KVQ_SELECT_CLUSTER", 0);
+                if (forced == 2 || forced == 4) cl = forced;
+                while (cl < kvq::kSelMaxCluster && max_n > cl * T * 32) cl *= 2;
+                int64_t cap = 0;  // keys of the largest slice: T * keys per lane
+                for (size_t k = v0; k < v1; ++k)
+                    if (sp.score_off[idx[k]] >= 0)
+                        cap = std::max(cap, T * ((views[idx[k]].n_packed + cl * T - 1) / (cl * T)));
+                a.key_cap = (int32_t)cap;
+                const size_t keys = (size_t)cap * 6;  // keys and first-pass bins
+                const dim3 grid((unsigned)((v1 - v0) * cl), (unsigned)n_kv_heads);
+                auto kernel = cl > 1 ? kvq::select_cluster_kernel<kvq::kSelClusterThreads, true>
+                                     : kvq::select_cluster_kernel<kvq::kSelClusterThreads, false>;
+                // (the opt-in above 48 KiB counts the kernel's ~25 KiB of
+                // static shared memory too)
+                if (keys + 26 * 1024 > 48 * 1024 &&
+                    cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)keys) !=
+                        cudaSuccess) {
                     (void)cudaGetLastError();
                     return KVQ_ERR_CUDA;
                 }
-                // (latency-bound: more warps beat fewer keys per warp, also for
-                // short views)
-                es = launch_pdl(kvq::select_fast_kernel<1024>, grid, 1024, keys, st, a);
+                es = cl > 1 ? launch_pdl_cluster(kernel, grid, kvq::kSelClusterThreads, (unsigned)cl, keys, st, a)
+                            : launch_pdl(kernel, grid, kvq::kSelClusterThreads, keys, st, a);
             } else {
-                if (smem > 48 * 1024 &&
+                if (smem + 2 * 1024 > 48 * 1024 &&  // (with its 1 KiB of static shared memory)
                     cudaFuncSetAttribute(kvq::select_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
                         cudaSuccess) {
                     (void)cudaGetLastError();
                     return KVQ_ERR_CUDA;
                 }
+                const dim3 grid((unsigned)(v1 - v0), (unsigned)n_kv_heads);
                 es = launch_pdl(kvq::select_kernel, grid, kvq::kSelectThreads, smem, st, a);
             }
             if (es != KVQ_OK) return es;

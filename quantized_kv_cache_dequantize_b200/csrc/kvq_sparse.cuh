@@ -25,8 +25,11 @@ constexpr int kScoreBlocks = 4;      // blocks of kScoreTok tokens per score CTA
 constexpr int kScoreHeads = 8;       // query heads per register batch
 constexpr int kSelectThreads = 512;
 constexpr int kSelectStageMax = 45056;  // keys a select CTA stages in shared memory (176 KiB)
-constexpr int kSelFastMax = 32768;      // select_fast_kernel: views of up to 32 keys per thread
-constexpr int kSelBins = 2048;          // histogram bins of a select_fast_kernel pass
+constexpr int kSelClusterThreads = 1024;  // select_cluster_kernel CTA
+constexpr int kSelMaxCluster = 4;         // CTAs per (view, KV head) at most
+constexpr int kSelFastMax = kSelMaxCluster * kSelClusterThreads * 32;  // 32 keys per thread at most
+constexpr int kSelBins = 2048;            // histogram bins of a select_cluster_kernel pass
+constexpr int kSelWarpMax = 64;           // candidates one warp finishes
 
 struct ScoreView {
     const uint8_t *k_codes;   // [H_kv][cap][RB]
@@ -167,6 +170,7 @@ struct SelectArgs {
     int32_t *sel;             // int32 [n_views][H_kv][top_k], ascending, -1 padded
     int64_t n_scores;         // floats of the score array,
     int32_t n_sel_rows;       // rows of sel (the debug build's checks)
+    int32_t key_cap;          // keys a select_cluster_kernel CTA's dynamic shared memory holds
     int32_t top_k;
     int32_t n_kv_heads;
     SelectView views[kSparseMaxViews];
@@ -318,279 +322,518 @@ __global__ void __launch_bounds__(kSelectThreads) select_kernel(const __grid_con
     }
 }
 
-// ---- select with a float-range first pass (views of up to 32768 tokens)
+// ---- select over keys in shared memory (views of up to kSelFastMax tokens)
 
-// Inverse of order_key.
-__device__ __forceinline__ float key_float(uint32_t k) {
-    return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+// Bin of a score x (order key k) on the first pass: kSelBins equal-width bins
+// over [lo, lo + kSelBins / scl] with scores below and above the range in the
+// end bins, or, without a usable range, the key's top 11 bits.  Monotone in
+// the key (NaNs sort beyond the infinities of their sign); computed without
+// contraction so that every use agrees.
+__device__ __forceinline__ uint32_t first_bin(float x, uint32_t k, bool use_float, float lo, float scl) {
+    if (!use_float) return k >> 21;
+    // clamped into [0, kSelBins - 1] (the infinities into the end bins), then
+    // truncated; a NaN goes to the end bin of its sign
+    const float y = fminf(fmaxf(__fmul_rn(__fsub_rn(x, lo), scl), 0.f), (float)(kSelBins - 1));
+    return x != x ? ((k >> 31) ? (uint32_t)(kSelBins - 1) : 0u) : (uint32_t)y;
 }
 
-// Bin of order key k among kSelBins equal-width bins over [lo, lo + kSelBins
-// / scl], keys below and above the range in the end bins: monotone in the
-// key's float value, computed without contraction so that every use agrees.
-__device__ __forceinline__ uint32_t float_bin(uint32_t k, float lo, float scl) {
-    const float y = __fmul_rn(__fsub_rn(key_float(k), lo), scl);
-    return y <= 0.f ? 0u : min((uint32_t)(kSelBins - 1), (uint32_t)y);
+// Butterfly sum over a warp (every lane ends with the same result).
+__device__ __forceinline__ uint32_t warp_sum_u32(uint32_t x) {
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) x += __shfl_xor_sync(0xFFFFFFFFu, x, o);
+    return x;
 }
 
-// One CTA of THREADS per (view, KV head) with 32 * THREADS packed tokens at
-// most.  Keys (order keys of the scores) are staged in shared memory; thread
-// t owns keys t, t + kSelFastThreads, ... and marks which of them are still
-// candidates in one register.  The K-th largest key T comes from histogram
-// passes over the candidates: first kSelBins equal-width bins over the
-// scores' float range (scores spread evenly there, so the counters rarely
-// collide), then 11-bit digits of the candidates' keys below the bits they
-// all share.  The keys in the bins above the boundary bin are taken; those
-// in it stay candidates.  Each warp then walks one contiguous segment of the
-// keys and writes every key above T and the first (by index) of those equal
-// to T in ascending order.
-template <int THREADS>
-__global__ void __launch_bounds__(THREADS) select_fast_kernel(const __grid_constant__ SelectArgs a) {
-    static_assert(THREADS >= 64 && THREADS <= 1024 && kSelBins % THREADS == 0, "threads");
-    constexpr int kSelFastThreads = THREADS;
-    extern __shared__ uint32_t fkeys[];
-    __shared__ uint32_t hist[kSelBins];
-    __shared__ uint32_t red[5 * 32];
-    __shared__ uint32_t pick[2];
+// Top-K selection of one (view, KV head) by one CTA, or, with CLUSTER, by a
+// thread-block cluster of CL CTAs (CL from the launch).  CTA r owns the keys
+// [r*S, (r+1)*S) of the view, warp w of it the 32*kpt keys from r*S +
+// 32*kpt*w, lane l the keys l, l+32, ... of those, kpt <= 32 per lane (bit j
+// of a lane's masks: its key j).  The scores arrive by asynchronous 4-byte
+// copies straight into shared memory, where they become order keys; the
+// first-pass bins are kept beside them.
+//   1. 256 evenly spaced scores of the CTA (of each CTA of the cluster) give
+//      the first pass's range (mean +- 6 standard deviations within their min
+//      and max; any range gives the exact selection: scores outside it go to
+//      the end bins).
+//   2. First pass: counts of every key's bin; the boundary bin from the
+//      counts (of the whole cluster: each CTA sums its peers' histograms), the
+//      same in every CTA.  Keys in higher bins are taken ("above"); those in
+//      it stay candidates.
+//   3. While more than kSelWarpMax candidates remain and they differ: 11-bit
+//      digit passes below the bits they share.  Then the candidates are
+//      gathered into one list, where one warp finds the K-th largest key T:
+//      the candidate with fewer than rem larger ones and at least rem not
+//      smaller.
+//   4. Ordered compaction: the keys above T and the first (by index) of
+//      those equal to T, the output position of every warp from the counts
+//      of the warps and CTAs before it.
+// In a cluster, every decision that gates a cluster barrier is taken on
+// cluster-wide values, so all its CTAs pass the same barriers; values from
+// the peers are read by one warp and handed on in shared memory.
+template <int THREADS, bool CLUSTER>
+__global__ void __launch_bounds__(THREADS) select_cluster_kernel(const __grid_constant__ SelectArgs a) {
+    static_assert(THREADS % 32 == 0 && THREADS >= 128 && THREADS <= 1024 && kSelBins % THREADS == 0 &&
+                      kSelBins / 4 <= THREADS && (THREADS / 32) * 64 <= kSelBins, "threads");
     constexpr int kWarps = THREADS / 32;
-    constexpr int kKeys = 32;                         // keys per thread at most
-    constexpr int kBpt = kSelBins / THREADS;          // bins per thread of the boundary search
+    constexpr int kBpt = kSelBins / THREADS;  // bins per thread of the boundary search
+    constexpr int kSample = 8;                // scores per lane of warp 0 behind the first pass's range
+    constexpr uint32_t kFull = 0xFFFFFFFFu;
+    extern __shared__ __align__(16) uint32_t skeys[];  // [S] scores, then keys; then [S] uint16 first-pass bins
+    __shared__ __align__(16) uint32_t hist[2][kSelBins];  // this CTA's counts, by pass parity
+    __shared__ __align__(16) uint32_t hm[CLUSTER ? kSelBins : 4];  // the cluster's counts
+    __shared__ uint32_t lst[kSelWarpMax];                 // this CTA's candidates at the end
+    __shared__ uint32_t gl[CLUSTER ? kSelWarpMax : 4];    // the cluster's candidates
+    __shared__ uint32_t xch[12];                          // what the cluster's CTAs read from each other
+    __shared__ uint32_t red[5][32];
+    __shared__ uint32_t bc[6];                            // values handed on to the CTA
+    __shared__ uint32_t pick[2];
     pdl_wait();  // the scores of the preceding grid
     pdl_launch_dependents();
-    const SelectView &v = a.views[blockIdx.x];
+    const uint32_t CL = CLUSTER ? cluster_nctarank() : 1u, rank = CLUSTER ? cluster_ctarank() : 0u;
+    const SelectView &v = a.views[blockIdx.x / CL];
     const int hk = blockIdx.y, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const int n = v.n_packed, K = a.top_k;
     int32_t *out = a.sel + ((int64_t)v.out_row * a.n_kv_heads + hk) * K;
+    const int kpt = (n + (int)CL * THREADS - 1) / ((int)CL * THREADS);
+    const int seg = 32 * kpt, S = kWarps * seg;
     // the selection row and the head's scores exist, and the keys fit (debug
-    // build; uniform over the CTA, so a refused CTA returns whole)
+    // build; uniform over the cluster, so a refused cluster returns whole)
     if (!dcheck(v.out_row >= 0 && v.out_row < a.n_sel_rows && hk < a.n_kv_heads &&
                     (n <= K || (v.score_off >= 0 && v.score_off + (int64_t)(hk + 1) * n <= a.n_scores &&
-                                n <= kKeys * THREADS)),
+                                kpt <= 32 && S <= a.key_cap)),
                 kDbgSelect))
         return;
     if (n <= K) {
-        for (int i = tid; i < K; i += kSelFastThreads) out[i] = i < n ? i : -1;
+        for (int i = (int)rank * THREADS + tid; i < K; i += (int)CL * THREADS) out[i] = i < n ? i : -1;
         return;
     }
+    auto csync = [&]() {
+        if constexpr (CLUSTER)
+            cluster_sync();
+        else
+            __syncthreads();
+    };
+    uint16_t *sbin = reinterpret_cast<uint16_t *>(skeys + S);
     const float *sc = a.scores + v.score_off + (int64_t)hk * n;
-    const int nk = tid < n ? (n - tid + kSelFastThreads - 1) / kSelFastThreads : 0;  // keys of this thread
-    uint32_t cand = 0;  // bit j: key tid + j * kSelFastThreads is a candidate
-    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
-    float s1 = 0.f, s2 = 0.f;  // sum and sum of squares of the finite scores
-#pragma unroll 8
-    for (int j = 0; j < kKeys; ++j) {
-        const int i = tid + j * kSelFastThreads;
-        if (i < n) {
-            const float x = __ldcg(sc + i);
-            const uint32_t k = order_key(x);
-            fkeys[i] = k;
-            cand |= 1u << j;
-            mn = min(mn, k);
-            mx = max(mx, k);
-            if (isfinite(x)) {
+    const int base = (int)rank * S + warp * seg + lane;  // index of this lane's key 0; key j at + 32 j
+    const int lbase = warp * seg + lane;                 // its place in skeys
+    const int nk = base < n ? min(kpt, (n - base + 31) / 32) : 0;
+    // every score of this lane in flight at once
+    for (int j = 0; j < nk; ++j) cp_async<4>(skeys + lbase + 32 * j, sc + base + 32 * j);
+    for (int i = tid; i < kSelBins; i += THREADS) hist[0][i] = 0u;
+    cp_async_wait_all();
+    __syncthreads();  // every lane's scores have landed
+
+    // 1. the range, from kSample evenly spaced scores per lane of warp 0 (the
+    //    cluster's CTAs: their samples together)
+    float s1 = 0.f, s2 = 0.f, smin = INFINITY, smax = -INFINITY;
+    uint32_t ns = 0;
+    auto reduce5 = [&]() {  // butterfly: the same result in every lane
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            s1 += __shfl_xor_sync(kFull, s1, o);
+            s2 += __shfl_xor_sync(kFull, s2, o);
+            smin = fminf(smin, __shfl_xor_sync(kFull, smin, o));
+            smax = fmaxf(smax, __shfl_xor_sync(kFull, smax, o));
+            ns += __shfl_xor_sync(kFull, ns, o);
+        }
+    };
+    if (warp == 0) {
+        const int nloc = min(max(n - (int)rank * S, 0), S);  // keys of this CTA
+#pragma unroll
+        for (int i = 0; i < kSample; ++i) {
+            const int li = (int)(((int64_t)(lane + 32 * i) * nloc) / (32 * kSample));
+            const float x = __uint_as_float(skeys[min(li, S - 1)]);
+            if (li < nloc && isfinite(x)) {
                 s1 += x;
                 s2 = fmaf(x, x, s2);
+                smin = fminf(smin, x);
+                smax = fmaxf(smax, x);
+                ++ns;
             }
         }
+        reduce5();
     }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
-        s2 += __shfl_xor_sync(0xFFFFFFFFu, s2, o);
+    if constexpr (CLUSTER) {
+        if (tid == 0) {
+            xch[0] = __float_as_uint(s1);
+            xch[1] = __float_as_uint(s2);
+            xch[2] = __float_as_uint(smin);
+            xch[3] = __float_as_uint(smax);
+            xch[4] = ns;
+        }
+        cluster_sync();
+        if (warp == 0) {  // lane q < CL: CTA q's values
+            const bool in = (uint32_t)lane < CL;
+            s1 = in ? __uint_as_float(ld_cluster_u32(&xch[0], lane)) : 0.f;
+            s2 = in ? __uint_as_float(ld_cluster_u32(&xch[1], lane)) : 0.f;
+            smin = in ? __uint_as_float(ld_cluster_u32(&xch[2], lane)) : INFINITY;
+            smax = in ? __uint_as_float(ld_cluster_u32(&xch[3], lane)) : -INFINITY;
+            ns = in ? ld_cluster_u32(&xch[4], lane) : 0u;
+            reduce5();
+        }
     }
-    if (lane == 0) {
-        reinterpret_cast<float *>(red)[96 + warp] = s1;
-        reinterpret_cast<float *>(red)[128 + warp] = s2;
+    if (tid == 0) {
+        bc[0] = __float_as_uint(s1);
+        bc[1] = __float_as_uint(s2);
+        bc[2] = __float_as_uint(smin);
+        bc[3] = __float_as_uint(smax);
+        bc[4] = ns;
     }
     __syncthreads();
-    s1 = lane < kWarps ? reinterpret_cast<const float *>(red)[96 + lane] : 0.f;
-    s2 = lane < kWarps ? reinterpret_cast<const float *>(red)[128 + lane] : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-        s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, o);
-        s2 += __shfl_xor_sync(0xFFFFFFFFu, s2, o);
-    }
-    // the first pass's range: mean +- 6 standard deviations within [min, max]
-    // (any range gives the exact selection: scores outside it fall into the
-    // end bins; a range that leaves out a few outliers keeps the bins where
-    // the K-th score lies from collapsing into one)
-    const float mean = s1 / (float)n, sd = sqrtf(fmaxf(s2 / (float)n - mean * mean, 0.f));
-    uint32_t rem = (uint32_t)K;
-    bool first = true, done = false, failed = false;
-    // at most one float pass and three digit passes; the bound and the
-    // boundary check only guard against a broken count
-    for (int pass = 0; pass < 5; ++pass) {
-        // block-wide min and max of the candidates (shuffles, then warp 0's
-        // partials in shared memory)
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
-            mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-        }
-        if (lane == 0) {
-            red[warp] = mn;
-            red[32 + warp] = mx;
-        }
-        __syncthreads();
-        mn = lane < kWarps ? red[lane] : 0xFFFFFFFFu;
-        mx = lane < kWarps ? red[32 + lane] : 0u;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            mn = min(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, o));
-            mx = max(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, o));
-        }
-        if (mn == mx) {  // the candidates are all T (uniform)
-            done = true;
-            break;
-        }
-        // this pass's bins: the float range on the first pass when its ends
-        // are finite and distinct, else 11-bit digits below the shared bits
-        // (every candidate finite: the smallest and largest are)
-        const bool ends_finite = isfinite(key_float(mn)) && isfinite(key_float(mx));
-        float lo = key_float(mn), hi = key_float(mx);
-        if (first && ends_finite && isfinite(mean) && isfinite(sd) && sd > 0.f) {
-            lo = fmaxf(lo, mean - 6.f * sd);
-            hi = fminf(hi, mean + 6.f * sd);
-        }
-        const float span = hi - lo;
-        const float scl = (float)kSelBins / span;
-        const bool use_float = first && ends_finite && isfinite(span) && span > 0.f && isfinite(scl);
-        first = false;
-        const int top_bit = 31 - __clz(mn ^ mx);
-        const int shift = top_bit > 10 ? top_bit - 10 : 0;
-        for (int i = tid; i < kSelBins; i += kSelFastThreads) hist[i] = 0u;
-        if (tid == 0) {
-            pick[0] = 0xFFFFFFFFu;  // stays so if no bin holds the boundary
-            pick[1] = 0u;
-        }
-        __syncthreads();
-        // the candidates: on the first pass every key of the thread (an
-        // unrolled loop, several in flight), later the set bits
-        if (pass == 0) {
+    s1 = __uint_as_float(bc[0]);
+    s2 = __uint_as_float(bc[1]);
+    smin = __uint_as_float(bc[2]);
+    smax = __uint_as_float(bc[3]);
+    ns = bc[4];
+    const float mean = s1 / (float)max(ns, 1u);
+    const float sd = sqrtf(fmaxf(s2 / (float)max(ns, 1u) - mean * mean, 0.f));
+    const float lo = fmaxf(smin, mean - 6.f * sd), hi = fminf(smax, mean + 6.f * sd);
+    const float span = hi - lo, scl = (float)kSelBins / span;
+    const bool use_float = ns > 0 && isfinite(mean) && isfinite(sd) && isfinite(span) && span > 0.f && isfinite(scl);
+
+    // 2. first pass: keys in place of the scores, bins beside them, counts
 #pragma unroll 8
-            for (int j = 0; j < nk; ++j) {
-                const uint32_t k = fkeys[tid + j * kSelFastThreads];
-                const uint32_t b = use_float ? float_bin(k, lo, scl) : (k >> shift) & (uint32_t)(kSelBins - 1);
-                atomicAdd(&hist[b], 1u);
+    for (int j = 0; j < nk; ++j) {
+        const float x = __uint_as_float(skeys[lbase + 32 * j]);
+        const uint32_t k = order_key(x);
+        const uint32_t b = first_bin(x, k, use_float, lo, scl);
+        skeys[lbase + 32 * j] = k;
+        sbin[lbase + 32 * j] = (uint16_t)b;
+        atomicAdd(&hist[0][b], 1u);
+    }
+    csync();  // every CTA's counts are complete
+
+    // boundary bin of this pass's counts (the cluster's: summed from the
+    // peers' histograms with 16-byte loads): thread t sums bins kSelBins -
+    // (t+1)*kBpt .. kSelBins - t*kBpt - 1 (highest first), one block scan of
+    // the sums; pick = {bin, keys in higher bins}, or {kSelBins, 0} when no
+    // bin holds the rem-th key (a broken count)
+    uint32_t rem = (uint32_t)K;
+    auto boundary = [&](int p) {
+        const uint32_t *h = hist[p];
+        if constexpr (CLUSTER) {
+            if (tid < kSelBins / 4) {
+                uint4 s = make_uint4(0u, 0u, 0u, 0u);
+                for (uint32_t q = 0; q < CL; ++q) {
+                    const uint4 y = ld_cluster_v4(&hist[p][4 * tid], q);
+                    s.x += y.x;
+                    s.y += y.y;
+                    s.z += y.z;
+                    s.w += y.w;
+                }
+                *reinterpret_cast<uint4 *>(&hm[4 * tid]) = s;
             }
-        } else {
-            for (uint32_t cb = cand; cb != 0u; cb &= cb - 1u) {
-                const int j = __ffs(cb) - 1;
-                const uint32_t k = fkeys[tid + j * kSelFastThreads];
-                const uint32_t b = use_float ? float_bin(k, lo, scl) : (k >> shift) & (uint32_t)(kSelBins - 1);
-                atomicAdd(&hist[b], 1u);
-            }
+            __syncthreads();
+            h = hm;
         }
-        __syncthreads();
-        // boundary bin: thread t sums bins kSelBins - (t+1)*kBpt .. kSelBins
-        // - t*kBpt - 1 (the highest bins first), one block scan of the sums
         const int top = kSelBins - tid * kBpt;
-        uint32_t c = 0;
+        uint32_t hc[kBpt], c = 0;
 #pragma unroll
-        for (int i = 1; i <= kBpt; ++i) c += hist[top - i];
+        for (int i = 0; i < kBpt; ++i) {
+            hc[i] = h[top - 1 - i];
+            c += hc[i];
+        }
         uint32_t inc = c;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, inc, o);
+            const uint32_t y = __shfl_up_sync(kFull, inc, o);
             if (lane >= o) inc += y;
         }
-        if (lane == 31) red[64 + warp] = inc;
+        if (tid == 0) {
+            pick[0] = (uint32_t)kSelBins;
+            pick[1] = 0u;
+        }
+        if (lane == 31) red[0][warp] = inc;
         __syncthreads();
-        uint32_t wtot = lane < kWarps ? red[64 + lane] : 0u, winc = wtot;
+        const uint32_t wtot = lane < kWarps ? red[0][lane] : 0u;
+        uint32_t winc = wtot;
 #pragma unroll
         for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(0xFFFFFFFFu, winc, o);
+            const uint32_t y = __shfl_up_sync(kFull, winc, o);
             if (lane >= o) winc += y;
         }
-        uint32_t above = __shfl_sync(0xFFFFFFFFu, winc - wtot, warp) + inc - c;
+        uint32_t above = __shfl_sync(kFull, winc - wtot, warp) + inc - c;
         if (above < rem && rem <= above + c) {
 #pragma unroll
-            for (int i = 1; i <= kBpt; ++i) {
-                const uint32_t h = hist[top - i];
-                if (above + h >= rem) {
-                    pick[0] = (uint32_t)(top - i);
+            for (int i = 0; i < kBpt; ++i) {
+                if (above + hc[i] >= rem) {
+                    pick[0] = (uint32_t)(top - 1 - i);
                     pick[1] = above;
                     break;
                 }
-                above += h;
+                above += hc[i];
             }
         }
         __syncthreads();
-        const uint32_t pb = pick[0], pabove = pick[1];
+    };
+    boundary(0);
+    uint32_t pb = pick[0];
+    bool failed = pb >= (uint32_t)kSelBins, done = false;
+    rem -= pick[1];
+    uint32_t above = 0u, cand = 0u;  // bit j: key j is above the candidates / a candidate
+    uint32_t mn = 0xFFFFFFFFu, mx = 0u;
+#pragma unroll 8
+    for (int j = 0; j < nk; ++j) {
+        const uint32_t b = sbin[lbase + 32 * j];
+        above |= (b > pb ? 1u : 0u) << j;
+        if (b == pb) {
+            cand |= 1u << j;
+            const uint32_t k = skeys[lbase + 32 * j];
+            mn = min(mn, k);
+            mx = max(mx, k);
+        }
+    }
+
+    // 3. digit passes while many candidates differ, then the warp finish
+    for (int pass = 1; pass <= 4 && !failed; ++pass) {
+        uint32_t cnt = __popc(cand);
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            mn = min(mn, __shfl_xor_sync(kFull, mn, o));
+            mx = max(mx, __shfl_xor_sync(kFull, mx, o));
+            cnt += __shfl_xor_sync(kFull, cnt, o);
+        }
+        if (lane == 0) {
+            red[1][warp] = mn;
+            red[2][warp] = mx;
+            red[3][warp] = cnt;
+        }
+        __syncthreads();
+        mn = lane < kWarps ? red[1][lane] : 0xFFFFFFFFu;
+        mx = lane < kWarps ? red[2][lane] : 0u;
+        cnt = lane < kWarps ? red[3][lane] : 0u;
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            mn = min(mn, __shfl_xor_sync(kFull, mn, o));
+            mx = max(mx, __shfl_xor_sync(kFull, mx, o));
+            cnt += __shfl_xor_sync(kFull, cnt, o);
+        }
+        if constexpr (CLUSTER) {
+            if (tid == 0) {
+                xch[5] = mn;
+                xch[6] = mx;
+                xch[7] = cnt;
+            }
+            cluster_sync();
+            if (warp == 0) {
+                const bool in = (uint32_t)lane < CL;
+                mn = in ? ld_cluster_u32(&xch[5], lane) : 0xFFFFFFFFu;
+                mx = in ? ld_cluster_u32(&xch[6], lane) : 0u;
+                cnt = in ? ld_cluster_u32(&xch[7], lane) : 0u;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) {
+                    mn = min(mn, __shfl_xor_sync(kFull, mn, o));
+                    mx = max(mx, __shfl_xor_sync(kFull, mx, o));
+                    cnt += __shfl_xor_sync(kFull, cnt, o);
+                }
+                if (lane == 0) {
+                    bc[0] = mn;
+                    bc[1] = mx;
+                    bc[2] = cnt;
+                }
+            }
+            __syncthreads();
+            mn = bc[0];
+            mx = bc[1];
+            cnt = bc[2];
+        }
+        if (mn == mx) {  // the candidates are all T
+            done = true;
+            break;
+        }
+        if (cnt <= (uint32_t)kSelWarpMax) {
+            // this CTA's candidates to its list (and the cluster's lists
+            // into one), then warp 0: lane l tests candidates l and l + 32
+            if (tid == 0) pick[0] = 0u;
+            __syncthreads();
+            const uint32_t my = __popc(cand);
+            if (my) {
+                uint32_t at = atomicAdd(&pick[0], my);
+                for (uint32_t cb = cand; cb != 0u; cb &= cb - 1u) {
+                    const uint32_t k = skeys[lbase + 32 * (__ffs(cb) - 1)];
+                    if (dcheck(at < (uint32_t)kSelWarpMax, kDbgSelect)) lst[at] = k;
+                    ++at;
+                }
+            }
+            __syncthreads();
+            const uint32_t *g = lst;
+            uint32_t m = min(pick[0], (uint32_t)kSelWarpMax);
+            if constexpr (CLUSTER) {
+                if (tid == 0) xch[8] = pick[0];
+                cluster_sync();
+                g = gl;
+                m = 0;
+                if (warp == 0)
+                    for (uint32_t q = 0; q < CL; ++q) {
+                        const uint32_t cq = min(ld_cluster_u32(&xch[8], q), (uint32_t)kSelWarpMax);
+                        for (uint32_t i = lane; i < cq; i += 32)
+                            if (dcheck(m + i < (uint32_t)kSelWarpMax, kDbgSelect)) gl[m + i] = ld_cluster_u32(&lst[i], q);
+                        m = min(m + cq, (uint32_t)kSelWarpMax);
+                    }
+                __syncwarp();
+            }
+            if (warp == 0) {
+#pragma unroll
+                for (int h = 0; h < kSelWarpMax / 32; ++h) {
+                    const uint32_t i0 = (uint32_t)(lane + 32 * h);
+                    const uint32_t c = i0 < m ? g[i0] : 0u;
+                    uint32_t n_gt = 0, n_ge = 0;
+                    for (uint32_t i = 0; i < m; ++i) {
+                        const uint32_t y = g[i];
+                        n_gt += y > c ? 1u : 0u;
+                        n_ge += y >= c ? 1u : 0u;
+                    }
+                    // T: fewer than rem candidates above it, at least rem not
+                    // below it (equal candidates write the same values)
+                    if (i0 < m && n_gt < rem && rem <= n_ge) {
+                        pick[0] = c;
+                        pick[1] = rem - n_gt;  // keys equal to T still to take (>= 1)
+                    }
+                }
+            }
+            __syncthreads();
+            mn = pick[0];
+            rem = pick[1];
+            done = true;
+            break;
+        }
+        // a digit pass: 11 bits below the bits the candidates share
+        const int p = pass & 1;
+        const int top_bit = 31 - __clz(mn ^ mx);
+        const int shift = top_bit > 10 ? top_bit - 10 : 0;
+        for (int i = tid; i < kSelBins; i += THREADS) hist[p][i] = 0u;
+        __syncthreads();
+        for (uint32_t cb = cand; cb != 0u; cb &= cb - 1u) {
+            const uint32_t k = skeys[lbase + 32 * (__ffs(cb) - 1)];
+            atomicAdd(&hist[p][(k >> shift) & (uint32_t)(kSelBins - 1)], 1u);
+        }
+        csync();
+        boundary(p);
+        pb = pick[0];
         if (pb >= (uint32_t)kSelBins) {
             failed = true;
             break;
         }
-        rem -= pabove;
+        rem -= pick[1];
         mn = 0xFFFFFFFFu;
         mx = 0u;
-        if (pass == 0) {
-#pragma unroll 8
-            for (int j = 0; j < nk; ++j) {
-                const uint32_t k = fkeys[tid + j * kSelFastThreads];
-                const uint32_t b = use_float ? float_bin(k, lo, scl) : (k >> shift) & (uint32_t)(kSelBins - 1);
-                if (b != pb) {
-                    cand &= ~(1u << j);
-                } else {
-                    mn = min(mn, k);
-                    mx = max(mx, k);
+        for (uint32_t cb = cand; cb != 0u; cb &= cb - 1u) {
+            const int j = __ffs(cb) - 1;
+            const uint32_t k = skeys[lbase + 32 * j];
+            const uint32_t b = (k >> shift) & (uint32_t)(kSelBins - 1);
+            if (b != pb) {
+                cand &= ~(1u << j);
+                if (b > pb) above |= 1u << j;
+            } else {
+                mn = min(mn, k);
+                mx = max(mx, k);
+            }
+        }
+    }
+
+    // 4. ordered compaction (T = mn; rem keys equal to T to take).  Per lane
+    //    the masks of its keys above T (gtm) and equal to T (eqm); per warp
+    //    the counts, and from the counts of the warps (and CTAs) before it
+    //    its first output position and the equal keys it takes.  Then row j
+    //    of a warp (its keys j of every lane, in index order) is one ballot;
+    //    a key's position is its warp's, plus the rows before its own, plus
+    //    the lanes before it in its row.
+    if (!dcheck(done && !failed && rem >= 1u && rem <= (uint32_t)K, kDbgSelect) || !done || failed) {
+        for (int i = (int)rank * THREADS + tid; i < K; i += (int)CL * THREADS) out[i] = -1;
+    } else {
+        const uint32_t T = mn;
+        uint32_t gtm = above, eqm = 0u;
+        for (uint32_t cb = cand; cb != 0u; cb &= cb - 1u) {
+            const int j = __ffs(cb) - 1;
+            const uint32_t k = skeys[lbase + 32 * j];
+            gtm |= (k > T ? 1u : 0u) << j;
+            eqm |= (k == T ? 1u : 0u) << j;
+        }
+        const uint32_t gt = warp_sum_u32(__popc(gtm)), eq = warp_sum_u32(__popc(eqm));
+        uint32_t *wcnt = hist[1];  // [0, 32): warps' keys above T, [32, 64): equal; [64, 128): before them
+        if (lane == 0) {
+            wcnt[warp] = gt;
+            wcnt[32 + warp] = eq;
+        }
+        __syncthreads();
+        if (warp == 0) {
+            const uint32_t g = lane < kWarps ? wcnt[lane] : 0u, e = lane < kWarps ? wcnt[32 + lane] : 0u;
+            uint32_t gi = g, ei = e;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t yg = __shfl_up_sync(kFull, gi, o), ye = __shfl_up_sync(kFull, ei, o);
+                if (lane >= o) {
+                    gi += yg;
+                    ei += ye;
                 }
             }
-        } else {
-            for (uint32_t cb = cand; cb != 0u; cb &= cb - 1u) {
-                const int j = __ffs(cb) - 1;
-                const uint32_t k = fkeys[tid + j * kSelFastThreads];
-                const uint32_t b = use_float ? float_bin(k, lo, scl) : (k >> shift) & (uint32_t)(kSelBins - 1);
-                if (b != pb) {
-                    cand &= ~(1u << j);
-                } else {
-                    mn = min(mn, k);
-                    mx = max(mx, k);
+            wcnt[64 + lane] = gi - g;
+            wcnt[96 + lane] = ei - e;
+            if constexpr (CLUSTER) {
+                const uint32_t cta_gt = __shfl_sync(kFull, gi, 31), cta_eq = __shfl_sync(kFull, ei, 31);
+                if (lane == 0) {
+                    xch[9] = cta_gt;
+                    xch[10] = cta_eq;
                 }
             }
         }
-        __syncthreads();  // red, hist and pick are rewritten by the next pass
+        if constexpr (CLUSTER) {
+            cluster_sync();
+            if (warp == 0) {  // the CTAs before this one
+                const bool in = (uint32_t)lane < rank;
+                const uint32_t cg = warp_sum_u32(in ? ld_cluster_u32(&xch[9], lane) : 0u);
+                const uint32_t ce = warp_sum_u32(in ? ld_cluster_u32(&xch[10], lane) : 0u);
+                if (lane == 0) {
+                    bc[0] = cg;
+                    bc[1] = ce;
+                }
+            }
+        }
+        __syncthreads();
+        uint32_t gt_before = wcnt[64 + warp], eq_before = wcnt[96 + warp];
+        if constexpr (CLUSTER) {
+            gt_before += bc[0];
+            eq_before += bc[1];
+        }
+        const uint32_t take = eq_before >= rem ? 0u : min(eq, rem - eq_before);
+        const uint32_t pos = gt_before + min(eq_before, rem);
+        const uint32_t below = (1u << lane) - 1u;
+        uint32_t selm = gtm;  // this lane's keys taken
+        if (take >= eq) {
+            selm |= eqm;
+        } else if (take > 0u) {  // the first `take` equal keys of the warp
+            uint32_t t = 0;
+            for (int j = 0; j < kpt; ++j) {
+                const uint32_t em = __ballot_sync(kFull, (eqm >> j) & 1u);
+                if (((eqm >> j) & 1u) && t + __popc(em & below) < take) selm |= 1u << j;
+                t += __popc(em);
+            }
+        }
+        // rows: lane j keeps row j; its keys' count before it by a scan
+        uint32_t myrow = 0u;
+        for (int j = 0; j < kpt; ++j) {
+            const uint32_t r = __ballot_sync(kFull, (selm >> j) & 1u);
+            myrow = lane == j ? r : myrow;
+        }
+        const uint32_t rc = __popc(myrow);
+        uint32_t ri = rc;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(kFull, ri, o);
+            if (lane >= o) ri += y;
+        }
+        uint32_t *wrow = hist[0] + 64 * warp;  // [row masks | keys in the rows before], kWarps * 64 <= kSelBins
+        wrow[lane] = myrow;
+        wrow[32 + lane] = ri - rc;
+        __syncwarp();
+        for (uint32_t sb = selm; sb != 0u; sb &= sb - 1u) {
+            const int j = __ffs(sb) - 1;
+            const uint32_t at = pos + wrow[32 + j] + __popc(wrow[j] & below);
+            if (dcheck(at < (uint32_t)K, kDbgSelect)) out[at] = base + 32 * j;
+        }
     }
-    if (!dcheck(done && !failed && rem >= 1u && rem <= (uint32_t)K, kDbgSelect) || !done || failed) {
-        for (int i = tid; i < K; i += kSelFastThreads) out[i] = -1;
-        return;
-    }
-    const uint32_t T = mn;  // rem keys equal to T remain to be taken
-    // ordered compaction: warp w walks keys [w0, w1), 32 at a time
-    const int seg = (n + kWarps - 1) / kWarps;
-    const int w0 = min(n, warp * seg), w1 = min(n, w0 + seg);
-    uint32_t gt = 0, eq = 0;
-    for (int i0 = w0; i0 < w1; i0 += 32) {
-        const int i = i0 + lane;
-        const uint32_t k = i < w1 ? fkeys[i] : 0u;
-        gt += __popc(__ballot_sync(0xFFFFFFFFu, i < w1 && k > T));
-        eq += __popc(__ballot_sync(0xFFFFFFFFu, i < w1 && k == T));
-    }
-    if (lane == 0) {
-        red[96 + warp] = gt;
-        red[128 + warp] = eq;
-    }
-    __syncthreads();
-    // this warp's first output position and the equal keys it takes
-    uint32_t g_before = 0, e_before = 0;
-    for (int w = 0; w < warp; ++w) {
-        g_before += red[96 + w];
-        e_before += red[128 + w];
-    }
-    const uint32_t take = e_before >= rem ? 0u : min(eq, rem - e_before);
-    uint32_t pos = g_before + min(e_before, rem), taken = 0;
-    const uint32_t below = (1u << lane) - 1u;
-    for (int i0 = w0; i0 < w1; i0 += 32) {
-        const int i = i0 + lane;
-        const uint32_t k = i < w1 ? fkeys[i] : 0u;
-        const uint32_t eqm = __ballot_sync(0xFFFFFFFFu, i < w1 && k == T);
-        const bool pick_me = i < w1 && (k > T || (k == T && taken + __popc(eqm & below) < take));
-        const uint32_t pm = __ballot_sync(0xFFFFFFFFu, pick_me);
-        const uint32_t at = pos + __popc(pm & below);
-        if (pick_me && dcheck(at < (uint32_t)K, kDbgSelect)) out[at] = i;
-        pos += __popc(pm);
-        taken += min((uint32_t)__popc(eqm), take - min(take, taken));
-    }
+    if constexpr (CLUSTER) cluster_sync();  // no CTA leaves while a peer may still read its shared memory
 }
 
 }  // namespace kvq

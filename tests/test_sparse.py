@@ -206,10 +206,10 @@ def test_sparse_many_views_and_workspace_reuse_while_growing(cuda_device):
 
 
 def test_sparse_long_views_both_select_paths(cuda_device):
-    # 32768 packed tokens (keys in registers, 1024 threads), 40000 (keys
-    # staged in shared memory) and 5000 (256 threads), top_k in the
-    # thousands
-    specs = [ViewSpec(32768, 16, 16, 4, head=2, seed=810), ViewSpec(40000, 16, 16, 4, head=0, seed=811),
+    # 32768 packed tokens (one select CTA, 32 keys a lane), 140000 (beyond
+    # the shared-memory select: the radix select reading the scores from
+    # memory) and 5000, top_k in the thousands
+    specs = [ViewSpec(32768, 16, 16, 4, head=2, seed=810), ViewSpec(140000, 16, 16, 4, head=0, seed=811),
              ViewSpec(5000, 0, 0, 2, seed=812)]
     case = build_case(8, 2, 128, specs, q_seed=21)
     scale = 1 / np.sqrt(128)
@@ -217,15 +217,32 @@ def test_sparse_long_views_both_select_paths(cuda_device):
     check(case, scale, k, "long views")
 
 
-def dup_case(n_packed, n_window, bits, D, hq, hkv, block, copies, seed):
-    """One view whose first `block` packed tokens repeat `copies` times in
-    aligned blocks (equal K and V rows, so equal scores on both sides)."""
+@pytest.mark.parametrize("cluster", ["1", "2", "4"])
+def test_sparse_select_cluster_sizes(cuda_device, monkeypatch, cluster):
+    # the same selections whatever the number of CTAs a (view, KV head) is
+    # split over (a view whose keys would exceed 32 a lane takes more);
+    # ragged slices: views shorter than one CTA's share, and lengths that are
+    # no multiple of 32
+    monkeypatch.setenv("KVQ_SELECT_CLUSTER", cluster)
+    specs = [ViewSpec(3001, 16, 16, 4, head=1, seed=840), ViewSpec(9000, 0, 0, 3, seed=841),
+             ViewSpec(20011, 8, 8, 4, head=5, seed=842), ViewSpec(700, 4, 4, 8, head=0, seed=843)]
+    case = build_case(8, 2, 64, specs, q_seed=23)
+    scale = 0.125
+    k = pick_top_k(case, scale, range(400, 690, 3))
+    check(case, scale, k, f"cluster {cluster}")
+
+
+def dup_case(n_packed, n_window, bits, D, hq, hkv, block, copies, seed, stride=None):
+    """One view whose first `block` packed tokens repeat `copies` times, at
+    multiples of `stride` (default `block`; equal K and V rows, so equal
+    scores on both sides)."""
+    stride = stride or block
     g = wl.generator(seed)
     mask = wl.outlier_mask(g, hkv, D, 0.0)
     k, v = wl.kv_pair(g, hkv, n_packed + n_window, D, mask)
     for m in range(1, copies):
-        k[:, m * block:(m + 1) * block] = k[:, :block]
-        v[:, m * block:(m + 1) * block] = v[:, :block]
+        k[:, m * stride:m * stride + block] = k[:, :block]
+        v[:, m * stride:m * stride + block] = v[:, :block]
     view = kvq.View(hkv, D, bits, n_packed + 2, n_window, device="cuda")
     view.fill_packed(k[:, :n_packed].cuda(), v[:, :n_packed].cuda())
     view.fill_window(k[:, n_packed:].cuda(), v[:, n_packed:].cuda(), head=0)
@@ -239,9 +256,10 @@ def dup_case(n_packed, n_window, bits, D, hq, hkv, block, copies, seed):
 def test_sparse_exact_ties_take_lowest_indices(cuda_device):
     # 8 copies of a 32-token block: the K-th score falls inside a group of 8
     # equal scores for at least one KV head, where the tie rule (lowest index
-    # first) decides; the other heads have a clear gap at K
-    for n, seed in ((4096, 830), (20000, 831)):
-        case = dup_case(n, 16, 4, 128, 8, 2, 32, 8, seed)
+    # first) decides; the other heads have a clear gap at K.  20000 tokens:
+    # the copies 2500 tokens apart, in different CTAs of the cluster
+    for n, seed, stride in ((4096, 830, 32), (20000, 831, 2500)):
+        case = dup_case(n, 16, 4, 128, 8, 2, 32, 8, seed, stride)
         scale = 1 / np.sqrt(128)
         sc = oracle_scores(case, 0, scale)
         chosen = None
