@@ -351,7 +351,8 @@ __device__ __forceinline__ uint32_t warp_sum_u32(uint32_t x) {
 // of a lane's masks: its key j).  The scores arrive by asynchronous 4-byte
 // copies straight into shared memory, where they become order keys; the
 // first-pass bins are kept beside them.
-//   1. 256 evenly spaced scores of the CTA (of each CTA of the cluster) give
+//   1. 256 scores of the CTA in 8 evenly spaced runs (of each CTA of the
+//      cluster) give
 //      the first pass's range (mean +- 6 standard deviations within their min
 //      and max; any range gives the exact selection: scores outside it go to
 //      the end bins).
@@ -371,7 +372,7 @@ __device__ __forceinline__ uint32_t warp_sum_u32(uint32_t x) {
 // cluster-wide values, so all its CTAs pass the same barriers; values from
 // the peers are read by one warp and handed on in shared memory.
 template <int THREADS, bool CLUSTER>
-__global__ void __launch_bounds__(THREADS) select_cluster_kernel(const __grid_constant__ SelectArgs a) {
+__global__ void __launch_bounds__(THREADS, 1) select_cluster_kernel(const __grid_constant__ SelectArgs a) {
     static_assert(THREADS % 32 == 0 && THREADS >= 128 && THREADS <= 1024 && kSelBins % THREADS == 0 &&
                       kSelBins / 4 <= THREADS && (THREADS / 32) * 64 <= kSelBins, "threads");
     constexpr int kWarps = THREADS / 32;
@@ -387,6 +388,7 @@ __global__ void __launch_bounds__(THREADS) select_cluster_kernel(const __grid_co
     __shared__ uint32_t red[5][32];
     __shared__ uint32_t bc[6];                            // values handed on to the CTA
     __shared__ uint32_t pick[2];
+    __shared__ uint32_t pc[3];                            // the candidates' min, max and count
     pdl_wait();  // the scores of the preceding grid
     pdl_launch_dependents();
     const uint32_t CL = CLUSTER ? cluster_nctarank() : 1u, rank = CLUSTER ? cluster_ctarank() : 0u;
@@ -441,8 +443,8 @@ __global__ void __launch_bounds__(THREADS) select_cluster_kernel(const __grid_co
     if (warp == 0) {
         const int nloc = min(max(n - (int)rank * S, 0), S);  // keys of this CTA
 #pragma unroll
-        for (int i = 0; i < kSample; ++i) {
-            const int li = (int)(((int64_t)(lane + 32 * i) * nloc) / (32 * kSample));
+        for (int i = 0; i < kSample; ++i) {  // kSample runs of 32 consecutive scores
+            const int li = (int)((((int64_t)i * nloc) / kSample) & ~31) + lane;
             const float x = __uint_as_float(skeys[min(li, S - 1)]);
             if (li < nloc && isfinite(x)) {
                 s1 += x;
@@ -543,6 +545,9 @@ __global__ void __launch_bounds__(THREADS) select_cluster_kernel(const __grid_co
         if (tid == 0) {
             pick[0] = (uint32_t)kSelBins;
             pick[1] = 0u;
+            pc[0] = 0xFFFFFFFFu;  // for the next pass's candidate counts
+            pc[1] = 0u;
+            pc[2] = 0u;
         }
         if (lane == 31) red[0][warp] = inc;
         __syncthreads();
@@ -587,28 +592,17 @@ __global__ void __launch_bounds__(THREADS) select_cluster_kernel(const __grid_co
 
     // 3. digit passes while many candidates differ, then the warp finish
     for (int pass = 1; pass <= 4 && !failed; ++pass) {
-        uint32_t cnt = __popc(cand);
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            mn = min(mn, __shfl_xor_sync(kFull, mn, o));
-            mx = max(mx, __shfl_xor_sync(kFull, mx, o));
-            cnt += __shfl_xor_sync(kFull, cnt, o);
-        }
-        if (lane == 0) {
-            red[1][warp] = mn;
-            red[2][warp] = mx;
-            red[3][warp] = cnt;
+        // the CTA's candidates' min, max and count: shared atomics of the
+        // lanes that hold any (few after the first pass)
+        if (cand != 0u) {
+            atomicMin(&pc[0], mn);
+            atomicMax(&pc[1], mx);
+            atomicAdd(&pc[2], (uint32_t)__popc(cand));
         }
         __syncthreads();
-        mn = lane < kWarps ? red[1][lane] : 0xFFFFFFFFu;
-        mx = lane < kWarps ? red[2][lane] : 0u;
-        cnt = lane < kWarps ? red[3][lane] : 0u;
-#pragma unroll
-        for (int o = 16; o > 0; o >>= 1) {
-            mn = min(mn, __shfl_xor_sync(kFull, mn, o));
-            mx = max(mx, __shfl_xor_sync(kFull, mx, o));
-            cnt += __shfl_xor_sync(kFull, cnt, o);
-        }
+        mn = pc[0];
+        mx = pc[1];
+        uint32_t cnt = pc[2];
         if constexpr (CLUSTER) {
             if (tid == 0) {
                 xch[5] = mn;
@@ -733,12 +727,13 @@ __global__ void __launch_bounds__(THREADS) select_cluster_kernel(const __grid_co
     }
 
     // 4. ordered compaction (T = mn; rem keys equal to T to take).  Per lane
-    //    the masks of its keys above T (gtm) and equal to T (eqm); per warp
-    //    the counts, and from the counts of the warps (and CTAs) before it
-    //    its first output position and the equal keys it takes.  Then row j
-    //    of a warp (its keys j of every lane, in index order) is one ballot;
-    //    a key's position is its warp's, plus the rows before its own, plus
-    //    the lanes before it in its row.
+    //    the masks of its keys above T (gtm) and equal to T (eqm).  Row j of
+    //    a warp (its keys j of every lane, in index order) is one ballot,
+    //    kept by lane j; the rows give the warp's counts, and the counts of
+    //    the warps (and CTAs) before it give its first output position and
+    //    the equal keys it takes.  A key's position is its warp's, plus the
+    //    keys taken in the rows before its own, plus the lanes before it in
+    //    its row.
     if (!dcheck(done && !failed && rem >= 1u && rem <= (uint32_t)K, kDbgSelect) || !done || failed) {
         for (int i = (int)rank * THREADS + tid; i < K; i += (int)CL * THREADS) out[i] = -1;
     } else {
@@ -750,7 +745,28 @@ __global__ void __launch_bounds__(THREADS) select_cluster_kernel(const __grid_co
             gtm |= (k > T ? 1u : 0u) << j;
             eqm |= (k == T ? 1u : 0u) << j;
         }
-        const uint32_t gt = warp_sum_u32(__popc(gtm)), eq = warp_sum_u32(__popc(eqm));
+        // this lane's rows, and the warp's counts from a scan of the rows
+        uint32_t rgt = 0u, req = 0u, eq = 0u;
+#pragma unroll 8
+        for (int j = 0; j < kpt; ++j) {
+            const uint32_t r = __ballot_sync(kFull, (gtm >> j) & 1u);
+            rgt = lane == j ? r : rgt;
+        }
+        if (__any_sync(kFull, eqm != 0u)) {
+            for (int j = 0; j < kpt; ++j) {
+                const uint32_t r = __ballot_sync(kFull, (eqm >> j) & 1u);
+                req = lane == j ? r : req;
+            }
+            eq = warp_sum_u32(__popc(req));
+        }
+        const uint32_t rcg = __popc(rgt);
+        uint32_t rig = rcg;
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+            const uint32_t y = __shfl_up_sync(kFull, rig, o);
+            if (lane >= o) rig += y;
+        }
+        const uint32_t gt = __shfl_sync(kFull, rig, 31);
         uint32_t *wcnt = hist[1];  // [0, 32): warps' keys above T, [32, 64): equal; [64, 128): before them
         if (lane == 0) {
             wcnt[warp] = gt;
@@ -799,34 +815,45 @@ __global__ void __launch_bounds__(THREADS) select_cluster_kernel(const __grid_co
         const uint32_t take = eq_before >= rem ? 0u : min(eq, rem - eq_before);
         const uint32_t pos = gt_before + min(eq_before, rem);
         const uint32_t below = (1u << lane) - 1u;
-        uint32_t selm = gtm;  // this lane's keys taken
+        // the equal keys taken: the warp's first `take`, by row then lane
+        uint32_t keep = 0u;
         if (take >= eq) {
-            selm |= eqm;
-        } else if (take > 0u) {  // the first `take` equal keys of the warp
-            uint32_t t = 0;
-            for (int j = 0; j < kpt; ++j) {
-                const uint32_t em = __ballot_sync(kFull, (eqm >> j) & 1u);
-                if (((eqm >> j) & 1u) && t + __popc(em & below) < take) selm |= 1u << j;
-                t += __popc(em);
+            keep = req;
+        } else if (take > 0u) {
+            const uint32_t ec = __popc(req);
+            uint32_t ei = ec;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(kFull, ei, o);
+                if (lane >= o) ei += y;
+            }
+            const uint32_t epre = ei - ec;
+            uint32_t kk = take > epre ? min(ec, take - epre) : 0u, m = req;
+            for (; kk > 0u; --kk) {  // the lowest kk lanes of the row
+                keep |= m & (0u - m);
+                m &= m - 1u;
             }
         }
-        // rows: lane j keeps row j; its keys' count before it by a scan
-        uint32_t myrow = 0u;
-        for (int j = 0; j < kpt; ++j) {
-            const uint32_t r = __ballot_sync(kFull, (selm >> j) & 1u);
-            myrow = lane == j ? r : myrow;
-        }
-        const uint32_t rc = __popc(myrow);
-        uint32_t ri = rc;
+        const uint32_t myrow = rgt | keep;
+        uint32_t rc = rcg, ri = rig;  // the rows' counts, again when equal keys join them
+        if (__any_sync(kFull, keep != 0u)) {
+            rc = __popc(myrow);
+            ri = rc;
 #pragma unroll
-        for (int o = 1; o < 32; o <<= 1) {
-            const uint32_t y = __shfl_up_sync(kFull, ri, o);
-            if (lane >= o) ri += y;
+            for (int o = 1; o < 32; o <<= 1) {
+                const uint32_t y = __shfl_up_sync(kFull, ri, o);
+                if (lane >= o) ri += y;
+            }
         }
         uint32_t *wrow = hist[0] + 64 * warp;  // [row masks | keys in the rows before], kWarps * 64 <= kSelBins
         wrow[lane] = myrow;
         wrow[32 + lane] = ri - rc;
         __syncwarp();
+        uint32_t selm = gtm;  // this lane's keys taken
+        for (uint32_t eb = take > 0u ? eqm : 0u; eb != 0u; eb &= eb - 1u) {
+            const int j = __ffs(eb) - 1;
+            selm |= ((wrow[j] >> lane) & 1u) << j;
+        }
         for (uint32_t sb = selm; sb != 0u; sb &= sb - 1u) {
             const int j = __ffs(sb) - 1;
             const uint32_t at = pos + wrow[32 + j] + __popc(wrow[j] & below);
