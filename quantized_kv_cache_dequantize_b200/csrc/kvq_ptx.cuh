@@ -1,8 +1,7 @@
 // kvq_ptx.cuh -- thin inline-PTX wrappers used by the sm_100a kernels:
 // bf16 tensor-core MMA (m16n8k16, fp32 accumulate), 8x8 b16 transpose
-// (movmatrix), mbarrier waits with a wall-clock bound, 1-D bulk async
-// copies global -> shared completed on an mbarrier (no cluster multicast),
-// and the cluster barrier and shared-memory loads from a cluster peer.
+// (movmatrix), mbarrier waits with a wall-clock bound, and 1-D bulk async
+// copies global -> shared completed on an mbarrier (no cluster multicast).
 #pragma once
 
 #include <cstdint>
@@ -164,71 +163,23 @@ __device__ __forceinline__ void bulk_copy_g2s_if(bool issue, void *dst, const vo
         : "memory");
 }
 
-// Per-thread asynchronous copy global -> shared of 4, 8 or 16 bytes (both
+// Per-thread asynchronous copy global -> shared of 8 or 16 bytes (both
 // addresses aligned to the size).  Their completion reaches an mbarrier
-// through cp_async_mbar_arrive, or the issuing thread through
-// cp_async_wait_all.
+// through cp_async_mbar_arrive.
 template <int BYTES>
 __device__ __forceinline__ void cp_async(void *dst, const void *src) {
-    static_assert(BYTES == 4 || BYTES == 8 || BYTES == 16, "cp.async size");
+    static_assert(BYTES == 8 || BYTES == 16, "cp.async size");
     if constexpr (BYTES == 16)
         asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
-    else if constexpr (BYTES == 8)
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
     else
-        asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+        asm volatile("cp.async.ca.shared.global [%0], [%1], 8;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
 }
-
-// Wait until every cp.async this thread issued has landed (visible to it).
-__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
 
 // One arrival on `bar`, made once every cp.async this thread issued before
 // it has landed.  The arrival is counted in the barrier's initial count
 // (noinc), so a barrier fed this way by n threads is initialised with n.
 __device__ __forceinline__ void cp_async_mbar_arrive(uint64_t *bar) {
     asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];\n" ::"r"(smem_u32(bar)) : "memory");
-}
-
-// ------------------------------------------------------------ clusters ----
-
-__device__ __forceinline__ uint32_t cluster_ctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
-    return r;
-}
-
-__device__ __forceinline__ uint32_t cluster_nctarank() {
-    uint32_t r;
-    asm volatile("mov.u32 %0, %%cluster_nctarank;\n" : "=r"(r));
-    return r;
-}
-
-// Barrier over every thread of the cluster: shared-memory writes before it
-// (this CTA's and the peers') are visible to the cluster's reads after it.
-// A launch without clusters is a cluster of one CTA.
-__device__ __forceinline__ void cluster_sync() {
-    asm volatile("barrier.cluster.arrive.release;\nbarrier.cluster.wait.acquire;\n" ::: "memory");
-}
-
-// Load of the 32-bit word at `p` in the shared memory of the cluster's CTA
-// `rank` (p: this CTA's address of the same variable).
-__device__ __forceinline__ uint32_t ld_cluster_u32(const void *p, uint32_t rank) {
-    uint32_t a, v;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
-    asm volatile("ld.shared::cluster.u32 %0, [%1];\n" : "=r"(v) : "r"(a) : "memory");
-    return v;
-}
-
-// 16-byte load from the cluster's CTA `rank` (p 16-byte aligned).
-__device__ __forceinline__ uint4 ld_cluster_v4(const void *p, uint32_t rank) {
-    uint32_t a;
-    uint4 v;
-    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
-    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];\n"
-                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
-                 : "r"(a)
-                 : "memory");
-    return v;
 }
 
 // Programmatic dependent launch: wait until the preceding grid in the stream

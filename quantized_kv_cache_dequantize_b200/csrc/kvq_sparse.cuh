@@ -19,6 +19,56 @@
 
 namespace kvq {
 
+// ---- inline PTX used by the select only
+
+// Per-thread asynchronous 4-byte copy global -> shared (both addresses
+// 4-byte aligned), completed for the issuing thread by cp_async_wait_all.
+__device__ __forceinline__ void cp_async4(void *dst, const void *src) {
+    asm volatile("cp.async.ca.shared.global [%0], [%1], 4;\n" ::"r"(smem_u32(dst)), "l"(src) : "memory");
+}
+
+// Wait until every cp.async this thread issued has landed (visible to it).
+__device__ __forceinline__ void cp_async_wait_all() { asm volatile("cp.async.wait_all;\n" ::: "memory"); }
+
+__device__ __forceinline__ uint32_t cluster_ctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;\n" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ uint32_t cluster_nctarank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_nctarank;\n" : "=r"(r));
+    return r;
+}
+
+// Barrier over every thread of the cluster: shared-memory writes before it
+// (this CTA's and the peers') are visible to the cluster's reads after it.
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release;\nbarrier.cluster.wait.acquire;\n" ::: "memory");
+}
+
+// Load of the 32-bit word at `p` in the shared memory of the cluster's CTA
+// `rank` (p: this CTA's address of the same variable).
+__device__ __forceinline__ uint32_t ld_cluster_u32(const void *p, uint32_t rank) {
+    uint32_t a, v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+    asm volatile("ld.shared::cluster.u32 %0, [%1];\n" : "=r"(v) : "r"(a) : "memory");
+    return v;
+}
+
+// 16-byte load from the cluster's CTA `rank` (p 16-byte aligned).
+__device__ __forceinline__ uint4 ld_cluster_v4(const void *p, uint32_t rank) {
+    uint32_t a;
+    uint4 v;
+    asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(a) : "r"(smem_u32(p)), "r"(rank));
+    asm volatile("ld.shared::cluster.v4.u32 {%0, %1, %2, %3}, [%4];\n"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "r"(a)
+                 : "memory");
+    return v;
+}
+
 constexpr int kSparseMaxViews = 96;  // views per score / select launch
 constexpr int kScoreTok = 128;       // threads of a score CTA, one token each at a time
 constexpr int kScoreBlocks = 4;      // blocks of kScoreTok tokens per score CTA
@@ -421,7 +471,7 @@ __global__ void __launch_bounds__(THREADS, 1) select_cluster_kernel(const __grid
     const int lbase = warp * seg + lane;                 // its place in skeys
     const int nk = base < n ? min(kpt, (n - base + 31) / 32) : 0;
     // every score of this lane in flight at once
-    for (int j = 0; j < nk; ++j) cp_async<4>(skeys + lbase + 32 * j, sc + base + 32 * j);
+    for (int j = 0; j < nk; ++j) cp_async4(skeys + lbase + 32 * j, sc + base + 32 * j);
     for (int i = tid; i < kSelBins; i += THREADS) hist[0][i] = 0u;
     cp_async_wait_all();
     __syncthreads();  // every lane's scores have landed
