@@ -86,60 +86,77 @@ __device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], con
     } else if (s != 0.0f) {
         // Fast path: y = fma(x, r, -RN(mn*r)) with r = RN(1/s) lies within
         // 2^(B-23) + |mn*r|*2^-24 of the quotient (x - mn)/s (quotients are
-        // <= 2^B), so unless y is within 2^(B-21) + |mn*r|*2^-21 of a
-        // half-integer it rounds to the same integer as the correctly rounded
-        // quotient RN((x - mn)/s) (and every code is in range).  Elements
-        // closer than that (bf16 grids make exact ties common) are redone
-        // exactly below, without a division.
-        // A group whose min is large against its scale (|mn*r| >= 2^(B+2))
-        // takes y = (x - mn) * r instead (within 3*2^(B-24) of the quotient;
-        // window 2^(B-21)), which keeps y > -1/2 there.
+        // <= 2^B).  A group whose min is large against its scale (|mn*r| >=
+        // 2^(B+2)) takes y = (x - mn) * r instead (within 3*2^(B-24) of the
+        // quotient), which keeps y > -1/2 there.  With W = 2^(B-21) (plus
+        // |mn*r|*2^-21 on the fma form), at least four times that error, y1
+        // and y2 are y shifted by +W and -W (on the fma form: the addend
+        // -mn*r +- W): they bracket the quotient strictly, so when they round
+        // to the same integer the quotient lies strictly inside that
+        // integer's interval and the correctly rounded RN((x - mn)/s) is it
+        // (and every code is in range).  Elements whose brackets round apart
+        // (bf16 grids make exact ties common) are redone exactly below,
+        // without a division.
         const float r = __frcp_rn(s);
         const float mr = __fmul_rn(mn, r);
         const bool fma_ok = fabsf(mr) < __uint_as_float((uint32_t)(127 + B + 2) << 23);
-        const float lim = __fsub_rn(0.5f - __uint_as_float((uint32_t)(127 + B - 21) << 23),
+        const float win = __fadd_rn(__uint_as_float((uint32_t)(127 + B - 21) << 23),
                                     fma_ok ? __fmul_rn(fabsf(mr), 0x1p-21f) : 0.0f);
-        uint32_t near = 0u;
+        const float c1 = __fsub_rn(win, mr), c2 = __fsub_rn(-win, mr);
+        // codes of y1 packed, and those of y2 in `apart`, which then becomes
+        // the difference: per element y1's code minus y2's (0 or 1) in its
+        // field (B = 3: fields straddle words, so a 32-bit mask of the
+        // elements instead)
+        uint32_t apart[B == 3 ? 1 : B];
+#pragma unroll
+        for (int w = 0; w < (B == 3 ? 1 : B); ++w) apart[w] = 0u;
         auto fast = [&](auto use_fma) {
 #pragma unroll
             for (int i = 0; i < 32; ++i) {
                 const float xf = (i & 1) ? bf16hi_to_f32(x[i >> 1]) : bf16lo_to_f32(x[i >> 1]);
-                const float y = use_fma ? __fmaf_rn(xf, r, -mr) : __fmul_rn(__fsub_rn(xf, mn), r);
-                const float t = __fadd_rn(y, kRoundMagic);
-                const float d = __fsub_rn(y, __fsub_rn(t, kRoundMagic));
-                near |= (fabsf(d) <= lim) ? 0u : (1u << i);
-                // the magic sum's bits, 0x4B400000 + c; the constant goes below
-                const uint32_t tb = __float_as_uint(t);
+                float y1, y2;
+                if constexpr (decltype(use_fma)::value) {
+                    y1 = __fmaf_rn(xf, r, c1);
+                    y2 = __fmaf_rn(xf, r, c2);
+                } else {
+                    const float y = __fmul_rn(__fsub_rn(xf, mn), r);
+                    y1 = __fadd_rn(y, win);
+                    y2 = __fsub_rn(y, win);
+                }
+                // the magic sums' bits, 0x4B400000 + code; the constant goes below
+                const uint32_t t1 = __float_as_uint(__fadd_rn(y1, kRoundMagic));
+                const uint32_t t2 = __float_as_uint(__fadd_rn(y2, kRoundMagic));
                 const int bit = i * B;
-                packed[bit >> 5] += tb << (bit & 31);
-                if ((bit & 31) + B > 32) packed[(bit >> 5) + 1] += tb >> (32 - (bit & 31));
+                packed[bit >> 5] += t1 << (bit & 31);
+                if ((bit & 31) + B > 32) packed[(bit >> 5) + 1] += t1 >> (32 - (bit & 31));
+                if constexpr (B == 3) apart[0] |= (t1 - t2) << i;
+                else apart[bit >> 5] += t2 << (bit & 31);  // y2's codes; subtracted below
             }
         };
         if (fma_ok) fast(std::true_type{});
         else fast(std::false_type{});
 #pragma unroll
+        for (int w = 0; w < (B == 3 ? 0 : B); ++w) apart[w] = packed[w] - apart[w];
+#pragma unroll
         for (int w = 0; w < B; ++w) packed[w] -= magic_pack_word<B>(w);
-        while (near) {
-            const int i = __ffs(near) - 1;
-            near &= near - 1u;
-            // element i again from memory: the lane has just read the row, so
-            // it is a cache hit, and one load costs the integer pipe (the
-            // kernel's bound) less than a select tree over the 16 registers
-            // (handoff K cache: 628.5 vs 637.7 us)
+        // element i again from memory: the lane has just read the row, so it
+        // is a cache hit, and one load costs the integer pipe (the kernel's
+        // bound) less than a select tree over the 16 registers
+        auto redo = [&](int i) -> uint32_t {
             const float xf = __uint_as_float((uint32_t)__ldg(src + i) << 16);
             const float a = __fsub_rn(xf, mn);
-            // the code the fast path packed (the same arithmetic), and the
-            // half-integer the quotient is near
+            // the code the fast path packed (y1's), and the half-integer h
+            // that y is near (within W: the brackets straddle it)
             const float y = fma_ok ? __fmaf_rn(xf, r, -mr) : __fmul_rn(a, r);
-            const float t = __fadd_rn(y, kRoundMagic);
-            const float ri = __fsub_rn(t, kRoundMagic);
-            const uint32_t c_fast = __float_as_uint(t) - kRoundMagicBits;
-            // h = the half-integer y is near; e = a - h*s is exact (|e| <
-            // s*2^(B-20) on a grid no finer than ulp(s)/4, i.e. <= B+6
-            // significant bits), so a/s = h + e/s exactly.  RN(a/s) == h iff
-            // |e| <= s*ulp(h)/2 (h has few significant bits, so a tie at that
-            // distance rounds to h); then the code is h rounded half to even,
-            // otherwise the integer on the side of h that e points to.
+            const float y1 = fma_ok ? __fmaf_rn(xf, r, c1) : __fadd_rn(y, win);
+            const uint32_t c_fast = __float_as_uint(__fadd_rn(y1, kRoundMagic)) - kRoundMagicBits;
+            const float ri = __fsub_rn(__fadd_rn(y, kRoundMagic), kRoundMagic);
+            // e = a - h*s is exact (|e| < s*2^(B-20) on a grid no finer than
+            // ulp(s)/4, i.e. <= B+6 significant bits), so a/s = h + e/s
+            // exactly.  RN(a/s) == h iff |e| <= s*ulp(h)/2 (h has few
+            // significant bits, so a tie at that distance rounds to h); then
+            // the code is h rounded half to even, otherwise the integer on
+            // the side of h that e points to.
             const float h = __fadd_rn(ri, (y >= ri) ? 0.5f : -0.5f);
             const float e = __fmaf_rn(-h, s, a);
             const float half_ulp = __uint_as_float((__float_as_uint(h) & 0x7F800000u) - (24u << 23));
@@ -147,14 +164,26 @@ __device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], con
             uint32_t c;
             if (fabsf(e) <= __fmul_rn(s, half_ulp)) c = n + (n & 1u);
             else c = (e > 0.0f) ? n + 1u : n;
-            // patch the packed field of element i (XOR: no carries across fields)
-            const uint32_t flip = c ^ c_fast;
-            const int bit = i * B;
+            return c ^ c_fast;  // the field's correction (XOR: no carries across fields)
+        };
+        if constexpr (B == 3) {
+            for (uint32_t near = apart[0]; near != 0u; near &= near - 1u) {
+                const int i = __ffs(near) - 1;
+                const uint32_t flip = redo(i);
+                const int bit = i * B;
 #pragma unroll
-            for (int k = 0; k < B; ++k) {
-                if ((bit >> 5) == k) packed[k] ^= flip << (bit & 31);
-                if (B == 3 && (bit >> 5) + 1 == k && (bit & 31) + B > 32) packed[k] ^= flip >> (32 - (bit & 31));
+                for (int k = 0; k < B; ++k) {
+                    if ((bit >> 5) == k) packed[k] ^= flip << (bit & 31);
+                    if ((bit >> 5) + 1 == k && (bit & 31) + B > 32) packed[k] ^= flip >> (32 - (bit & 31));
+                }
             }
+        } else {
+#pragma unroll
+            for (int w = 0; w < B; ++w)
+                for (uint32_t near = apart[w]; near != 0u; near &= near - 1u) {
+                    const int b = __ffs(near) - 1;  // the low bit of element (32 w + b) / B's field
+                    packed[w] ^= redo((32 * w + b) / B) << b;
+                }
         }
     }
     s_out = s;
