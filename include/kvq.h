@@ -305,8 +305,14 @@ kvq_status kvq_decode_attn_seq(const kvq_view *views, int32_t n_views, const int
  *             top_k, while the sizes of the views change.
  * Scores are fp32; the attention is that of kvq_decode_attn over one view
  * per (view, KV head) whose packed part is the selected rows, read in place
- * through the selection list (in `selected` or the workspace).
- * Errors: as kvq_decode_attn, and KVQ_ERR_INVALID_ARG for top_k < 1.
+ * through the selection list (in `selected` or the workspace).  The
+ * selection of a view with more than 32768 packed tokens (up to 131072) runs
+ * on a thread-block cluster of 2 or 4 CTAs.
+ * Tuning and tests (environment, read once per call): KVQ_SELECT_CLUSTER = 2
+ * or 4 splits every selection over that many CTAs; KVQ_CHUNK_TOKENS forces
+ * the attention's chunk length.  Neither changes a result.
+ * Errors: as kvq_decode_attn, KVQ_ERR_INVALID_ARG for top_k < 1, and
+ * KVQ_ERR_CUDA when a launch is refused (e.g. no room for a cluster).
  */
 size_t kvq_sparse_decode_attn_workspace_size(const kvq_view *views, int32_t n_views,
                                              int32_t n_q_heads, int32_t n_kv_heads,
