@@ -308,9 +308,10 @@ kvq_status kvq_decode_attn_seq(const kvq_view *views, int32_t n_views, const int
  * through the selection list (in `selected` or the workspace).  The
  * selection of a view with more than 32768 packed tokens (up to 131072) runs
  * on a thread-block cluster of 2 or 4 CTAs.
- * Tuning and tests (environment, read once per call): KVQ_SELECT_CLUSTER = 2
- * or 4 splits every selection over that many CTAs; KVQ_CHUNK_TOKENS forces
- * the attention's chunk length.  Neither changes a result.
+ * Tuning and tests (environment, read at every call): KVQ_SELECT_CLUSTER = 2
+ * or 4 splits every selection over that many CTAs (same selection);
+ * KVQ_CHUNK_TOKENS forces the attention's chunk length (only the rounding of
+ * the split-K merge changes).
  * Errors: as kvq_decode_attn, KVQ_ERR_INVALID_ARG for top_k < 1, and
  * KVQ_ERR_CUDA when a launch is refused (e.g. no room for a cluster).
  */
