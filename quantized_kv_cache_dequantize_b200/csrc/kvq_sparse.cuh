@@ -402,10 +402,9 @@ __device__ __forceinline__ uint32_t warp_sum_u32(uint32_t x) {
 // copies straight into shared memory, where they become order keys; the
 // first-pass bins are kept beside them.
 //   1. 256 scores of the CTA in 8 evenly spaced runs (of each CTA of the
-//      cluster) give
-//      the first pass's range (mean +- 6 standard deviations within their min
-//      and max; any range gives the exact selection: scores outside it go to
-//      the end bins).
+//      cluster) give the first pass's range (mean +- 6 standard deviations
+//      within their min and max; any range gives the exact selection: scores
+//      outside it go to the end bins).
 //   2. First pass: counts of every key's bin; the boundary bin from the
 //      counts (of the whole cluster: each CTA sums its peers' histograms), the
 //      same in every CTA.  Keys in higher bins are taken ("above"); those in
@@ -414,10 +413,11 @@ __device__ __forceinline__ uint32_t warp_sum_u32(uint32_t x) {
 //      digit passes below the bits they share.  Then the candidates are
 //      gathered into one list, where one warp finds the K-th largest key T:
 //      the candidate with fewer than rem larger ones and at least rem not
-//      smaller.
+//      smaller (rem: K less the keys already taken above the candidates).
 //   4. Ordered compaction: the keys above T and the first (by index) of
-//      those equal to T, the output position of every warp from the counts
-//      of the warps and CTAs before it.
+//      those equal to T; each warp's output position from the counts of the
+//      warps and CTAs before it, each key's from one ballot per row of its
+//      warp's keys.
 // In a cluster, every decision that gates a cluster barrier is taken on
 // cluster-wide values, so all its CTAs pass the same barriers; values from
 // the peers are read by one warp and handed on in shared memory.
