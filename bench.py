@@ -634,6 +634,7 @@ def codec_leg(args, local, peak):
     n_el = 2 * H * hw.n_tokens * hw.head_dim
     codec_bytes = n_el * 2 + 2 * (kc.numel() + ks.numel() * 4)
     qt, dt = [], []
+    torch.cuda.synchronize()  # the inputs come from the current stream; the timed stream starts after them
     with ClockSampler(local) as codec_clk, torch.cuda.stream(stream):
         for it in range(args.warmup + args.steps):
             if it == args.warmup:

@@ -56,7 +56,11 @@ from . import (card_info, card_pack, card_unpack, decode_attn, dequantize, new_w
 def _time(fn, reps):
     """Mean device time of one call: 3 eager warm-up calls, then the call
     captured in a CUDA graph and replayed `reps` times (host launch cost stays
-    out of the timing)."""
+    out of the timing).  The inputs were made on the current stream: it is
+    drained first, so that the side stream never touches memory that work
+    still queued there reads or writes (the allocator recycles blocks in
+    the current stream's order only)."""
+    torch.cuda.synchronize()
     st = torch.cuda.Stream()
     with torch.cuda.stream(st):
         for _ in range(3):
