@@ -206,12 +206,13 @@ def test_sparse_many_views_and_workspace_reuse_while_growing(cuda_device):
 
 
 def test_sparse_long_views_both_select_paths(cuda_device):
-    # 32768 packed tokens (one select CTA, 32 keys a lane), 70001 (a cluster
-    # of 4 select CTAs, 18 keys a lane), 140000 (beyond the shared-memory
-    # select: the radix select reading the scores from memory) and 5000,
-    # top_k in the thousands
+    # 32768 packed tokens (one select CTA, 32 keys a lane), 65536 (a cluster
+    # of 2, 32 keys a lane), 70001 (a cluster of 4, 18 keys a lane), 140000
+    # (beyond the shared-memory select: the radix select reading the scores
+    # from memory) and 5000, top_k in the thousands
     specs = [ViewSpec(32768, 16, 16, 4, head=2, seed=810), ViewSpec(140000, 16, 16, 4, head=0, seed=811),
-             ViewSpec(5000, 0, 0, 2, seed=812), ViewSpec(70001, 8, 8, 3, head=5, seed=813)]
+             ViewSpec(5000, 0, 0, 2, seed=812), ViewSpec(70001, 8, 8, 3, head=5, seed=813),
+             ViewSpec(65536, 4, 4, 8, head=1, seed=814)]
     case = build_case(8, 2, 128, specs, q_seed=21)
     scale = 1 / np.sqrt(128)
     k = pick_top_k(case, scale, range(1500, 2400, 7))
