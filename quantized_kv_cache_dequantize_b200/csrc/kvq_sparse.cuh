@@ -73,11 +73,13 @@ constexpr int kSparseMaxViews = 96;  // views per score / select launch
 constexpr int kScoreTok = 128;       // threads of a score CTA, one token each at a time
 constexpr int kScoreBlocks = 4;      // blocks of kScoreTok tokens per score CTA
 constexpr int kScoreHeads = 8;       // query heads per register batch
-constexpr int kSelectThreads = 512;
-constexpr int kSelectStageMax = 45056;  // keys a select CTA stages in shared memory (176 KiB)
+constexpr int kSelectThreads = 512;     // select_kernel CTA (views longer than kSelFastMax)
+constexpr int kSelectStageMax = 45056;  // keys a select_kernel CTA stages in shared memory (176 KiB)
 constexpr int kSelClusterThreads = 1024;  // select_cluster_kernel CTA
 constexpr int kSelMaxCluster = 4;         // CTAs per (view, KV head) at most
-constexpr int kSelFastMax = kSelMaxCluster * kSelClusterThreads * 32;  // 32 keys per thread at most
+// views of up to kSelFastMax packed tokens select in shared memory (32 keys a
+// thread at most)
+constexpr int kSelFastMax = kSelMaxCluster * kSelClusterThreads * 32;
 constexpr int kSelBins = 2048;            // histogram bins of a select_cluster_kernel pass
 constexpr int kSelWarpMax = 64;           // candidates one warp finishes
 
