@@ -139,9 +139,9 @@ __device__ __forceinline__ void quantize_half_group(const uint32_t (&x)[16], con
         for (int w = 0; w < (B == 3 ? 0 : B); ++w) apart[w] = packed[w] - apart[w];
 #pragma unroll
         for (int w = 0; w < B; ++w) packed[w] -= magic_pack_word<B>(w);
-        // element i again from memory: the lane has just read the row, so it
-        // is a cache hit, and one load costs the integer pipe (the kernel's
-        // bound) less than a select tree over the 16 registers
+        // element i again from memory: the lane has just read the row through
+        // L1 (read-only cached loads), so it is a cache hit, and one load
+        // costs the integer pipe less than a select tree over the 16 registers
         auto redo = [&](int i) -> uint32_t {
             const float xf = __uint_as_float((uint32_t)__ldg(src + i) << 16);
             const float a = __fsub_rn(xf, mn);
@@ -264,7 +264,7 @@ __global__ void __launch_bounds__(256) quantize_kernel(CodecArgs a) {
         const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
 #pragma unroll
         for (int v = 0; v < 4; ++v) {
-            const uint4 q = ok ? __ldcs(s4 + v) : make_uint4(0, 0, 0, 0);
+            const uint4 q = ok ? __ldg(s4 + v) : make_uint4(0, 0, 0, 0);
             x[4 * v + 0] = q.x; x[4 * v + 1] = q.y; x[4 * v + 2] = q.z; x[4 * v + 3] = q.w;
         }
         uint32_t packed[B];
